@@ -1,0 +1,195 @@
+"""Pins for the block-allocator reference model (CPU only).
+
+The model is pinned to the pages' block-table figure (vLLM 初探 §1.4), to
+hand-worked copy-on-write cases, and to invariants that hold after any sequence
+of operations: every table entry is one reference, free + live blocks = pool,
+a free block never sits in a live table, and a table always has
+ceil(length / block_size) entries.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import workloads as wl
+from oracle.block_manager import ERR_INVALID, ERR_OOM, BlockManagerError, BlockManagerModel
+
+
+def check_invariants(m: BlockManagerModel):
+    refs = [0] * m.num_blocks
+    for table in m.tables.values():
+        for b in table:
+            refs[b] += 1
+    assert refs == m.ref, "reference counts must equal the number of table entries"
+    live = {b for b in range(m.num_blocks) if m.ref[b] > 0}
+    assert len(m.free) + len(live) == m.num_blocks
+    assert not (set(m.free) & live)
+    assert len(set(m.free)) == len(m.free)
+    for s, table in m.tables.items():
+        assert len(table) == -(-m.lens[s] // m.block_size)
+
+
+def test_block_table_figure():
+    fig = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "block_table_figure.json")))
+    sc, ex = fig["scenario"], fig["expected"]
+    m = BlockManagerModel(8, sc["block_size"], sc["initial_free_order"])
+    A, B = 1, 2
+    m.add_seq(A, 16)
+    m.add_seq(B, 16)
+    for _ in range(16):
+        m.append_slots([A])
+    for _ in range(16):
+        m.append_slots([B])
+    assert m.tables[A] == ex["table_A"] == [fig["printed"]["logical_table"]["Block 0"],
+                                            fig["printed"]["logical_table"]["Block 1"]]
+    assert m.tables[B] == ex["table_B"]
+    assert sorted(m.free) == ex["free_after"] == fig["printed"]["free_blocks"]
+    for pos, slot in ex["slots_A_positions"].items():
+        assert m.slots(A, int(pos), 1) == [slot]
+    for pos, slot in ex["slots_B_positions"].items():
+        assert m.slots(B, int(pos), 1) == [slot]
+    check_invariants(m)
+
+
+def test_blocks_return_to_pool_on_finish():
+    """Outcome School explainer: a finished request's blocks go straight back to the pool."""
+    m = BlockManagerModel(10, 4, list(range(10)))
+    m.add_seq(0, 9)          # blocks 0,1,2
+    m.add_seq(1, 4)          # block 3
+    assert m.num_free() == 6
+    m.free_seq(0)
+    assert list(m.free) == [4, 5, 6, 7, 8, 9, 0, 1, 2]
+    m.add_seq(2, 20)         # takes 5 blocks from the front
+    assert m.tables[2] == [4, 5, 6, 7, 8]
+    check_invariants(m)
+
+
+def test_new_block_only_when_last_is_full():
+    m = BlockManagerModel(6, 4)
+    m.add_seq(7, 0)
+    slots_seen = []
+    for _ in range(9):
+        slots, pairs = m.append_slots([7])
+        slots_seen += slots
+        assert pairs == []
+    assert m.tables[7] == [0, 1, 2]
+    assert slots_seen == [0, 1, 2, 3, 4, 5, 6, 7, 8]
+    assert m.num_free() == 3
+
+
+def test_beam_fork_copy_on_write_by_hand():
+    """Four beams share a partial last block; appending in id order, beams 0-2 copy
+    it and beam 3, by then its only holder, writes in place."""
+    m = BlockManagerModel(16, 4, list(range(16)))
+    m.add_seq(0, 6)                      # blocks [0, 1], last block has 2 of 4 rows
+    for child in (1, 2, 3):
+        m.fork(0, child)
+    assert m.ref[0] == 4 and m.ref[1] == 4
+    slots, pairs = m.append_slots([0, 1, 2, 3])
+    assert pairs == [(1, 2), (1, 3), (1, 4)]
+    assert [m.tables[s] for s in range(4)] == [[0, 2], [0, 3], [0, 4], [0, 1]]
+    assert slots == [2 * 4 + 2, 3 * 4 + 2, 4 * 4 + 2, 1 * 4 + 2]
+    assert m.ref[0] == 4 and m.ref[1] == 1
+    check_invariants(m)
+
+
+def test_fork_at_block_boundary_needs_no_copy():
+    m = BlockManagerModel(8, 4, list(range(8)))
+    m.add_seq(0, 8)                      # two full blocks
+    m.fork(0, 1)
+    slots, pairs = m.append_slots([0, 1])
+    assert pairs == [] and slots == [2 * 4, 3 * 4]
+    assert m.tables[0][:2] == m.tables[1][:2] == [0, 1]
+    check_invariants(m)
+
+
+def test_shared_prefix_refcounts():
+    """Outcome School explainer, "内存共享": identical prefixes stored once."""
+    m = BlockManagerModel(400, 16, list(range(400)))
+    m.add_seq(0, 1024 + 30)
+    prefix = m.tables[0][:64]
+    for s in range(1, 128):
+        m.add_seq(s, 1024 + s % 16 + 1, prefix)
+    assert all(m.ref[b] == 128 for b in prefix)
+    assert all(m.tables[s][:64] == prefix for s in range(128))
+    check_invariants(m)
+    for s in range(128):
+        m.free_seq(s)
+    assert m.num_free() == 400 and sum(m.ref) == 0
+
+
+def test_oom_is_all_or_nothing():
+    m = BlockManagerModel(3, 4, [2, 0, 1])
+    m.add_seq(0, 4)
+    m.add_seq(1, 4)
+    before = (list(m.free), dict((k, list(v)) for k, v in m.tables.items()), dict(m.lens), list(m.ref))
+    with pytest.raises(BlockManagerError) as e:
+        m.append_slots([0, 1])           # both need a new block, only one is free
+    assert e.value.code == ERR_OOM
+    assert before == (list(m.free), dict((k, list(v)) for k, v in m.tables.items()), dict(m.lens), list(m.ref))
+    with pytest.raises(BlockManagerError) as e:
+        m.add_seq(2, 9)
+    assert e.value.code == ERR_OOM
+
+
+def test_invalid_operations():
+    m = BlockManagerModel(4, 4)
+    m.add_seq(0, 3)
+    for call in (lambda: m.add_seq(0, 1), lambda: m.fork(5, 6), lambda: m.fork(0, 0),
+                 lambda: m.append_slots([0, 0]), lambda: m.append_slots([9]),
+                 lambda: m.free_seq(3), lambda: m.decref(3), lambda: m.incref(2),
+                 lambda: m.slots(0, 2, 2), lambda: m.add_seq(1, 3, [0, 1])):
+        with pytest.raises(BlockManagerError) as e:
+            call()
+        assert e.value.code == ERR_INVALID
+
+
+def random_ops(seed, steps=400, num_blocks=48, block_size=4):
+    """A seeded random mix of every operation; checks invariants after each one."""
+    rng = wl.rng_for(seed)
+    m = BlockManagerModel(num_blocks, block_size, rng.permutation(num_blocks))
+    next_id = 0
+    for _ in range(steps):
+        op = rng.integers(0, 5)
+        live = sorted(m.tables)
+        try:
+            if op == 0 or not live:
+                shared = []
+                if live and rng.random() < 0.5:
+                    donor = live[rng.integers(len(live))]
+                    full = m.lens[donor] // block_size
+                    shared = m.tables[donor][:rng.integers(0, full + 1)]
+                m.add_seq(next_id, len(shared) * block_size + int(rng.integers(0, 9)), shared)
+                next_id += 1
+            elif op == 1:
+                m.fork(live[rng.integers(len(live))], next_id)
+                next_id += 1
+            elif op == 2:
+                pick = rng.permutation(live)[:rng.integers(1, len(live) + 1)]
+                m.append_slots([int(s) for s in pick])
+            elif op == 3:
+                m.free_seq(live[rng.integers(len(live))])
+            else:
+                s = live[rng.integers(len(live))]
+                if m.lens[s]:
+                    start = int(rng.integers(0, m.lens[s]))
+                    m.slots(s, start, m.lens[s] - start)
+        except BlockManagerError as e:
+            assert e.code == ERR_OOM
+        check_invariants(m)
+    return m
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_invariants_under_random_operations(seed):
+    random_ops(seed)
+
+
+def test_slots_follow_tables():
+    m = random_ops(42, steps=200)
+    for s, table in m.tables.items():
+        got = m.slots(s, 0, m.lens[s])
+        for p, slot in enumerate(got):
+            assert slot // m.block_size == table[p // m.block_size]
+            assert slot % m.block_size == p % m.block_size

@@ -1,0 +1,469 @@
+"""Benchmark of the paged decode step on B200.
+
+One step = one decode step of one attention layer over the whole batch, i.e. every
+row of the hot path:
+  host block allocator (a fresh slot per sequence, CoW pairs) -> copy_blocks (when
+  there are CoW pairs) -> reshape_and_cache (the new token's K/V) ->
+  paged_attention_decode (plan + streaming kernel).
+
+`value`  KV-read GB/s of the decode = sum_s L_s * Hkv * D * 2 (K and V) * 2 B per step,
+         divided by the device time of the whole step, inputs resident in HBM (the
+         allocator's slots/tables of every step are prepared before timing).
+`e2e`    the same metric through the public API with host buffers: per step the
+         allocator runs on the host, q / new K,V / slots / tables / lengths are copied
+         from pinned host memory, the kernels run, and the output is read back.
+`roofline` the decode call (plan + streaming kernel) against the measured HBM copy
+         bandwidth, algorithmic bytes = KV + q + out + tables + lengths.
+
+Default workload: the LLaMA-13B-shaped mixed-length batch (256 sequences, 40 heads,
+head_dim 128, block size 16, lengths 70% geometric(mean 50) / 30% U{1000..2000}),
+the batch on which the 70%-of-HBM target is stated.  Its KV (2.5 GB) is ~20x the
+L2, so consecutive steps cannot hit in L2.
+
+`--impl reference` times the CPU oracle (float64 NumPy, one thread) on a bounded
+sample of the same workload and prints the same JSON line with "impl": "reference".
+Multi-GPU (`torchrun`): independent replicas per GPU (weak scaling), no collective on
+the data path; timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); seq-steps/sec"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_hbm_gbs():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def rank_info():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# Workload preparation (allocator + per-step inputs)
+# ---------------------------------------------------------------------------
+
+def decode_bytes(lens, Hq, Hkv, D, bs):
+    """Algorithmic bytes of one decode call: KV of every valid token once, q, out (bf16),
+    the used table entries and the lengths."""
+    lens = np.asarray(lens, np.int64)
+    kv = int(lens.sum()) * Hkv * D * 2 * 2
+    blocks = int(np.sum(-(-lens // bs)))
+    return kv, kv + 2 * len(lens) * Hq * D * 2 + blocks * 4 + len(lens) * 4
+
+
+class Workload:
+    def __init__(self, name: str, steps: int, seed: int, device):
+        import torch
+        import paged_kv_cache_423_b200 as pkv
+        self.name = name
+        b = wl.make_decode_batch(name, with_data=False, extra_blocks=0)
+        self.B, self.Hq, self.Hkv, self.D, self.bs = b.num_seqs, b.num_heads, b.num_kv_heads, b.head_dim, b.block_size
+        self.scale = b.scale
+        self.lens0 = b.context_lens.copy()            # context lengths after the first appended token
+        growth = steps + 1
+        need_final = int(np.sum(-(-(self.lens0 + growth) // self.bs)))
+        self.NB = max(b.num_blocks, int(math.ceil(1.2 * need_final)))
+        self.free_order = wl.rng_for(seed).permutation(self.NB).astype(np.int32)
+        self.max_blocks = int(np.max(-(-(self.lens0 + growth) // self.bs)))
+        self.device = device
+        self.pkv = pkv
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        shape = (self.NB, self.Hkv, self.bs, self.D)
+        self.key_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        self.value_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        self.rng = wl.rng_for(seed + 1)
+
+    def new_manager(self):
+        bm = self.pkv.BlockManager(self.NB, self.bs, self.free_order)
+        for s in range(self.B):
+            bm.add_seq(s, int(self.lens0[s]) - 1)
+        return bm
+
+    def host_step_inputs(self):
+        q = wl.bf16_normal(self.rng, (self.B, self.Hq, self.D))
+        k, v = wl.new_tokens(self.rng, self.B, self.Hkv, self.D)
+        return q, k, v
+
+
+def to_dev(bits, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import paged_kv_cache_423_b200 as pkv
+
+    device = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device)
+    total = args.warmup + args.steps
+    w = Workload(args.workload, total, seed=1000 + rank, device=device)
+    seq_ids = list(range(w.B))
+
+    # ---- prepare every step's device inputs (allocator run ahead of timing)
+    bm = w.new_manager()
+    steps = []
+    for _ in range(total):
+        slots, pairs = bm.append_slots(seq_ids)
+        tables, lens = bm.export_tables(seq_ids, w.max_blocks)
+        q, k, v = w.host_step_inputs()
+        steps.append(dict(q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
+                          slots=torch.from_numpy(slots).to(device), pairs=torch.from_numpy(pairs).to(device),
+                          n_pairs=len(pairs), tables=torch.from_numpy(tables).to(device),
+                          lens=torch.from_numpy(lens).to(device), max_len=int(lens.max()), host_lens=lens))
+    bm.close()
+    max_len_all = max(s["max_len"] for s in steps)
+    ws = torch.empty(pkv.paged_attention_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.bs, max_len_all),
+                     dtype=torch.uint8, device=device)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    path = {"auto": 0, "simt": 1, "tensor": 2}[args.path]
+
+    def step(i, ev=None):
+        st = steps[i]
+        if st["n_pairs"]:
+            pkv.copy_blocks([w.key_cache], [w.value_cache], st["pairs"], status=status)
+        pkv.reshape_and_cache(st["k"], st["v"], w.key_cache, w.value_cache, st["slots"], status=status)
+        if ev is not None:
+            ev[0].record(stream)
+        pkv.paged_attention_decode(out, st["q"], w.key_cache, w.value_cache, st["tables"], st["lens"], max_len_all,
+                                   w.scale, ws, path=path, status=status)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    launches = 0
+    kv_total = bytes_total = 0
+    for i in range(args.warmup, total):
+        kv, alg = decode_bytes(steps[i]["host_lens"], w.Hq, w.Hkv, w.D, w.bs)
+        kv_total += kv
+        bytes_total += alg
+        launches += 3 + (1 if steps[i]["n_pairs"] else 0)
+    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        t0.record(stream)
+        for j, i in enumerate(range(args.warmup, total)):
+            step(i, dec_events[j])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    dec_ms = sum(a.elapsed_time(b) for a, b in dec_events)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item():#x}")
+    ms_max = ms
+    if dist:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    value = world * kv_total / (ms_max * 1e-3) / 1e9
+    seq_steps = world * w.B * args.steps / (ms_max * 1e-3)
+
+    # ---- e2e through the public API with host buffers
+    e2e = run_e2e(args, w, pkv, device, path, ws, out, status, max_len_all) if not args.no_e2e else None
+
+    peak, peak_kind = measured_hbm_gbs()
+    dec_gbs = bytes_total / (dec_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "num_seqs": w.B, "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D,
+                   "block_size": w.bs, "mean_context": float(np.mean(w.lens0)), "num_blocks": w.NB,
+                   "kv_bytes_per_step": kv_total // args.steps, "path": args.path,
+                   "l2": "inputs larger than L2 (KV per step >> 126 MB)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "seq_steps_per_s": round(seq_steps, 1),
+        "pct_hbm_peak": round(100 * value / world / peak, 2),
+        "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(dec_gbs / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "paged_attention_decode (plan + streaming kernel)",
+                     "ms_per_launch": round(dec_ms / args.steps, 4)},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, steps[args.warmup], budget_s=args.cpu_budget)
+    if dist:
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
+    import torch
+    bm = w.new_manager()
+    seq_ids = list(range(w.B))
+    stream = torch.cuda.current_stream()
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+    host = []
+    for _ in range(args.warmup + args.steps):
+        q, k, v = w.host_step_inputs()
+        host.append((pin(q.view(np.int16)), pin(k.view(np.int16)), pin(v.view(np.int16))))
+    out_host = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    dq = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=device)
+    dk = torch.empty((w.B, w.Hkv, w.D), dtype=torch.bfloat16, device=device)
+    dv = torch.empty_like(dk)
+    d_slots = torch.empty(w.B, dtype=torch.int64, device=device)
+    d_pairs = torch.empty((w.B, 2), dtype=torch.int64, device=device)
+    d_tables = torch.empty((w.B, w.max_blocks), dtype=torch.int32, device=device)
+    d_lens = torch.empty(w.B, dtype=torch.int32, device=device)
+    tab_host = torch.empty((w.B, w.max_blocks), dtype=torch.int32).pin_memory()
+    len_host = torch.empty(w.B, dtype=torch.int32).pin_memory()
+    slot_host = torch.empty(w.B, dtype=torch.int64).pin_memory()
+    pair_host = torch.empty((w.B, 2), dtype=torch.int64).pin_memory()
+    h2d = d2h = 0
+
+    def step(i):
+        nonlocal h2d, d2h
+        slots, pairs = bm.append_slots(seq_ids)
+        tables, lens = bm.export_tables(seq_ids, w.max_blocks)
+        slot_host.numpy()[:] = slots
+        tab_host.numpy()[:] = tables
+        len_host.numpy()[:] = lens
+        q, k, v = host[i]
+        dq.view(torch.int16).copy_(q.view(dq.shape), non_blocking=True)
+        dk.view(torch.int16).copy_(k.view(dk.shape), non_blocking=True)
+        dv.view(torch.int16).copy_(v.view(dv.shape), non_blocking=True)
+        d_slots.copy_(slot_host, non_blocking=True)
+        d_tables.copy_(tab_host, non_blocking=True)
+        d_lens.copy_(len_host, non_blocking=True)
+        nbytes = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + slots.nbytes + tables.nbytes + lens.nbytes
+        if len(pairs):
+            pair_host.numpy()[:len(pairs)] = pairs
+            d_pairs[:len(pairs)].copy_(pair_host[:len(pairs)], non_blocking=True)
+            pkv.copy_blocks([w.key_cache], [w.value_cache], d_pairs[:len(pairs)], status=status)
+            nbytes += pairs.nbytes
+        pkv.reshape_and_cache(dk, dv, w.key_cache, w.value_cache, d_slots, status=status)
+        pkv.paged_attention_decode(out, dq, w.key_cache, w.value_cache, d_tables, d_lens, max_len_bound, w.scale, ws,
+                                   path=path, status=status)
+        out_host.copy_(out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return nbytes, out_host.numel() * 2, lens
+
+    for i in range(args.warmup):
+        step(i)
+    kv_total = 0
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.warmup, args.warmup + args.steps):
+        bi, bo, lens = step(i)
+        h2d += bi
+        d2h += bo
+        kv_total += int(np.asarray(lens, np.int64).sum()) * w.Hkv * w.D * 4
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    bm.close()
+    return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d // args.steps, "d2h_bytes_per_step": d2h // args.steps,
+            "ms_per_step": round(ms / args.steps, 4)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, step_inputs, n_seqs, rng):
+    """Host copies of a sample of sequences (their blocks only) for the oracle."""
+    import torch
+    seqs = sorted(rng.choice(w.B, size=min(n_seqs, w.B), replace=False).tolist())
+    lens = step_inputs["host_lens"] if "host_lens" in step_inputs else None
+    tables = step_inputs["tables"].cpu().numpy()
+    q = step_inputs["q"].view(torch.int16).cpu().numpy().view(np.uint16)
+    items = []
+    for s in seqs:
+        need = -(-int(lens[s]) // w.bs)
+        idx = torch.from_numpy(tables[s][:need].astype(np.int64)).to(w.device)
+        kc = w.key_cache[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+        vc = w.value_cache[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+        items.append((q[s:s + 1], kc, vc, np.arange(need, dtype=np.int32)[None, :], lens[s:s + 1]))
+    return items
+
+
+def time_oracle(w, items, budget_s):
+    from threadpoolctl import threadpool_limits
+    from oracle import paged_attention
+    done_bytes = 0
+    t0 = time.perf_counter()
+    n = 0
+    with threadpool_limits(limits=1):
+        for q, kc, vc, table, lens in items:
+            paged_attention.paged_decode(q, kc, vc, table, lens, w.scale)
+            done_bytes += int(lens.sum()) * w.Hkv * w.D * 4
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+    dt = time.perf_counter() - t0
+    return done_bytes, dt, n
+
+
+def cpu_baseline(w, step_inputs, budget_s=10.0):
+    items = oracle_sample(w, step_inputs, 64, wl.rng_for(77))
+    done, dt, n = time_oracle(w, items, budget_s)
+    return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} sequences of the {w.name} batch (all {w.Hq} heads each), float64 NumPy, 1 thread, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, rank, world, local_rank):
+    """The CPU oracle as the reference arm, on a bounded sample of the same workload."""
+    import torch
+    if rank != 0:
+        return None
+    device = torch.device(f"cuda:{local_rank}") if torch.cuda.is_available() else None
+    if device is None:
+        return {"impl": "reference", "unavailable": "no CUDA device to hold the synthetic workload"}
+    torch.cuda.set_device(device)
+    w = Workload(args.workload, args.warmup + args.steps, seed=1000, device=device)
+    bm = w.new_manager()
+    ids = list(range(w.B))
+    bm.append_slots(ids)
+    tables, lens = bm.export_tables(ids, w.max_blocks)
+    q, _, _ = w.host_step_inputs()
+    st = {"tables": torch.from_numpy(tables), "host_lens": lens, "q": to_dev(q, device)}
+    rng = wl.rng_for(78)
+    per_step = max(1, int(args.ref_seqs))
+    for _ in range(args.warmup):
+        time_oracle(w, oracle_sample(w, st, per_step, rng), 1e9)
+    kv = 0
+    dt_total = 0.0
+    n_total = 0
+    for _ in range(args.steps):
+        items = oracle_sample(w, st, per_step, rng)
+        b, dt, n = time_oracle(w, items, 1e9)
+        kv += b
+        dt_total += dt
+        n_total += n
+    value = kv / dt_total / 1e9
+    sample = (f"{per_step} random sequences of the {w.name} batch per step (all {w.Hq} heads), float64 NumPy oracle, "
+              f"1 thread")
+    return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * dt_total / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "num_seqs": w.B, "num_heads": w.Hq, "num_kv_heads": w.Hkv,
+                       "head_dim": w.D, "block_size": w.bs},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama13b_mixed_bs16", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-seqs", type=int, default=8)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local_rank = rank_info()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world, local_rank)
+    else:
+        res = run_ours(args, rank, world, local_rank)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

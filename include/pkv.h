@@ -1,0 +1,232 @@
+/*
+ * pkv.h — C ABI of the B200 paged KV-cache decode library (libpkv.so).
+ *
+ * The scheme: the KV cache of every sequence is cut into fixed-size blocks of
+ * `block_size` tokens (16 or 32) that sit anywhere in one shared physical pool;
+ * each sequence reaches its blocks through a block table that keeps their order
+ * (vLLM 初探 §1.4 PagedAttention 原理简介, block-table figure; Outcome School vLLM
+ * explainer, "vLLM的核心创新：PagedAttention").  Decode attention follows the
+ * paged_attention pseudo-code of the intelliparadigm article
+ * "PagedAttention：操作系统分页思想的跨界创新" §2.1: logical block = position //
+ * block_size, physical block = block_tables[seq][logical block], then
+ * softmax(scale * q·Kᵀ)·V over the sequence's tokens.
+ *
+ * Conventions for every call
+ *   - "device" pointers are CUDA device memory owned by the caller (the library
+ *     never allocates, frees or keeps them); "host" pointers are ordinary memory.
+ *   - Tensors are dense and row-major with the shapes given; bf16 is IEEE bfloat16.
+ *     Device tensors must start on a 16-byte boundary (PKV_ERR_INVALID otherwise).
+ *   - Kernel calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  A return of PKV_OK means the work was enqueued.
+ *   - Argument errors are reported before anything is enqueued and leave all
+ *     memory untouched.  Data-dependent errors found on the device (an index out
+ *     of range) never trap: the offending row/block is skipped and a bit is OR-ed
+ *     into the optional device word `status` (int32, caller-zeroed; may be NULL).
+ *   - pkv_last_error_string() returns the text of the last failure on the calling
+ *     host thread.
+ *
+ * Pool layout (one layer): key_cache, value_cache = [num_blocks, num_kv_heads,
+ * block_size, head_dim] bf16.  A (block, kv head) tile of block_size x head_dim is
+ * contiguous (4 KiB for 16 x 128), the unit the kernels stage into shared memory.
+ * Slot of a token = physical_block * block_size + row in the block.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ---- */
+#define PKV_OK 0
+#define PKV_ERR_INVALID (-1)     /* bad argument, shape, pointer alignment or id */
+#define PKV_ERR_OOM (-2)         /* block pool exhausted; nothing was changed */
+#define PKV_ERR_CUDA (-3)        /* a CUDA runtime call or launch failed */
+#define PKV_ERR_UNSUPPORTED (-4) /* head_dim not in {64,128}, block_size not in {16,32},
+                                    num_heads % num_kv_heads != 0, ... */
+
+/* ---- bits of the device status word ---- */
+#define PKV_DEV_BAD_SLOT 0x1     /* reshape_and_cache: slot >= num_blocks*block_size */
+#define PKV_DEV_BAD_BLOCK 0x2    /* a block-table entry outside [0, num_blocks) */
+#define PKV_DEV_BAD_CONTEXT 0x4  /* context_len < 0, > max_context_len or > max_blocks*block_size */
+#define PKV_DEV_BAD_PAIR 0x8     /* copy_blocks: src or dst outside [0, num_blocks) */
+#define PKV_DEV_TIMEOUT 0x10     /* a bounded on-chip wait gave up (the kernel returned early) */
+
+/* ---- output dtypes and decode paths ---- */
+#define PKV_DTYPE_BF16 0
+#define PKV_DTYPE_F32 1
+#define PKV_PATH_AUTO 0          /* tensor-core path for grouped heads where supported, else CUDA cores */
+#define PKV_PATH_SIMT 1          /* CUDA-core streaming kernel, any head grouping */
+#define PKV_PATH_TENSOR 2        /* tcgen05 query-group kernel; PKV_ERR_UNSUPPORTED where it does not apply */
+
+typedef void* pkv_stream_t;      /* a cudaStream_t */
+typedef struct pkv_bm pkv_bm;    /* opaque host block manager */
+
+/* Text of the last error on this host thread ("" if none). Never NULL. */
+PKV_API const char* pkv_last_error_string(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+PKV_API int pkv_version(void);
+
+/*
+ * reshape_and_cache — write each new token's K and V into the pool.
+ * Outcome School explainer, "LLM serving的基本流程与KV缓存": every decoded token adds
+ * one K/V pair that stays resident until its request ends; the intelliparadigm
+ * article §2.2: growth only takes a new page and a table update, nothing moves.
+ *
+ *   key, value       device [num_tokens, num_kv_heads, head_dim] bf16 (read)
+ *   key_cache,
+ *   value_cache      device [num_blocks, num_kv_heads, block_size, head_dim] bf16 (written)
+ *   slot_mapping     device [num_tokens] int64: destination slot of token t;
+ *                    slot < 0 skips the token; slot >= num_blocks*block_size is
+ *                    skipped and sets PKV_DEV_BAD_SLOT.
+ *   Two tokens with the same slot in one call: which one lands is unspecified.
+ *   num_tokens == 0 is a no-op.  Bit-exact copy.
+ */
+PKV_API int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
+                          const int64_t* slot_mapping, int num_tokens, int num_blocks,
+                          int num_kv_heads, int head_dim, int block_size, int32_t* status,
+                          pkv_stream_t stream);
+
+/*
+ * copy_blocks — copy-on-write copies of shared blocks that diverge.
+ * Outcome School explainer, "内存共享": beams share blocks until they diverge; the
+ * copy itself is this library's reading (see pkv_bm_append_slots).
+ *
+ *   key_caches,
+ *   value_caches     HOST arrays of num_layers DEVICE pointers, each a pool of
+ *                    [num_blocks, block_elems] bf16 (block_elems = Hkv*bs*D)
+ *   block_mapping    device [num_pairs, 2] int64: (src, dst) physical block ids;
+ *                    out-of-range pairs are skipped and set PKV_DEV_BAD_PAIR.
+ *   Every dst must be distinct and no dst may also be a src in the same call.
+ *   num_pairs == 0 or num_layers == 0 is a no-op.  Bit-exact copy.
+ */
+PKV_API int pkv_copy_blocks(void* const* key_caches, void* const* value_caches, int num_layers,
+                    const int64_t* block_mapping, int num_pairs, int num_blocks,
+                    int64_t block_elems, int32_t* status, pkv_stream_t stream);
+
+/*
+ * Bytes of device workspace pkv_paged_attention_decode needs for these sizes
+ * (the plan of work items and the split-context partials).  Returns 0 on bad
+ * arguments.  partition_tokens: 0 = automatic, else the split size (below).
+ */
+PKV_API size_t pkv_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                          int head_dim, int block_size, int max_context_len,
+                                          int partition_tokens);
+
+/* Split size the automatic choice picks for these sizes (64..512 tokens). */
+PKV_API int pkv_paged_attention_partition_tokens(int num_seqs, int num_kv_heads, int block_size,
+                                         int max_context_len);
+
+/*
+ * paged_attention_decode — single-token decode attention through block tables.
+ * intelliparadigm article §2.1 (paged_attention pseudo-code; mapping table; kernel
+ * that splices non-contiguous pages through shared memory with prefetch).
+ *
+ * For every sequence s and query head h, with g = num_heads / num_kv_heads,
+ * kv = h / g and L = context_lens[s] (the current token included):
+ *   out[s,h,:] = sum_t softmax_t(scale * q[s,h,:]·K_t) V_t,   t = 0..L-1,
+ *   K_t = key_cache[block_tables[s][t / bs], kv, t % bs, :]  (V likewise).
+ * L == 0 gives a zero row.  Scores, softmax and sums are fp32; the bf16 output
+ * is the round-to-nearest-even of the fp32 result.
+ *
+ *   out              device [num_seqs, num_heads, head_dim], bf16 or f32 (out_dtype)
+ *   query            device [num_seqs, num_heads, head_dim] bf16
+ *   key_cache,
+ *   value_cache      device [num_blocks, num_kv_heads, block_size, head_dim] bf16
+ *   block_tables     device [num_seqs, max_blocks_per_seq] int32; entries past
+ *                    ceil(L/bs) are never read
+ *   context_lens     device [num_seqs] int32; each must be <= max_context_len and
+ *                    <= max_blocks_per_seq*block_size, else the row is zeroed and
+ *                    PKV_DEV_BAD_CONTEXT is set
+ *   max_context_len  host upper bound of context_lens (sizes the split)
+ *   head_dim 64 or 128; block_size 16 or 32; num_heads % num_kv_heads == 0
+ *   partition_tokens 0 = automatic; else 64, 128, 256 or 512 (a multiple of block_size):
+ *                    sequences longer than this are split into partitions that run
+ *                    in parallel and are merged by log-sum-exp rescaling
+ *   path             PKV_PATH_AUTO / PKV_PATH_SIMT / PKV_PATH_TENSOR
+ *   workspace        device scratch of >= pkv_paged_attention_workspace_size(...)
+ *                    bytes, 256-byte aligned; its contents need no initialisation
+ *                    and are clobbered; calls sharing one workspace must not overlap
+ *                    on the GPU.
+ */
+PKV_API int pkv_paged_attention_decode(void* out, int out_dtype, const void* query, const void* key_cache,
+                               const void* value_cache, const int32_t* block_tables,
+                               int max_blocks_per_seq, const int32_t* context_lens,
+                               int max_context_len, int num_seqs, int num_heads, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, float scale,
+                               int partition_tokens, int path, void* workspace,
+                               size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
+
+/*
+ * Host block manager — free list + reference counts + per-sequence block tables.
+ * Outcome School explainer, "vLLM的核心创新：PagedAttention" (a block only when needed,
+ * any free block serves any request, finished requests return all blocks at once)
+ * and "内存共享" (shared prefixes, beams).  Not thread-safe: one manager per host
+ * thread, or external locking.  All ids are host values; nothing touches the GPU.
+ *
+ * Free list: FIFO.  Its initial order is `initial_order` (a permutation of
+ * 0..num_blocks-1; NULL = ascending); freed blocks join the back in table order.
+ */
+PKV_API pkv_bm* pkv_bm_create(int num_blocks, int block_size, const int32_t* initial_order);
+PKV_API void pkv_bm_destroy(pkv_bm* bm);
+PKV_API int pkv_bm_num_blocks(const pkv_bm* bm);
+PKV_API int pkv_bm_block_size(const pkv_bm* bm);
+PKV_API int pkv_bm_num_free(const pkv_bm* bm);
+/* Copy the free list, front first, into host `out` (up to cap); returns the count. */
+PKV_API int pkv_bm_free_list(const pkv_bm* bm, int32_t* out, int cap);
+/* Take the front free block with reference count 1 (PKV_ERR_OOM if none). */
+PKV_API int pkv_bm_alloc(pkv_bm* bm, int32_t* block_out);
+PKV_API int pkv_bm_incref(pkv_bm* bm, int32_t block);   /* block must be live */
+PKV_API int pkv_bm_decref(pkv_bm* bm, int32_t block);   /* at 0 the block joins the free list */
+PKV_API int pkv_bm_refcount(const pkv_bm* bm, int32_t block);   /* >= 0, or PKV_ERR_INVALID */
+/*
+ * New sequence of num_tokens tokens.  Its first n_shared table entries are the
+ * given live blocks (a shared prefix; each gains a reference; they must be full:
+ * n_shared*block_size <= num_tokens); the rest are fresh blocks.  All-or-nothing.
+ */
+PKV_API int pkv_bm_add_seq(pkv_bm* bm, int64_t seq_id, int num_tokens, const int32_t* shared_prefix_blocks,
+                   int n_shared);
+/* Child gets a copy of the parent's table and length; every block gains a reference. */
+PKV_API int pkv_bm_fork(pkv_bm* bm, int64_t parent, int64_t child);
+/*
+ * One new token for each of the n sequences (distinct ids), in order.  For each:
+ * if its next position starts a block, a fresh block is appended; else if its last
+ * block is shared (reference count > 1) a fresh block replaces it, the pair
+ * (old, new) is appended to cow_pairs_out and old loses one reference.
+ * slots_out[i] = slot of the new token of seq_ids[i].
+ *   slots_out     host [n] int64
+ *   cow_pairs_out host [n, 2] int64 (capacity n pairs), *n_cow_out = pairs written;
+ *                 feed them to pkv_copy_blocks before writing the new tokens.
+ * All-or-nothing: PKV_ERR_OOM if the pool cannot cover every fresh block.
+ */
+PKV_API int pkv_bm_append_slots(pkv_bm* bm, const int64_t* seq_ids, int n, int64_t* slots_out,
+                        int64_t* cow_pairs_out, int* n_cow_out);
+/* Slots of positions start..start+count-1 of a sequence (host [count] int64). */
+PKV_API int pkv_bm_slots(const pkv_bm* bm, int64_t seq_id, int start, int count, int64_t* slots_out);
+/* Drop the sequence; each of its blocks loses a reference, in table order. */
+PKV_API int pkv_bm_free_seq(pkv_bm* bm, int64_t seq_id);
+PKV_API int pkv_bm_seq_len(const pkv_bm* bm, int64_t seq_id);      /* >= 0, or PKV_ERR_INVALID */
+PKV_API int pkv_bm_seq_blocks(const pkv_bm* bm, int64_t seq_id);   /* table length, or PKV_ERR_INVALID */
+/*
+ * Padded tables of the listed sequences: host tables [n, max_blocks] int32
+ * (padding 0) and host context_lens [n] int32.  PKV_ERR_INVALID if a table is
+ * longer than max_blocks or an id is unknown.
+ */
+PKV_API int pkv_bm_export_tables(const pkv_bm* bm, const int64_t* seq_ids, int n, int32_t* tables,
+                         int max_blocks, int32_t* context_lens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

@@ -1,0 +1,334 @@
+"""Python binding of libpkv.so, the B200 paged KV-cache decode library.
+
+A thin ctypes layer with the same names as the C ABI in ``include/pkv.h``: it
+checks tensor shapes/dtypes, passes raw pointers, sizes and the current CUDA
+stream, and turns return codes into exceptions.  Every step of the decode path
+runs in the library's kernels; nothing here computes.  If the library has not
+been built, importing the binding's entry points raises -- there is no fallback.
+
+PyTorch provides device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = [
+    "PKV_OK", "PKV_ERR_INVALID", "PKV_ERR_OOM", "PKV_ERR_CUDA", "PKV_ERR_UNSUPPORTED",
+    "PKV_DEV_BAD_SLOT", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_CONTEXT", "PKV_DEV_BAD_PAIR", "PKV_DEV_TIMEOUT",
+    "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR", "PkvError", "library", "library_path",
+    "reshape_and_cache", "copy_blocks", "paged_attention_workspace_size", "paged_attention_partition_tokens",
+    "paged_attention_decode", "BlockManager",
+]
+
+PKV_OK = 0
+PKV_ERR_INVALID = -1
+PKV_ERR_OOM = -2
+PKV_ERR_CUDA = -3
+PKV_ERR_UNSUPPORTED = -4
+PKV_DEV_BAD_SLOT = 0x1
+PKV_DEV_BAD_BLOCK = 0x2
+PKV_DEV_BAD_CONTEXT = 0x4
+PKV_DEV_BAD_PAIR = 0x8
+PKV_DEV_TIMEOUT = 0x10
+PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
+DTYPE_BF16, DTYPE_F32 = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libpkv.so")
+
+
+class PkvError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+_lib = None
+
+c_int, c_int64, c_size_t, c_float, c_void_p = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p
+P_i32 = ctypes.POINTER(ctypes.c_int32)
+P_i64 = ctypes.POINTER(ctypes.c_int64)
+
+_SIGNATURES = {
+    "pkv_last_error_string": (ctypes.c_char_p, []),
+    "pkv_version": (c_int, []),
+    "pkv_reshape_and_cache": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                                      c_int, c_void_p, c_void_p]),
+    "pkv_copy_blocks": (c_int, [ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_int, c_void_p, c_int, c_int,
+                                c_int64, c_void_p, c_void_p]),
+    "pkv_paged_attention_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int, c_int]),
+    "pkv_paged_attention_partition_tokens": (c_int, [c_int, c_int, c_int, c_int]),
+    "pkv_paged_attention_decode": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                           c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
+                                           c_void_p, c_size_t, c_void_p, c_void_p]),
+    "pkv_bm_create": (c_void_p, [c_int, c_int, c_void_p]),
+    "pkv_bm_destroy": (None, [c_void_p]),
+    "pkv_bm_num_blocks": (c_int, [c_void_p]),
+    "pkv_bm_block_size": (c_int, [c_void_p]),
+    "pkv_bm_num_free": (c_int, [c_void_p]),
+    "pkv_bm_free_list": (c_int, [c_void_p, c_void_p, c_int]),
+    "pkv_bm_alloc": (c_int, [c_void_p, P_i32]),
+    "pkv_bm_incref": (c_int, [c_void_p, ctypes.c_int32]),
+    "pkv_bm_decref": (c_int, [c_void_p, ctypes.c_int32]),
+    "pkv_bm_refcount": (c_int, [c_void_p, ctypes.c_int32]),
+    "pkv_bm_add_seq": (c_int, [c_void_p, c_int64, c_int, c_void_p, c_int]),
+    "pkv_bm_fork": (c_int, [c_void_p, c_int64, c_int64]),
+    "pkv_bm_append_slots": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, ctypes.POINTER(c_int)]),
+    "pkv_bm_slots": (c_int, [c_void_p, c_int64, c_int, c_int, c_void_p]),
+    "pkv_bm_free_seq": (c_int, [c_void_p, c_int64]),
+    "pkv_bm_seq_len": (c_int, [c_void_p, c_int64]),
+    "pkv_bm_seq_blocks": (c_int, [c_void_p, c_int64]),
+    "pkv_bm_export_tables": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p]),
+}
+
+
+def library():
+    """Load libpkv.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing; build it with `python -m paged_kv_cache_423_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != PKV_OK:
+        raise PkvError(rc, f"{what}: {library().pkv_last_error_string().decode()}")
+    return rc
+
+
+# ---------------------------------------------------------------------------
+# torch plumbing: pointers and streams only
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+# ---------------------------------------------------------------------------
+# Kernels
+# ---------------------------------------------------------------------------
+
+def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, status=None, stream=None):
+    """Write key/value [T, Hkv, D] bf16 into the pools [NB, Hkv, bs, D] at slot_mapping [T] int64."""
+    torch = _torch()
+    T, Hkv, D = key.shape
+    NB, Hkv2, bs, D2 = key_cache.shape
+    if value.shape != key.shape or value_cache.shape != key_cache.shape or (Hkv, D) != (Hkv2, D2):
+        raise ValueError("reshape_and_cache: shape mismatch")
+    if slot_mapping.shape != (T,):
+        raise ValueError("reshape_and_cache: slot_mapping must be [T]")
+    rc = library().pkv_reshape_and_cache(
+        _ptr(key, torch.bfloat16, "key"), _ptr(value, torch.bfloat16, "value"),
+        _ptr(key_cache, torch.bfloat16, "key_cache"), _ptr(value_cache, torch.bfloat16, "value_cache"),
+        _ptr(slot_mapping, torch.int64, "slot_mapping"), T, NB, Hkv, D, bs,
+        _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "reshape_and_cache")
+
+
+def copy_blocks(key_caches, value_caches, block_mapping, status=None, stream=None):
+    """Copy (src, dst) blocks of block_mapping [n, 2] int64 in every layer's K and V pool."""
+    torch = _torch()
+    if len(key_caches) != len(value_caches):
+        raise ValueError("copy_blocks: layer count mismatch")
+    n = int(block_mapping.shape[0]) if block_mapping.numel() else 0
+    if block_mapping.numel() and tuple(block_mapping.shape) != (n, 2):
+        raise ValueError("copy_blocks: block_mapping must be [n, 2]")
+    if not key_caches:
+        return
+    NB = key_caches[0].shape[0]
+    block_elems = int(np.prod(key_caches[0].shape[1:]))
+    for kc, vc in zip(key_caches, value_caches):
+        if kc.shape != key_caches[0].shape or vc.shape != key_caches[0].shape:
+            raise ValueError("copy_blocks: every pool must have the same shape")
+    ks = (c_void_p * len(key_caches))(*[_ptr(k, torch.bfloat16, "key_cache").value for k in key_caches])
+    vs = (c_void_p * len(value_caches))(*[_ptr(v, torch.bfloat16, "value_cache").value for v in value_caches])
+    mapping = _ptr(block_mapping, torch.int64, "block_mapping") if n else c_void_p(0)
+    rc = library().pkv_copy_blocks(ks, vs, len(key_caches), mapping, n, NB, block_elems,
+                                   _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "copy_blocks")
+
+
+def paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                                   partition_tokens=0) -> int:
+    n = library().pkv_paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                     max_context_len, partition_tokens)
+    if n == 0:
+        raise PkvError(PKV_ERR_INVALID, "paged_attention_workspace_size: bad arguments")
+    return int(n)
+
+
+def paged_attention_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len) -> int:
+    r = library().pkv_paged_attention_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len)
+    if r < 0:
+        _check(r, "paged_attention_partition_tokens")
+    return int(r)
+
+
+def paged_attention_decode(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len, scale,
+                           workspace, partition_tokens=0, path=PATH_AUTO, status=None, stream=None):
+    """Decode attention: out [B, Hq, D] (bf16 or f32) from query [B, Hq, D] bf16 over the paged pools.
+
+    block_tables [B, max_blocks] int32, context_lens [B] int32 (device), max_context_len
+    a host bound, workspace a uint8 device tensor of paged_attention_workspace_size bytes."""
+    torch = _torch()
+    B, Hq, D = query.shape
+    NB, Hkv, bs, D2 = key_cache.shape
+    if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
+        raise ValueError("paged_attention_decode: shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("paged_attention_decode: block_tables must be [B, max_blocks], context_lens [B]")
+    if out.dtype == torch.bfloat16:
+        out_dtype = DTYPE_BF16
+    elif out.dtype == torch.float32:
+        out_dtype = DTYPE_F32
+    else:
+        raise TypeError("paged_attention_decode: out must be bf16 or f32")
+    rc = library().pkv_paged_attention_decode(
+        _ptr(out, None, "out"), out_dtype, _ptr(query, torch.bfloat16, "query"),
+        _ptr(key_cache, torch.bfloat16, "key_cache"), _ptr(value_cache, torch.bfloat16, "value_cache"),
+        _ptr(block_tables, torch.int32, "block_tables"), int(block_tables.shape[1]),
+        _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len), B, Hq, Hkv, D, bs, NB,
+        float(scale), int(partition_tokens), int(path), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "paged_attention_decode")
+
+
+# ---------------------------------------------------------------------------
+# Host block manager
+# ---------------------------------------------------------------------------
+
+def _np_ptr(a):
+    return c_void_p(a.ctypes.data) if a is not None and a.size else c_void_p(0)
+
+
+class BlockManager:
+    """Free list + reference counts + per-sequence block tables (host, C++)."""
+
+    def __init__(self, num_blocks: int, block_size: int, initial_order=None):
+        lib = library()
+        order = None if initial_order is None else np.ascontiguousarray(initial_order, dtype=np.int32)
+        if order is not None and order.shape != (num_blocks,):
+            raise ValueError("initial_order must have num_blocks entries")
+        h = lib.pkv_bm_create(num_blocks, block_size, _np_ptr(order) if order is not None else None)
+        if not h:
+            raise PkvError(PKV_ERR_INVALID, lib.pkv_last_error_string().decode())
+        self._h = c_void_p(h)
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if getattr(self, "_h", None):
+            library().pkv_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def num_free(self) -> int:
+        return library().pkv_bm_num_free(self._h)
+
+    def free_list(self) -> list[int]:
+        buf = np.zeros(self.num_blocks, np.int32)
+        n = library().pkv_bm_free_list(self._h, _np_ptr(buf), self.num_blocks)
+        return buf[:n].tolist()
+
+    def alloc(self) -> int:
+        b = ctypes.c_int32()
+        _check(library().pkv_bm_alloc(self._h, ctypes.byref(b)), "bm_alloc")
+        return b.value
+
+    def incref(self, block: int):
+        _check(library().pkv_bm_incref(self._h, block), "bm_incref")
+
+    def decref(self, block: int):
+        _check(library().pkv_bm_decref(self._h, block), "bm_decref")
+
+    def refcount(self, block: int) -> int:
+        r = library().pkv_bm_refcount(self._h, block)
+        if r < 0:
+            _check(r, "bm_refcount")
+        return r
+
+    def add_seq(self, seq_id: int, num_tokens: int, shared_prefix_blocks=()):
+        shared = np.ascontiguousarray(list(shared_prefix_blocks), dtype=np.int32)
+        _check(library().pkv_bm_add_seq(self._h, seq_id, num_tokens, _np_ptr(shared), len(shared)), "bm_add_seq")
+
+    def fork(self, parent: int, child: int):
+        _check(library().pkv_bm_fork(self._h, parent, child), "bm_fork")
+
+    def append_slots(self, seq_ids):
+        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        slots = np.zeros(len(ids), np.int64)
+        pairs = np.zeros((max(len(ids), 1), 2), np.int64)
+        n_cow = c_int(0)
+        _check(library().pkv_bm_append_slots(self._h, _np_ptr(ids), len(ids), _np_ptr(slots), _np_ptr(pairs),
+                                             ctypes.byref(n_cow)), "bm_append_slots")
+        return slots, pairs[:n_cow.value].copy()
+
+    def slots(self, seq_id: int, start: int, count: int) -> np.ndarray:
+        out = np.zeros(count, np.int64)
+        _check(library().pkv_bm_slots(self._h, seq_id, start, count, _np_ptr(out)), "bm_slots")
+        return out
+
+    def free_seq(self, seq_id: int):
+        _check(library().pkv_bm_free_seq(self._h, seq_id), "bm_free_seq")
+
+    def seq_len(self, seq_id: int) -> int:
+        r = library().pkv_bm_seq_len(self._h, seq_id)
+        if r < 0:
+            _check(r, "bm_seq_len")
+        return r
+
+    def seq_blocks(self, seq_id: int) -> int:
+        r = library().pkv_bm_seq_blocks(self._h, seq_id)
+        if r < 0:
+            _check(r, "bm_seq_blocks")
+        return r
+
+    def export_tables(self, seq_ids, max_blocks: int):
+        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        tables = np.zeros((len(ids), max_blocks), np.int32)
+        lens = np.zeros(len(ids), np.int32)
+        _check(library().pkv_bm_export_tables(self._h, _np_ptr(ids), len(ids), _np_ptr(tables), max_blocks,
+                                              _np_ptr(lens)), "bm_export_tables")
+        return tables, lens

@@ -1,0 +1,278 @@
+// Host block manager: FIFO free list, per-block reference counts and per-sequence
+// block tables.
+//
+// Outcome School vLLM explainer, "vLLM的核心创新：PagedAttention": blocks are taken
+// only when a request needs room, need not be contiguous, are recorded in order in
+// the request's block table, and all go back to the shared pool when it finishes;
+// "内存共享": identical prefixes and beams point their tables at the same blocks.
+// The copy-on-write rule for a shared, partially filled last block and the FIFO
+// order of the free list are this library's readings (documented in pkv.h).
+#include <deque>
+#include <new>
+#include <unordered_map>
+#include <utility>
+#include <vector>
+
+#include "pkv_internal.h"
+
+using pkv::set_error;
+
+struct pkv_bm {
+  struct Seq {
+    std::vector<int32_t> table;
+    int len = 0;
+  };
+  int num_blocks = 0;
+  int block_size = 0;
+  std::deque<int32_t> free_list;
+  std::vector<int32_t> ref;
+  std::unordered_map<int64_t, Seq> seqs;
+  // Scratch for the dry run of append_slots: per-block pending reference change.
+  std::vector<int32_t> pending;
+  std::vector<int32_t> touched;
+
+  bool valid_block(int32_t b) const { return b >= 0 && b < num_blocks; }
+  int blocks_for(int tokens) const { return (tokens + block_size - 1) / block_size; }
+
+  int32_t take() {
+    int32_t b = free_list.front();
+    free_list.pop_front();
+    ref[b] = 1;
+    return b;
+  }
+  void drop(int32_t b) {
+    if (--ref[b] == 0) free_list.push_back(b);
+  }
+};
+
+extern "C" pkv_bm* pkv_bm_create(int num_blocks, int block_size, const int32_t* initial_order) {
+  if (num_blocks <= 0 || block_size <= 0) {
+    set_error(PKV_ERR_INVALID, "pkv_bm_create: num_blocks and block_size must be positive");
+    return nullptr;
+  }
+  pkv_bm* bm = new (std::nothrow) pkv_bm();
+  if (!bm) {
+    set_error(PKV_ERR_OOM, "pkv_bm_create: host allocation failed");
+    return nullptr;
+  }
+  bm->num_blocks = num_blocks;
+  bm->block_size = block_size;
+  bm->ref.assign(num_blocks, 0);
+  bm->pending.assign(num_blocks, 0);
+  if (initial_order) {
+    std::vector<char> seen(num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+      int32_t b = initial_order[i];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete bm;
+        set_error(PKV_ERR_INVALID, "pkv_bm_create: initial_order is not a permutation of 0..%d", num_blocks - 1);
+        return nullptr;
+      }
+      seen[b] = 1;
+      bm->free_list.push_back(b);
+    }
+  } else {
+    for (int i = 0; i < num_blocks; ++i) bm->free_list.push_back(i);
+  }
+  return bm;
+}
+
+extern "C" void pkv_bm_destroy(pkv_bm* bm) { delete bm; }
+
+extern "C" int pkv_bm_num_blocks(const pkv_bm* bm) { return bm ? bm->num_blocks : PKV_ERR_INVALID; }
+extern "C" int pkv_bm_block_size(const pkv_bm* bm) { return bm ? bm->block_size : PKV_ERR_INVALID; }
+extern "C" int pkv_bm_num_free(const pkv_bm* bm) {
+  return bm ? static_cast<int>(bm->free_list.size()) : PKV_ERR_INVALID;
+}
+
+extern "C" int pkv_bm_free_list(const pkv_bm* bm, int32_t* out, int cap) {
+  if (!bm || (cap > 0 && !out)) return set_error(PKV_ERR_INVALID, "pkv_bm_free_list: bad arguments");
+  int n = 0;
+  for (int32_t b : bm->free_list) {
+    if (n >= cap) break;
+    out[n++] = b;
+  }
+  return n;
+}
+
+extern "C" int pkv_bm_alloc(pkv_bm* bm, int32_t* block_out) {
+  if (!bm || !block_out) return set_error(PKV_ERR_INVALID, "pkv_bm_alloc: bad arguments");
+  if (bm->free_list.empty()) return set_error(PKV_ERR_OOM, "pkv_bm_alloc: pool exhausted");
+  *block_out = bm->take();
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_incref(pkv_bm* bm, int32_t block) {
+  if (!bm || !bm->valid_block(block) || bm->ref[block] <= 0)
+    return set_error(PKV_ERR_INVALID, "pkv_bm_incref: block %d is not live", block);
+  ++bm->ref[block];
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_decref(pkv_bm* bm, int32_t block) {
+  if (!bm || !bm->valid_block(block) || bm->ref[block] <= 0)
+    return set_error(PKV_ERR_INVALID, "pkv_bm_decref: block %d is not live", block);
+  bm->drop(block);
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_refcount(const pkv_bm* bm, int32_t block) {
+  if (!bm || !bm->valid_block(block)) return set_error(PKV_ERR_INVALID, "pkv_bm_refcount: bad block %d", block);
+  return bm->ref[block];
+}
+
+extern "C" int pkv_bm_add_seq(pkv_bm* bm, int64_t seq_id, int num_tokens, const int32_t* shared_prefix_blocks,
+                              int n_shared) {
+  if (!bm || num_tokens < 0 || n_shared < 0 || (n_shared > 0 && !shared_prefix_blocks))
+    return set_error(PKV_ERR_INVALID, "pkv_bm_add_seq: bad arguments");
+  if (bm->seqs.count(seq_id)) return set_error(PKV_ERR_INVALID, "pkv_bm_add_seq: sequence %lld exists", (long long)seq_id);
+  if (static_cast<int64_t>(n_shared) * bm->block_size > num_tokens)
+    return set_error(PKV_ERR_INVALID, "pkv_bm_add_seq: shared prefix longer than the sequence");
+  for (int i = 0; i < n_shared; ++i) {
+    int32_t b = shared_prefix_blocks[i];
+    if (!bm->valid_block(b) || bm->ref[b] <= 0)
+      return set_error(PKV_ERR_INVALID, "pkv_bm_add_seq: shared block %d is not live", b);
+  }
+  int fresh = bm->blocks_for(num_tokens) - n_shared;
+  if (fresh > static_cast<int>(bm->free_list.size()))
+    return set_error(PKV_ERR_OOM, "pkv_bm_add_seq: pool exhausted (%d blocks needed, %zu free)", fresh,
+                     bm->free_list.size());
+  pkv_bm::Seq seq;
+  seq.table.reserve(n_shared + fresh);
+  for (int i = 0; i < n_shared; ++i) {
+    ++bm->ref[shared_prefix_blocks[i]];
+    seq.table.push_back(shared_prefix_blocks[i]);
+  }
+  for (int i = 0; i < fresh; ++i) seq.table.push_back(bm->take());
+  seq.len = num_tokens;
+  bm->seqs.emplace(seq_id, std::move(seq));
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_fork(pkv_bm* bm, int64_t parent, int64_t child) {
+  if (!bm) return set_error(PKV_ERR_INVALID, "pkv_bm_fork: null manager");
+  auto it = bm->seqs.find(parent);
+  if (it == bm->seqs.end() || bm->seqs.count(child))
+    return set_error(PKV_ERR_INVALID, "pkv_bm_fork: unknown parent %lld or existing child %lld", (long long)parent,
+                     (long long)child);
+  pkv_bm::Seq copy = it->second;
+  for (int32_t b : copy.table) ++bm->ref[b];
+  bm->seqs.emplace(child, std::move(copy));
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_append_slots(pkv_bm* bm, const int64_t* seq_ids, int n, int64_t* slots_out,
+                                   int64_t* cow_pairs_out, int* n_cow_out) {
+  if (!bm || n < 0 || (n > 0 && (!seq_ids || !slots_out || !cow_pairs_out)) || !n_cow_out)
+    return set_error(PKV_ERR_INVALID, "pkv_bm_append_slots: bad arguments");
+  *n_cow_out = 0;
+  // Validate ids (known, distinct) and resolve them once.
+  std::vector<pkv_bm::Seq*> seqs(n);
+  std::unordered_map<int64_t, int> seen;
+  seen.reserve(static_cast<size_t>(n) * 2);
+  for (int i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end() || !seen.emplace(seq_ids[i], i).second)
+      return set_error(PKV_ERR_INVALID, "pkv_bm_append_slots: unknown or repeated sequence %lld", (long long)seq_ids[i]);
+    seqs[i] = &it->second;
+  }
+  // Dry run: count fresh blocks, following reference counts as earlier sequences
+  // of this call give up their share of a block.
+  int need = 0;
+  for (int i = 0; i < n; ++i) {
+    pkv_bm::Seq& s = *seqs[i];
+    if (s.len % bm->block_size == 0) {
+      ++need;
+    } else {
+      int32_t last = s.table.back();
+      if (bm->ref[last] + bm->pending[last] > 1) {
+        ++need;
+        if (bm->pending[last] == 0) bm->touched.push_back(last);
+        --bm->pending[last];
+      }
+    }
+  }
+  for (int32_t b : bm->touched) bm->pending[b] = 0;
+  bm->touched.clear();
+  if (need > static_cast<int>(bm->free_list.size()))
+    return set_error(PKV_ERR_OOM, "pkv_bm_append_slots: pool exhausted (%d blocks needed, %zu free)", need,
+                     bm->free_list.size());
+  int n_cow = 0;
+  for (int i = 0; i < n; ++i) {
+    pkv_bm::Seq& s = *seqs[i];
+    const int row = s.len % bm->block_size;
+    if (row == 0) {
+      s.table.push_back(bm->take());
+    } else if (bm->ref[s.table.back()] > 1) {
+      int32_t old = s.table.back();
+      int32_t fresh = bm->take();
+      cow_pairs_out[2 * n_cow] = old;
+      cow_pairs_out[2 * n_cow + 1] = fresh;
+      ++n_cow;
+      bm->drop(old);
+      s.table.back() = fresh;
+    }
+    slots_out[i] = static_cast<int64_t>(s.table.back()) * bm->block_size + row;
+    ++s.len;
+  }
+  *n_cow_out = n_cow;
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_slots(const pkv_bm* bm, int64_t seq_id, int start, int count, int64_t* slots_out) {
+  if (!bm || start < 0 || count < 0 || (count > 0 && !slots_out))
+    return set_error(PKV_ERR_INVALID, "pkv_bm_slots: bad arguments");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end() || static_cast<int64_t>(start) + count > it->second.len)
+    return set_error(PKV_ERR_INVALID, "pkv_bm_slots: unknown sequence or range past its length");
+  const auto& table = it->second.table;
+  for (int i = 0; i < count; ++i) {
+    int p = start + i;
+    slots_out[i] = static_cast<int64_t>(table[p / bm->block_size]) * bm->block_size + p % bm->block_size;
+  }
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_free_seq(pkv_bm* bm, int64_t seq_id) {
+  if (!bm) return set_error(PKV_ERR_INVALID, "pkv_bm_free_seq: null manager");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) return set_error(PKV_ERR_INVALID, "pkv_bm_free_seq: unknown sequence %lld", (long long)seq_id);
+  for (int32_t b : it->second.table) bm->drop(b);
+  bm->seqs.erase(it);
+  return PKV_OK;
+}
+
+extern "C" int pkv_bm_seq_len(const pkv_bm* bm, int64_t seq_id) {
+  if (!bm) return set_error(PKV_ERR_INVALID, "pkv_bm_seq_len: null manager");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) return set_error(PKV_ERR_INVALID, "pkv_bm_seq_len: unknown sequence");
+  return it->second.len;
+}
+
+extern "C" int pkv_bm_seq_blocks(const pkv_bm* bm, int64_t seq_id) {
+  if (!bm) return set_error(PKV_ERR_INVALID, "pkv_bm_seq_blocks: null manager");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) return set_error(PKV_ERR_INVALID, "pkv_bm_seq_blocks: unknown sequence");
+  return static_cast<int>(it->second.table.size());
+}
+
+extern "C" int pkv_bm_export_tables(const pkv_bm* bm, const int64_t* seq_ids, int n, int32_t* tables,
+                                    int max_blocks, int32_t* context_lens) {
+  if (!bm || n < 0 || max_blocks < 0 || (n > 0 && (!seq_ids || !context_lens || (max_blocks > 0 && !tables))))
+    return set_error(PKV_ERR_INVALID, "pkv_bm_export_tables: bad arguments");
+  for (int i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end() || static_cast<int>(it->second.table.size()) > max_blocks)
+      return set_error(PKV_ERR_INVALID, "pkv_bm_export_tables: unknown sequence %lld or table longer than %d",
+                       (long long)seq_ids[i], max_blocks);
+  }
+  for (int i = 0; i < n; ++i) {
+    const auto& s = bm->seqs.find(seq_ids[i])->second;
+    int32_t* row = tables + static_cast<size_t>(i) * max_blocks;
+    size_t k = 0;
+    for (; k < s.table.size(); ++k) row[k] = s.table[k];
+    for (; k < static_cast<size_t>(max_blocks); ++k) row[k] = 0;
+    context_lens[i] = s.len;
+  }
+  return PKV_OK;
+}

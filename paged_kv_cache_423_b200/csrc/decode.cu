@@ -1,0 +1,571 @@
+// Paged decode attention: the work plan, the CUDA-core streaming kernel and the
+// C-ABI entry points.
+//
+// What is computed (intelliparadigm article "PagedAttention：操作系统分页思想的跨界创新",
+// §2.1, paged_attention pseudo-code): for each sequence and query head, the logical
+// block of token t is t // block_size, the block table gives its physical block,
+// K and V are read from there, and the output is softmax(scale * q·Kᵀ)·V over the
+// sequence's context.  §2.1 also states the kernel idea this file keeps: splice the
+// non-contiguous pages on the fly through shared memory, with prefetch.
+//
+// How it maps to sm_100a:
+//   * plan kernel (one CTA): splits every sequence into partitions of at most
+//     `partition` tokens and counting-sorts the (sequence, partition) entries by
+//     length, longest first, so the persistent kernel hands out big items first and
+//     fills the tail with small ones.
+//   * streaming kernel (persistent, CUDA cores): every warp is an independent
+//     consumer with its own ring of shared-memory stages.  Lane 0 streams 16-token
+//     slices of (block, kv head) tiles into the ring with 1-D bulk copies (TMA
+//     engine, mbarrier completion), several stages ahead of the math, and runs ahead
+//     across item boundaries (block-table slices of the next item are prefetched one
+//     item early).  Scores use a transposed warp reduction (one shuffle per token),
+//     the softmax is online in fp32 and base 2, P·V accumulates in fp32 registers.
+//   * split partitions write an unnormalised partial (o, m, l); the last partition
+//     of a (sequence, head) to arrive (device-scope atomic counter) merges all
+//     partials by log-sum-exp rescaling and writes the output, so there is no
+//     separate reduce launch.  No thread ever waits for another CTA.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "decode_common.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// Plan kernel
+// ---------------------------------------------------------------------------
+
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads)
+    plan_kernel(const int32_t* __restrict__ context_lens, int num_seqs, int max_context_len, int max_table_tokens,
+                int partition, PlanEntry* __restrict__ entries, int32_t* __restrict__ plan_count,
+                int32_t* __restrict__ arrive, int n_arrive, int32_t* status) {
+  __shared__ int bucket[kMaxPartition + 1];  // bucket k holds entries of partition - k tokens
+  __shared__ int warp_total[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i <= partition; i += blockDim.x) bucket[i] = 0;
+  for (int i = tid; i < n_arrive; i += blockDim.x) arrive[i] = 0;
+  __syncthreads();
+  for (int s = tid; s < num_seqs; s += blockDim.x) {
+    int L = context_lens[s];
+    if (L < 0 || L > max_context_len || L > max_table_tokens) {
+      set_status(status, PKV_DEV_BAD_CONTEXT);
+      L = 0;
+    }
+    const int np = L == 0 ? 1 : (L + partition - 1) / partition;
+    for (int p = 0; p < np; ++p) {
+      const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
+      atomicAdd(&bucket[partition - ntok], 1);
+    }
+  }
+  __syncthreads();
+  // Exclusive scan of the bucket counts (partition + 1 <= 513 <= 1024 threads).
+  const int v = tid <= partition ? bucket[tid] : 0;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_total[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (blockDim.x >> 5) ? warp_total[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_total[lane] = w;
+  }
+  __syncthreads();
+  const int excl = x - v + (warp > 0 ? warp_total[warp - 1] : 0);
+  __syncthreads();
+  if (tid <= partition) bucket[tid] = excl;
+  if (tid == 0) plan_count[0] = warp_total[31];
+  __syncthreads();
+  for (int s = tid; s < num_seqs; s += blockDim.x) {
+    int L = context_lens[s];
+    if (L < 0 || L > max_context_len || L > max_table_tokens) L = 0;
+    const int np = L == 0 ? 1 : (L + partition - 1) / partition;
+    for (int p = 0; p < np; ++p) {
+      const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
+      const int pos = atomicAdd(&bucket[partition - ntok], 1);
+      entries[pos] = make_int4(s, p, np, L);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core streaming kernel
+// ---------------------------------------------------------------------------
+
+template <int D, int STAGES>
+struct __align__(128) WarpRing {
+  __nv_bfloat16 k[STAGES][kStageTokens * D];
+  __nv_bfloat16 v[STAGES][kStageTokens * D];
+  __nv_bfloat16 q[STAGES][D];
+  uint64_t full[STAGES];
+  int4 meta[STAGES];  // x seq, y query head, z part | nparts << 16, w n_valid | first << 8 | last << 9
+};
+
+// Per-item state of the issuing side (warp-uniform except `table`).
+struct IssueItem {
+  int64_t id;      // item index, or -1 when there is none
+  PlanEntry e;     // seq, part, nparts, L
+  int table;       // lane j: physical block of the item's j-th block (prefetched)
+};
+
+__device__ __forceinline__ int item_stages(const PlanEntry& e, int partition) {
+  const int ntok = e.w == 0 ? 0 : min(partition, e.w - e.y * partition);
+  return ntok == 0 ? 1 : (ntok + kStageTokens - 1) / kStageTokens;
+}
+
+// Load lane j's table entry for the item (block tok0/bs + j), 0 past the item.
+__device__ __forceinline__ int load_item_table(const DecodeArgs& a, const PlanEntry& e, int lane) {
+  const int tok0 = e.y * a.partition;
+  const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - tok0);
+  const int nblk = (ntok + a.block_size - 1) / a.block_size;
+  if (lane >= nblk) return 0;
+  return __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + lane);
+}
+
+template <int D, bool OUT_F32>
+__device__ __forceinline__ void store_row(const DecodeArgs& a, int seq, int qh, int lane, const float* o,
+                                          float inv) {
+  constexpr int EPL = D / 32;
+  const int64_t base = (static_cast<int64_t>(seq) * a.num_heads + qh) * D + lane * EPL;
+  if constexpr (OUT_F32) {
+    float* out = static_cast<float*>(a.out) + base;
+    if constexpr (EPL == 4)
+      *reinterpret_cast<float4*>(out) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+    else
+      *reinterpret_cast<float2*>(out) = make_float2(o[0] * inv, o[1] * inv);
+  } else {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + base;
+    if constexpr (EPL == 4)
+      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv));
+    else
+      *reinterpret_cast<uint32_t*>(out) = pack_bf16x2(o[0] * inv, o[1] * inv);
+  }
+}
+
+template <int D, bool OUT_F32, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int EPL = D / 32;                                  // elements per lane: 2 or 4
+  constexpr uint32_t kKVBytes = kStageTokens * D * sizeof(__nv_bfloat16);
+  constexpr uint32_t kQBytes = D * sizeof(__nv_bfloat16);
+  using Ring = WarpRing<D, STAGES>;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Ring& ring = reinterpret_cast<Ring*>(smem_raw)[warp];
+
+  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_heads;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * WARPS;
+  const int64_t first_item = static_cast<int64_t>(blockIdx.x) * WARPS + warp;
+  if (first_item >= n_items) return;
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) mbar_init(&ring.full[s], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const uint64_t policy = l2_policy_evict_first();
+
+  // ---- issuing side: current item, next item (table prefetched), item after (entry prefetched)
+  auto entry_of = [&](int64_t id) -> PlanEntry {
+    return id < n_items ? a.entries[id / a.num_heads] : make_int4(0, 0, 0, 0);
+  };
+  IssueItem cur, nxt;
+  PlanEntry nx2_e;
+  int64_t nx2_id;
+  cur.id = first_item;
+  cur.e = entry_of(cur.id);
+  cur.table = load_item_table(a, cur.e, lane);
+  nxt.id = first_item + stride < n_items ? first_item + stride : -1;
+  nxt.e = entry_of(first_item + stride);
+  nxt.table = nxt.id >= 0 ? load_item_table(a, nxt.e, lane) : 0;
+  nx2_id = first_item + 2 * stride < n_items ? first_item + 2 * stride : -1;
+  nx2_e = entry_of(first_item + 2 * stride);
+  int cur_stage = 0;
+  int cur_nstages = item_stages(cur.e, a.partition);
+  bool issue_done = false;
+
+  // Issue the next stage into `slot`; false when every item has been issued.
+  auto issue = [&](int slot) -> bool {
+    if (issue_done) return false;
+    if (cur_stage == cur_nstages) {
+      if (nxt.id < 0) {
+        issue_done = true;
+        return false;
+      }
+      cur = nxt;
+      nxt.id = nx2_id;
+      nxt.e = nx2_e;
+      nxt.table = nxt.id >= 0 ? load_item_table(a, nxt.e, lane) : 0;
+      nx2_id = nx2_id >= 0 && nx2_id + stride < n_items ? nx2_id + stride : -1;
+      nx2_e = entry_of(nx2_id >= 0 ? nx2_id : n_items);
+      cur_stage = 0;
+      cur_nstages = item_stages(cur.e, a.partition);
+    }
+    const PlanEntry e = cur.e;
+    const int qh = static_cast<int>(cur.id % a.num_heads);
+    const int kvh = qh / a.group;
+    const int tok = e.y * a.partition + cur_stage * kStageTokens;        // first token of the stage
+    const int n_tok = e.w == 0 ? 0 : min(kStageTokens, e.w - tok);
+    const int local_tok = cur_stage * kStageTokens;
+    const int phys = __shfl_sync(kFull, cur.table, local_tok / a.block_size);
+    const bool ok = n_tok > 0 && phys >= 0 && phys < a.num_blocks;
+    const bool first = cur_stage == 0, last = cur_stage == cur_nstages - 1;
+    const bool with_q = first && n_tok > 0;
+    if (lane == 0) {
+      if (n_tok > 0 && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
+      ring.meta[slot] = make_int4(e.x, qh, e.y | (e.z << 16),
+                                  (ok ? n_tok : 0) | (first ? 0x100 : 0) | (last ? 0x200 : 0) | (with_q ? 0x400 : 0));
+      const uint32_t bytes = (ok ? 2 * kKVBytes : 0) + (with_q ? kQBytes : 0);
+      mbar_arrive_expect_tx(&ring.full[slot], bytes);
+      if (with_q)
+        bulk_copy_g2s(ring.q[slot], a.query + (static_cast<int64_t>(e.x) * a.num_heads + qh) * D, kQBytes,
+                      &ring.full[slot], policy);
+      if (ok) {
+        const int64_t row = (static_cast<int64_t>(phys) * a.num_kv_heads + kvh) * a.block_size + local_tok % a.block_size;
+        bulk_copy_g2s(ring.k[slot], a.key_cache + row * D, kKVBytes, &ring.full[slot], policy);
+        bulk_copy_g2s(ring.v[slot], a.value_cache + row * D, kKVBytes, &ring.full[slot], policy);
+      }
+    }
+    ++cur_stage;
+    return true;
+  };
+
+  // ---- consuming side
+  float qf[EPL], o[EPL];
+  float m = -INFINITY, lsum = 0.f;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) qf[j] = o[j] = 0.f;
+
+  int issued = 0;
+  for (int s = 0; s < STAGES; ++s) {
+    if (!issue(s)) break;
+    ++issued;
+  }
+  int consumed = 0;
+  bool timed_out = false;
+  while (consumed < issued) {
+    const int slot = consumed % STAGES;
+    if (!mbar_wait(&ring.full[slot], (consumed / STAGES) & 1)) {
+      timed_out = true;
+      break;
+    }
+    const int4 mt = ring.meta[slot];
+    const int n_valid = mt.w & 0xff;
+    const bool first = mt.w & 0x100, last = mt.w & 0x200;
+    if (first) {
+      m = -INFINITY;
+      lsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) o[j] = 0.f;
+      if (mt.w & 0x400) {
+        const __nv_bfloat16* qs = ring.q[slot] + lane * EPL;
+        if constexpr (EPL == 4) {
+          const uint2 w = *reinterpret_cast<const uint2*>(qs);
+          qf[0] = bf16lo(w.x) * a.scale_log2;
+          qf[1] = bf16hi(w.x) * a.scale_log2;
+          qf[2] = bf16lo(w.y) * a.scale_log2;
+          qf[3] = bf16hi(w.y) * a.scale_log2;
+        } else {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(qs);
+          qf[0] = bf16lo(w) * a.scale_log2;
+          qf[1] = bf16hi(w) * a.scale_log2;
+        }
+      }
+    }
+    if (n_valid > 0) {
+      // Scores of the 16 rows: per-lane partial dot products over EPL dims.
+      const __nv_bfloat16* kb = ring.k[slot] + lane * EPL;
+      float sc[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        if constexpr (EPL == 4) {
+          const uint2 w = *reinterpret_cast<const uint2*>(kb + t * D);
+          sc[t] = fmaf(qf[3], bf16hi(w.y), fmaf(qf[2], bf16lo(w.y), fmaf(qf[1], bf16hi(w.x), qf[0] * bf16lo(w.x))));
+        } else {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(kb + t * D);
+          sc[t] = fmaf(qf[1], bf16hi(w), qf[0] * bf16lo(w));
+        }
+      }
+      // Transposed reduction: after the steps on lane bits 4..1 lane holds the sum
+      // over 16 lanes of row (lane >> 1); the xor-1 step completes it.
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? sc[i] : sc[i + 8];
+        const float keep = up ? sc[i + 8] : sc[i];
+        sc[i] = keep + __shfl_xor_sync(kFull, send, 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? sc[i] : sc[i + 4];
+        const float keep = up ? sc[i + 4] : sc[i];
+        sc[i] = keep + __shfl_xor_sync(kFull, send, 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? sc[i] : sc[i + 2];
+        const float keep = up ? sc[i + 2] : sc[i];
+        sc[i] = keep + __shfl_xor_sync(kFull, send, 4);
+      }
+      {
+        const bool up = lane & 2;
+        const float send = up ? sc[0] : sc[1];
+        const float keep = up ? sc[1] : sc[0];
+        sc[0] = keep + __shfl_xor_sync(kFull, send, 2);
+      }
+      sc[0] += __shfl_xor_sync(kFull, sc[0], 1);
+      const bool valid = (lane >> 1) < n_valid;
+      const float x = valid ? sc[0] : -INFINITY;
+      float mx = x;
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+      const float m_new = fmaxf(m, mx);
+      const float alpha = exp2f(m - m_new);
+      const float p = valid ? exp2f(x - m_new) : 0.f;
+      m = m_new;
+      lsum = fmaf(lsum, alpha, p);
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) o[j] *= alpha;
+      const __nv_bfloat16* vb = ring.v[slot] + lane * EPL;
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const float pt = __shfl_sync(kFull, p, 2 * t);
+        if (t < n_valid) {
+          if constexpr (EPL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(vb + t * D);
+            o[0] = fmaf(pt, bf16lo(w.x), o[0]);
+            o[1] = fmaf(pt, bf16hi(w.x), o[1]);
+            o[2] = fmaf(pt, bf16lo(w.y), o[2]);
+            o[3] = fmaf(pt, bf16hi(w.y), o[3]);
+          } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(vb + t * D);
+            o[0] = fmaf(pt, bf16lo(w), o[0]);
+            o[1] = fmaf(pt, bf16hi(w), o[1]);
+          }
+        }
+      }
+    }
+    if (last) {
+      const int seq = mt.x, qh = mt.y, part = mt.z & 0xffff, nparts = mt.z >> 16;
+      float l = lsum;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
+      l *= 0.5f;  // every row was counted by its two lanes
+      if (nparts == 1) {
+        store_row<D, OUT_F32>(a, seq, qh, lane, o, l > 0.f ? 1.f / l : 0.f);
+      } else {
+        const int64_t unit = static_cast<int64_t>(seq) * a.num_heads + qh;
+        const int64_t pidx = unit * a.max_parts + part;
+        float* po = a.part_o + pidx * D + lane * EPL;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) po[j] = o[j];
+        if (lane == 0) a.part_ml[pidx] = make_float2(m, l);
+        __threadfence();
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(a.arrive + unit, 1);
+        prev = __shfl_sync(kFull, prev, 0);
+        if (prev == nparts - 1) {
+          // Last partition in: merge every partial of this (sequence, head).
+          __threadfence();
+          const float2* ml = a.part_ml + unit * a.max_parts;
+          float M = -INFINITY;
+          for (int p = 0; p < nparts; ++p) M = fmaxf(M, __ldcg(&ml[p].x));
+          float acc[EPL], Ls = 0.f;
+#pragma unroll
+          for (int j = 0; j < EPL; ++j) acc[j] = 0.f;
+          const float* pb = a.part_o + unit * a.max_parts * D + lane * EPL;
+          for (int p = 0; p < nparts; ++p) {
+            const float2 mlp = __ldcg(&ml[p]);
+            const float w = exp2f(mlp.x - M);
+            Ls = fmaf(w, mlp.y, Ls);
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) acc[j] = fmaf(w, __ldcg(pb + static_cast<int64_t>(p) * D + j), acc[j]);
+          }
+          store_row<D, OUT_F32>(a, seq, qh, lane, acc, Ls > 0.f ? 1.f / Ls : 0.f);
+          if (lane == 0) a.arrive[unit] = 0;
+        }
+      }
+    }
+    fence_proxy_async_smem();  // this slot's reads are ordered before a bulk copy refills it
+    __syncwarp();
+    ++consumed;
+    if (issue(slot)) ++issued;
+  }
+  if (timed_out) {
+    if (lane == 0) set_status(a.status, PKV_DEV_TIMEOUT);
+    // Let copies already in flight into this warp's ring land before the CTA exits.
+    for (int n = consumed; n < issued; ++n) mbar_wait(&ring.full[n % STAGES], (n / STAGES) & 1);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+constexpr int kSimtWarps = 4;
+constexpr int kSimtStages = 3;
+
+template <int D, bool OUT_F32>
+static int launch_simt(const DecodeArgs& a, cudaStream_t stream) {
+  auto kernel = decode_simt_kernel<D, OUT_F32, kSimtWarps, kSimtStages>;
+  const size_t smem = sizeof(WarpRing<D, kSimtStages>) * kSimtWarps;
+  static std::once_flag once;
+  static int blocks_per_sm = 0;
+  static cudaError_t setup_err = cudaSuccess;
+  std::call_once(once, [&] {
+    setup_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (setup_err == cudaSuccess)
+      setup_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kSimtWarps * 32, smem);
+  });
+  if (setup_err != cudaSuccess)
+    return set_error(PKV_ERR_CUDA, "decode (simt) setup: %s", cudaGetErrorString(setup_err));
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::max(1, sms * std::max(1, blocks_per_sm));
+  kernel<<<grid, kSimtWarps * 32, smem, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (simt) launch: %s", cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+static int launch_plan(const DecodeArgs& a, const int32_t* context_lens, int max_context_len, cudaStream_t stream) {
+  plan_kernel<<<1, kPlanThreads, 0, stream>>>(context_lens, a.num_seqs, max_context_len,
+                                              a.max_blocks * a.block_size, a.partition,
+                                              const_cast<PlanEntry*>(a.entries),
+                                              const_cast<int32_t*>(a.plan_count), a.arrive,
+                                              a.num_seqs * a.num_heads, a.status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode plan launch: %s", cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+static int resolve_partition(int partition_tokens, int num_seqs, int num_kv_heads, int block_size,
+                             int max_context_len) {
+  if (partition_tokens == 0) return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len);
+  if (partition_tokens != 64 && partition_tokens != 128 && partition_tokens != 256 && partition_tokens != 512)
+    return -1;
+  if (partition_tokens % block_size != 0) return -1;
+  return partition_tokens;
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" int pkv_paged_attention_partition_tokens(int num_seqs, int num_kv_heads, int block_size,
+                                                    int max_context_len) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || (block_size != 16 && block_size != 32) || max_context_len < 0)
+    return set_error(PKV_ERR_INVALID, "partition_tokens: bad arguments");
+  return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len);
+}
+
+extern "C" size_t pkv_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                                     int block_size, int max_context_len, int partition_tokens) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+      (block_size != 16 && block_size != 32))
+    return 0;
+  const int p = resolve_partition(partition_tokens, num_seqs, num_kv_heads, block_size, max_context_len);
+  if (p < 0) return 0;
+  return workspace_layout(num_seqs, num_heads, head_dim, max_context_len, p).total;
+}
+
+extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* query, const void* key_cache,
+                                          const void* value_cache, const int32_t* block_tables,
+                                          int max_blocks_per_seq, const int32_t* context_lens,
+                                          int max_context_len, int num_seqs, int num_heads, int num_kv_heads,
+                                          int head_dim, int block_size, int num_blocks, float scale,
+                                          int partition_tokens, int path, void* workspace, size_t workspace_bytes,
+                                          int32_t* status, pkv_stream_t stream) {
+  clear_error();
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
+      max_context_len < 0)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: bad sizes");
+  if (num_seqs > 65535 * 1024) return set_error(PKV_ERR_INVALID, "paged_attention_decode: too many sequences");
+  if (out_dtype != PKV_DTYPE_BF16 && out_dtype != PKV_DTYPE_F32)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: out_dtype %d", out_dtype);
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: head_dim %d not in {64,128}", head_dim);
+  if (block_size != 16 && block_size != 32)
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: block_size %d not in {16,32}", block_size);
+  if (num_heads % num_kv_heads != 0)
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: num_heads %d not a multiple of num_kv_heads %d",
+                     num_heads, num_kv_heads);
+  if (path != PKV_PATH_AUTO && path != PKV_PATH_SIMT && path != PKV_PATH_TENSOR)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: path %d", path);
+  const int group = num_heads / num_kv_heads;
+  if (path == PKV_PATH_TENSOR && !tensor_path_supports(group, head_dim))
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: tensor path needs 2 <= group <= 16 and head_dim 128"
+                     " (group %d, head_dim %d)", group, head_dim);
+  const int partition = resolve_partition(partition_tokens, num_seqs, num_kv_heads, block_size, max_context_len);
+  if (partition < 0)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: partition_tokens %d (64/128/256/512, multiple of "
+                     "block_size)", partition_tokens);
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(65535) * partition)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: max_context_len too large for the split");
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !workspace)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: null pointer");
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: tensors must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: workspace must be 256-byte aligned");
+  const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim, max_context_len, partition);
+  if (workspace_bytes < w.total)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: workspace of %zu bytes, %zu needed", workspace_bytes,
+                     w.total);
+  if (static_cast<int64_t>(num_blocks) * num_kv_heads * block_size > (static_cast<int64_t>(1) << 31))
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: pool too large");
+
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  DecodeArgs a{};
+  a.out = out;
+  a.query = static_cast<const __nv_bfloat16*>(query);
+  a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
+  a.value_cache = static_cast<const __nv_bfloat16*>(value_cache);
+  a.block_tables = block_tables;
+  a.plan_count = reinterpret_cast<const int32_t*>(ws + w.off_count);
+  a.entries = reinterpret_cast<const PlanEntry*>(ws + w.off_entries);
+  a.arrive = reinterpret_cast<int32_t*>(ws + w.off_arrive);
+  a.part_o = reinterpret_cast<float*>(ws + w.off_part_o);
+  a.part_ml = reinterpret_cast<float2*>(ws + w.off_part_ml);
+  a.status = status;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.group = group;
+  a.partition = partition;
+  a.max_parts = w.max_parts;
+  a.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = launch_plan(a, context_lens, max_context_len, s);
+  if (rc != PKV_OK) return rc;
+  const bool out_f32 = out_dtype == PKV_DTYPE_F32;
+  const bool use_tensor = path == PKV_PATH_TENSOR || (path == PKV_PATH_AUTO && tensor_path_supports(group, head_dim));
+  if (use_tensor) return launch_decode_tensor(a, head_dim, out_f32, s);
+  if (head_dim == 128) return out_f32 ? launch_simt<128, true>(a, s) : launch_simt<128, false>(a, s);
+  return out_f32 ? launch_simt<64, true>(a, s) : launch_simt<64, false>(a, s);
+}

@@ -1,0 +1,91 @@
+// Shared definitions of the decode-attention kernels: launch arguments, the
+// work plan (entries of (sequence, partition) sorted longest first) and the
+// workspace layout.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "device_common.cuh"
+
+namespace pkv {
+
+// Tokens that one pipeline stage carries: one 16-row slice of a (block, kv head)
+// tile (a whole block at block_size 16, half a block at 32).
+constexpr int kStageTokens = 16;
+constexpr int kMaxPartition = 512;
+
+// One plan entry: a (sequence, partition) pair.  x = seq, y = partition index,
+// z = number of partitions of the sequence, w = validated context length.
+using PlanEntry = int4;
+
+struct DecodeArgs {
+  void* out;
+  const __nv_bfloat16* query;
+  const __nv_bfloat16* key_cache;
+  const __nv_bfloat16* value_cache;
+  const int32_t* block_tables;
+  const int32_t* plan_count;   // number of plan entries (written by the plan kernel)
+  const PlanEntry* entries;    // sorted plan
+  int32_t* arrive;             // [B * Hq] partition arrival counters (zeroed by the plan kernel)
+  float* part_o;               // [B * Hq * max_parts * D] unnormalised partial outputs
+  float2* part_ml;             // [B * Hq * max_parts] (running max in log2 units, sum of weights)
+  int32_t* status;
+  int max_blocks;
+  int num_seqs;
+  int num_heads;
+  int num_kv_heads;
+  int block_size;
+  int num_blocks;
+  int group;                   // num_heads / num_kv_heads
+  int partition;               // tokens per partition
+  int max_parts;
+  float scale_log2;            // scale * log2(e): scores are kept in base-2 units
+};
+
+// Workspace layout, identical for every decode path.
+struct WorkspaceLayout {
+  int partition = 0;
+  int max_parts = 0;
+  size_t off_count = 0, off_arrive = 0, off_entries = 0, off_part_o = 0, off_part_ml = 0, total = 0;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_context_len) {
+  // Largest split (fewest partials to merge) that still leaves enough work items
+  // to spread over every SM of the GPU.
+  int p = kMaxPartition;
+  while (p > 64 && static_cast<int64_t>(num_seqs) * num_kv_heads * ((max_context_len + p - 1) / p) < 4096) p /= 2;
+  return p < block_size ? block_size : p;
+}
+
+inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int max_context_len,
+                                        int partition) {
+  WorkspaceLayout w;
+  w.partition = partition;
+  w.max_parts = max_context_len <= 0 ? 1 : (max_context_len + partition - 1) / partition;
+  size_t off = 0;
+  w.off_count = off;
+  off = align256(off + sizeof(int32_t));
+  w.off_arrive = off;
+  off = align256(off + static_cast<size_t>(num_seqs) * num_heads * sizeof(int32_t));
+  w.off_entries = off;
+  off = align256(off + static_cast<size_t>(num_seqs) * w.max_parts * sizeof(PlanEntry));
+  w.off_part_o = off;
+  if (w.max_parts > 1) {
+    off = align256(off + static_cast<size_t>(num_seqs) * num_heads * w.max_parts * head_dim * sizeof(float));
+    w.off_part_ml = off;
+    off = align256(off + static_cast<size_t>(num_seqs) * num_heads * w.max_parts * sizeof(float2));
+  } else {
+    w.off_part_ml = off;
+  }
+  w.total = off;
+  return w;
+}
+
+// Launchers living in other translation units.
+int launch_decode_tensor(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
+bool tensor_path_supports(int group, int head_dim);
+
+}  // namespace pkv

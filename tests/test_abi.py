@@ -1,0 +1,192 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, rejects
+bad arguments before touching a GPU, and its block manager matches the reference
+model of the allocator operation for operation (all CPU-only)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import workloads as wl
+from oracle.block_manager import BlockManagerError, BlockManagerModel
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"PKV_API\s+[\w\s\*]*?\b(pkv_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_loads_and_exports_every_declared_symbol(pkv):
+    lib = pkv.library()
+    names = declared_symbols()
+    assert len(names) >= 20
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert lib.pkv_version() >= 10000
+
+
+def test_binding_covers_every_symbol(pkv):
+    from paged_kv_cache_423_b200 import _SIGNATURES
+    assert set(declared_symbols()) <= set(_SIGNATURES)
+
+
+def test_header_entry_points_cite_their_passage():
+    text = open(os.path.join(ROOT, "include", "pkv.h")).read()
+    for anchor in ("§2.1", "§1.4", "内存共享", "LLM serving的基本流程与KV缓存", "vLLM的核心创新"):
+        assert anchor in text
+
+
+def test_argument_errors_before_any_device_work(pkv):
+    lib = pkv.library()
+    fake = ctypes.c_void_p(0x1000)
+    # unsupported head_dim / block size / grouping; bad out dtype; misaligned pointer
+    args = dict(out=fake, out_dtype=0, query=fake, kc=fake, vc=fake, tables=fake, max_blocks=4, lens=fake,
+                max_ctx=64, B=2, Hq=4, Hkv=2, D=128, bs=16, NB=8, scale=0.1, part=0, path=0, ws=fake,
+                ws_bytes=1 << 20)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.pkv_paged_attention_decode(a["out"], a["out_dtype"], a["query"], a["kc"], a["vc"], a["tables"],
+                                              a["max_blocks"], a["lens"], a["max_ctx"], a["B"], a["Hq"], a["Hkv"],
+                                              a["D"], a["bs"], a["NB"], a["scale"], a["part"], a["path"], a["ws"],
+                                              a["ws_bytes"], None, None)
+
+    assert call(D=96) == pkv.PKV_ERR_UNSUPPORTED
+    assert call(bs=8) == pkv.PKV_ERR_UNSUPPORTED
+    assert call(Hq=5) == pkv.PKV_ERR_UNSUPPORTED
+    assert call(out_dtype=7) == pkv.PKV_ERR_INVALID
+    assert call(part=100) == pkv.PKV_ERR_INVALID
+    assert call(query=ctypes.c_void_p(0x1008)) == pkv.PKV_ERR_INVALID
+    assert call(ws=ctypes.c_void_p(0x1010)) == pkv.PKV_ERR_INVALID
+    assert call(ws_bytes=16) == pkv.PKV_ERR_INVALID
+    assert b"workspace" in lib.pkv_last_error_string()
+    assert call(B=0) == pkv.PKV_OK       # empty batch: nothing to do
+    assert lib.pkv_reshape_and_cache(fake, fake, fake, fake, fake, 4, 8, 2, 96, 16, None, None) == pkv.PKV_ERR_UNSUPPORTED
+    assert lib.pkv_reshape_and_cache(fake, fake, fake, fake, fake, 0, 8, 2, 128, 16, None, None) == pkv.PKV_OK
+    assert lib.pkv_copy_blocks(None, None, 0, None, 0, 8, 4096, None, None) == pkv.PKV_OK
+    assert lib.pkv_copy_blocks(None, None, 1, None, 3, 8, 4095, None, None) == pkv.PKV_ERR_INVALID
+
+
+def test_workspace_size_and_partition_choice(pkv):
+    assert pkv.paged_attention_partition_tokens(256, 40, 16, 2000) == 512
+    assert pkv.paged_attention_partition_tokens(4, 2, 16, 33) == 64
+    small = pkv.paged_attention_workspace_size(4, 2, 2, 64, 16, 33)
+    big = pkv.paged_attention_workspace_size(16, 64, 8, 128, 32, 32000)
+    assert 0 < small < big
+    # partials: B * Hq * parts * (D + 2) floats dominate
+    assert big >= 16 * 64 * 63 * 130 * 4
+    with pytest.raises(pkv.PkvError):
+        pkv.paged_attention_workspace_size(4, 2, 2, 64, 16, 33, partition_tokens=48)
+
+
+# ---------------------------------------------------------------------------
+# Block manager: C++ vs the reference model, operation by operation
+# ---------------------------------------------------------------------------
+
+def same_state(cpp, model: BlockManagerModel):
+    assert cpp.num_free() == model.num_free()
+    assert cpp.free_list() == list(model.free)
+    for b in range(model.num_blocks):
+        assert cpp.refcount(b) == model.ref[b]
+    ids = sorted(model.tables)
+    if ids:
+        mb = max(len(t) for t in model.tables.values()) or 1
+        tables, lens = cpp.export_tables(ids, mb)
+        exp_t, exp_l = model.export_tables(ids, mb)
+        assert tables.tolist() == exp_t and lens.tolist() == exp_l
+
+
+def run_both(op, cpp, model, pkv):
+    """Run op on both; they must agree on success or on the error code."""
+    err_m = err_c = None
+    res_m = res_c = None
+    try:
+        res_m = op(model)
+    except BlockManagerError as e:
+        err_m = e.code
+    try:
+        res_c = op(cpp)
+    except pkv.PkvError as e:
+        err_c = e.code
+    assert err_m == err_c
+    return res_m, res_c
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_block_manager_matches_model(pkv, seed):
+    rng = wl.rng_for(100 + seed)
+    nb, bs = 40, 4
+    order = rng.permutation(nb).astype(np.int32)
+    cpp = pkv.BlockManager(nb, bs, order)
+    model = BlockManagerModel(nb, bs, order)
+    next_id = 0
+    for _ in range(300):
+        live = sorted(model.tables)
+        op = int(rng.integers(0, 6))
+        if op == 0 or not live:
+            shared = []
+            if live and rng.random() < 0.5:
+                donor = live[int(rng.integers(len(live)))]
+                shared = model.tables[donor][:int(rng.integers(0, model.lens[donor] // bs + 1))]
+            n_tok = len(shared) * bs + int(rng.integers(0, 10))
+            sid = next_id
+            next_id += 1
+            run_both(lambda m: m.add_seq(sid, n_tok, shared), cpp, model, pkv)
+        elif op == 1:
+            parent = live[int(rng.integers(len(live)))]
+            child = next_id
+            next_id += 1
+            run_both(lambda m: m.fork(parent, child), cpp, model, pkv)
+        elif op == 2:
+            pick = [int(s) for s in rng.permutation(live)[:int(rng.integers(1, len(live) + 1))]]
+            (sm, pm), (sc, pc) = [r if r is not None else (None, None) for r in run_both(
+                lambda m: m.append_slots(pick), cpp, model, pkv)]
+            if sm is not None:
+                assert list(sc) == sm and [tuple(p) for p in pc.tolist()] == pm
+        elif op == 3:
+            victim = live[int(rng.integers(len(live)))]
+            run_both(lambda m: m.free_seq(victim), cpp, model, pkv)
+        elif op == 4:
+            s = live[int(rng.integers(len(live)))]
+            L = model.lens[s]
+            rm, rc = run_both(lambda m: m.slots(s, 0, L), cpp, model, pkv)
+            assert list(rc) == rm
+        else:
+            bad = int(rng.integers(-2, nb + 2))
+            run_both(lambda m: m.decref(bad) if m.refcount(bad) == 0 else m.incref(bad), cpp, model, pkv)
+        same_state(cpp, model)
+    cpp.close()
+
+
+def test_block_manager_errors_and_oom(pkv):
+    bm = pkv.BlockManager(3, 4, [2, 0, 1])
+    bm.add_seq(0, 4)
+    bm.add_seq(1, 4)
+    with pytest.raises(pkv.PkvError) as e:
+        bm.append_slots([0, 1])
+    assert e.value.code == pkv.PKV_ERR_OOM
+    assert bm.num_free() == 1 and bm.seq_len(0) == 4 and bm.seq_len(1) == 4
+    with pytest.raises(pkv.PkvError) as e:
+        bm.append_slots([0, 0])
+    assert e.value.code == pkv.PKV_ERR_INVALID
+    with pytest.raises(pkv.PkvError):
+        pkv.BlockManager(4, 4, [0, 1, 1, 2])
+
+
+def test_block_manager_cow_example(pkv):
+    bm = pkv.BlockManager(16, 4)
+    bm.add_seq(0, 6)
+    for c in (1, 2, 3):
+        bm.fork(0, c)
+    slots, pairs = bm.append_slots([0, 1, 2, 3])
+    assert pairs.tolist() == [[1, 2], [1, 3], [1, 4]]
+    assert slots.tolist() == [10, 14, 18, 6]
+    tables, lens = bm.export_tables([0, 1, 2, 3], 2)
+    assert tables.tolist() == [[0, 2], [0, 3], [0, 4], [0, 1]] and lens.tolist() == [7] * 4

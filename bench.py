@@ -32,9 +32,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -67,52 +65,69 @@ def rank_info():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event reasons through NVML every ~1 ms
+    while the timed region runs (a thread; NVML reads only, nothing is set)."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.max_mhz = None
+        self.err = None
+        self._stop = None
+        self._thread = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: record why
+            self.err = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((mhz, rs))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(0.001)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
 
     def summary(self):
-        if self.proc is None or not self.path:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [self.err or "no samples"], "samples": 0}
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({name for _, rs in self.samples for name, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "sm_mhz_min": min(mhz)}
 
 
 # ---------------------------------------------------------------------------
@@ -163,6 +178,20 @@ class Workload:
         return q, k, v
 
 
+def aggregate_over_ranks(ms_local, units_local, dist=None, device=None):
+    """Whole-job timing: the slowest rank's time and the units all ranks processed.
+
+    Every rank must call this with the same collective sequence (MAX then SUM)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms_local), int(units_local)
+    import torch
+    t = torch.tensor([float(ms_local)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([int(units_local)], dtype=torch.int64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(u.item())
+
+
 def to_dev(bits, device):
     import torch
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
@@ -179,22 +208,27 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", device_id=device)
     total = args.warmup + args.steps
-    w = Workload(args.workload, total, seed=1000 + rank, device=device)
+    n_states = min(total, args.states)
+    w = Workload(args.workload, max(n_states, min(total, args.e2e_steps + args.warmup)), seed=1000 + rank,
+                 device=device)
     seq_ids = list(range(w.B))
 
-    # ---- prepare every step's device inputs (allocator run ahead of timing)
+    # ---- the allocator runs ahead of timing: `n_states` consecutive decode steps of
+    # the batch.  Timed step i replays state i % n_states, so the batch keeps its
+    # configured length mix however many steps are timed (a replayed state rewrites
+    # its own token into its own slot, then decodes the same contexts).
     bm = w.new_manager()
-    steps = []
-    for _ in range(total):
+    states = []
+    for _ in range(n_states):
         slots, pairs = bm.append_slots(seq_ids)
         tables, lens = bm.export_tables(seq_ids, w.max_blocks)
         q, k, v = w.host_step_inputs()
-        steps.append(dict(q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
-                          slots=torch.from_numpy(slots).to(device), pairs=torch.from_numpy(pairs).to(device),
-                          n_pairs=len(pairs), tables=torch.from_numpy(tables).to(device),
-                          lens=torch.from_numpy(lens).to(device), max_len=int(lens.max()), host_lens=lens))
+        states.append(dict(q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
+                           slots=torch.from_numpy(slots).to(device), pairs=torch.from_numpy(pairs).to(device),
+                           n_pairs=len(pairs), tables=torch.from_numpy(tables).to(device),
+                           lens=torch.from_numpy(lens).to(device), max_len=int(lens.max()), host_lens=lens))
     bm.close()
-    max_len_all = max(s["max_len"] for s in steps)
+    max_len_all = int(w.lens0.max()) + max(n_states, args.e2e_steps + args.warmup) + 1
     ws = torch.empty(pkv.paged_attention_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.bs, max_len_all),
                      dtype=torch.uint8, device=device)
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=device)
@@ -203,7 +237,7 @@ def run_ours(args, rank, world, local_rank):
     path = {"auto": 0, "simt": 1, "tensor": 2}[args.path]
 
     def step(i, ev=None):
-        st = steps[i]
+        st = states[i % n_states]
         if st["n_pairs"]:
             pkv.copy_blocks([w.key_cache], [w.value_cache], st["pairs"], status=status)
         pkv.reshape_and_cache(st["k"], st["v"], w.key_cache, w.value_cache, st["slots"], status=status)
@@ -220,17 +254,18 @@ def run_ours(args, rank, world, local_rank):
     launches = 0
     kv_total = bytes_total = 0
     for i in range(args.warmup, total):
-        kv, alg = decode_bytes(steps[i]["host_lens"], w.Hq, w.Hkv, w.D, w.bs)
+        st = states[i % n_states]
+        kv, alg = decode_bytes(st["host_lens"], w.Hq, w.Hkv, w.D, w.bs)
         kv_total += kv
         bytes_total += alg
-        launches += 3 + (1 if steps[i]["n_pairs"] else 0)
+        launches += 3 + (1 if st["n_pairs"] else 0)
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clocks:
+    with ClockSampler(device) as clocks:
         t0.record(stream)
         for j, i in enumerate(range(args.warmup, total)):
             step(i, dec_events[j])
@@ -242,12 +277,8 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_events)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item():#x}")
-    ms_max = ms
-    if dist:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    value = world * kv_total / (ms_max * 1e-3) / 1e9
+    ms_max, kv_all = aggregate_over_ranks(ms, kv_total, dist, device)
+    value = kv_all / (ms_max * 1e-3) / 1e9
     seq_steps = world * w.B * args.steps / (ms_max * 1e-3)
 
     # ---- e2e through the public API with host buffers
@@ -276,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
     if e2e is not None:
         result["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, steps[args.warmup], budget_s=args.cpu_budget)
+        result["cpu_baseline"] = cpu_baseline(w, states[0], budget_s=args.cpu_budget)
     if dist:
         dist.destroy_process_group()
     return result
@@ -284,12 +315,13 @@ def run_ours(args, rank, world, local_rank):
 
 def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     import torch
+    ke = max(1, min(args.steps, args.e2e_steps))
     bm = w.new_manager()
     seq_ids = list(range(w.B))
     stream = torch.cuda.current_stream()
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
     host = []
-    for _ in range(args.warmup + args.steps):
+    for _ in range(args.warmup + ke):
         q, k, v = w.host_step_inputs()
         host.append((pin(q.view(np.int16)), pin(k.view(np.int16)), pin(v.view(np.int16))))
     out_host = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
@@ -339,7 +371,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     t0.record(stream)
-    for i in range(args.warmup, args.warmup + args.steps):
+    for i in range(args.warmup, args.warmup + ke):
         bi, bo, lens = step(i)
         h2d += bi
         d2h += bo
@@ -349,8 +381,9 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     ms = t0.elapsed_time(t1)
     bm.close()
     return {"value": round(kv_total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
-            "h2d_bytes_per_step": h2d // args.steps, "d2h_bytes_per_step": d2h // args.steps,
-            "ms_per_step": round(ms / args.steps, 4)}
+            "h2d_bytes_per_step": h2d // ke, "d2h_bytes_per_step": d2h // ke,
+            "ms_per_step": round(ms / ke, 4), "steps": ke,
+            "seq_steps_per_s": round(w.B * ke / (ms * 1e-3), 1)}
 
 
 # ---------------------------------------------------------------------------
@@ -408,7 +441,7 @@ def run_reference(args, rank, world, local_rank):
     if device is None:
         return {"impl": "reference", "unavailable": "no CUDA device to hold the synthetic workload"}
     torch.cuda.set_device(device)
-    w = Workload(args.workload, args.warmup + args.steps, seed=1000, device=device)
+    w = Workload(args.workload, 2, seed=1000, device=device)
     bm = w.new_manager()
     ids = list(range(w.B))
     bm.append_slots(ids)
@@ -416,18 +449,19 @@ def run_reference(args, rank, world, local_rank):
     q, _, _ = w.host_step_inputs()
     st = {"tables": torch.from_numpy(tables), "host_lens": lens, "q": to_dev(q, device)}
     rng = wl.rng_for(78)
-    per_step = max(1, int(args.ref_seqs))
+    # size each step's sample so the whole run stays near --ref-budget seconds
+    probe = oracle_sample(w, st, 2, rng)
+    _, dt_probe, n_probe = time_oracle(w, probe, 1e9)
+    per_seq = dt_probe / max(n_probe, 1)
+    per_step = int(max(1, min(64, args.ref_budget / max(per_seq, 1e-6) / (args.warmup + args.steps))))
     for _ in range(args.warmup):
         time_oracle(w, oracle_sample(w, st, per_step, rng), 1e9)
     kv = 0
     dt_total = 0.0
-    n_total = 0
     for _ in range(args.steps):
-        items = oracle_sample(w, st, per_step, rng)
-        b, dt, n = time_oracle(w, items, 1e9)
+        b, dt, _n = time_oracle(w, oracle_sample(w, st, per_step, rng), 1e9)
         kv += b
         dt_total += dt
-        n_total += n
     value = kv / dt_total / 1e9
     sample = (f"{per_step} random sequences of the {w.name} batch per step (all {w.Hq} heads), float64 NumPy oracle, "
               f"1 thread")
@@ -444,15 +478,17 @@ def run_reference(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--states", type=int, default=16, help="distinct precomputed decode steps replayed in turn")
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama13b_mixed_bs16", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
-    ap.add_argument("--ref-seqs", type=int, default=8)
+    ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work in --impl reference")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -1,0 +1,53 @@
+"""Host-side logic of bench.py: byte accounting and the multi-rank aggregation
+(world size 2 over gloo on CPU; the GPU runs use the same calls over NCCL)."""
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_decode_bytes_counts_each_token_once():
+    kv, alg = bench.decode_bytes([1, 16, 17], Hq=8, Hkv=2, D=128, bs=16)
+    assert kv == 34 * 2 * 128 * 2 * 2
+    blocks = 1 + 1 + 2
+    assert alg == kv + 2 * 3 * 8 * 128 * 2 + blocks * 4 + 3 * 4
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    ms, units = bench.aggregate_over_ranks(10.0 + 5 * rank, 100 * (rank + 1), dist, torch.device("cpu"))
+    results[rank] = (ms, units)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_aggregate_over_two_gloo_ranks():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    results = manager.dict()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    # every rank sees the slowest rank's time and the units of all ranks
+    assert results[0] == results[1] == (15.0, 300)
+
+
+def test_single_process_aggregation_is_identity():
+    assert bench.aggregate_over_ranks(3.5, 7) == (3.5, 7)

@@ -111,8 +111,9 @@ struct __align__(128) WarpRing {
   __nv_bfloat16 k[STAGES][kStageTokens * D];
   __nv_bfloat16 v[STAGES][kStageTokens * D];
   __nv_bfloat16 q[STAGES][D];
+  float2 p[kStageTokens];  // (p_t, p_t) of the stage being consumed, read back as packed pairs
   uint64_t full[STAGES];
-  int4 meta[STAGES];  // x seq, y query head, z part | nparts << 16, w n_valid | first << 8 | last << 9
+  int4 meta[STAGES];  // x seq, y query head, z part | nparts << 16, w n_valid | flags (first, last, q present)
 };
 
 // Per-item state of the issuing side (warp-uniform except `table`).
@@ -136,6 +137,42 @@ __device__ __forceinline__ int load_item_table(const DecodeArgs& a, const PlanEn
   return __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + lane);
 }
 
+// ---- packed fp32x2 arithmetic (two lanes of fp32 in one 64-bit register pair)
+__device__ __forceinline__ uint64_t f2pack(float x, float y) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// bf16 pair word -> packed (lo, hi) fp32 pair, exactly.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2pack(bf16lo(w), bf16hi(w)); }
+
+// a0 += q.lo * k.lo, a1 += q.hi * k.hi with bf16 operands and fp32 accumulation
+// (sm_100 mixed-precision FMA; the bf16 x bf16 product is exact in fp32).
+__device__ __forceinline__ void dot_bf16x2(float& a0, float& a1, uint32_t q, uint32_t k) {
+  asm("{\n\t.reg .b16 ql, qh, kl, kh;\n\t"
+      "mov.b32 {ql, qh}, %2;\n\t"
+      "mov.b32 {kl, kh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, ql, kl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, qh, kh, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(q), "r"(k));
+}
+
 template <int D, bool OUT_F32>
 __device__ __forceinline__ void store_row(const DecodeArgs& a, int seq, int qh, int lane, const float* o,
                                           float inv) {
@@ -156,15 +193,39 @@ __device__ __forceinline__ void store_row(const DecodeArgs& a, int seq, int qh, 
   }
 }
 
+// Lane roles inside a warp.
+//   q·K: two lanes per row, each over half of head_dim (64 or 32 values, NC 16-byte
+//        chunks).  Lane k of a row visits its chunks in the rotated order
+//        (k + i) mod NC, so the 8 lanes of each shared-memory phase always hit 8
+//        different 16-byte bank groups although every row starts at bank 0.
+//   P·V: lane l owns head_dim/32 consecutive output values of every row.
+template <int D>
+struct LaneMap {
+  static constexpr int NC = D / 16;                  // 16-byte chunks per half row
+  static constexpr int PARTNER = D == 128 ? 16 : 4;  // the lane holding the other half of the row
+  __device__ static int row(int lane) { return D == 128 ? (lane & 15) : ((lane & 3) | ((lane >> 3) << 2)); }
+  __device__ static int half(int lane) { return D == 128 ? (lane >> 4) : ((lane >> 2) & 1); }
+  __device__ static float max_rows(float x) {  // max over the 16 rows (lanes with the same half)
+    constexpr int m0 = 1, m1 = 2, m2 = D == 128 ? 4 : 8, m3 = D == 128 ? 8 : 16;
+    x = fmaxf(x, __shfl_xor_sync(kFull, x, m0));
+    x = fmaxf(x, __shfl_xor_sync(kFull, x, m1));
+    x = fmaxf(x, __shfl_xor_sync(kFull, x, m2));
+    return fmaxf(x, __shfl_xor_sync(kFull, x, m3));
+  }
+};
+
 template <int D, bool OUT_F32, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int EPL = D / 32;                                  // elements per lane: 2 or 4
+  constexpr int EPL = D / 32;                                  // output values per lane: 2 or 4
+  constexpr int NPAIR = EPL / 2;                               // packed fp32 pairs per lane
+  constexpr int NC = LaneMap<D>::NC;
   constexpr uint32_t kKVBytes = kStageTokens * D * sizeof(__nv_bfloat16);
   constexpr uint32_t kQBytes = D * sizeof(__nv_bfloat16);
   using Ring = WarpRing<D, STAGES>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Ring& ring = reinterpret_cast<Ring*>(smem_raw)[warp];
+  const int qk_row = LaneMap<D>::row(lane), qk_half = LaneMap<D>::half(lane);
 
   const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_heads;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * WARPS;
@@ -218,9 +279,9 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
     const PlanEntry e = cur.e;
     const int qh = static_cast<int>(cur.id % a.num_heads);
     const int kvh = qh / a.group;
-    const int tok = e.y * a.partition + cur_stage * kStageTokens;        // first token of the stage
-    const int n_tok = e.w == 0 ? 0 : min(kStageTokens, e.w - tok);
     const int local_tok = cur_stage * kStageTokens;
+    const int tok = e.y * a.partition + local_tok;                       // first token of the stage
+    const int n_tok = e.w == 0 ? 0 : min(kStageTokens, e.w - tok);
     const int phys = __shfl_sync(kFull, cur.table, local_tok / a.block_size);
     const bool ok = n_tok > 0 && phys >= 0 && phys < a.num_blocks;
     const bool first = cur_stage == 0, last = cur_stage == cur_nstages - 1;
@@ -245,10 +306,13 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   };
 
   // ---- consuming side
-  float qf[EPL], o[EPL];
+  uint4 qv[NC];                 // this lane's half of q (raw bf16 pairs), chunks in rotated order
+  uint64_t o[NPAIR];            // packed fp32 output accumulators
   float m = -INFINITY, lsum = 0.f;
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) qf[j] = o[j] = 0.f;
+  for (int i = 0; i < NC; ++i) qv[i] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
 
   int issued = 0;
   for (int s = 0; s < STAGES; ++s) {
@@ -270,113 +334,92 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       m = -INFINITY;
       lsum = 0.f;
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) o[j] = 0.f;
+      for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
       if (mt.w & 0x400) {
-        const __nv_bfloat16* qs = ring.q[slot] + lane * EPL;
-        if constexpr (EPL == 4) {
-          const uint2 w = *reinterpret_cast<const uint2*>(qs);
-          qf[0] = bf16lo(w.x) * a.scale_log2;
-          qf[1] = bf16hi(w.x) * a.scale_log2;
-          qf[2] = bf16lo(w.y) * a.scale_log2;
-          qf[3] = bf16hi(w.y) * a.scale_log2;
-        } else {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(qs);
-          qf[0] = bf16lo(w) * a.scale_log2;
-          qf[1] = bf16hi(w) * a.scale_log2;
-        }
+        const uint4* qs = reinterpret_cast<const uint4*>(ring.q[slot]);
+#pragma unroll
+        for (int i = 0; i < NC; ++i) qv[i] = qs[qk_half * NC + ((i + qk_row) & (NC - 1))];
       }
     }
     if (n_valid > 0) {
-      // Scores of the 16 rows: per-lane partial dot products over EPL dims.
-      const __nv_bfloat16* kb = ring.k[slot] + lane * EPL;
-      float sc[16];
+      // ---- scores: two lanes per row, bf16 x bf16 products accumulated in fp32
+      const uint4* krow = reinterpret_cast<const uint4*>(ring.k[slot] + qk_row * D) + qk_half * NC;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        if constexpr (EPL == 4) {
-          const uint2 w = *reinterpret_cast<const uint2*>(kb + t * D);
-          sc[t] = fmaf(qf[3], bf16hi(w.y), fmaf(qf[2], bf16lo(w.y), fmaf(qf[1], bf16hi(w.x), qf[0] * bf16lo(w.x))));
-        } else {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(kb + t * D);
-          sc[t] = fmaf(qf[1], bf16hi(w), qf[0] * bf16lo(w));
-        }
+      for (int i = 0; i < NC; ++i) {
+        const uint4 kw = krow[(i + qk_row) & (NC - 1)];
+        dot_bf16x2(a0, a1, qv[i].x, kw.x);
+        dot_bf16x2(a2, a3, qv[i].y, kw.y);
+        dot_bf16x2(a0, a1, qv[i].z, kw.z);
+        dot_bf16x2(a2, a3, qv[i].w, kw.w);
       }
-      // Transposed reduction: after the steps on lane bits 4..1 lane holds the sum
-      // over 16 lanes of row (lane >> 1); the xor-1 step completes it.
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const bool up = lane & 16;
-        const float send = up ? sc[i] : sc[i + 8];
-        const float keep = up ? sc[i + 8] : sc[i];
-        sc[i] = keep + __shfl_xor_sync(kFull, send, 16);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool up = lane & 8;
-        const float send = up ? sc[i] : sc[i + 4];
-        const float keep = up ? sc[i + 4] : sc[i];
-        sc[i] = keep + __shfl_xor_sync(kFull, send, 8);
-      }
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const bool up = lane & 4;
-        const float send = up ? sc[i] : sc[i + 2];
-        const float keep = up ? sc[i + 2] : sc[i];
-        sc[i] = keep + __shfl_xor_sync(kFull, send, 4);
-      }
-      {
-        const bool up = lane & 2;
-        const float send = up ? sc[0] : sc[1];
-        const float keep = up ? sc[1] : sc[0];
-        sc[0] = keep + __shfl_xor_sync(kFull, send, 2);
-      }
-      sc[0] += __shfl_xor_sync(kFull, sc[0], 1);
-      const bool valid = (lane >> 1) < n_valid;
-      const float x = valid ? sc[0] : -INFINITY;
-      float mx = x;
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-      const float m_new = fmaxf(m, mx);
+      float sc = (a0 + a1) + (a2 + a3);
+      sc += __shfl_xor_sync(kFull, sc, LaneMap<D>::PARTNER);
+      // ---- online softmax in base 2 over the stage's rows
+      const bool valid = qk_row < n_valid;
+      const float x = valid ? sc * a.scale_log2 : -INFINITY;
+      const float m_new = fmaxf(m, LaneMap<D>::max_rows(x));
       const float alpha = exp2f(m - m_new);
       const float p = valid ? exp2f(x - m_new) : 0.f;
       m = m_new;
       lsum = fmaf(lsum, alpha, p);
+      if (qk_half == 0) ring.p[qk_row] = make_float2(p, p);
+      __syncwarp();
+      // ---- P·V: packed fp32 pairs, rows past n_valid never touched (stale rows may be NaN)
+      const uint64_t alpha2 = f2pack(alpha, alpha);
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) o[j] *= alpha;
+      for (int j = 0; j < NPAIR; ++j) o[j] = fmul2(o[j], alpha2);
+      const uint64_t* pp = reinterpret_cast<const uint64_t*>(ring.p);
       const __nv_bfloat16* vb = ring.v[slot] + lane * EPL;
+      if (n_valid == kStageTokens) {
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        const float pt = __shfl_sync(kFull, p, 2 * t);
-        if (t < n_valid) {
+        for (int t = 0; t < kStageTokens; ++t) {
+          const uint64_t p2 = pp[t];
           if constexpr (EPL == 4) {
             const uint2 w = *reinterpret_cast<const uint2*>(vb + t * D);
-            o[0] = fmaf(pt, bf16lo(w.x), o[0]);
-            o[1] = fmaf(pt, bf16hi(w.x), o[1]);
-            o[2] = fmaf(pt, bf16lo(w.y), o[2]);
-            o[3] = fmaf(pt, bf16hi(w.y), o[3]);
+            o[0] = ffma2(p2, bf16x2_to_f2(w.x), o[0]);
+            o[1] = ffma2(p2, bf16x2_to_f2(w.y), o[1]);
           } else {
             const uint32_t w = *reinterpret_cast<const uint32_t*>(vb + t * D);
-            o[0] = fmaf(pt, bf16lo(w), o[0]);
-            o[1] = fmaf(pt, bf16hi(w), o[1]);
+            o[0] = ffma2(p2, bf16x2_to_f2(w), o[0]);
+          }
+        }
+      } else {
+#pragma unroll 4
+        for (int t = 0; t < n_valid; ++t) {
+          const uint64_t p2 = pp[t];
+          if constexpr (EPL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(vb + t * D);
+            o[0] = ffma2(p2, bf16x2_to_f2(w.x), o[0]);
+            o[1] = ffma2(p2, bf16x2_to_f2(w.y), o[1]);
+          } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(vb + t * D);
+            o[0] = ffma2(p2, bf16x2_to_f2(w), o[0]);
           }
         }
       }
     }
     if (last) {
       const int seq = mt.x, qh = mt.y, part = mt.z & 0xffff, nparts = mt.z >> 16;
+      float of[EPL];
+#pragma unroll
+      for (int j = 0; j < NPAIR; ++j) {
+        const float2 f = f2unpack(o[j]);
+        of[2 * j] = f.x;
+        of[2 * j + 1] = f.y;
+      }
       float l = lsum;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
-      l *= 0.5f;  // every row was counted by its two lanes
+      l *= 0.5f;  // every row's weight was held by its two lanes
       if (nparts == 1) {
-        store_row<D, OUT_F32>(a, seq, qh, lane, o, l > 0.f ? 1.f / l : 0.f);
+        store_row<D, OUT_F32>(a, seq, qh, lane, of, l > 0.f ? 1.f / l : 0.f);
       } else {
         const int64_t unit = static_cast<int64_t>(seq) * a.num_heads + qh;
         const int64_t pidx = unit * a.max_parts + part;
         float* po = a.part_o + pidx * D + lane * EPL;
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) po[j] = o[j];
+        for (int j = 0; j < EPL; ++j) po[j] = of[j];
         if (lane == 0) a.part_ml[pidx] = make_float2(m, l);
         __threadfence();
         __syncwarp();
@@ -421,8 +464,15 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
 // Host side
 // ---------------------------------------------------------------------------
 
-constexpr int kSimtWarps = 4;
-constexpr int kSimtStages = 3;
+// Warps per CTA and ring stages per warp (compile-time overridable for tuning sweeps).
+#ifndef PKV_SIMT_WARPS
+#define PKV_SIMT_WARPS 4
+#endif
+#ifndef PKV_SIMT_STAGES
+#define PKV_SIMT_STAGES 2
+#endif
+constexpr int kSimtWarps = PKV_SIMT_WARPS;
+constexpr int kSimtStages = PKV_SIMT_STAGES;
 
 template <int D, bool OUT_F32>
 static int launch_simt(const DecodeArgs& a, cudaStream_t stream) {

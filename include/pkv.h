@@ -168,6 +168,39 @@ PKV_API int pkv_paged_attention_decode(void* out, int out_dtype, const void* que
                                size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
 
 /*
+ * paged_attention_decode_static — pkv_paged_attention_decode without a workspace
+ * argument, for callers that cannot allocate device memory.  The source pages have
+ * no counterpart: this is a deployment convenience of this library.
+ *
+ * Who needs it: code that only receives its input and output buffers (for example
+ * a plugin called through a runtime's custom-operator interface that offers no
+ * scratch space), or applications that hand all device memory to their own
+ * allocator or forbid device allocations while running.
+ *
+ * How it works: the scratch lives in a fixed array of PKV_STATIC_SCRATCH_BYTES
+ * compiled into libpkv.so, present on every GPU that loads the library until the
+ * process exits.  This call allocates nothing.  Arguments, results and device
+ * status bits are those of pkv_paged_attention_decode.
+ *   - Sizes whose workspace (pkv_paged_attention_workspace_size) exceeds
+ *     PKV_STATIC_SCRATCH_BYTES return PKV_ERR_INVALID with an explanation; nothing
+ *     is enqueued.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture starts.
+ *   - All calls on one device share the array.  Calls whose kernels overlap on the
+ *     GPU (for example on two streams without ordering between them) race and give
+ *     wrong results; order them on one stream or use the workspace variant.
+ */
+#define PKV_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+PKV_API int pkv_paged_attention_decode_static(void* out, int out_dtype, const void* query, const void* key_cache,
+                                              const void* value_cache, const int32_t* block_tables,
+                                              int max_blocks_per_seq, const int32_t* context_lens,
+                                              int max_context_len, int num_seqs, int num_heads, int num_kv_heads,
+                                              int head_dim, int block_size, int num_blocks, float scale,
+                                              int partition_tokens, int path, int32_t* status,
+                                              pkv_stream_t stream);
+
+/*
  * Host block manager — free list + reference counts + per-sequence block tables.
  * Outcome School explainer, "vLLM的核心创新：PagedAttention" (a block only when needed,
  * any free block serves any request, finished requests return all blocks at once)

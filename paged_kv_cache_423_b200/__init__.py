@@ -20,7 +20,7 @@ __all__ = [
     "PKV_DEV_BAD_SLOT", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_CONTEXT", "PKV_DEV_BAD_PAIR", "PKV_DEV_TIMEOUT",
     "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR", "PkvError", "library", "library_path",
     "reshape_and_cache", "copy_blocks", "paged_attention_workspace_size", "paged_attention_partition_tokens",
-    "paged_attention_decode", "BlockManager",
+    "paged_attention_decode", "paged_attention_decode_static", "STATIC_SCRATCH_BYTES", "BlockManager",
 ]
 
 PKV_OK = 0
@@ -67,6 +67,9 @@ _SIGNATURES = {
     "pkv_paged_attention_decode": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                            c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
                                            c_void_p, c_size_t, c_void_p, c_void_p]),
+    "pkv_paged_attention_decode_static": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                                  c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
+                                                  c_int, c_int, c_void_p, c_void_p]),
     "pkv_bm_create": (c_void_p, [c_int, c_int, c_void_p]),
     "pkv_bm_destroy": (None, [c_void_p]),
     "pkv_bm_num_blocks": (c_int, [c_void_p]),
@@ -228,6 +231,34 @@ def paged_attention_decode(out, query, key_cache, value_cache, block_tables, con
         float(scale), int(partition_tokens), int(path), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
     _check(rc, "paged_attention_decode")
+
+
+STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def paged_attention_decode_static(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len,
+                                  scale, partition_tokens=0, path=PATH_AUTO, status=None, stream=None):
+    """paged_attention_decode without a workspace, for callers that cannot allocate
+    device memory: the scratch is a fixed array inside the library (STATIC_SCRATCH_BYTES
+    per GPU).  Calls on one device must not overlap on the GPU; the first call on a
+    device should come before any stream capture."""
+    torch = _torch()
+    B, Hq, D = query.shape
+    NB, Hkv, bs, D2 = key_cache.shape
+    if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
+        raise ValueError("paged_attention_decode_static: shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("paged_attention_decode_static: block_tables must be [B, max_blocks], context_lens [B]")
+    out_dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(out.dtype)
+    if out_dtype is None:
+        raise TypeError("paged_attention_decode_static: out must be bf16 or f32")
+    rc = library().pkv_paged_attention_decode_static(
+        _ptr(out, None, "out"), out_dtype, _ptr(query, torch.bfloat16, "query"),
+        _ptr(key_cache, torch.bfloat16, "key_cache"), _ptr(value_cache, torch.bfloat16, "value_cache"),
+        _ptr(block_tables, torch.int32, "block_tables"), int(block_tables.shape[1]),
+        _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len), B, Hq, Hkv, D, bs, NB,
+        float(scale), int(partition_tokens), int(path), _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "paged_attention_decode_static")
 
 
 # ---------------------------------------------------------------------------

@@ -13,7 +13,14 @@ from tests.gpu_helpers import DeviceBatch, compare, dev_bf16, host_bits
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1}
+PATHS = {"simt": 1, "tensor": 2}
+
+
+def path_applies(b, path):
+    """The tensor-core path covers grouped heads (2 <= g <= 16) at head_dim 128."""
+    g = b.num_heads // b.num_kv_heads
+    if path == "tensor" and not (b.head_dim == 128 and 2 <= g <= 16):
+        pytest.skip("tensor-core path needs grouped query heads and head_dim 128")
 
 
 def oracle_out(b):
@@ -29,6 +36,9 @@ CASES = {
     "long_trace": dict(name="long_trace", num_seqs=3, length_scale=0.08),
     "d64_bs32": dict(name="llama7b", num_seqs=6, length_scale=0.2, head_dim=64, block_size=32, num_heads=8,
                      num_kv_heads=8),
+    "gqa2_bs16": dict(name="llama7b", num_seqs=6, length_scale=0.3, num_heads=8, num_kv_heads=4),
+    "gqa16_bs32": dict(name="long_trace", num_seqs=2, length_scale=0.05, num_heads=32, num_kv_heads=2),
+    "gqa8_d64": dict(name="llama7b", num_seqs=4, length_scale=0.2, head_dim=64, num_heads=16, num_kv_heads=2),
 }
 
 
@@ -36,6 +46,7 @@ CASES = {
 @pytest.mark.parametrize("path", sorted(PATHS))
 def test_decode_matches_oracle(pkv, case, path):
     b = wl.make_decode_batch(**CASES[case])
+    path_applies(b, path)
     out = DeviceBatch(b).decode(pkv, path=PATHS[path])
     compare(out.cpu().numpy(), oracle_out(b))
 
@@ -44,24 +55,28 @@ def test_decode_matches_oracle(pkv, case, path):
 @pytest.mark.parametrize("path", sorted(PATHS))
 def test_split_sizes_agree(pkv, partition, path):
     """Split-context partitions of every size give the oracle's result."""
-    b = wl.make_decode_batch("llama7b", num_seqs=5, num_heads=4, num_kv_heads=4,
-                             lengths=[1, 63, 64, 65, 1500])
+    heads = (4, 4) if path == "simt" else (16, 4)
+    b = wl.make_decode_batch("llama7b", num_seqs=6, num_heads=heads[0], num_kv_heads=heads[1],
+                             lengths=[1, 63, 64, 65, 129, 1500])
     ref = oracle_out(b)
     out = DeviceBatch(b).decode(pkv, partition=partition, path=PATHS[path])
     compare(out.cpu().numpy(), ref)
 
 
-def test_bf16_output_is_rounded_fp32(pkv):
-    b = wl.make_decode_batch("llama13b_mixed_bs16", num_seqs=16, length_scale=0.3)
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_bf16_output_is_rounded_fp32(pkv, path):
+    name = "llama13b_mixed_bs16" if path == "simt" else "prefix_beams"
+    b = wl.make_decode_batch(name, num_seqs=16, length_scale=0.3)
     db = DeviceBatch(b)
-    f32 = db.decode(pkv, out_dtype=torch.float32)
-    bf = db.decode(pkv, out_dtype=torch.bfloat16)
+    f32 = db.decode(pkv, out_dtype=torch.float32, path=PATHS[path])
+    bf = db.decode(pkv, out_dtype=torch.bfloat16, path=PATHS[path])
     assert torch.equal(bf, f32.to(torch.bfloat16))
 
 
-def test_zero_length_and_single_token(pkv):
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_zero_length_and_single_token(pkv, path):
     b = wl.make_decode_batch("llama7b", num_seqs=4, num_heads=4, num_kv_heads=2, lengths=[0, 1, 0, 17])
-    out = DeviceBatch(b).decode(pkv).cpu().numpy()
+    out = DeviceBatch(b).decode(pkv, path=PATHS[path]).cpu().numpy()
     assert np.all(out[0] == 0) and np.all(out[2] == 0)
     compare(out, oracle_out(b))
     # one token: the output is exactly that token's V (softmax weight 1)
@@ -69,15 +84,17 @@ def test_zero_length_and_single_token(pkv):
     assert np.array_equal(out[1], np.repeat(v, 2, axis=0))
 
 
-def test_stale_nan_rows_do_not_leak(pkv):
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_stale_nan_rows_do_not_leak(pkv, path):
     """Rows past a context's end (stale pool rows) never enter the result, even as NaN."""
-    b = wl.make_decode_batch("llama13b_mixed_bs32", num_seqs=8, num_heads=4, num_kv_heads=4, length_scale=0.1)
+    b = wl.make_decode_batch("llama13b_mixed_bs32", num_seqs=8, num_heads=8, num_kv_heads=4 if path == "tensor" else 8,
+                             length_scale=0.1)
     nan = np.uint16(0x7FC1)
     for s, L in enumerate(b.context_lens):
         last = b.block_tables[s][(L - 1) // b.block_size]
         b.key_cache[last, :, (L - 1) % b.block_size + 1:, :] = nan
         b.value_cache[last, :, (L - 1) % b.block_size + 1:, :] = nan
-    out = DeviceBatch(b).decode(pkv).cpu().numpy()
+    out = DeviceBatch(b).decode(pkv, path=PATHS[path]).cpu().numpy()
     compare(out, oracle_out(b))
 
 
@@ -94,25 +111,28 @@ def test_permuted_pool_gives_same_output(pkv):
     assert torch.equal(base, DeviceBatch(b).decode(pkv))
 
 
-def test_bad_table_entry_and_context_are_flagged(pkv):
-    b = wl.make_decode_batch("llama7b", num_seqs=3, num_heads=2, num_kv_heads=2, lengths=[40, 20, 30])
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_bad_table_entry_and_context_are_flagged(pkv, path):
+    heads = (2, 2) if path == "simt" else (8, 2)
+    b = wl.make_decode_batch("llama7b", num_seqs=3, num_heads=heads[0], num_kv_heads=heads[1], lengths=[40, 20, 30])
     b.block_tables[0][1] = b.num_blocks + 5            # out of the pool
     db = DeviceBatch(b)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = db.decode(pkv, status=status).cpu().numpy()
+    out = db.decode(pkv, status=status, path=PATHS[path]).cpu().numpy()
     assert status.item() & pkv.PKV_DEV_BAD_BLOCK
     # sequences with valid tables are unaffected
-    good = wl.make_decode_batch("llama7b", num_seqs=3, num_heads=2, num_kv_heads=2, lengths=[40, 20, 30])
+    good = wl.make_decode_batch("llama7b", num_seqs=3, num_heads=heads[0], num_kv_heads=heads[1], lengths=[40, 20, 30])
     compare(out[1:], oracle_out(good)[1:])
     # a context longer than the bound: row zeroed, flagged
     db.lens[2] = 10_000
     status.zero_()
-    out = db.decode(pkv, status=status, max_context_len=64).cpu().numpy()
+    out = db.decode(pkv, status=status, max_context_len=64, path=PATHS[path]).cpu().numpy()
     assert status.item() & pkv.PKV_DEV_BAD_CONTEXT
     assert np.all(out[2] == 0)
 
 
-def test_repeated_calls_reuse_workspace(pkv):
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_repeated_calls_reuse_workspace(pkv, path):
     """The arrival counters are re-armed by every call: back-to-back calls on one
     workspace give identical outputs."""
     b = wl.make_decode_batch("long_trace", num_seqs=2, length_scale=0.05)
@@ -123,7 +143,7 @@ def test_repeated_calls_reuse_workspace(pkv):
     for _ in range(3):
         out = torch.empty((2, 64, 128), dtype=torch.float32, device="cuda")
         pkv.paged_attention_decode(out, db.query, db.key_cache, db.value_cache, db.tables, db.lens, maxl, b.scale, ws,
-                                   partition_tokens=64, path=1)
+                                   partition_tokens=64, path=PATHS[path])
         outs.append(out)
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
@@ -156,13 +176,15 @@ def sampled_oracle(b, kc_dev, vc_dev, seqs):
 
 @pytest.mark.parametrize("name", ["llama7b", "llama13b_mixed_bs16", "llama13b_mixed_bs32", "prefix_beams",
                                   "long_trace"])
-def test_full_size_sampled(pkv, name):
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_full_size_sampled(pkv, name, path):
     b = wl.make_decode_batch(name, with_data=False)
+    path_applies(b, path)
     rng = wl.rng_for(300)
     b.query = wl.bf16_normal(rng, (b.num_seqs, b.num_heads, b.head_dim))
     shape = (b.num_blocks, b.num_kv_heads, b.block_size, b.head_dim)
     kc, vc = device_pool(shape, 1), device_pool(shape, 2)
-    out = DeviceBatch(b, kc, vc).decode(pkv).cpu().numpy()
+    out = DeviceBatch(b, kc, vc).decode(pkv, path=PATHS[path]).cpu().numpy()
     assert np.all(np.isfinite(out))
     order = np.argsort(b.context_lens)
     seqs = sorted(set([int(order[0]), int(order[-1]), int(order[len(order) // 2])] +

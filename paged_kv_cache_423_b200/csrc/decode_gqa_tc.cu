@@ -46,9 +46,12 @@ constexpr int kChunks = kTile / kChunk;
 constexpr int kD = 128;                // head_dim of this path
 constexpr int kHalfBytes = kTile * 128;  // one 64-column half of a K or V tile: 16 KiB
 constexpr int kTileBytes = 2 * kHalfBytes;
-constexpr int kConsumers = 128;        // warps 0-3
-constexpr int kThreads = kConsumers + 32;
-constexpr int kTmemCols = 32;          // S in columns [0,16), O in [16,32)
+constexpr int kConsumers = 128;        // warps 0-3: softmax, one thread per TMEM lane
+constexpr int kProducerWarp = 4;       // TMA loads
+constexpr int kMmaWarp = 5;            // tcgen05.mma issue
+constexpr int kThreads = kConsumers + 64;
+constexpr int kTmemCols = 64;          // S double buffer in columns [0,16) and [16,32), O in [32,48)
+constexpr uint32_t kColO = 32;
 constexpr uint32_t kChunkTx = 4 * kChunk * 128;  // K and V, two halves each
 
 struct alignas(64) Args {
@@ -123,6 +126,20 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Named barrier that also returns the OR of `pred` over the participating threads.
+__device__ __forceinline__ bool named_barrier_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // Shared-memory matrix descriptor (sm_100 layout): start, leading/stride byte
 // offsets (16-byte units), version 1, swizzle mode 2 = 128-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -147,11 +164,12 @@ struct Layout {
   static constexpr int off_v = off_k + STAGES * kTileBytes;
   static constexpr int off_q = off_v + STAGES * kTileBytes;
   static constexpr int off_p = off_q + kQSlots * 4096;    // q slots sized for N <= 16
-  static constexpr int off_red = off_p + 4096;            // P: 2 K-atoms of N rows x 128 B
+  static constexpr int off_red = off_p + 2 * 4096;        // P double buffer: 2 K-atoms of N rows x 128 B each
   static constexpr int off_meta = off_red + 2 * 4 * 16 * 4;
   static constexpr int off_bar = off_meta + STAGES * 16;
-  static constexpr int off_misc = off_bar + (2 * STAGES + 2) * 8;
-  static constexpr int bytes = off_misc + 16;
+  static constexpr int kBars = 2 * STAGES + 8;            // full, empty, s_full[2], s_free[2], p_full[2], o_bar[2]
+  static constexpr int off_misc = off_bar + kBars * 8;
+  static constexpr int bytes = off_misc + 32;
   static constexpr int alloc = bytes + 1024;              // slack to align the base to 1024
 };
 
@@ -163,42 +181,62 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, floa
     static_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
 }
 
-// Column-wise maximum over the 32 rows a warp holds, for 16 columns at once: a
+// Column-wise reduction over the 32 rows a warp holds, for 16 columns at once: a
 // transposed butterfly (16 shuffles) that leaves column (lane >> 1) in both lanes
 // of each pair.
-__device__ __forceinline__ float warp_colmax16(const float (&x)[16], int lane) {
+template <bool MAX>
+__device__ __forceinline__ float warp_col16(const float (&x)[16], int lane) {
+  auto op = [](float u, float w) { return MAX ? fmaxf(u, w) : u + w; };
   float v[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const bool up = lane & 16;
     const float send = up ? x[i] : x[i + 8];
     const float keep = up ? x[i + 8] : x[i];
-    v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const bool up = lane & 8;
     const float send = up ? v[i] : v[i + 4];
     const float keep = up ? v[i + 4] : v[i];
-    v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
   }
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const bool up = lane & 4;
     const float send = up ? v[i] : v[i + 2];
     const float keep = up ? v[i + 2] : v[i];
-    v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
   }
   {
     const bool up = lane & 2;
     const float send = up ? v[0] : v[1];
     const float keep = up ? v[1] : v[0];
-    v[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+    v[0] = op(keep, __shfl_xor_sync(0xffffffffu, send, 2));
   }
-  return fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
+  return op(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
 }
 
-// meta.w bits: n_valid (8) | chunk mask << 8 (8) | first << 16 | last << 17 | with_q << 18
+// Softmax rows are rescaled only when a score exceeds the held maximum by more
+// than 2^kRescaleLog2 (weights up to 256 before normalisation, harmless in bf16
+// and fp32); otherwise P uses the held maximum and P·V keeps accumulating in TMEM.
+constexpr float kRescaleLog2 = 8.f;
+
+// Stage metadata, written by the producer:
+//   x = sequence, y = kv head | q slot << 16, z = partition | partitions << 16,
+//   w = valid rows (8 bits) | chunk mask << 8 | first << 16 | last << 17 | end of stream << 18
+constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
+
+// Pipeline (per CTA, persistent over work items):
+//   producer warp  -> full[s]      : K, V (and q on an item's first tile) landed in stage s
+//   MMA warp       -> s_full[b]    : S = K·Qᵀ of a tile is in TMEM buffer b (two buffers)
+//   softmax warps  -> s_free[b]    : S buffer b has been read
+//   softmax warps  -> p_full[b]    : P of the tile is in shared buffer b (two buffers)
+//   MMA warp       -> o_bar[b]     : O += Vᵀ·P of that tile is done (P buffer b reusable)
+//   MMA warp       -> empty[s]     : stage s may be refilled
+// The MMA warp never blocks on one side while the other could proceed: it polls
+// both (QK of the next landed tile, PV of the next tile whose P is ready).
 template <int STAGES, int N, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid_constant__ Args args) {
   static_assert(N == 16, "the tile is M = 128 rows, whose narrowest MMA is N = 16");
@@ -209,16 +247,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   unsigned char* k_ring = smem + L::off_k;
   unsigned char* v_ring = smem + L::off_v;
   unsigned char* q_ring = smem + L::off_q;
-  unsigned char* p_tile = smem + L::off_p;
+  unsigned char* p_buf = smem + L::off_p;                    // [2][4096]
   float* red = reinterpret_cast<float*>(smem + L::off_red);  // [2][4 warps][16]
   int4* meta = reinterpret_cast<int4*>(smem + L::off_meta);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* empty = full + STAGES;
-  uint64_t* s_bar = empty + STAGES;   // S of a tile is ready
-  uint64_t* o_bar = s_bar + 1;        // O of a tile is ready
+  uint64_t* s_full = empty + STAGES;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* o_bar = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::off_misc + 4);
-  int* merge_flag = reinterpret_cast<int*>(smem + L::off_misc + 8);
+  volatile int* restart_flag = reinterpret_cast<volatile int*>(smem + L::off_misc + 8);  // [2]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = a.group;
@@ -229,13 +269,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(s_bar, 1);
-    mbar_init(o_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 4);  // one arrival per softmax warp
+      mbar_init(&p_full[b], 4);
+      mbar_init(&o_bar[b], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
   // P rows of unused heads (g..N-1) stay zero for the whole kernel.
-  for (int i = tid; i < 4096 / 16; i += blockDim.x) reinterpret_cast<uint4*>(p_tile)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < 2 * 4096 / 16; i += blockDim.x) reinterpret_cast<uint4*>(p_buf)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -243,39 +287,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ================= producer =================
     const uint64_t policy = l2_policy_evict_first();
-    int n = 0;  // fills issued
-    int item_ord = 0;
-    for (int64_t item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x, ++item_ord) {
-      const PlanEntry e = a.entries[item / a.num_kv_heads];
-      const int kvh = static_cast<int>(item % a.num_kv_heads);
+    const int64_t G = gridDim.x;
+    auto load_entry = [&](int64_t it) -> PlanEntry {
+      return it < n_items ? a.entries[it / a.num_kv_heads] : make_int4(0, 0, 0, 0);
+    };
+    auto load_tab = [&](const PlanEntry& e) -> int {
       const int tok0 = e.y * a.partition;
       const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - tok0);
       const int nblk = (ntok + a.block_size - 1) / a.block_size;
-      const int tab = lane < nblk ? __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + lane) : 0;
+      return lane < nblk ? __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + lane)
+                         : 0;
+    };
+    // Plan entries and table slices are fetched one and two items ahead.
+    int64_t item = blockIdx.x;
+    PlanEntry e_cur = load_entry(item);
+    int tab_cur = item < n_items ? load_tab(e_cur) : 0;
+    PlanEntry e_nxt = load_entry(item + G);
+    int tab_nxt = item + G < n_items ? load_tab(e_nxt) : 0;
+    PlanEntry e_nx2 = load_entry(item + 2 * G);
+    int n = 0;  // fills issued
+    int item_ord = 0;
+    bool failed = false;
+    auto acquire = [&](int slot) -> bool {
+      if (n >= STAGES && !mbar_wait(&empty[slot], ((n / STAGES) - 1) & 1)) {
+        *abort_flag = 1;
+        set_status(a.status, PKV_DEV_TIMEOUT);
+        return false;
+      }
+      return true;
+    };
+    while (item < n_items && !failed && !*abort_flag) {
+      const PlanEntry e = e_cur;
+      const int kvh = static_cast<int>(item % a.num_kv_heads);
+      const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - e.y * a.partition);
       const int ntiles = ntok == 0 ? 1 : (ntok + kTile - 1) / kTile;
+      const int qslot = item_ord % L::kQSlots;
       for (int tile = 0; tile < ntiles; ++tile, ++n) {
         const int slot = n % STAGES;
-        if (n >= STAGES && !mbar_wait(&empty[slot], ((n / STAGES) - 1) & 1)) {
-          *abort_flag = 1;
-          set_status(a.status, PKV_DEV_TIMEOUT);
+        if (!acquire(slot)) {
+          failed = true;
           break;
         }
         const int n_valid = max(0, min(kTile, ntok - tile * kTile));
         const int nchunks = (n_valid + kChunk - 1) / kChunk;
         const int ltok = tile * kTile + lane * kChunk;  // this lane's chunk (lane < nchunks)
-        const int phys = __shfl_sync(0xffffffffu, tab, min(31, ltok / a.block_size));
+        const int phys = __shfl_sync(0xffffffffu, tab_cur, min(31, ltok / a.block_size));
         const bool mine = lane < nchunks;
         const bool ok = mine && phys >= 0 && phys < a.num_blocks;
         const uint32_t mask = __ballot_sync(0xffffffffu, ok);
         if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
         const bool with_q = tile == 0 && ntok > 0;
         if (lane == 0) {
-          meta[slot] = make_int4(e.x, kvh, e.y | (e.z << 16),
-                                 n_valid | (mask << 8) | (tile == 0 ? 1 << 16 : 0) | (tile == ntiles - 1 ? 1 << 17 : 0) |
-                                     (with_q ? 1 << 18 : 0));
+          meta[slot] = make_int4(e.x, kvh | (qslot << 16), e.y | (e.z << 16),
+                                 n_valid | (mask << 8) | (tile == 0 ? kMetaFirst : 0) | (tile == ntiles - 1 ? kMetaLast : 0));
           mbar_arrive_expect_tx(&full[slot], __popc(mask) * kChunkTx + (with_q ? L::kQBytes : 0));
         }
         __syncwarp();
@@ -289,211 +356,291 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           tma_load_2d(vd + kHalfBytes, &args.tm_v, 64, row, &full[slot], policy);
         }
         if (with_q && lane == 0) {
-          // The producer runs at most STAGES tiles (so STAGES items) ahead of the
-          // consumers: STAGES + 1 q slots never overwrite the q still in use.
+          // The producer runs at most STAGES fills (so STAGES items) ahead of the
+          // last released stage: STAGES + 1 q slots never overwrite a q in use.
           const int qrow = e.x * a.num_heads + kvh * g;
-          unsigned char* qd = q_ring + (item_ord % L::kQSlots) * 4096;
+          unsigned char* qd = q_ring + qslot * 4096;
           tma_load_2d(qd, &args.tm_q, 0, qrow, &full[slot], policy);
           tma_load_2d(qd + N * 128, &args.tm_q, 64, qrow, &full[slot], policy);
         }
       }
+      item += G;
+      ++item_ord;
+      e_cur = e_nxt;
+      tab_cur = tab_nxt;
+      e_nxt = e_nx2;
+      tab_nxt = item + G < n_items ? load_tab(e_nxt) : 0;
+      e_nx2 = load_entry(item + 2 * G);
+    }
+    if (!failed && !*abort_flag) {
+      // end-of-stream marker: a fill with no data
+      const int slot = n % STAGES;
+      if (acquire(slot)) {
+        if (lane == 0) {
+          meta[slot] = make_int4(0, 0, 0, kMetaEnd);
+          mbar_arrive_expect_tx(&full[slot], 0);
+        }
+        ++n;
+      }
+      __syncwarp();
     }
     // Let this CTA's last copies land before the final barrier.
     for (int k = max(0, n - STAGES); k < n; ++k) mbar_wait(&full[k % STAGES], (k / STAGES) & 1);
-  } else {
-    // ================= consumers (one thread per TMEM lane) =================
-    constexpr uint32_t idesc_qk = instr_desc(kTile, N, false, false);
-    constexpr uint32_t idesc_pv = instr_desc(kD, N, true, false);
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tmem_s = tmem + lane_base;
-    const uint32_t tmem_o = tmem + lane_base + 16;
-    const uint32_t p_addr = smem_addr(p_tile);
-
-    // S = K · Qᵀ for the tile in `slot` (thread 0 only).
-    auto issue_qk = [&](int slot, int ord) {
-      const uint32_t k_addr = smem_addr(k_ring + slot * kTileBytes);
-      const uint32_t q_addr = smem_addr(q_ring + (ord % L::kQSlots) * 4096);
-      tc_fence_after();
+  } else if (warp == kMmaWarp) {
+    // ================= MMA issuer (one thread) =================
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = instr_desc(kTile, N, false, false);
+      constexpr uint32_t idesc_pv = instr_desc(kD, N, true, false);
+      const uint32_t p_addr0 = smem_addr(p_buf);
+      int qk_n = 0, pv_n = 0, end_n = 0x7fffffff;
+      int q_valid = 0, p_valid = 0;  // valid (non-empty) tiles that got their QK / PV
+      uint64_t idle_since = 0;
+      int idle = 0;
+      while (pv_n < end_n) {
+        bool progress = false;
+        // ---- QK of the next landed tile, if its S buffer is free
+        if (qk_n < end_n && mbar_test(&full[qk_n % STAGES], (qk_n / STAGES) & 1)) {
+          const int4 mt = meta[qk_n % STAGES];
+          if (mt.w & kMetaEnd) {
+            end_n = qk_n;
+            progress = true;
+          } else if ((mt.w & 0xff) == 0) {
+            ++qk_n;
+            progress = true;
+          } else {
+            const int b = q_valid & 1;
+            if (q_valid < 2 || mbar_test(&s_free[b], ((q_valid >> 1) - 1) & 1)) {
+              tc_fence_after();
+              const int slot = qk_n % STAGES;
+              const uint32_t k_addr = smem_addr(k_ring + slot * kTileBytes);
+              const uint32_t q_addr = smem_addr(q_ring + (mt.y >> 16) * 4096);
 #pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        const uint32_t qoff = (kk >> 2) * (N * 128) + (kk & 3) * 32;
-        umma(tmem, smem_desc_sw128(k_addr + koff, 16, 1024), smem_desc_sw128(q_addr + qoff, 16, 1024), idesc_qk,
-             kk > 0);
+              for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                const uint32_t qoff = (kk >> 2) * (N * 128) + (kk & 3) * 32;
+                umma(tmem + b * 16, smem_desc_sw128(k_addr + koff, 16, 1024),
+                     smem_desc_sw128(q_addr + qoff, 16, 1024), idesc_qk, kk > 0);
+              }
+              umma_commit(&s_full[b]);
+              ++q_valid;
+              ++qk_n;
+              progress = true;
+            }
+          }
+        }
+        // ---- PV of the oldest tile whose P is ready
+        if (pv_n < qk_n) {
+          const int slot = pv_n % STAGES;
+          const int4 mt = meta[slot];
+          if ((mt.w & 0xff) == 0) {
+            mbar_arrive(&empty[slot]);
+            ++pv_n;
+            progress = true;
+          } else {
+            const int b = p_valid & 1;
+            if (mbar_test(&p_full[b], (p_valid >> 1) & 1)) {
+              tc_fence_after();
+              const bool restart = restart_flag[b] != 0;
+              const uint32_t v_addr = smem_addr(v_ring + slot * kTileBytes);
+              const uint32_t p_addr = p_addr0 + b * 4096;
+              const int kt = ((mt.w & 0xff) + 15) / 16;
+              for (int kk = 0; kk < kt; ++kk) {
+                const uint32_t poff = (kk >> 2) * (N * 128) + (kk & 3) * 32;
+                umma(tmem + kColO, smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024),
+                     smem_desc_sw128(p_addr + poff, 16, 1024), idesc_pv, kk > 0 || !restart);
+              }
+              umma_commit(&o_bar[b]);
+              umma_commit(&empty[slot]);
+              ++p_valid;
+              ++pv_n;
+              progress = true;
+            }
+          }
+        }
+        if (progress) {
+          idle = 0;
+        } else if (++idle == 64) {
+          idle_since = global_timer_ns();
+        } else if (idle > 64 && (idle & 63) == 0) {
+          if (*abort_flag || global_timer_ns() - idle_since > kWaitLimitNs) {
+            *abort_flag = 1;
+            set_status(a.status, PKV_DEV_TIMEOUT);
+            break;
+          }
+        }
       }
-      umma_commit(s_bar);
+    }
+    __syncwarp();
+  } else {
+    // ================= softmax warps (one thread per TMEM lane) =================
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m_used[N], lp[N], o_reg[N];
+#pragma unroll
+    for (int h = 0; h < N; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f;
+    bool restart = true;           // the next P·V starts a fresh TMEM accumulation
+    bool pv_since_restart = false;
+    int n_valid_tiles = 0;
+    uint32_t ob_next = 0;     // bit b: parity of the phase the next P·V on o_bar[b] completes
+    uint32_t ob_pending = 0;  // bit b: the last P·V on o_bar[b] has not been waited for yet
+    auto wait_ob = [&](int b) -> bool {
+      if (!((ob_pending >> b) & 1)) return true;
+      ob_pending &= ~(1u << b);
+      return mbar_wait(&o_bar[b], ((ob_next >> b) & 1) ^ 1u);
     };
 
-    float m[N], lp[N], oacc[N], alpha[N];
+    for (int n = 0;; ++n) {
+      const int slot = n % STAGES;
+      bool bad = !mbar_wait(&full[slot], (n / STAGES) & 1);
+      const int4 mt = meta[slot];
+      if (mt.w & kMetaEnd) break;
+      const int n_valid = mt.w & 0xff;
+      const uint32_t mask = (mt.w >> 8) & 0xff;
+      const bool first = mt.w & kMetaFirst, last = mt.w & kMetaLast;
+      if (first) {
 #pragma unroll
-    for (int h = 0; h < N; ++h) m[h] = -INFINITY, lp[h] = 0.f, oacc[h] = 0.f, alpha[h] = 1.f;
-    int s_phase = 0, o_phase = 0;
-    int n = 0;
-    int item_ord = 0;
-    // Thread 0 issues the first tile's S before the loop; afterwards S of tile n+1
-    // is issued right behind O of tile n, so the tensor core computes it while the
-    // other threads finish tile n.
-    if (tid == 0 && n_items > blockIdx.x) {
-      if (!mbar_wait(&full[0], 0)) *abort_flag = 1;
-      else if ((meta[0].w & 0xff) > 0) issue_qk(0, 0);
-    }
-    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ord) {
-      const PlanEntry e = a.entries[item / a.num_kv_heads];
-      const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - e.y * a.partition);
-      const int ntiles = ntok == 0 ? 1 : (ntok + kTile - 1) / kTile;
-      const bool more_items = item + gridDim.x < n_items;
-      bool stop = false;
-      for (int tile = 0; tile < ntiles; ++tile, ++n) {
-        const int slot = n % STAGES;
-        if (!mbar_wait(&full[slot], (n / STAGES) & 1)) *abort_flag = 1;
-        named_barrier_sync(1, kConsumers);
-        if (*abort_flag) {
-          stop = true;
-          break;
+        for (int h = 0; h < N; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f;
+        restart = true;
+        pv_since_restart = false;
+      }
+      if (n_valid > 0) {
+        const int b = n_valid_tiles & 1;
+        unsigned char* p_tile = p_buf + b * 4096;
+        bad |= !mbar_wait(&s_full[b], (n_valid_tiles >> 1) & 1);
+        tc_fence_after();
+        float s[N];
+        tmem_load_row<N>(tmem + lane_base + b * 16, s);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[b]);
+        bad |= !wait_ob(b);  // P buffer b: the P·V of two valid tiles back is done
+        const int t = tid;   // this thread's row = token of the tile
+        const bool valid = t < n_valid && ((mask >> (t / kChunk)) & 1);
+        float x[N];
+        bool need = false;
+#pragma unroll
+        for (int h = 0; h < N; ++h) {
+          x[h] = (valid && h < g) ? s[h] * a.scale_log2 : -INFINITY;
+          need |= x[h] > m_used[h] + kRescaleLog2;
         }
-        const int4 mt = meta[slot];
-        const int n_valid = mt.w & 0xff;
-        const uint32_t mask = (mt.w >> 8) & 0xff;
-        const bool first = (mt.w >> 16) & 1, last = (mt.w >> 17) & 1;
-        if (first) {
-#pragma unroll
-          for (int h = 0; h < N; ++h) m[h] = -INFINITY, lp[h] = 0.f, oacc[h] = 0.f;
-        }
-        // the tile after this one (in this CTA's stream), whose S thread 0 issues early
-        const bool has_next = tile + 1 < ntiles || more_items;
-        const int next_slot = (n + 1) % STAGES;
-        const int next_ord = tile + 1 < ntiles ? item_ord : item_ord + 1;
-        if (n_valid > 0) {
-          const uint32_t v_addr = smem_addr(v_ring + slot * kTileBytes);
-          if (!mbar_wait(s_bar, s_phase)) *abort_flag = 1;
-          s_phase ^= 1;
-          tc_fence_after();
-          float s[N];
-          tmem_load_row<N>(tmem_s, s);
-          // ---- online softmax over this tile's rows, per query head (column)
-          const int t = tid;  // this thread's row = token of the tile
-          const bool valid = t < n_valid && ((mask >> (t / kChunk)) & 1);
-          float x[N];
-#pragma unroll
-          for (int h = 0; h < N; ++h) x[h] = (valid && h < g) ? s[h] * a.scale_log2 : -INFINITY;
-          const float wmax = warp_colmax16(x, lane);
-          if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = wmax;
-          named_barrier_sync(1, kConsumers);
+        // P[t][h] into the K-major, 128-byte-swizzled B operand (rows = heads)
+        const int katom = t >> 6, chunk = (t & 63) >> 3;
+        float pv[N];
+        auto write_p = [&]() {
 #pragma unroll
           for (int h = 0; h < N; ++h) {
             if (h >= g) break;
-            const float tmax = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
-            const float m_new = fmaxf(m[h], tmax);
-            alpha[h] = m_new == -INFINITY ? 1.f : exp2f(m[h] - m_new);
-            m[h] = m_new;
-            const float p = valid ? exp2f(x[h] - m_new) : 0.f;
+            const float p = (valid && m_used[h] > -INFINITY) ? exp2f(x[h] - m_used[h]) : 0.f;
             const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-            lp[h] = fmaf(lp[h], alpha[h], __bfloat162float(pb));
-            // P[t][h] into the K-major, 128-byte-swizzled B operand (rows = heads)
-            const int katom = t >> 6, chunk = (t & 63) >> 3;
+            pv[h] = __bfloat162float(pb);
             const int off = katom * (N * 128) + h * 128 + ((chunk ^ (h & 7)) << 4) + ((t & 7) << 1);
             *reinterpret_cast<__nv_bfloat16*>(p_tile + off) = pb;
           }
-          if (!valid) {
-            // rows of V outside the context may hold anything (even NaN): zero them
-            uint4* r0 = reinterpret_cast<uint4*>(v_ring + slot * kTileBytes + t * 128);
-            uint4* r1 = reinterpret_cast<uint4*>(v_ring + slot * kTileBytes + kHalfBytes + t * 128);
+        };
+        write_p();
+        if (!valid) {
+          // rows of V outside the context may hold anything (even NaN): zero them
+          uint4* r0 = reinterpret_cast<uint4*>(v_ring + slot * kTileBytes + t * 128);
+          uint4* r1 = reinterpret_cast<uint4*>(v_ring + slot * kTileBytes + kHalfBytes + t * 128);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) r0[c] = r1[c] = make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          named_barrier_sync(1, kConsumers);
-          if (tid == 0) {
-            // ---- O = Vᵀ · P over the tile's valid 16-row slices
-            tc_fence_after();
-            const int kt = (n_valid + 15) / 16;
-            for (int kk = 0; kk < kt; ++kk) {
-              const uint32_t poff = (kk >> 2) * (N * 128) + (kk & 3) * 32;
-              umma(tmem + 16, smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024),
-                   smem_desc_sw128(p_addr + poff, 16, 1024), idesc_pv, kk > 0);
-            }
-            umma_commit(o_bar);
-            umma_commit(&empty[slot]);
-            // ---- S of the next tile (S of this tile has been read by every thread)
-            if (has_next) {
-              if (!mbar_wait(&full[next_slot], ((n + 1) / STAGES) & 1)) *abort_flag = 1;
-              else if ((meta[next_slot].w & 0xff) > 0) issue_qk(next_slot, next_ord);
-            }
-          }
-          if (!mbar_wait(o_bar, o_phase)) *abort_flag = 1;
-          o_phase ^= 1;
-          tc_fence_after();
-          float o[N];
-          tmem_load_row<N>(tmem_o, o);
-#pragma unroll
-          for (int h = 0; h < N; ++h) oacc[h] = fmaf(oacc[h], alpha[h], o[h]);
-          tc_fence_before();
-        } else if (tid == 0) {
-          mbar_arrive(&empty[slot]);  // nothing to compute: hand the stage back
-          if (has_next) {
-            if (!mbar_wait(&full[next_slot], ((n + 1) / STAGES) & 1)) *abort_flag = 1;
-            else if ((meta[next_slot].w & 0xff) > 0) issue_qk(next_slot, next_ord);
-          }
+          for (int c = 0; c < 8; ++c) r0[c] = r1[c] = make_uint4(0, 0, 0, 0);
         }
-        if (last) {
-          // ---- finalize the item: softmax denominators, then the output (or a partial)
-          float* red2 = red + 64;
+        if (tid == 0) restart_flag[b] = restart;
+        if (bad) *abort_flag = 1;
+        fence_proxy_async_smem();
+        const bool need_any = named_barrier_or(1, kConsumers, need || bad);
+        if (*abort_flag) break;
+        if (need_any) {
+          // A score outgrew the held maximum: take the tile maximum, fold the
+          // accumulated P·V into registers at the old scale, and redo P.
+          const float wmax = warp_col16<true>(x, lane);
+          if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = wmax;
+          bool ok = wait_ob(0);
+          ok &= wait_ob(1);
+          named_barrier_sync(1, kConsumers);
+          float alpha[N];
 #pragma unroll
           for (int h = 0; h < N; ++h) {
-            if (h >= g) break;
-            float w = lp[h];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) w += __shfl_xor_sync(0xffffffffu, w, off);
-            if (lane == 0) red2[warp * 16 + h] = w;
+            const float tmax = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
+            if (h < g) {
+              // nothing is accumulated yet while the held maximum is -inf
+              const float m_new = fmaxf(m_used[h], tmax);
+              alpha[h] = m_used[h] == -INFINITY ? 0.f : exp2f(m_used[h] - m_new);
+              m_used[h] = m_new;
+            } else {
+              alpha[h] = 1.f;
+            }
           }
-          named_barrier_sync(1, kConsumers);
-          const int seq = mt.x, kvh = mt.y, part = mt.z & 0xffff, nparts = mt.z >> 16;
-          const int d = tid;
-          if (nparts == 1) {
+          tc_fence_after();
+          if (pv_since_restart) {
+            float o[N];
+            tmem_load_row<N>(tmem + lane_base + kColO, o);
 #pragma unroll
-            for (int h = 0; h < N; ++h) {
-              if (h >= g) break;
-              const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
-              store_out<OUT_F32>(a, (static_cast<int64_t>(seq) * a.num_heads + kvh * g + h) * kD + d,
-                                 l > 0.f ? oacc[h] / l : 0.f);
-            }
+            for (int h = 0; h < N; ++h) o_reg[h] = (o_reg[h] + o[h]) * alpha[h];
           } else {
-            const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
 #pragma unroll
-            for (int h = 0; h < N; ++h) {
-              if (h >= g) break;
-              const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
-              const int64_t pidx = (unit0 + h) * a.max_parts + part;
-              a.part_o[pidx * kD + d] = oacc[h];
-              if (d == 0) a.part_ml[pidx] = make_float2(m[h], l);
-            }
-            __threadfence();
-            named_barrier_sync(1, kConsumers);
-            if (tid == 0) *merge_flag = atomicAdd(a.arrive + unit0, 1) == nparts - 1;
-            named_barrier_sync(1, kConsumers);
-            if (*merge_flag) {
-              __threadfence();
-              for (int h = 0; h < g; ++h) {
-                const float2* ml = a.part_ml + (unit0 + h) * a.max_parts;
-                const float* po = a.part_o + (unit0 + h) * a.max_parts * kD + d;
-                float M = -INFINITY;
-                for (int p = 0; p < nparts; ++p) M = fmaxf(M, __ldcg(&ml[p].x));
-                float acc = 0.f, Ls = 0.f;
-                for (int p = 0; p < nparts; ++p) {
-                  const float2 mlp = __ldcg(&ml[p]);
-                  const float w = exp2f(mlp.x - M);
-                  Ls = fmaf(w, mlp.y, Ls);
-                  acc = fmaf(w, __ldcg(po + static_cast<int64_t>(p) * kD), acc);
-                }
-                store_out<OUT_F32>(a, (unit0 + h) * kD + d, Ls > 0.f ? acc / Ls : 0.f);
-              }
-              if (tid == 0) a.arrive[unit0] = 0;
-            }
+            for (int h = 0; h < N; ++h) o_reg[h] *= alpha[h];
+          }
+          tc_fence_before();
+#pragma unroll
+          for (int h = 0; h < N; ++h) lp[h] *= alpha[h];
+          restart = true;
+          pv_since_restart = false;
+          write_p();
+          if (tid == 0) restart_flag[b] = 1;
+          if (!ok) *abort_flag = 1;
+          fence_proxy_async_smem();
+          named_barrier_sync(1, kConsumers);
+        }
+#pragma unroll
+        for (int h = 0; h < N; ++h)
+          if (h < g) lp[h] += pv[h];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+        ob_next ^= 1u << b;
+        ob_pending |= 1u << b;
+        restart = false;
+        pv_since_restart = true;
+        ++n_valid_tiles;
+      }
+      if (last) {
+        // ---- finalize the item: O = registers + TMEM, denominators, output or partial
+        bool ok = wait_ob(0);
+        ok &= wait_ob(1);
+        tc_fence_after();
+        float ot[N];
+        if (pv_since_restart) {
+          float o[N];
+          tmem_load_row<N>(tmem + lane_base + kColO, o);
+#pragma unroll
+          for (int h = 0; h < N; ++h) ot[h] = o_reg[h] + o[h];
+        } else {
+#pragma unroll
+          for (int h = 0; h < N; ++h) ot[h] = o_reg[h];
+        }
+        tc_fence_before();
+        if (!ok) *abort_flag = 1;
+        float* red2 = red + 64;
+        const float wsum = warp_col16<false>(lp, lane);
+        if ((lane & 1) == 0) red2[warp * 16 + (lane >> 1)] = wsum;
+        named_barrier_sync(1, kConsumers);
+        const int seq = mt.x, kvh = mt.y & 0xffff, part = mt.z & 0xffff, nparts = mt.z >> 16;
+        const int d = tid;
+        const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
+#pragma unroll
+        for (int h = 0; h < N; ++h) {
+          if (h >= g) break;
+          const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
+          if (nparts == 1) {
+            store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[h] / l : 0.f);
+          } else {
+            // unnormalised partial; a separate kernel merges the partitions
+            const int64_t pidx = (unit0 + h) * a.max_parts + part;
+            a.part_o[pidx * kD + d] = ot[h];
+            if (d == 0) a.part_ml[pidx] = make_float2(m_used[h], l);
           }
         }
+        // red2 is rewritten only after the next item's barriers
       }
-      if (stop) break;
     }
     if (*abort_flag && tid == 0) set_status(a.status, PKV_DEV_TIMEOUT);
   }
@@ -501,6 +648,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Merge of split partitions: one warp per (sequence, query head) whose context was
+// split, o = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.  Runs after the main
+// kernel on the same stream; lane l owns output values 4l .. 4l+3.
+template <bool OUT_F32>
+__global__ void __launch_bounds__(256) merge_partials_kernel(const DecodeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n_units = static_cast<int64_t>(a.plan_count[0]) * a.num_heads;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); u < n_units;
+       u += stride) {
+    const PlanEntry e = a.entries[u / a.num_heads];
+    if (e.y != 0 || e.z <= 1) continue;  // one warp per split sequence and head
+    const int h = static_cast<int>(u % a.num_heads);
+    const int nparts = e.z;
+    const int64_t unit = static_cast<int64_t>(e.x) * a.num_heads + h;
+    const float2* ml = a.part_ml + unit * a.max_parts;
+    const float* po = a.part_o + unit * a.max_parts * kD + lane * 4;
+    float M = -INFINITY;
+    for (int p = lane; p < nparts; p += 32) M = fmaxf(M, ml[p].x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Ls = 0.f;
+    for (int base = 0; base < nparts; base += 32) {
+      const int p = base + lane;
+      float w = 0.f;
+      if (p < nparts) {
+        const float2 v = ml[p];
+        w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+        Ls = fmaf(w, v.y, Ls);
+      }
+      const int cnt = min(32, nparts - base);
+#pragma unroll 8
+      for (int j = 0; j < cnt; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, j);
+        const float4 o = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(base + j) * kD);
+        acc.x = fmaf(wj, o.x, acc.x);
+        acc.y = fmaf(wj, o.y, acc.y);
+        acc.z = fmaf(wj, o.z, acc.z);
+        acc.w = fmaf(wj, o.w, acc.w);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    const int64_t base = unit * kD + lane * 4;
+    store_out<OUT_F32>(a, base + 0, acc.x * inv);
+    store_out<OUT_F32>(a, base + 1, acc.y * inv);
+    store_out<OUT_F32>(a, base + 2, acc.z * inv);
+    store_out<OUT_F32>(a, base + 3, acc.w * inv);
+  }
 }
 
 // ---- host side -----------------------------------------------------------
@@ -549,6 +749,11 @@ static int launch(const Args& args, cudaStream_t stream) {
   kernel<<<std::max(1, sms), kThreads, smem, stream>>>(args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) launch: %s", cudaGetErrorString(e));
+  if (args.a.max_parts > 1) {
+    merge_partials_kernel<OUT_F32><<<std::max(1, sms) * 4, 256, 0, stream>>>(args.a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) merge launch: %s", cudaGetErrorString(e));
+  }
   return PKV_OK;
 }
 

@@ -147,6 +147,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// Same, without swizzle (core matrices of 8 rows x 16 bytes).
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFF) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
+}
+
+// 2^x with the SFU's approximate exponential (relative error ~2^-22, tiny inputs
+// flush to zero); used for softmax weights that are rounded to bf16 anyway.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A/B major-ness,
 // N >> 3 and M >> 4.
 __host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn_major, bool b_mn_major) {
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
     // ================= MMA issuer (one thread) =================
     if (lane == 0) {
       constexpr uint32_t idesc_qk = instr_desc(kTile, N, false, false);
-      constexpr uint32_t idesc_pv = instr_desc(kD, N, true, false);
+      constexpr uint32_t idesc_pv = instr_desc(kD, N, true, true);
       const uint32_t p_addr0 = smem_addr(p_buf);
       int qk_n = 0, pv_n = 0, end_n = 0x7fffffff;
       int q_valid = 0, p_valid = 0;  // valid (non-empty) tiles that got their QK / PV
@@ -445,9 +459,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
               const uint32_t p_addr = p_addr0 + b * 4096;
               const int kt = ((mt.w & 0xff) + 15) / 16;
               for (int kk = 0; kk < kt; ++kk) {
-                const uint32_t poff = (kk >> 2) * (N * 128) + (kk & 3) * 32;
+                // P: MN-major, unswizzled; 8-token groups 128 B apart, heads 8..15 2 KiB on
                 umma(tmem + kColO, smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024),
-                     smem_desc_sw128(p_addr + poff, 16, 1024), idesc_pv, kk > 0 || !restart);
+                     smem_desc_plain(p_addr + kk * 256, 128, 2048), idesc_pv, kk > 0 || !restart);
               }
               umma_commit(&o_bar[b]);
               umma_commit(&empty[slot]);
@@ -459,13 +473,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         }
         if (progress) {
           idle = 0;
-        } else if (++idle == 64) {
-          idle_since = global_timer_ns();
-        } else if (idle > 64 && (idle & 63) == 0) {
-          if (*abort_flag || global_timer_ns() - idle_since > kWaitLimitNs) {
-            *abort_flag = 1;
-            set_status(a.status, PKV_DEV_TIMEOUT);
-            break;
+        } else {
+          // Back off briefly: this warp shares its scheduler with a softmax warp.
+          __nanosleep(32);
+          if (++idle == 64) {
+            idle_since = global_timer_ns();
+          } else if (idle > 64 && (idle & 63) == 0) {
+            if (*abort_flag || global_timer_ns() - idle_since > kWaitLimitNs) {
+              *abort_flag = 1;
+              set_status(a.status, PKV_DEV_TIMEOUT);
+              break;
+            }
           }
         }
       }
@@ -522,21 +540,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           x[h] = (valid && h < g) ? s[h] * a.scale_log2 : -INFINITY;
           need |= x[h] > m_used[h] + kRescaleLog2;
         }
-        // P[t][h] into the K-major, 128-byte-swizzled B operand (rows = heads)
-        const int katom = t >> 6, chunk = (t & 63) >> 3;
+        // P row of this token (B operand, MN-major, unswizzled): heads 0..7 as one
+        // 16-byte chunk at (t/8)*128 + (t%8)*16, heads 8..15 2 KiB further.
         float pv[N];
         auto write_p = [&]() {
+          uint32_t w[N / 2];
 #pragma unroll
-          for (int h = 0; h < N; ++h) {
-            if (h >= g) break;
-            const float p = (valid && m_used[h] > -INFINITY) ? exp2f(x[h] - m_used[h]) : 0.f;
-            const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-            pv[h] = __bfloat162float(pb);
-            const int off = katom * (N * 128) + h * 128 + ((chunk ^ (h & 7)) << 4) + ((t & 7) << 1);
-            *reinterpret_cast<__nv_bfloat16*>(p_tile + off) = pb;
+          for (int j = 0; j < N / 2; ++j) {
+            const int h0 = 2 * j, h1 = 2 * j + 1;
+            const float p0 = (valid && h0 < g && m_used[h0] > -INFINITY) ? fast_exp2(x[h0] - m_used[h0]) : 0.f;
+            const float p1 = (valid && h1 < g && m_used[h1] > -INFINITY) ? fast_exp2(x[h1] - m_used[h1]) : 0.f;
+            w[j] = pack_bf16x2(p0, p1);
+            pv[h0] = bf16lo(w[j]);
+            pv[h1] = bf16hi(w[j]);
           }
+          unsigned char* row = p_tile + (t >> 3) * 128 + (t & 7) * 16;
+          *reinterpret_cast<uint4*>(row) = make_uint4(w[0], w[1], w[2], w[3]);
+          if (g > 8) *reinterpret_cast<uint4*>(row + 2048) = make_uint4(w[4], w[5], w[6], w[7]);
         };
-        write_p();
         if (!valid) {
           // rows of V outside the context may hold anything (even NaN): zero them
           uint4* r0 = reinterpret_cast<uint4*>(v_ring + slot * kTileBytes + t * 128);
@@ -544,19 +565,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
 #pragma unroll
           for (int c = 0; c < 8; ++c) r0[c] = r1[c] = make_uint4(0, 0, 0, 0);
         }
-        if (tid == 0) restart_flag[b] = restart;
         if (bad) *abort_flag = 1;
-        fence_proxy_async_smem();
-        const bool need_any = named_barrier_or(1, kConsumers, need || bad);
-        if (*abort_flag) break;
+        bool need_any = true;  // an item's first tile always sets the held maximum
+        if (!first) {
+          write_p();
+          if (tid == 0) restart_flag[b] = restart;
+          fence_proxy_async_smem();
+          need_any = named_barrier_or(1, kConsumers, need || bad);
+          if (*abort_flag) break;
+        }
         if (need_any) {
-          // A score outgrew the held maximum: take the tile maximum, fold the
-          // accumulated P·V into registers at the old scale, and redo P.
+          // A score outgrew the held maximum (or none is held yet): take the tile
+          // maximum, fold the accumulated P·V into registers at the old scale, and
+          // (re)write P.
           const float wmax = warp_col16<true>(x, lane);
           if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = wmax;
           bool ok = wait_ob(0);
           ok &= wait_ob(1);
+          if (!ok) *abort_flag = 1;
           named_barrier_sync(1, kConsumers);
+          if (*abort_flag) break;
           float alpha[N];
 #pragma unroll
           for (int h = 0; h < N; ++h) {
@@ -564,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
             if (h < g) {
               // nothing is accumulated yet while the held maximum is -inf
               const float m_new = fmaxf(m_used[h], tmax);
-              alpha[h] = m_used[h] == -INFINITY ? 0.f : exp2f(m_used[h] - m_new);
+              alpha[h] = m_used[h] == -INFINITY ? 0.f : fast_exp2(m_used[h] - m_new);
               m_used[h] = m_new;
             } else {
               alpha[h] = 1.f;
@@ -587,7 +615,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           pv_since_restart = false;
           write_p();
           if (tid == 0) restart_flag[b] = 1;
-          if (!ok) *abort_flag = 1;
           fence_proxy_async_smem();
           named_barrier_sync(1, kConsumers);
         }

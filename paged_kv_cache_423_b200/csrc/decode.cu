@@ -42,14 +42,20 @@ constexpr unsigned kFull = 0xffffffffu;
 
 constexpr int kPlanThreads = 1024;
 
+// Bucket of an entry of `ntok` tokens: longest first, 513 buckets whatever the
+// split size (exact for splits up to 512 tokens, coarser beyond).
+__device__ __forceinline__ int plan_bucket(int ntok, int partition) {
+  return static_cast<int>((static_cast<int64_t>(partition - ntok) * (kPlanBuckets - 1)) / partition);
+}
+
 __global__ void __launch_bounds__(kPlanThreads)
     plan_kernel(const int32_t* __restrict__ context_lens, int num_seqs, int max_context_len, int max_table_tokens,
                 int partition, PlanEntry* __restrict__ entries, int32_t* __restrict__ plan_count,
                 int32_t* __restrict__ arrive, int n_arrive, int32_t* status) {
-  __shared__ int bucket[kMaxPartition + 1];  // bucket k holds entries of partition - k tokens
+  __shared__ int bucket[kPlanBuckets];
   __shared__ int warp_total[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i <= partition; i += blockDim.x) bucket[i] = 0;
+  for (int i = tid; i < kPlanBuckets; i += blockDim.x) bucket[i] = 0;
   for (int i = tid; i < n_arrive; i += blockDim.x) arrive[i] = 0;
   __syncthreads();
   for (int s = tid; s < num_seqs; s += blockDim.x) {
@@ -61,12 +67,12 @@ __global__ void __launch_bounds__(kPlanThreads)
     const int np = L == 0 ? 1 : (L + partition - 1) / partition;
     for (int p = 0; p < np; ++p) {
       const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
-      atomicAdd(&bucket[partition - ntok], 1);
+      atomicAdd(&bucket[plan_bucket(ntok, partition)], 1);
     }
   }
   __syncthreads();
-  // Exclusive scan of the bucket counts (partition + 1 <= 513 <= 1024 threads).
-  const int v = tid <= partition ? bucket[tid] : 0;
+  // Exclusive scan of the bucket counts (513 buckets <= 1024 threads).
+  const int v = tid < kPlanBuckets ? bucket[tid] : 0;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -87,7 +93,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   __syncthreads();
   const int excl = x - v + (warp > 0 ? warp_total[warp - 1] : 0);
   __syncthreads();
-  if (tid <= partition) bucket[tid] = excl;
+  if (tid < kPlanBuckets) bucket[tid] = excl;
   if (tid == 0) plan_count[0] = warp_total[31];
   __syncthreads();
   for (int s = tid; s < num_seqs; s += blockDim.x) {
@@ -96,7 +102,7 @@ __global__ void __launch_bounds__(kPlanThreads)
     const int np = L == 0 ? 1 : (L + partition - 1) / partition;
     for (int p = 0; p < np; ++p) {
       const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
-      const int pos = atomicAdd(&bucket[partition - ntok], 1);
+      const int pos = atomicAdd(&bucket[plan_bucket(ntok, partition)], 1);
       entries[pos] = make_int4(s, p, np, L);
     }
   }
@@ -509,12 +515,20 @@ static int launch_plan(const DecodeArgs& a, const int32_t* context_lens, int max
   return PKV_OK;
 }
 
-static int resolve_partition(int partition_tokens, int num_seqs, int num_kv_heads, int block_size,
+static bool valid_partition(int p) {
+  return p == 64 || p == 128 || p == 256 || p == 512 || p == 1024 || p == 2048;
+}
+
+// Split size for one call: the caller's choice if given (checked against the
+// path's table-slice limit), else the path's automatic choice.  -1: invalid,
+// -2: not supported by the chosen path.
+static int resolve_partition(int partition_tokens, bool tensor, int num_seqs, int num_kv_heads, int block_size,
                              int max_context_len) {
-  if (partition_tokens == 0) return auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len);
-  if (partition_tokens != 64 && partition_tokens != 128 && partition_tokens != 256 && partition_tokens != 512)
-    return -1;
-  if (partition_tokens % block_size != 0) return -1;
+  if (partition_tokens == 0)
+    return tensor ? auto_partition_tokens_tensor(num_seqs, num_kv_heads, block_size, max_context_len)
+                  : auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len);
+  if (!valid_partition(partition_tokens) || partition_tokens % block_size != 0) return -1;
+  if (!tensor && partition_tokens / block_size > 32) return -2;
   return partition_tokens;
 }
 
@@ -534,7 +548,10 @@ extern "C" size_t pkv_paged_attention_workspace_size(int num_seqs, int num_heads
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
       (block_size != 16 && block_size != 32))
     return 0;
-  const int p = resolve_partition(partition_tokens, num_seqs, num_kv_heads, block_size, max_context_len);
+  // sized for the CUDA-core split, the shortest (so the largest workspace) of the two paths
+  const int p = partition_tokens == 0 ? auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len)
+                                      : resolve_partition(partition_tokens, true, num_seqs, num_kv_heads, block_size,
+                                                          max_context_len);
   if (p < 0) return 0;
   return workspace_layout(num_seqs, num_heads, head_dim, max_context_len, p).total;
 }
@@ -566,10 +583,15 @@ extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* 
   if (path == PKV_PATH_TENSOR && !tensor_path_supports(group, head_dim))
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: tensor path needs 2 <= group <= 16 and head_dim 128"
                      " (group %d, head_dim %d)", group, head_dim);
-  const int partition = resolve_partition(partition_tokens, num_seqs, num_kv_heads, block_size, max_context_len);
-  if (partition < 0)
-    return set_error(PKV_ERR_INVALID, "paged_attention_decode: partition_tokens %d (64/128/256/512, multiple of "
-                     "block_size)", partition_tokens);
+  const bool use_tensor = path == PKV_PATH_TENSOR || (path == PKV_PATH_AUTO && tensor_path_supports(group, head_dim));
+  const int partition =
+      resolve_partition(partition_tokens, use_tensor, num_seqs, num_kv_heads, block_size, max_context_len);
+  if (partition == -1)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode: partition_tokens %d (64..2048, a power of two and a "
+                     "multiple of block_size)", partition_tokens);
+  if (partition == -2)
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: the CUDA-core path splits at most 32 blocks "
+                     "(partition_tokens %d, block_size %d)", partition_tokens, block_size);
   if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(65535) * partition)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: max_context_len too large for the split");
   if (num_seqs == 0) return PKV_OK;
@@ -599,6 +621,8 @@ extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* 
   a.part_o = reinterpret_cast<float*>(ws + w.off_part_o);
   a.part_ml = reinterpret_cast<float2*>(ws + w.off_part_ml);
   a.status = status;
+  a.context_lens = context_lens;
+  a.max_context_len = max_context_len;
   a.max_blocks = max_blocks_per_seq;
   a.num_seqs = num_seqs;
   a.num_heads = num_heads;
@@ -614,7 +638,6 @@ extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* 
   int rc = launch_plan(a, context_lens, max_context_len, s);
   if (rc != PKV_OK) return rc;
   const bool out_f32 = out_dtype == PKV_DTYPE_F32;
-  const bool use_tensor = path == PKV_PATH_TENSOR || (path == PKV_PATH_AUTO && tensor_path_supports(group, head_dim));
   if (use_tensor) return launch_decode_tensor(a, head_dim, out_f32, s);
   if (head_dim == 128) return out_f32 ? launch_simt<128, true>(a, s) : launch_simt<128, false>(a, s);
   return out_f32 ? launch_simt<64, true>(a, s) : launch_simt<64, false>(a, s);

@@ -13,7 +13,9 @@ namespace pkv {
 // Tokens that one pipeline stage carries: one 16-row slice of a (block, kv head)
 // tile (a whole block at block_size 16, half a block at 32).
 constexpr int kStageTokens = 16;
-constexpr int kMaxPartition = 512;
+constexpr int kMaxPartition = 2048;       // the tensor-core path reads up to 128 table entries per item
+constexpr int kMaxPartitionSimt = 512;    // the CUDA-core path keeps one table entry per lane (32 blocks)
+constexpr int kPlanBuckets = 513;         // counting-sort buckets of the plan (item length, coarsened)
 
 // One plan entry: a (sequence, partition) pair.  x = seq, y = partition index,
 // z = number of partitions of the sequence, w = validated context length.
@@ -31,6 +33,8 @@ struct DecodeArgs {
   float* part_o;               // [B * Hq * max_parts * D] unnormalised partial outputs
   float2* part_ml;             // [B * Hq * max_parts] (running max in log2 units, sum of weights)
   int32_t* status;
+  const int32_t* context_lens;
+  int max_context_len;
   int max_blocks;
   int num_seqs;
   int num_heads;
@@ -55,9 +59,21 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 inline int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size, int max_context_len) {
   // Largest split (fewest partials to merge) that still leaves enough work items
   // to spread over every SM of the GPU.
-  int p = kMaxPartition;
+  int p = kMaxPartitionSimt;
   while (p > 64 && static_cast<int64_t>(num_seqs) * num_kv_heads * ((max_context_len + p - 1) / p) < 4096) p /= 2;
   return p < block_size ? block_size : p;
+}
+
+// The tensor-core path pays a fixed cost per item (softmax denominators, output or
+// partial, and later a merge): it takes longer splits, up to 2048 tokens, as long
+// as about 16 items per SM remain for load balance.  Never shorter than the
+// CUDA-core split, so a workspace sized for that split always suffices.
+inline int auto_partition_tokens_tensor(int num_seqs, int num_kv_heads, int block_size, int max_context_len) {
+  const int base = auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len);
+  int p = kMaxPartition;
+  while (p > base && static_cast<int64_t>(num_seqs) * num_kv_heads * ((max_context_len + p - 1) / p) < 16 * 148)
+    p /= 2;
+  return p > base ? p : base;
 }
 
 inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int max_context_len,

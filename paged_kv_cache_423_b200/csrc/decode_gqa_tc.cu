@@ -308,19 +308,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
     auto load_entry = [&](int64_t it) -> PlanEntry {
       return it < n_items ? a.entries[it / a.num_kv_heads] : make_int4(0, 0, 0, 0);
     };
-    auto load_tab = [&](const PlanEntry& e) -> int {
+    // The item's block-table slice: lane l holds entries l, l+32, l+64, l+96 (an
+    // item spans at most 2048 tokens = 128 blocks of 16).
+    auto load_tab = [&](const PlanEntry& e) -> int4 {
       const int tok0 = e.y * a.partition;
       const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - tok0);
       const int nblk = (ntok + a.block_size - 1) / a.block_size;
-      return lane < nblk ? __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + lane)
-                         : 0;
+      const int32_t* row = a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size;
+      int4 t = make_int4(0, 0, 0, 0);
+      if (lane < nblk) t.x = __ldg(row + lane);
+      if (lane + 32 < nblk) t.y = __ldg(row + lane + 32);
+      if (lane + 64 < nblk) t.z = __ldg(row + lane + 64);
+      if (lane + 96 < nblk) t.w = __ldg(row + lane + 96);
+      return t;
     };
     // Plan entries and table slices are fetched one and two items ahead.
     int64_t item = blockIdx.x;
     PlanEntry e_cur = load_entry(item);
-    int tab_cur = item < n_items ? load_tab(e_cur) : 0;
+    int4 tab_cur = item < n_items ? load_tab(e_cur) : make_int4(0, 0, 0, 0);
     PlanEntry e_nxt = load_entry(item + G);
-    int tab_nxt = item + G < n_items ? load_tab(e_nxt) : 0;
+    int4 tab_nxt = item + G < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
     PlanEntry e_nx2 = load_entry(item + 2 * G);
     int n = 0;  // fills issued
     int item_ord = 0;
@@ -348,7 +355,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         const int n_valid = max(0, min(kTile, ntok - tile * kTile));
         const int nchunks = (n_valid + kChunk - 1) / kChunk;
         const int ltok = tile * kTile + lane * kChunk;  // this lane's chunk (lane < nchunks)
-        const int phys = __shfl_sync(0xffffffffu, tab_cur, min(31, ltok / a.block_size));
+        const int blk = min(127, ltok / a.block_size);
+        const int p0 = __shfl_sync(0xffffffffu, tab_cur.x, blk & 31);
+        const int p1 = __shfl_sync(0xffffffffu, tab_cur.y, blk & 31);
+        const int p2 = __shfl_sync(0xffffffffu, tab_cur.z, blk & 31);
+        const int p3 = __shfl_sync(0xffffffffu, tab_cur.w, blk & 31);
+        const int phys = blk < 32 ? p0 : blk < 64 ? p1 : blk < 96 ? p2 : p3;
         const bool mine = lane < nchunks;
         const bool ok = mine && phys >= 0 && phys < a.num_blocks;
         const uint32_t mask = __ballot_sync(0xffffffffu, ok);
@@ -383,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       e_cur = e_nxt;
       tab_cur = tab_nxt;
       e_nxt = e_nx2;
-      tab_nxt = item + G < n_items ? load_tab(e_nxt) : 0;
+      tab_nxt = item + G < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
       e_nx2 = load_entry(item + 2 * G);
     }
     if (!failed && !*abort_flag) {
@@ -677,56 +689,73 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Merge of split partitions: one warp per (sequence, query head) whose context was
-// split, o = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.  Runs after the main
-// kernel on the same stream; lane l owns output values 4l .. 4l+3.
+// Merge of split partitions: one CTA of 4 warps per (sequence, query head) whose
+// context was split, o = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.  Runs
+// after the main kernel on the same stream.  Warp w takes partitions w, w+4, ...;
+// lane l owns output values 4l .. 4l+3; the four warps' sums meet in shared memory.
+constexpr int kMergeWarps = 4;
+
 template <bool OUT_F32>
-__global__ void __launch_bounds__(256) merge_partials_kernel(const DecodeArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int64_t n_units = static_cast<int64_t>(a.plan_count[0]) * a.num_heads;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); u < n_units;
-       u += stride) {
-    const PlanEntry e = a.entries[u / a.num_heads];
-    if (e.y != 0 || e.z <= 1) continue;  // one warp per split sequence and head
-    const int h = static_cast<int>(u % a.num_heads);
-    const int nparts = e.z;
-    const int64_t unit = static_cast<int64_t>(e.x) * a.num_heads + h;
-    const float2* ml = a.part_ml + unit * a.max_parts;
-    const float* po = a.part_o + unit * a.max_parts * kD + lane * 4;
-    float M = -INFINITY;
-    for (int p = lane; p < nparts; p += 32) M = fmaxf(M, ml[p].x);
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_partials_kernel(const DecodeArgs a) {
+  __shared__ float s_max[kMergeWarps];
+  __shared__ float s_l[kMergeWarps];
+  __shared__ float4 s_acc[kMergeWarps][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq = blockIdx.x / a.num_heads, h = blockIdx.x % a.num_heads;
+  int L = a.context_lens[seq];
+  if (L < 0 || L > a.max_context_len || L > a.max_blocks * a.block_size) L = 0;  // as the plan does
+  const int nparts = L == 0 ? 1 : (L + a.partition - 1) / a.partition;
+  if (nparts <= 1) return;  // written directly by the main kernel
+  const int64_t unit = static_cast<int64_t>(seq) * a.num_heads + h;
+  const float2* ml = a.part_ml + unit * a.max_parts;
+  const float* po = a.part_o + unit * a.max_parts * kD + lane * 4;
+  float M = -INFINITY;
+  for (int p = warp + kMergeWarps * lane; p < nparts; p += kMergeWarps * 32) M = fmaxf(M, ml[p].x);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Ls = 0.f;
-    for (int base = 0; base < nparts; base += 32) {
-      const int p = base + lane;
-      float w = 0.f;
-      if (p < nparts) {
-        const float2 v = ml[p];
-        w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-        Ls = fmaf(w, v.y, Ls);
-      }
-      const int cnt = min(32, nparts - base);
-#pragma unroll 8
-      for (int j = 0; j < cnt; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, w, j);
-        const float4 o = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(base + j) * kD);
-        acc.x = fmaf(wj, o.x, acc.x);
-        acc.y = fmaf(wj, o.y, acc.y);
-        acc.z = fmaf(wj, o.z, acc.z);
-        acc.w = fmaf(wj, o.w, acc.w);
-      }
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (lane == 0) s_max[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float Ls = 0.f;
+  for (int base = warp; base < nparts; base += kMergeWarps * 32) {
+    const int p = base + kMergeWarps * lane;  // this lane's partition of the round
+    float w = 0.f;
+    if (p < nparts) {
+      const float2 v = ml[p];
+      w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+      Ls = fmaf(w, v.y, Ls);
     }
+    const int cnt = min(32, (nparts - base + kMergeWarps - 1) / kMergeWarps);
+#pragma unroll 8
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, w, j);
+      const float4 o = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(base + kMergeWarps * j) * kD);
+      acc.x = fmaf(wj, o.x, acc.x);
+      acc.y = fmaf(wj, o.y, acc.y);
+      acc.z = fmaf(wj, o.z, acc.z);
+      acc.w = fmaf(wj, o.w, acc.w);
+    }
+  }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
-    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+  for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+  if (lane == 0) s_l[warp] = Ls;
+  s_acc[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    const float Lt = s_l[0] + s_l[1] + s_l[2] + s_l[3];
+    const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+    float4 r = s_acc[0][lane];
+#pragma unroll
+    for (int w2 = 1; w2 < kMergeWarps; ++w2) {
+      const float4 t = s_acc[w2][lane];
+      r.x += t.x, r.y += t.y, r.z += t.z, r.w += t.w;
+    }
     const int64_t base = unit * kD + lane * 4;
-    store_out<OUT_F32>(a, base + 0, acc.x * inv);
-    store_out<OUT_F32>(a, base + 1, acc.y * inv);
-    store_out<OUT_F32>(a, base + 2, acc.z * inv);
-    store_out<OUT_F32>(a, base + 3, acc.w * inv);
+    store_out<OUT_F32>(a, base + 0, r.x * inv);
+    store_out<OUT_F32>(a, base + 1, r.y * inv);
+    store_out<OUT_F32>(a, base + 2, r.z * inv);
+    store_out<OUT_F32>(a, base + 3, r.w * inv);
   }
 }
 
@@ -777,7 +806,7 @@ static int launch(const Args& args, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) launch: %s", cudaGetErrorString(e));
   if (args.a.max_parts > 1) {
-    merge_partials_kernel<OUT_F32><<<std::max(1, sms) * 4, 256, 0, stream>>>(args.a);
+    merge_partials_kernel<OUT_F32><<<args.a.num_seqs * args.a.num_heads, kMergeWarps * 32, 0, stream>>>(args.a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) merge launch: %s", cudaGetErrorString(e));
   }

@@ -51,13 +51,19 @@ def test_decode_matches_oracle(pkv, case, path):
     compare(out.cpu().numpy(), oracle_out(b))
 
 
-@pytest.mark.parametrize("partition", [64, 128, 256, 512])
+@pytest.mark.parametrize("partition", [64, 128, 256, 512, 1024, 2048])
 @pytest.mark.parametrize("path", sorted(PATHS))
 def test_split_sizes_agree(pkv, partition, path):
-    """Split-context partitions of every size give the oracle's result."""
+    """Split-context partitions of every size give the oracle's result (the CUDA-core
+    path reads at most 32 table entries per item and refuses longer splits)."""
     heads = (4, 4) if path == "simt" else (16, 4)
-    b = wl.make_decode_batch("llama7b", num_seqs=6, num_heads=heads[0], num_kv_heads=heads[1],
-                             lengths=[1, 63, 64, 65, 129, 1500])
+    b = wl.make_decode_batch("llama7b", num_seqs=7, num_heads=heads[0], num_kv_heads=heads[1],
+                             lengths=[1, 63, 64, 65, 129, 1500, 4500])
+    if path == "simt" and partition // b.block_size > 32:
+        with pytest.raises(pkv.PkvError) as e:
+            DeviceBatch(b).decode(pkv, partition=partition, path=PATHS[path])
+        assert e.value.code == pkv.PKV_ERR_UNSUPPORTED
+        return
     ref = oracle_out(b)
     out = DeviceBatch(b).decode(pkv, partition=partition, path=PATHS[path])
     compare(out.cpu().numpy(), ref)

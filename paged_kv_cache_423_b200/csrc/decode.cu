@@ -58,16 +58,23 @@ __global__ void __launch_bounds__(kPlanThreads)
   for (int i = tid; i < kPlanBuckets; i += blockDim.x) bucket[i] = 0;
   for (int i = tid; i < n_arrive; i += blockDim.x) arrive[i] = 0;
   __syncthreads();
-  for (int s = tid; s < num_seqs; s += blockDim.x) {
+  // One warp per sequence, lanes over its partitions; lanes that hit the same
+  // bucket add to it once (warp-aggregated shared-memory atomics).
+  const int nwarps = blockDim.x >> 5;
+  for (int s = warp; s < num_seqs; s += nwarps) {
     int L = context_lens[s];
     if (L < 0 || L > max_context_len || L > max_table_tokens) {
-      set_status(status, PKV_DEV_BAD_CONTEXT);
+      if (lane == 0) set_status(status, PKV_DEV_BAD_CONTEXT);
       L = 0;
     }
     const int np = L == 0 ? 1 : (L + partition - 1) / partition;
-    for (int p = 0; p < np; ++p) {
+    for (int p0 = 0; p0 < np; p0 += 32) {
+      const int p = p0 + lane;
+      const bool live = p < np;
       const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
-      atomicAdd(&bucket[plan_bucket(ntok, partition)], 1);
+      const int b = live ? plan_bucket(ntok, partition) : -1;
+      const unsigned same = __match_any_sync(kFull, b);
+      if (live && (__ffs(same) - 1) == lane) atomicAdd(&bucket[b], __popc(same));
     }
   }
   __syncthreads();
@@ -94,16 +101,26 @@ __global__ void __launch_bounds__(kPlanThreads)
   const int excl = x - v + (warp > 0 ? warp_total[warp - 1] : 0);
   __syncthreads();
   if (tid < kPlanBuckets) bucket[tid] = excl;
-  if (tid == 0) plan_count[0] = warp_total[31];
+  if (tid == 0) {
+    plan_count[0] = warp_total[31];
+    plan_count[1] = 0;  // work-item counter of the tensor-core kernel
+  }
   __syncthreads();
-  for (int s = tid; s < num_seqs; s += blockDim.x) {
+  for (int s = warp; s < num_seqs; s += nwarps) {
     int L = context_lens[s];
     if (L < 0 || L > max_context_len || L > max_table_tokens) L = 0;
     const int np = L == 0 ? 1 : (L + partition - 1) / partition;
-    for (int p = 0; p < np; ++p) {
+    for (int p0 = 0; p0 < np; p0 += 32) {
+      const int p = p0 + lane;
+      const bool live = p < np;
       const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
-      const int pos = atomicAdd(&bucket[plan_bucket(ntok, partition)], 1);
-      entries[pos] = make_int4(s, p, np, L);
+      const int b = live ? plan_bucket(ntok, partition) : -1;
+      const unsigned same = __match_any_sync(kFull, b);
+      const int leader = __ffs(same) - 1;
+      int base = 0;
+      if (live && leader == lane) base = atomicAdd(&bucket[b], __popc(same));
+      base = __shfl_sync(kFull, base, leader);
+      if (live) entries[base + __popc(same & ((1u << lane) - 1))] = make_int4(s, p, np, L);
     }
   }
 }

@@ -27,7 +27,7 @@ struct DecodeArgs {
   const __nv_bfloat16* key_cache;
   const __nv_bfloat16* value_cache;
   const int32_t* block_tables;
-  const int32_t* plan_count;   // number of plan entries (written by the plan kernel)
+  const int32_t* plan_count;   // [0] number of plan entries, [1] work-item counter (both set by the plan kernel)
   const PlanEntry* entries;    // sorted plan
   int32_t* arrive;             // [B * Hq] partition arrival counters (zeroed by the plan kernel)
   float* part_o;               // [B * Hq * max_parts * D] unnormalised partial outputs

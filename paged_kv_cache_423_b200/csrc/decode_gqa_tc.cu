@@ -304,7 +304,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   if (warp == kProducerWarp) {
     // ================= producer =================
     const uint64_t policy = l2_policy_evict_first();
-    const int64_t G = gridDim.x;
     auto load_entry = [&](int64_t it) -> PlanEntry {
       return it < n_items ? a.entries[it / a.num_kv_heads] : make_int4(0, 0, 0, 0);
     };
@@ -322,13 +321,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       if (lane + 96 < nblk) t.w = __ldg(row + lane + 96);
       return t;
     };
-    // Plan entries and table slices are fetched one and two items ahead.
-    int64_t item = blockIdx.x;
+    // Items are taken from a global counter in plan order (longest first), so CTAs
+    // that finish early take more.  Item ids, plan entries and table slices are
+    // fetched up to two items ahead.
+    int* work_counter = const_cast<int*>(a.plan_count) + 1;
+    auto grab = [&]() -> int64_t {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(work_counter, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    int64_t item = grab();
+    int64_t item_nxt = grab();
+    int64_t item_nx2 = grab();
     PlanEntry e_cur = load_entry(item);
     int4 tab_cur = item < n_items ? load_tab(e_cur) : make_int4(0, 0, 0, 0);
-    PlanEntry e_nxt = load_entry(item + G);
-    int4 tab_nxt = item + G < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
-    PlanEntry e_nx2 = load_entry(item + 2 * G);
+    PlanEntry e_nxt = load_entry(item_nxt);
+    int4 tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
+    PlanEntry e_nx2 = load_entry(item_nx2);
     int n = 0;  // fills issued
     int item_ord = 0;
     bool failed = false;
@@ -390,13 +399,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           tma_load_2d(qd + N * 128, &args.tm_q, 64, qrow, &full[slot], policy);
         }
       }
-      item += G;
+      item = item_nxt;
+      item_nxt = item_nx2;
+      item_nx2 = grab();
       ++item_ord;
       e_cur = e_nxt;
       tab_cur = tab_nxt;
       e_nxt = e_nx2;
-      tab_nxt = item + G < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
-      e_nx2 = load_entry(item + 2 * G);
+      tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
+      e_nx2 = load_entry(item_nx2);
     }
     if (!failed && !*abort_flag) {
       // end-of-stream marker: a fill with no data

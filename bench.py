@@ -56,6 +56,32 @@ def measured_hbm_gbs():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def source_digest() -> str:
+    """Digest of the library sources; a recorded ncu traffic figure is only reported
+    while the kernels are the ones it was measured on."""
+    import hashlib
+    h = hashlib.sha256()
+    for sub in (os.path.join("paged_kv_cache_423_b200", "csrc"), "include"):
+        d = os.path.join(ROOT, sub)
+        for f in sorted(os.listdir(d)):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes (read + write) per decode launch from profiles/traffic.json, or None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f).get(workload)
+    except Exception:
+        return None
+    if not entry or entry.get("sources") != source_digest():
+        return None
+    return int(entry["dram_bytes_per_launch"])
+
+
 def rank_info():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
@@ -285,6 +311,8 @@ def run_ours(args, rank, world, local_rank):
     e2e = run_e2e(args, w, pkv, device, path, ws, out, status, max_len_all) if not args.no_e2e else None
 
     peak, peak_kind = measured_hbm_gbs()
+    g = w.Hq // w.Hkv
+    uses_tensor = path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16)
     dec_gbs = bytes_total / (dec_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -298,8 +326,10 @@ def run_ours(args, rank, world, local_rank):
         "seq_steps_per_s": round(seq_steps, 1),
         "pct_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(dec_gbs / peak, 4), "traffic": None, "peak_kind": peak_kind,
-                     "kernel": "paged_attention_decode (plan + streaming kernel)",
+                     "frac": round(dec_gbs / peak, 4), "traffic": recorded_traffic(w.name),
+                     "algorithmic_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
+                     "kernel": ("paged_attention_decode: plan + tcgen05 kernel + split merge" if uses_tensor
+                                else "paged_attention_decode: plan + CUDA-core streaming kernel"),
                      "ms_per_launch": round(dec_ms / args.steps, 4)},
         "gpu_launches": launches,
         "clocks": clocks.summary(),

@@ -58,24 +58,18 @@ __global__ void __launch_bounds__(kPlanThreads)
   for (int i = tid; i < kPlanBuckets; i += blockDim.x) bucket[i] = 0;
   for (int i = tid; i < n_arrive; i += blockDim.x) arrive[i] = 0;
   __syncthreads();
-  // One warp per sequence, lanes over its partitions; lanes that hit the same
-  // bucket add to it once (warp-aggregated shared-memory atomics).
-  const int nwarps = blockDim.x >> 5;
-  for (int s = warp; s < num_seqs; s += nwarps) {
+  // One thread per sequence.  Its full-length partitions all fall in bucket 0 and
+  // only the last may be shorter, so a sequence costs at most two atomics.
+  for (int s = tid; s < num_seqs; s += blockDim.x) {
     int L = context_lens[s];
     if (L < 0 || L > max_context_len || L > max_table_tokens) {
-      if (lane == 0) set_status(status, PKV_DEV_BAD_CONTEXT);
+      set_status(status, PKV_DEV_BAD_CONTEXT);
       L = 0;
     }
-    const int np = L == 0 ? 1 : (L + partition - 1) / partition;
-    for (int p0 = 0; p0 < np; p0 += 32) {
-      const int p = p0 + lane;
-      const bool live = p < np;
-      const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
-      const int b = live ? plan_bucket(ntok, partition) : -1;
-      const unsigned same = __match_any_sync(kFull, b);
-      if (live && (__ffs(same) - 1) == lane) atomicAdd(&bucket[b], __popc(same));
-    }
+    const int full = L / partition;
+    const int tail = L - full * partition;
+    if (full > 0) atomicAdd(&bucket[0], full);
+    if (tail > 0 || L == 0) atomicAdd(&bucket[plan_bucket(tail, partition)], 1);
   }
   __syncthreads();
   // Exclusive scan of the bucket counts (513 buckets <= 1024 threads).
@@ -106,21 +100,19 @@ __global__ void __launch_bounds__(kPlanThreads)
     plan_count[1] = 0;  // work-item counter of the tensor-core kernel
   }
   __syncthreads();
-  for (int s = warp; s < num_seqs; s += nwarps) {
+  for (int s = tid; s < num_seqs; s += blockDim.x) {
     int L = context_lens[s];
     if (L < 0 || L > max_context_len || L > max_table_tokens) L = 0;
-    const int np = L == 0 ? 1 : (L + partition - 1) / partition;
-    for (int p0 = 0; p0 < np; p0 += 32) {
-      const int p = p0 + lane;
-      const bool live = p < np;
-      const int ntok = L == 0 ? 0 : min(partition, L - p * partition);
-      const int b = live ? plan_bucket(ntok, partition) : -1;
-      const unsigned same = __match_any_sync(kFull, b);
-      const int leader = __ffs(same) - 1;
-      int base = 0;
-      if (live && leader == lane) base = atomicAdd(&bucket[b], __popc(same));
-      base = __shfl_sync(kFull, base, leader);
-      if (live) entries[base + __popc(same & ((1u << lane) - 1))] = make_int4(s, p, np, L);
+    const int full = L / partition;
+    const int tail = L - full * partition;
+    const int np = L == 0 ? 1 : full + (tail > 0);
+    if (full > 0) {
+      const int pos = atomicAdd(&bucket[0], full);
+      for (int p = 0; p < full; ++p) entries[pos + p] = make_int4(s, p, np, L);
+    }
+    if (tail > 0 || L == 0) {
+      const int pos = atomicAdd(&bucket[plan_bucket(tail, partition)], 1);
+      entries[pos] = make_int4(s, full, np, L);
     }
   }
 }

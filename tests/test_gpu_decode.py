@@ -156,6 +156,23 @@ def test_repeated_calls_reuse_workspace(pkv, path):
     compare(outs[0].cpu().numpy(), oracle_out(b))
 
 
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_longest_context(pkv, path):
+    """One 131072-token context (4096 blocks of 32): 256 partitions of 512 tokens on the
+    CUDA-core path, 64 of 2048 on the tensor path, merged into one row per head."""
+    L = 131072
+    heads = (4, 4) if path == "simt" else (32, 4)
+    b = wl.make_decode_batch("long_trace", num_seqs=1, num_heads=heads[0], num_kv_heads=heads[1], lengths=[L],
+                             pool_factor=1.0, with_data=False)
+    rng = wl.rng_for(310)
+    b.query = wl.bf16_normal(rng, (1, b.num_heads, 128))
+    shape = (b.num_blocks, b.num_kv_heads, b.block_size, 128)
+    kc, vc = device_pool(shape, 3), device_pool(shape, 4)
+    part = 512 if path == "simt" else 2048
+    out = DeviceBatch(b, kc, vc).decode(pkv, partition=part, path=PATHS[path]).cpu().numpy()
+    compare(out, sampled_oracle(b, kc, vc, [0]))
+
+
 # ---------------------------------------------------------------------------
 # Full-size workloads: sampled sequences checked one by one against the oracle
 # ---------------------------------------------------------------------------

@@ -417,6 +417,110 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
 
 
 # ---------------------------------------------------------------------------
+# Continuous-batching trace (the fifth workload, run step by step)
+# ---------------------------------------------------------------------------
+
+def run_trace(args, rank, world, local_rank):
+    """Long-context trace: every step appends one token per running sequence
+    (reshape_and_cache), decodes, frees finished sequences and admits seeded arrivals
+    while the pool allows (their prompt K/V is written by one reshape_and_cache call,
+    a synthetic prefill, outside the timed decode work).  Device time of the decode
+    work (copy_blocks if any, reshape_and_cache, paged_attention_decode) is summed
+    over the timed steps with CUDA events."""
+    import torch
+    import paged_kv_cache_423_b200 as pkv
+
+    device = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(device)
+    p = wl.TraceParams(steps=args.warmup + args.steps)
+    initial, arrivals = wl.trace_events(p, seed=2000 + rank)
+    rng = wl.rng_for(2001 + rank)
+    order = rng.permutation(p.num_blocks).astype(np.int32)
+    bm = pkv.BlockManager(p.num_blocks, p.block_size, order)
+    g = torch.Generator(device=device)
+    g.manual_seed(2002 + rank)
+    shape = (p.num_blocks, p.num_kv_heads, p.block_size, p.head_dim)
+    kc = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    max_blocks = (p.len_hi + p.steps + p.block_size) // p.block_size + 1
+    max_len = max_blocks * p.block_size
+    ws = torch.empty(pkv.paged_attention_workspace_size(p.max_batch, p.num_heads, p.num_kv_heads, p.head_dim,
+                                                        p.block_size, max_len), dtype=torch.uint8, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    scale = wl.fp32_scale(p.head_dim)
+    running = {}
+    next_id = 0
+
+    def admit(length, budget):
+        nonlocal next_id
+        if -(-length // p.block_size) > bm.num_free():
+            return
+        sid = next_id
+        next_id += 1
+        bm.add_seq(sid, length - 1)
+        slots = torch.from_numpy(bm.slots(sid, 0, length - 1)).to(device)
+        k = torch.randn((length - 1, p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
+        pkv.reshape_and_cache(k, k, kc, vc, slots, status=status)
+        running[sid] = budget
+
+    for length, budget in initial:
+        admit(length, budget)
+    t_ms = 0.0
+    seq_steps = 0
+    kv_bytes = 0
+    launches = 0
+    with ClockSampler(device) as clocks:
+        for step in range(p.steps):
+            ids = sorted(running)
+            if ids:
+                slots, pairs = bm.append_slots(ids)
+                tables, lens = bm.export_tables(ids, max_blocks)
+                d_slots = torch.from_numpy(slots).to(device)
+                d_tables = torch.from_numpy(tables).to(device)
+                d_lens = torch.from_numpy(lens).to(device)
+                q = torch.randn((len(ids), p.num_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
+                k = torch.randn((len(ids), p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
+                out = torch.empty((len(ids), p.num_heads, p.head_dim), dtype=torch.bfloat16, device=device)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                if len(pairs):
+                    pkv.copy_blocks([kc], [vc], torch.from_numpy(pairs).to(device), status=status)
+                pkv.reshape_and_cache(k, k, kc, vc, d_slots, status=status)
+                pkv.paged_attention_decode(out, q, kc, vc, d_tables, d_lens, max_len, scale, ws, status=status)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if step >= args.warmup:
+                    t_ms += e0.elapsed_time(e1)
+                    seq_steps += len(ids)
+                    kv_bytes += int(lens.astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 4
+                    launches += 3 + (1 if len(pairs) else 0) + 1  # + the split merge
+                for sid in ids:
+                    running[sid] -= 1
+                    if running[sid] == 0:
+                        bm.free_seq(sid)
+                        del running[sid]
+            for length, budget in arrivals[step]:
+                if len(running) < p.max_batch:
+                    admit(length, budget)
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item():#x}")
+    bm.close()
+    peak, peak_kind = measured_hbm_gbs()
+    value = kv_bytes / (t_ms * 1e-3) / 1e9
+    return {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t_ms / max(1, args.steps), 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "long_trace_continuous", "max_batch": p.max_batch, "num_heads": p.num_heads,
+                       "num_kv_heads": p.num_kv_heads, "head_dim": p.head_dim, "block_size": p.block_size,
+                       "num_blocks": p.num_blocks, "admitted": next_id,
+                       "timed": "copy_blocks + reshape_and_cache + paged_attention_decode per step"},
+            "seq_steps_per_s": round(seq_steps / (t_ms * 1e-3), 1), "pct_hbm_peak": round(100 * value / peak, 2),
+            "gpu_launches": launches, "clocks": clocks.summary()}
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle timing (baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
@@ -515,6 +619,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama13b_mixed_bs16", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--trace", action="store_true",
+                    help="run the long-context continuous-batching trace step by step (the fifth workload)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
@@ -525,6 +631,8 @@ def main():
     rank, world, local_rank = rank_info()
     if args.impl == "reference":
         res = run_reference(args, rank, world, local_rank)
+    elif args.trace:
+        res = run_trace(args, rank, world, local_rank)
     else:
         res = run_ours(args, rank, world, local_rank)
     if rank == 0 and res is not None:

@@ -32,6 +32,18 @@
 #include "decode_common.cuh"
 #include "pkv_internal.h"
 
+// Warps per CTA, ring stages per warp, and dynamic (counter) instead of static
+// work distribution of the CUDA-core kernel; compile-time overridable for sweeps.
+#ifndef PKV_SIMT_WARPS
+#define PKV_SIMT_WARPS 4
+#endif
+#ifndef PKV_SIMT_STAGES
+#define PKV_SIMT_STAGES 2
+#endif
+#ifndef PKV_SIMT_DYNAMIC
+#define PKV_SIMT_DYNAMIC 1
+#endif
+
 namespace pkv {
 
 constexpr unsigned kFull = 0xffffffffu;
@@ -243,8 +255,19 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   const int qk_row = LaneMap<D>::row(lane), qk_half = LaneMap<D>::half(lane);
 
   const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_heads;
+  // Work distribution over the plan (longest items first): every warp starts with
+  // items w and w + #warps; after that it takes the next unclaimed item from a
+  // global counter, so warps that finish early do more of the tail.
   const int64_t stride = static_cast<int64_t>(gridDim.x) * WARPS;
   const int64_t first_item = static_cast<int64_t>(blockIdx.x) * WARPS + warp;
+#if PKV_SIMT_DYNAMIC
+  int* work_counter = const_cast<int*>(a.plan_count) + 1;
+  auto take = [&]() -> int64_t {
+    int v = 0;
+    if (lane == 0) v = atomicAdd(work_counter, 1);
+    return 2 * stride + __shfl_sync(kFull, v, 0);
+  };
+#endif
   if (first_item >= n_items) return;
 
   if (lane == 0) {
@@ -253,7 +276,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
     fence_barrier_init();
   }
   __syncwarp();
-  const uint64_t policy = l2_policy_evict_first();
+  const uint64_t policy = l2_policy_kv();
 
   // ---- issuing side: current item, next item (table prefetched), item after (entry prefetched)
   auto entry_of = [&](int64_t id) -> PlanEntry {
@@ -267,9 +290,17 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   cur.table = load_item_table(a, cur.e, lane);
   nxt.id = first_item + stride < n_items ? first_item + stride : -1;
   nxt.e = entry_of(first_item + stride);
-  nxt.table = nxt.id >= 0 ? load_item_table(a, nxt.e, lane) : 0;
+#if PKV_SIMT_DYNAMIC
+  {
+    const int64_t i2 = nxt.id >= 0 ? take() : n_items;
+    nx2_id = i2 < n_items ? i2 : -1;
+    nx2_e = entry_of(i2);
+  }
+#else
   nx2_id = first_item + 2 * stride < n_items ? first_item + 2 * stride : -1;
   nx2_e = entry_of(first_item + 2 * stride);
+#endif
+  nxt.table = nxt.id >= 0 ? load_item_table(a, nxt.e, lane) : 0;
   int cur_stage = 0;
   int cur_nstages = item_stages(cur.e, a.partition);
   bool issue_done = false;
@@ -286,7 +317,14 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       nxt.id = nx2_id;
       nxt.e = nx2_e;
       nxt.table = nxt.id >= 0 ? load_item_table(a, nxt.e, lane) : 0;
+#if PKV_SIMT_DYNAMIC
+      if (nx2_id >= 0) {
+        const int64_t i2 = take();
+        nx2_id = i2 < n_items ? i2 : -1;
+      }
+#else
       nx2_id = nx2_id >= 0 && nx2_id + stride < n_items ? nx2_id + stride : -1;
+#endif
       nx2_e = entry_of(nx2_id >= 0 ? nx2_id : n_items);
       cur_stage = 0;
       cur_nstages = item_stages(cur.e, a.partition);
@@ -479,13 +517,6 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
 // Host side
 // ---------------------------------------------------------------------------
 
-// Warps per CTA and ring stages per warp (compile-time overridable for tuning sweeps).
-#ifndef PKV_SIMT_WARPS
-#define PKV_SIMT_WARPS 4
-#endif
-#ifndef PKV_SIMT_STAGES
-#define PKV_SIMT_STAGES 2
-#endif
 constexpr int kSimtWarps = PKV_SIMT_WARPS;
 constexpr int kSimtStages = PKV_SIMT_STAGES;
 

@@ -42,7 +42,6 @@ namespace tc {
 
 constexpr int kTile = 128;             // tokens per tile (MMA M)
 constexpr int kChunk = 16;             // rows per TMA box
-constexpr int kChunks = kTile / kChunk;
 constexpr int kD = 128;                // head_dim of this path
 constexpr int kHalfBytes = kTile * 128;  // one 64-column half of a K or V tile: 16 KiB
 constexpr int kTileBytes = 2 * kHalfBytes;
@@ -303,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
 
   if (warp == kProducerWarp) {
     // ================= producer =================
-    const uint64_t policy = l2_policy_evict_first();
+    const uint64_t policy = l2_policy_kv();
     auto load_entry = [&](int64_t it) -> PlanEntry {
       return it < n_items ? a.entries[it / a.num_kv_heads] : make_int4(0, 0, 0, 0);
     };

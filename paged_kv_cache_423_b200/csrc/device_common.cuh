@@ -103,6 +103,26 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// L2 policy of the K/V tile loads.  Evict-first keeps streamed tiles from
+// displacing other data; evict-normal lets blocks that several tables share (a
+// common prompt) stay in L2 for the other sequences that read them.
+#ifndef PKV_KV_EVICT_FIRST
+#define PKV_KV_EVICT_FIRST 1
+#endif
+__device__ __forceinline__ uint64_t l2_policy_kv() {
+#if PKV_KV_EVICT_FIRST
+  return l2_policy_evict_first();
+#else
+  return l2_policy_evict_normal();
+#endif
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));

@@ -8,11 +8,16 @@ import or call anything here; the product path never does.
 
 Modules
   paged_attention  decode attention through block tables (gather + textbook softmax)
-  cache_ops        reshape_and_cache (slot scatter) and copy_blocks (copy-on-write copy)
-  block_manager    reference model of the block allocator and per-sequence tables
+  prefill          prefill / chunked-prefill attention (causal, multi-token queries)
+  fp8              e4m3 codec, the quantising cache write, decode over an 8-bit pool
+  cache_ops        reshape_and_cache (slot scatter), copy_blocks (copy-on-write copy),
+                   swap_blocks (device <-> host pool copy)
+  block_manager    reference model of the block allocator and per-sequence tables,
+                   with swap space and automatic prefix caching
 
-Every function is pinned by ``tests/test_oracle_pins.py`` and
+Every function is pinned by ``tests/test_oracle_pins.py``,
+``tests/test_oracle_prefill_pins.py``, ``tests/test_oracle_fp8_pins.py`` and
 ``tests/test_oracle_block_manager.py`` to closed forms, library routines,
 invariants the pages state, and the pages' own block-table example.
 """
-from . import block_manager, cache_ops, paged_attention  # noqa: F401
+from . import block_manager, cache_ops, fp8, paged_attention, prefill  # noqa: F401

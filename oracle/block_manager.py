@@ -26,8 +26,36 @@ Rules the pages leave open (readings):
   * add_seq with shared prefix blocks: they must be full blocks; the remaining
     blocks are taken fresh (all-or-nothing).
 
+Swap space (intelliparadigm article, §4.2 OOM错误: swap_space extends the pool into
+host memory).  Readings:
+  * A second pool of host blocks with its own FIFO free list (initial order 0..H-1)
+    and reference counts.
+  * swap_out(seqs) moves the listed sequences' tables to host blocks: every distinct
+    device block among them (in order of first appearance, sequence by sequence)
+    gets one host block, the pair (device, host) is returned for the copy, the
+    table entry becomes the host block and the device block loses one reference.
+    swap_in(seqs) is the mirror image.  Both are all-or-nothing.  A swapped-out
+    sequence can only be swapped in or freed.
+
+Automatic prefix caching (Outcome School explainer, "内存共享": requests with an
+identical prefix, e.g. one long system prompt, keep a single copy of its blocks;
+vLLM 初探 §1.4: shared system prompts save 30-50% of the memory).  Readings:
+  * A full block is identified by the chain hash h_i = FNV-1a-64 of the 8
+    little-endian bytes of h_(i-1) (h_(-1) = 0) followed by the block's token ids
+    as 4-byte little-endian integers.  FNV-1a-64: start from 0xcbf29ce484222325;
+    per byte, xor it in, then multiply by 0x100000001b3 modulo 2^64.
+  * add_seq_tokens(seq, tokens) takes the longest run of leading blocks whose hashes
+    are registered, but never the block holding the last token (that token is
+    always computed again), so at most (n - 1) // bs blocks.  Blocks taken from
+    the cache gain a reference; a cached block with no references is taken back
+    out of the free list.  The other blocks are fresh; each fresh FULL block
+    registers its hash unless the hash is already registered.
+  * A registered block whose references drop to zero stays registered while it
+    waits in the free list; when the free list hands it out again its
+    registration is dropped (eviction in free-list order).
+
 Parity status: pinned (invariants, the pages' block-table example, hand-worked
-copy-on-write cases).
+copy-on-write, swap and prefix-cache cases, FNV-1a test vectors).
 """
 from __future__ import annotations
 
@@ -44,9 +72,25 @@ class BlockManagerError(Exception):
         self.code = code
 
 
+FNV_OFFSET = 0xCBF29CE484222325
+FNV_PRIME = 0x100000001B3
+
+
+def fnv1a64(data: bytes, h: int = FNV_OFFSET) -> int:
+    for byte in data:
+        h ^= byte
+        h = (h * FNV_PRIME) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def block_hash(parent: int, tokens) -> int:
+    data = int(parent).to_bytes(8, "little") + b"".join(int(t).to_bytes(4, "little", signed=True) for t in tokens)
+    return fnv1a64(data)
+
+
 class BlockManagerModel:
-    def __init__(self, num_blocks: int, block_size: int, initial_order=None):
-        if num_blocks <= 0 or block_size <= 0:
+    def __init__(self, num_blocks: int, block_size: int, initial_order=None, num_host_blocks: int = 0):
+        if num_blocks <= 0 or block_size <= 0 or num_host_blocks < 0:
             raise BlockManagerError(ERR_INVALID, "bad sizes")
         order = list(range(num_blocks)) if initial_order is None else [int(b) for b in initial_order]
         if sorted(order) != list(range(num_blocks)):
@@ -57,6 +101,11 @@ class BlockManagerModel:
         self.ref = [0] * num_blocks
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        self.host_free = deque(range(num_host_blocks))
+        self.host_ref = [0] * num_host_blocks
+        self.swapped: set[int] = set()
+        self.cached: dict[int, int] = {}        # hash -> device block
+        self.block_hash: dict[int, int] = {}    # device block -> its registered hash
 
     # -- blocks -------------------------------------------------------------
     def num_free(self) -> int:
@@ -67,6 +116,9 @@ class BlockManagerModel:
             raise BlockManagerError(ERR_OOM, "pool exhausted")
         b = self.free.popleft()
         self.ref[b] = 1
+        h = self.block_hash.pop(b, None)        # handing a cached block out evicts it
+        if h is not None:
+            del self.cached[h]
         return b
 
     def _check_block(self, b: int):
@@ -115,7 +167,7 @@ class BlockManagerModel:
         self.lens[seq_id] = num_tokens
 
     def fork(self, parent: int, child: int):
-        if parent not in self.tables or child in self.tables:
+        if parent not in self.tables or child in self.tables or parent in self.swapped:
             raise BlockManagerError(ERR_INVALID, "bad fork")
         table = list(self.tables[parent])
         for b in table:
@@ -126,8 +178,9 @@ class BlockManagerModel:
     def append_slots(self, seq_ids):
         """One new token per listed sequence; returns (slots, cow_pairs)."""
         seq_ids = [int(s) for s in seq_ids]
-        if len(set(seq_ids)) != len(seq_ids) or any(s not in self.tables for s in seq_ids):
-            raise BlockManagerError(ERR_INVALID, "unknown or repeated sequence")
+        if (len(set(seq_ids)) != len(seq_ids) or any(s not in self.tables for s in seq_ids)
+                or any(s in self.swapped for s in seq_ids)):
+            raise BlockManagerError(ERR_INVALID, "unknown, repeated or swapped-out sequence")
         # Dry run: count fresh blocks, following the reference counts as they change.
         need = 0
         pending = {}
@@ -160,7 +213,8 @@ class BlockManagerModel:
 
     def slots(self, seq_id: int, start: int, count: int):
         """Slots of positions start .. start+count-1 of an existing sequence."""
-        if seq_id not in self.tables or start < 0 or count < 0 or start + count > self.lens[seq_id]:
+        if (seq_id not in self.tables or seq_id in self.swapped or start < 0 or count < 0
+                or start + count > self.lens[seq_id]):
             raise BlockManagerError(ERR_INVALID, "bad range")
         table = self.tables[seq_id]
         return [table[p // self.block_size] * self.block_size + p % self.block_size
@@ -169,15 +223,21 @@ class BlockManagerModel:
     def free_seq(self, seq_id: int):
         if seq_id not in self.tables:
             raise BlockManagerError(ERR_INVALID, "unknown sequence")
-        for b in self.tables.pop(seq_id):
-            self.decref(b)
+        table = self.tables.pop(seq_id)
+        if seq_id in self.swapped:
+            self.swapped.discard(seq_id)
+            for b in table:
+                self._host_decref(b)
+        else:
+            for b in table:
+                self.decref(b)
         del self.lens[seq_id]
 
     def export_tables(self, seq_ids, max_blocks: int):
         tables = []
         lens = []
         for s in seq_ids:
-            if s not in self.tables or len(self.tables[s]) > max_blocks:
+            if s not in self.tables or s in self.swapped or len(self.tables[s]) > max_blocks:
                 raise BlockManagerError(ERR_INVALID, "unknown sequence or table too long")
             row = list(self.tables[s]) + [0] * (max_blocks - len(self.tables[s]))
             tables.append(row)
@@ -186,3 +246,122 @@ class BlockManagerModel:
 
     def seq_len(self, seq_id: int) -> int:
         return self.lens[seq_id]
+
+    # -- swap space -----------------------------------------------------------
+    def num_host_free(self) -> int:
+        return len(self.host_free)
+
+    def host_refcount(self, b: int) -> int:
+        return self.host_ref[b]
+
+    def is_swapped(self, seq_id: int) -> bool:
+        return seq_id in self.swapped
+
+    def _host_decref(self, b: int):
+        self.host_ref[b] -= 1
+        if self.host_ref[b] == 0:
+            self.host_free.append(b)
+
+    def _check_swap_ids(self, seq_ids, want_swapped: bool):
+        if len(set(seq_ids)) != len(seq_ids):
+            raise BlockManagerError(ERR_INVALID, "repeated sequence")
+        for s in seq_ids:
+            if s not in self.tables or (s in self.swapped) != want_swapped:
+                raise BlockManagerError(ERR_INVALID, "sequence in the wrong place")
+
+    def _distinct_blocks(self, seq_ids):
+        seen = []
+        marked = set()
+        for s in seq_ids:
+            for b in self.tables[s]:
+                if b not in marked:
+                    marked.add(b)
+                    seen.append(b)
+        return seen
+
+    def swap_out(self, seq_ids):
+        """Move the listed resident sequences to host blocks; returns (device, host) pairs."""
+        seq_ids = [int(s) for s in seq_ids]
+        self._check_swap_ids(seq_ids, want_swapped=False)
+        if len(self._distinct_blocks(seq_ids)) > len(self.host_free):
+            raise BlockManagerError(ERR_OOM, "host pool exhausted")
+        mapping, pairs = {}, []
+        for s in seq_ids:
+            table = self.tables[s]
+            for j, b in enumerate(table):
+                if b in mapping:
+                    self.host_ref[mapping[b]] += 1
+                else:
+                    hb = self.host_free.popleft()
+                    self.host_ref[hb] = 1
+                    mapping[b] = hb
+                    pairs.append((b, hb))
+                table[j] = mapping[b]
+                self.decref(b)
+            self.swapped.add(s)
+        return pairs
+
+    def swap_in(self, seq_ids):
+        """Bring the listed swapped-out sequences back; returns (host, device) pairs."""
+        seq_ids = [int(s) for s in seq_ids]
+        self._check_swap_ids(seq_ids, want_swapped=True)
+        if len(self._distinct_blocks(seq_ids)) > len(self.free):
+            raise BlockManagerError(ERR_OOM, "pool exhausted")
+        mapping, pairs = {}, []
+        for s in seq_ids:
+            table = self.tables[s]
+            for j, hb in enumerate(table):
+                if hb in mapping:
+                    self.ref[mapping[hb]] += 1
+                else:
+                    mapping[hb] = self.alloc()
+                    pairs.append((hb, mapping[hb]))
+                table[j] = mapping[hb]
+                self._host_decref(hb)
+            self.swapped.discard(s)
+        return pairs
+
+    # -- automatic prefix caching ---------------------------------------------
+    def num_cached_blocks(self) -> int:
+        return len(self.cached)
+
+    def add_seq_tokens(self, seq_id: int, tokens) -> int:
+        """New sequence from its prompt token ids; returns the number of leading
+        tokens whose K/V came from cached blocks."""
+        tokens = [int(t) for t in tokens]
+        n = len(tokens)
+        bs = self.block_size
+        if seq_id in self.tables:
+            raise BlockManagerError(ERR_INVALID, "bad sequence")
+        hashes = []
+        parent = 0
+        for i in range(n // bs):
+            parent = block_hash(parent, tokens[i * bs:(i + 1) * bs])
+            hashes.append(parent)
+        cap = (n - 1) // bs if n > 0 else 0
+        hits = []
+        for i in range(cap):
+            b = self.cached.get(hashes[i])
+            if b is None:
+                break
+            hits.append(b)
+        revive = sum(1 for b in hits if self.ref[b] == 0)
+        fresh = self._blocks_for(n) - len(hits)
+        if fresh > len(self.free) - revive:
+            raise BlockManagerError(ERR_OOM, "pool exhausted")
+        for b in hits:
+            if self.ref[b] == 0:
+                self.free.remove(b)
+                self.ref[b] = 1
+            else:
+                self.ref[b] += 1
+        table = list(hits)
+        for i in range(len(hits), self._blocks_for(n)):
+            b = self.alloc()
+            table.append(b)
+            if i < len(hashes) and hashes[i] not in self.cached:
+                self.cached[hashes[i]] = b
+                self.block_hash[b] = hashes[i]
+        self.tables[seq_id] = table
+        self.lens[seq_id] = n
+        return len(hits) * bs

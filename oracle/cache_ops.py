@@ -11,6 +11,11 @@ copy_blocks
   Copy-on-write of shared blocks (Outcome School explainer, "内存共享": beams share
   blocks until they diverge): for every (src, dst) pair, dst <- src in every layer,
   K and V.  All reads happen before any write (pairs are applied as one parallel copy).
+swap_blocks
+  The pool's overflow path (intelliparadigm article, §4.2 OOM错误: swap_space extends
+  the cache into host memory): for every (src, dst) pair, block dst of the destination
+  pool (host or device) <- block src of the source pool, K and V alike.  The two pools
+  are different memories, so no pair can read what another writes.
 
 Parity status: pinned (explicit element loops on tiny inputs, invariants).
 """
@@ -47,3 +52,14 @@ def copy_blocks(key_caches, value_caches, block_mapping):
         out_k.append(new_k)
         out_v.append(new_v)
     return out_k, out_v
+
+
+def swap_blocks(src_pool, dst_pool, block_mapping):
+    """Return a new destination pool with dst_pool[dst] = src_pool[src] for every pair.
+
+    Pools [NB, ...] of any element type (the two pools may differ in NB)."""
+    pairs = np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+    out = dst_pool.copy()
+    for src, dst in pairs:
+        out[dst] = src_pool[src]
+    return out

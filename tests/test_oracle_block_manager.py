@@ -13,21 +13,34 @@ import numpy as np
 import pytest
 
 import workloads as wl
-from oracle.block_manager import ERR_INVALID, ERR_OOM, BlockManagerError, BlockManagerModel
+from oracle.block_manager import (ERR_INVALID, ERR_OOM, BlockManagerError, BlockManagerModel, block_hash,
+                                  fnv1a64)
 
 
 def check_invariants(m: BlockManagerModel):
     refs = [0] * m.num_blocks
-    for table in m.tables.values():
+    host_refs = [0] * len(m.host_ref)
+    for s, table in m.tables.items():
         for b in table:
-            refs[b] += 1
+            if s in m.swapped:
+                host_refs[b] += 1
+            else:
+                refs[b] += 1
     assert refs == m.ref, "reference counts must equal the number of table entries"
+    assert host_refs == m.host_ref, "host reference counts must equal the swapped-out table entries"
     live = {b for b in range(m.num_blocks) if m.ref[b] > 0}
     assert len(m.free) + len(live) == m.num_blocks
     assert not (set(m.free) & live)
     assert len(set(m.free)) == len(m.free)
+    host_live = {b for b in range(len(m.host_ref)) if m.host_ref[b] > 0}
+    assert len(m.host_free) + len(host_live) == len(m.host_ref)
+    assert not (set(m.host_free) & host_live)
     for s, table in m.tables.items():
         assert len(table) == -(-m.lens[s] // m.block_size)
+    # the prefix cache maps each registered hash to one block and back
+    assert len(m.cached) == len(m.block_hash)
+    for h, b in m.cached.items():
+        assert m.block_hash[b] == h
 
 
 def test_block_table_figure():
@@ -145,15 +158,34 @@ def test_invalid_operations():
         assert e.value.code == ERR_INVALID
 
 
-def random_ops(seed, steps=400, num_blocks=48, block_size=4):
-    """A seeded random mix of every operation; checks invariants after each one."""
+def random_ops(seed, steps=400, num_blocks=48, block_size=4, extended=False):
+    """A seeded random mix of every operation; checks invariants after each one.
+    ``extended`` adds swap-out / swap-in and prompt-token (prefix-cached) admission."""
     rng = wl.rng_for(seed)
-    m = BlockManagerModel(num_blocks, block_size, rng.permutation(num_blocks))
+    m = BlockManagerModel(num_blocks, block_size, rng.permutation(num_blocks),
+                          num_host_blocks=num_blocks // 2 if extended else 0)
+    prompts = [list(rng.integers(0, 5, size=40)) for _ in range(3)]   # few distinct prompts: many hits
     next_id = 0
     for _ in range(steps):
-        op = rng.integers(0, 5)
-        live = sorted(m.tables)
+        op = rng.integers(0, 8 if extended else 5)
+        live = sorted(s for s in m.tables if s not in m.swapped)
+        gone = sorted(m.swapped)
         try:
+            if op == 5:
+                if live:
+                    m.swap_out([int(x) for x in rng.permutation(live)[:rng.integers(1, min(3, len(live)) + 1)]])
+                continue
+            if op == 6:
+                if gone:
+                    m.swap_in([int(x) for x in rng.permutation(gone)[:rng.integers(1, len(gone) + 1)]])
+                continue
+            if op == 7:
+                p = prompts[rng.integers(len(prompts))]
+                n = int(rng.integers(1, len(p) + 1))
+                tail = list(rng.integers(0, 5, size=int(rng.integers(0, 3))))
+                m.add_seq_tokens(next_id, p[:n] + tail)
+                next_id += 1
+                continue
             if op == 0 or not live:
                 shared = []
                 if live and rng.random() < 0.5:
@@ -169,7 +201,8 @@ def random_ops(seed, steps=400, num_blocks=48, block_size=4):
                 pick = rng.permutation(live)[:rng.integers(1, len(live) + 1)]
                 m.append_slots([int(s) for s in pick])
             elif op == 3:
-                m.free_seq(live[rng.integers(len(live))])
+                every = sorted(m.tables)
+                m.free_seq(every[rng.integers(len(every))])
             else:
                 s = live[rng.integers(len(live))]
                 if m.lens[s]:
@@ -177,7 +210,8 @@ def random_ops(seed, steps=400, num_blocks=48, block_size=4):
                     m.slots(s, start, m.lens[s] - start)
         except BlockManagerError as e:
             assert e.code == ERR_OOM
-        check_invariants(m)
+        finally:
+            check_invariants(m)
     return m
 
 
@@ -193,3 +227,126 @@ def test_slots_follow_tables():
         for p, slot in enumerate(got):
             assert slot // m.block_size == table[p // m.block_size]
             assert slot % m.block_size == p % m.block_size
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_invariants_under_random_operations_with_swap_and_prefix_cache(seed):
+    m = random_ops(100 + seed, extended=True)
+    assert m.num_cached_blocks() > 0
+
+
+# ---------------------------------------------------------------------------
+# Swap space
+# ---------------------------------------------------------------------------
+
+def test_swap_out_and_in_by_hand():
+    m = BlockManagerModel(8, 4, list(range(8)), num_host_blocks=4)
+    m.add_seq(0, 6)                    # device blocks 0, 1
+    m.fork(0, 1)                       # shares 0, 1
+    m.add_seq(2, 3)                    # block 2
+    pairs = m.swap_out([0, 1])
+    assert pairs == [(0, 0), (1, 1)]   # each distinct device block gets one host block
+    assert m.tables[0] == m.tables[1] == [0, 1] and m.host_ref[:2] == [2, 2]
+    assert m.num_free() == 7 and list(m.free) == [3, 4, 5, 6, 7, 0, 1]
+    assert m.is_swapped(0) and not m.is_swapped(2)
+    with pytest.raises(BlockManagerError) as e:
+        m.append_slots([0])
+    assert e.value.code == ERR_INVALID
+    pairs = m.swap_in([1, 0])
+    assert pairs == [(0, 3), (1, 4)]   # fresh device blocks from the front of the free list
+    assert m.tables[0] == m.tables[1] == [3, 4] and m.ref[3] == m.ref[4] == 2
+    assert m.num_host_free() == 4
+    check_invariants(m)
+
+
+def test_swap_partial_sharing_keeps_device_copy():
+    """A block still used by a resident sequence stays on the device; the swapped
+    sequence takes a host copy of it."""
+    m = BlockManagerModel(6, 4, list(range(6)), num_host_blocks=3)
+    m.add_seq(0, 8)                    # blocks 0, 1
+    m.fork(0, 1)
+    pairs = m.swap_out([1])
+    assert pairs == [(0, 0), (1, 1)] and m.ref[0] == m.ref[1] == 1
+    m.free_seq(1)                      # freeing a swapped-out sequence frees its host blocks
+    assert m.num_host_free() == 3
+    check_invariants(m)
+
+
+def test_swap_is_all_or_nothing():
+    m = BlockManagerModel(6, 4, list(range(6)), num_host_blocks=2)
+    m.add_seq(0, 9)                    # 3 blocks > 2 host blocks
+    with pytest.raises(BlockManagerError) as e:
+        m.swap_out([0])
+    assert e.value.code == ERR_OOM
+    assert m.tables[0] == [0, 1, 2] and not m.is_swapped(0) and m.num_host_free() == 2
+    m2 = BlockManagerModel(3, 4, list(range(3)), num_host_blocks=3)
+    m2.add_seq(0, 8)
+    m2.swap_out([0])
+    m2.add_seq(1, 12)                  # takes every device block
+    with pytest.raises(BlockManagerError) as e:
+        m2.swap_in([0])
+    assert e.value.code == ERR_OOM and m2.is_swapped(0)
+    check_invariants(m2)
+
+
+# ---------------------------------------------------------------------------
+# Prefix caching
+# ---------------------------------------------------------------------------
+
+def test_fnv1a64_published_vectors():
+    """FNV-1a 64-bit test vectors from the algorithm's published test suite."""
+    assert fnv1a64(b"") == 0xCBF29CE484222325
+    assert fnv1a64(b"a") == 0xAF63DC4C8601EC8C
+    assert fnv1a64(b"foobar") == 0x85944171F73967E8
+
+
+def test_block_hash_layout():
+    """Parent hash as 8 little-endian bytes, then int32 little-endian token ids."""
+    data = bytes([1, 0, 0, 0, 0, 0, 0, 0]) + bytes([7, 0, 0, 0]) + bytes([0xFF, 0xFF, 0xFF, 0xFF])
+    assert block_hash(1, [7, -1]) == fnv1a64(data)
+
+
+def test_prefix_cache_by_hand():
+    bs = 4
+    m = BlockManagerModel(12, bs, list(range(12)))
+    a = list(range(100, 110))                         # 10 tokens: 2 full blocks + 2
+    assert m.add_seq_tokens(0, a) == 0                # nothing cached yet
+    assert m.tables[0] == [0, 1, 2] and m.num_cached_blocks() == 2
+    b = a[:8] + [7, 7, 7]
+    assert m.add_seq_tokens(1, b) == 8                # both full blocks shared
+    assert m.tables[1][:2] == [0, 1] and m.ref[0] == m.ref[1] == 2
+    c = a[:8]                                         # the last token sits in block 1:
+    assert m.add_seq_tokens(2, c) == 4                # only block 0 is taken
+    assert m.tables[2] == [0, 4] and m.num_cached_blocks() == 2   # block 4 holds a registered hash: not re-registered
+    d = [5] + a[1:8]                                  # first block differs: no hit at all
+    assert m.add_seq_tokens(3, d) == 0
+    check_invariants(m)
+
+
+def test_prefix_cache_revive_and_evict():
+    bs = 4
+    m = BlockManagerModel(8, bs, list(range(8)))
+    p = list(range(12))
+    m.add_seq_tokens(0, p + [99])                     # blocks 0,1,2 full (registered), 3 partial
+    m.free_seq(0)                                     # all free again, 3 still registered
+    assert m.num_free() == 8 and m.num_cached_blocks() == 3
+    assert list(m.free) == [4, 5, 6, 7, 0, 1, 2, 3]
+    assert m.add_seq_tokens(1, p + [98]) == 12        # revived from the free list
+    assert m.tables[1] == [0, 1, 2, 4] and list(m.free) == [5, 6, 7, 3]
+    m.free_seq(1)
+    m.add_seq(2, 24)                                  # takes 5, 6, 7, 3, 0, 1: evicts 0 and 1
+    assert m.tables[2] == [5, 6, 7, 3, 0, 1] and m.num_cached_blocks() == 1
+    assert m.add_seq_tokens(3, p[:4] + [1]) == 0      # block 0's hash is gone
+    assert m.tables[3] == [2, 4]                      # block 2 handed out: its old hash evicted,
+    assert m.num_cached_blocks() == 1                 # the new prompt's first block registered
+    check_invariants(m)
+
+
+def test_prefix_cache_oom_is_all_or_nothing():
+    m = BlockManagerModel(4, 4, list(range(4)))
+    m.add_seq_tokens(0, list(range(9)))               # 3 blocks
+    before = (list(m.free), list(m.ref), dict(m.cached))
+    with pytest.raises(BlockManagerError) as e:
+        m.add_seq_tokens(1, list(range(8)) + list(range(50, 60)))   # 2 cached + 3 fresh > 1 free
+    assert e.value.code == ERR_OOM
+    assert before == (list(m.free), list(m.ref), dict(m.cached)) and 1 not in m.tables

@@ -316,6 +316,21 @@ def test_copy_blocks_parallel_semantics():
             assert np.array_equal(k1[b], k0[b]) and np.array_equal(v1[b], v0[b])
 
 
+def test_swap_blocks_matches_element_loop():
+    rng = wl.rng_for(32)
+    src = wl.bf16_normal(rng, (6, 2, 4, 3))          # e.g. the device pool
+    dst = wl.bf16_normal(rng, (4, 2, 4, 3))          # e.g. a smaller host pool
+    pairs = np.array([[5, 0], [1, 3], [5, 2]], np.int64)
+    got = cache_ops.swap_blocks(src, dst, pairs)
+    exp = dst.copy()
+    for s_blk, d_blk in pairs:
+        for h in range(2):
+            for r in range(4):
+                for d in range(3):
+                    exp[d_blk, h, r, d] = src[s_blk, h, r, d]
+    assert np.array_equal(got, exp) and np.array_equal(got[1], dst[1])
+
+
 # ---------------------------------------------------------------------------
 # Mutation tests: plausible mistakes planted in copies of the oracle source
 # ---------------------------------------------------------------------------

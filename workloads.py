@@ -255,3 +255,116 @@ def trace_events(params: TraceParams, seed: int):
                                int(rng.integers(params.budget_lo, params.budget_hi + 1))))
         arrivals.append(offers)
     return initial, arrivals
+
+
+# ---------------------------------------------------------------------------
+# Prefill / chunked-prefill batches
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PrefillBatch:
+    """One prefill-attention call's worth of inputs (one layer).
+
+    Sequence s already holds context_lens[s] tokens in the pool, of which the last
+    query_lens[s] are this call's new tokens (its chunk); their query rows are packed
+    at query_start[s] .. query_start[s+1]-1."""
+
+    name: str
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    query_lens: np.ndarray          # [B] int32
+    context_lens: np.ndarray        # [B] int32 (earlier tokens + this chunk)
+    query_start: np.ndarray         # [B+1] int32
+    block_tables: np.ndarray        # [B, max_blocks] int32, pad 0
+    scale: float
+    free_order: np.ndarray
+    seed: int
+    query: np.ndarray | None = None         # [T, Hq, D] uint16
+    key_cache: np.ndarray | None = None     # [NB, Hkv, bs, D] uint16
+    value_cache: np.ndarray | None = None
+
+    @property
+    def total_q(self) -> int:
+        return int(self.query_start[-1])
+
+    @property
+    def max_query_len(self) -> int:
+        return int(self.query_lens.max()) if self.num_seqs else 0
+
+    @property
+    def max_context_len(self) -> int:
+        return int(self.context_lens.max()) if self.num_seqs else 0
+
+    @property
+    def max_blocks(self) -> int:
+        return int(self.block_tables.shape[1])
+
+
+PREFILL_WORKLOADS = {
+    # name: (B, Hq, Hkv, D, bs, chunk, earlier_lo, earlier_hi)
+    # 8 chunks of 512 tokens = 4096 batched tokens (intelliparadigm article §4.1/§4.2:
+    # chunked_prefill_token_size=512, max_num_batched_tokens=4096), LLaMA-13B heads.
+    "chunked_prefill_13b": (8, 40, 40, 128, 16, 512, 0, 8192),
+    # the same chunking on 10k+-token contexts (§4.2) with grouped-query heads
+    "chunked_prefill_long_gqa": (8, 64, 8, 128, 32, 512, 4096, 28672),
+}
+
+PREFILL_SUB_SEED = {name: 100 + i for i, name in enumerate(PREFILL_WORKLOADS)}
+
+
+def make_prefill_batch(name: str, *, seed: int | None = None, num_seqs: int | None = None,
+                       length_scale: float = 1.0, with_data: bool = True, num_heads: int | None = None,
+                       num_kv_heads: int | None = None, head_dim: int | None = None,
+                       block_size: int | None = None, query_lens=None, earlier_lens=None,
+                       pool_factor: float = 1.2) -> PrefillBatch:
+    """Draw one prefill batch.  A quarter of the sequences (at least one when B > 1) end
+    their prompt inside this call with a shorter, ragged chunk U{1..chunk}; the rest
+    take a full chunk.  Earlier (already cached) lengths are U{lo..hi}, scaled by
+    ``length_scale``.  Explicit ``query_lens`` / ``earlier_lens`` override the draws."""
+    B0, Hq0, Hkv0, D0, bs0, chunk0, lo, hi = PREFILL_WORKLOADS[name]
+    B = B0 if num_seqs is None else num_seqs
+    Hq = Hq0 if num_heads is None else num_heads
+    Hkv = Hkv0 if num_kv_heads is None else num_kv_heads
+    D = D0 if head_dim is None else head_dim
+    bs = bs0 if block_size is None else block_size
+    seed = BASE_SEED * 1000 + PREFILL_SUB_SEED[name] if seed is None else seed
+    rng = rng_for(seed)
+    chunk = max(1, int(round(chunk0 * length_scale)))
+    if query_lens is None:
+        qlens = np.full(B, chunk, dtype=np.int32)
+        ragged = rng.random(B) < 0.25
+        if B > 1 and not ragged.any():
+            ragged[rng.integers(B)] = True
+        qlens[ragged] = rng.integers(1, chunk + 1, size=int(ragged.sum()))
+    else:
+        qlens = np.asarray(query_lens, np.int32)
+    B = len(qlens)
+    if earlier_lens is None:
+        earlier = rng.integers(int(round(lo * length_scale)), int(round(hi * length_scale)) + 1, size=B)
+    else:
+        earlier = np.asarray(earlier_lens)
+    lens = (earlier + qlens).astype(np.int32)
+    qstart = np.zeros(B + 1, dtype=np.int32)
+    qstart[1:] = np.cumsum(qlens)
+    need = blocks_needed(lens, bs)
+    nb = max(int(math.ceil(pool_factor * int(need.sum()))), 1)
+    free_order = rng.permutation(nb).astype(np.int32)
+    tables = place_blocks(lens, bs, free_order)
+    batch = PrefillBatch(name=name, num_seqs=B, num_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=bs,
+                         num_blocks=nb, query_lens=qlens, context_lens=lens, query_start=qstart,
+                         block_tables=tables, scale=fp32_scale(D), free_order=free_order, seed=seed)
+    if with_data:
+        batch.query = bf16_normal(rng, (int(qstart[-1]), Hq, D))
+        batch.key_cache = bf16_normal(rng, (nb, Hkv, bs, D))
+        batch.value_cache = bf16_normal(rng, (nb, Hkv, bs, D))
+    return batch
+
+
+def kv_scales(rng: np.random.Generator, num_kv_heads: int, lo: float = 1.0 / 64, hi: float = 1.0 / 32) -> np.ndarray:
+    """Seeded per-kv-head float32 scales of an 8-bit cache: N(0,1) data divided by a
+    scale in [1/64, 1/32] spans about +-320 before saturation at 448."""
+    return rng.uniform(lo, hi, size=num_kv_heads).astype(np.float32)

@@ -20,6 +20,17 @@ head_dim 128, block size 16, lengths 70% geometric(mean 50) / 30% U{1000..2000})
 the batch on which the 70%-of-HBM target is stated.  Its KV (2.5 GB) is ~20x the
 L2, so consecutive steps cannot hit in L2.
 
+Other rows, same JSON line (`--workload` / `--kv`):
+  --kv fp8                 the same decode step over an 8-bit (e4m3) pool: KV bytes at
+                           1 byte per value, reshape_and_cache_fp8 + paged_attention_decode_fp8.
+  --workload chunked_prefill_13b | chunked_prefill_long_gqa
+                           one step = the chunks' K/V written + paged_attention_prefill;
+                           value in TFLOP/s (4 * D per visible (row, key) per head),
+                           roofline against the measured bf16 tensor peak.
+  --workload swap_llama13b one step = 256 13B-shaped blocks swapped out to pinned host
+                           memory and 256 swapped in (K and V); GB/s against the
+                           pinned-memory copy bandwidth measured in the same run.
+
 `--impl reference` times the CPU oracle (float64 NumPy, one thread) on a bounded
 sample of the same workload and prints the same JSON line with "impl": "reference".
 Multi-GPU (`torchrun`): independent replicas per GPU (weak scaling), no collective on
@@ -44,7 +55,21 @@ if ROOT not in sys.path:
 import workloads as wl  # noqa: E402
 
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); seq-steps/sec"
+METRIC_PREFILL = "paged prefill attention TFLOP/s (% of B200 bf16 tensor peak)"
+METRIC_SWAP = "swap_blocks device<->pinned-host GB/s (% of the pinned memcpy bandwidth)"
+SWAP_WORKLOAD = "swap_llama13b"
 FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_bf16_tflops():
+    """The sustained cuBLAS bf16 figure: the prefill kernel is timed inside a loop of
+    back-to-back launches lasting seconds."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        return 1400.0, "fallback (sustained)"
 
 
 def measured_hbm_gbs():
@@ -160,20 +185,32 @@ class ClockSampler:
 # Workload preparation (allocator + per-step inputs)
 # ---------------------------------------------------------------------------
 
-def decode_bytes(lens, Hq, Hkv, D, bs):
+def decode_bytes(lens, Hq, Hkv, D, bs, kv_elem_bytes=2):
     """Algorithmic bytes of one decode call: KV of every valid token once, q, out (bf16),
     the used table entries and the lengths."""
     lens = np.asarray(lens, np.int64)
-    kv = int(lens.sum()) * Hkv * D * 2 * 2
+    kv = int(lens.sum()) * Hkv * D * 2 * kv_elem_bytes
     blocks = int(np.sum(-(-lens // bs)))
     return kv, kv + 2 * len(lens) * Hq * D * 2 + blocks * 4 + len(lens) * 4
 
 
+def e4m3_pool(shape, gen, device):
+    """Seeded e4m3 codes drawn as bit patterns on the device (sign, exponent around 8,
+    uniform mantissa, never NaN), like workloads.e4m3_codes."""
+    import torch
+    sign = torch.randint(0, 2, shape, generator=gen, device=device, dtype=torch.int32)
+    exp = (torch.randn(shape, generator=gen, device=device) * 1.5 + 8).round().clamp(0, 15).to(torch.int32)
+    mant = torch.randint(0, 8, shape, generator=gen, device=device, dtype=torch.int32)
+    mant = torch.where((exp == 15) & (mant == 7), torch.full_like(mant, 6), mant)
+    return ((sign << 7) | (exp << 3) | mant).to(torch.uint8)
+
+
 class Workload:
-    def __init__(self, name: str, steps: int, seed: int, device):
+    def __init__(self, name: str, steps: int, seed: int, device, kv8: bool = False):
         import torch
         import paged_kv_cache_423_b200 as pkv
         self.name = name
+        self.kv8 = kv8
         b = wl.make_decode_batch(name, with_data=False, extra_blocks=0)
         self.B, self.Hq, self.Hkv, self.D, self.bs = b.num_seqs, b.num_heads, b.num_kv_heads, b.head_dim, b.block_size
         self.scale = b.scale
@@ -188,9 +225,34 @@ class Workload:
         g = torch.Generator(device=device)
         g.manual_seed(seed)
         shape = (self.NB, self.Hkv, self.bs, self.D)
-        self.key_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
-        self.value_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        if kv8:
+            self.key_cache = e4m3_pool(shape, g, device)
+            self.value_cache = e4m3_pool(shape, g, device)
+            srng = wl.rng_for(seed + 2)
+            self.k_scale = torch.from_numpy(wl.kv_scales(srng, self.Hkv)).to(device)
+            self.v_scale = torch.from_numpy(wl.kv_scales(srng, self.Hkv)).to(device)
+        else:
+            self.key_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+            self.value_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
         self.rng = wl.rng_for(seed + 1)
+
+    def write(self, k, v, slots, status):
+        if self.kv8:
+            self.pkv.reshape_and_cache_fp8(k, v, self.key_cache, self.value_cache, slots, self.k_scale, self.v_scale,
+                                           status=status)
+        else:
+            self.pkv.reshape_and_cache(k, v, self.key_cache, self.value_cache, slots, status=status)
+
+    def copy(self, pairs, status):
+        self.pkv.copy_blocks([self.key_cache], [self.value_cache], pairs, status=status)
+
+    def decode(self, out, q, tables, lens, max_len, ws, path, status):
+        if self.kv8:
+            self.pkv.paged_attention_decode_fp8(out, q, self.key_cache, self.value_cache, self.k_scale, self.v_scale,
+                                                tables, lens, max_len, self.scale, ws, status=status)
+        else:
+            self.pkv.paged_attention_decode(out, q, self.key_cache, self.value_cache, tables, lens, max_len, self.scale,
+                                            ws, path=path, status=status)
 
     def new_manager(self):
         bm = self.pkv.BlockManager(self.NB, self.bs, self.free_order)
@@ -235,8 +297,9 @@ def run_ours(args, rank, world, local_rank):
         dist.init_process_group("nccl", device_id=device)
     total = args.warmup + args.steps
     n_states = min(total, args.states)
+    kv8 = args.kv == "fp8"
     w = Workload(args.workload, max(n_states, min(total, args.e2e_steps + args.warmup)), seed=1000 + rank,
-                 device=device)
+                 device=device, kv8=kv8)
     seq_ids = list(range(w.B))
 
     # ---- the allocator runs ahead of timing: `n_states` consecutive decode steps of
@@ -265,12 +328,11 @@ def run_ours(args, rank, world, local_rank):
     def step(i, ev=None):
         st = states[i % n_states]
         if st["n_pairs"]:
-            pkv.copy_blocks([w.key_cache], [w.value_cache], st["pairs"], status=status)
-        pkv.reshape_and_cache(st["k"], st["v"], w.key_cache, w.value_cache, st["slots"], status=status)
+            w.copy(st["pairs"], status)
+        w.write(st["k"], st["v"], st["slots"], status)
         if ev is not None:
             ev[0].record(stream)
-        pkv.paged_attention_decode(out, st["q"], w.key_cache, w.value_cache, st["tables"], st["lens"], max_len_all,
-                                   w.scale, ws, path=path, status=status)
+        w.decode(out, st["q"], st["tables"], st["lens"], max_len_all, ws, path, status)
         if ev is not None:
             ev[1].record(stream)
 
@@ -281,7 +343,7 @@ def run_ours(args, rank, world, local_rank):
     kv_total = bytes_total = 0
     for i in range(args.warmup, total):
         st = states[i % n_states]
-        kv, alg = decode_bytes(st["host_lens"], w.Hq, w.Hkv, w.D, w.bs)
+        kv, alg = decode_bytes(st["host_lens"], w.Hq, w.Hkv, w.D, w.bs, 1 if kv8 else 2)
         kv_total += kv
         bytes_total += alg
         launches += 3 + (1 if st["n_pairs"] else 0)
@@ -312,13 +374,13 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_kind = measured_hbm_gbs()
     g = w.Hq // w.Hkv
-    uses_tensor = path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16)
+    uses_tensor = not kv8 and (path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16))
     dec_gbs = bytes_total / (dec_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "num_seqs": w.B, "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 KV, bf16 q" if kv8 else "bf16", "data": "synthetic",
+        "config": {"workload": w.name + ("+fp8" if kv8 else ""), "kv_dtype": args.kv, "num_seqs": w.B, "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D,
                    "block_size": w.bs, "mean_context": float(np.mean(w.lens0)), "num_blocks": w.NB,
                    "kv_bytes_per_step": kv_total // args.steps, "path": args.path,
                    "l2": "inputs larger than L2 (KV per step >> 126 MB)",
@@ -328,7 +390,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4), "traffic": recorded_traffic(w.name),
                      "algorithmic_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
-                     "kernel": ("paged_attention_decode: plan + tcgen05 kernel + split merge" if uses_tensor
+                     "kernel": ("paged_attention_decode_fp8: plan + CUDA-core streaming kernel (e4m3 tiles)" if kv8
+                                else "paged_attention_decode: plan + tcgen05 kernel + split merge" if uses_tensor
                                 else "paged_attention_decode: plan + CUDA-core streaming kernel"),
                      "ms_per_launch": round(dec_ms / args.steps, 4)},
         "gpu_launches": launches,
@@ -336,8 +399,10 @@ def run_ours(args, rank, world, local_rank):
     }
     if e2e is not None:
         result["e2e"] = e2e
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not kv8:
         result["cpu_baseline"] = cpu_baseline(w, states[0], budget_s=args.cpu_budget)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and kv8:
+        result["cpu_baseline"] = cpu_baseline_fp8(w, states[0], budget_s=args.cpu_budget)
     if dist:
         dist.destroy_process_group()
     return result
@@ -407,10 +472,9 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
         d_lens = dm[o_lens:o_lens + 4 * w.B].view(torch.int32)
         if len(pairs):
             d_pairs = dm[o_pairs:o_pairs + pairs.nbytes].view(torch.int64).view(-1, 2)
-            pkv.copy_blocks([w.key_cache], [w.value_cache], d_pairs, status=status)
-        pkv.reshape_and_cache(dk, dv, w.key_cache, w.value_cache, d_slots, status=status)
-        pkv.paged_attention_decode(outs[b], dq, w.key_cache, w.value_cache, d_tables, d_lens, max_len_bound, w.scale,
-                                   ws, path=path, status=status)
+            w.copy(d_pairs, status)
+        w.write(dk, dv, d_slots, status)
+        w.decode(outs[b], dq, d_tables, d_lens, max_len_bound, ws, path, status)
         out_host[b].copy_(outs[b], non_blocking=True)
         comp_done[i].record(compute)
         if i >= 1:                                 # read the previous step's result on the host
@@ -419,7 +483,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
         if i >= args.warmup:
             stats["h2d"] += host_qkv[i].numel() * 2 + slots.nbytes + pairs.nbytes + tables.nbytes + lens.nbytes
             stats["d2h"] += out_host[b].numel() * 2
-            stats["kv"] += int(np.asarray(lens, np.int64).sum()) * w.Hkv * w.D * 4
+            stats["kv"] += int(np.asarray(lens, np.int64).sum()) * w.Hkv * w.D * 2 * (1 if w.kv8 else 2)
 
     for i in range(args.warmup):
         step(i)
@@ -592,6 +656,334 @@ def cpu_baseline(w, step_inputs, budget_s=10.0):
                       f"{dt:.1f} s"}
 
 
+def oracle_sample_fp8(w, step_inputs, n_seqs, rng):
+    """Host copies of a sample of sequences of an 8-bit pool (their blocks only)."""
+    import torch
+    seqs = sorted(rng.choice(w.B, size=min(n_seqs, w.B), replace=False).tolist())
+    lens = step_inputs["host_lens"]
+    tables = step_inputs["tables"].cpu().numpy()
+    q = step_inputs["q"].view(torch.int16).cpu().numpy().view(np.uint16)
+    ks, vs = w.k_scale.cpu().numpy(), w.v_scale.cpu().numpy()
+    items = []
+    for s in seqs:
+        need = -(-int(lens[s]) // w.bs)
+        idx = torch.from_numpy(tables[s][:need].astype(np.int64)).to(w.device)
+        items.append((q[s:s + 1], w.key_cache[idx].cpu().numpy(), w.value_cache[idx].cpu().numpy(), ks, vs,
+                      np.arange(need, dtype=np.int32)[None, :], lens[s:s + 1]))
+    return items
+
+
+def cpu_baseline_fp8(w, step_inputs, budget_s=10.0):
+    from threadpoolctl import threadpool_limits
+    from oracle import fp8
+    items = oracle_sample_fp8(w, step_inputs, 64, wl.rng_for(77))
+    done = n = 0
+    t0 = time.perf_counter()
+    with threadpool_limits(limits=1):
+        for q, kc, vc, ks, vs, table, lens in items:
+            fp8.paged_decode_fp8(q, kc, vc, ks, vs, table, lens, w.scale)
+            done += int(lens.sum()) * w.Hkv * w.D * 2
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+    dt = time.perf_counter() - t0
+    return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} sequences of the {w.name} batch over the 8-bit pool (all {w.Hq} heads each), "
+                      f"float64 NumPy, 1 thread, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# Prefill / chunked prefill
+# ---------------------------------------------------------------------------
+
+def prefill_flops(query_lens, context_lens, num_heads, head_dim):
+    """Algorithmic FLOPs of one prefill call: every query row of every head sees
+    p + 1 keys (p its position); scores and the weighted sum cost 2 * D each per key."""
+    visible = 0
+    for n, L in zip(np.asarray(query_lens, np.int64), np.asarray(context_lens, np.int64)):
+        visible += int(n) * (int(L) - int(n)) + int(n) * (int(n) + 1) // 2
+    return 4 * head_dim * num_heads * visible
+
+
+class PrefillWorkload:
+    """One chunked-prefill batch resident on the device; per-step query/K/V states
+    drawn on the host and uploaded before timing; the allocator gives tables and the
+    chunk tokens' slots."""
+
+    def __init__(self, name, n_states, seed, device):
+        import torch
+        import paged_kv_cache_423_b200 as pkv
+        self.pkv = pkv
+        b = wl.make_prefill_batch(name, with_data=False)
+        self.b = b
+        self.name = name
+        bm = pkv.BlockManager(b.num_blocks, b.block_size, b.free_order)
+        ids = list(range(b.num_seqs))
+        slots = []
+        for s in ids:
+            bm.add_seq(s, int(b.context_lens[s]))
+            n = int(b.query_lens[s])
+            slots.append(bm.slots(s, int(b.context_lens[s]) - n, n))
+        tables, lens = bm.export_tables(ids, b.max_blocks)
+        bm.close()
+        self.slots = torch.from_numpy(np.concatenate(slots)).to(device)
+        self.tables = torch.from_numpy(tables).to(device)
+        self.lens = torch.from_numpy(lens).to(device)
+        self.qstart = torch.from_numpy(b.query_start).to(device)
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        shape = (b.num_blocks, b.num_kv_heads, b.block_size, b.head_dim)
+        self.key_cache = torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+        self.value_cache = torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+        rng = wl.rng_for(seed + 1)
+        T = b.total_q
+        self.host = []
+        for _ in range(n_states):
+            q = wl.bf16_normal(rng, (T, b.num_heads, b.head_dim))
+            k, v = wl.new_tokens(rng, T, b.num_kv_heads, b.head_dim)
+            self.host.append((q, k, v))
+        self.ws = torch.empty(pkv.paged_attention_prefill_workspace_size(b.num_seqs, T, b.num_heads, b.num_kv_heads),
+                              dtype=torch.uint8, device=device)
+        self.flops = prefill_flops(b.query_lens, b.context_lens, b.num_heads, b.head_dim)
+
+    def step(self, q, k, v, out, status, ev=None, stream=None):
+        b = self.b
+        self.pkv.reshape_and_cache(k, v, self.key_cache, self.value_cache, self.slots, status=status)
+        if ev is not None:
+            ev[0].record(stream)
+        self.pkv.paged_attention_prefill(out, q, self.key_cache, self.value_cache, self.tables, self.qstart, self.lens,
+                                         b.max_context_len, b.scale, self.ws, status=status)
+        if ev is not None:
+            ev[1].record(stream)
+
+
+def prefill_oracle_rate(pw, q_bits, budget_s, rng):
+    """FLOPs done and seconds spent by the float64 prefill oracle on randomly sampled
+    query rows (1 thread).  Only the oracle call is timed; fetching the row's pages
+    from the device is not.  Runs until about `budget_s` seconds have passed."""
+    import torch
+    from threadpoolctl import threadpool_limits
+    from oracle import prefill
+    b = pw.b
+    tables = pw.tables.cpu().numpy()
+    done, work_t, n = 0, 0.0, 0
+    wall0 = time.perf_counter()
+    with threadpool_limits(limits=1):
+        while n == 0 or time.perf_counter() - wall0 < budget_s:
+            s = int(rng.integers(b.num_seqs))
+            nq = int(b.query_lens[s])
+            if nq == 0:
+                continue
+            i = int(rng.integers(nq))
+            pos = int(b.context_lens[s]) - nq + i
+            need = pos // b.block_size + 1
+            idx = torch.from_numpy(tables[s][:need].astype(np.int64)).to(pw.key_cache.device)
+            kc = pw.key_cache[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+            vc = pw.value_cache[idx].view(torch.int16).cpu().numpy().view(np.uint16)
+            row = int(b.query_start[s]) + i
+            tq = time.perf_counter()
+            prefill.prefill_rows(q_bits[row:row + 1], kc, vc, np.arange(need, dtype=np.int32)[None, :],
+                                 np.array([0, 1], np.int32), np.array([pos + 1], np.int32), b.scale, [0])
+            work_t += time.perf_counter() - tq
+            done += 4 * b.head_dim * b.num_heads * (pos + 1)
+            n += 1
+    return done, work_t, n
+
+
+def run_prefill(args, rank, world, local_rank):
+    import torch
+    device = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device)
+    n_states = 2
+    pw = PrefillWorkload(args.workload, n_states, seed=2000 + rank, device=device)
+    b = pw.b
+    dev_states = [(to_dev(q, device), to_dev(k, device), to_dev(v, device)) for q, k, v in pw.host]
+    out = torch.empty((b.total_q, b.num_heads, b.head_dim), dtype=torch.bfloat16, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        pw.step(*dev_states[i % n_states], out, status)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device) as clocks:
+        t0.record(stream)
+        for j in range(args.steps):
+            pw.step(*dev_states[j % n_states], out, status, ev[j], stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item():#x}")
+    ms = t0.elapsed_time(t1)
+    k_ms = sum(a.elapsed_time(c) for a, c in ev)
+    ms_max, flops_all = aggregate_over_ranks(ms, pw.flops * args.steps, dist, device)
+    value = flops_all / (ms_max * 1e-3) / 1e12
+    peak, peak_kind = measured_bf16_tflops()
+    achieved = pw.flops * args.steps / (k_ms * 1e-3) / 1e12
+
+    # e2e: q, chunk K/V from pinned host memory, output back to pinned memory, every step
+    ke = max(1, min(args.steps, args.e2e_steps))
+    host_in = [tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+                     for a in st) for st in pw.host]
+    out_host = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * 2 for t in host_in[0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for j in range(ke):
+        hq, hk, hv = host_in[j % n_states]
+        dq, dk, dv = dev_states[j % n_states]
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        pw.step(dq, dk, dv, out, status)
+        out_host.copy_(out, non_blocking=True)
+        stream.synchronize()
+        _ = float(out_host[0, 0, 0])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    result = {
+        "metric": METRIC_PREFILL, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": b.name, "num_seqs": b.num_seqs, "num_heads": b.num_heads,
+                   "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim, "block_size": b.block_size,
+                   "query_tokens": b.total_q, "query_lens": b.query_lens.tolist(),
+                   "context_lens": b.context_lens.tolist(), "flops_per_step": pw.flops,
+                   "l2": "K/V of the batch (>= 0.6 GB) larger than L2; no flush",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "pct_tensor_peak": round(100 * value / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(b.name),
+                     "algorithmic_flops_per_launch": pw.flops, "peak_kind": peak_kind,
+                     "kernel": "paged_attention_prefill: plan + tcgen05 kernel",
+                     "ms_per_launch": round(k_ms / args.steps, 4)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": {"value": round(pw.flops * ke / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_host.numel() * 2,
+                "ms_per_step": round(e_ms / ke, 4), "steps": ke, "pipelining": "none (copy, compute, copy back, sync)"},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        done, dt, n = prefill_oracle_rate(pw, pw.host[0][0], args.cpu_budget, wl.rng_for(79))
+        result["cpu_baseline"] = {"value": round(done / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                  "sample": f"{n} random query rows of the {b.name} batch (all {b.num_heads} heads), "
+                                            f"float64 NumPy oracle, 1 thread, {dt:.1f} s"}
+    if dist:
+        dist.destroy_process_group()
+    return result
+
+
+# ---------------------------------------------------------------------------
+# Swap (device <-> pinned host)
+# ---------------------------------------------------------------------------
+
+SWAP_SHAPE = (40, 16, 128)      # LLaMA-13B: 40 kv heads x 16 tokens x 128 (bf16): 160 KiB per K or V block
+SWAP_PAIRS = 256
+
+
+def run_swap(args, rank, world, local_rank):
+    import torch
+    import paged_kv_cache_423_b200 as pkv
+    device = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device)
+    NB, HB = 4096, 1024
+    g = torch.Generator(device=device)
+    g.manual_seed(3000 + rank)
+    dk = torch.randn((NB,) + SWAP_SHAPE, generator=g, device=device).to(torch.bfloat16)
+    dv = torch.randn((NB,) + SWAP_SHAPE, generator=g, device=device).to(torch.bfloat16)
+    hk = torch.empty((HB,) + SWAP_SHAPE, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty((HB,) + SWAP_SHAPE, dtype=torch.bfloat16).pin_memory()
+    rng = wl.rng_for(3100 + rank)
+    plans = []
+    for _ in range(8):
+        src = rng.permutation(NB)[:SWAP_PAIRS]
+        dst = rng.permutation(HB)[:SWAP_PAIRS]
+        back = rng.permutation(NB)[:SWAP_PAIRS]
+        plans.append((torch.from_numpy(np.stack([src, dst], 1).astype(np.int64)).to(device),
+                      torch.from_numpy(np.stack([dst, back], 1).astype(np.int64)).to(device)))
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    block_bytes = int(np.prod(SWAP_SHAPE)) * 2
+    step_bytes = 4 * SWAP_PAIRS * block_bytes          # out and in, K and V
+
+    def step(j):
+        out_pairs, in_pairs = plans[j % len(plans)]
+        pkv.swap_blocks(dk, hk, out_pairs, status=status)
+        pkv.swap_blocks(dv, hv, out_pairs, status=status)
+        pkv.swap_blocks(hk, dk, in_pairs, status=status)
+        pkv.swap_blocks(hv, dv, in_pairs, status=status)
+
+    for j in range(args.warmup):
+        step(j)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    with ClockSampler(device) as clocks:
+        t0.record(stream)
+        for j in range(args.steps):
+            step(j)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item():#x}")
+    ms = t0.elapsed_time(t1)
+    ms_max, bytes_all = aggregate_over_ranks(ms, step_bytes * args.steps, dist, device)
+    value = bytes_all / (ms_max * 1e-3) / 1e9
+    # the link's own copy bandwidth: one pinned cudaMemcpyAsync each way of the same bytes per step
+    big_d = torch.empty(step_bytes // 2, dtype=torch.uint8, device=device)
+    big_h = torch.empty(step_bytes // 2, dtype=torch.uint8).pin_memory()
+    m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        big_h.copy_(big_d, non_blocking=True)
+        big_d.copy_(big_h, non_blocking=True)
+    torch.cuda.synchronize()
+    m0.record(stream)
+    for _ in range(args.steps):
+        big_h.copy_(big_d, non_blocking=True)
+        big_d.copy_(big_h, non_blocking=True)
+    m1.record(stream)
+    torch.cuda.synchronize()
+    link = step_bytes * args.steps / (m0.elapsed_time(m1) * 1e-3) / 1e9
+    result = {
+        "metric": METRIC_SWAP, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bytes", "data": "synthetic",
+        "config": {"workload": SWAP_WORKLOAD, "block_shape": list(SWAP_SHAPE), "block_bytes": block_bytes,
+                   "pairs_per_direction": SWAP_PAIRS, "bytes_per_step": step_bytes,
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "roofline": {"bound": "host link", "achieved": round(value / world, 2), "peak": round(link, 2), "unit": "GB/s",
+                     "frac": round(value / world / link, 4), "traffic": None,
+                     "peak_kind": "measured in this run: pinned cudaMemcpyAsync D2H + H2D of the same bytes",
+                     "kernel": "swap_blocks (4 launches per step)"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": {"value": round(value, 2), "unit": "GB/s", "h2d_bytes_per_step": step_bytes // 2,
+                "d2h_bytes_per_step": step_bytes // 2,
+                "note": "the timed step is itself a host<->device transfer of pinned memory"},
+    }
+    if dist:
+        dist.destroy_process_group()
+    return result
+
+
 def run_reference(args, rank, world, local_rank):
     """The CPU oracle as the reference arm, on a bounded sample of the same workload."""
     import torch
@@ -601,6 +993,10 @@ def run_reference(args, rank, world, local_rank):
     if device is None:
         return {"impl": "reference", "unavailable": "no CUDA device to hold the synthetic workload"}
     torch.cuda.set_device(device)
+    if args.workload in wl.PREFILL_WORKLOADS:
+        return run_reference_prefill(args, world, device)
+    if args.workload == SWAP_WORKLOAD:
+        return run_reference_swap(args, world)
     w = Workload(args.workload, 2, seed=1000, device=device)
     bm = w.new_manager()
     ids = list(range(w.B))
@@ -635,6 +1031,56 @@ def run_reference(args, rank, world, local_rank):
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_reference_prefill(args, world, device):
+    pw = PrefillWorkload(args.workload, 1, seed=2000, device=device)
+    rng = wl.rng_for(80)
+    per_step = max(0.05, args.ref_budget / (args.warmup + args.steps))
+    for _ in range(args.warmup):
+        prefill_oracle_rate(pw, pw.host[0][0], per_step, rng)
+    done = dt = 0.0
+    for _ in range(args.steps):
+        d, t, _n = prefill_oracle_rate(pw, pw.host[0][0], per_step, rng)
+        done += d
+        dt += t
+    value = done / dt / 1e12
+    b = pw.b
+    sample = f"random query rows of the {b.name} batch (all {b.num_heads} heads), {per_step:.2f} s per step, " \
+             "float64 NumPy oracle, 1 thread"
+    return {"metric": METRIC_PREFILL, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": b.name, "num_seqs": b.num_seqs, "num_heads": b.num_heads,
+                       "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim, "block_size": b.block_size},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_reference_swap(args, world):
+    from oracle import cache_ops
+    rng = wl.rng_for(81)
+    src = np.zeros((512,) + SWAP_SHAPE, np.uint16)
+    dst = np.zeros((256,) + SWAP_SHAPE, np.uint16)
+    block_bytes = int(np.prod(SWAP_SHAPE)) * 2
+    pairs_n = 64
+    for _ in range(args.warmup):
+        cache_ops.swap_blocks(src, dst, np.stack([rng.permutation(512)[:pairs_n], rng.permutation(256)[:pairs_n]], 1))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cache_ops.swap_blocks(src, dst, np.stack([rng.permutation(512)[:pairs_n], rng.permutation(256)[:pairs_n]], 1))
+    dt = time.perf_counter() - t0
+    # the oracle copies the whole destination pool once per call plus the pairs; count the pairs' bytes
+    value = args.steps * pairs_n * block_bytes / dt / 1e9
+    sample = f"{pairs_n} 13B-shaped blocks per step between two host arrays (NumPy), 1 thread"
+    return {"metric": METRIC_SWAP, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bytes", "data": "synthetic",
+            "config": {"workload": SWAP_WORKLOAD, "block_shape": list(SWAP_SHAPE)}, "impl": "reference",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -643,7 +1089,9 @@ def main():
     ap.add_argument("--states", type=int, default=16, help="distinct precomputed decode steps replayed in turn")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama13b_mixed_bs16", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="llama13b_mixed_bs16",
+                    choices=sorted(wl.WORKLOADS) + sorted(wl.PREFILL_WORKLOADS) + [SWAP_WORKLOAD])
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16", help="element type of the decode pool")
     ap.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--trace", action="store_true",
                     help="run the long-context continuous-batching trace step by step (the fifth workload)")
@@ -659,6 +1107,10 @@ def main():
         res = run_reference(args, rank, world, local_rank)
     elif args.trace:
         res = run_trace(args, rank, world, local_rank)
+    elif args.workload in wl.PREFILL_WORKLOADS:
+        res = run_prefill(args, rank, world, local_rank)
+    elif args.workload == SWAP_WORKLOAD:
+        res = run_swap(args, rank, world, local_rank)
     else:
         res = run_ours(args, rank, world, local_rank)
     if rank == 0 and res is not None:

@@ -104,7 +104,8 @@ PKV_API int pkv_reshape_and_cache(const void* key, const void* value, void* key_
  *
  *   key_caches,
  *   value_caches     HOST arrays of num_layers DEVICE pointers, each a pool of
- *                    [num_blocks, block_elems] bf16 (block_elems = Hkv*bs*D)
+ *                    [num_blocks, block_elems] bf16 (block_elems = Hkv*bs*D; the copy is
+ *                    bytewise, so an 8-bit pool passes half its bytes per block)
  *   block_mapping    device [num_pairs, 2] int64: (src, dst) physical block ids;
  *                    out-of-range pairs are skipped and set PKV_DEV_BAD_PAIR.
  *   Every dst must be distinct and no dst may also be a src in the same call.
@@ -201,6 +202,92 @@ PKV_API int pkv_paged_attention_decode_static(void* out, int out_dtype, const vo
                                               pkv_stream_t stream);
 
 /*
+ * 8-bit (e4m3) KV cache.  intelliparadigm article §4.2 (初始化速度慢: loading in low-bit
+ * fp8) and §5 (quantisation combined with vLLM shrinks memory and raises throughput).
+ * The pages fix no format; this library stores K and V as OCP e4m3 codes (1 sign,
+ * 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448, no infinities)
+ * with one float32 scale per kv head for K and one for V:
+ *   code = e4m3(x / scale[h])   (float32 division, round to nearest even, saturate)
+ *   value = e4m3_value(code) * scale[h]
+ * Pools: key_cache, value_cache = [num_blocks, num_kv_heads, block_size, head_dim]
+ * uint8, half the bytes of the bf16 pool; k_scale, v_scale = device [num_kv_heads] float32.
+ *
+ * reshape_and_cache_fp8 — pkv_reshape_and_cache for an 8-bit pool: key/value are the
+ * new tokens' bf16 [num_tokens, num_kv_heads, head_dim], quantised on the way in.
+ * Slot rules and status bits as for pkv_reshape_and_cache.
+ */
+PKV_API int pkv_reshape_and_cache_fp8(const void* key, const void* value, void* key_cache, void* value_cache,
+                                      const int64_t* slot_mapping, const float* k_scale, const float* v_scale,
+                                      int num_tokens, int num_blocks, int num_kv_heads, int head_dim,
+                                      int block_size, int32_t* status, pkv_stream_t stream);
+/*
+ * paged_attention_decode_fp8 — pkv_paged_attention_decode over an 8-bit pool: the
+ * attention of the dequantised values (K_j = e4m3_value * k_scale[h], V_j likewise).
+ * head_dim 128; CUDA cores (the e4m3 tiles are widened to f16 in registers, products
+ * accumulate in fp32).  Workspace, splits and status bits as for
+ * pkv_paged_attention_decode (size it with pkv_paged_attention_workspace_size).
+ */
+PKV_API int pkv_paged_attention_decode_fp8(void* out, int out_dtype, const void* query, const void* key_cache,
+                                           const void* value_cache, const float* k_scale, const float* v_scale,
+                                           const int32_t* block_tables, int max_blocks_per_seq,
+                                           const int32_t* context_lens, int max_context_len, int num_seqs,
+                                           int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                           int num_blocks, float scale, int partition_tokens, void* workspace,
+                                           size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
+
+/*
+ * swap_blocks — the pool's overflow path (intelliparadigm article §4.2 OOM错误:
+ * swap_space extends the cache into host memory).  For each (src, dst) pair of
+ * block_mapping, block dst of dst_pool <- block src of src_pool, block_bytes bytes,
+ * in one kernel launch.  One pool is normally device memory and the other pinned host
+ * memory (cudaHostAlloc / cudaHostRegister, mapped at the same address on the
+ * device); either may be device memory.  The two pools must not overlap.
+ *   src_pool, dst_pool  16-byte aligned, [src_blocks] / [dst_blocks] blocks of block_bytes
+ *   block_mapping       [num_pairs, 2] int64 in device or pinned host memory
+ *   block_bytes         a multiple of 16 (one layer's K or V block; call once per pool)
+ * A pair outside either pool sets PKV_DEV_BAD_PAIR and is skipped.  Memory that is
+ * neither device nor pinned-and-mapped is PKV_ERR_INVALID (checked on the host).
+ */
+PKV_API int pkv_swap_blocks(const void* src_pool, void* dst_pool, const int64_t* block_mapping, int num_pairs,
+                            int src_blocks, int dst_blocks, int64_t block_bytes, int32_t* status,
+                            pkv_stream_t stream);
+
+/*
+ * paged_attention_prefill — causal attention of a batch of prompt chunks over the
+ * paged pool (tensor cores).  Outcome School explainer, "LLM serving的基本流程与KV缓存"
+ * (prefill reads the whole prompt and stores every token's K/V) and intelliparadigm
+ * article §4.1/§4.2 (chunked prefill: a long prompt in pieces, e.g. 512 tokens).
+ *
+ * Sequence s holds context_lens[s] = L tokens in the pool, the last n = query_start[s+1]
+ * - query_start[s] of which are this call's new tokens (write them with
+ * pkv_reshape_and_cache first).  Row query_start[s] + i of `query` is the token at
+ * position p = L - n + i; for every query head h it gets
+ *   out[row, h] = softmax_j(scale * q·k_j) · v_j   over positions j = 0 .. p
+ * with K/V of kv head h / (num_heads / num_kv_heads), read through block_tables[s].
+ *   out          device [total_q, num_heads, 128], out_dtype BF16 or F32
+ *   query        device [total_q, num_heads, 128] bf16 (rows of all sequences packed)
+ *   key_cache, value_cache, block_tables, num_blocks, block_size: as for decode
+ *   query_start  device [num_seqs + 1] int32, non-decreasing, query_start[num_seqs] <= total_q
+ *   context_lens device [num_seqs] int32, n <= L <= min(max_context_len, max_blocks_per_seq*block_size)
+ *   workspace    device, pkv_paged_attention_prefill_workspace_size() bytes, 256-byte aligned
+ * head_dim must be 128 and num_heads / num_kv_heads must divide 128 (PKV_ERR_UNSUPPORTED).
+ * A sequence whose numbers break the rules above sets PKV_DEV_BAD_CONTEXT and its rows
+ * (when their range is valid) are written as zeros; a table entry outside the pool sets
+ * PKV_DEV_BAD_BLOCK and its 16-row slice of keys is skipped.  The pages leave the
+ * visibility rule open; the reading here is the causal one of a prompt: a token sees
+ * itself and every earlier token, never a later one.
+ */
+PKV_API size_t pkv_paged_attention_prefill_workspace_size(int num_seqs, int total_q, int num_heads,
+                                                          int num_kv_heads);
+PKV_API int pkv_paged_attention_prefill(void* out, int out_dtype, const void* query, const void* key_cache,
+                                        const void* value_cache, const int32_t* block_tables,
+                                        int max_blocks_per_seq, const int32_t* query_start,
+                                        const int32_t* context_lens, int num_seqs, int total_q,
+                                        int max_context_len, int num_heads, int num_kv_heads, int head_dim,
+                                        int block_size, int num_blocks, float scale, void* workspace,
+                                        size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
+
+/*
  * Host block manager — free list + reference counts + per-sequence block tables.
  * Outcome School explainer, "vLLM的核心创新：PagedAttention" (a block only when needed,
  * any free block serves any request, finished requests return all blocks at once)
@@ -257,6 +344,57 @@ PKV_API int pkv_bm_seq_blocks(const pkv_bm* bm, int64_t seq_id);   /* table leng
  */
 PKV_API int pkv_bm_export_tables(const pkv_bm* bm, const int64_t* seq_ids, int n, int32_t* tables,
                          int max_blocks, int32_t* context_lens);
+
+/*
+ * Swap space (intelliparadigm article §4.2 OOM错误: swap_space extends the pool into
+ * host memory).  A manager created with num_host_blocks > 0 also owns a pool of host
+ * block ids (FIFO free list, initial order 0..num_host_blocks-1, reference counts).
+ * pkv_bm_create(...) equals pkv_bm_create_with_swap_space(..., 0).
+ *
+ * swap_out moves the listed resident sequences to host blocks: every distinct device
+ * block among their tables (in order of first appearance, sequence by sequence, table
+ * order) gets one host block; the pair (device, host) goes to pairs_out; the table
+ * entry becomes the host block and the device block loses one reference (a block still
+ * used by a resident sequence stays on the device).  swap_in is the mirror image:
+ * pairs (host, device), fresh device blocks from the front of the free list.  Copy
+ * every pair with pkv_swap_blocks (every layer, K and V) before the freed blocks are
+ * written again.  Both calls are all-or-nothing: PKV_ERR_OOM if the destination pool
+ * lacks blocks, PKV_ERR_INVALID if pairs_out (host [cap, 2] int64) is too small.
+ * While swapped out, a sequence can only be swapped in or freed (free_seq releases its
+ * host blocks); append_slots, slots, fork and export_tables refuse it.
+ */
+PKV_API pkv_bm* pkv_bm_create_with_swap_space(int num_blocks, int block_size, const int32_t* initial_order,
+                                              int num_host_blocks);
+PKV_API int pkv_bm_num_host_free(const pkv_bm* bm);
+PKV_API int pkv_bm_host_refcount(const pkv_bm* bm, int32_t block);   /* >= 0, or PKV_ERR_INVALID */
+PKV_API int pkv_bm_is_swapped(const pkv_bm* bm, int64_t seq_id);     /* 1, 0, or PKV_ERR_INVALID */
+PKV_API int pkv_bm_swap_out(pkv_bm* bm, const int64_t* seq_ids, int n, int64_t* pairs_out, int cap,
+                            int* n_pairs_out);
+PKV_API int pkv_bm_swap_in(pkv_bm* bm, const int64_t* seq_ids, int n, int64_t* pairs_out, int cap,
+                           int* n_pairs_out);
+
+/*
+ * Automatic prefix caching (Outcome School explainer, "内存共享": requests with the same
+ * prefix keep one copy of its blocks; vLLM 初探 §1.4: a shared system prompt saves
+ * 30-50% of the memory).  A full block is identified by the chain hash
+ *   h_i = FNV-1a-64( h_(i-1) as 8 little-endian bytes || the block's token ids as
+ *                    4-byte little-endian integers ),  h_(-1) = 0
+ * (FNV-1a-64: start at 0xcbf29ce484222325; per byte xor, then multiply by
+ * 0x100000001b3 modulo 2^64).
+ *
+ * add_seq_tokens creates a sequence from its prompt token ids (host [num_tokens]
+ * int32).  It takes the longest run of leading blocks whose hashes are registered, but
+ * never the block holding the last token (at most (num_tokens-1)/block_size blocks);
+ * those gain a reference (a registered block with no references is taken back out of
+ * the free list).  The remaining blocks are fresh; each fresh full block registers its
+ * hash unless the hash is already registered.  *cached_tokens_out = tokens whose K/V
+ * are already in the pool; the caller computes and writes the rest.  All-or-nothing
+ * (PKV_ERR_OOM).  A registered block whose references drop to zero stays registered
+ * in the free list until the list hands it out again (eviction in free-list order).
+ */
+PKV_API int pkv_bm_add_seq_tokens(pkv_bm* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
+                                  int* cached_tokens_out);
+PKV_API int pkv_bm_num_cached_blocks(const pkv_bm* bm);
 
 #ifdef __cplusplus
 }

@@ -20,7 +20,9 @@ __all__ = [
     "PKV_DEV_BAD_SLOT", "PKV_DEV_BAD_BLOCK", "PKV_DEV_BAD_CONTEXT", "PKV_DEV_BAD_PAIR", "PKV_DEV_TIMEOUT",
     "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR", "PkvError", "library", "library_path",
     "reshape_and_cache", "copy_blocks", "paged_attention_workspace_size", "paged_attention_partition_tokens",
-    "paged_attention_decode", "paged_attention_decode_static", "STATIC_SCRATCH_BYTES", "BlockManager",
+    "paged_attention_decode", "paged_attention_decode_static", "STATIC_SCRATCH_BYTES",
+    "paged_attention_prefill_workspace_size", "paged_attention_prefill", "reshape_and_cache_fp8",
+    "paged_attention_decode_fp8", "swap_blocks", "BlockManager",
 ]
 
 PKV_OK = 0
@@ -70,7 +72,25 @@ _SIGNATURES = {
     "pkv_paged_attention_decode_static": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                                   c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                                   c_int, c_int, c_void_p, c_void_p]),
+    "pkv_paged_attention_prefill_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "pkv_paged_attention_prefill": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                            c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                            c_int, c_float, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "pkv_reshape_and_cache_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                          c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
+    "pkv_paged_attention_decode_fp8": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                               c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                               c_int, c_float, c_int, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "pkv_swap_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int64, c_void_p, c_void_p]),
     "pkv_bm_create": (c_void_p, [c_int, c_int, c_void_p]),
+    "pkv_bm_create_with_swap_space": (c_void_p, [c_int, c_int, c_void_p, c_int]),
+    "pkv_bm_num_host_free": (c_int, [c_void_p]),
+    "pkv_bm_host_refcount": (c_int, [c_void_p, ctypes.c_int32]),
+    "pkv_bm_is_swapped": (c_int, [c_void_p, c_int64]),
+    "pkv_bm_swap_out": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, ctypes.POINTER(c_int)]),
+    "pkv_bm_swap_in": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, ctypes.POINTER(c_int)]),
+    "pkv_bm_add_seq_tokens": (c_int, [c_void_p, c_int64, c_void_p, c_int, ctypes.POINTER(c_int)]),
+    "pkv_bm_num_cached_blocks": (c_int, [c_void_p]),
     "pkv_bm_destroy": (None, [c_void_p]),
     "pkv_bm_num_blocks": (c_int, [c_void_p]),
     "pkv_bm_block_size": (c_int, [c_void_p]),
@@ -261,6 +281,118 @@ def paged_attention_decode_static(out, query, key_cache, value_cache, block_tabl
     _check(rc, "paged_attention_decode_static")
 
 
+def reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale, status=None,
+                          stream=None):
+    """Quantising write of key/value [T, Hkv, D] bf16 into 8-bit pools [NB, Hkv, bs, D] uint8
+    (e4m3 codes) with per-kv-head float32 scales k_scale, v_scale [Hkv]."""
+    torch = _torch()
+    T, Hkv, D = key.shape
+    NB, Hkv2, bs, D2 = key_cache.shape
+    if value.shape != key.shape or value_cache.shape != key_cache.shape or (Hkv, D) != (Hkv2, D2):
+        raise ValueError("reshape_and_cache_fp8: shape mismatch")
+    if slot_mapping.shape != (T,) or tuple(k_scale.shape) != (Hkv,) or tuple(v_scale.shape) != (Hkv,):
+        raise ValueError("reshape_and_cache_fp8: slot_mapping must be [T], scales [Hkv]")
+    rc = library().pkv_reshape_and_cache_fp8(
+        _ptr(key, torch.bfloat16, "key"), _ptr(value, torch.bfloat16, "value"),
+        _ptr(key_cache, torch.uint8, "key_cache"), _ptr(value_cache, torch.uint8, "value_cache"),
+        _ptr(slot_mapping, torch.int64, "slot_mapping"), _ptr(k_scale, torch.float32, "k_scale"),
+        _ptr(v_scale, torch.float32, "v_scale"), T, NB, Hkv, D, bs, _ptr(status, torch.int32, "status"),
+        _stream(stream))
+    _check(rc, "reshape_and_cache_fp8")
+
+
+def paged_attention_decode_fp8(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, context_lens,
+                               max_context_len, scale, workspace, partition_tokens=0, status=None, stream=None):
+    """Decode attention over 8-bit pools [NB, Hkv, bs, 128] uint8 with per-kv-head scales;
+    otherwise as paged_attention_decode (same workspace size)."""
+    torch = _torch()
+    B, Hq, D = query.shape
+    NB, Hkv, bs, D2 = key_cache.shape
+    if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
+        raise ValueError("paged_attention_decode_fp8: shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("paged_attention_decode_fp8: block_tables must be [B, max_blocks], context_lens [B]")
+    out_dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(out.dtype)
+    if out_dtype is None:
+        raise TypeError("paged_attention_decode_fp8: out must be bf16 or f32")
+    rc = library().pkv_paged_attention_decode_fp8(
+        _ptr(out, None, "out"), out_dtype, _ptr(query, torch.bfloat16, "query"),
+        _ptr(key_cache, torch.uint8, "key_cache"), _ptr(value_cache, torch.uint8, "value_cache"),
+        _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
+        _ptr(block_tables, torch.int32, "block_tables"), int(block_tables.shape[1]),
+        _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len), B, Hq, Hkv, D, bs, NB,
+        float(scale), int(partition_tokens), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "paged_attention_decode_fp8")
+
+
+def _any_ptr(t, name):
+    """Pointer of a contiguous tensor in device memory or pinned host memory."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda and not t.is_pinned():
+        raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    return c_void_p(t.data_ptr())
+
+
+def swap_blocks(src_pool, dst_pool, block_mapping, status=None, stream=None):
+    """Copy blocks between pools [NB, ...] (device and/or pinned host, same block shape and
+    dtype): dst_pool[d] = src_pool[s] for every (s, d) of block_mapping [n, 2] int64 (device or
+    pinned host).  One kernel launch."""
+    torch = _torch()
+    if src_pool.dtype != dst_pool.dtype or src_pool.shape[1:] != dst_pool.shape[1:]:
+        raise ValueError("swap_blocks: pools must share dtype and block shape")
+    n = int(block_mapping.shape[0]) if block_mapping.numel() else 0
+    if block_mapping.numel() and (tuple(block_mapping.shape) != (n, 2) or block_mapping.dtype != torch.int64):
+        raise ValueError("swap_blocks: block_mapping must be [n, 2] int64")
+    if n == 0:
+        return
+    block_bytes = int(np.prod(src_pool.shape[1:])) * src_pool.element_size()
+    rc = library().pkv_swap_blocks(_any_ptr(src_pool, "src_pool"), _any_ptr(dst_pool, "dst_pool"),
+                                   _any_ptr(block_mapping, "block_mapping"), n, int(src_pool.shape[0]),
+                                   int(dst_pool.shape[0]), block_bytes, _ptr(status, torch.int32, "status"),
+                                   _stream(stream))
+    _check(rc, "swap_blocks")
+
+
+def paged_attention_prefill_workspace_size(num_seqs, total_q, num_heads, num_kv_heads) -> int:
+    n = library().pkv_paged_attention_prefill_workspace_size(num_seqs, total_q, num_heads, num_kv_heads)
+    if n == 0:
+        raise PkvError(PKV_ERR_INVALID, "paged_attention_prefill_workspace_size: bad arguments")
+    return int(n)
+
+
+def paged_attention_prefill(out, query, key_cache, value_cache, block_tables, query_start, context_lens,
+                            max_context_len, scale, workspace, status=None, stream=None):
+    """Causal prefill / chunked-prefill attention: out [T, Hq, 128] (bf16 or f32) from the
+    packed query rows [T, Hq, 128] bf16 of every sequence's new tokens.
+
+    query_start [B+1] int32 and context_lens [B] int32 (device), max_context_len a host
+    bound, workspace a uint8 device tensor of paged_attention_prefill_workspace_size bytes."""
+    torch = _torch()
+    T, Hq, D = query.shape
+    NB, Hkv, bs, D2 = key_cache.shape
+    B = int(context_lens.shape[0])
+    if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
+        raise ValueError("paged_attention_prefill: shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(query_start.shape) != (B + 1,):
+        raise ValueError("paged_attention_prefill: block_tables must be [B, max_blocks], query_start [B+1]")
+    out_dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(out.dtype)
+    if out_dtype is None:
+        raise TypeError("paged_attention_prefill: out must be bf16 or f32")
+    rc = library().pkv_paged_attention_prefill(
+        _ptr(out, None, "out"), out_dtype, _ptr(query, torch.bfloat16, "query"),
+        _ptr(key_cache, torch.bfloat16, "key_cache"), _ptr(value_cache, torch.bfloat16, "value_cache"),
+        _ptr(block_tables, torch.int32, "block_tables"), int(block_tables.shape[1]),
+        _ptr(query_start, torch.int32, "query_start"), _ptr(context_lens, torch.int32, "context_lens"), B, T,
+        int(max_context_len), Hq, Hkv, D, bs, NB, float(scale), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "paged_attention_prefill")
+
+
 # ---------------------------------------------------------------------------
 # Host block manager
 # ---------------------------------------------------------------------------
@@ -272,17 +404,19 @@ def _np_ptr(a):
 class BlockManager:
     """Free list + reference counts + per-sequence block tables (host, C++)."""
 
-    def __init__(self, num_blocks: int, block_size: int, initial_order=None):
+    def __init__(self, num_blocks: int, block_size: int, initial_order=None, num_host_blocks: int = 0):
         lib = library()
         order = None if initial_order is None else np.ascontiguousarray(initial_order, dtype=np.int32)
         if order is not None and order.shape != (num_blocks,):
             raise ValueError("initial_order must have num_blocks entries")
-        h = lib.pkv_bm_create(num_blocks, block_size, _np_ptr(order) if order is not None else None)
+        h = lib.pkv_bm_create_with_swap_space(num_blocks, block_size,
+                                              _np_ptr(order) if order is not None else None, num_host_blocks)
         if not h:
             raise PkvError(PKV_ERR_INVALID, lib.pkv_last_error_string().decode())
         self._h = c_void_p(h)
         self.num_blocks = num_blocks
         self.block_size = block_size
+        self.num_host_blocks = num_host_blocks
 
     def close(self):
         if getattr(self, "_h", None):
@@ -363,3 +497,48 @@ class BlockManager:
         _check(library().pkv_bm_export_tables(self._h, _np_ptr(ids), len(ids), _np_ptr(tables), max_blocks,
                                               _np_ptr(lens)), "bm_export_tables")
         return tables, lens
+
+    # -- swap space ---------------------------------------------------------------
+    def num_host_free(self) -> int:
+        return library().pkv_bm_num_host_free(self._h)
+
+    def host_refcount(self, block: int) -> int:
+        r = library().pkv_bm_host_refcount(self._h, block)
+        if r < 0:
+            _check(r, "bm_host_refcount")
+        return r
+
+    def is_swapped(self, seq_id: int) -> bool:
+        r = library().pkv_bm_is_swapped(self._h, seq_id)
+        if r < 0:
+            _check(r, "bm_is_swapped")
+        return bool(r)
+
+    def _swap(self, fn, seq_ids, what):
+        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        cap = max(self.num_blocks, self.num_host_blocks, 1)
+        pairs = np.zeros((cap, 2), np.int64)
+        n = c_int(0)
+        _check(fn(self._h, _np_ptr(ids), len(ids), _np_ptr(pairs), cap, ctypes.byref(n)), what)
+        return pairs[:n.value].copy()
+
+    def swap_out(self, seq_ids) -> np.ndarray:
+        """(device, host) block pairs to copy, [n, 2] int64."""
+        return self._swap(library().pkv_bm_swap_out, seq_ids, "bm_swap_out")
+
+    def swap_in(self, seq_ids) -> np.ndarray:
+        """(host, device) block pairs to copy, [n, 2] int64."""
+        return self._swap(library().pkv_bm_swap_in, seq_ids, "bm_swap_in")
+
+    # -- automatic prefix caching ---------------------------------------------------
+    def add_seq_tokens(self, seq_id: int, tokens) -> int:
+        """New sequence from its prompt token ids; returns the number of leading tokens
+        whose K/V are already in the pool (taken from cached blocks)."""
+        toks = np.ascontiguousarray(list(tokens), dtype=np.int32)
+        cached = c_int(0)
+        _check(library().pkv_bm_add_seq_tokens(self._h, seq_id, _np_ptr(toks), len(toks), ctypes.byref(cached)),
+               "bm_add_seq_tokens")
+        return cached.value
+
+    def num_cached_blocks(self) -> int:
+        return library().pkv_bm_num_cached_blocks(self._h)

@@ -6,6 +6,10 @@
 // intelliparadigm article §2.2: growth needs only a new page and a table update.
 // Both kernels are plain 16-byte vector copies: bit-exact, HBM-bound, and tiny next
 // to the attention read that follows them.
+//
+// Also here: the quantising write of an 8-bit (e4m3) pool (intelliparadigm article
+// §4.2/§5: low-bit storage), and swap_blocks, the pool's overflow path to pinned
+// host memory (§4.2 OOM错误: swap_space), as one kernel over every block pair.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -43,6 +47,84 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4* __r
     const int64_t dst = ((block * num_kv_heads + h) * block_size + r) * chunks_per_row + c;
     key_cache[dst] = key[i];
     value_cache[dst] = value[i];
+  }
+}
+
+// e4m3 quantisation of 16 values: x / scale, correctly rounded in fp32, then round
+// to nearest even into e4m3 with saturation to +-448.
+__device__ __forceinline__ uint32_t e4m3x4(float x0, float x1, float x2, float x3) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(x1), "f"(x0));  // first operand -> high byte
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(x3), "f"(x2));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+__device__ __forceinline__ uint4 quantize16(const uint4 a, const uint4 b, float s) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t r[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    r[i] = e4m3x4(__fdiv_rn(bf16lo(w[2 * i]), s), __fdiv_rn(bf16hi(w[2 * i]), s), __fdiv_rn(bf16lo(w[2 * i + 1]), s),
+                  __fdiv_rn(bf16hi(w[2 * i + 1]), s));
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// One thread writes one 16-byte chunk (16 codes) of one (token, kv head) row of K and V.
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
+    const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ key_cache,
+    uint4* __restrict__ value_cache, const int64_t* __restrict__ slot_mapping, const float* __restrict__ k_scale,
+    const float* __restrict__ v_scale, int64_t total_chunks, int chunks_per_row, int num_kv_heads, int block_size,
+    int64_t num_slots, int32_t* status) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks; i += stride) {
+    const int c = static_cast<int>(i % chunks_per_row);
+    const int64_t row = i / chunks_per_row;              // token * Hkv + head
+    const int h = static_cast<int>(row % num_kv_heads);
+    const int64_t t = row / num_kv_heads;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (c == 0 && h == 0) set_status(status, PKV_DEV_BAD_SLOT);
+      continue;
+    }
+    const int64_t block = slot / block_size;
+    const int64_t r = slot - block * block_size;
+    const int64_t dst = ((block * num_kv_heads + h) * block_size + r) * chunks_per_row + c;
+    key_cache[dst] = quantize16(key[2 * i], key[2 * i + 1], __ldg(k_scale + h));
+    value_cache[dst] = quantize16(value[2 * i], value[2 * i + 1], __ldg(v_scale + h));
+  }
+}
+
+// swap_blocks: grid-stride over (pair, 16-byte chunk); each thread keeps 4 loads in
+// flight before its stores, so reads across the host link overlap.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                          const int64_t* __restrict__ block_mapping, int num_pairs,
+                                                          int src_blocks, int dst_blocks, int64_t chunks_per_block,
+                                                          int32_t* status) {
+  const int64_t total = static_cast<int64_t>(num_pairs) * chunks_per_block;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  constexpr int kUnroll = 4;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
+       base += stride * kUnroll) {
+    uint4 v[kUnroll];
+    int64_t to[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      to[u] = -1;
+      const int64_t i = base + u * stride;
+      if (i >= total) continue;
+      const int64_t pair = i / chunks_per_block, c = i - pair * chunks_per_block;
+      const int64_t s = block_mapping[2 * pair], d = block_mapping[2 * pair + 1];
+      if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) {
+        if (c == 0) set_status(status, PKV_DEV_BAD_PAIR);
+        continue;
+      }
+      v[u] = src[s * chunks_per_block + c];
+      to[u] = d * chunks_per_block + c;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (to[u] >= 0) dst[to[u]] = v[u];
   }
 }
 
@@ -142,4 +224,70 @@ extern "C" int pkv_copy_blocks(void* const* key_caches, void* const* value_cache
     if (rc != PKV_OK) return rc;
   }
   return PKV_OK;
+}
+
+extern "C" int pkv_reshape_and_cache_fp8(const void* key, const void* value, void* key_cache, void* value_cache,
+                                         const int64_t* slot_mapping, const float* k_scale, const float* v_scale,
+                                         int num_tokens, int num_blocks, int num_kv_heads, int head_dim,
+                                         int block_size, int32_t* status, pkv_stream_t stream) {
+  clear_error();
+  if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0)
+    return set_error(PKV_ERR_INVALID, "reshape_and_cache_fp8: bad sizes");
+  if (head_dim != 64 && head_dim != 128)
+    return set_error(PKV_ERR_UNSUPPORTED, "reshape_and_cache_fp8: head_dim %d not in {64,128}", head_dim);
+  if (block_size != 16 && block_size != 32)
+    return set_error(PKV_ERR_UNSUPPORTED, "reshape_and_cache_fp8: block_size %d not in {16,32}", block_size);
+  if (num_tokens == 0) return PKV_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping || !k_scale || !v_scale)
+    return set_error(PKV_ERR_INVALID, "reshape_and_cache_fp8: null pointer");
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return set_error(PKV_ERR_INVALID, "reshape_and_cache_fp8: tensors must be 16-byte aligned");
+  const int chunks_per_row = head_dim / 16;
+  const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * chunks_per_row;
+  const int threads = 256;
+  const int64_t want = (total + threads - 1) / threads;
+  const int blocks = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8));
+  reshape_and_cache_fp8_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(key_cache),
+      static_cast<uint4*>(value_cache), slot_mapping, k_scale, v_scale, total, chunks_per_row, num_kv_heads,
+      block_size, static_cast<int64_t>(num_blocks) * block_size, status);
+  return check_launch("reshape_and_cache_fp8 launch");
+}
+
+extern "C" int pkv_swap_blocks(const void* src_pool, void* dst_pool, const int64_t* block_mapping, int num_pairs,
+                               int src_blocks, int dst_blocks, int64_t block_bytes, int32_t* status,
+                               pkv_stream_t stream) {
+  clear_error();
+  if (num_pairs < 0 || src_blocks <= 0 || dst_blocks <= 0 || block_bytes <= 0)
+    return set_error(PKV_ERR_INVALID, "swap_blocks: bad sizes");
+  if (block_bytes % 16 != 0) return set_error(PKV_ERR_INVALID, "swap_blocks: block bytes must be a multiple of 16");
+  if (num_pairs == 0) return PKV_OK;
+  if (!src_pool || !dst_pool || !block_mapping) return set_error(PKV_ERR_INVALID, "swap_blocks: null pointer");
+  if (!aligned16(src_pool) || !aligned16(dst_pool))
+    return set_error(PKV_ERR_INVALID, "swap_blocks: pools must be 16-byte aligned");
+  // Every pointer the kernel dereferences must be device memory or pinned host
+  // memory mapped into the device's address space.
+  const void* ptrs[3] = {src_pool, dst_pool, block_mapping};
+  const char* names[3] = {"src_pool", "dst_pool", "block_mapping"};
+  for (int i = 0; i < 3; ++i) {
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, ptrs[i]) != cudaSuccess) {
+      cudaGetLastError();
+      return set_error(PKV_ERR_INVALID, "swap_blocks: %s is not CUDA-visible memory", names[i]);
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeHost && attr.type != cudaMemoryTypeManaged)
+      return set_error(PKV_ERR_INVALID, "swap_blocks: %s must be device or pinned host memory", names[i]);
+    if (attr.type == cudaMemoryTypeHost && attr.devicePointer != ptrs[i])
+      return set_error(PKV_ERR_INVALID, "swap_blocks: pinned %s is not mapped at the same address on the device",
+                       names[i]);
+  }
+  const int64_t chunks = block_bytes / 16;
+  const int64_t total = chunks * num_pairs;
+  const int threads = 256;
+  const int64_t want = (total + threads * 4 - 1) / (threads * 4);
+  const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8)));
+  swap_blocks_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src_pool), static_cast<uint4*>(dst_pool), block_mapping, num_pairs, src_blocks,
+      dst_blocks, chunks, status);
+  return check_launch("swap_blocks launch");
 }

@@ -28,6 +28,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "decode_common.cuh"
 #include "pkv_internal.h"
@@ -42,6 +43,10 @@
 #endif
 #ifndef PKV_SIMT_DYNAMIC
 #define PKV_SIMT_DYNAMIC 1
+#endif
+// Ring stages per warp for an 8-bit pool (half the bytes per stage).
+#ifndef PKV_SIMT_STAGES8
+#define PKV_SIMT_STAGES8 4
 #endif
 
 namespace pkv {
@@ -133,12 +138,14 @@ __global__ void __launch_bounds__(kPlanThreads)
 // CUDA-core streaming kernel
 // ---------------------------------------------------------------------------
 
-template <int D, int STAGES>
+template <int D, int STAGES, bool KV8 = false>
 struct __align__(128) WarpRing {
-  __nv_bfloat16 k[STAGES][kStageTokens * D];
-  __nv_bfloat16 v[STAGES][kStageTokens * D];
+  using KvT = std::conditional_t<KV8, uint8_t, __nv_bfloat16>;  // bf16 or e4m3 pool elements
+  KvT k[STAGES][kStageTokens * D];
+  KvT v[STAGES][kStageTokens * D];
   __nv_bfloat16 q[STAGES][D];
   float2 p[kStageTokens];  // (p_t, p_t) of the stage being consumed, read back as packed pairs
+                           // (8-bit pool: p_t rounded to f16 in the low half of .x)
   uint64_t full[STAGES];
   int4 meta[STAGES];  // x seq, y query head, z part | nparts << 16, w n_valid | flags (first, last, q present)
 };
@@ -226,7 +233,7 @@ __device__ __forceinline__ void store_row(const DecodeArgs& a, int seq, int qh, 
 //        (k + i) mod NC, so the 8 lanes of each shared-memory phase always hit 8
 //        different 16-byte bank groups although every row starts at bank 0.
 //   P·V: lane l owns head_dim/32 consecutive output values of every row.
-template <int D>
+template <int D, bool KV8 = false>
 struct LaneMap {
   static constexpr int NC = D / 16;                  // 16-byte chunks per half row
   static constexpr int PARTNER = D == 128 ? 16 : 4;  // the lane holding the other half of the row
@@ -241,18 +248,76 @@ struct LaneMap {
   }
 };
 
-template <int D, bool OUT_F32, int WARPS, int STAGES>
+// 8-bit pool, head_dim 128: a K row is 128 bytes, a half row 64 bytes = 4 chunks.
+// The two halves of a row sit in adjacent lanes (row = lane / 2), so each group of 8
+// lanes covers 4 rows x both halves and, with the rotated chunk order, 8 different
+// 16-byte bank groups.
+template <>
+struct LaneMap<128, true> {
+  static constexpr int NC = 4;
+  static constexpr int PARTNER = 1;
+  __device__ static int row(int lane) { return lane >> 1; }
+  __device__ static int half(int lane) { return lane & 1; }
+  __device__ static float max_rows(float x) {
+    x = fmaxf(x, __shfl_xor_sync(kFull, x, 2));
+    x = fmaxf(x, __shfl_xor_sync(kFull, x, 4));
+    x = fmaxf(x, __shfl_xor_sync(kFull, x, 8));
+    return fmaxf(x, __shfl_xor_sync(kFull, x, 16));
+  }
+};
+
+// ---- e4m3 helpers (8-bit pool)
+// Two e4m3 codes (low byte first) -> f16x2, exactly (every e4m3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair16) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(r) : "r"(pair16));
+  return r;
+}
+// a0 += x.lo * y.lo, a1 += x.hi * y.hi with f16 operands and fp32 accumulation
+// (sm_100 mixed-precision FMA; the f16 x f16 product is exact in fp32).
+__device__ __forceinline__ void dot_f16x2(float& a0, float& a1, uint32_t x, uint32_t y) {
+  asm("{\n\t.reg .b16 xl, xh, yl, yh;\n\t"
+      "mov.b32 {xl, xh}, %2;\n\t"
+      "mov.b32 {yl, yh}, %3;\n\t"
+      "fma.rn.f32.f16 %0, xl, yl, %0;\n\t"
+      "fma.rn.f32.f16 %1, xh, yh, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(x), "r"(y));
+}
+// a += p * x.lo, b += p * x.hi (p an f16 in the low half of `p16`)
+__device__ __forceinline__ void axpy_f16x2(float& a, float& b, uint32_t p16, uint32_t x) {
+  asm("{\n\t.reg .b16 pl, ph, xl, xh;\n\t"
+      "mov.b32 {pl, ph}, %2;\n\t"
+      "mov.b32 {xl, xh}, %3;\n\t"
+      "fma.rn.f32.f16 %0, pl, xl, %0;\n\t"
+      "fma.rn.f32.f16 %1, pl, xh, %1;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "r"(p16), "r"(x));
+}
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float f16lo_to_f32(uint32_t w) {
+  float r;
+  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.f32.f16 %0, lo;\n\t}" : "=f"(r) : "r"(w));
+  return r;
+}
+
+template <int D, bool OUT_F32, int WARPS, int STAGES, bool KV8 = false>
 __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_constant__ DecodeArgs a) {
+  static_assert(!KV8 || D == 128, "the 8-bit pool path is head_dim 128");
   constexpr int EPL = D / 32;                                  // output values per lane: 2 or 4
   constexpr int NPAIR = EPL / 2;                               // packed fp32 pairs per lane
-  constexpr int NC = LaneMap<D>::NC;
-  constexpr uint32_t kKVBytes = kStageTokens * D * sizeof(__nv_bfloat16);
+  constexpr int NC = LaneMap<D, KV8>::NC;
+  using Ring = WarpRing<D, STAGES, KV8>;
+  constexpr uint32_t kKVBytes = kStageTokens * D * sizeof(typename Ring::KvT);
   constexpr uint32_t kQBytes = D * sizeof(__nv_bfloat16);
-  using Ring = WarpRing<D, STAGES>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Ring& ring = reinterpret_cast<Ring*>(smem_raw)[warp];
-  const int qk_row = LaneMap<D>::row(lane), qk_half = LaneMap<D>::half(lane);
+  const int qk_row = LaneMap<D, KV8>::row(lane), qk_half = LaneMap<D, KV8>::half(lane);
 
   const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_heads;
   // Work distribution over the plan (longest items first): every warp starts with
@@ -350,8 +415,13 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
                       &ring.full[slot], policy);
       if (ok) {
         const int64_t row = (static_cast<int64_t>(phys) * a.num_kv_heads + kvh) * a.block_size + local_tok % a.block_size;
-        bulk_copy_g2s(ring.k[slot], a.key_cache + row * D, kKVBytes, &ring.full[slot], policy);
-        bulk_copy_g2s(ring.v[slot], a.value_cache + row * D, kKVBytes, &ring.full[slot], policy);
+        if constexpr (KV8) {
+          bulk_copy_g2s(ring.k[slot], a.key_cache8 + row * D, kKVBytes, &ring.full[slot], policy);
+          bulk_copy_g2s(ring.v[slot], a.value_cache8 + row * D, kKVBytes, &ring.full[slot], policy);
+        } else {
+          bulk_copy_g2s(ring.k[slot], a.key_cache + row * D, kKVBytes, &ring.full[slot], policy);
+          bulk_copy_g2s(ring.v[slot], a.value_cache + row * D, kKVBytes, &ring.full[slot], policy);
+        }
       }
     }
     ++cur_stage;
@@ -359,11 +429,18 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   };
 
   // ---- consuming side
-  uint4 qv[NC];                 // this lane's half of q (raw bf16 pairs), chunks in rotated order
+  // this lane's half of q in rotated chunk order: raw bf16 pairs, or (8-bit pool)
+  // f16 pairs, two uint4 per 16-code chunk
+  constexpr int NQ = KV8 ? 2 * NC : NC;
+  uint4 qv[NQ];
   uint64_t o[NPAIR];            // packed fp32 output accumulators
+  float o8[KV8 ? EPL : 1];      // 8-bit pool: scalar fp32 accumulators
+  float score_scale = a.scale_log2, out_scale = 1.f;
   float m = -INFINITY, lsum = 0.f;
 #pragma unroll
-  for (int i = 0; i < NC; ++i) qv[i] = make_uint4(0, 0, 0, 0);
+  for (int i = 0; i < NQ; ++i) qv[i] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int j = 0; j < (KV8 ? EPL : 1); ++j) o8[j] = 0.f;
 #pragma unroll
   for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
 
@@ -388,37 +465,109 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       lsum = 0.f;
 #pragma unroll
       for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
-      if (mt.w & 0x400) {
+      if constexpr (KV8) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) o8[j] = 0.f;
+        if (mt.w & 0x400) {
+          // q to f16 for the mixed-precision products.  bf16 values of magnitude
+          // >= 2^15 would overflow f16: then the whole vector is scaled by 2^-16
+          // (and the score scale by 2^16).
+          const uint4* qs = reinterpret_cast<const uint4*>(ring.q[slot]);
+          bool big = false;
+#pragma unroll
+          for (int i = 0; i < NC; ++i) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint4 w = qs[qk_half * 2 * NC + 2 * ((i + qk_row) & (NC - 1)) + h];
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                big |= fabsf(bf16lo(ws[c])) >= 32768.f || fabsf(bf16hi(ws[c])) >= 32768.f;
+            }
+          }
+          const float qscale = __any_sync(kFull, big) ? 1.f / 65536.f : 1.f;
+#pragma unroll
+          for (int i = 0; i < NC; ++i) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint4 w = qs[qk_half * 2 * NC + 2 * ((i + qk_row) & (NC - 1)) + h];
+              qv[2 * i + h] = make_uint4(f32x2_to_f16x2(bf16lo(w.x) * qscale, bf16hi(w.x) * qscale),
+                                         f32x2_to_f16x2(bf16lo(w.y) * qscale, bf16hi(w.y) * qscale),
+                                         f32x2_to_f16x2(bf16lo(w.z) * qscale, bf16hi(w.z) * qscale),
+                                         f32x2_to_f16x2(bf16lo(w.w) * qscale, bf16hi(w.w) * qscale));
+            }
+          }
+          const int kvh = mt.y / a.group;
+          score_scale = a.scale_log2 * __ldg(a.k_scale + kvh) / qscale;
+          out_scale = __ldg(a.v_scale + kvh);
+        }
+      } else if (mt.w & 0x400) {
         const uint4* qs = reinterpret_cast<const uint4*>(ring.q[slot]);
 #pragma unroll
         for (int i = 0; i < NC; ++i) qv[i] = qs[qk_half * NC + ((i + qk_row) & (NC - 1))];
       }
     }
     if (n_valid > 0) {
-      // ---- scores: two lanes per row, bf16 x bf16 products accumulated in fp32
+      // ---- scores: two lanes per row, bf16 x bf16 (or f16 x e4m3) products accumulated in fp32
       const uint4* krow = reinterpret_cast<const uint4*>(ring.k[slot] + qk_row * D) + qk_half * NC;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
       for (int i = 0; i < NC; ++i) {
         const uint4 kw = krow[(i + qk_row) & (NC - 1)];
-        dot_bf16x2(a0, a1, qv[i].x, kw.x);
-        dot_bf16x2(a2, a3, qv[i].y, kw.y);
-        dot_bf16x2(a0, a1, qv[i].z, kw.z);
-        dot_bf16x2(a2, a3, qv[i].w, kw.w);
+        if constexpr (KV8) {
+          const uint32_t kws[4] = {kw.x, kw.y, kw.z, kw.w};
+          const uint4 q0 = qv[2 * i], q1 = qv[2 * i + 1];
+          const uint32_t qs[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            dot_f16x2(a0, a1, qs[2 * c], e4m3x2_to_f16x2(kws[c] & 0xffffu));
+            dot_f16x2(a2, a3, qs[2 * c + 1], e4m3x2_to_f16x2(kws[c] >> 16));
+          }
+        } else {
+          dot_bf16x2(a0, a1, qv[i].x, kw.x);
+          dot_bf16x2(a2, a3, qv[i].y, kw.y);
+          dot_bf16x2(a0, a1, qv[i].z, kw.z);
+          dot_bf16x2(a2, a3, qv[i].w, kw.w);
+        }
       }
       float sc = (a0 + a1) + (a2 + a3);
-      sc += __shfl_xor_sync(kFull, sc, LaneMap<D>::PARTNER);
+      sc += __shfl_xor_sync(kFull, sc, LaneMap<D, KV8>::PARTNER);
       // ---- online softmax in base 2 over the stage's rows
       const bool valid = qk_row < n_valid;
-      const float x = valid ? sc * a.scale_log2 : -INFINITY;
-      const float m_new = fmaxf(m, LaneMap<D>::max_rows(x));
+      const float x = valid ? sc * score_scale : -INFINITY;
+      const float m_new = fmaxf(m, LaneMap<D, KV8>::max_rows(x));
       const float alpha = exp2f(m - m_new);
-      const float p = valid ? exp2f(x - m_new) : 0.f;
+      float p = valid ? exp2f(x - m_new) : 0.f;
+      uint32_t p16 = 0;
+      if constexpr (KV8) {
+        // the weight the P·V products use: p rounded to f16; the sum adds the same value
+        p16 = f32x2_to_f16x2(p, 0.f);
+        p = f16lo_to_f32(p16);
+      }
       m = m_new;
       lsum = fmaf(lsum, alpha, p);
-      if (qk_half == 0) ring.p[qk_row] = make_float2(p, p);
+      if (qk_half == 0) {
+        if constexpr (KV8)
+          ring.p[qk_row] = make_float2(__uint_as_float(p16), 0.f);
+        else
+          ring.p[qk_row] = make_float2(p, p);
+      }
       __syncwarp();
       // ---- P·V: packed fp32 pairs, rows past n_valid never touched (stale rows may be NaN)
+      if constexpr (KV8) {
+        // ---- P·V over e4m3 rows: lane l owns values 4l..4l+3; f16 x f16 products, fp32 sums
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) o8[j] *= alpha;
+        const uint8_t* vb = ring.v[slot] + lane * EPL;
+        const float2* pr = ring.p;
+#pragma unroll 4
+        for (int t = 0; t < n_valid; ++t) {
+          const uint32_t pw = __float_as_uint(pr[t].x);
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(vb + t * D);
+          axpy_f16x2(o8[0], o8[1], pw, e4m3x2_to_f16x2(w & 0xffffu));
+          axpy_f16x2(o8[2], o8[3], pw, e4m3x2_to_f16x2(w >> 16));
+        }
+      } else {
       const uint64_t alpha2 = f2pack(alpha, alpha);
 #pragma unroll
       for (int j = 0; j < NPAIR; ++j) o[j] = fmul2(o[j], alpha2);
@@ -451,15 +600,21 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
           }
         }
       }
+      }  // bf16 P·V
     }
     if (last) {
       const int seq = mt.x, qh = mt.y, part = mt.z & 0xffff, nparts = mt.z >> 16;
       float of[EPL];
+      if constexpr (KV8) {
 #pragma unroll
-      for (int j = 0; j < NPAIR; ++j) {
-        const float2 f = f2unpack(o[j]);
-        of[2 * j] = f.x;
-        of[2 * j + 1] = f.y;
+        for (int j = 0; j < EPL; ++j) of[j] = o8[j] * out_scale;  // the value scale of the kv head
+      } else {
+#pragma unroll
+        for (int j = 0; j < NPAIR; ++j) {
+          const float2 f = f2unpack(o[j]);
+          of[2 * j] = f.x;
+          of[2 * j + 1] = f.y;
+        }
       }
       float l = lsum;
 #pragma unroll
@@ -519,11 +674,13 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
 
 constexpr int kSimtWarps = PKV_SIMT_WARPS;
 constexpr int kSimtStages = PKV_SIMT_STAGES;
+constexpr int kSimtStages8 = PKV_SIMT_STAGES8;
 
-template <int D, bool OUT_F32>
+template <int D, bool OUT_F32, bool KV8 = false>
 static int launch_simt(const DecodeArgs& a, cudaStream_t stream) {
-  auto kernel = decode_simt_kernel<D, OUT_F32, kSimtWarps, kSimtStages>;
-  const size_t smem = sizeof(WarpRing<D, kSimtStages>) * kSimtWarps;
+  constexpr int stages = KV8 ? kSimtStages8 : kSimtStages;
+  auto kernel = decode_simt_kernel<D, OUT_F32, kSimtWarps, stages, KV8>;
+  const size_t smem = sizeof(WarpRing<D, stages, KV8>) * kSimtWarps;
   static std::once_flag once;
   static int blocks_per_sm = 0;
   static cudaError_t setup_err = cudaSuccess;
@@ -596,14 +753,15 @@ extern "C" size_t pkv_paged_attention_workspace_size(int num_seqs, int num_heads
   return workspace_layout(num_seqs, num_heads, head_dim, max_context_len, p).total;
 }
 
-extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* query, const void* key_cache,
-                                          const void* value_cache, const int32_t* block_tables,
-                                          int max_blocks_per_seq, const int32_t* context_lens,
-                                          int max_context_len, int num_seqs, int num_heads, int num_kv_heads,
-                                          int head_dim, int block_size, int num_blocks, float scale,
-                                          int partition_tokens, int path, void* workspace, size_t workspace_bytes,
-                                          int32_t* status, pkv_stream_t stream) {
-  clear_error();
+// Shared by the bf16 and the 8-bit entry points; `k_scale` != null selects the
+// 8-bit (e4m3) pool, which the CUDA-core kernel reads at head_dim 128.
+static int decode_impl(void* out, int out_dtype, const void* query, const void* key_cache, const void* value_cache,
+                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                       int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
+                       int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                       int partition_tokens, int path, void* workspace, size_t workspace_bytes, int32_t* status,
+                       pkv_stream_t stream) {
+  const bool kv8 = k_scale != nullptr;
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: bad sizes");
@@ -619,6 +777,11 @@ extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* 
                      num_heads, num_kv_heads);
   if (path != PKV_PATH_AUTO && path != PKV_PATH_SIMT && path != PKV_PATH_TENSOR)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: path %d", path);
+  if (kv8 && head_dim != 128)
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_fp8: head_dim %d (only 128)", head_dim);
+  if (kv8 && path == PKV_PATH_TENSOR)
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_fp8: the 8-bit pool is read on CUDA cores");
+  if (kv8) path = PKV_PATH_SIMT;
   const int group = num_heads / num_kv_heads;
   if (path == PKV_PATH_TENSOR && !tensor_path_supports(group, head_dim))
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: tensor path needs 2 <= group <= 16 and head_dim 128"
@@ -635,7 +798,8 @@ extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* 
   if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(65535) * partition)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: max_context_len too large for the split");
   if (num_seqs == 0) return PKV_OK;
-  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !workspace)
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !workspace ||
+      (kv8 && !v_scale))
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: null pointer");
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: tensors must be 16-byte aligned");
@@ -652,8 +816,15 @@ extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* 
   DecodeArgs a{};
   a.out = out;
   a.query = static_cast<const __nv_bfloat16*>(query);
-  a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
-  a.value_cache = static_cast<const __nv_bfloat16*>(value_cache);
+  if (kv8) {
+    a.key_cache8 = static_cast<const uint8_t*>(key_cache);
+    a.value_cache8 = static_cast<const uint8_t*>(value_cache);
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+  } else {
+    a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
+    a.value_cache = static_cast<const __nv_bfloat16*>(value_cache);
+  }
   a.block_tables = block_tables;
   a.plan_count = reinterpret_cast<const int32_t*>(ws + w.off_count);
   a.entries = reinterpret_cast<const PlanEntry*>(ws + w.off_entries);
@@ -678,7 +849,37 @@ extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* 
   int rc = launch_plan(a, context_lens, max_context_len, s);
   if (rc != PKV_OK) return rc;
   const bool out_f32 = out_dtype == PKV_DTYPE_F32;
+  if (kv8) return out_f32 ? launch_simt<128, true, true>(a, s) : launch_simt<128, false, true>(a, s);
   if (use_tensor) return launch_decode_tensor(a, head_dim, out_f32, s);
   if (head_dim == 128) return out_f32 ? launch_simt<128, true>(a, s) : launch_simt<128, false>(a, s);
   return out_f32 ? launch_simt<64, true>(a, s) : launch_simt<64, false>(a, s);
+}
+
+extern "C" int pkv_paged_attention_decode(void* out, int out_dtype, const void* query, const void* key_cache,
+                                          const void* value_cache, const int32_t* block_tables,
+                                          int max_blocks_per_seq, const int32_t* context_lens,
+                                          int max_context_len, int num_seqs, int num_heads, int num_kv_heads,
+                                          int head_dim, int block_size, int num_blocks, float scale,
+                                          int partition_tokens, int path, void* workspace, size_t workspace_bytes,
+                                          int32_t* status, pkv_stream_t stream) {
+  clear_error();
+  return decode_impl(out, out_dtype, query, key_cache, value_cache, nullptr, nullptr, block_tables,
+                     max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads, num_kv_heads, head_dim,
+                     block_size, num_blocks, scale, partition_tokens, path, workspace, workspace_bytes, status,
+                     stream);
+}
+
+extern "C" int pkv_paged_attention_decode_fp8(void* out, int out_dtype, const void* query, const void* key_cache,
+                                              const void* value_cache, const float* k_scale, const float* v_scale,
+                                              const int32_t* block_tables, int max_blocks_per_seq,
+                                              const int32_t* context_lens, int max_context_len, int num_seqs,
+                                              int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                              int num_blocks, float scale, int partition_tokens, void* workspace,
+                                              size_t workspace_bytes, int32_t* status, pkv_stream_t stream) {
+  clear_error();
+  if (!k_scale) return set_error(PKV_ERR_INVALID, "paged_attention_decode_fp8: null k_scale");
+  return decode_impl(out, out_dtype, query, key_cache, value_cache, k_scale, v_scale, block_tables,
+                     max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads, num_kv_heads, head_dim,
+                     block_size, num_blocks, scale, partition_tokens, PKV_PATH_SIMT, workspace, workspace_bytes,
+                     status, stream);
 }

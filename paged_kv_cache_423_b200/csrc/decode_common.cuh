@@ -26,6 +26,10 @@ struct DecodeArgs {
   const __nv_bfloat16* query;
   const __nv_bfloat16* key_cache;
   const __nv_bfloat16* value_cache;
+  const uint8_t* key_cache8;   // 8-bit (e4m3) pools of the fp8 entry point, else null
+  const uint8_t* value_cache8;
+  const float* k_scale;        // [num_kv_heads] scales of the 8-bit pools
+  const float* v_scale;
   const int32_t* block_tables;
   const int32_t* plan_count;   // [0] number of plan entries, [1] work-item counter (both set by the plan kernel)
   const PlanEntry* entries;    // sorted plan

@@ -74,6 +74,46 @@ def test_argument_errors_before_any_device_work(pkv):
     assert lib.pkv_copy_blocks(None, None, 1, None, 3, 8, 4095, None, None) == pkv.PKV_ERR_INVALID
 
 
+def test_prefill_argument_errors_before_any_device_work(pkv):
+    lib = pkv.library()
+    fake = ctypes.c_void_p(0x1000)
+    args = dict(out=fake, out_dtype=0, query=fake, kc=fake, vc=fake, tables=fake, max_blocks=4, qstart=fake,
+                lens=fake, B=2, T=10, max_ctx=64, Hq=8, Hkv=2, D=128, bs=16, NB=8, scale=0.1, ws=fake,
+                ws_bytes=1 << 20)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.pkv_paged_attention_prefill(a["out"], a["out_dtype"], a["query"], a["kc"], a["vc"], a["tables"],
+                                               a["max_blocks"], a["qstart"], a["lens"], a["B"], a["T"],
+                                               a["max_ctx"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"],
+                                               a["scale"], a["ws"], a["ws_bytes"], None, None)
+    assert call(D=64) == pkv.PKV_ERR_UNSUPPORTED          # the tensor-core prefill is head_dim 128
+    assert call(bs=8) == pkv.PKV_ERR_UNSUPPORTED
+    assert call(Hq=6, Hkv=2) == pkv.PKV_ERR_UNSUPPORTED   # group 3 does not divide 128
+    assert call(Hq=7) == pkv.PKV_ERR_UNSUPPORTED
+    assert call(out_dtype=3) == pkv.PKV_ERR_INVALID
+    assert call(T=-1) == pkv.PKV_ERR_INVALID
+    assert call(query=ctypes.c_void_p(0x1004)) == pkv.PKV_ERR_INVALID
+    assert call(ws=ctypes.c_void_p(0x1080)) == pkv.PKV_ERR_INVALID
+    assert call(ws_bytes=64) == pkv.PKV_ERR_INVALID
+    assert b"workspace" in lib.pkv_last_error_string()
+    assert call(qstart=None) == pkv.PKV_ERR_INVALID
+    assert call(T=0) == pkv.PKV_OK                        # no rows: nothing to do
+    assert call(B=0) == pkv.PKV_OK
+
+
+def test_prefill_workspace_size(pkv):
+    # 256 bytes of counters + one 16-byte entry per query tile (upper bound: T / (128 / g) + B),
+    # rounded up to 256 bytes
+    def up(x):
+        return -(-x // 256) * 256
+    assert pkv.paged_attention_prefill_workspace_size(8, 4096, 40, 40) == 256 + up(16 * (32 + 8))
+    assert pkv.paged_attention_prefill_workspace_size(8, 4096, 64, 8) == 256 + up(16 * (256 + 8))
+    assert pkv.paged_attention_prefill_workspace_size(1, 1, 128, 1) == 256 + up(16 * 2)
+    with pytest.raises(pkv.PkvError):
+        pkv.paged_attention_prefill_workspace_size(2, 10, 6, 2)
+
+
 def test_workspace_size_and_partition_choice(pkv):
     assert pkv.paged_attention_partition_tokens(256, 40, 16, 2000) == 512
     assert pkv.paged_attention_partition_tokens(4, 2, 16, 33) == 64
@@ -95,7 +135,13 @@ def same_state(cpp, model: BlockManagerModel):
     assert cpp.free_list() == list(model.free)
     for b in range(model.num_blocks):
         assert cpp.refcount(b) == model.ref[b]
-    ids = sorted(model.tables)
+    assert cpp.num_host_free() == model.num_host_free()
+    for b in range(len(model.host_ref)):
+        assert cpp.host_refcount(b) == model.host_ref[b]
+    assert cpp.num_cached_blocks() == model.num_cached_blocks()
+    for s in model.tables:
+        assert cpp.is_swapped(s) == model.is_swapped(s)
+    ids = sorted(s for s in model.tables if not model.is_swapped(s))
     if ids:
         mb = max(len(t) for t in model.tables.values()) or 1
         tables, lens = cpp.export_tables(ids, mb)
@@ -120,17 +166,46 @@ def run_both(op, cpp, model, pkv):
 
 
 @pytest.mark.parametrize("seed", range(5))
-def test_block_manager_matches_model(pkv, seed):
+@pytest.mark.parametrize("extended", [False, True], ids=["base", "swap_and_prefix_cache"])
+def test_block_manager_matches_model(pkv, seed, extended):
     rng = wl.rng_for(100 + seed)
     nb, bs = 40, 4
     order = rng.permutation(nb).astype(np.int32)
-    cpp = pkv.BlockManager(nb, bs, order)
-    model = BlockManagerModel(nb, bs, order)
+    hb = 20 if extended else 0
+    cpp = pkv.BlockManager(nb, bs, order, num_host_blocks=hb)
+    model = BlockManagerModel(nb, bs, order, num_host_blocks=hb)
+    prompts = [list(rng.integers(0, 4, size=30)) for _ in range(3)]
     next_id = 0
     for _ in range(300):
-        live = sorted(model.tables)
-        op = int(rng.integers(0, 6))
-        if op == 0 or not live:
+        every = sorted(model.tables)
+        live = [x for x in every if not model.is_swapped(x)]
+        gone = [x for x in every if model.is_swapped(x)]
+        op = int(rng.integers(0, 9 if extended else 6))
+        if op >= 6:
+            # swap out / swap in (sometimes of a sequence in the wrong pool) / prompt admission
+            if op == 6 and every:
+                pick = [int(x) for x in rng.permutation(every)[:int(rng.integers(1, min(3, len(every)) + 1))]]
+                rm, rc = run_both(lambda m: m.swap_out(pick), cpp, model, pkv)
+                if rm is not None:
+                    assert [tuple(p) for p in rc.tolist()] == rm
+            elif op == 7 and every:
+                pick = [int(x) for x in rng.permutation(gone if gone and rng.random() < 0.8 else every)
+                        [:int(rng.integers(1, 3))]]
+                rm, rc = run_both(lambda m: m.swap_in(pick), cpp, model, pkv)
+                if rm is not None:
+                    assert [tuple(p) for p in rc.tolist()] == rm
+            else:
+                p = prompts[int(rng.integers(len(prompts)))]
+                toks = p[:int(rng.integers(1, len(p) + 1))] + [int(t) for t in rng.integers(0, 4, size=int(rng.integers(0, 3)))]
+                sid = next_id
+                next_id += 1
+                rm, rc = run_both(lambda m: m.add_seq_tokens(sid, toks), cpp, model, pkv)
+                assert rm == rc
+            same_state(cpp, model)
+            continue
+        if not live:
+            op = 0
+        if op == 0:
             shared = []
             if live and rng.random() < 0.5:
                 donor = live[int(rng.integers(len(live)))]
@@ -151,7 +226,7 @@ def test_block_manager_matches_model(pkv, seed):
             if sm is not None:
                 assert list(sc) == sm and [tuple(p) for p in pc.tolist()] == pm
         elif op == 3:
-            victim = live[int(rng.integers(len(live)))]
+            victim = every[int(rng.integers(len(every)))]
             run_both(lambda m: m.free_seq(victim), cpp, model, pkv)
         elif op == 4:
             s = live[int(rng.integers(len(live)))]
@@ -190,3 +265,25 @@ def test_block_manager_cow_example(pkv):
     assert slots.tolist() == [10, 14, 18, 6]
     tables, lens = bm.export_tables([0, 1, 2, 3], 2)
     assert tables.tolist() == [[0, 2], [0, 3], [0, 4], [0, 1]] and lens.tolist() == [7] * 4
+
+
+def test_block_manager_swap_and_prefix_examples(pkv):
+    """The hand-worked allocator cases of the oracle, through the C++ manager."""
+    bm = pkv.BlockManager(8, 4, list(range(8)), num_host_blocks=4)
+    bm.add_seq(0, 6)
+    bm.fork(0, 1)
+    bm.add_seq(2, 3)
+    assert bm.swap_out([0, 1]).tolist() == [[0, 0], [1, 1]]
+    assert bm.host_refcount(0) == 2 and bm.free_list() == [3, 4, 5, 6, 7, 0, 1]
+    with pytest.raises(pkv.PkvError) as e:
+        bm.append_slots([0])
+    assert e.value.code == pkv.PKV_ERR_INVALID
+    assert bm.swap_in([1, 0]).tolist() == [[0, 3], [1, 4]]
+    assert bm.refcount(3) == 2 and bm.num_host_free() == 4
+    pc = pkv.BlockManager(8, 4, list(range(8)))
+    p = list(range(12))
+    assert pc.add_seq_tokens(0, p + [99]) == 0 and pc.num_cached_blocks() == 3
+    pc.free_seq(0)
+    assert pc.add_seq_tokens(1, p + [98]) == 12
+    tables, _ = pc.export_tables([1], 4)
+    assert tables.tolist() == [[0, 1, 2, 4]] and pc.free_list() == [5, 6, 7, 3]

@@ -51,3 +51,16 @@ def test_aggregate_over_two_gloo_ranks():
 
 def test_single_process_aggregation_is_identity():
     assert bench.aggregate_over_ranks(3.5, 7) == (3.5, 7)
+
+
+def test_prefill_flops_counts_every_visible_key():
+    """4 * D FLOPs per (query row, head, visible key): the closed form against a
+    brute-force count of the causal window of every row."""
+    import bench
+    qlens = np.array([3, 0, 7, 1])
+    lens = np.array([10, 4, 7, 1])
+    brute = 0
+    for n, L in zip(qlens, lens):
+        for i in range(n):
+            brute += (L - n + i) + 1
+    assert bench.prefill_flops(qlens, lens, 5, 128) == 4 * 128 * 5 * brute

@@ -217,3 +217,102 @@ def test_continuous_batching_trace(pkv):
                 admit(length, budget)
     pool.check()
     assert next_id > len(initial)           # the trace admitted new requests
+
+
+def test_preempt_by_swap_then_resume(pkv):
+    """Sequences swapped out to pinned host blocks (intelliparadigm article §4.2:
+    swap_space), their device blocks reused by new requests, then swapped back in:
+    tables, pools and attention still match the oracle."""
+    from oracle import cache_ops as co
+    rng = wl.rng_for(900)
+    Hq, Hkv, D, bs, nb, hb = 16, 4, 128, 16, 160, 96
+    order = rng.permutation(nb).astype(np.int32)
+    cpp = pkv.BlockManager(nb, bs, order, num_host_blocks=hb)
+    model = BlockManagerModel(nb, bs, order, num_host_blocks=hb)
+    ls = Lockstep.__new__(Lockstep)
+    ls.cpp, ls.ref, ls.bs = cpp, model, bs
+    pool = Pool(pkv, rng, nb, Hkv, bs, D)
+    host_k = np.zeros((hb, Hkv, bs, D), np.uint16)
+    host_v = np.zeros((hb, Hkv, bs, D), np.uint16)
+    hk = torch.zeros((hb, Hkv, bs, D), dtype=torch.bfloat16).pin_memory()
+    hv = torch.zeros((hb, Hkv, bs, D), dtype=torch.bfloat16).pin_memory()
+    lens = rng.integers(40, 300, size=6)
+    for s, L in enumerate(lens):
+        ls.add_seq(s, int(L))
+        slots = ls.slots(s, 0, int(L))
+        k, v = wl.new_tokens(rng, len(slots), Hkv, D)
+        pool.write(k, v, slots)
+    ids = list(range(6))
+    cpp.fork(2, 10)
+    model.fork(2, 10)
+    ids.append(10)
+    max_blocks = 40
+    tables, clens = ls.tables(ids, max_blocks)
+    decode_and_compare(pkv, pool, wl.bf16_normal(rng, (len(ids), Hq, D)), tables, clens, wl.fp32_scale(D), Hq)
+
+    # preempt 1, 2 and its fork 10 (they share blocks): one host copy of each block
+    out_ids = [1, 2, 10]
+    pairs = cpp.swap_out(out_ids)
+    assert [tuple(p) for p in pairs.tolist()] == model.swap_out(out_ids)
+    dp = torch.from_numpy(pairs).cuda()
+    pkv.swap_blocks(pool.dk, hk, dp)
+    pkv.swap_blocks(pool.dv, hv, dp)
+    host_k = co.swap_blocks(pool.k, host_k, pairs)
+    host_v = co.swap_blocks(pool.v, host_v, pairs)
+    torch.cuda.synchronize()
+    assert np.array_equal(hk.view(torch.int16).numpy().view(np.uint16), host_k)
+    # new requests take the freed device blocks and overwrite them
+    for s in (20, 21):
+        L = int(rng.integers(200, 400))
+        ls.add_seq(s, L)
+        slots = ls.slots(s, 0, L)
+        k, v = wl.new_tokens(rng, len(slots), Hkv, D)
+        pool.write(k, v, slots)
+    ls.free_seq(20)
+    # resume
+    pairs = cpp.swap_in(out_ids)
+    assert [tuple(p) for p in pairs.tolist()] == model.swap_in(out_ids)
+    dp = torch.from_numpy(pairs).cuda()
+    pkv.swap_blocks(hk, pool.dk, dp)
+    pkv.swap_blocks(hv, pool.dv, dp)
+    pool.k = co.swap_blocks(host_k, pool.k, pairs)
+    pool.v = co.swap_blocks(host_v, pool.v, pairs)
+    pool.check()
+    ids = [0, 1, 2, 3, 4, 5, 10, 21]
+    slots, pairs = ls.append(ids)
+    pool.copy(pairs)
+    k, v = wl.new_tokens(rng, len(ids), Hkv, D)
+    pool.write(k, v, slots)
+    tables, clens = ls.tables(ids, max_blocks)
+    decode_and_compare(pkv, pool, wl.bf16_normal(rng, (len(ids), Hq, D)), tables, clens, wl.fp32_scale(D), Hq)
+
+
+def test_prefix_cached_admission(pkv):
+    """Requests sharing a long system prompt (Outcome School explainer, "内存共享"):
+    the second and later requests take the prompt's full blocks from the prefix cache,
+    only their uncached tokens are written, and attention matches the oracle."""
+    rng = wl.rng_for(910)
+    Hq, Hkv, D, bs, nb = 32, 8, 128, 16, 400
+    order = rng.permutation(nb).astype(np.int32)
+    ls = Lockstep(pkv, nb, bs, order)
+    pool = Pool(pkv, rng, nb, Hkv, bs, D)
+    prompt = [int(t) for t in rng.integers(0, 32000, size=203)]           # 12 full blocks + 11
+    pk, pv = wl.new_tokens(rng, len(prompt), Hkv, D)                      # its K/V, one copy
+    ids = []
+    for r in range(5):
+        tail = [int(t) for t in rng.integers(0, 32000, size=int(rng.integers(1, 60)))]
+        toks = prompt + tail
+        got = ls.cpp.add_seq_tokens(r, toks)
+        assert got == ls.ref.add_seq_tokens(r, toks)
+        assert got == (0 if r == 0 else 12 * bs)
+        slots = ls.slots(r, got, len(toks) - got)
+        tk, tv = wl.new_tokens(rng, len(tail), Hkv, D)
+        k = np.concatenate([pk[got:], tk])
+        v = np.concatenate([pv[got:], tv])
+        pool.write(k, v, slots)
+        ids.append(r)
+    pool.check()
+    assert ls.cpp.num_cached_blocks() == ls.ref.num_cached_blocks() >= 12
+    tables, clens = ls.tables(ids, 20)
+    assert all(tables[r][:12].tolist() == tables[0][:12].tolist() for r in ids)
+    decode_and_compare(pkv, pool, wl.bf16_normal(rng, (len(ids), Hq, D)), tables, clens, wl.fp32_scale(D), Hq)

@@ -368,3 +368,14 @@ def kv_scales(rng: np.random.Generator, num_kv_heads: int, lo: float = 1.0 / 64,
     """Seeded per-kv-head float32 scales of an 8-bit cache: N(0,1) data divided by a
     scale in [1/64, 1/32] spans about +-320 before saturation at 448."""
     return rng.uniform(lo, hi, size=num_kv_heads).astype(np.float32)
+
+
+def e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
+    """Seeded 8-bit (e4m3) pool contents drawn directly as bit patterns: random sign,
+    exponent field around 8 (values of magnitude ~1..4 before the scale), uniform
+    mantissa, never the NaN pattern.  Pure integer draws, no rounding arithmetic."""
+    sign = rng.integers(0, 2, size=shape)
+    exp = np.clip(np.rint(rng.normal(8.0, 1.5, size=shape)), 0, 15).astype(np.int64)
+    mant = rng.integers(0, 8, size=shape)
+    mant = np.where((exp == 15) & (mant == 7), 6, mant)
+    return ((sign << 7) | (exp << 3) | mant).astype(np.uint8)

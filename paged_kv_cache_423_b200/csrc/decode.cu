@@ -44,9 +44,9 @@
 #ifndef PKV_SIMT_DYNAMIC
 #define PKV_SIMT_DYNAMIC 1
 #endif
-// Ring stages per warp for an 8-bit pool (half the bytes per stage).
+// Ring stages per warp for an 8-bit pool (32-token stages of the same 8 KiB).
 #ifndef PKV_SIMT_STAGES8
-#define PKV_SIMT_STAGES8 4
+#define PKV_SIMT_STAGES8 2
 #endif
 
 namespace pkv {
@@ -138,14 +138,21 @@ __global__ void __launch_bounds__(kPlanThreads)
 // CUDA-core streaming kernel
 // ---------------------------------------------------------------------------
 
+// Tokens per ring stage: 16-row slices for bf16 (4 KiB of K at D = 128); an 8-bit
+// pool takes 32 tokens per stage, so a stage still moves 8 KiB of K and V and the
+// fixed cost of a stage (wait, reductions, softmax) is spread over as many bytes.
+template <bool KV8>
+constexpr int stage_tokens() { return KV8 ? 2 * kStageTokens : kStageTokens; }
+
 template <int D, int STAGES, bool KV8 = false>
 struct __align__(128) WarpRing {
   using KvT = std::conditional_t<KV8, uint8_t, __nv_bfloat16>;  // bf16 or e4m3 pool elements
-  KvT k[STAGES][kStageTokens * D];
-  KvT v[STAGES][kStageTokens * D];
+  static constexpr int ST = stage_tokens<KV8>();
+  KvT k[STAGES][ST * D];
+  KvT v[STAGES][ST * D];
   __nv_bfloat16 q[STAGES][D];
-  float2 p[kStageTokens];  // (p_t, p_t) of the stage being consumed, read back as packed pairs
-                           // (8-bit pool: p_t rounded to f16 in the low half of .x)
+  float2 p[ST];  // (p_t, p_t) of the stage being consumed, read back as packed pairs
+                 // (8-bit pool: p_t rounded to f16 in the low half of .x)
   uint64_t full[STAGES];
   int4 meta[STAGES];  // x seq, y query head, z part | nparts << 16, w n_valid | flags (first, last, q present)
 };
@@ -157,9 +164,9 @@ struct IssueItem {
   int table;       // lane j: physical block of the item's j-th block (prefetched)
 };
 
-__device__ __forceinline__ int item_stages(const PlanEntry& e, int partition) {
+__device__ __forceinline__ int item_stages(const PlanEntry& e, int partition, int stage_tok) {
   const int ntok = e.w == 0 ? 0 : min(partition, e.w - e.y * partition);
-  return ntok == 0 ? 1 : (ntok + kStageTokens - 1) / kStageTokens;
+  return ntok == 0 ? 1 : (ntok + stage_tok - 1) / stage_tok;
 }
 
 // Load lane j's table entry for the item (block tok0/bs + j), 0 past the item.
@@ -267,11 +274,13 @@ struct LaneMap<128, true> {
 };
 
 // ---- e4m3 helpers (8-bit pool)
-// Two e4m3 codes (low byte first) -> f16x2, exactly (every e4m3 value is an f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair16) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(r) : "r"(pair16));
-  return r;
+// Four e4m3 codes of a word (low byte first) -> two f16x2 (bytes 0,1 and 2,3), exactly
+// (every e4m3 value is an f16 value).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 // a0 += x.lo * y.lo, a1 += x.hi * y.hi with f16 operands and fp32 accumulation
 // (sm_100 mixed-precision FMA; the f16 x f16 product is exact in fp32).
@@ -312,7 +321,9 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   constexpr int NPAIR = EPL / 2;                               // packed fp32 pairs per lane
   constexpr int NC = LaneMap<D, KV8>::NC;
   using Ring = WarpRing<D, STAGES, KV8>;
-  constexpr uint32_t kKVBytes = kStageTokens * D * sizeof(typename Ring::KvT);
+  constexpr int ST = Ring::ST;
+  constexpr uint32_t kKVBytes = ST * D * sizeof(typename Ring::KvT);          // a full stage of K (or V)
+  constexpr uint32_t kSliceBytes = kStageTokens * D * sizeof(typename Ring::KvT);  // one 16-row slice
   constexpr uint32_t kQBytes = D * sizeof(__nv_bfloat16);
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -367,7 +378,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
 #endif
   nxt.table = nxt.id >= 0 ? load_item_table(a, nxt.e, lane) : 0;
   int cur_stage = 0;
-  int cur_nstages = item_stages(cur.e, a.partition);
+  int cur_nstages = item_stages(cur.e, a.partition, ST);
   bool issue_done = false;
 
   // Issue the next stage into `slot`; false when every item has been issued.
@@ -392,23 +403,27 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
 #endif
       nx2_e = entry_of(nx2_id >= 0 ? nx2_id : n_items);
       cur_stage = 0;
-      cur_nstages = item_stages(cur.e, a.partition);
+      cur_nstages = item_stages(cur.e, a.partition, ST);
     }
     const PlanEntry e = cur.e;
     const int qh = static_cast<int>(cur.id % a.num_heads);
     const int kvh = qh / a.group;
-    const int local_tok = cur_stage * kStageTokens;
+    const int local_tok = cur_stage * ST;
     const int tok = e.y * a.partition + local_tok;                       // first token of the stage
-    const int n_tok = e.w == 0 ? 0 : min(kStageTokens, e.w - tok);
+    const int n_tok = e.w == 0 ? 0 : min(ST, e.w - tok);
     const int phys = __shfl_sync(kFull, cur.table, local_tok / a.block_size);
-    const bool ok = n_tok > 0 && phys >= 0 && phys < a.num_blocks;
+    // 8-bit pool: the stage's second 16-row slice (maybe in the next block at bs 16)
+    const int phys2 = KV8 ? __shfl_sync(kFull, cur.table, (local_tok + kStageTokens) / a.block_size) : 0;
+    const bool two = KV8 && n_tok > kStageTokens;
+    const bool ok = n_tok > 0 && phys >= 0 && phys < a.num_blocks && (!two || (phys2 >= 0 && phys2 < a.num_blocks));
     const bool first = cur_stage == 0, last = cur_stage == cur_nstages - 1;
     const bool with_q = first && n_tok > 0;
     if (lane == 0) {
       if (n_tok > 0 && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
       ring.meta[slot] = make_int4(e.x, qh, e.y | (e.z << 16),
                                   (ok ? n_tok : 0) | (first ? 0x100 : 0) | (last ? 0x200 : 0) | (with_q ? 0x400 : 0));
-      const uint32_t bytes = (ok ? 2 * kKVBytes : 0) + (with_q ? kQBytes : 0);
+      const uint32_t kv_bytes = KV8 ? (two ? 2 : 1) * 2 * kSliceBytes : 2 * kKVBytes;
+      const uint32_t bytes = (ok ? kv_bytes : 0) + (with_q ? kQBytes : 0);
       mbar_arrive_expect_tx(&ring.full[slot], bytes);
       if (with_q)
         bulk_copy_g2s(ring.q[slot], a.query + (static_cast<int64_t>(e.x) * a.num_heads + qh) * D, kQBytes,
@@ -416,8 +431,17 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       if (ok) {
         const int64_t row = (static_cast<int64_t>(phys) * a.num_kv_heads + kvh) * a.block_size + local_tok % a.block_size;
         if constexpr (KV8) {
-          bulk_copy_g2s(ring.k[slot], a.key_cache8 + row * D, kKVBytes, &ring.full[slot], policy);
-          bulk_copy_g2s(ring.v[slot], a.value_cache8 + row * D, kKVBytes, &ring.full[slot], policy);
+          bulk_copy_g2s(ring.k[slot], a.key_cache8 + row * D, kSliceBytes, &ring.full[slot], policy);
+          bulk_copy_g2s(ring.v[slot], a.value_cache8 + row * D, kSliceBytes, &ring.full[slot], policy);
+          if (two) {
+            const int t2 = local_tok + kStageTokens;
+            const int64_t row2 =
+                (static_cast<int64_t>(phys2) * a.num_kv_heads + kvh) * a.block_size + t2 % a.block_size;
+            bulk_copy_g2s(ring.k[slot] + kStageTokens * D, a.key_cache8 + row2 * D, kSliceBytes, &ring.full[slot],
+                          policy);
+            bulk_copy_g2s(ring.v[slot] + kStageTokens * D, a.value_cache8 + row2 * D, kSliceBytes,
+                          &ring.full[slot], policy);
+          }
         } else {
           bulk_copy_g2s(ring.k[slot], a.key_cache + row * D, kKVBytes, &ring.full[slot], policy);
           bulk_copy_g2s(ring.v[slot], a.value_cache + row * D, kKVBytes, &ring.full[slot], policy);
@@ -434,13 +458,13 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   constexpr int NQ = KV8 ? 2 * NC : NC;
   uint4 qv[NQ];
   uint64_t o[NPAIR];            // packed fp32 output accumulators
-  float o8[KV8 ? EPL : 1];      // 8-bit pool: scalar fp32 accumulators
+  float o8[KV8 ? 2 * EPL : 1];  // 8-bit pool: scalar fp32 accumulators, two sets (even / odd tokens)
   float score_scale = a.scale_log2, out_scale = 1.f;
   float m = -INFINITY, lsum = 0.f;
 #pragma unroll
   for (int i = 0; i < NQ; ++i) qv[i] = make_uint4(0, 0, 0, 0);
 #pragma unroll
-  for (int j = 0; j < (KV8 ? EPL : 1); ++j) o8[j] = 0.f;
+  for (int j = 0; j < (KV8 ? 2 * EPL : 1); ++j) o8[j] = 0.f;
 #pragma unroll
   for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
 
@@ -467,7 +491,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
       if constexpr (KV8) {
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) o8[j] = 0.f;
+        for (int j = 0; j < 2 * EPL; ++j) o8[j] = 0.f;
         if (mt.w & 0x400) {
           // q to f16 for the mixed-precision products.  bf16 values of magnitude
           // >= 2^15 would overflow f16: then the whole vector is scaled by 2^-16
@@ -508,27 +532,64 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       }
     }
     if (n_valid > 0) {
-      // ---- scores: two lanes per row, bf16 x bf16 (or f16 x e4m3) products accumulated in fp32
+      float alpha;
+      if constexpr (KV8) {
+        // ---- scores, 8-bit pool: rows r and r + 16 of the 32-token stage; two lanes per
+        // row, f16 x e4m3 products accumulated in fp32
+        float sc[2];
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+          const int r = qk_row + pass * kStageTokens;
+          const uint4* krow = reinterpret_cast<const uint4*>(ring.k[slot] + r * D) + qk_half * NC;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
+#pragma unroll
+          for (int i = 0; i < NC; ++i) {
+            const uint4 kw = krow[(i + qk_row) & (NC - 1)];
+            const uint32_t kws[4] = {kw.x, kw.y, kw.z, kw.w};
+            const uint4 q0 = qv[2 * i], q1 = qv[2 * i + 1];
+            const uint32_t qs[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t k01, k23;
+              e4m3x4_to_f16x2x2(kws[c], k01, k23);
+              if (c & 1) {
+                dot_f16x2(b0, b1, qs[2 * c], k01);
+                dot_f16x2(b2, b3, qs[2 * c + 1], k23);
+              } else {
+                dot_f16x2(a0, a1, qs[2 * c], k01);
+                dot_f16x2(a2, a3, qs[2 * c + 1], k23);
+              }
+            }
+          }
+          sc[pass] = (a0 + a1) + (a2 + a3) + ((b0 + b1) + (b2 + b3));
+        }
+        sc[0] += __shfl_xor_sync(kFull, sc[0], LaneMap<D, KV8>::PARTNER);
+        sc[1] += __shfl_xor_sync(kFull, sc[1], LaneMap<D, KV8>::PARTNER);
+        const bool v0 = qk_row < n_valid, v1 = qk_row + kStageTokens < n_valid;
+        const float x0 = v0 ? sc[0] * score_scale : -INFINITY;
+        const float x1 = v1 ? sc[1] * score_scale : -INFINITY;
+        const float m_new = fmaxf(m, LaneMap<D, KV8>::max_rows(fmaxf(x0, x1)));
+        alpha = exp2f(m - m_new);
+        // the weights the P·V products use: p rounded to f16; the sum adds the same values
+        const uint32_t p16a = f32x2_to_f16x2(v0 ? exp2f(x0 - m_new) : 0.f, 0.f);
+        const uint32_t p16b = f32x2_to_f16x2(v1 ? exp2f(x1 - m_new) : 0.f, 0.f);
+        m = m_new;
+        lsum = fmaf(lsum, alpha, f16lo_to_f32(p16a) + f16lo_to_f32(p16b));
+        if (qk_half == 0) {
+          ring.p[qk_row] = make_float2(__uint_as_float(p16a), 0.f);
+          ring.p[qk_row + kStageTokens] = make_float2(__uint_as_float(p16b), 0.f);
+        }
+      } else {
+      // ---- scores: two lanes per row, bf16 x bf16 products accumulated in fp32
       const uint4* krow = reinterpret_cast<const uint4*>(ring.k[slot] + qk_row * D) + qk_half * NC;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
       for (int i = 0; i < NC; ++i) {
         const uint4 kw = krow[(i + qk_row) & (NC - 1)];
-        if constexpr (KV8) {
-          const uint32_t kws[4] = {kw.x, kw.y, kw.z, kw.w};
-          const uint4 q0 = qv[2 * i], q1 = qv[2 * i + 1];
-          const uint32_t qs[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            dot_f16x2(a0, a1, qs[2 * c], e4m3x2_to_f16x2(kws[c] & 0xffffu));
-            dot_f16x2(a2, a3, qs[2 * c + 1], e4m3x2_to_f16x2(kws[c] >> 16));
-          }
-        } else {
-          dot_bf16x2(a0, a1, qv[i].x, kw.x);
-          dot_bf16x2(a2, a3, qv[i].y, kw.y);
-          dot_bf16x2(a0, a1, qv[i].z, kw.z);
-          dot_bf16x2(a2, a3, qv[i].w, kw.w);
-        }
+        dot_bf16x2(a0, a1, qv[i].x, kw.x);
+        dot_bf16x2(a2, a3, qv[i].y, kw.y);
+        dot_bf16x2(a0, a1, qv[i].z, kw.z);
+        dot_bf16x2(a2, a3, qv[i].w, kw.w);
       }
       float sc = (a0 + a1) + (a2 + a3);
       sc += __shfl_xor_sync(kFull, sc, LaneMap<D, KV8>::PARTNER);
@@ -536,36 +597,41 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       const bool valid = qk_row < n_valid;
       const float x = valid ? sc * score_scale : -INFINITY;
       const float m_new = fmaxf(m, LaneMap<D, KV8>::max_rows(x));
-      const float alpha = exp2f(m - m_new);
-      float p = valid ? exp2f(x - m_new) : 0.f;
-      uint32_t p16 = 0;
-      if constexpr (KV8) {
-        // the weight the P·V products use: p rounded to f16; the sum adds the same value
-        p16 = f32x2_to_f16x2(p, 0.f);
-        p = f16lo_to_f32(p16);
-      }
+      alpha = exp2f(m - m_new);
+      const float p = valid ? exp2f(x - m_new) : 0.f;
       m = m_new;
       lsum = fmaf(lsum, alpha, p);
-      if (qk_half == 0) {
-        if constexpr (KV8)
-          ring.p[qk_row] = make_float2(__uint_as_float(p16), 0.f);
-        else
-          ring.p[qk_row] = make_float2(p, p);
+      if (qk_half == 0) ring.p[qk_row] = make_float2(p, p);
       }
       __syncwarp();
       // ---- P·V: packed fp32 pairs, rows past n_valid never touched (stale rows may be NaN)
       if constexpr (KV8) {
         // ---- P·V over e4m3 rows: lane l owns values 4l..4l+3; f16 x f16 products, fp32 sums
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) o8[j] *= alpha;
+        for (int j = 0; j < 2 * EPL; ++j) o8[j] *= alpha;
         const uint8_t* vb = ring.v[slot] + lane * EPL;
         const float2* pr = ring.p;
+        // even and odd tokens accumulate into separate sets (shorter dependency chains)
+        int t = 0;
 #pragma unroll 4
-        for (int t = 0; t < n_valid; ++t) {
-          const uint32_t pw = __float_as_uint(pr[t].x);
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(vb + t * D);
-          axpy_f16x2(o8[0], o8[1], pw, e4m3x2_to_f16x2(w & 0xffffu));
-          axpy_f16x2(o8[2], o8[3], pw, e4m3x2_to_f16x2(w >> 16));
+        for (; t + 1 < n_valid; t += 2) {
+          const uint32_t pw0 = __float_as_uint(pr[t].x), pw1 = __float_as_uint(pr[t + 1].x);
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vb + t * D);
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vb + (t + 1) * D);
+          uint32_t v01, v23, u01, u23;
+          e4m3x4_to_f16x2x2(w0, v01, v23);
+          e4m3x4_to_f16x2x2(w1, u01, u23);
+          axpy_f16x2(o8[0], o8[1], pw0, v01);
+          axpy_f16x2(o8[2], o8[3], pw0, v23);
+          axpy_f16x2(o8[4], o8[5], pw1, u01);
+          axpy_f16x2(o8[6], o8[7], pw1, u23);
+        }
+        if (t < n_valid) {
+          const uint32_t pw0 = __float_as_uint(pr[t].x);
+          uint32_t v01, v23;
+          e4m3x4_to_f16x2x2(*reinterpret_cast<const uint32_t*>(vb + t * D), v01, v23);
+          axpy_f16x2(o8[0], o8[1], pw0, v01);
+          axpy_f16x2(o8[2], o8[3], pw0, v23);
         }
       } else {
       const uint64_t alpha2 = f2pack(alpha, alpha);
@@ -607,7 +673,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       float of[EPL];
       if constexpr (KV8) {
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) of[j] = o8[j] * out_scale;  // the value scale of the kv head
+        for (int j = 0; j < EPL; ++j) of[j] = (o8[j] + o8[EPL + j]) * out_scale;  // the value scale of the kv head
       } else {
 #pragma unroll
         for (int j = 0; j < NPAIR; ++j) {

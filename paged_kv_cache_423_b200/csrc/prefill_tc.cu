@@ -6,24 +6,32 @@
 // already in the pool.  Chunk row i is the token at position p = L - n + i and
 // attends causally to positions 0 .. p, read page by page through the block table.
 //
-// Unlike decode, the query side is dense: a tile is 128 query rows = 128 / g tokens
-// x the g query heads of one kv head (row m = token * g + head), and every K/V tile
-// is shared by all of them.  Per 128-key tile:
-//   S[128 x 128] = Q[128 x D] · K[128 x D]ᵀ       (A = Q, B = K; both K-major, TMA-swizzled)
+// Unlike decode, the query side is dense.  A query tile is 128 rows = 128 / g tokens
+// x the g query heads of one kv head (row m = token * g + head).  A CTA holds TWO
+// consecutive query tiles (A and B) of one (sequence, kv head) and streams the K/V
+// pages once for both, 64 keys per stage:
+//   S_t[128 x 64]  = Q_t[128 x D] · K[64 x D]ᵀ      (A = Q_t, B = K; K-major, TMA-swizzled)
 //   online softmax of each row (one thread per TMEM lane; causal mask on the diagonal)
-//   O[128 x D]  += P[128 x 128] · V[128 x D]      (A = P, K-major, written by the softmax
-//                                                   threads; B = V, MN-major)
-// S is double-buffered in tensor memory (columns 0-127, 128-255), O lives in columns
-// 256-383 for the whole item.  O is rescaled in tensor memory only when a row's
+//   O_t[128 x D]  += P_t[128 x 64] · V[64 x D]      (A = P_t, K-major, written by the
+//                                                     softmax threads; B = V, MN-major)
+// Sharing a K/V stage between two tiles doubles the math per byte staged.  P is
+// double-buffered per tile, so a softmax group writes P of stage n+1 while the
+// tensor cores still multiply P of stage n: the MMA's issue-to-completion latency
+// stays off the per-stage critical path.
+//
+// Tensor memory (512 columns): S of tile t double-buffered in columns t*128 + {0, 64},
+// O of tile t in 256 + t*128.  O is rescaled in tensor memory only when a row's
 // maximum grows by more than 2^8; P is rounded to bf16 for the MMA and the row sums
 // add the same rounded values.
 //
-// Work item = (query tile, kv head), from a plan ordered longest sequence first with
-// every tile of a sequence adjacent, so the tiles that read the same K/V pages run
-// at the same time and share them through L2.  CTAs are persistent and take items
-// from a counter.  Roles: warps 0-3 softmax + epilogue, warp 4 TMA producer, warp 5
-// MMA issuer.  Every wait is bounded; on a timeout the CTA flags PKV_DEV_TIMEOUT,
-// lets its copies land, frees its tensor memory and exits.
+// Work item = (pair of query tiles, kv head), from a plan ordered longest sequence
+// first with every tile pair of a sequence adjacent, so items that read the same
+// K/V pages run at the same time and share them through L2.  CTAs are persistent and
+// take items from a counter.  Roles: warps 0-3 softmax + epilogue of tile A, warps
+// 4-7 of tile B, warp 8 TMA producer, warp 9 MMA issuer.  Per-stage metadata travels
+// in its own ring, so the softmax warps never wait for a V tile they do not touch.
+// Every wait is bounded; on a timeout the CTA flags PKV_DEV_TIMEOUT, lets its copies
+// land, waits for its MMAs, frees its tensor memory and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -39,42 +47,46 @@ namespace pf {
 
 using tc::fast_exp2;
 
-constexpr int kRows = 128;                // query rows per tile (MMA M)
-constexpr int kKeys = 128;                // keys per tile
-constexpr int kD = 128;                   // head_dim of this path
-constexpr int kHalf = 128 * 128;          // one 64-column half of a 128-row bf16 tile: 16 KiB
-constexpr int kTileBytes = 2 * kHalf;
-constexpr int kChunk = 16;                // key rows per TMA box (a 16-row slice of one block)
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kRows = 128;                  // query rows per tile (MMA M)
+constexpr int kKeys = 64;                   // keys per stage
+constexpr int kD = 128;                     // head_dim of this path
+constexpr int kQHalf = kRows * 128;         // one 64-column half of a 128-row bf16 tile: 16 KiB
+constexpr int kQBytes = 2 * kQHalf;         // a query tile: 32 KiB
+constexpr int kKvHalf = kKeys * 128;        // one 64-column half of a 64-row K or V tile: 8 KiB
+constexpr int kKvBytes = 2 * kKvHalf;       // 16 KiB
+constexpr int kPBytes = kRows * kKeys * 2;  // P of one tile: 128 rows x 128 bytes
+constexpr int kChunk = 16;                  // key rows per TMA box (a 16-row slice of one block)
+constexpr int kStages = 3;
+constexpr int kMetaSlots = 8;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;
 
 // shared memory (offsets from a 1024-aligned base)
-constexpr int kOffQ = 0;
-constexpr int kOffP = kOffQ + kTileBytes;
-constexpr int kOffK = kOffP + kTileBytes;
-constexpr int kOffV = kOffK + kKStages * kTileBytes;
-constexpr int kOffMetaV = kOffV + kVStages * kTileBytes;
-constexpr int kOffMetaK = kOffMetaV + kVStages * 16;
-constexpr int kOffBar = kOffMetaK + 16;
-constexpr int kBars = 19;
+constexpr int kOffQ = 0;                                  // [2 tiles][32 KiB]
+constexpr int kOffP = kOffQ + 2 * kQBytes;                // [2 tiles][2 buffers][16 KiB]
+constexpr int kOffKV = kOffP + 4 * kPBytes;               // [3 stages][K 16 KiB | V 16 KiB]
+constexpr int kOffMeta = kOffKV + kStages * 2 * kKvBytes; // [8] int4
+constexpr int kOffBar = kOffMeta + kMetaSlots * 16;
+constexpr int kBars = 2 + 3 * kStages + 2 * kMetaSlots + 4 + 4 + 4 + 4 + 1;
 constexpr int kOffMisc = kOffBar + kBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;          // + slack to align the base
+static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 
-// V-slot metadata: x = packed row of the tile's first token, y = its position,
-// z = tokens in the tile | kv head << 8, w = key tile | chunk mask << 20 | flags.
-constexpr int kFirst = 1 << 28, kLast = 1 << 29, kEnd = 1 << 30;
+// Stage metadata: x = packed row of tile A's first token, y = its position,
+// z = tokens of tile A | tokens of tile B << 8 | kv head << 16,
+// w = stage index in the item | chunk mask << 20 | flags.
+constexpr int kFirst = 1 << 24, kLast = 1 << 25, kEnd = 1 << 26;
 
 struct PrefillArgs {
   void* out;
   const int32_t* block_tables;
   const int32_t* plan_count;  // [0] entries, [1] work-item counter
-  const int4* entries;        // x = first packed row, y = its position, z = tokens, w = sequence
+  const int4* entries;        // x = first packed row, y = its position, z = tokens A | tokens B << 8, w = sequence
   int32_t* status;
   int max_blocks;
   int num_heads;
@@ -83,6 +95,7 @@ struct PrefillArgs {
   int num_blocks;
   int group;
   int group_shift;            // log2(group)
+  int tile_tokens;            // 128 / group
   float scale_log2;
 };
 
@@ -101,22 +114,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_buf = smem + kOffQ;
   unsigned char* p_buf = smem + kOffP;
-  unsigned char* k_ring = smem + kOffK;
-  unsigned char* v_ring = smem + kOffV;
-  int4* meta_v = reinterpret_cast<int4*>(smem + kOffMetaV);
-  int* meta_k = reinterpret_cast<int*>(smem + kOffMetaK);
+  unsigned char* kv_ring = smem + kOffKV;
+  int4* meta = reinterpret_cast<int4*>(smem + kOffMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;   // [3]
-  uint64_t* k_empty = bars + 5;  // [3]
-  uint64_t* v_full = bars + 8;   // [2]
-  uint64_t* v_empty = bars + 10; // [2]
-  uint64_t* s_full = bars + 12;  // [2]
-  uint64_t* s_free = bars + 14;  // [2]
-  uint64_t* p_full = bars + 16;
-  uint64_t* o_bar = bars + 17;
-  uint64_t* drain = bars + 18;   // the MMA thread's last commit, before tensor memory is freed
+  uint64_t* k_full = bars + 2;                        // [stage]
+  uint64_t* v_full = k_full + kStages;                // [stage]
+  uint64_t* kv_empty = v_full + kStages;              // [stage]
+  uint64_t* meta_full = kv_empty + kStages;           // [8]
+  uint64_t* meta_free = meta_full + kMetaSlots;       // [8]
+  uint64_t* s_full = meta_free + kMetaSlots;          // [tile][buffer]
+  uint64_t* s_free = s_full + 4;                      // [tile][buffer]
+  uint64_t* p_full = s_free + 4;                      // [tile][P buffer]
+  uint64_t* o_bar = p_full + 4;                       // [tile][P buffer]: that buffer's P·V done
+  uint64_t* drain = o_bar + 4;                        // the MMA thread's last commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -127,20 +139,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+      mbar_init(&kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);  // one arrival per softmax warp
+    for (int s = 0; s < kMetaSlots; ++s) {
+      mbar_init(&meta_full[s], 1);
+      mbar_init(&meta_free[s], kSoftmaxWarps);
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_bar, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);  // one arrival per warp of the tile's group
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_bar[i], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -151,192 +166,208 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  auto fail = [&]() {
+    *abort_flag = 1;
+    set_status(a.status, PKV_DEV_TIMEOUT);
+  };
+
   if (warp == kProducerWarp) {
     // ================= producer =================
     const uint64_t pol_q = l2_policy_evict_first();
-    const uint64_t pol_kv = l2_policy_evict_normal();  // every query tile of the sequence re-reads these pages
+    const uint64_t pol_kv = l2_policy_evict_normal();  // every tile pair of the sequence re-reads these pages
     int* work_counter = const_cast<int*>(a.plan_count) + 1;
     auto grab = [&]() -> int64_t {
       int v = 0;
       if (lane == 0) v = atomicAdd(work_counter, 1);
       return __shfl_sync(0xffffffffu, v, 0);
     };
-    auto acquire = [&](uint64_t* bar, int fills, int stages) -> bool {
-      if (fills >= stages && !mbar_wait(bar, ((fills / stages) - 1) & 1)) {
-        *abort_flag = 1;
-        set_status(a.status, PKV_DEV_TIMEOUT);
-        return false;
-      }
-      return true;
-    };
-    int kn = 0, vn = 0, item_ord = 0, q_loads = 0;
+    int n = 0, q_loads = 0;  // stages issued, query loads issued
     bool failed = false;
-    for (int64_t item = grab(); item < n_items && !failed && !*abort_flag; item = grab(), ++item_ord) {
+    // Claim stage slot n: its K/V buffers free (the pair's P·V of stage n-3 done) and
+    // its metadata slot read by every softmax warp (stage n-8).
+    auto acquire = [&]() -> bool {
+      bool ok = true;
+      if (n >= kStages) ok = mbar_wait(&kv_empty[n % kStages], ((n / kStages) - 1) & 1);
+      if (ok && n >= kMetaSlots) ok = mbar_wait(&meta_free[n % kMetaSlots], ((n / kMetaSlots) - 1) & 1);
+      if (!ok) fail();
+      return ok;
+    };
+    for (int64_t item = grab(); item < n_items && !failed && !*abort_flag; item = grab()) {
       const int4 e = a.entries[item / a.num_kv_heads];
       const int kvh = static_cast<int>(item % a.num_kv_heads);
-      const int row0 = e.x, pos0 = e.y, ntok = e.z, seq = e.w;
-      const int nkeys = pos0 + ntok;
-      const int nkt = (nkeys + kKeys - 1) / kKeys;
-      // Q: the previous item's last S = Q·Kᵀ must be done with the buffer
-      if (item_ord > 0 && !mbar_wait(q_empty, (item_ord - 1) & 1)) {
-        *abort_flag = 1;
-        set_status(a.status, PKV_DEV_TIMEOUT);
+      const int row0 = e.x, pos0 = e.y, ntok_a = e.z & 0xff, ntok_b = (e.z >> 8) & 0xff, seq = e.w;
+      const int nkeys = pos0 + ntok_a + ntok_b;
+      const int nst = (nkeys + kKeys - 1) / kKeys;
+      // queries: the previous item's last S = Q·Kᵀ must be done with the buffers
+      if (q_loads > 0 && !mbar_wait(q_empty, (q_loads - 1) & 1)) {
+        fail();
         failed = true;
         break;
       }
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, kTileBytes);
+        mbar_arrive_expect_tx(q_full, (ntok_b > 0 ? 2 : 1) * kQBytes);
         tc::tma_load_3d(q_buf, &args.tm_q, 0, kvh * g, row0, q_full, pol_q);
-        tc::tma_load_3d(q_buf + kHalf, &args.tm_q, 64, kvh * g, row0, q_full, pol_q);
+        tc::tma_load_3d(q_buf + kQHalf, &args.tm_q, 64, kvh * g, row0, q_full, pol_q);
+        if (ntok_b > 0) {
+          tc::tma_load_3d(q_buf + kQBytes, &args.tm_q, 0, kvh * g, row0 + a.tile_tokens, q_full, pol_q);
+          tc::tma_load_3d(q_buf + kQBytes + kQHalf, &args.tm_q, 64, kvh * g, row0 + a.tile_tokens, q_full, pol_q);
+        }
       }
       ++q_loads;
       const int32_t* table = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks;
-      for (int j = 0; j < nkt; ++j) {
+      // Table entries come 32 slices (8 stages) at a time, one window ahead: lane l
+      // holds the physical block of slice 32 w + l of window w.
+      auto load_window = [&](int w) -> int {
+        const int kp = (w * 32 + lane) * kChunk;
+        return kp < nkeys ? __ldg(table + kp / a.block_size) : -1;
+      };
+      int win = 0;
+      int tab_cur = load_window(0);
+      int tab_nxt = load_window(1);
+      for (int j = 0; j < nst; ++j) {
+        if (j / 8 != win) {
+          ++win;
+          tab_cur = tab_nxt;
+          tab_nxt = load_window(win + 1);
+        }
         const int kbase = j * kKeys;
         const int nvalid = min(kKeys, nkeys - kbase);
         const int nch = (nvalid + kChunk - 1) / kChunk;
         const int kp = kbase + lane * kChunk;  // this lane's 16-row slice (lanes < nch)
         const bool mine = lane < nch;
-        int phys = -1;
-        if (mine) phys = __ldg(table + kp / a.block_size);
+        int phys = __shfl_sync(0xffffffffu, tab_cur, (j % 8) * 4 + (lane & 3));
+        if (!mine) phys = -1;
         const bool ok = mine && phys >= 0 && phys < a.num_blocks;
-        const uint32_t mask = __ballot_sync(0xffffffffu, ok) & 0xffu;
+        const uint32_t mask = __ballot_sync(0xffffffffu, ok) & 0xfu;
         if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
         const int row = (phys * a.num_kv_heads + kvh) * a.block_size + kp % a.block_size;
-        const int flags = (j == 0 ? kFirst : 0) | (j == nkt - 1 ? kLast : 0);
-        // K
-        const int ks = kn % kKStages;
-        if (!acquire(&k_empty[ks], kn, kKStages)) {
+        if (!acquire()) {
           failed = true;
           break;
         }
+        const int st = n % kStages;
+        unsigned char* kd = kv_ring + st * 2 * kKvBytes + lane * kChunk * 128;
         if (lane == 0) {
-          meta_k[ks] = flags;
-          mbar_arrive_expect_tx(&k_full[ks], __popc(mask) * kChunk * 256);
+          meta[n % kMetaSlots] = make_int4(row0, pos0, ntok_a | (ntok_b << 8) | (kvh << 16),
+                                           j | static_cast<int>(mask << 20) | (j == 0 ? kFirst : 0) |
+                                               (j == nst - 1 ? kLast : 0));
+          mbar_arrive(&meta_full[n % kMetaSlots]);
+          mbar_arrive_expect_tx(&k_full[st], __popc(mask) * kChunk * 256);
         }
         __syncwarp();
         if (ok) {
-          unsigned char* kd = k_ring + ks * kTileBytes + lane * kChunk * 128;
-          tc::tma_load_2d(kd, &args.tm_k, 0, row, &k_full[ks], pol_kv);
-          tc::tma_load_2d(kd + kHalf, &args.tm_k, 64, row, &k_full[ks], pol_kv);
+          tc::tma_load_2d(kd, &args.tm_k, 0, row, &k_full[st], pol_kv);
+          tc::tma_load_2d(kd + kKvHalf, &args.tm_k, 64, row, &k_full[st], pol_kv);
         }
-        ++kn;
-        // V
-        const int vs = vn % kVStages;
-        if (!acquire(&v_empty[vs], vn, kVStages)) {
-          failed = true;
-          break;
-        }
-        if (lane == 0) {
-          meta_v[vs] = make_int4(row0, pos0, ntok | (kvh << 8), j | static_cast<int>(mask << 20) | flags);
-          mbar_arrive_expect_tx(&v_full[vs], __popc(mask) * kChunk * 256);
-        }
+        if (lane == 0) mbar_arrive_expect_tx(&v_full[st], __popc(mask) * kChunk * 256);
         __syncwarp();
         if (ok) {
-          unsigned char* vd = v_ring + vs * kTileBytes + lane * kChunk * 128;
-          tc::tma_load_2d(vd, &args.tm_v, 0, row, &v_full[vs], pol_kv);
-          tc::tma_load_2d(vd + kHalf, &args.tm_v, 64, row, &v_full[vs], pol_kv);
+          tc::tma_load_2d(kd + kKvBytes, &args.tm_v, 0, row, &v_full[st], pol_kv);
+          tc::tma_load_2d(kd + kKvBytes + kKvHalf, &args.tm_v, 64, row, &v_full[st], pol_kv);
         }
-        ++vn;
+        ++n;
       }
     }
-    if (!failed && !*abort_flag) {
-      // end-of-stream markers: fills with no data
-      const int ks = kn % kKStages, vs = vn % kVStages;
-      if (acquire(&k_empty[ks], kn, kKStages)) {
-        if (lane == 0) {
-          meta_k[ks] = kEnd;
-          mbar_arrive_expect_tx(&k_full[ks], 0);
-        }
-        ++kn;
-        if (acquire(&v_empty[vs], vn, kVStages)) {
-          if (lane == 0) {
-            meta_v[vs] = make_int4(0, 0, 0, kEnd);
-            mbar_arrive_expect_tx(&v_full[vs], 0);
-          }
-          ++vn;
-        }
+    if (!failed && !*abort_flag && acquire()) {
+      // end-of-stream: a stage with no data
+      if (lane == 0) {
+        meta[n % kMetaSlots] = make_int4(0, 0, 0, kEnd);
+        mbar_arrive(&meta_full[n % kMetaSlots]);
+        mbar_arrive_expect_tx(&k_full[n % kStages], 0);
+        mbar_arrive_expect_tx(&v_full[n % kStages], 0);
       }
+      ++n;
       __syncwarp();
     }
     // Let this CTA's last copies land before the final barrier.
-    for (int k = max(0, kn - kKStages); k < kn; ++k) mbar_wait(&k_full[k % kKStages], (k / kKStages) & 1);
-    for (int k = max(0, vn - kVStages); k < vn; ++k) mbar_wait(&v_full[k % kVStages], (k / kVStages) & 1);
+    for (int k = max(0, n - kStages); k < n; ++k) {
+      mbar_wait(&k_full[k % kStages], (k / kStages) & 1);
+      mbar_wait(&v_full[k % kStages], (k / kStages) & 1);
+    }
     if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1);
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer (one thread) =================
+    // A fixed order with blocking waits, one barrier at a time: S of stage n+1 for
+    // both tiles first (the tensor cores work while the softmax groups handle stage
+    // n), then P·V of stage n as each group's P lands.  At an item boundary P·V of
+    // the old item's last stage goes first, so its epilogue is not held up by the
+    // next item's query load.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc::instr_desc(kRows, kKeys, false, false);
       constexpr uint32_t idesc_pv = tc::instr_desc(kRows, kD, false, true);
-      const uint32_t q_addr = smem_addr(q_buf);
-      const uint32_t p_addr = smem_addr(p_buf);
-      int qn = 0, pn = 0, end_n = 0x7fffffff, q_items = 0;
-      bool q_ready = false;
-      uint64_t idle_since = 0;
-      int idle = 0;
-      while (pn < end_n) {
-        bool progress = false;
-        // ---- S = Q·Kᵀ of the next landed key tile
-        if (qn < end_n && mbar_test(&k_full[qn % kKStages], (qn / kKStages) & 1)) {
-          const int f = meta_k[qn % kKStages];
-          if (f & kEnd) {
-            end_n = qn;
-            progress = true;
-          } else {
-            if ((f & kFirst) && !q_ready) {
-              q_ready = mbar_test(q_full, q_items & 1);
-              if (q_ready) ++q_items;
-            }
-            const int b = qn & 1;
-            if (q_ready && (qn < 2 || mbar_test(&s_free[b], ((qn >> 1) - 1) & 1))) {
-              tc::tc_fence_after();
-              const uint32_t k_addr = smem_addr(k_ring + (qn % kKStages) * kTileBytes);
-#pragma unroll
-              for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                tc::umma(tmem + b * kKeys, tc::smem_desc_sw128(q_addr + off, 16, 1024),
-                         tc::smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0);
-              }
-              tc::umma_commit(&s_full[b]);
-              tc::umma_commit(&k_empty[qn % kKStages]);
-              if (f & kLast) {
-                tc::umma_commit(q_empty);
-                q_ready = false;
-              }
-              ++qn;
-              progress = true;
-            }
-          }
+      int qc[2] = {0, 0}, pc[2] = {0, 0};  // per tile: stages whose S / P·V were issued
+      int q_items = 0;
+      bool ok = true;
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        if (ok && !mbar_wait(bar, parity)) {
+          ok = false;
+          fail();
         }
-        // ---- O += P·V of the oldest tile whose P is ready
-        if (pn < qn && mbar_test(p_full, pn & 1) && mbar_test(&v_full[pn % kVStages], (pn / kVStages) & 1)) {
-          const int vs = pn % kVStages;
-          const int w = meta_v[vs].w;  // the softmax warps waited for this fill before arriving
+        return ok;
+      };
+      // Issue S_t = Q_t·Kᵀ of stage n for every tile present; false at end of stream.
+      auto issue_qk = [&](int n) -> bool {
+        if (!wait(&k_full[n % kStages], (n / kStages) & 1)) return false;
+        const int4 mt = meta[n % kMetaSlots];
+        if (mt.w & kEnd) return false;
+        const bool has_b = ((mt.z >> 8) & 0xff) != 0;
+        if (mt.w & kFirst) {
+          if (!wait(q_full, q_items & 1)) return false;
+          ++q_items;
+        }
+        const uint32_t k_addr = smem_addr(kv_ring + (n % kStages) * 2 * kKvBytes);
+        for (int t = 0; t < (has_b ? 2 : 1); ++t) {
+          const int b = qc[t] & 1;
+          if (qc[t] >= 2 && !wait(&s_free[t * 2 + b], ((qc[t] >> 1) - 1) & 1)) return false;
           tc::tc_fence_after();
-          const uint32_t v_addr = smem_addr(v_ring + vs * kTileBytes);
+          const uint32_t q_addr = smem_addr(q_buf + t * kQBytes);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            tc::umma(tmem + t * 128 + b * kKeys,
+                     tc::smem_desc_sw128(q_addr + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024),
+                     tc::smem_desc_sw128(k_addr + (kk >> 2) * kKvHalf + (kk & 3) * 32, 16, 1024), idesc_qk, kk > 0);
+          }
+          tc::umma_commit(&s_full[t * 2 + b]);
+          ++qc[t];
+        }
+        if (mt.w & kLast) tc::umma_commit(q_empty);
+        return true;
+      };
+      // Issue O_t += P_t·V of stage n for every tile present, then release the stage.
+      auto issue_pv = [&](int n) -> bool {
+        const int4 mt = meta[n % kMetaSlots];
+        const bool has_b = ((mt.z >> 8) & 0xff) != 0;
+        if (!wait(&v_full[n % kStages], (n / kStages) & 1)) return false;
+        const uint32_t v_addr = smem_addr(kv_ring + (n % kStages) * 2 * kKvBytes + kKvBytes);
+        for (int t = 0; t < (has_b ? 2 : 1); ++t) {
+          const int pb = pc[t] & 1;
+          if (!wait(&p_full[t * 2 + pb], (pc[t] >> 1) & 1)) return false;
+          tc::tc_fence_after();
+          const uint32_t p_addr = smem_addr(p_buf + (t * 2 + pb) * kPBytes);
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
-            // P: K-major, 128-byte swizzle (as TMA writes it); V: MN-major, 16 key rows per step
-            tc::umma(tmem + kColO, tc::smem_desc_sw128(p_addr + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024),
-                     tc::smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024), idesc_pv, kk > 0 || !(w & kFirst));
+            // P: K-major, 128-byte swizzle; V: MN-major, 16 key rows per step
+            tc::umma(tmem + kColO + t * 128, tc::smem_desc_sw128(p_addr + kk * 32, 16, 1024),
+                     tc::smem_desc_sw128(v_addr + kk * 2048, kKvHalf, 1024), idesc_pv, kk > 0 || !(mt.w & kFirst));
           }
-          tc::umma_commit(o_bar);
-          tc::umma_commit(&v_empty[vs]);
-          ++pn;
-          progress = true;
+          tc::umma_commit(&o_bar[t * 2 + pb]);
+          ++pc[t];
         }
-        if (progress) {
-          idle = 0;
-        } else {
-          __nanosleep(32);
-          if (++idle == 64) {
-            idle_since = global_timer_ns();
-          } else if (idle > 64 && (idle & 63) == 0) {
-            if (*abort_flag || global_timer_ns() - idle_since > kWaitLimitNs) {
-              *abort_flag = 1;
-              set_status(a.status, PKV_DEV_TIMEOUT);
-              break;
-            }
+        tc::umma_commit(&kv_empty[n % kStages]);
+        return true;
+      };
+      if (issue_qk(0)) {
+        for (int n = 0; ok; ++n) {
+          // stage n+1: does it start a new item (or end the stream)?
+          const bool next_ready = wait(&k_full[(n + 1) % kStages], ((n + 1) / kStages) & 1);
+          if (!next_ready) break;
+          const int wnext = meta[(n + 1) % kMetaSlots].w;
+          if ((wnext & kEnd) || (wnext & kFirst)) {
+            if (!issue_pv(n)) break;
+            if ((wnext & kEnd) || !issue_qk(n + 1)) break;
+          } else {
+            if (!issue_qk(n + 1)) break;
+            if (!issue_pv(n)) break;
           }
         }
       }
@@ -346,24 +377,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
     __syncwarp();
   } else {
-    // ================= softmax warps: thread = query row = TMEM lane =================
-    const int m = tid;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // ================= softmax warps: thread = query row of tile t = TMEM lane =================
+    const int t = warp >> 2;                 // 0: tile A (warps 0-3), 1: tile B (warps 4-7)
+    const int m = tid & 127;                 // row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t col_s = t * 128, col_o = kColO + t * 128;
     float m_used = -INFINITY, lsum = 0.f;
     bool has_pv = false;
-    int waited_pv = 0;  // P·V completions this thread has observed
-    for (int t = 0;; ++t) {
-      const int vs = t % kVStages;
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&v_full[vs], (t / kVStages) & 1));
-      const int4 mt = meta_v[vs];
+    int c = 0;  // stages of this tile processed (S and P buffers)
+    // P buffer k's P·V: uses issued and completions observed (wait for each in order)
+    int uses[2] = {0, 0}, seen[2] = {0, 0};
+    auto wait_pv = [&](int k) -> bool {
+      if (seen[k] == uses[k]) return true;
+      seen[k] = uses[k];
+      return mbar_wait(&o_bar[t * 2 + k], (uses[k] - 1) & 1);
+    };
+    for (int n = 0;; ++n) {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&meta_full[n % kMetaSlots], (n / kMetaSlots) & 1));
+      const int4 mt = meta[n % kMetaSlots];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&meta_free[n % kMetaSlots]);
       if (!ok || (mt.w & kEnd)) {  // warp-uniform: every lane leaves together
         if (!ok) *abort_flag = 1;
         break;
       }
+      const int ntok_a = mt.z & 0xff, ntok_b = (mt.z >> 8) & 0xff, kvh = mt.z >> 16;
+      const int ntok = t == 0 ? ntok_a : ntok_b;
+      if (ntok == 0) continue;  // tile B absent from this item
       const int j = mt.w & 0xfffff;
-      const uint32_t mask = (mt.w >> 20) & 0xffu;
+      const uint32_t mask = (mt.w >> 20) & 0xfu;
       const bool first = mt.w & kFirst, last = mt.w & kLast;
-      const int row0 = mt.x, pos0 = mt.y, ntok = mt.z & 0xff, kvh = mt.z >> 8;
+      const int row0 = mt.x + t * a.tile_tokens, pos0 = mt.y + t * a.tile_tokens;
       if (first) {
         m_used = -INFINITY;
         lsum = 0.f;
@@ -373,54 +417,53 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const bool valid_row = tl < ntok;
       const int limit = pos0 + (valid_row ? tl : ntok - 1);  // last visible key position
       const int kbase = j * kKeys;
-      const int nvalid = min(kKeys, pos0 + ntok - kbase);
-      // V rows past the context or in a slice that was not loaded may hold anything
-      // (even NaN): zero them before P·V reads the tile.
-      if (m >= nvalid || !((mask >> (m / kChunk)) & 1u)) {
-        uint4* r0 = reinterpret_cast<uint4*>(v_ring + vs * kTileBytes + m * 128);
-        uint4* r1 = reinterpret_cast<uint4*>(v_ring + vs * kTileBytes + kHalf + m * 128);
+      const int nvalid = min(kKeys, mt.y + ntok_a + ntok_b - kbase);
+      const bool partial = nvalid < kKeys || mask != 0xfu;
+      if (t == 0 && partial) {
+        // V rows past the context or in a slice that was not loaded may hold anything
+        // (even NaN): zero them once the stage's copies have landed, before P·V.
+        const int st = n % kStages;
+        ok &= mbar_wait(&v_full[st], (n / kStages) & 1);
+        if (m < kKeys && (m >= nvalid || !((mask >> (m / kChunk)) & 1u))) {
+          unsigned char* vrow = kv_ring + st * 2 * kKvBytes + kKvBytes + m * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) r0[c] = r1[c] = make_uint4(0, 0, 0, 0);
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) reinterpret_cast<uint4*>(vrow + h * kKvHalf)[q] = make_uint4(0, 0, 0, 0);
+        }
       }
       // ---- S row
-      const int b = t & 1;
-      ok = mbar_wait(&s_full[b], (t >> 1) & 1);
+      const int b = c & 1;
+      ok &= mbar_wait(&s_full[t * 2 + b], (c >> 1) & 1);
       tc::tc_fence_after();
       float s[kKeys];
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          tc::tmem_load32_nowait(tmem + lane_base + b * kKeys + q4 * 32, r);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[q4 * 32 + c] = __uint_as_float(r[c]);
-        }
-      }
+      tc::tmem_load32f_nowait(tmem + lane_base + col_s + b * kKeys, s);
+      tc::tmem_load32f_nowait(tmem + lane_base + col_s + b * kKeys + 32, s + 32);
+      tc::tmem_wait_ld();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
+      if (lane == 0) mbar_arrive(&s_free[t * 2 + b]);
       // ---- causal / context mask and the row maximum
-      const bool full_tile = kbase + kKeys - 1 <= pos0 && mask == 0xffu;
-      if (!full_tile) {
+      if (!(kbase + kKeys - 1 <= pos0 && mask == 0xfu)) {
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c) {
-          const bool vis = kbase + c <= limit && ((mask >> (c / kChunk)) & 1u);
-          s[c] = vis ? s[c] : -INFINITY;
+        for (int k = 0; k < kKeys; ++k) {
+          const bool vis = kbase + k <= limit && ((mask >> (k / kChunk)) & 1u);
+          s[k] = vis ? s[k] : -INFINITY;
         }
       }
-      float mx = s[0];
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < kKeys; ++c) mx = fmaxf(mx, s[c]);
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int k = 8; k < kKeys; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], s[k]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mxs = mx * a.scale_log2;
-      // The single P buffer and O: the previous tile's P·V must be done.
-      if (t > waited_pv) {
-        ok &= mbar_wait(o_bar, (t - 1) & 1);
-        waited_pv = t;
-      }
+      const int pb = c & 1;
+      ok &= wait_pv(pb);  // this P buffer's previous P·V (two stages back) is done
       // A row rescales only when its maximum grew past the threshold; the tensor-memory
-      // accesses are warp-collective, so the warp rescales together (alpha = 1 for
-      // the rows that keep their maximum).
+      // accesses are warp-collective, so the warp rescales together (alpha = 1 for the
+      // rows that keep their maximum).
       const bool need = mxs > m_used + kRescaleLog2;
       float alpha = 1.f;
       if (need) {
@@ -429,15 +472,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         m_used = m_new;
       }
       if (has_pv && __any_sync(0xffffffffu, need)) {
+        ok &= wait_pv(pb ^ 1);  // O must hold every issued P·V before it is rescaled
         tc::tc_fence_after();
-        uint32_t r[32];
+        uint32_t r[2][32];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          tc::tmem_load32_nowait(tmem + lane_base + kColO + q4 * 32, r);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          tc::tmem_load32_nowait(tmem + lane_base + col_o + h2 * 64, r[0]);
+          tc::tmem_load32_nowait(tmem + lane_base + col_o + h2 * 64 + 32, r[1]);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-          tc::tmem_store32(tmem + lane_base + kColO + q4 * 32, r);
+          for (int k = 0; k < 32; ++k) {
+            r[0][k] = __float_as_uint(__uint_as_float(r[0][k]) * alpha);
+            r[1][k] = __float_as_uint(__uint_as_float(r[1][k]) * alpha);
+          }
+          tc::tmem_store32(tmem + lane_base + col_o + h2 * 64, r[0]);
+          tc::tmem_store32(tmem + lane_base + col_o + h2 * 64 + 32, r[1]);
         }
         tc::tmem_wait_st();
       }
@@ -445,7 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       // ---- P = 2^(s * scale_log2 - m), bf16, written as the K-major swizzled A operand
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const bool any = m_used != -INFINITY;
-      unsigned char* prow = p_buf + m * 128;
+      unsigned char* prow = p_buf + (t * 2 + pb) * kPBytes + m * 128;
+      float ls8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ls8[i] = 0.f;
 #pragma unroll
       for (int c8 = 0; c8 < kKeys / 8; ++c8) {
         uint32_t w[4];
@@ -455,41 +507,44 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           const float p0 = any ? fast_exp2(fmaf(x0, a.scale_log2, neg_m)) : 0.f;
           const float p1 = any ? fast_exp2(fmaf(x1, a.scale_log2, neg_m)) : 0.f;
           w[i] = pack_bf16x2(p0, p1);
-          lsum += bf16lo(w[i]) + bf16hi(w[i]);
+          ls8[2 * i] += bf16lo(w[i]);
+          ls8[2 * i + 1] += bf16hi(w[i]);
         }
-        const int half = c8 >> 3, chunk = c8 & 7;
-        *reinterpret_cast<uint4*>(prow + half * kHalf + ((chunk ^ (m & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (m & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      lsum += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async_smem();  // P and the zeroed V rows, before the MMA reads them
       tc::tc_fence_before();     // the rescaled O, before the next P·V
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[t * 2 + pb]);
+      ++uses[pb];
       has_pv = true;
+      ++c;
       if (last) {
-        // ---- epilogue: O / l of this row
-        ok &= mbar_wait(o_bar, t & 1);
-        waited_pv = t + 1;
+        // ---- epilogue: O / l of this row, once every P·V of the item is done
+        ok &= wait_pv(0);
+        ok &= wait_pv(1);
         tc::tc_fence_after();
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         const int64_t orow = (static_cast<int64_t>(row0 + tl) * a.num_heads + kvh * g + (m & (g - 1))) * kD;
         uint32_t r[32];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          tc::tmem_load32_nowait(tmem + lane_base + kColO + q4 * 32, r);
+          tc::tmem_load32_nowait(tmem + lane_base + col_o + q4 * 32, r);
           tc::tmem_wait_ld();
           if (valid_row) {
             if constexpr (OUT_F32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow + q4 * 32);
 #pragma unroll
-              for (int c = 0; c < 8; ++c)
-                dst[c] = make_float4(__uint_as_float(r[4 * c]) * inv, __uint_as_float(r[4 * c + 1]) * inv,
-                                     __uint_as_float(r[4 * c + 2]) * inv, __uint_as_float(r[4 * c + 3]) * inv);
+              for (int k = 0; k < 8; ++k)
+                dst[k] = make_float4(__uint_as_float(r[4 * k]) * inv, __uint_as_float(r[4 * k + 1]) * inv,
+                                     __uint_as_float(r[4 * k + 2]) * inv, __uint_as_float(r[4 * k + 3]) * inv);
             } else {
               uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow + q4 * 32);
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const uint32_t* v = r + 8 * c;
-                dst[c] = make_uint4(pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t* v = r + 8 * k;
+                dst[k] = make_uint4(pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
                                     pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
                                     pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
                                     pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
@@ -502,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       if (!ok) *abort_flag = 1;
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) break;  // warp-uniform
     }
-    if (*abort_flag && tid == 0) set_status(a.status, PKV_DEV_TIMEOUT);
+    if (*abort_flag && (tid & 127) == 0) set_status(a.status, PKV_DEV_TIMEOUT);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -512,9 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
 // ---- plan ---------------------------------------------------------------------
 //
-// One CTA.  Validates every sequence, then lays the query tiles out longest
+// One CTA.  Validates every sequence, then lays the query-tile pairs out longest
 // sequence first (counting sort on the context length, coarsened to 512 buckets),
-// each sequence's tiles adjacent and its longest tile first.  A sequence whose
+// each sequence's pairs adjacent and its longest pair first.  A sequence whose
 // numbers are inconsistent is flagged PKV_DEV_BAD_CONTEXT and its rows, when their
 // range is itself valid, are written as zeros.
 constexpr int kPlanThreads = 1024;
@@ -546,6 +601,7 @@ __global__ void __launch_bounds__(kPlanThreads) prefill_plan_kernel(const PlanAr
   __shared__ int total;
   for (int i = threadIdx.x; i < kPlanBuckets; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
+  const int pair_tokens = 2 * p.tile_tokens;
   auto check = [&](int s, int& q0, int& n, int& L) -> bool {
     q0 = p.query_start[s];
     const int q1 = p.query_start[s + 1];
@@ -569,7 +625,7 @@ __global__ void __launch_bounds__(kPlanThreads) prefill_plan_kernel(const PlanAr
       }
       continue;
     }
-    if (n > 0) atomicAdd(&cnt[plan_bucket(L, p.max_context_len)], (n + p.tile_tokens - 1) / p.tile_tokens);
+    if (n > 0) atomicAdd(&cnt[plan_bucket(L, p.max_context_len)], (n + pair_tokens - 1) / pair_tokens);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -594,12 +650,14 @@ __global__ void __launch_bounds__(kPlanThreads) prefill_plan_kernel(const PlanAr
   for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
     int q0, n, L;
     if (!check(s, q0, n, L) || n == 0) continue;
-    const int ntiles = (n + p.tile_tokens - 1) / p.tile_tokens;
-    const int pos = atomicAdd(&cnt[plan_bucket(L, p.max_context_len)], ntiles);
-    for (int k = 0; k < ntiles; ++k) {
-      const int tile = ntiles - 1 - k;  // longest (last) tile first
-      const int t0 = tile * p.tile_tokens;
-      p.entries[pos + k] = make_int4(q0 + t0, L - n + t0, min(p.tile_tokens, n - t0), s);
+    const int npairs = (n + pair_tokens - 1) / pair_tokens;
+    const int pos = atomicAdd(&cnt[plan_bucket(L, p.max_context_len)], npairs);
+    for (int k = 0; k < npairs; ++k) {
+      const int pair = npairs - 1 - k;  // longest (last) pair first
+      const int t0 = pair * pair_tokens;
+      const int na = min(p.tile_tokens, n - t0);
+      const int nb = max(0, min(p.tile_tokens, n - t0 - p.tile_tokens));
+      p.entries[pos + k] = make_int4(q0 + t0, L - n + t0, na | (nb << 8), s);
     }
   }
   if (threadIdx.x == 0) {
@@ -655,9 +713,10 @@ static int launch_main(const Args& args, int grid, cudaStream_t stream) {
   return PKV_OK;
 }
 
+// Plan entries the workspace must hold: one per pair of query tiles.
 static int max_entries(int num_seqs, int total_q, int group) {
-  const int tile_tokens = kRows / group;
-  return (total_q + tile_tokens - 1) / tile_tokens + num_seqs;
+  const int pair_tokens = 2 * (kRows / group);
+  return (total_q + pair_tokens - 1) / pair_tokens + num_seqs;
 }
 
 }  // namespace pf
@@ -696,7 +755,7 @@ extern "C" int pkv_paged_attention_prefill(void* out, int out_dtype, const void*
   const int group = num_heads / num_kv_heads;
   if (group > pf::kRows || pf::kRows % group != 0)
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_prefill: group %d does not divide 128", group);
-  if (num_kv_heads >= (1 << 23) || max_context_len >= (1 << 27))
+  if (num_kv_heads >= (1 << 15) || max_context_len >= (1 << 25))
     return set_error(PKV_ERR_INVALID, "paged_attention_prefill: sizes out of range");
   if (static_cast<int64_t>(num_blocks) * num_kv_heads * block_size > (static_cast<int64_t>(1) << 31))
     return set_error(PKV_ERR_INVALID, "paged_attention_prefill: pool too large");
@@ -752,6 +811,7 @@ extern "C" int pkv_paged_attention_prefill(void* out, int out_dtype, const void*
   a.num_blocks = num_blocks;
   a.group = group;
   a.group_shift = __builtin_ctz(static_cast<unsigned>(group));
+  a.tile_tokens = pf::kRows / group;
   a.scale_log2 = scale * 1.4426950408889634f;
   const uint64_t pool_rows = static_cast<uint64_t>(num_blocks) * num_kv_heads * block_size;
   int rc = pf::encode_kv_map(&args.tm_k, key_cache, pool_rows, "key_cache");

@@ -9,27 +9,30 @@
 // Unlike decode, the query side is dense.  A query tile is 128 rows = 128 / g tokens
 // x the g query heads of one kv head (row m = token * g + head).  A CTA holds TWO
 // consecutive query tiles (A and B) of one (sequence, kv head) and streams the K/V
-// pages once for both, 64 keys per stage:
-//   S_t[128 x 64]  = Q_t[128 x D] · K[64 x D]ᵀ      (A = Q_t, B = K; K-major, TMA-swizzled)
+// pages once for both, 128 keys per stage:
+//   S_t[128 x 128] = Q_t[128 x D] · K[128 x D]ᵀ     (A = Q_t in shared memory, B = K;
+//                                                    both K-major, TMA-swizzled)
 //   online softmax of each row (one thread per TMEM lane; causal mask on the diagonal)
-//   O_t[128 x D]  += P_t[128 x 64] · V[64 x D]      (A = P_t, K-major, written by the
-//                                                     softmax threads; B = V, MN-major)
-// Sharing a K/V stage between two tiles doubles the math per byte staged.  P is
-// double-buffered per tile, so a softmax group writes P of stage n+1 while the
-// tensor cores still multiply P of stage n: the MMA's issue-to-completion latency
-// stays off the per-stage critical path.
+//   O_t[128 x D]  += P_t[128 x 128] · V[128 x D]    (A = P_t in TENSOR memory, written
+//                                                    over S_t by the softmax threads;
+//                                                    B = V, MN-major)
+// Shared-memory bandwidth is what bounds these MMAs: keeping P in tensor memory and
+// using 128-wide S tiles leaves only Q, K and V to cross shared memory.
 //
-// Tensor memory (512 columns): S of tile t double-buffered in columns t*128 + {0, 64},
-// O of tile t in 256 + t*128.  O is rescaled in tensor memory only when a row's
-// maximum grows by more than 2^8; P is rounded to bf16 for the MMA and the row sums
-// add the same rounded values.
+// Tensor memory (512 columns): S_t / P_t in columns t*128 .. t*128+127 (P_t, bf16,
+// takes the first 64), O_t in 256 + t*128.  Per tile the MMA order is
+// ... S_t(n) -> [softmax] -> O_t += P_t(n)·V(n) -> S_t(n+1) ..., so S_t(n+1) never
+// overwrites P_t(n) before its P·V has read it, and once a softmax group sees S_t(n+1)
+// every earlier MMA of the tile is complete (a commit covers all prior MMAs), so O_t
+// may be rescaled without a further wait.  O is rescaled only when a row's maximum
+// grows by more than 2^8; P is rounded to bf16 and the row sums add the same values.
 //
 // Work item = (pair of query tiles, kv head), from a plan ordered longest sequence
 // first with every tile pair of a sequence adjacent, so items that read the same
 // K/V pages run at the same time and share them through L2.  CTAs are persistent and
 // take items from a counter.  Roles: warps 0-3 softmax + epilogue of tile A, warps
-// 4-7 of tile B, warp 8 TMA producer, warp 9 MMA issuer.  Per-stage metadata travels
-// in its own ring, so the softmax warps never wait for a V tile they do not touch.
+// 4-7 of tile B, warp 8 TMA producer (K one stage ahead of V), warp 9 MMA issuer (a
+// fixed order with blocking waits).  Per-stage metadata travels in its own ring.
 // Every wait is bounded; on a timeout the CTA flags PKV_DEV_TIMEOUT, lets its copies
 // land, waits for its MMAs, frees its tensor memory and exits.
 #include <cuda.h>
@@ -48,39 +51,45 @@ namespace pf {
 using tc::fast_exp2;
 
 constexpr int kRows = 128;                  // query rows per tile (MMA M)
-constexpr int kKeys = 64;                   // keys per stage
+constexpr int kKeys = 128;                  // keys per stage (MMA N of S, K of P·V)
 constexpr int kD = 128;                     // head_dim of this path
-constexpr int kQHalf = kRows * 128;         // one 64-column half of a 128-row bf16 tile: 16 KiB
-constexpr int kQBytes = 2 * kQHalf;         // a query tile: 32 KiB
-constexpr int kKvHalf = kKeys * 128;        // one 64-column half of a 64-row K or V tile: 8 KiB
-constexpr int kKvBytes = 2 * kKvHalf;       // 16 KiB
-constexpr int kPBytes = kRows * kKeys * 2;  // P of one tile: 128 rows x 128 bytes
+constexpr int kHalf = 128 * 128;            // one 64-column half of a 128-row bf16 tile: 16 KiB
+constexpr int kTileBytes = 2 * kHalf;       // a Q, K or V tile: 32 KiB
 constexpr int kChunk = 16;                  // key rows per TMA box (a 16-row slice of one block)
-constexpr int kStages = 3;
+constexpr int kChunks = kKeys / kChunk;     // 8
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
 constexpr int kMetaSlots = 8;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;              // 3 warpgroups; warps 10-11 only lend registers
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); the
+// producer/MMA warpgroup drops to 88 and the two softmax warpgroups rise to 208:
+// 128 x (208 + 208 + 88) = 64512 <= 64512, and per scheduler (one warp of each
+// group) 32 x 504 = 16128 <= 16384 registers.
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsControl = 88;
+static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;
 
 // shared memory (offsets from a 1024-aligned base)
-constexpr int kOffQ = 0;                                  // [2 tiles][32 KiB]
-constexpr int kOffP = kOffQ + 2 * kQBytes;                // [2 tiles][2 buffers][16 KiB]
-constexpr int kOffKV = kOffP + 4 * kPBytes;               // [3 stages][K 16 KiB | V 16 KiB]
-constexpr int kOffMeta = kOffKV + kStages * 2 * kKvBytes; // [8] int4
+constexpr int kOffQ = 0;                                   // [2 tiles]
+constexpr int kOffK = kOffQ + 2 * kTileBytes;              // [3 stages]
+constexpr int kOffV = kOffK + kKStages * kTileBytes;       // [2 stages]
+constexpr int kOffMeta = kOffV + kVStages * kTileBytes;    // [8] int4
 constexpr int kOffBar = kOffMeta + kMetaSlots * 16;
-constexpr int kBars = 2 + 3 * kStages + 2 * kMetaSlots + 4 + 4 + 4 + 4 + 1;
+constexpr int kBars = 2 + 2 * kKStages + 2 * kVStages + 2 * kMetaSlots + 2 + 2 + 2 + 1;
 constexpr int kOffMisc = kOffBar + kBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;          // + slack to align the base
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;           // + slack to align the base
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 
 // Stage metadata: x = packed row of tile A's first token, y = its position,
 // z = tokens of tile A | tokens of tile B << 8 | kv head << 16,
-// w = stage index in the item | chunk mask << 20 | flags.
-constexpr int kFirst = 1 << 24, kLast = 1 << 25, kEnd = 1 << 26;
+// w = stage index in the item (18 bits) | chunk mask << 18 | flags.
+constexpr int kFirst = 1 << 26, kLast = 1 << 27, kEnd = 1 << 28;
 
 struct PrefillArgs {
   void* out;
@@ -113,22 +122,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_buf = smem + kOffQ;
-  unsigned char* p_buf = smem + kOffP;
-  unsigned char* kv_ring = smem + kOffKV;
+  unsigned char* k_ring = smem + kOffK;
+  unsigned char* v_ring = smem + kOffV;
   int4* meta = reinterpret_cast<int4*>(smem + kOffMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;                        // [stage]
-  uint64_t* v_full = k_full + kStages;                // [stage]
-  uint64_t* kv_empty = v_full + kStages;              // [stage]
-  uint64_t* meta_full = kv_empty + kStages;           // [8]
-  uint64_t* meta_free = meta_full + kMetaSlots;       // [8]
-  uint64_t* s_full = meta_free + kMetaSlots;          // [tile][buffer]
-  uint64_t* s_free = s_full + 4;                      // [tile][buffer]
-  uint64_t* p_full = s_free + 4;                      // [tile][P buffer]
-  uint64_t* o_bar = p_full + 4;                       // [tile][P buffer]: that buffer's P·V done
-  uint64_t* drain = o_bar + 4;                        // the MMA thread's last commit
+  uint64_t* k_full = bars + 2;                        // [K stage]
+  uint64_t* k_empty = k_full + kKStages;              // [K stage]
+  uint64_t* v_full = k_empty + kKStages;              // [V stage]
+  uint64_t* v_empty = v_full + kVStages;              // [V stage]
+  uint64_t* meta_full = v_empty + kVStages;           // [meta slot]
+  uint64_t* meta_free = meta_full + kMetaSlots;       // [meta slot]
+  uint64_t* s_full = meta_free + kMetaSlots;          // [tile]: S_t of the stage is in tensor memory
+  uint64_t* p_full = s_full + 2;                      // [tile]: P_t of the stage is in tensor memory
+  uint64_t* o_bar = p_full + 2;                       // [tile]: O_t += P_t·V of the stage done
+  uint64_t* drain = o_bar + 2;                        // the MMA thread's last commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -139,22 +148,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < kMetaSlots; ++s) {
       mbar_init(&meta_full[s], 1);
       mbar_init(&meta_free[s], kSoftmaxWarps);
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);  // one arrival per warp of the tile's group
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&p_full[i], 4);
-      mbar_init(&o_bar[i], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 4);  // one arrival per warp of the tile's group
+      mbar_init(&o_bar[t], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -165,14 +174,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
   auto fail = [&]() {
     *abort_flag = 1;
     set_status(a.status, PKV_DEV_TIMEOUT);
   };
 
+  if (warp >= kProducerWarp) {
+  // The control warpgroup gives registers back; the branch is uniform per warpgroup,
+  // as setmaxnreg requires, and dominates the code that runs with the new count.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == kProducerWarp) {
     // ================= producer =================
+    // Stages form one stream across items.  K of stage n+1 (with its metadata) is
+    // issued before V of stage n, so the QK side runs a stage ahead; at an item
+    // boundary V of the old item goes first, then the new item's queries.
     const uint64_t pol_q = l2_policy_evict_first();
     const uint64_t pol_kv = l2_policy_evict_normal();  // every tile pair of the sequence re-reads these pages
     int* work_counter = const_cast<int*>(a.plan_count) + 1;
@@ -181,121 +196,164 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       if (lane == 0) v = atomicAdd(work_counter, 1);
       return __shfl_sync(0xffffffffu, v, 0);
     };
-    int n = 0, q_loads = 0;  // stages issued, query loads issued
     bool failed = false;
-    // Claim stage slot n: its K/V buffers free (the pair's P·V of stage n-3 done) and
-    // its metadata slot read by every softmax warp (stage n-8).
-    auto acquire = [&]() -> bool {
-      bool ok = true;
-      if (n >= kStages) ok = mbar_wait(&kv_empty[n % kStages], ((n / kStages) - 1) & 1);
-      if (ok && n >= kMetaSlots) ok = mbar_wait(&meta_free[n % kMetaSlots], ((n / kMetaSlots) - 1) & 1);
-      if (!ok) fail();
-      return ok;
-    };
-    for (int64_t item = grab(); item < n_items && !failed && !*abort_flag; item = grab()) {
-      const int4 e = a.entries[item / a.num_kv_heads];
-      const int kvh = static_cast<int>(item % a.num_kv_heads);
-      const int row0 = e.x, pos0 = e.y, ntok_a = e.z & 0xff, ntok_b = (e.z >> 8) & 0xff, seq = e.w;
-      const int nkeys = pos0 + ntok_a + ntok_b;
-      const int nst = (nkeys + kKeys - 1) / kKeys;
-      // queries: the previous item's last S = Q·Kᵀ must be done with the buffers
-      if (q_loads > 0 && !mbar_wait(q_empty, (q_loads - 1) & 1)) {
+    auto wait_slot = [&](uint64_t* bar, int fills, int depth) -> bool {
+      if (failed) return false;
+      if (fills >= depth && !mbar_wait(bar, ((fills / depth) - 1) & 1)) {
         fail();
         failed = true;
-        break;
       }
+      return !failed;
+    };
+    // the item whose stages the K side is issuing
+    int64_t item = grab();
+    int kvh = 0, row0 = 0, pos0 = 0, ntok_a = 0, ntok_b = 0, nkeys = 0, nst = 0, j = 0;
+    const int32_t* table = nullptr;
+    int tab_cur = -1, tab_nxt = -1, win = 0;
+    // Table entries come 32 slices (4 stages) at a time, one window ahead: lane l
+    // holds the physical block of slice 32 w + l of window w.
+    auto load_window = [&](int w) -> int {
+      const int kp = (w * 32 + lane) * kChunk;
+      return kp < nkeys ? __ldg(table + kp / a.block_size) : -1;
+    };
+    auto start_item = [&]() {
+      const int4 e = a.entries[item / a.num_kv_heads];
+      kvh = static_cast<int>(item % a.num_kv_heads);
+      row0 = e.x;
+      pos0 = e.y;
+      ntok_a = e.z & 0xff;
+      ntok_b = (e.z >> 8) & 0xff;
+      nkeys = pos0 + ntok_a + ntok_b;
+      nst = (nkeys + kKeys - 1) / kKeys;
+      j = 0;
+      table = a.block_tables + static_cast<int64_t>(e.w) * a.max_blocks;
+      win = 0;
+      tab_cur = load_window(0);
+      tab_nxt = load_window(1);
+    };
+    int kn = 0, vn = 0, q_loads = 0;  // K fills, V fills, query loads issued
+    auto load_q = [&]() -> bool {
+      if (q_loads > 0 && !wait_slot(q_empty, q_loads, 1)) return false;
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, (ntok_b > 0 ? 2 : 1) * kQBytes);
+        mbar_arrive_expect_tx(q_full, (ntok_b > 0 ? 2 : 1) * kTileBytes);
         tc::tma_load_3d(q_buf, &args.tm_q, 0, kvh * g, row0, q_full, pol_q);
-        tc::tma_load_3d(q_buf + kQHalf, &args.tm_q, 64, kvh * g, row0, q_full, pol_q);
+        tc::tma_load_3d(q_buf + kHalf, &args.tm_q, 64, kvh * g, row0, q_full, pol_q);
         if (ntok_b > 0) {
-          tc::tma_load_3d(q_buf + kQBytes, &args.tm_q, 0, kvh * g, row0 + a.tile_tokens, q_full, pol_q);
-          tc::tma_load_3d(q_buf + kQBytes + kQHalf, &args.tm_q, 64, kvh * g, row0 + a.tile_tokens, q_full, pol_q);
+          tc::tma_load_3d(q_buf + kTileBytes, &args.tm_q, 0, kvh * g, row0 + a.tile_tokens, q_full, pol_q);
+          tc::tma_load_3d(q_buf + kTileBytes + kHalf, &args.tm_q, 64, kvh * g, row0 + a.tile_tokens, q_full, pol_q);
         }
       }
       ++q_loads;
-      const int32_t* table = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks;
-      // Table entries come 32 slices (8 stages) at a time, one window ahead: lane l
-      // holds the physical block of slice 32 w + l of window w.
-      auto load_window = [&](int w) -> int {
-        const int kp = (w * 32 + lane) * kChunk;
-        return kp < nkeys ? __ldg(table + kp / a.block_size) : -1;
-      };
-      int win = 0;
-      int tab_cur = load_window(0);
-      int tab_nxt = load_window(1);
-      for (int j = 0; j < nst; ++j) {
-        if (j / 8 != win) {
-          ++win;
-          tab_cur = tab_nxt;
-          tab_nxt = load_window(win + 1);
-        }
-        const int kbase = j * kKeys;
-        const int nvalid = min(kKeys, nkeys - kbase);
-        const int nch = (nvalid + kChunk - 1) / kChunk;
-        const int kp = kbase + lane * kChunk;  // this lane's 16-row slice (lanes < nch)
-        const bool mine = lane < nch;
-        int phys = __shfl_sync(0xffffffffu, tab_cur, (j % 8) * 4 + (lane & 3));
-        if (!mine) phys = -1;
-        const bool ok = mine && phys >= 0 && phys < a.num_blocks;
-        const uint32_t mask = __ballot_sync(0xffffffffu, ok) & 0xfu;
-        if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
-        const int row = (phys * a.num_kv_heads + kvh) * a.block_size + kp % a.block_size;
-        if (!acquire()) {
-          failed = true;
-          break;
-        }
-        const int st = n % kStages;
-        unsigned char* kd = kv_ring + st * 2 * kKvBytes + lane * kChunk * 128;
-        if (lane == 0) {
-          meta[n % kMetaSlots] = make_int4(row0, pos0, ntok_a | (ntok_b << 8) | (kvh << 16),
-                                           j | static_cast<int>(mask << 20) | (j == 0 ? kFirst : 0) |
-                                               (j == nst - 1 ? kLast : 0));
-          mbar_arrive(&meta_full[n % kMetaSlots]);
-          mbar_arrive_expect_tx(&k_full[st], __popc(mask) * kChunk * 256);
-        }
-        __syncwarp();
-        if (ok) {
-          tc::tma_load_2d(kd, &args.tm_k, 0, row, &k_full[st], pol_kv);
-          tc::tma_load_2d(kd + kKvHalf, &args.tm_k, 64, row, &k_full[st], pol_kv);
-        }
-        if (lane == 0) mbar_arrive_expect_tx(&v_full[st], __popc(mask) * kChunk * 256);
-        __syncwarp();
-        if (ok) {
-          tc::tma_load_2d(kd + kKvBytes, &args.tm_v, 0, row, &v_full[st], pol_kv);
-          tc::tma_load_2d(kd + kKvBytes + kKvHalf, &args.tm_v, 64, row, &v_full[st], pol_kv);
-        }
-        ++n;
+      return true;
+    };
+    // K (and metadata) of the cursor's stage j; returns this lane's V source row
+    // and the slice mask through the references, for the matching V fill.
+    auto issue_k = [&](int& vrow, uint32_t& vmask) -> bool {
+      if (j / 4 != win) {
+        ++win;
+        tab_cur = tab_nxt;
+        tab_nxt = load_window(win + 1);
+      }
+      const int kbase = j * kKeys;
+      const int nvalid = min(kKeys, nkeys - kbase);
+      const int nch = (nvalid + kChunk - 1) / kChunk;
+      const int kp = kbase + lane * kChunk;  // this lane's 16-row slice (lanes < nch)
+      const bool mine = lane < nch;
+      int phys = __shfl_sync(0xffffffffu, tab_cur, (j % 4) * 8 + (lane & 7));
+      if (!mine) phys = -1;
+      const bool ok = mine && phys >= 0 && phys < a.num_blocks;
+      const uint32_t mask = __ballot_sync(0xffffffffu, ok) & 0xffu;
+      if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
+      vrow = ok ? (phys * a.num_kv_heads + kvh) * a.block_size + kp % a.block_size : -1;
+      vmask = mask;
+      if (!wait_slot(&k_empty[kn % kKStages], kn, kKStages)) return false;
+      if (!wait_slot(&meta_free[kn % kMetaSlots], kn, kMetaSlots)) return false;
+      const int ks = kn % kKStages;
+      if (lane == 0) {
+        meta[kn % kMetaSlots] = make_int4(row0, pos0, ntok_a | (ntok_b << 8) | (kvh << 16),
+                                          j | static_cast<int>(mask << 18) | (j == 0 ? kFirst : 0) |
+                                              (j == nst - 1 ? kLast : 0));
+        mbar_arrive(&meta_full[kn % kMetaSlots]);
+        mbar_arrive_expect_tx(&k_full[ks], __popc(mask) * kChunk * 256);
+      }
+      __syncwarp();
+      if (ok) {
+        unsigned char* kd = k_ring + ks * kTileBytes + lane * kChunk * 128;
+        tc::tma_load_2d(kd, &args.tm_k, 0, vrow, &k_full[ks], pol_kv);
+        tc::tma_load_2d(kd + kHalf, &args.tm_k, 64, vrow, &k_full[ks], pol_kv);
+      }
+      ++kn;
+      return true;
+    };
+    auto issue_v = [&](int vrow, uint32_t vmask) -> bool {
+      if (!wait_slot(&v_empty[vn % kVStages], vn, kVStages)) return false;
+      const int vs = vn % kVStages;
+      if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], __popc(vmask) * kChunk * 256);
+      __syncwarp();
+      if (vrow >= 0) {
+        unsigned char* vd = v_ring + vs * kTileBytes + lane * kChunk * 128;
+        tc::tma_load_2d(vd, &args.tm_v, 0, vrow, &v_full[vs], pol_kv);
+        tc::tma_load_2d(vd + kHalf, &args.tm_v, 64, vrow, &v_full[vs], pol_kv);
+      }
+      ++vn;
+      return true;
+    };
+    int pend_row = -1;
+    uint32_t pend_mask = 0;
+    bool pending = false;  // V of the last K-issued stage still to go
+    if (item < n_items) {
+      start_item();
+      if (load_q() && issue_k(pend_row, pend_mask)) pending = true;
+    }
+    while (pending && !failed && !*abort_flag) {
+      // advance the cursor to the next stage
+      ++j;
+      bool new_item = false;
+      if (j == nst) {
+        item = grab();
+        new_item = true;
+      }
+      int nrow;
+      uint32_t nmask;
+      if (new_item) {
+        if (!issue_v(pend_row, pend_mask)) break;
+        pending = false;
+        if (item >= n_items) break;
+        start_item();
+        if (!load_q() || !issue_k(pend_row, pend_mask)) break;
+        pending = true;
+      } else {
+        if (!issue_k(nrow, nmask)) break;
+        if (!issue_v(pend_row, pend_mask)) break;
+        pend_row = nrow;
+        pend_mask = nmask;
       }
     }
-    if (!failed && !*abort_flag && acquire()) {
-      // end-of-stream: a stage with no data
+    if (!failed && !*abort_flag && wait_slot(&k_empty[kn % kKStages], kn, kKStages) &&
+        wait_slot(&meta_free[kn % kMetaSlots], kn, kMetaSlots)) {
+      // end-of-stream: a K fill and metadata with no data
       if (lane == 0) {
-        meta[n % kMetaSlots] = make_int4(0, 0, 0, kEnd);
-        mbar_arrive(&meta_full[n % kMetaSlots]);
-        mbar_arrive_expect_tx(&k_full[n % kStages], 0);
-        mbar_arrive_expect_tx(&v_full[n % kStages], 0);
+        meta[kn % kMetaSlots] = make_int4(0, 0, 0, kEnd);
+        mbar_arrive(&meta_full[kn % kMetaSlots]);
+        mbar_arrive_expect_tx(&k_full[kn % kKStages], 0);
       }
-      ++n;
+      ++kn;
       __syncwarp();
     }
     // Let this CTA's last copies land before the final barrier.
-    for (int k = max(0, n - kStages); k < n; ++k) {
-      mbar_wait(&k_full[k % kStages], (k / kStages) & 1);
-      mbar_wait(&v_full[k % kStages], (k / kStages) & 1);
-    }
+    for (int k = max(0, kn - kKStages); k < kn; ++k) mbar_wait(&k_full[k % kKStages], (k / kKStages) & 1);
+    for (int k = max(0, vn - kVStages); k < vn; ++k) mbar_wait(&v_full[k % kVStages], (k / kVStages) & 1);
     if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1);
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer (one thread) =================
-    // A fixed order with blocking waits, one barrier at a time: S of stage n+1 for
-    // both tiles first (the tensor cores work while the softmax groups handle stage
-    // n), then P·V of stage n as each group's P lands.  At an item boundary P·V of
-    // the old item's last stage goes first, so its epilogue is not held up by the
-    // next item's query load.
+    // Fixed order with blocking waits, one barrier at a time:
+    //   S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) S_A(2) ...
+    // P·V of a tile goes before its next S (P lives in S's columns), and the other
+    // tile's MMAs fill the tensor pipe while one group runs its softmax.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc::instr_desc(kRows, kKeys, false, false);
       constexpr uint32_t idesc_pv = tc::instr_desc(kRows, kD, false, true);
-      int qc[2] = {0, 0}, pc[2] = {0, 0};  // per tile: stages whose S / P·V were issued
+      int sc[2] = {0, 0}, pc[2] = {0, 0};  // per tile: S and P·V issued
       int q_items = 0;
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -305,70 +363,74 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         return ok;
       };
-      // Issue S_t = Q_t·Kᵀ of stage n for every tile present; false at end of stream.
-      auto issue_qk = [&](int n) -> bool {
-        if (!wait(&k_full[n % kStages], (n / kStages) & 1)) return false;
-        const int4 mt = meta[n % kMetaSlots];
-        if (mt.w & kEnd) return false;
-        const bool has_b = ((mt.z >> 8) & 0xff) != 0;
-        if (mt.w & kFirst) {
+      auto stage_meta = [&](int n) -> int4 { return meta[n % kMetaSlots]; };
+      auto has_b = [](const int4& mt) { return ((mt.z >> 8) & 0xff) != 0; };
+      // S_t = Q_t·Kᵀ of stage n (K landed, queries of a new item landed).
+      auto issue_s = [&](int n, int t, const int4& mt) -> bool {
+        if (t == 0 && (mt.w & kFirst)) {
           if (!wait(q_full, q_items & 1)) return false;
           ++q_items;
         }
-        const uint32_t k_addr = smem_addr(kv_ring + (n % kStages) * 2 * kKvBytes);
-        for (int t = 0; t < (has_b ? 2 : 1); ++t) {
-          const int b = qc[t] & 1;
-          if (qc[t] >= 2 && !wait(&s_free[t * 2 + b], ((qc[t] >> 1) - 1) & 1)) return false;
-          tc::tc_fence_after();
-          const uint32_t q_addr = smem_addr(q_buf + t * kQBytes);
+        tc::tc_fence_after();
+        const uint32_t q_addr = smem_addr(q_buf + t * kTileBytes);
+        const uint32_t k_addr = smem_addr(k_ring + (n % kKStages) * kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            tc::umma(tmem + t * 128 + b * kKeys,
-                     tc::smem_desc_sw128(q_addr + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024),
-                     tc::smem_desc_sw128(k_addr + (kk >> 2) * kKvHalf + (kk & 3) * 32, 16, 1024), idesc_qk, kk > 0);
-          }
-          tc::umma_commit(&s_full[t * 2 + b]);
-          ++qc[t];
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          tc::umma(tmem + t * 128, tc::smem_desc_sw128(q_addr + off, 16, 1024),
+                   tc::smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0);
         }
-        if (mt.w & kLast) tc::umma_commit(q_empty);
+        tc::umma_commit(&s_full[t]);
+        ++sc[t];
+        const bool stage_done = t == 1 || !has_b(mt);
+        if (stage_done) {
+          tc::umma_commit(&k_empty[n % kKStages]);
+          if (mt.w & kLast) tc::umma_commit(q_empty);
+        }
         return true;
       };
-      // Issue O_t += P_t·V of stage n for every tile present, then release the stage.
-      auto issue_pv = [&](int n) -> bool {
-        const int4 mt = meta[n % kMetaSlots];
-        const bool has_b = ((mt.z >> 8) & 0xff) != 0;
-        if (!wait(&v_full[n % kStages], (n / kStages) & 1)) return false;
-        const uint32_t v_addr = smem_addr(kv_ring + (n % kStages) * 2 * kKvBytes + kKvBytes);
-        for (int t = 0; t < (has_b ? 2 : 1); ++t) {
-          const int pb = pc[t] & 1;
-          if (!wait(&p_full[t * 2 + pb], (pc[t] >> 1) & 1)) return false;
-          tc::tc_fence_after();
-          const uint32_t p_addr = smem_addr(p_buf + (t * 2 + pb) * kPBytes);
+      // O_t += P_t·V of stage n (P in tensor memory, V landed).
+      auto issue_pv = [&](int n, int t, const int4& mt) -> bool {
+        if (t == 0 && !wait(&v_full[n % kVStages], (n / kVStages) & 1)) return false;
+        if (!wait(&p_full[t], pc[t] & 1)) return false;
+        tc::tc_fence_after();
+        const uint32_t v_addr = smem_addr(v_ring + (n % kVStages) * kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < kKeys / 16; ++kk) {
-            // P: K-major, 128-byte swizzle; V: MN-major, 16 key rows per step
-            tc::umma(tmem + kColO + t * 128, tc::smem_desc_sw128(p_addr + kk * 32, 16, 1024),
-                     tc::smem_desc_sw128(v_addr + kk * 2048, kKvHalf, 1024), idesc_pv, kk > 0 || !(mt.w & kFirst));
-          }
-          tc::umma_commit(&o_bar[t * 2 + pb]);
-          ++pc[t];
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          // P: 8 columns (16 keys) per step; V: MN-major, 16 key rows per step
+          tc::umma_ts(tmem + kColO + t * 128, tmem + t * 128 + kk * 8,
+                      tc::smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024), idesc_pv,
+                      kk > 0 || !(mt.w & kFirst));
         }
-        tc::umma_commit(&kv_empty[n % kStages]);
+        tc::umma_commit(&o_bar[t]);
+        ++pc[t];
+        if (t == 1 || !has_b(mt)) tc::umma_commit(&v_empty[n % kVStages]);
         return true;
       };
-      if (issue_qk(0)) {
-        for (int n = 0; ok; ++n) {
-          // stage n+1: does it start a new item (or end the stream)?
-          const bool next_ready = wait(&k_full[(n + 1) % kStages], ((n + 1) / kStages) & 1);
-          if (!next_ready) break;
-          const int wnext = meta[(n + 1) % kMetaSlots].w;
-          if ((wnext & kEnd) || (wnext & kFirst)) {
-            if (!issue_pv(n)) break;
-            if ((wnext & kEnd) || !issue_qk(n + 1)) break;
-          } else {
-            if (!issue_qk(n + 1)) break;
-            if (!issue_pv(n)) break;
-          }
+      // stage 0
+      bool more = wait(&k_full[0], 0) && !(stage_meta(0).w & kEnd);
+      if (more) {
+        const int4 m0 = stage_meta(0);
+        more = issue_s(0, 0, m0) && (!has_b(m0) || issue_s(0, 1, m0));
+      }
+      for (int n = 0; more && ok; ++n) {
+        const int4 mt = stage_meta(n);
+        // the next stage's K (or the end marker)
+        if (!wait(&k_full[(n + 1) % kKStages], ((n + 1) / kKStages) & 1)) break;
+        const int4 mn = stage_meta(n + 1);
+        const bool next = !(mn.w & kEnd);
+        if (next && !(mn.w & kFirst)) {
+          // same item: interleave per tile
+          if (!issue_pv(n, 0, mt) || !issue_s(n + 1, 0, mn)) break;
+          if (has_b(mt) && !issue_pv(n, 1, mt)) break;
+          if (has_b(mn) && !issue_s(n + 1, 1, mn)) break;
+        } else {
+          // item boundary or end: finish this item's P·V first
+          if (!issue_pv(n, 0, mt)) break;
+          if (has_b(mt) && !issue_pv(n, 1, mt)) break;
+          if (!next) break;
+          if (!issue_s(n + 1, 0, mn)) break;
+          if (has_b(mn) && !issue_s(n + 1, 1, mn)) break;
         }
       }
       // every MMA this thread issued has finished before tensor memory is freed
@@ -376,7 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       mbar_wait(drain, 0);
     }
     __syncwarp();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ================= softmax warps: thread = query row of tile t = TMEM lane =================
     const int t = warp >> 2;                 // 0: tile A (warps 0-3), 1: tile B (warps 4-7)
     const int m = tid & 127;                 // row within the tile
@@ -384,14 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     const uint32_t col_s = t * 128, col_o = kColO + t * 128;
     float m_used = -INFINITY, lsum = 0.f;
     bool has_pv = false;
-    int c = 0;  // stages of this tile processed (S and P buffers)
-    // P buffer k's P·V: uses issued and completions observed (wait for each in order)
-    int uses[2] = {0, 0}, seen[2] = {0, 0};
-    auto wait_pv = [&](int k) -> bool {
-      if (seen[k] == uses[k]) return true;
-      seen[k] = uses[k];
-      return mbar_wait(&o_bar[t * 2 + k], (uses[k] - 1) & 1);
-    };
+    int c = 0;  // stages of this tile processed (phases of s_full / p_full / o_bar)
     for (int n = 0;; ++n) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(&meta_full[n % kMetaSlots], (n / kMetaSlots) & 1));
       const int4 mt = meta[n % kMetaSlots];
@@ -404,8 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int ntok_a = mt.z & 0xff, ntok_b = (mt.z >> 8) & 0xff, kvh = mt.z >> 16;
       const int ntok = t == 0 ? ntok_a : ntok_b;
       if (ntok == 0) continue;  // tile B absent from this item
-      const int j = mt.w & 0xfffff;
-      const uint32_t mask = (mt.w >> 20) & 0xfu;
+      const int j = mt.w & 0x3ffff;
+      const uint32_t mask = (mt.w >> 18) & 0xffu;
       const bool first = mt.w & kFirst, last = mt.w & kLast;
       const int row0 = mt.x + t * a.tile_tokens, pos0 = mt.y + t * a.tile_tokens;
       if (first) {
@@ -418,33 +475,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int limit = pos0 + (valid_row ? tl : ntok - 1);  // last visible key position
       const int kbase = j * kKeys;
       const int nvalid = min(kKeys, mt.y + ntok_a + ntok_b - kbase);
-      const bool partial = nvalid < kKeys || mask != 0xfu;
-      if (t == 0 && partial) {
+      if (t == 0 && (nvalid < kKeys || mask != 0xffu)) {
         // V rows past the context or in a slice that was not loaded may hold anything
         // (even NaN): zero them once the stage's copies have landed, before P·V.
-        const int st = n % kStages;
-        ok &= mbar_wait(&v_full[st], (n / kStages) & 1);
-        if (m < kKeys && (m >= nvalid || !((mask >> (m / kChunk)) & 1u))) {
-          unsigned char* vrow = kv_ring + st * 2 * kKvBytes + kKvBytes + m * 128;
+        const int vs = n % kVStages;
+        ok &= mbar_wait(&v_full[vs], (n / kVStages) & 1);
+        if (m >= nvalid || !((mask >> (m / kChunk)) & 1u)) {
+          unsigned char* vrow = v_ring + vs * kTileBytes + m * 128;
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int q = 0; q < 8; ++q) reinterpret_cast<uint4*>(vrow + h * kKvHalf)[q] = make_uint4(0, 0, 0, 0);
+            for (int q = 0; q < 8; ++q) reinterpret_cast<uint4*>(vrow + h * kHalf)[q] = make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
       }
-      // ---- S row
-      const int b = c & 1;
-      ok &= mbar_wait(&s_full[t * 2 + b], (c >> 1) & 1);
+      // ---- S row (its arrival also means every earlier MMA of this tile is done)
+      ok &= mbar_wait(&s_full[t], c & 1);
       tc::tc_fence_after();
       float s[kKeys];
-      tc::tmem_load32f_nowait(tmem + lane_base + col_s + b * kKeys, s);
-      tc::tmem_load32f_nowait(tmem + lane_base + col_s + b * kKeys + 32, s + 32);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tc::tmem_load32f_nowait(tmem + lane_base + col_s + q4 * 32, s + q4 * 32);
       tc::tmem_wait_ld();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[t * 2 + b]);
       // ---- causal / context mask and the row maximum
-      if (!(kbase + kKeys - 1 <= pos0 && mask == 0xfu)) {
+      if (!(kbase + kKeys - 1 <= pos0 && mask == 0xffu)) {
 #pragma unroll
         for (int k = 0; k < kKeys; ++k) {
           const bool vis = kbase + k <= limit && ((mask >> (k / kChunk)) & 1u);
@@ -459,11 +512,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mxs = mx * a.scale_log2;
-      const int pb = c & 1;
-      ok &= wait_pv(pb);  // this P buffer's previous P·V (two stages back) is done
       // A row rescales only when its maximum grew past the threshold; the tensor-memory
       // accesses are warp-collective, so the warp rescales together (alpha = 1 for the
-      // rows that keep their maximum).
+      // rows that keep their maximum).  Every P·V of the tile is complete here.
       const bool need = mxs > m_used + kRescaleLog2;
       float alpha = 1.f;
       if (need) {
@@ -472,58 +523,48 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         m_used = m_new;
       }
       if (has_pv && __any_sync(0xffffffffu, need)) {
-        ok &= wait_pv(pb ^ 1);  // O must hold every issued P·V before it is rescaled
-        tc::tc_fence_after();
-        uint32_t r[2][32];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          tc::tmem_load32_nowait(tmem + lane_base + col_o + h2 * 64, r[0]);
-          tc::tmem_load32_nowait(tmem + lane_base + col_o + h2 * 64 + 32, r[1]);
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t r[32];
+          tc::tmem_load32_nowait(tmem + lane_base + col_o + q4 * 32, r);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            r[0][k] = __float_as_uint(__uint_as_float(r[0][k]) * alpha);
-            r[1][k] = __float_as_uint(__uint_as_float(r[1][k]) * alpha);
-          }
-          tc::tmem_store32(tmem + lane_base + col_o + h2 * 64, r[0]);
-          tc::tmem_store32(tmem + lane_base + col_o + h2 * 64 + 32, r[1]);
+          for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+          tc::tmem_store32(tmem + lane_base + col_o + q4 * 32, r);
         }
-        tc::tmem_wait_st();
       }
       lsum *= alpha;
-      // ---- P = 2^(s * scale_log2 - m), bf16, written as the K-major swizzled A operand
+      // ---- P = 2^(s * scale_log2 - m) as bf16 pairs, stored over S (columns 0-63 of
+      //      the tile's block: keys 2i, 2i+1 in column i)
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const bool any = m_used != -INFINITY;
-      unsigned char* prow = p_buf + (t * 2 + pb) * kPBytes + m * 128;
       float ls8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) ls8[i] = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < kKeys / 8; ++c8) {
-        uint32_t w[4];
+      for (int h = 0; h < 4; ++h) {
+        uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float x0 = s[c8 * 8 + 2 * i], x1 = s[c8 * 8 + 2 * i + 1];
+        for (int i = 0; i < 16; ++i) {
+          const float x0 = s[h * 32 + 2 * i], x1 = s[h * 32 + 2 * i + 1];
           const float p0 = any ? fast_exp2(fmaf(x0, a.scale_log2, neg_m)) : 0.f;
           const float p1 = any ? fast_exp2(fmaf(x1, a.scale_log2, neg_m)) : 0.f;
           w[i] = pack_bf16x2(p0, p1);
-          ls8[2 * i] += bf16lo(w[i]);
-          ls8[2 * i + 1] += bf16hi(w[i]);
+          ls8[(2 * i) & 7] += bf16lo(w[i]);
+          ls8[(2 * i + 1) & 7] += bf16hi(w[i]);
         }
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (m & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        tc::tmem_store16(tmem + lane_base + col_s + h * 16, w);
       }
       lsum += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-      fence_proxy_async_smem();  // P and the zeroed V rows, before the MMA reads them
-      tc::tc_fence_before();     // the rescaled O, before the next P·V
+      tc::tmem_wait_st();
+      tc::tc_fence_before();     // P and the rescaled O, before the MMA reads them
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t * 2 + pb]);
-      ++uses[pb];
+      if (lane == 0) mbar_arrive(&p_full[t]);
       has_pv = true;
       ++c;
       if (last) {
-        // ---- epilogue: O / l of this row, once every P·V of the item is done
-        ok &= wait_pv(0);
-        ok &= wait_pv(1);
+        // ---- epilogue: O / l of this row, once the item's last P·V is done
+        ok &= mbar_wait(&o_bar[t], (c - 1) & 1);
         tc::tc_fence_after();
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         const int64_t orow = (static_cast<int64_t>(row0 + tl) * a.num_heads + kvh * g + (m & (g - 1))) * kD;

@@ -103,12 +103,12 @@ def test_prefill_argument_errors_before_any_device_work(pkv):
 
 
 def test_prefill_workspace_size(pkv):
-    # 256 bytes of counters + one 16-byte entry per query tile (upper bound: T / (128 / g) + B),
-    # rounded up to 256 bytes
+    # 256 bytes of counters + one 16-byte entry per pair of 128-row query tiles (upper
+    # bound: T / (2 * 128 / g) + B), rounded up to 256 bytes
     def up(x):
         return -(-x // 256) * 256
-    assert pkv.paged_attention_prefill_workspace_size(8, 4096, 40, 40) == 256 + up(16 * (32 + 8))
-    assert pkv.paged_attention_prefill_workspace_size(8, 4096, 64, 8) == 256 + up(16 * (256 + 8))
+    assert pkv.paged_attention_prefill_workspace_size(8, 4096, 40, 40) == 256 + up(16 * (16 + 8))
+    assert pkv.paged_attention_prefill_workspace_size(8, 4096, 64, 8) == 256 + up(16 * (128 + 8))
     assert pkv.paged_attention_prefill_workspace_size(1, 1, 128, 1) == 256 + up(16 * 2)
     with pytest.raises(pkv.PkvError):
         pkv.paged_attention_prefill_workspace_size(2, 10, 6, 2)

@@ -81,28 +81,33 @@ def measured_hbm_gbs():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest() -> str:
-    """Digest of the library sources; a recorded ncu traffic figure is only reported
-    while the kernels are the ones it was measured on."""
+# Sources each kernel family is compiled from: a recorded ncu traffic figure is only
+# reported while these files are the ones it was measured on.
+KERNEL_SOURCES = {
+    "decode": ["decode.cu", "decode_gqa_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
+    "prefill": ["prefill_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
+}
+
+
+def source_digest(kind: str = "decode") -> str:
     import hashlib
     h = hashlib.sha256()
-    for sub in (os.path.join("paged_kv_cache_423_b200", "csrc"), "include"):
-        d = os.path.join(ROOT, sub)
-        for f in sorted(os.listdir(d)):
-            h.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
+    d = os.path.join(ROOT, "paged_kv_cache_423_b200", "csrc")
+    for f in KERNEL_SOURCES[kind]:
+        h.update(f.encode())
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes (read + write) per decode launch from profiles/traffic.json, or None."""
+def recorded_traffic(key: str, kind: str = "decode"):
+    """DRAM bytes (read + write) per launch of the profiled kernel from profiles/traffic.json, or None."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            entry = json.load(f).get(workload)
+            entry = json.load(f).get(key)
     except Exception:
         return None
-    if not entry or entry.get("sources") != source_digest():
+    if not entry or entry.get("sources") != source_digest(kind):
         return None
     return int(entry["dram_bytes_per_launch"])
 
@@ -388,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
         "seq_steps_per_s": round(seq_steps, 1),
         "pct_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(dec_gbs / peak, 4), "traffic": recorded_traffic(w.name),
+                     "frac": round(dec_gbs / peak, 4), "traffic": recorded_traffic(w.name + ("+fp8" if kv8 else "")),
                      "algorithmic_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
                      "kernel": ("paged_attention_decode_fp8: plan + CUDA-core streaming kernel (e4m3 tiles)" if kv8
                                 else "paged_attention_decode: plan + tcgen05 kernel + split merge" if uses_tensor
@@ -864,7 +869,7 @@ def run_prefill(args, rank, world, local_rank):
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "pct_tensor_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(b.name),
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(b.name, "prefill"),
                      "algorithmic_flops_per_launch": pw.flops, "peak_kind": peak_kind,
                      "kernel": "paged_attention_prefill: plan + tcgen05 kernel",
                      "ms_per_launch": round(k_ms / args.steps, 4)},

@@ -223,8 +223,12 @@ PKV_API int pkv_reshape_and_cache_fp8(const void* key, const void* value, void* 
 /*
  * paged_attention_decode_fp8 — pkv_paged_attention_decode over an 8-bit pool: the
  * attention of the dequantised values (K_j = e4m3_value * k_scale[h], V_j likewise).
- * head_dim 128; CUDA cores (the e4m3 tiles are widened to f16 in registers, products
- * accumulate in fp32).  Workspace, splits and status bits as for
+ * head_dim 128.  path PKV_PATH_SIMT: CUDA cores (the e4m3 tiles are widened to f16
+ * in registers, products accumulate in fp32); PKV_PATH_TENSOR (2 <= group <= 16):
+ * the tiles are widened to f16 on chip and both products run on the tensor cores
+ * with fp32 accumulators (the queries are rounded to f16, after a 2^-16 scale when
+ * one of a kv head's queries reaches 2^15; P is rounded to f16); PKV_PATH_AUTO takes
+ * the tensor cores whenever they apply.  Workspace, splits and status bits as for
  * pkv_paged_attention_decode (size it with pkv_paged_attention_workspace_size).
  */
 PKV_API int pkv_paged_attention_decode_fp8(void* out, int out_dtype, const void* query, const void* key_cache,
@@ -232,8 +236,9 @@ PKV_API int pkv_paged_attention_decode_fp8(void* out, int out_dtype, const void*
                                            const int32_t* block_tables, int max_blocks_per_seq,
                                            const int32_t* context_lens, int max_context_len, int num_seqs,
                                            int num_heads, int num_kv_heads, int head_dim, int block_size,
-                                           int num_blocks, float scale, int partition_tokens, void* workspace,
-                                           size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
+                                           int num_blocks, float scale, int partition_tokens, int path,
+                                           void* workspace, size_t workspace_bytes, int32_t* status,
+                                           pkv_stream_t stream);
 
 /*
  * swap_blocks — the pool's overflow path (intelliparadigm article §4.2 OOM错误:

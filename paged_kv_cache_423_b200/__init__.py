@@ -80,7 +80,8 @@ _SIGNATURES = {
                                           c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
     "pkv_paged_attention_decode_fp8": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                                c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
-                                               c_int, c_float, c_int, c_void_p, c_size_t, c_void_p, c_void_p]),
+                                               c_int, c_float, c_int, c_int, c_void_p, c_size_t, c_void_p,
+                                               c_void_p]),
     "pkv_swap_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int64, c_void_p, c_void_p]),
     "pkv_bm_create": (c_void_p, [c_int, c_int, c_void_p]),
     "pkv_bm_create_with_swap_space": (c_void_p, [c_int, c_int, c_void_p, c_int]),
@@ -302,9 +303,11 @@ def reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_sc
 
 
 def paged_attention_decode_fp8(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, context_lens,
-                               max_context_len, scale, workspace, partition_tokens=0, status=None, stream=None):
+                               max_context_len, scale, workspace, partition_tokens=0, path=PATH_AUTO, status=None,
+                               stream=None):
     """Decode attention over 8-bit pools [NB, Hkv, bs, 128] uint8 with per-kv-head scales;
-    otherwise as paged_attention_decode (same workspace size)."""
+    otherwise as paged_attention_decode (same workspace size).  path: PATH_AUTO (tensor
+    cores for 2 <= group <= 16), PATH_SIMT or PATH_TENSOR."""
     torch = _torch()
     B, Hq, D = query.shape
     NB, Hkv, bs, D2 = key_cache.shape
@@ -321,7 +324,7 @@ def paged_attention_decode_fp8(out, query, key_cache, value_cache, k_scale, v_sc
         _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
         _ptr(block_tables, torch.int32, "block_tables"), int(block_tables.shape[1]),
         _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len), B, Hq, Hkv, D, bs, NB,
-        float(scale), int(partition_tokens), _ptr(workspace, None, "workspace"),
+        float(scale), int(partition_tokens), int(path), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
     _check(rc, "paged_attention_decode_fp8")
 

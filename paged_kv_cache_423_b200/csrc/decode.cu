@@ -820,7 +820,8 @@ extern "C" size_t pkv_paged_attention_workspace_size(int num_seqs, int num_heads
 }
 
 // Shared by the bf16 and the 8-bit entry points; `k_scale` != null selects the
-// 8-bit (e4m3) pool, which the CUDA-core kernel reads at head_dim 128.
+// 8-bit (e4m3) pool (head_dim 128), read by the CUDA-core kernel or, for grouped
+// query heads, by the tensor-core kernel that widens each tile to f16.
 static int decode_impl(void* out, int out_dtype, const void* query, const void* key_cache, const void* value_cache,
                        const float* k_scale, const float* v_scale, const int32_t* block_tables,
                        int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
@@ -845,9 +846,6 @@ static int decode_impl(void* out, int out_dtype, const void* query, const void* 
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: path %d", path);
   if (kv8 && head_dim != 128)
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_fp8: head_dim %d (only 128)", head_dim);
-  if (kv8 && path == PKV_PATH_TENSOR)
-    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_fp8: the 8-bit pool is read on CUDA cores");
-  if (kv8) path = PKV_PATH_SIMT;
   const int group = num_heads / num_kv_heads;
   if (path == PKV_PATH_TENSOR && !tensor_path_supports(group, head_dim))
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: tensor path needs 2 <= group <= 16 and head_dim 128"
@@ -915,6 +913,7 @@ static int decode_impl(void* out, int out_dtype, const void* query, const void* 
   int rc = launch_plan(a, context_lens, max_context_len, s);
   if (rc != PKV_OK) return rc;
   const bool out_f32 = out_dtype == PKV_DTYPE_F32;
+  if (kv8 && use_tensor) return launch_decode_tensor_fp8(a, head_dim, out_f32, s);
   if (kv8) return out_f32 ? launch_simt<128, true, true>(a, s) : launch_simt<128, false, true>(a, s);
   if (use_tensor) return launch_decode_tensor(a, head_dim, out_f32, s);
   if (head_dim == 128) return out_f32 ? launch_simt<128, true>(a, s) : launch_simt<128, false>(a, s);
@@ -940,12 +939,13 @@ extern "C" int pkv_paged_attention_decode_fp8(void* out, int out_dtype, const vo
                                               const int32_t* block_tables, int max_blocks_per_seq,
                                               const int32_t* context_lens, int max_context_len, int num_seqs,
                                               int num_heads, int num_kv_heads, int head_dim, int block_size,
-                                              int num_blocks, float scale, int partition_tokens, void* workspace,
-                                              size_t workspace_bytes, int32_t* status, pkv_stream_t stream) {
+                                              int num_blocks, float scale, int partition_tokens, int path,
+                                              void* workspace, size_t workspace_bytes, int32_t* status,
+                                              pkv_stream_t stream) {
   clear_error();
   if (!k_scale) return set_error(PKV_ERR_INVALID, "paged_attention_decode_fp8: null k_scale");
   return decode_impl(out, out_dtype, query, key_cache, value_cache, k_scale, v_scale, block_tables,
                      max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads, num_kv_heads, head_dim,
-                     block_size, num_blocks, scale, partition_tokens, PKV_PATH_SIMT, workspace, workspace_bytes,
+                     block_size, num_blocks, scale, partition_tokens, path, workspace, workspace_bytes,
                      status, stream);
 }

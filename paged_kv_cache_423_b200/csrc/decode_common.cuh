@@ -106,6 +106,9 @@ inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_di
 
 // Launchers living in other translation units.
 int launch_decode_tensor(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
+int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
 bool tensor_path_supports(int group, int head_dim);
+// Merge of split partitions (no launch when max_parts <= 1), after a tensor-core decode.
+int launch_merge_partials(const DecodeArgs& a, bool out_f32, cudaStream_t stream);
 
 }  // namespace pkv

@@ -88,43 +88,6 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, floa
     static_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
 }
 
-// Column-wise reduction over the 32 rows a warp holds, for 16 columns at once: a
-// transposed butterfly (16 shuffles) that leaves column (lane >> 1) in both lanes
-// of each pair.
-template <bool MAX>
-__device__ __forceinline__ float warp_col16(const float (&x)[16], int lane) {
-  auto op = [](float u, float w) { return MAX ? fmaxf(u, w) : u + w; };
-  float v[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const bool up = lane & 16;
-    const float send = up ? x[i] : x[i + 8];
-    const float keep = up ? x[i + 8] : x[i];
-    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const bool up = lane & 8;
-    const float send = up ? v[i] : v[i + 4];
-    const float keep = up ? v[i + 4] : v[i];
-    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
-  }
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const bool up = lane & 4;
-    const float send = up ? v[i] : v[i + 2];
-    const float keep = up ? v[i + 2] : v[i];
-    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-  }
-  {
-    const bool up = lane & 2;
-    const float send = up ? v[0] : v[1];
-    const float keep = up ? v[1] : v[0];
-    v[0] = op(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-  }
-  return op(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
-}
-
 // Softmax rows are rescaled only when a score exceeds the held maximum by more
 // than 2^kRescaleLog2 (weights up to 256 before normalisation, harmless in bf16
 // and fp32); otherwise P uses the held maximum and P·V keeps accumulating in TMEM.
@@ -141,7 +104,9 @@ constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
 //   softmax warps  -> s_free[b]    : S buffer b has been read
 //   softmax warps  -> p_full[b]    : P of the tile is in shared buffer b (two buffers)
 //   MMA warp       -> o_bar[b]     : O += Vᵀ·P of that tile is done (P buffer b reusable)
-//   MMA warp       -> empty[s]     : stage s may be refilled
+//   MMA warp and the 4 softmax warps -> empty[s] : stage s may be refilled (its
+//                    P·V is done and its metadata has been read; a tile with no
+//                    valid rows must not be refilled before the softmax has seen it)
 // The MMA warp never blocks on one side while the other could proceed: it polls
 // both (QK of the next landed tile, PV of the next tile whose P is ready).
 template <int STAGES, int N, bool OUT_F32>
@@ -174,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 5);  // the MMA commit after P·V, and each softmax warp once it has read the metadata
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -427,6 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       bool bad = !mbar_wait(&full[slot], (n / STAGES) & 1);
       const int4 mt = meta[slot];
       if (mt.w & kMetaEnd) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
       const int n_valid = mt.w & 0xff;
       const uint32_t mask = (mt.w >> 8) & 0xff;
       const bool first = mt.w & kMetaFirst, last = mt.w & kMetaLast;
@@ -696,15 +663,22 @@ static int launch(const Args& args, cudaStream_t stream) {
   kernel<<<std::max(1, sms), kThreads, smem, stream>>>(args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) launch: %s", cudaGetErrorString(e));
-  if (args.a.max_parts > 1) {
-    merge_partials_kernel<OUT_F32><<<args.a.num_seqs * args.a.num_heads, kMergeWarps * 32, 0, stream>>>(args.a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) merge launch: %s", cudaGetErrorString(e));
-  }
-  return PKV_OK;
+  return launch_merge_partials(args.a, OUT_F32, stream);
 }
 
 }  // namespace tc
+
+int launch_merge_partials(const DecodeArgs& a, bool out_f32, cudaStream_t stream) {
+  if (a.max_parts <= 1) return PKV_OK;
+  const int grid = a.num_seqs * a.num_heads;
+  if (out_f32)
+    tc::merge_partials_kernel<true><<<grid, tc::kMergeWarps * 32, 0, stream>>>(a);
+  else
+    tc::merge_partials_kernel<false><<<grid, tc::kMergeWarps * 32, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
+  return PKV_OK;
+}
 
 bool tensor_path_supports(int group, int head_dim) { return head_dim == tc::kD && group >= 2 && group <= 16; }
 

@@ -1,0 +1,769 @@
+// Tensor-core (tcgen05) decode over an 8-bit (e4m3) pool for grouped query heads.
+//
+// The contraction of the bf16 tensor-core decode (S = K·Qᵀ over 128-token tiles,
+// online softmax of the g query heads of a kv head, O = Vᵀ·P; intelliparadigm
+// article "PagedAttention：操作系统分页思想的跨界创新" §2.1), over a pool that holds
+// e4m3 codes with one float32 scale per kv head.  Both products run as kind::f8f6f4
+// MMAs straight from the e4m3 K and V tiles that TMA staged (128-byte swizzled):
+//
+//   S = K·Qᵀ   A = K (K-major).  B = the queries as two e4m3 terms, q·2^e = hi + lo,
+//              with a power of two 2^e per head that puts the head's largest |q| in
+//              [128, 256): hi is q·2^e rounded to e4m3 and lo the exact remainder
+//              rounded to e4m3, which holds all 8 significant bits of a bf16 value
+//              down to 2^-2 (below that the error is at most 2^-10 · 2^-e).  [hi; lo]
+//              is one N = 32 operand; the softmax adds the two halves of S.
+//   O = Vᵀ·P   A = V (MN-major: a token row of 128 codes is one swizzle span).  B = P
+//              (times 2^7) as three e5m2 terms: hi and mid are the f16 value of P cut
+//              to e5m2 and lo the rest rounded to e5m2, about 9 significant bits, and
+//              e5m2's range keeps every weight above 2^-23 of the held maximum (e4m3
+//              would drop those below 2^-9).  [hi | mid | lo] is one N = 48 operand;
+//              the softmax adds the three thirds of O, and the denominators add the
+//              same represented values.
+//   The K scale and 2^-e join the score scale, the V scale the output.
+//
+// Roles: warps 0-3 softmax (thread = TMEM lane = token row of a tile), warp 4 TMA
+// producer, warp 5 MMA issuer (fixed order: S of tile n+1, then O += Vᵀ·P of tile
+// n), warp 6 splits each item's queries as soon as they land.  Work items, plan,
+// workspace and the merge of split partitions are those of the bf16 decode paths.
+// Every wait is bounded; on a timeout the CTA flags PKV_DEV_TIMEOUT, lets its copies
+// land, waits for its MMAs, frees its tensor memory and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "decode_common.cuh"
+#include "pkv_internal.h"
+#include "tcgen05_common.cuh"
+
+namespace pkv {
+namespace tc8 {
+
+using tc::fast_exp2;
+
+constexpr int kTile = 128;                 // tokens per tile (MMA M of S)
+constexpr int kChunk = 16;                 // rows per TMA box: a 16-row slice of one (block, kv head)
+constexpr int kD = 128;
+constexpr int kN = 16;                     // query heads of one kv head (g <= 16)
+constexpr int kStages = 5;                 // e4m3 staging ring
+constexpr int kRow8 = kD;                  // bytes of one e4m3 row
+constexpr int kStage8 = 2 * kTile * kRow8; // K then V: 32 KiB
+constexpr int kVOff = kTile * kRow8;       // V within a stage
+constexpr int kQSlot = 4096;               // bf16 queries (2 halves x 16 rows x 128 B), then e4m3 [hi; lo] in place
+constexpr int kQSlots = 6;                 // by item ordinal; a slot is refilled 6 items later
+constexpr int kPTerm = kTile * 16;         // one e5m2 term of P: 128 tokens x 16 heads
+constexpr int kPBytes = 3 * kPTerm;        // [hi | mid | lo]
+constexpr int kConsumers = 128;            // warps 0-3
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kQueryWarp = 6;
+constexpr int kThreads = 224;
+constexpr uint32_t kTmemCols = 128;        // S double buffer [0,32), [32,64) (hi | lo); O [64,112) (3 terms)
+constexpr uint32_t kColO = 64;
+constexpr uint32_t kChunkTx = 2 * kChunk * kRow8;  // K and V of one slice
+constexpr float kRescaleLog2 = 8.f;
+constexpr float kPShift = 7.f;             // P is stored times 2^7 (at most 2^15)
+// Stage metadata: x = sequence, y = kv head | q slot << 16, z = partition | partitions << 16,
+// w = valid rows (8 bits) | slice mask << 8 | first << 16 | last << 17 | end of stream << 18
+constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
+
+// shared memory
+constexpr int kOffStage = 0;
+constexpr int kOffQ = kOffStage + kStages * kStage8;
+constexpr int kOffP = kOffQ + kQSlots * kQSlot;
+constexpr int kOffRed = kOffP + 2 * kPBytes;
+constexpr int kOffMeta = kOffRed + 2 * 4 * 16 * 4;
+constexpr int kOffScale = kOffMeta + kStages * 16;  // [stage] (k_scale, v_scale) of the item
+constexpr int kOffQinv = kOffScale + kStages * 8;   // [q slot][16] 2^-e of each head
+constexpr int kOffBar = kOffQinv + kQSlots * 16 * 4;
+constexpr int kBars = 2 * kStages + kQSlots + 2 * 4 + 1;
+constexpr int kOffMisc = kOffBar + kBars * 8;
+constexpr int kSmemBytes = kOffMisc + 32 + 1024;
+static_assert(kOffBar % 8 == 0 && kOffMeta % 16 == 0 && kOffQ % 1024 == 0, "alignment");
+static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+
+struct alignas(64) Args {
+  CUtensorMap tm_k;  // e4m3 pool as [rows, 128] bytes, box 128 x 16, 128-byte swizzle
+  CUtensorMap tm_v;
+  CUtensorMap tm_q;  // bf16 queries as [B * Hq, 128], box 64 x 16, 128-byte swizzle
+  DecodeArgs a;
+};
+
+// Two floats -> two e4m3 codes (round to nearest even, saturating), x0 in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_rn(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+
+// Two e4m3 codes (low byte first) -> their values as f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t codes) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l;\n\tcvt.u16.u32 l, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}" : "=r"(r) : "r"(codes));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t sub_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ float f16lo(uint32_t w) {
+  float r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(r) : "r"(w));
+  return r;
+}
+
+__device__ __forceinline__ float f16hi(uint32_t w) {
+  float r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, h;\n\t}" : "=f"(r) : "r"(w));
+  return r;
+}
+
+// hi + lo split of two scaled query values: the e4m3 codes of hi in the low 16 bits
+// and of lo in the high 16 bits, x0's code in the low byte of each.
+__device__ __forceinline__ uint32_t split_q2(float x0, float x1) {
+  const uint32_t h = e4m3x2_rn(x0, x1);
+  const uint32_t hf = e4m3x2_f16x2(h);
+  const uint32_t l = e4m3x2_rn(x0 - f16lo(hf), x1 - f16hi(hf));
+  return h | (l << 16);
+}
+
+// Three e5m2 terms of two non-negative f16 values p (f16x2): hi and mid are p cut to
+// the top byte (an e5m2 code is the top byte of an f16) and lo the remainder rounded
+// at its third significant bit.  Returns the three f16x2 words whose top bytes are
+// the codes; `sum` gets hi + mid + lo (exact in f16).
+__device__ __forceinline__ void split_p2(uint32_t p, uint32_t& hi, uint32_t& mid, uint32_t& lo, uint32_t& sum) {
+  hi = p & 0xFF00FF00u;
+  const uint32_t r1 = sub_f16x2(p, hi);
+  mid = r1 & 0xFF00FF00u;
+  const uint32_t r2 = sub_f16x2(r1, mid);
+  lo = (r2 + 0x00800080u) & 0xFF00FF00u;
+  sum = add_f16x2(add_f16x2(hi, mid), lo);
+}
+
+template <bool OUT_F32>
+__device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, float v) {
+  if constexpr (OUT_F32)
+    static_cast<float*>(a.out)[idx] = v;
+  else
+    static_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
+}
+
+// Pipeline (per CTA, persistent over work items; n counts tiles):
+//   producer     -> full[s]    : e4m3 K, V (and the bf16 queries on an item's first tile) in stage s
+//   query warp   -> q_ready[j] : the queries of the item in q slot j split into e4m3 hi/lo
+//   MMA          -> s_full[b]  : S of the b-th valid tile (mod 2) in TMEM
+//   softmax      -> s_free[b]  : that S read
+//   softmax      -> p_full[b]  : P of that tile in shared buffer b (and its stale V rows zeroed)
+//   MMA          -> o_bar[b]   : its O += Vᵀ·P done (P buffer b reusable)
+//   MMA + softmax + query warp -> empty[s] : stage s done with: its P·V complete
+//                  (commit; a plain arrival for a tile with no rows), metadata read by
+//                  the 4 softmax warps and the query warp (6 arrivals)
+template <bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __grid_constant__ Args args) {
+  const DecodeArgs& a = args.a;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* stage8 = smem + kOffStage;
+  unsigned char* q_ring = smem + kOffQ;
+  unsigned char* p_buf = smem + kOffP;
+  float* red = reinterpret_cast<float*>(smem + kOffRed);
+  int4* meta = reinterpret_cast<int4*>(smem + kOffMeta);
+  float2* mscale = reinterpret_cast<float2*>(smem + kOffScale);
+  float* qinv = reinterpret_cast<float*>(smem + kOffQinv);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kStages;
+  uint64_t* q_ready = empty + kStages;
+  uint64_t* s_full = q_ready + kQSlots;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* o_bar = p_full + 2;
+  uint64_t* drain = o_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  volatile int* restart_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [2]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = a.group;
+  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + 4 + 1);
+    }
+    for (int j = 0; j < kQSlots; ++j) mbar_init(&q_ready[j], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 4);
+      mbar_init(&p_full[b], 4);
+      mbar_init(&o_bar[b], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tc::tmem_alloc(tmem_slot, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    // ================= producer: e4m3 slices and an item's queries =================
+    const uint64_t policy = l2_policy_kv();
+    auto load_entry = [&](int64_t it) -> PlanEntry {
+      return it < n_items ? a.entries[it / a.num_kv_heads] : make_int4(0, 0, 0, 0);
+    };
+    // The item's block-table slice: lane l holds entries l, l+32, l+64, l+96 (an item
+    // spans at most 2048 tokens = 128 blocks of 16).
+    auto load_tab = [&](const PlanEntry& e) -> int4 {
+      const int tok0 = e.y * a.partition;
+      const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - tok0);
+      const int nblk = (ntok + a.block_size - 1) / a.block_size;
+      const int32_t* row = a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size;
+      int4 t = make_int4(0, 0, 0, 0);
+      if (lane < nblk) t.x = __ldg(row + lane);
+      if (lane + 32 < nblk) t.y = __ldg(row + lane + 32);
+      if (lane + 64 < nblk) t.z = __ldg(row + lane + 64);
+      if (lane + 96 < nblk) t.w = __ldg(row + lane + 96);
+      return t;
+    };
+    auto load_scales = [&](int64_t it) -> float2 {
+      if (it >= n_items) return make_float2(0.f, 0.f);
+      const int kvh = static_cast<int>(it % a.num_kv_heads);
+      return make_float2(__ldg(a.k_scale + kvh), __ldg(a.v_scale + kvh));
+    };
+    int* work_counter = const_cast<int*>(a.plan_count) + 1;
+    auto grab = [&]() -> int64_t {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(work_counter, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    // item ids, entries, scales and table slices are fetched ahead, as in the bf16 kernel
+    int64_t item = grab();
+    int64_t item_nxt = grab();
+    int64_t item_nx2 = grab();
+    PlanEntry e_cur = load_entry(item);
+    int4 tab_cur = item < n_items ? load_tab(e_cur) : make_int4(0, 0, 0, 0);
+    float2 sc_cur = load_scales(item);
+    PlanEntry e_nxt = load_entry(item_nxt);
+    int4 tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
+    float2 sc_nxt = load_scales(item_nxt);
+    PlanEntry e_nx2 = load_entry(item_nx2);
+    int n = 0, item_ord = 0;
+    bool failed = false;
+    auto acquire = [&](int slot) -> bool {
+      if (n >= kStages && !mbar_wait(&empty[slot], ((n / kStages) - 1) & 1)) {
+        *abort_flag = 1;
+        set_status(a.status, PKV_DEV_TIMEOUT);
+        return false;
+      }
+      return true;
+    };
+    while (item < n_items && !failed && !*abort_flag) {
+      const PlanEntry e = e_cur;
+      const int kvh = static_cast<int>(item % a.num_kv_heads);
+      const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - e.y * a.partition);
+      const int ntiles = ntok == 0 ? 1 : (ntok + kTile - 1) / kTile;
+      const int qslot = item_ord % kQSlots;
+      for (int tile = 0; tile < ntiles; ++tile, ++n) {
+        const int slot = n % kStages;
+        const int n_valid = max(0, min(kTile, ntok - tile * kTile));
+        const int nchunks = (n_valid + kChunk - 1) / kChunk;
+        const int ltok = tile * kTile + lane * kChunk;  // this lane's slice (lane < nchunks)
+        const int blk = min(127, ltok / a.block_size);
+        const int p0 = __shfl_sync(0xffffffffu, tab_cur.x, blk & 31);
+        const int p1 = __shfl_sync(0xffffffffu, tab_cur.y, blk & 31);
+        const int p2 = __shfl_sync(0xffffffffu, tab_cur.z, blk & 31);
+        const int p3 = __shfl_sync(0xffffffffu, tab_cur.w, blk & 31);
+        const int phys = blk < 32 ? p0 : blk < 64 ? p1 : blk < 96 ? p2 : p3;
+        const bool mine = lane < nchunks;
+        const bool ok = mine && phys >= 0 && phys < a.num_blocks;
+        const uint32_t mask = __ballot_sync(0xffffffffu, ok);
+        if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
+        if (!acquire(slot)) {
+          failed = true;
+          break;
+        }
+        const bool with_q = tile == 0 && ntok > 0;
+        if (lane == 0) {
+          meta[slot] = make_int4(e.x, kvh | (qslot << 16), e.y | (e.z << 16),
+                                 n_valid | (mask << 8) | (tile == 0 ? kMetaFirst : 0) |
+                                     (tile == ntiles - 1 ? kMetaLast : 0));
+          mscale[slot] = sc_cur;
+          mbar_arrive_expect_tx(&full[slot], __popc(mask) * kChunkTx + (with_q ? kQSlot : 0));
+        }
+        __syncwarp();
+        if (ok) {
+          const int r = (phys * a.num_kv_heads + kvh) * a.block_size + ltok % a.block_size;
+          unsigned char* dst = stage8 + slot * kStage8 + lane * kChunk * kRow8;
+          tc::tma_load_2d(dst, &args.tm_k, 0, r, &full[slot], policy);
+          tc::tma_load_2d(dst + kVOff, &args.tm_v, 0, r, &full[slot], policy);
+        }
+        if (with_q && lane == 0) {
+          const int qrow = e.x * a.num_heads + kvh * g;
+          unsigned char* qd = q_ring + qslot * kQSlot;
+          tc::tma_load_2d(qd, &args.tm_q, 0, qrow, &full[slot], policy);
+          tc::tma_load_2d(qd + kN * 128, &args.tm_q, 64, qrow, &full[slot], policy);
+        }
+      }
+      item = item_nxt;
+      item_nxt = item_nx2;
+      item_nx2 = grab();
+      ++item_ord;
+      e_cur = e_nxt;
+      tab_cur = tab_nxt;
+      sc_cur = sc_nxt;
+      e_nxt = e_nx2;
+      tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
+      sc_nxt = load_scales(item_nxt);
+      e_nx2 = load_entry(item_nx2);
+    }
+    if (!failed && !*abort_flag) {
+      const int slot = n % kStages;
+      if (acquire(slot)) {
+        if (lane == 0) {
+          meta[slot] = make_int4(0, 0, 0, kMetaEnd);
+          mbar_arrive_expect_tx(&full[slot], 0);
+        }
+        ++n;
+      }
+      __syncwarp();
+    }
+    // Let this CTA's last copies land before the final barrier.
+    for (int k = max(0, n - kStages); k < n; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1);
+  } else if (warp == kQueryWarp) {
+    // ================= query split: bf16 -> e4m3 [hi; lo] with a power of two per head =================
+    // Lane l takes head r = l / 2 and half h = l % 2 (dims 64h .. 64h+63) of the bf16 slot.
+    const int r = lane >> 1, h = lane & 1;
+    for (int n = 0;; ++n) {
+      const int slot = n % kStages;
+      if (!mbar_wait(&full[slot], (n / kStages) & 1)) {
+        *abort_flag = 1;
+        set_status(a.status, PKV_DEV_TIMEOUT);
+        break;
+      }
+      const int4 mt = meta[slot];
+      if (mt.w & kMetaEnd) break;
+      if ((mt.w & kMetaFirst) && (mt.w & 0xff) > 0) {
+        const int qs = mt.y >> 16;
+        unsigned char* qb = q_ring + qs * kQSlot;
+        // bf16 row r of half h: 128 bytes, 16-byte chunk c at (c ^ (r % 8)) * 16
+        uint4 v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          v[c] = *reinterpret_cast<const uint4*>(qb + h * 2048 + r * 128 + ((c ^ (r & 7)) << 4));
+        float m = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
+        }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        // 2^e with the head's largest |q| * 2^e in [128, 256)
+        const int E = static_cast<int>((__float_as_uint(m) >> 23) & 0xff);
+        const int e = E == 0 ? 0 : min(134 - E, 126);
+        const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+        __syncwarp();  // every bf16 value read before the slot is rewritten
+        // e4m3 rows: hi of head r at row r, lo at row 16 + r (128 bytes, 128-byte
+        // swizzle); dims 64h + 16j .. sit in 16-byte chunk 4h + j
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 x0 = v[2 * j], x1 = v[2 * j + 1];  // dims 64h + 16j + 0..7, + 8..15
+          const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          uint32_t s[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) s[i] = split_q2(bf16lo(w[i]) * up, bf16hi(w[i]) * up);
+          uint4 hi4, lo4;
+          hi4.x = __byte_perm(s[0], s[1], 0x5410);
+          hi4.y = __byte_perm(s[2], s[3], 0x5410);
+          hi4.z = __byte_perm(s[4], s[5], 0x5410);
+          hi4.w = __byte_perm(s[6], s[7], 0x5410);
+          lo4.x = __byte_perm(s[0], s[1], 0x7632);
+          lo4.y = __byte_perm(s[2], s[3], 0x7632);
+          lo4.z = __byte_perm(s[4], s[5], 0x7632);
+          lo4.w = __byte_perm(s[6], s[7], 0x7632);
+          const int pc = ((4 * h + j) ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4*>(qb + r * 128 + pc) = hi4;
+          *reinterpret_cast<uint4*>(qb + (16 + r) * 128 + pc) = lo4;
+        }
+        if (h == 0) qinv[qs * 16 + r] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        fence_proxy_async_smem();  // the split queries, before the MMAs read them
+      }
+      __syncwarp();
+      // every item's first tile completes one phase of its slot's barrier (an empty
+      // item's too), so the phase of item i in slot i % 6 is (i / 6) & 1 for all roles
+      if ((mt.w & kMetaFirst) && lane == 0) mbar_arrive(&q_ready[mt.y >> 16]);
+      if (lane == 0) mbar_arrive(&empty[slot]);  // metadata read
+    }
+  } else if (warp == kMmaWarp) {
+    // ================= MMA issuer (one thread) =================
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = tc::instr_desc_e4m3(kTile, 2 * kN);
+      // A = V e4m3 MN-major, B = P e5m2 (format 1) MN-major, N = 48
+      constexpr uint32_t idesc_pv = tc::instr_desc_e4m3(kD, 3 * kN) | (1u << 10) | (1u << 15) | (1u << 16);
+      const uint32_t p_addr0 = smem_addr(p_buf);
+      int q_valid = 0, p_valid = 0;  // valid tiles that got their QK / PV
+      int items = 0;                 // items whose first tile has been seen
+      int prev_slot = -1, prev_nv = 0;
+      bool ok = true;
+      auto wait = [&](uint64_t* bar, uint32_t parity) {
+        if (ok && !mbar_wait(bar, parity)) {
+          ok = false;
+          *abort_flag = 1;
+          set_status(a.status, PKV_DEV_TIMEOUT);
+        }
+        return ok;
+      };
+      // O += Vᵀ·P of the held tile (its P in buffer p_valid & 1)
+      auto issue_pv = [&]() {
+        const int b = p_valid & 1;
+        if (!wait(&p_full[b], (p_valid >> 1) & 1)) return;
+        tc::tc_fence_after();
+        const bool restart = restart_flag[b] != 0;
+        const uint32_t v_addr = smem_addr(stage8 + prev_slot * kStage8 + kVOff);
+        const uint32_t p_addr = p_addr0 + b * kPBytes;
+        const int kt = (prev_nv + 31) / 32;
+        for (int kk = 0; kk < kt; ++kk) {
+          // V: 32 tokens = 4 swizzle atoms of 8 rows; P: 4 groups of 8 tokens x 16 bytes, terms 2 KiB apart
+          tc::umma_f8(tmem + kColO, tc::smem_desc_sw128(v_addr + kk * 4096, kTile * kRow8, 1024),
+                      tc::smem_desc_plain(p_addr + kk * 512, 128, kPTerm), idesc_pv, kk > 0 || !restart);
+        }
+        tc::umma_commit(&o_bar[b]);
+        tc::umma_commit(&empty[prev_slot]);
+        ++p_valid;
+        prev_slot = -1;
+      };
+      for (int n = 0; ok; ++n) {
+        const int slot = n % kStages;
+        if (!wait(&full[slot], (n / kStages) & 1)) break;
+        const int4 mt = meta[slot];
+        if (mt.w & kMetaEnd) break;
+        const int nv = mt.w & 0xff;
+        const bool first = mt.w & kMetaFirst;
+        if (nv == 0) {
+          if (prev_slot >= 0) issue_pv();
+          mbar_arrive(&empty[slot]);
+          items += first;
+          continue;
+        }
+        // S = K·[hi; lo]ᵀ of tile n
+        const int qs = mt.y >> 16;
+        if (first && !wait(&q_ready[qs], (items / kQSlots) & 1)) break;
+        items += first;
+        const int b = q_valid & 1;
+        if (q_valid >= 2 && !wait(&s_free[b], ((q_valid >> 1) - 1) & 1)) break;
+        tc::tc_fence_after();
+        const uint32_t k_addr = smem_addr(stage8 + slot * kStage8);
+        const uint32_t q_addr = smem_addr(q_ring + qs * kQSlot);
+#pragma unroll
+        for (int kk = 0; kk < kD / 32; ++kk)
+          tc::umma_f8(tmem + b * 32, tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024),
+                      tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024), idesc_qk, kk > 0);
+        tc::umma_commit(&s_full[b]);
+        ++q_valid;
+        // then O += Vᵀ·P of the previous valid tile
+        if (prev_slot >= 0) issue_pv();
+        prev_slot = slot;
+        prev_nv = nv;
+      }
+      if (ok && prev_slot >= 0) issue_pv();
+      // every MMA of this CTA is done before the tensor memory is freed
+      tc::umma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ================= softmax warps (one thread per TMEM lane) =================
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m_used[kN], lp[kN], o_reg[kN], hscale[kN];
+#pragma unroll
+    for (int h = 0; h < kN; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f, hscale[h] = 0.f;
+    float out_scale = 1.f;
+    bool restart = true;
+    bool pv_since_restart = false;
+    int n_valid_tiles = 0, items = 0;
+    uint32_t ob_next = 0, ob_pending = 0;
+    auto wait_ob = [&](int b) -> bool {
+      if (!((ob_pending >> b) & 1)) return true;
+      ob_pending &= ~(1u << b);
+      return mbar_wait(&o_bar[b], ((ob_next >> b) & 1) ^ 1u);
+    };
+    // O (sum of the three terms' columns) of this thread's row
+    auto load_o = [&](float (&o)[kN]) {
+      float o3[3 * kN];
+      tc::tmem_load32f_nowait(tmem + lane_base + kColO, o3);
+      tc::tmem_load32f_nowait(tmem + lane_base + kColO + 32, o3 + 32);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int h = 0; h < kN; ++h) o[h] = o3[h] + o3[kN + h] + o3[2 * kN + h];
+    };
+    for (int n = 0;; ++n) {
+      const int slot = n % kStages;
+      bool bad = !mbar_wait(&full[slot], (n / kStages) & 1);
+      const int4 mt = meta[slot];
+      const float2 sc = mscale[slot];
+      if (bad) *abort_flag = 1;
+      if ((mt.w & kMetaEnd) || bad) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);  // metadata read
+      const int n_valid = mt.w & 0xff;
+      const uint32_t mask = (mt.w >> 8) & 0xff;
+      const bool first = mt.w & kMetaFirst, last = mt.w & kMetaLast;
+      if (first) {
+#pragma unroll
+        for (int h = 0; h < kN; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f;
+        restart = true;
+        pv_since_restart = false;
+        out_scale = sc.y;
+        if (n_valid > 0) {
+          const int qs = mt.y >> 16;
+          bad |= !mbar_wait(&q_ready[qs], (items / kQSlots) & 1);
+          const float base = a.scale_log2 * sc.x;
+#pragma unroll
+          for (int h = 0; h < kN; ++h) hscale[h] = base * qinv[qs * 16 + h];
+        }
+        ++items;
+      }
+      if (n_valid > 0) {
+        const int b = n_valid_tiles & 1;
+        unsigned char* p_tile = p_buf + b * kPBytes;
+        bad |= !mbar_wait(&s_full[b], (n_valid_tiles >> 1) & 1);
+        tc::tc_fence_after();
+        float s[2 * kN];
+        tc::tmem_load32f_nowait(tmem + lane_base + b * 32, s);
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[b]);
+        bad |= !wait_ob(b);  // P buffer b: the P·V of two valid tiles back is done
+        const int t = tid;
+        const bool valid = t < n_valid && ((mask >> (t / kChunk)) & 1);
+        if (!valid) {
+          // V rows outside the context may hold anything (even NaN codes): zero them
+          uint4* vr = reinterpret_cast<uint4*>(stage8 + slot * kStage8 + kVOff + t * kRow8);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) vr[c] = make_uint4(0, 0, 0, 0);
+        }
+        float x[kN];
+        bool need = false;
+#pragma unroll
+        for (int h = 0; h < kN; ++h) {
+          x[h] = (valid && h < g) ? (s[h] + s[kN + h]) * hscale[h] : -INFINITY;
+          need |= x[h] > m_used[h] + kRescaleLog2;
+        }
+        // P row of this token: each term is a 16-byte chunk (heads 0..15) at
+        // (t/8)*128 + (t%8)*16 of its 2 KiB third of the buffer.
+        float pv[kN];
+        auto write_p = [&]() {
+          uint32_t ph[kN / 2], pm[kN / 2], pl[kN / 2];
+#pragma unroll
+          for (int j = 0; j < kN / 2; ++j) {
+            const int h0 = 2 * j, h1 = 2 * j + 1;
+            const float p0 =
+                (valid && h0 < g && m_used[h0] > -INFINITY) ? fast_exp2(x[h0] - m_used[h0] + kPShift) : 0.f;
+            const float p1 =
+                (valid && h1 < g && m_used[h1] > -INFINITY) ? fast_exp2(x[h1] - m_used[h1] + kPShift) : 0.f;
+            uint32_t sum;
+            split_p2(pack_f16x2(p0, p1), ph[j], pm[j], pl[j], sum);
+            pv[h0] = f16lo(sum);
+            pv[h1] = f16hi(sum);
+          }
+          unsigned char* row = p_tile + (t >> 3) * 128 + (t & 7) * 16;
+          *reinterpret_cast<uint4*>(row) =
+              make_uint4(__byte_perm(ph[0], ph[1], 0x7531), __byte_perm(ph[2], ph[3], 0x7531),
+                         __byte_perm(ph[4], ph[5], 0x7531), __byte_perm(ph[6], ph[7], 0x7531));
+          *reinterpret_cast<uint4*>(row + kPTerm) =
+              make_uint4(__byte_perm(pm[0], pm[1], 0x7531), __byte_perm(pm[2], pm[3], 0x7531),
+                         __byte_perm(pm[4], pm[5], 0x7531), __byte_perm(pm[6], pm[7], 0x7531));
+          *reinterpret_cast<uint4*>(row + 2 * kPTerm) =
+              make_uint4(__byte_perm(pl[0], pl[1], 0x7531), __byte_perm(pl[2], pl[3], 0x7531),
+                         __byte_perm(pl[4], pl[5], 0x7531), __byte_perm(pl[6], pl[7], 0x7531));
+        };
+        if (bad) *abort_flag = 1;
+        bool need_any = true;  // an item's first tile always sets the held maximum
+        if (!first) {
+          write_p();
+          if (tid == 0) restart_flag[b] = restart;
+          fence_proxy_async_smem();
+          need_any = tc::named_barrier_or(1, kConsumers, need || bad);
+          if (*abort_flag) break;
+        }
+        if (need_any) {
+          // a score outgrew the held maximum (or none is held yet): take the tile
+          // maximum, fold the accumulated P·V into registers at the old scale, rewrite P
+          const float wmax = tc::warp_col16<true>(x, lane);
+          if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = wmax;
+          bool ok = wait_ob(0);
+          ok &= wait_ob(1);
+          if (!ok) *abort_flag = 1;
+          tc::named_barrier_sync(1, kConsumers);
+          if (*abort_flag) break;
+          float alpha[kN];
+#pragma unroll
+          for (int h = 0; h < kN; ++h) {
+            const float tmax = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
+            if (h < g) {
+              const float m_new = fmaxf(m_used[h], tmax);
+              alpha[h] = m_used[h] == -INFINITY ? 0.f : fast_exp2(m_used[h] - m_new);
+              m_used[h] = m_new;
+            } else {
+              alpha[h] = 1.f;
+            }
+          }
+          tc::tc_fence_after();
+          if (pv_since_restart) {
+            float o[kN];
+            load_o(o);
+#pragma unroll
+            for (int h = 0; h < kN; ++h) o_reg[h] = (o_reg[h] + o[h]) * alpha[h];
+          } else {
+#pragma unroll
+            for (int h = 0; h < kN; ++h) o_reg[h] *= alpha[h];
+          }
+          tc::tc_fence_before();
+#pragma unroll
+          for (int h = 0; h < kN; ++h) lp[h] *= alpha[h];
+          restart = true;
+          pv_since_restart = false;
+          write_p();
+          if (tid == 0) restart_flag[b] = 1;
+          fence_proxy_async_smem();
+          tc::named_barrier_sync(1, kConsumers);
+        }
+#pragma unroll
+        for (int h = 0; h < kN; ++h)
+          if (h < g) lp[h] += pv[h];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+        ob_next ^= 1u << b;
+        ob_pending |= 1u << b;
+        restart = false;
+        pv_since_restart = true;
+        ++n_valid_tiles;
+      }
+      if (last) {
+        // ---- finalize the item: O = registers + TMEM, times the V scale; denominators
+        bool ok = wait_ob(0);
+        ok &= wait_ob(1);
+        tc::tc_fence_after();
+        float ot[kN];
+        if (pv_since_restart) {
+          float o[kN];
+          load_o(o);
+#pragma unroll
+          for (int h = 0; h < kN; ++h) ot[h] = (o_reg[h] + o[h]) * out_scale;
+        } else {
+#pragma unroll
+          for (int h = 0; h < kN; ++h) ot[h] = o_reg[h] * out_scale;
+        }
+        tc::tc_fence_before();
+        if (!ok) *abort_flag = 1;
+        float* red2 = red + 64;
+        const float wsum = tc::warp_col16<false>(lp, lane);
+        if ((lane & 1) == 0) red2[warp * 16 + (lane >> 1)] = wsum;
+        tc::named_barrier_sync(1, kConsumers);
+        const int seq = mt.x, kvh = mt.y & 0xffff, part = mt.z & 0xffff, nparts = mt.z >> 16;
+        const int d = tid;
+        const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
+#pragma unroll
+        for (int h = 0; h < kN; ++h) {
+          if (h >= g) break;
+          const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
+          if (nparts == 1) {
+            store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[h] / l : 0.f);
+          } else {
+            // unnormalised partial (weights times 2^7 in both o and l); the merge
+            // kernel combines the partitions
+            const int64_t pidx = (unit0 + h) * a.max_parts + part;
+            a.part_o[pidx * kD + d] = ot[h];
+            if (d == 0) a.part_ml[pidx] = make_float2(m_used[h], l);
+          }
+        }
+      }
+    }
+    if (*abort_flag && tid == 0) set_status(a.status, PKV_DEV_TIMEOUT);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---- host side -----------------------------------------------------------------
+
+// 2-D view [rows, 128] with a 128-byte swizzle: the e4m3 pool (box 128 codes x 16
+// rows) or the bf16 queries (box 64 values x 16 rows).
+static int encode_map(CUtensorMap* map, const void* base, uint64_t rows, bool e4m3, const char* what) {
+  auto encode = tc::tensor_map_encoder();
+  if (!encode) return set_error(PKV_ERR_CUDA, "decode (8-bit tensor): cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * (e4m3 ? 1 : 2)};
+  cuuint32_t box[2] = {e4m3 ? 128u : 64u, e4m3 ? static_cast<cuuint32_t>(kChunk) : static_cast<cuuint32_t>(kN)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(PKV_ERR_CUDA, "decode (8-bit tensor): tensor map for %s failed (%d)", what, (int)r);
+  return PKV_OK;
+}
+
+template <bool OUT_F32>
+static int launch(const Args& args, cudaStream_t stream) {
+  auto kernel = decode_gqa_tc_fp8_kernel<OUT_F32>;
+  static std::once_flag once;
+  static cudaError_t setup = cudaSuccess;
+  std::call_once(once,
+                 [&] { setup = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes); });
+  if (setup != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) setup: %s", cudaGetErrorString(setup));
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  kernel<<<std::max(1, sms), kThreads, kSmemBytes, stream>>>(args);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) launch: %s", cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+}  // namespace tc8
+
+int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream) {
+  if (!tensor_path_supports(a.group, head_dim))
+    return set_error(PKV_ERR_UNSUPPORTED, "decode (8-bit tensor): group %d / head_dim %d not supported", a.group,
+                     head_dim);
+  tc8::Args args;
+  args.a = a;
+  const uint64_t pool_rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
+  int rc = tc8::encode_map(&args.tm_k, a.key_cache8, pool_rows, true, "key_cache");
+  if (rc == PKV_OK) rc = tc8::encode_map(&args.tm_v, a.value_cache8, pool_rows, true, "value_cache");
+  if (rc == PKV_OK)
+    rc = tc8::encode_map(&args.tm_q, a.query, static_cast<uint64_t>(a.num_seqs) * a.num_heads, false, "query");
+  if (rc != PKV_OK) return rc;
+  rc = out_f32 ? tc8::launch<true>(args, stream) : tc8::launch<false>(args, stream);
+  if (rc != PKV_OK) return rc;
+  return launch_merge_partials(a, out_f32, stream);
+}
+
+}  // namespace pkv

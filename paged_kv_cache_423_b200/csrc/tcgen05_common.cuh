@@ -61,6 +61,19 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] · B[smem desc], kind::f8f6f4 with 8-bit operands (the
+// formats are in the instruction descriptor; fp32 accumulate).  One MMA covers 32
+// elements of K (32 bytes of a K-major row).
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
 // Arrive once on `bar` when every previously issued MMA of this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
@@ -125,12 +138,56 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A/B major-ness,
-// N >> 3 and M >> 4.
-__host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn_major, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn_major ? 1u << 15 : 0u) | (b_mn_major ? 1u << 16 : 0u) |
-         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+// Instruction descriptor, kind::f16: fp32 accumulator, A and B both bf16 (or both f16),
+// A/B major-ness, N >> 3 and M >> 4.
+__host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn_major, bool b_mn_major, bool f16 = false) {
+  return (1u << 4) | (f16 ? 0u : (1u << 7) | (1u << 10)) | (a_mn_major ? 1u << 15 : 0u) |
+         (b_mn_major ? 1u << 16 : 0u) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
+
+// Instruction descriptor, kind::f8f6f4: fp32 accumulator, A and B e4m3 (format code 0),
+// both K-major, N >> 3 and M >> 4.
+__host__ __device__ constexpr uint32_t instr_desc_e4m3(int m, int n) {
+  return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// Column-wise reduction over the 32 rows a warp holds, for 16 columns at once: a
+// transposed butterfly (16 shuffles) that leaves column (lane >> 1) in both lanes
+// of each pair.
+template <bool MAX>
+__device__ __forceinline__ float warp_col16(const float (&x)[16], int lane) {
+  auto op = [](float u, float w) { return MAX ? fmaxf(u, w) : u + w; };
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool up = lane & 16;
+    const float send = up ? x[i] : x[i + 8];
+    const float keep = up ? x[i + 8] : x[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool up = lane & 8;
+    const float send = up ? v[i] : v[i + 4];
+    const float keep = up ? v[i + 4] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool up = lane & 4;
+    const float send = up ? v[i] : v[i + 2];
+    const float keep = up ? v[i + 2] : v[i];
+    v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+  }
+  {
+    const bool up = lane & 2;
+    const float send = up ? v[0] : v[1];
+    const float keep = up ? v[1] : v[0];
+    v[0] = op(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+  }
+  return op(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
+}
+
 
 
 // 3-D tensor-map load (coordinates innermost first).

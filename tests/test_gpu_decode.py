@@ -91,6 +91,20 @@ def test_zero_length_and_single_token(pkv, path):
 
 
 @pytest.mark.parametrize("path", sorted(PATHS))
+def test_runs_of_empty_contexts(pkv, path):
+    """Runs of zero-length sequences between long ones (each gives one empty work item;
+    the plan puts them last, right behind the longest items' final tiles)."""
+    lengths = [0] * 6 + [700] + [0] * 9 + [1, 0, 0, 0, 0, 300, 0, 17] + [0] * 12 + [2049]
+    b = wl.make_decode_batch("llama7b", num_heads=8, num_kv_heads=2 if path == "tensor" else 8, lengths=lengths)
+    db = DeviceBatch(b)
+    ref = oracle_out(b)
+    for _ in range(3):
+        out = db.decode(pkv, path=PATHS[path]).cpu().numpy()
+        assert np.all(out[np.array(lengths) == 0] == 0)
+        compare(out, ref)
+
+
+@pytest.mark.parametrize("path", sorted(PATHS))
 def test_stale_nan_rows_do_not_leak(pkv, path):
     """Rows past a context's end (stale pool rows) never enter the result, even as NaN."""
     b = wl.make_decode_batch("llama13b_mixed_bs32", num_seqs=8, num_heads=8, num_kv_heads=4 if path == "tensor" else 8,

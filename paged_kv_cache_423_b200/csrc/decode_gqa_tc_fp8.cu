@@ -175,7 +175,9 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, floa
 //   MMA + softmax + query warp -> empty[s] : stage s done with: its P·V complete
 //                  (commit; a plain arrival for a tile with no rows), metadata read by
 //                  the 4 softmax warps and the query warp (6 arrivals)
-template <bool OUT_F32>
+// NH (4, 8 or 16 >= g) bounds the heads the softmax works on; the operand layouts
+// keep 16 head slots.
+template <bool OUT_F32, int NH>
 __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __grid_constant__ Args args) {
   const DecodeArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
@@ -496,9 +498,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   } else {
     // ================= softmax warps (one thread per TMEM lane) =================
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m_used[kN], lp[kN], o_reg[kN], hscale[kN];
+    float m_used[NH], lp[NH], o_reg[NH], hscale[NH];
 #pragma unroll
-    for (int h = 0; h < kN; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f, hscale[h] = 0.f;
+    for (int h = 0; h < NH; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f, hscale[h] = 0.f;
     float out_scale = 1.f;
     bool restart = true;
     bool pv_since_restart = false;
@@ -510,14 +512,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       return mbar_wait(&o_bar[b], ((ob_next >> b) & 1) ^ 1u);
     };
     // O (sum of the three terms' columns) of this thread's row
-    auto load_o = [&](float (&o)[kN]) {
+    auto load_o = [&](float (&o)[NH]) {
       float o3[3 * kN];
       tc::tmem_load32f_nowait(tmem + lane_base + kColO, o3);
       tc::tmem_load32f_nowait(tmem + lane_base + kColO + 32, o3 + 32);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int h = 0; h < kN; ++h) o[h] = o3[h] + o3[kN + h] + o3[2 * kN + h];
+      for (int h = 0; h < NH; ++h) o[h] = o3[h] + o3[kN + h] + o3[2 * kN + h];
     };
+    constexpr int kColLanes = 32 / NH;  // lanes sharing one column after warp_col
     for (int n = 0;; ++n) {
       const int slot = n % kStages;
       bool bad = !mbar_wait(&full[slot], (n / kStages) & 1);
@@ -532,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       const bool first = mt.w & kMetaFirst, last = mt.w & kMetaLast;
       if (first) {
 #pragma unroll
-        for (int h = 0; h < kN; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f;
+        for (int h = 0; h < NH; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f;
         restart = true;
         pv_since_restart = false;
         out_scale = sc.y;
@@ -541,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           bad |= !mbar_wait(&q_ready[qs], (items / kQSlots) & 1);
           const float base = a.scale_log2 * sc.x;
 #pragma unroll
-          for (int h = 0; h < kN; ++h) hscale[h] = base * qinv[qs * 16 + h];
+          for (int h = 0; h < NH; ++h) hscale[h] = base * qinv[qs * 16 + h];
         }
         ++items;
       }
@@ -565,20 +568,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
 #pragma unroll
           for (int c = 0; c < 8; ++c) vr[c] = make_uint4(0, 0, 0, 0);
         }
-        float x[kN];
+        float x[NH];
         bool need = false;
 #pragma unroll
-        for (int h = 0; h < kN; ++h) {
+        for (int h = 0; h < NH; ++h) {
           x[h] = (valid && h < g) ? (s[h] + s[kN + h]) * hscale[h] : -INFINITY;
           need |= x[h] > m_used[h] + kRescaleLog2;
         }
         // P row of this token: each term is a 16-byte chunk (heads 0..15) at
         // (t/8)*128 + (t%8)*16 of its 2 KiB third of the buffer.
-        float pv[kN];
+        float pv[NH];
         auto write_p = [&]() {
-          uint32_t ph[kN / 2], pm[kN / 2], pl[kN / 2];
+          uint32_t ph[kN / 2], pm[kN / 2], pl[kN / 2];  // pairs of heads; those from NH on stay 0
 #pragma unroll
-          for (int j = 0; j < kN / 2; ++j) {
+          for (int j = NH / 2; j < kN / 2; ++j) ph[j] = pm[j] = pl[j] = 0u;
+#pragma unroll
+          for (int j = 0; j < NH / 2; ++j) {
             const int h0 = 2 * j, h1 = 2 * j + 1;
             const float p0 =
                 (valid && h0 < g && m_used[h0] > -INFINITY) ? fast_exp2(x[h0] - m_used[h0] + kPShift) : 0.f;
@@ -612,16 +617,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         if (need_any) {
           // a score outgrew the held maximum (or none is held yet): take the tile
           // maximum, fold the accumulated P·V into registers at the old scale, rewrite P
-          const float wmax = tc::warp_col16<true>(x, lane);
-          if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = wmax;
+          const float wmax = tc::warp_col<true, NH>(x, lane);
+          if (lane % kColLanes == 0) red[warp * 16 + lane / kColLanes] = wmax;
           bool ok = wait_ob(0);
           ok &= wait_ob(1);
           if (!ok) *abort_flag = 1;
           tc::named_barrier_sync(1, kConsumers);
           if (*abort_flag) break;
-          float alpha[kN];
+          float alpha[NH];
 #pragma unroll
-          for (int h = 0; h < kN; ++h) {
+          for (int h = 0; h < NH; ++h) {
             const float tmax = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
             if (h < g) {
               const float m_new = fmaxf(m_used[h], tmax);
@@ -633,17 +638,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           }
           tc::tc_fence_after();
           if (pv_since_restart) {
-            float o[kN];
+            float o[NH];
             load_o(o);
 #pragma unroll
-            for (int h = 0; h < kN; ++h) o_reg[h] = (o_reg[h] + o[h]) * alpha[h];
+            for (int h = 0; h < NH; ++h) o_reg[h] = (o_reg[h] + o[h]) * alpha[h];
           } else {
 #pragma unroll
-            for (int h = 0; h < kN; ++h) o_reg[h] *= alpha[h];
+            for (int h = 0; h < NH; ++h) o_reg[h] *= alpha[h];
           }
           tc::tc_fence_before();
 #pragma unroll
-          for (int h = 0; h < kN; ++h) lp[h] *= alpha[h];
+          for (int h = 0; h < NH; ++h) lp[h] *= alpha[h];
           restart = true;
           pv_since_restart = false;
           write_p();
@@ -652,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           tc::named_barrier_sync(1, kConsumers);
         }
 #pragma unroll
-        for (int h = 0; h < kN; ++h)
+        for (int h = 0; h < NH; ++h)
           if (h < g) lp[h] += pv[h];
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
@@ -667,27 +672,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         bool ok = wait_ob(0);
         ok &= wait_ob(1);
         tc::tc_fence_after();
-        float ot[kN];
+        float ot[NH];
         if (pv_since_restart) {
-          float o[kN];
+          float o[NH];
           load_o(o);
 #pragma unroll
-          for (int h = 0; h < kN; ++h) ot[h] = (o_reg[h] + o[h]) * out_scale;
+          for (int h = 0; h < NH; ++h) ot[h] = (o_reg[h] + o[h]) * out_scale;
         } else {
 #pragma unroll
-          for (int h = 0; h < kN; ++h) ot[h] = o_reg[h] * out_scale;
+          for (int h = 0; h < NH; ++h) ot[h] = o_reg[h] * out_scale;
         }
         tc::tc_fence_before();
         if (!ok) *abort_flag = 1;
         float* red2 = red + 64;
-        const float wsum = tc::warp_col16<false>(lp, lane);
-        if ((lane & 1) == 0) red2[warp * 16 + (lane >> 1)] = wsum;
+        const float wsum = tc::warp_col<false, NH>(lp, lane);
+        if (lane % kColLanes == 0) red2[warp * 16 + lane / kColLanes] = wsum;
         tc::named_barrier_sync(1, kConsumers);
         const int seq = mt.x, kvh = mt.y & 0xffff, part = mt.z & 0xffff, nparts = mt.z >> 16;
         const int d = tid;
         const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
 #pragma unroll
-        for (int h = 0; h < kN; ++h) {
+        for (int h = 0; h < NH; ++h) {
           if (h >= g) break;
           const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
           if (nparts == 1) {
@@ -730,9 +735,9 @@ static int encode_map(CUtensorMap* map, const void* base, uint64_t rows, bool e4
   return PKV_OK;
 }
 
-template <bool OUT_F32>
+template <bool OUT_F32, int NH>
 static int launch(const Args& args, cudaStream_t stream) {
-  auto kernel = decode_gqa_tc_fp8_kernel<OUT_F32>;
+  auto kernel = decode_gqa_tc_fp8_kernel<OUT_F32, NH>;
   static std::once_flag once;
   static cudaError_t setup = cudaSuccess;
   std::call_once(once,
@@ -761,7 +766,12 @@ int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cu
   if (rc == PKV_OK)
     rc = tc8::encode_map(&args.tm_q, a.query, static_cast<uint64_t>(a.num_seqs) * a.num_heads, false, "query");
   if (rc != PKV_OK) return rc;
-  rc = out_f32 ? tc8::launch<true>(args, stream) : tc8::launch<false>(args, stream);
+  if (a.group <= 4)
+    rc = out_f32 ? tc8::launch<true, 4>(args, stream) : tc8::launch<false, 4>(args, stream);
+  else if (a.group <= 8)
+    rc = out_f32 ? tc8::launch<true, 8>(args, stream) : tc8::launch<false, 8>(args, stream);
+  else
+    rc = out_f32 ? tc8::launch<true, 16>(args, stream) : tc8::launch<false, 16>(args, stream);
   if (rc != PKV_OK) return rc;
   return launch_merge_partials(a, out_f32, stream);
 }

@@ -190,6 +190,32 @@ __device__ __forceinline__ float warp_col16(const float (&x)[16], int lane) {
 
 
 
+// The same reduction for NH = 4, 8 or 16 columns: log2(NH) transposing rounds, then
+// plain butterfly rounds over the rest of the warp.  Column lane / (32 / NH) ends up
+// in every lane of its group of 32 / NH lanes.
+template <bool MAX, int NH>
+__device__ __forceinline__ float warp_col(const float (&x)[NH], int lane) {
+  static_assert(NH == 4 || NH == 8 || NH == 16, "4, 8 or 16 columns");
+  auto op = [](float u, float w) { return MAX ? fmaxf(u, w) : u + w; };
+  float v[NH];
+#pragma unroll
+  for (int i = 0; i < NH; ++i) v[i] = x[i];
+  int off = 16;
+#pragma unroll
+  for (int w = NH; w > 1; w >>= 1, off >>= 1) {
+    const bool up = lane & off;
+#pragma unroll
+    for (int i = 0; i < w / 2; ++i) {
+      const float send = up ? v[i] : v[i + w / 2];
+      const float keep = up ? v[i + w / 2] : v[i];
+      v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, off));
+    }
+  }
+#pragma unroll
+  for (; off >= 1; off >>= 1) v[0] = op(v[0], __shfl_xor_sync(0xffffffffu, v[0], off));
+  return v[0];
+}
+
 // 3-D tensor-map load (coordinates innermost first).
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar,
                                             uint64_t policy) {

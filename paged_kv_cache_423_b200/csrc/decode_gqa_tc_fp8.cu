@@ -55,17 +55,25 @@ constexpr int kQSlot = 4096;               // bf16 queries (2 halves x 16 rows x
 constexpr int kQSlots = 6;                 // by item ordinal; a slot is refilled 6 items later
 constexpr int kPTerm = kTile * 16;         // one e5m2 term of P: 128 tokens x 16 heads
 constexpr int kPBytes = 3 * kPTerm;        // [hi | mid | lo]
-constexpr int kConsumers = 128;            // warps 0-3
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kQueryWarp = 6;
-constexpr int kThreads = 224;
+constexpr int kSoftmax = 256;              // warps 0-7: two groups of 4 (head pairs 0, 2, .. and 1, 3, ..)
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kQueryWarp = 10;
+constexpr int kThreads = 384;              // 3 warpgroups; warp 11 only lends registers
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); the
+// control warpgroup drops to 88 and the two softmax warpgroups rise to 208:
+// 128 x (208 + 208 + 88) = 64512, and per scheduler (one warp of each group)
+// 32 x 504 = 16128 <= 16384 registers.
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsControl = 88;
+static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 128;        // S double buffer [0,32), [32,64) (hi | lo); O [64,112) (3 terms)
 constexpr uint32_t kColO = 64;
 constexpr uint32_t kChunkTx = 2 * kChunk * kRow8;  // K and V of one slice
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kPShift = 7.f;             // P is stored times 2^7 (at most 2^15)
-// Stage metadata: x = sequence, y = kv head | q slot << 16, z = partition | partitions << 16,
+// Stage metadata: x = sequence, y = kv head | q slot << 16 | phase of the slot's barrier << 20,
+// z = partition | partitions << 16,
 // w = valid rows (8 bits) | slice mask << 8 | first << 16 | last << 17 | end of stream << 18
 constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
 
@@ -74,7 +82,7 @@ constexpr int kOffStage = 0;
 constexpr int kOffQ = kOffStage + kStages * kStage8;
 constexpr int kOffP = kOffQ + kQSlots * kQSlot;
 constexpr int kOffRed = kOffP + 2 * kPBytes;
-constexpr int kOffMeta = kOffRed + 2 * 4 * 16 * 4;
+constexpr int kOffMeta = kOffRed + 2 * 2 * 4 * 16 * 4;  // [group][maxima | sums][4 warps][16]
 constexpr int kOffScale = kOffMeta + kStages * 16;  // [stage] (k_scale, v_scale) of the item
 constexpr int kOffQinv = kOffScale + kStages * 8;   // [q slot][16] 2^-e of each head
 constexpr int kOffBar = kOffQinv + kQSlots * 16 * 4;
@@ -169,12 +177,14 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, floa
 //   producer     -> full[s]    : e4m3 K, V (and the bf16 queries on an item's first tile) in stage s
 //   query warp   -> q_ready[j] : the queries of the item in q slot j split into e4m3 hi/lo
 //   MMA          -> s_full[b]  : S of the b-th valid tile (mod 2) in TMEM
-//   softmax      -> s_free[b]  : that S read
-//   softmax      -> p_full[b]  : P of that tile in shared buffer b (and its stale V rows zeroed)
+//   softmax      -> s_free[b]  : that S read (8 warps)
+//   softmax      -> p_full[b]  : P of that tile in shared buffer b (and its stale V rows zeroed; 8 warps)
 //   MMA          -> o_bar[b]   : its O += Vᵀ·P done (P buffer b reusable)
 //   MMA + softmax + query warp -> empty[s] : stage s done with: its P·V complete
 //                  (commit; a plain arrival for a tile with no rows), metadata read by
-//                  the 4 softmax warps and the query warp (6 arrivals)
+//                  the 8 softmax warps and the query warp (10 arrivals)
+// Each tile's heads are split between the two softmax groups; they take every
+// decision that touches the shared O accumulator (a rescale restarts it) together.
 // NH (4, 8 or 16 >= g) bounds the heads the softmax works on; the operand layouts
 // keep 16 head slots.
 template <bool OUT_F32, int NH>
@@ -210,25 +220,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4 + 1);
+      mbar_init(&empty[s], 1 + 8 + 1);
     }
     for (int j = 0; j < kQSlots; ++j) mbar_init(&q_ready[j], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&s_free[b], 8);
+      mbar_init(&p_full[b], 8);
       mbar_init(&o_bar[b], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
+  // P bytes of head pairs from NH / 2 on are never written: they stay zero.
+  for (int i = tid; i < 2 * kPBytes / 16; i += blockDim.x) reinterpret_cast<uint4*>(p_buf)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
   if (warp == 0) tc::tmem_alloc(tmem_slot, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= kProducerWarp) {
+  // The control warpgroup gives registers back; the branch is uniform per warpgroup,
+  // as setmaxnreg requires, and dominates the code that runs with the new count.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == kProducerWarp) {
     // ================= producer: e4m3 slices and an item's queries =================
     const uint64_t policy = l2_policy_kv();
@@ -308,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         }
         const bool with_q = tile == 0 && ntok > 0;
         if (lane == 0) {
-          meta[slot] = make_int4(e.x, kvh | (qslot << 16), e.y | (e.z << 16),
+          meta[slot] = make_int4(e.x, kvh | (qslot << 16) | (((item_ord / kQSlots) & 1) << 20), e.y | (e.z << 16),
                                  n_valid | (mask << 8) | (tile == 0 ? kMetaFirst : 0) |
                                      (tile == ntiles - 1 ? kMetaLast : 0));
           mscale[slot] = sc_cur;
@@ -367,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       const int4 mt = meta[slot];
       if (mt.w & kMetaEnd) break;
       if ((mt.w & kMetaFirst) && (mt.w & 0xff) > 0) {
-        const int qs = mt.y >> 16;
+        const int qs = (mt.y >> 16) & 0xf;
         unsigned char* qb = q_ring + qs * kQSlot;
         // bf16 row r of half h: 128 bytes, 16-byte chunk c at (c ^ (r % 8)) * 16
         uint4 v[8];
@@ -415,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       __syncwarp();
       // every item's first tile completes one phase of its slot's barrier (an empty
       // item's too), so the phase of item i in slot i % 6 is (i / 6) & 1 for all roles
-      if ((mt.w & kMetaFirst) && lane == 0) mbar_arrive(&q_ready[mt.y >> 16]);
+      if ((mt.w & kMetaFirst) && lane == 0) mbar_arrive(&q_ready[(mt.y >> 16) & 0xf]);
       if (lane == 0) mbar_arrive(&empty[slot]);  // metadata read
     }
   } else if (warp == kMmaWarp) {
@@ -426,7 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       constexpr uint32_t idesc_pv = tc::instr_desc_e4m3(kD, 3 * kN) | (1u << 10) | (1u << 15) | (1u << 16);
       const uint32_t p_addr0 = smem_addr(p_buf);
       int q_valid = 0, p_valid = 0;  // valid tiles that got their QK / PV
-      int items = 0;                 // items whose first tile has been seen
       int prev_slot = -1, prev_nv = 0;
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -466,13 +482,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         if (nv == 0) {
           if (prev_slot >= 0) issue_pv();
           mbar_arrive(&empty[slot]);
-          items += first;
           continue;
         }
         // S = K·[hi; lo]ᵀ of tile n
-        const int qs = mt.y >> 16;
-        if (first && !wait(&q_ready[qs], (items / kQSlots) & 1)) break;
-        items += first;
+        const int qs = (mt.y >> 16) & 0xf;
+        if (first && !wait(&q_ready[qs], (mt.y >> 20) & 1)) break;
         const int b = q_valid & 1;
         if (q_valid >= 2 && !wait(&s_free[b], ((q_valid >> 1) - 1) & 1)) break;
         tc::tc_fence_after();
@@ -495,32 +509,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       mbar_wait(drain, 0);
     }
     __syncwarp();
+  }
   } else {
-    // ================= softmax warps (one thread per TMEM lane) =================
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m_used[NH], lp[NH], o_reg[NH], hscale[NH];
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    // ================= softmax: thread = token row of the tile = TMEM lane =================
+    // Group G (warps 4G .. 4G+3) takes head pairs G, G+2, G+4, ..: local head j is
+    // head 4 (j / 2) + 2G + j % 2.  Both groups walk every tile together.
+    constexpr int NL = NH / 2;               // heads of one group
+    constexpr int kColLanes = 32 / NL;       // lanes sharing one column after warp_col
+    const int G = warp >> 2;
+    const int t = tid & 127;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float* red_max = red + G * 128;          // [4 warps][16]
+    float* red_sum = red_max + 64;           // [4 warps][16]
+    auto head = [&](int j) { return 4 * (j >> 1) + 2 * G + (j & 1); };
+    float m_used[NL], lp[NL], o_reg[NL], hscale[NL];
 #pragma unroll
-    for (int h = 0; h < NH; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f, hscale[h] = 0.f;
+    for (int j = 0; j < NL; ++j) m_used[j] = -INFINITY, lp[j] = 0.f, o_reg[j] = 0.f, hscale[j] = 0.f;
     float out_scale = 1.f;
     bool restart = true;
     bool pv_since_restart = false;
-    int n_valid_tiles = 0, items = 0;
+    int n_valid_tiles = 0;
     uint32_t ob_next = 0, ob_pending = 0;
     auto wait_ob = [&](int b) -> bool {
       if (!((ob_pending >> b) & 1)) return true;
       ob_pending &= ~(1u << b);
       return mbar_wait(&o_bar[b], ((ob_next >> b) & 1) ^ 1u);
     };
-    // O (sum of the three terms' columns) of this thread's row
-    auto load_o = [&](float (&o)[NH]) {
+    // this group's heads of O (sum of the three terms' columns) in this thread's row
+    auto load_o = [&](float (&o)[NL]) {
       float o3[3 * kN];
       tc::tmem_load32f_nowait(tmem + lane_base + kColO, o3);
       tc::tmem_load32f_nowait(tmem + lane_base + kColO + 32, o3 + 32);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int h = 0; h < NH; ++h) o[h] = o3[h] + o3[kN + h] + o3[2 * kN + h];
+      for (int j = 0; j < NL; ++j) {
+        const int h0 = 4 * (j >> 1) + (j & 1);  // head of group 0; group 1's is h0 + 2
+        o[j] = G ? o3[h0 + 2] + o3[kN + h0 + 2] + o3[2 * kN + h0 + 2] : o3[h0] + o3[kN + h0] + o3[2 * kN + h0];
+      }
     };
-    constexpr int kColLanes = 32 / NH;  // lanes sharing one column after warp_col
     for (int n = 0;; ++n) {
       const int slot = n % kStages;
       bool bad = !mbar_wait(&full[slot], (n / kStages) & 1);
@@ -528,26 +555,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       const float2 sc = mscale[slot];
       if (bad) *abort_flag = 1;
       if ((mt.w & kMetaEnd) || bad) break;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);  // metadata read
       const int n_valid = mt.w & 0xff;
       const uint32_t mask = (mt.w >> 8) & 0xff;
       const bool first = mt.w & kMetaFirst, last = mt.w & kMetaLast;
       if (first) {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f;
+        for (int j = 0; j < NL; ++j) m_used[j] = -INFINITY, lp[j] = 0.f, o_reg[j] = 0.f;
         restart = true;
         pv_since_restart = false;
         out_scale = sc.y;
         if (n_valid > 0) {
-          const int qs = mt.y >> 16;
-          bad |= !mbar_wait(&q_ready[qs], (items / kQSlots) & 1);
+          const int qs = (mt.y >> 16) & 0xf;
+          bad |= !mbar_wait(&q_ready[qs], (mt.y >> 20) & 1);
           const float base = a.scale_log2 * sc.x;
 #pragma unroll
-          for (int h = 0; h < NH; ++h) hscale[h] = base * qinv[qs * 16 + h];
+          for (int j = 0; j < NL; ++j) hscale[j] = base * qinv[qs * 16 + head(j)];
         }
-        ++items;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);  // metadata (and this item's query scales) read
       if (n_valid > 0) {
         const int b = n_valid_tiles & 1;
         unsigned char* p_tile = p_buf + b * kPBytes;
@@ -560,50 +586,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[b]);
         bad |= !wait_ob(b);  // P buffer b: the P·V of two valid tiles back is done
-        const int t = tid;
         const bool valid = t < n_valid && ((mask >> (t / kChunk)) & 1);
         if (!valid) {
           // V rows outside the context may hold anything (even NaN codes): zero them
-          uint4* vr = reinterpret_cast<uint4*>(stage8 + slot * kStage8 + kVOff + t * kRow8);
+          // (each group half of the row)
+          uint4* vr = reinterpret_cast<uint4*>(stage8 + slot * kStage8 + kVOff + t * kRow8) + 4 * G;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) vr[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 4; ++c) vr[c] = make_uint4(0, 0, 0, 0);
         }
-        float x[NH];
+        float x[NL];
         bool need = false;
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          x[h] = (valid && h < g) ? (s[h] + s[kN + h]) * hscale[h] : -INFINITY;
-          need |= x[h] > m_used[h] + kRescaleLog2;
+        for (int j = 0; j < NL; ++j) {
+          const int h0 = 4 * (j >> 1) + (j & 1);
+          const float sv = G ? s[h0 + 2] + s[kN + h0 + 2] : s[h0] + s[kN + h0];
+          x[j] = (valid && head(j) < g) ? sv * hscale[j] : -INFINITY;
+          need |= x[j] > m_used[j] + kRescaleLog2;
         }
-        // P row of this token: each term is a 16-byte chunk (heads 0..15) at
-        // (t/8)*128 + (t%8)*16 of its 2 KiB third of the buffer.
-        float pv[NH];
+        // P of this token: head pair (2k, 2k+1) of each term is 2 bytes at 2k of the
+        // term's 16-byte chunk at (t/8)*128 + (t%8)*16 of its 2 KiB third of the buffer.
+        float pv[NL];
         auto write_p = [&]() {
-          uint32_t ph[kN / 2], pm[kN / 2], pl[kN / 2];  // pairs of heads; those from NH on stay 0
+          unsigned char* row = p_tile + (t >> 3) * 128 + (t & 7) * 16 + 2 * G;
 #pragma unroll
-          for (int j = NH / 2; j < kN / 2; ++j) ph[j] = pm[j] = pl[j] = 0u;
-#pragma unroll
-          for (int j = 0; j < NH / 2; ++j) {
-            const int h0 = 2 * j, h1 = 2 * j + 1;
-            const float p0 =
-                (valid && h0 < g && m_used[h0] > -INFINITY) ? fast_exp2(x[h0] - m_used[h0] + kPShift) : 0.f;
-            const float p1 =
-                (valid && h1 < g && m_used[h1] > -INFINITY) ? fast_exp2(x[h1] - m_used[h1] + kPShift) : 0.f;
-            uint32_t sum;
-            split_p2(pack_f16x2(p0, p1), ph[j], pm[j], pl[j], sum);
-            pv[h0] = f16lo(sum);
-            pv[h1] = f16hi(sum);
+          for (int k = 0; k < NL / 2; ++k) {
+            const int j0 = 2 * k, j1 = 2 * k + 1;
+            const float p0 = (valid && head(j0) < g && m_used[j0] > -INFINITY)
+                                 ? fast_exp2(x[j0] - m_used[j0] + kPShift) : 0.f;
+            const float p1 = (valid && head(j1) < g && m_used[j1] > -INFINITY)
+                                 ? fast_exp2(x[j1] - m_used[j1] + kPShift) : 0.f;
+            uint32_t ph, pm, pl, sum;
+            split_p2(pack_f16x2(p0, p1), ph, pm, pl, sum);
+            pv[j0] = f16lo(sum);
+            pv[j1] = f16hi(sum);
+            // the codes are the top bytes of the two f16 halves
+            *reinterpret_cast<uint16_t*>(row + 4 * k) = static_cast<uint16_t>(__byte_perm(ph, 0, 0x0031));
+            *reinterpret_cast<uint16_t*>(row + kPTerm + 4 * k) = static_cast<uint16_t>(__byte_perm(pm, 0, 0x0031));
+            *reinterpret_cast<uint16_t*>(row + 2 * kPTerm + 4 * k) = static_cast<uint16_t>(__byte_perm(pl, 0, 0x0031));
           }
-          unsigned char* row = p_tile + (t >> 3) * 128 + (t & 7) * 16;
-          *reinterpret_cast<uint4*>(row) =
-              make_uint4(__byte_perm(ph[0], ph[1], 0x7531), __byte_perm(ph[2], ph[3], 0x7531),
-                         __byte_perm(ph[4], ph[5], 0x7531), __byte_perm(ph[6], ph[7], 0x7531));
-          *reinterpret_cast<uint4*>(row + kPTerm) =
-              make_uint4(__byte_perm(pm[0], pm[1], 0x7531), __byte_perm(pm[2], pm[3], 0x7531),
-                         __byte_perm(pm[4], pm[5], 0x7531), __byte_perm(pm[6], pm[7], 0x7531));
-          *reinterpret_cast<uint4*>(row + 2 * kPTerm) =
-              make_uint4(__byte_perm(pl[0], pl[1], 0x7531), __byte_perm(pl[2], pl[3], 0x7531),
-                         __byte_perm(pl[4], pl[5], 0x7531), __byte_perm(pl[6], pl[7], 0x7531));
         };
         if (bad) *abort_flag = 1;
         bool need_any = true;  // an item's first tile always sets the held maximum
@@ -611,54 +631,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           write_p();
           if (tid == 0) restart_flag[b] = restart;
           fence_proxy_async_smem();
-          need_any = tc::named_barrier_or(1, kConsumers, need || bad);
+          // one decision for both groups: a rescale restarts the shared O
+          need_any = tc::named_barrier_or(1, kSoftmax, need || bad);
           if (*abort_flag) break;
         }
         if (need_any) {
           // a score outgrew the held maximum (or none is held yet): take the tile
           // maximum, fold the accumulated P·V into registers at the old scale, rewrite P
-          const float wmax = tc::warp_col<true, NH>(x, lane);
-          if (lane % kColLanes == 0) red[warp * 16 + lane / kColLanes] = wmax;
+          const float wmax = tc::warp_col<true, NL>(x, lane);
+          if (lane % kColLanes == 0) red_max[(warp & 3) * 16 + lane / kColLanes] = wmax;
           bool ok = wait_ob(0);
           ok &= wait_ob(1);
           if (!ok) *abort_flag = 1;
-          tc::named_barrier_sync(1, kConsumers);
+          // both groups: every P·V into the shared O is complete before either folds it
+          tc::named_barrier_sync(1, kSoftmax);
           if (*abort_flag) break;
-          float alpha[NH];
+          float alpha[NL];
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            const float tmax = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
-            if (h < g) {
-              const float m_new = fmaxf(m_used[h], tmax);
-              alpha[h] = m_used[h] == -INFINITY ? 0.f : fast_exp2(m_used[h] - m_new);
-              m_used[h] = m_new;
+          for (int j = 0; j < NL; ++j) {
+            const float tmax = fmaxf(fmaxf(red_max[j], red_max[16 + j]), fmaxf(red_max[32 + j], red_max[48 + j]));
+            if (head(j) < g) {
+              const float m_new = fmaxf(m_used[j], tmax);
+              alpha[j] = m_used[j] == -INFINITY ? 0.f : fast_exp2(m_used[j] - m_new);
+              m_used[j] = m_new;
             } else {
-              alpha[h] = 1.f;
+              alpha[j] = 1.f;
             }
           }
           tc::tc_fence_after();
           if (pv_since_restart) {
-            float o[NH];
+            float o[NL];
             load_o(o);
 #pragma unroll
-            for (int h = 0; h < NH; ++h) o_reg[h] = (o_reg[h] + o[h]) * alpha[h];
+            for (int j = 0; j < NL; ++j) o_reg[j] = (o_reg[j] + o[j]) * alpha[j];
           } else {
 #pragma unroll
-            for (int h = 0; h < NH; ++h) o_reg[h] *= alpha[h];
+            for (int j = 0; j < NL; ++j) o_reg[j] *= alpha[j];
           }
           tc::tc_fence_before();
 #pragma unroll
-          for (int h = 0; h < NH; ++h) lp[h] *= alpha[h];
+          for (int j = 0; j < NL; ++j) lp[j] *= alpha[j];
           restart = true;
           pv_since_restart = false;
           write_p();
           if (tid == 0) restart_flag[b] = 1;
           fence_proxy_async_smem();
-          tc::named_barrier_sync(1, kConsumers);
+          tc::named_barrier_sync(2 + G, 128);  // the group's maxima read before they are rewritten
         }
 #pragma unroll
-        for (int h = 0; h < NH; ++h)
-          if (h < g) lp[h] += pv[h];
+        for (int j = 0; j < NL; ++j)
+          if (head(j) < g) lp[j] += pv[j];
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
         ob_next ^= 1u << b;
@@ -672,37 +694,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         bool ok = wait_ob(0);
         ok &= wait_ob(1);
         tc::tc_fence_after();
-        float ot[NH];
+        float ot[NL];
         if (pv_since_restart) {
-          float o[NH];
+          float o[NL];
           load_o(o);
 #pragma unroll
-          for (int h = 0; h < NH; ++h) ot[h] = (o_reg[h] + o[h]) * out_scale;
+          for (int j = 0; j < NL; ++j) ot[j] = (o_reg[j] + o[j]) * out_scale;
         } else {
 #pragma unroll
-          for (int h = 0; h < NH; ++h) ot[h] = o_reg[h] * out_scale;
+          for (int j = 0; j < NL; ++j) ot[j] = o_reg[j] * out_scale;
         }
         tc::tc_fence_before();
         if (!ok) *abort_flag = 1;
-        float* red2 = red + 64;
-        const float wsum = tc::warp_col<false, NH>(lp, lane);
-        if (lane % kColLanes == 0) red2[warp * 16 + lane / kColLanes] = wsum;
-        tc::named_barrier_sync(1, kConsumers);
+        const float wsum = tc::warp_col<false, NL>(lp, lane);
+        if (lane % kColLanes == 0) red_sum[(warp & 3) * 16 + lane / kColLanes] = wsum;
+        tc::named_barrier_sync(2 + G, 128);
         const int seq = mt.x, kvh = mt.y & 0xffff, part = mt.z & 0xffff, nparts = mt.z >> 16;
-        const int d = tid;
+        const int d = t;
         const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          if (h >= g) break;
-          const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
+        for (int j = 0; j < NL; ++j) {
+          const int h = head(j);
+          if (h >= g) break;  // heads of a group increase with j
+          const float l = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
           if (nparts == 1) {
-            store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[h] / l : 0.f);
+            store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[j] / l : 0.f);
           } else {
             // unnormalised partial (weights times 2^7 in both o and l); the merge
             // kernel combines the partitions
             const int64_t pidx = (unit0 + h) * a.max_parts + part;
-            a.part_o[pidx * kD + d] = ot[h];
-            if (d == 0) a.part_ml[pidx] = make_float2(m_used[h], l);
+            a.part_o[pidx * kD + d] = ot[j];
+            if (d == 0) a.part_ml[pidx] = make_float2(m_used[j], l);
           }
         }
       }

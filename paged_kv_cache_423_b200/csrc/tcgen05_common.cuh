@@ -190,12 +190,12 @@ __device__ __forceinline__ float warp_col16(const float (&x)[16], int lane) {
 
 
 
-// The same reduction for NH = 4, 8 or 16 columns: log2(NH) transposing rounds, then
+// The same reduction for NH = 2, 4, 8 or 16 columns: log2(NH) transposing rounds, then
 // plain butterfly rounds over the rest of the warp.  Column lane / (32 / NH) ends up
 // in every lane of its group of 32 / NH lanes.
 template <bool MAX, int NH>
 __device__ __forceinline__ float warp_col(const float (&x)[NH], int lane) {
-  static_assert(NH == 4 || NH == 8 || NH == 16, "4, 8 or 16 columns");
+  static_assert(NH == 2 || NH == 4 || NH == 8 || NH == 16, "2, 4, 8 or 16 columns");
   auto op = [](float u, float w) { return MAX ? fmaxf(u, w) : u + w; };
   float v[NH];
 #pragma unroll

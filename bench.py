@@ -84,7 +84,8 @@ def measured_hbm_gbs():
 # Sources each kernel family is compiled from: a recorded ncu traffic figure is only
 # reported while these files are the ones it was measured on.
 KERNEL_SOURCES = {
-    "decode": ["decode.cu", "decode_gqa_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
+    "decode": ["decode.cu", "decode_gqa_tc.cu", "decode_gqa_tc_fp8.cu", "decode_common.cuh", "device_common.cuh",
+               "tcgen05_common.cuh"],
     "prefill": ["prefill_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
 }
 
@@ -110,6 +111,25 @@ def recorded_traffic(key: str, kind: str = "decode"):
     if not entry or entry.get("sources") != source_digest(kind):
         return None
     return int(entry["dram_bytes_per_launch"])
+
+
+def split_tokens(num_seqs, num_kv_heads, block_size, max_context_len, tensor):
+    """The library's automatic split of a context (tokens per partition) for a call:
+    the CUDA-core path takes the largest of 512..64 that leaves >= 4096 work items,
+    the tensor-core paths the largest of 2048.. down to that which leaves >= 16 items
+    per SM.  Used to count the launches of a step (a split context adds the merge)."""
+    def items(p):
+        return num_seqs * num_kv_heads * -(-max_context_len // p)
+    base = 512
+    while base > 64 and items(base) < 4096:
+        base //= 2
+    base = max(base, block_size)
+    if not tensor:
+        return base
+    p = 2048
+    while p > base and items(p) < 16 * 148:
+        p //= 2
+    return max(p, base)
 
 
 def rank_info():
@@ -254,7 +274,7 @@ class Workload:
     def decode(self, out, q, tables, lens, max_len, ws, path, status):
         if self.kv8:
             self.pkv.paged_attention_decode_fp8(out, q, self.key_cache, self.value_cache, self.k_scale, self.v_scale,
-                                                tables, lens, max_len, self.scale, ws, status=status)
+                                                tables, lens, max_len, self.scale, ws, path=path, status=status)
         else:
             self.pkv.paged_attention_decode(out, q, self.key_cache, self.value_cache, tables, lens, max_len, self.scale,
                                             ws, path=path, status=status)
@@ -346,12 +366,16 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     launches = 0
     kv_total = bytes_total = 0
+    g = w.Hq // w.Hkv
+    uses_tensor = path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16)
+    # write, plan, decode (+ copy_blocks when a fork copied blocks) (+ the merge of a split context)
+    merge = 1 if uses_tensor and max_len_all > split_tokens(w.B, w.Hkv, w.bs, max_len_all, True) else 0
     for i in range(args.warmup, total):
         st = states[i % n_states]
         kv, alg = decode_bytes(st["host_lens"], w.Hq, w.Hkv, w.D, w.bs, 1 if kv8 else 2)
         kv_total += kv
         bytes_total += alg
-        launches += 3 + (1 if st["n_pairs"] else 0)
+        launches += 3 + (1 if st["n_pairs"] else 0) + merge
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -378,8 +402,6 @@ def run_ours(args, rank, world, local_rank):
     e2e = run_e2e(args, w, pkv, device, path, ws, out, status, max_len_all) if not args.no_e2e else None
 
     peak, peak_kind = measured_hbm_gbs()
-    g = w.Hq // w.Hkv
-    uses_tensor = not kv8 and (path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16))
     dec_gbs = bytes_total / (dec_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -395,7 +417,9 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4), "traffic": recorded_traffic(w.name + ("+fp8" if kv8 else "")),
                      "algorithmic_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
-                     "kernel": ("paged_attention_decode_fp8: plan + CUDA-core streaming kernel (e4m3 tiles)" if kv8
+                     "kernel": ("paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"
+                                " + split merge" if kv8 and uses_tensor
+                                else "paged_attention_decode_fp8: plan + CUDA-core streaming kernel (e4m3 tiles)" if kv8
                                 else "paged_attention_decode: plan + tcgen05 kernel + split merge" if uses_tensor
                                 else "paged_attention_decode: plan + CUDA-core streaming kernel"),
                      "ms_per_launch": round(dec_ms / args.steps, 4)},

@@ -64,3 +64,18 @@ def test_prefill_flops_counts_every_visible_key():
         for i in range(n):
             brute += (L - n + i) + 1
     assert bench.prefill_flops(qlens, lens, 5, 128) == 4 * 128 * 5 * brute
+
+
+def test_split_tokens_mirrors_the_library():
+    """bench.split_tokens counts the merge launch of a split context; on the CUDA-core
+    path it must be the library's own automatic split, and the tensor-core split is
+    never shorter than it and at most 2048 tokens."""
+    import paged_kv_cache_423_b200 as pkv
+    for B in (1, 3, 16, 128, 256):
+        for hkv in (1, 8, 40):
+            for bs in (16, 32):
+                for L in (1, 100, 2049, 32768, 131072):
+                    simt = bench.split_tokens(B, hkv, bs, L, False)
+                    assert simt == pkv.paged_attention_partition_tokens(B, hkv, bs, L)
+                    tensor = bench.split_tokens(B, hkv, bs, L, True)
+                    assert simt <= tensor <= 2048 and tensor % bs == 0

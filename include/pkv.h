@@ -401,6 +401,16 @@ PKV_API int pkv_bm_add_seq_tokens(pkv_bm* bm, int64_t seq_id, const int32_t* tok
                                   int* cached_tokens_out);
 PKV_API int pkv_bm_num_cached_blocks(const pkv_bm* bm);
 
+/*
+ * stream_read — measurement helper, not part of the attention path: reads `bytes` of
+ * device memory once (16-byte non-caching loads, 4 CTAs of 512 threads per SM) and
+ * XORs every 32-bit word of it into *sink (device, 4-byte aligned; the caller sets it
+ * first, usually to 0).  Timing it gives the HBM read bandwidth reached in the same
+ * run as the decode kernels (the roofline's read-only reference next to the measured
+ * copy peak).  src 16-byte aligned, bytes a multiple of 16; PKV_ERR_INVALID otherwise.
+ */
+PKV_API int pkv_stream_read(const void* src, size_t bytes, uint32_t* sink, pkv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,7 +22,7 @@ __all__ = [
     "reshape_and_cache", "copy_blocks", "paged_attention_workspace_size", "paged_attention_partition_tokens",
     "paged_attention_decode", "paged_attention_decode_static", "STATIC_SCRATCH_BYTES",
     "paged_attention_prefill_workspace_size", "paged_attention_prefill", "reshape_and_cache_fp8",
-    "paged_attention_decode_fp8", "swap_blocks", "BlockManager",
+    "paged_attention_decode_fp8", "swap_blocks", "BlockManager", "stream_read",
 ]
 
 PKV_OK = 0
@@ -83,6 +83,7 @@ _SIGNATURES = {
                                                c_int, c_float, c_int, c_int, c_void_p, c_size_t, c_void_p,
                                                c_void_p]),
     "pkv_swap_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int64, c_void_p, c_void_p]),
+    "pkv_stream_read": (c_int, [c_void_p, c_size_t, c_void_p, c_void_p]),
     "pkv_bm_create": (c_void_p, [c_int, c_int, c_void_p]),
     "pkv_bm_create_with_swap_space": (c_void_p, [c_int, c_int, c_void_p, c_int]),
     "pkv_bm_num_host_free": (c_int, [c_void_p]),
@@ -359,6 +360,15 @@ def swap_blocks(src_pool, dst_pool, block_mapping, status=None, stream=None):
                                    int(dst_pool.shape[0]), block_bytes, _ptr(status, torch.int32, "status"),
                                    _stream(stream))
     _check(rc, "swap_blocks")
+
+
+def stream_read(buf, sink, stream=None):
+    """Read the contiguous device tensor `buf` once, XOR-folding its 32-bit words into
+    sink (a 1-element int32 device tensor, set by the caller).  A bandwidth reference."""
+    torch = _torch()
+    nbytes = buf.numel() * buf.element_size()
+    rc = library().pkv_stream_read(_ptr(buf, None, "buf"), nbytes, _ptr(sink, torch.int32, "sink"), _stream(stream))
+    _check(rc, "stream_read")
 
 
 def paged_attention_prefill_workspace_size(num_seqs, total_q, num_heads, num_kv_heads) -> int:

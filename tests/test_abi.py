@@ -72,6 +72,12 @@ def test_argument_errors_before_any_device_work(pkv):
     assert lib.pkv_reshape_and_cache(fake, fake, fake, fake, fake, 0, 8, 2, 128, 16, None, None) == pkv.PKV_OK
     assert lib.pkv_copy_blocks(None, None, 0, None, 0, 8, 4096, None, None) == pkv.PKV_OK
     assert lib.pkv_copy_blocks(None, None, 1, None, 3, 8, 4095, None, None) == pkv.PKV_ERR_INVALID
+    # the bandwidth reference: sizes and alignment are checked before any launch
+    assert lib.pkv_stream_read(fake, 0, fake, None) == pkv.PKV_OK
+    assert lib.pkv_stream_read(fake, 40, fake, None) == pkv.PKV_ERR_INVALID
+    assert lib.pkv_stream_read(None, 64, fake, None) == pkv.PKV_ERR_INVALID
+    assert lib.pkv_stream_read(ctypes.c_void_p(0x1008), 64, fake, None) == pkv.PKV_ERR_INVALID
+    assert lib.pkv_stream_read(fake, 64, ctypes.c_void_p(0x1002), None) == pkv.PKV_ERR_INVALID
 
 
 def test_prefill_argument_errors_before_any_device_work(pkv):

@@ -79,3 +79,20 @@ def test_split_tokens_mirrors_the_library():
                     assert simt == pkv.paged_attention_partition_tokens(B, hkv, bs, L)
                     tensor = bench.split_tokens(B, hkv, bs, L, True)
                     assert simt <= tensor <= 2048 and tensor % bs == 0
+
+
+def test_all_cores_oracle_counts_every_sequence():
+    """The all-cores oracle leg (spawned workers) processes every sampled sequence once."""
+    import types
+    import workloads as wl
+    b = wl.make_decode_batch("tiny")
+    w = types.SimpleNamespace(Hkv=b.num_kv_heads, D=b.head_dim, scale=b.scale)
+    items = []
+    for s in range(b.num_seqs):
+        need = -(-int(b.context_lens[s]) // b.block_size)
+        blocks = b.block_tables[s][:need]
+        items.append((b.query[s:s + 1], b.key_cache[blocks], b.value_cache[blocks],
+                      np.arange(need, dtype=np.int32)[None, :], b.context_lens[s:s + 1]))
+    done, dt, cores = bench.time_oracle_all_cores(w, items)
+    assert done == int(b.context_lens.sum()) * b.num_kv_heads * b.head_dim * 4
+    assert cores >= 1 and dt > 0

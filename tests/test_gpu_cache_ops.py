@@ -74,3 +74,17 @@ def test_copy_blocks_bad_pair(pkv):
     assert status.item() == pkv.PKV_DEV_BAD_PAIR
     exp, _ = cache_ops.copy_blocks([kc], [kc], np.array([[1, 2]]))
     assert np.array_equal(host_bits(dk), exp[0])
+
+
+@pytest.mark.parametrize("nbytes", [16, 48, 4096 + 32, (64 << 20) + 208])
+def test_stream_read_folds_every_word(pkv, nbytes):
+    """The bandwidth reference reads every byte once: its XOR of all 32-bit words equals
+    numpy's on seeded bytes (sizes down to one 16-byte chunk, ragged grid tails)."""
+    rng = np.random.default_rng(nbytes)
+    host = rng.integers(0, 256, size=nbytes, dtype=np.uint8)
+    buf = torch.from_numpy(host).cuda()
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.stream_read(buf, sink)
+    torch.cuda.synchronize()
+    want = np.bitwise_xor.reduce(host.view(np.uint32))
+    assert np.uint32(sink.cpu().numpy().view(np.uint32)[0]) == want

@@ -82,7 +82,7 @@ def test_split_tokens_mirrors_the_library():
 
 
 def test_all_cores_oracle_counts_every_sequence():
-    """The all-cores oracle leg (spawned workers) processes every sampled sequence once."""
+    """The all-cores oracle leg (spawned workers) processes every sampled sequence once per pass."""
     import types
     import workloads as wl
     b = wl.make_decode_batch("tiny")
@@ -94,5 +94,5 @@ def test_all_cores_oracle_counts_every_sequence():
         items.append((b.query[s:s + 1], b.key_cache[blocks], b.value_cache[blocks],
                       np.arange(need, dtype=np.int32)[None, :], b.context_lens[s:s + 1]))
     done, dt, cores = bench.time_oracle_all_cores(w, items)
-    assert done == int(b.context_lens.sum()) * b.num_kv_heads * b.head_dim * 4
+    assert done == cores * int(b.context_lens.sum()) * b.num_kv_heads * b.head_dim * 4  # `cores` passes
     assert cores >= 1 and dt > 0

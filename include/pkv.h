@@ -52,7 +52,8 @@ extern "C" {
 #define PKV_ERR_OOM (-2)         /* block pool exhausted; nothing was changed */
 #define PKV_ERR_CUDA (-3)        /* a CUDA runtime call or launch failed */
 #define PKV_ERR_UNSUPPORTED (-4) /* head_dim not in {64,128}, block_size not in {16,32},
-                                    num_heads % num_kv_heads != 0, ... */
+                                    num_heads % num_kv_heads != 0, num_kv_heads > 65535
+                                    (decode), ... */
 
 /* ---- bits of the device status word ---- */
 #define PKV_DEV_BAD_SLOT 0x1     /* reshape_and_cache: slot >= num_blocks*block_size */

@@ -839,6 +839,8 @@ static int decode_impl(void* out, int out_dtype, const void* query, const void* 
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: head_dim %d not in {64,128}", head_dim);
   if (block_size != 16 && block_size != 32)
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: block_size %d not in {16,32}", block_size);
+  if (num_kv_heads > 65535)  // the tensor-core kernels carry the kv head in 16 bits of their stage metadata
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: num_kv_heads %d above 65535", num_kv_heads);
   if (num_heads % num_kv_heads != 0)
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode: num_heads %d not a multiple of num_kv_heads %d",
                      num_heads, num_kv_heads);

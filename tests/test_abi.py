@@ -61,6 +61,7 @@ def test_argument_errors_before_any_device_work(pkv):
     assert call(D=96) == pkv.PKV_ERR_UNSUPPORTED
     assert call(bs=8) == pkv.PKV_ERR_UNSUPPORTED
     assert call(Hq=5) == pkv.PKV_ERR_UNSUPPORTED
+    assert call(Hq=70000, Hkv=70000) == pkv.PKV_ERR_UNSUPPORTED  # kv head ids are 16-bit in the kernels
     assert call(out_dtype=7) == pkv.PKV_ERR_INVALID
     assert call(part=100) == pkv.PKV_ERR_INVALID
     assert call(query=ctypes.c_void_p(0x1008)) == pkv.PKV_ERR_INVALID

@@ -67,8 +67,9 @@ constexpr int kThreads = 384;              // 3 warpgroups; warp 11 only lends r
 constexpr int kRegsSoftmax = 208;
 constexpr int kRegsControl = 88;
 static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kThreads * 168, "register split exceeds the launch");
-constexpr uint32_t kTmemCols = 128;        // S double buffer [0,32), [32,64) (hi | lo); O [64,112) (3 terms)
-constexpr uint32_t kColO = 64;
+constexpr uint32_t kTmemCols = 256;        // S double buffer [0,32), [32,64) (hi | lo); O of even / odd items
+constexpr uint32_t kColO = 64;             // at [64,112) / [128,176) (3 terms of 16 heads each)
+constexpr uint32_t kOStride = 64;
 constexpr uint32_t kChunkTx = 2 * kChunk * kRow8;  // K and V of one slice
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kPShift = 7.f;             // P is stored times 2^7 (at most 2^15)
@@ -82,7 +83,7 @@ constexpr int kOffStage = 0;
 constexpr int kOffQ = kOffStage + kStages * kStage8;
 constexpr int kOffP = kOffQ + kQSlots * kQSlot;
 constexpr int kOffRed = kOffP + 2 * kPBytes;
-constexpr int kOffMeta = kOffRed + 2 * 2 * 4 * 16 * 4;  // [group][maxima | sums][4 warps][16]
+constexpr int kOffMeta = kOffRed + 2 * 3 * 4 * 16 * 4;  // [group][maxima | sums of even | odd items][4 warps][16]
 constexpr int kOffScale = kOffMeta + kStages * 16;  // [stage] (k_scale, v_scale) of the item
 constexpr int kOffQinv = kOffScale + kStages * 8;   // [q slot][16] 2^-e of each head
 constexpr int kOffBar = kOffQinv + kQSlots * 16 * 4;
@@ -211,7 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   uint64_t* drain = o_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  volatile int* restart_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [2]
+  // [P buffer]: bit 0 = the P·V starts a fresh accumulation, bit 1 = O buffer of the item
+  volatile int* restart_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = a.group;
@@ -458,13 +460,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         const int b = p_valid & 1;
         if (!wait(&p_full[b], (p_valid >> 1) & 1)) return;
         tc::tc_fence_after();
-        const bool restart = restart_flag[b] != 0;
+        const int rf = restart_flag[b];
+        const bool restart = rf & 1;
+        const uint32_t o_col = kColO + ((rf >> 1) & 1) * kOStride;
         const uint32_t v_addr = smem_addr(stage8 + prev_slot * kStage8 + kVOff);
         const uint32_t p_addr = p_addr0 + b * kPBytes;
         const int kt = (prev_nv + 31) / 32;
         for (int kk = 0; kk < kt; ++kk) {
           // V: 32 tokens = 4 swizzle atoms of 8 rows; P: 4 groups of 8 tokens x 16 bytes, terms 2 KiB apart
-          tc::umma_f8(tmem + kColO, tc::smem_desc_sw128(v_addr + kk * 4096, kTile * kRow8, 1024),
+          tc::umma_f8(tmem + o_col, tc::smem_desc_sw128(v_addr + kk * 4096, kTile * kRow8, 1024),
                       tc::smem_desc_plain(p_addr + kk * 512, 128, kPTerm), idesc_pv, kk > 0 || !restart);
         }
         tc::umma_commit(&o_bar[b]);
@@ -520,8 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
     const int G = warp >> 2;
     const int t = tid & 127;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    float* red_max = red + G * 128;          // [4 warps][16]
-    float* red_sum = red_max + 64;           // [4 warps][16]
+    float* red_max = red + G * 192;          // [4 warps][16]
+    float* red_sums = red_max + 64;          // [item parity][4 warps][16]
     auto head = [&](int j) { return 4 * (j >> 1) + 2 * G + (j & 1); };
     float m_used[NL], lp[NL], o_reg[NL], hscale[NL];
 #pragma unroll
@@ -530,17 +534,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
     bool restart = true;
     bool pv_since_restart = false;
     int n_valid_tiles = 0;
+    int obuf = 1;  // O buffer of the current item (alternates per item)
+    // An item's output is written one tile later, after the next tile's P is released,
+    // so its last P·V completes meanwhile instead of being waited for.
+    bool fin = false;
+    int4 f_mt = make_int4(0, 0, 0, 0);
+    float f_o[NL], f_lp[NL], f_m[NL];
+    float f_scale = 1.f;
+    int f_ob = 0, f_b = 0;
+    bool f_has_o = false;
     uint32_t ob_next = 0, ob_pending = 0;
     auto wait_ob = [&](int b) -> bool {
       if (!((ob_pending >> b) & 1)) return true;
       ob_pending &= ~(1u << b);
       return mbar_wait(&o_bar[b], ((ob_next >> b) & 1) ^ 1u);
     };
-    // this group's heads of O (sum of the three terms' columns) in this thread's row
-    auto load_o = [&](float (&o)[NL]) {
+    // this group's heads of O buffer ob (sum of the three terms' columns) in this thread's row
+    auto load_o = [&](float (&o)[NL], int ob) {
       float o3[3 * kN];
-      tc::tmem_load32f_nowait(tmem + lane_base + kColO, o3);
-      tc::tmem_load32f_nowait(tmem + lane_base + kColO + 32, o3 + 32);
+      tc::tmem_load32f_nowait(tmem + lane_base + kColO + ob * kOStride, o3);
+      tc::tmem_load32f_nowait(tmem + lane_base + kColO + ob * kOStride + 32, o3 + 32);
       tc::tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < NL; ++j) {
@@ -548,13 +561,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         o[j] = G ? o3[h0 + 2] + o3[kN + h0 + 2] + o3[2 * kN + h0 + 2] : o3[h0] + o3[kN + h0] + o3[2 * kN + h0];
       }
     };
+    // ---- the held item's output: O = registers + TMEM, times the V scale; denominators
+    auto finalize = [&]() {
+      fin = false;
+      bool ok = true;
+      float ot[NL];
+      if (f_has_o) {
+        ok = wait_ob(f_b);  // its last P·V (the latest on P buffer f_b)
+        tc::tc_fence_after();
+        float o[NL];
+        load_o(o, f_ob);
+        tc::tc_fence_before();
+#pragma unroll
+        for (int j = 0; j < NL; ++j) ot[j] = (f_o[j] + o[j]) * f_scale;
+      } else {
+#pragma unroll
+        for (int j = 0; j < NL; ++j) ot[j] = f_o[j] * f_scale;
+      }
+      if (!ok) *abort_flag = 1;
+      float* red_sum = red_sums + f_ob * 64;  // consecutive items use different halves
+      const float wsum = tc::warp_col<false, NL>(f_lp, lane);
+      if (lane % kColLanes == 0) red_sum[(warp & 3) * 16 + lane / kColLanes] = wsum;
+      tc::named_barrier_sync(2 + G, 128);
+      const int seq = f_mt.x, kvh = f_mt.y & 0xffff, part = f_mt.z & 0xffff, nparts = f_mt.z >> 16;
+      const int d = t;
+      const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
+#pragma unroll
+      for (int j = 0; j < NL; ++j) {
+        const int h = head(j);
+        if (h >= g) break;  // heads of a group increase with j
+        const float l = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
+        if (nparts == 1) {
+          store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[j] / l : 0.f);
+        } else {
+          // unnormalised partial (weights times 2^7 in both o and l); the merge
+          // kernel combines the partitions
+          const int64_t pidx = (unit0 + h) * a.max_parts + part;
+          a.part_o[pidx * kD + d] = ot[j];
+          if (d == 0) a.part_ml[pidx] = make_float2(f_m[j], l);
+        }
+      }
+    };
+    bool ended = false;
     for (int n = 0;; ++n) {
       const int slot = n % kStages;
       bool bad = !mbar_wait(&full[slot], (n / kStages) & 1);
       const int4 mt = meta[slot];
       const float2 sc = mscale[slot];
       if (bad) *abort_flag = 1;
-      if ((mt.w & kMetaEnd) || bad) break;
+      if (bad) break;
+      if (mt.w & kMetaEnd) {
+        ended = true;
+        break;
+      }
       const int n_valid = mt.w & 0xff;
       const uint32_t mask = (mt.w >> 8) & 0xff;
       const bool first = mt.w & kMetaFirst, last = mt.w & kMetaLast;
@@ -564,6 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         restart = true;
         pv_since_restart = false;
         out_scale = sc.y;
+        obuf ^= 1;
         if (n_valid > 0) {
           const int qs = (mt.y >> 16) & 0xf;
           bad |= !mbar_wait(&q_ready[qs], (mt.y >> 20) & 1);
@@ -629,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         bool need_any = true;  // an item's first tile always sets the held maximum
         if (!first) {
           write_p();
-          if (tid == 0) restart_flag[b] = restart;
+          if (tid == 0) restart_flag[b] = (restart ? 1 : 0) | (obuf << 1);
           fence_proxy_async_smem();
           // one decision for both groups: a rescale restarts the shared O
           need_any = tc::named_barrier_or(1, kSoftmax, need || bad);
@@ -640,8 +700,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           // maximum, fold the accumulated P·V into registers at the old scale, rewrite P
           const float wmax = tc::warp_col<true, NL>(x, lane);
           if (lane % kColLanes == 0) red_max[(warp & 3) * 16 + lane / kColLanes] = wmax;
-          bool ok = wait_ob(0);
-          ok &= wait_ob(1);
+          bool ok = true;
+          if (pv_since_restart) {  // this item's O is folded below: its P·Vs must be complete
+            ok = wait_ob(0);
+            ok &= wait_ob(1);
+          }
           if (!ok) *abort_flag = 1;
           // both groups: every P·V into the shared O is complete before either folds it
           tc::named_barrier_sync(1, kSoftmax);
@@ -661,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           tc::tc_fence_after();
           if (pv_since_restart) {
             float o[NL];
-            load_o(o);
+            load_o(o, obuf);
 #pragma unroll
             for (int j = 0; j < NL; ++j) o_reg[j] = (o_reg[j] + o[j]) * alpha[j];
           } else {
@@ -674,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           restart = true;
           pv_since_restart = false;
           write_p();
-          if (tid == 0) restart_flag[b] = 1;
+          if (tid == 0) restart_flag[b] = 1 | (obuf << 1);
           fence_proxy_async_smem();
           tc::named_barrier_sync(2 + G, 128);  // the group's maxima read before they are rewritten
         }
@@ -689,46 +752,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         pv_since_restart = true;
         ++n_valid_tiles;
       }
+      if (fin) finalize();  // the previous item: its last P·V ran while this tile was processed
       if (last) {
-        // ---- finalize the item: O = registers + TMEM, times the V scale; denominators
-        bool ok = wait_ob(0);
-        ok &= wait_ob(1);
-        tc::tc_fence_after();
-        float ot[NL];
-        if (pv_since_restart) {
-          float o[NL];
-          load_o(o);
+        fin = true;
+        f_mt = mt;
 #pragma unroll
-          for (int j = 0; j < NL; ++j) ot[j] = (o_reg[j] + o[j]) * out_scale;
-        } else {
-#pragma unroll
-          for (int j = 0; j < NL; ++j) ot[j] = o_reg[j] * out_scale;
-        }
-        tc::tc_fence_before();
-        if (!ok) *abort_flag = 1;
-        const float wsum = tc::warp_col<false, NL>(lp, lane);
-        if (lane % kColLanes == 0) red_sum[(warp & 3) * 16 + lane / kColLanes] = wsum;
-        tc::named_barrier_sync(2 + G, 128);
-        const int seq = mt.x, kvh = mt.y & 0xffff, part = mt.z & 0xffff, nparts = mt.z >> 16;
-        const int d = t;
-        const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
-#pragma unroll
-        for (int j = 0; j < NL; ++j) {
-          const int h = head(j);
-          if (h >= g) break;  // heads of a group increase with j
-          const float l = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
-          if (nparts == 1) {
-            store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[j] / l : 0.f);
-          } else {
-            // unnormalised partial (weights times 2^7 in both o and l); the merge
-            // kernel combines the partitions
-            const int64_t pidx = (unit0 + h) * a.max_parts + part;
-            a.part_o[pidx * kD + d] = ot[j];
-            if (d == 0) a.part_ml[pidx] = make_float2(m_used[j], l);
-          }
-        }
+        for (int j = 0; j < NL; ++j) f_o[j] = o_reg[j], f_lp[j] = lp[j], f_m[j] = m_used[j];
+        f_scale = out_scale;
+        f_ob = obuf;
+        f_has_o = pv_since_restart;
+        f_b = (n_valid_tiles - 1) & 1;  // P buffer of the item's last valid tile
       }
     }
+    if (ended && fin) finalize();
     if (*abort_flag && tid == 0) set_status(a.status, PKV_DEV_TIMEOUT);
   }
   tc::tc_fence_before();

@@ -81,16 +81,17 @@ def measured_hbm_gbs():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# Sources each kernel family is compiled from: a recorded ncu traffic figure is only
+# Sources each profiled kernel is compiled from: a recorded ncu traffic figure is only
 # reported while these files are the ones it was measured on.
 KERNEL_SOURCES = {
-    "decode": ["decode.cu", "decode_gqa_tc.cu", "decode_gqa_tc_fp8.cu", "decode_common.cuh", "device_common.cuh",
-               "tcgen05_common.cuh"],
+    "decode_simt": ["decode.cu", "decode_common.cuh", "device_common.cuh"],
+    "decode_gqa_tc": ["decode_gqa_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
+    "decode_gqa_tc_fp8": ["decode_gqa_tc_fp8.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
     "prefill": ["prefill_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
 }
 
 
-def source_digest(kind: str = "decode") -> str:
+def source_digest(kind: str) -> str:
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "paged_kv_cache_423_b200", "csrc")
@@ -101,7 +102,7 @@ def source_digest(kind: str = "decode") -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(key: str, kind: str = "decode"):
+def recorded_traffic(key: str, kind: str):
     """DRAM bytes (read + write) per launch of the profiled kernel from profiles/traffic.json, or None."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
@@ -440,7 +441,10 @@ def run_ours(args, rank, world, local_rank):
         "seq_steps_per_s": round(seq_steps, 1),
         "pct_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(dec_gbs / peak, 4), "traffic": recorded_traffic(w.name + ("+fp8" if kv8 else "")),
+                     "frac": round(dec_gbs / peak, 4),
+                     "traffic": recorded_traffic(w.name + ("+fp8" if kv8 else ""),
+                                                 ("decode_gqa_tc_fp8" if kv8 else "decode_gqa_tc") if uses_tensor
+                                                 else "decode_simt"),
                      "algorithmic_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
                      "kernel": ("paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"
                                 " + split merge" if kv8 and uses_tensor

@@ -400,6 +400,19 @@ PKV_API int pkv_bm_swap_in(pkv_bm* bm, const int64_t* seq_ids, int n, int64_t* p
  */
 PKV_API int pkv_bm_add_seq_tokens(pkv_bm* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
                                   int* cached_tokens_out);
+/*
+ * append_tokens — pkv_bm_append_slots with the token id of each new position (host [n]
+ * int32; in decode the token whose K/V the slot will hold is known when its slot is
+ * taken).  A sequence created by add_seq_tokens keeps its token history (fork copies
+ * it); when a new token completes a block, that block registers under its chain hash
+ * exactly as a full prompt block does (unless the hash is registered already; in call
+ * order), so a later prompt that continues the generated text finds it.  A plain
+ * pkv_bm_append_slots ends a sequence's history (nothing it fills later registers);
+ * sequences created by add_seq have none.  Slots, copy-on-write pairs, all-or-nothing
+ * and errors as pkv_bm_append_slots.
+ */
+PKV_API int pkv_bm_append_tokens(pkv_bm* bm, const int64_t* seq_ids, const int32_t* tokens, int n,
+                                 int64_t* slots_out, int64_t* cow_pairs_out, int* n_cow_out);
 PKV_API int pkv_bm_num_cached_blocks(const pkv_bm* bm);
 
 /*

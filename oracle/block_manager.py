@@ -53,6 +53,13 @@ vLLM 初探 §1.4: shared system prompts save 30-50% of the memory).  Readings:
   * A registered block whose references drop to zero stays registered while it
     waits in the free list; when the free list hands it out again its
     registration is dropped (eviction in free-list order).
+  * Blocks filled during decode: a sequence created by add_seq_tokens keeps its
+    token history (the chain hash of its last full block and the ids of the block
+    being filled); fork copies it.  append_tokens(seqs, tokens) is append_slots
+    plus one token id per sequence: when a token completes its sequence's block,
+    the block registers under its chain hash like a full prompt block (unless the
+    hash is already registered; sequences in call order).  append_slots, which
+    carries no ids, ends a sequence's history; add_seq sequences have none.
 
 Parity status: pinned (invariants, the pages' block-table example, hand-worked
 copy-on-write, swap and prefix-cache cases, FNV-1a test vectors).
@@ -106,6 +113,7 @@ class BlockManagerModel:
         self.swapped: set[int] = set()
         self.cached: dict[int, int] = {}        # hash -> device block
         self.block_hash: dict[int, int] = {}    # device block -> its registered hash
+        self.hist: dict[int, tuple | None] = {}  # seq -> (parent hash, partial token ids) or None
 
     # -- blocks -------------------------------------------------------------
     def num_free(self) -> int:
@@ -165,6 +173,7 @@ class BlockManagerModel:
         table = shared + [self.alloc() for _ in range(fresh)]
         self.tables[seq_id] = table
         self.lens[seq_id] = num_tokens
+        self.hist[seq_id] = None
 
     def fork(self, parent: int, child: int):
         if parent not in self.tables or child in self.tables or parent in self.swapped:
@@ -174,9 +183,42 @@ class BlockManagerModel:
             self.ref[b] += 1
         self.tables[child] = table
         self.lens[child] = self.lens[parent]
+        h = self.hist.get(parent)
+        self.hist[child] = None if h is None else (h[0], list(h[1]))
 
     def append_slots(self, seq_ids):
-        """One new token per listed sequence; returns (slots, cow_pairs)."""
+        """One new token per listed sequence; returns (slots, cow_pairs).  The
+        sequences' token histories end (nothing they fill later registers)."""
+        slots, pairs = self._append(seq_ids)
+        for s in seq_ids:
+            self.hist[int(s)] = None
+        return slots, pairs
+
+    def append_tokens(self, seq_ids, tokens):
+        """append_slots with the token id of each new position; a tracked sequence
+        registers the block a token completes under its chain hash."""
+        seq_ids = [int(s) for s in seq_ids]
+        tokens = [int(t) for t in tokens]
+        if len(tokens) != len(seq_ids):
+            raise BlockManagerError(ERR_INVALID, "one token per sequence")
+        slots, pairs = self._append(seq_ids)
+        for s, tok in zip(seq_ids, tokens):
+            h = self.hist.get(s)
+            if h is None:
+                continue
+            parent, partial = h
+            partial = partial + [tok]
+            if len(partial) == self.block_size:
+                parent = block_hash(parent, partial)
+                partial = []
+                b = self.tables[s][-1]
+                if b not in self.block_hash and parent not in self.cached:
+                    self.cached[parent] = b
+                    self.block_hash[b] = parent
+            self.hist[s] = (parent, partial)
+        return slots, pairs
+
+    def _append(self, seq_ids):
         seq_ids = [int(s) for s in seq_ids]
         if (len(set(seq_ids)) != len(seq_ids) or any(s not in self.tables for s in seq_ids)
                 or any(s in self.swapped for s in seq_ids)):
@@ -232,6 +274,7 @@ class BlockManagerModel:
             for b in table:
                 self.decref(b)
         del self.lens[seq_id]
+        self.hist.pop(seq_id, None)
 
     def export_tables(self, seq_ids, max_blocks: int):
         tables = []
@@ -364,4 +407,5 @@ class BlockManagerModel:
                 self.block_hash[b] = hashes[i]
         self.tables[seq_id] = table
         self.lens[seq_id] = n
+        self.hist[seq_id] = (hashes[-1] if hashes else 0, tokens[len(hashes) * bs:])
         return len(hits) * bs

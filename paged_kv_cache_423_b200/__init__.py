@@ -105,6 +105,7 @@ _SIGNATURES = {
     "pkv_bm_add_seq": (c_int, [c_void_p, c_int64, c_int, c_void_p, c_int]),
     "pkv_bm_fork": (c_int, [c_void_p, c_int64, c_int64]),
     "pkv_bm_append_slots": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, ctypes.POINTER(c_int)]),
+    "pkv_bm_append_tokens": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p, ctypes.POINTER(c_int)]),
     "pkv_bm_slots": (c_int, [c_void_p, c_int64, c_int, c_int, c_void_p]),
     "pkv_bm_free_seq": (c_int, [c_void_p, c_int64]),
     "pkv_bm_seq_len": (c_int, [c_void_p, c_int64]),
@@ -481,6 +482,20 @@ class BlockManager:
         n_cow = c_int(0)
         _check(library().pkv_bm_append_slots(self._h, _np_ptr(ids), len(ids), _np_ptr(slots), _np_ptr(pairs),
                                              ctypes.byref(n_cow)), "bm_append_slots")
+        return slots, pairs[:n_cow.value].copy()
+
+    def append_tokens(self, seq_ids, tokens):
+        """append_slots with the token id of each new position; a sequence created from
+        token ids registers every block these tokens complete in the prefix cache."""
+        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        toks = np.ascontiguousarray(list(tokens), dtype=np.int32)
+        if len(toks) != len(ids):
+            raise ValueError("append_tokens: one token per sequence")
+        slots = np.zeros(len(ids), np.int64)
+        pairs = np.zeros((max(len(ids), 1), 2), np.int64)
+        n_cow = c_int(0)
+        _check(library().pkv_bm_append_tokens(self._h, _np_ptr(ids), _np_ptr(toks), len(ids), _np_ptr(slots),
+                                              _np_ptr(pairs), ctypes.byref(n_cow)), "bm_append_tokens")
         return slots, pairs[:n_cow.value].copy()
 
     def slots(self, seq_id: int, start: int, count: int) -> np.ndarray:

@@ -91,6 +91,11 @@ struct pkv_bm {
     std::vector<int32_t> table;  // device blocks, or host blocks while swapped out
     int len = 0;
     bool swapped = false;
+    // Token history for the prefix cache: known for sequences created from token
+    // ids and kept by append_tokens; lost (false) after a plain append_slots.
+    bool tracked = false;
+    uint64_t parent = 0;           // chain hash of the last full block
+    std::vector<int32_t> partial;  // token ids of the block being filled
   };
   int num_blocks = 0;
   int block_size = 0;
@@ -245,8 +250,11 @@ extern "C" int pkv_bm_fork(pkv_bm* bm, int64_t parent, int64_t child) {
   return PKV_OK;
 }
 
-extern "C" int pkv_bm_append_slots(pkv_bm* bm, const int64_t* seq_ids, int n, int64_t* slots_out,
-                                   int64_t* cow_pairs_out, int* n_cow_out) {
+// One new position per listed sequence (all-or-nothing), then, with token ids, the
+// prefix-cache bookkeeping of each tracked sequence; without them the sequences'
+// token history is lost.
+static int append_impl(pkv_bm* bm, const int64_t* seq_ids, const int32_t* tokens, int n, int64_t* slots_out,
+                       int64_t* cow_pairs_out, int* n_cow_out) {
   if (!bm || n < 0 || (n > 0 && (!seq_ids || !slots_out || !cow_pairs_out)) || !n_cow_out)
     return set_error(PKV_ERR_INVALID, "pkv_bm_append_slots: bad arguments");
   *n_cow_out = 0;
@@ -301,7 +309,38 @@ extern "C" int pkv_bm_append_slots(pkv_bm* bm, const int64_t* seq_ids, int n, in
     ++s.len;
   }
   *n_cow_out = n_cow;
+  for (int i = 0; i < n; ++i) {
+    pkv_bm::Seq& s = *seqs[i];
+    if (!tokens) {
+      s.tracked = false;
+      s.partial.clear();
+      continue;
+    }
+    if (!s.tracked) continue;
+    s.partial.push_back(tokens[i]);
+    if (static_cast<int>(s.partial.size()) < bm->block_size) continue;
+    // the token completed its block: register it under the chain hash, as a prompt block is
+    s.parent = block_hash(s.parent, s.partial.data(), bm->block_size);
+    s.partial.clear();
+    const int32_t b = s.table.back();
+    if (!bm->registered[b] && !bm->cached.count(s.parent)) {
+      bm->cached.emplace(s.parent, b);
+      bm->block_hash_of[b] = s.parent;
+      bm->registered[b] = 1;
+    }
+  }
   return PKV_OK;
+}
+
+extern "C" int pkv_bm_append_slots(pkv_bm* bm, const int64_t* seq_ids, int n, int64_t* slots_out,
+                                   int64_t* cow_pairs_out, int* n_cow_out) {
+  return append_impl(bm, seq_ids, nullptr, n, slots_out, cow_pairs_out, n_cow_out);
+}
+
+extern "C" int pkv_bm_append_tokens(pkv_bm* bm, const int64_t* seq_ids, const int32_t* tokens, int n,
+                                    int64_t* slots_out, int64_t* cow_pairs_out, int* n_cow_out) {
+  if (n > 0 && !tokens) return set_error(PKV_ERR_INVALID, "pkv_bm_append_tokens: null tokens");
+  return append_impl(bm, seq_ids, n > 0 ? tokens : nullptr, n, slots_out, cow_pairs_out, n_cow_out);
 }
 
 extern "C" int pkv_bm_slots(const pkv_bm* bm, int64_t seq_id, int start, int count, int64_t* slots_out) {
@@ -519,6 +558,9 @@ extern "C" int pkv_bm_add_seq_tokens(pkv_bm* bm, int64_t seq_id, const int32_t* 
     }
   }
   seq.len = num_tokens;
+  seq.tracked = true;
+  seq.parent = nfull > 0 ? hashes[nfull - 1] : 0;
+  seq.partial.assign(tokens + static_cast<size_t>(nfull) * bs, tokens + num_tokens);
   bm->seqs.emplace(seq_id, std::move(seq));
   *cached_tokens_out = static_cast<int>(hits.size()) * bs;
   return PKV_OK;

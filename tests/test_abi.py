@@ -182,13 +182,41 @@ def test_block_manager_matches_model(pkv, seed, extended):
     cpp = pkv.BlockManager(nb, bs, order, num_host_blocks=hb)
     model = BlockManagerModel(nb, bs, order, num_host_blocks=hb)
     prompts = [list(rng.integers(0, 4, size=30)) for _ in range(3)]
+    texts = {}  # seq -> token ids when known (prompt-token sequences and their decode appends)
     next_id = 0
     for _ in range(300):
         every = sorted(model.tables)
         live = [x for x in every if not model.is_swapped(x)]
         gone = [x for x in every if model.is_swapped(x)]
-        op = int(rng.integers(0, 9 if extended else 6))
-        if op >= 6:
+        op = int(rng.integers(0, 11 if extended else 6))
+        if op == 9 and live:
+            # decode appends with token ids: blocks they complete register in the prefix cache
+            pick = [int(x) for x in rng.permutation(live)[:int(rng.integers(1, len(live) + 1))]]
+            toks = [int(t) for t in rng.integers(0, 4, size=len(pick))]
+            (sm, pm), (sc, pc) = [r if r is not None else (None, None) for r in run_both(
+                lambda m: m.append_tokens(pick, toks), cpp, model, pkv)]
+            if sm is not None:
+                assert list(sc) == sm and [tuple(p) for p in pc.tolist()] == pm
+                for s_, t_ in zip(pick, toks):
+                    if texts.get(s_) is not None:
+                        texts[s_] = texts[s_] + [t_]
+            same_state(cpp, model)
+            continue
+        if op == 10:
+            # a prompt continuing a generated text
+            known = [x for x in live if texts.get(x) is not None]
+            if known:
+                src = known[int(rng.integers(len(known)))]
+                toks = texts[src] + [int(t) for t in rng.integers(0, 4, size=int(rng.integers(1, 3)))]
+                sid = next_id
+                next_id += 1
+                rm, rc = run_both(lambda m: m.add_seq_tokens(sid, toks), cpp, model, pkv)
+                assert rm == rc
+                if rm is not None:
+                    texts[sid] = toks
+            same_state(cpp, model)
+            continue
+        if op >= 6 and op <= 8:
             # swap out / swap in (sometimes of a sequence in the wrong pool) / prompt admission
             if op == 6 and every:
                 pick = [int(x) for x in rng.permutation(every)[:int(rng.integers(1, min(3, len(every)) + 1))]]
@@ -208,6 +236,8 @@ def test_block_manager_matches_model(pkv, seed, extended):
                 next_id += 1
                 rm, rc = run_both(lambda m: m.add_seq_tokens(sid, toks), cpp, model, pkv)
                 assert rm == rc
+                if rm is not None:
+                    texts[sid] = [int(t) for t in toks]
             same_state(cpp, model)
             continue
         if not live:
@@ -226,12 +256,15 @@ def test_block_manager_matches_model(pkv, seed, extended):
             child = next_id
             next_id += 1
             run_both(lambda m: m.fork(parent, child), cpp, model, pkv)
+            texts[child] = None if texts.get(parent) is None else list(texts[parent])
         elif op == 2:
             pick = [int(s) for s in rng.permutation(live)[:int(rng.integers(1, len(live) + 1))]]
             (sm, pm), (sc, pc) = [r if r is not None else (None, None) for r in run_both(
                 lambda m: m.append_slots(pick), cpp, model, pkv)]
             if sm is not None:
                 assert list(sc) == sm and [tuple(p) for p in pc.tolist()] == pm
+                for s_ in pick:
+                    texts[s_] = None
         elif op == 3:
             victim = every[int(rng.integers(len(every)))]
             run_both(lambda m: m.free_seq(victim), cpp, model, pkv)
@@ -294,3 +327,12 @@ def test_block_manager_swap_and_prefix_examples(pkv):
     assert pc.add_seq_tokens(1, p + [98]) == 12
     tables, _ = pc.export_tables([1], 4)
     assert tables.tolist() == [[0, 1, 2, 4]] and pc.free_list() == [5, 6, 7, 3]
+
+
+def test_block_manager_decode_registration_example(pkv):
+    """The hand-worked decode-registration case gives the same results in C++."""
+    from tests.test_oracle_block_manager import decode_registration_example
+    model = BlockManagerModel(8, 4, list(range(8)))
+    cpp = pkv.BlockManager(8, 4, list(range(8)))
+    assert decode_registration_example(cpp) == decode_registration_example(model)
+    same_state(cpp, model)

@@ -158,19 +158,57 @@ def test_invalid_operations():
         assert e.value.code == ERR_INVALID
 
 
+def check_histories(m: BlockManagerModel, texts):
+    """A sequence with a known token text holds the chain hash of its full blocks and the
+    ids of its partial block; one without holds none."""
+    bs = m.block_size
+    for s in m.tables:
+        txt = texts.get(s)
+        if txt is None:
+            assert m.hist[s] is None
+            continue
+        assert len(txt) == m.lens[s]
+        nf = len(txt) // bs
+        parent = 0
+        for i in range(nf):
+            parent = block_hash(parent, txt[i * bs:(i + 1) * bs])
+        assert m.hist[s] == (parent, txt[nf * bs:])
+
+
 def random_ops(seed, steps=400, num_blocks=48, block_size=4, extended=False):
     """A seeded random mix of every operation; checks invariants after each one.
-    ``extended`` adds swap-out / swap-in and prompt-token (prefix-cached) admission."""
+    ``extended`` adds swap-out / swap-in, prompt-token (prefix-cached) admission,
+    decode appends with token ids, and prompts that continue a generated text."""
     rng = wl.rng_for(seed)
     m = BlockManagerModel(num_blocks, block_size, rng.permutation(num_blocks),
                           num_host_blocks=num_blocks // 2 if extended else 0)
     prompts = [list(rng.integers(0, 5, size=40)) for _ in range(3)]   # few distinct prompts: many hits
+    texts = {}  # seq -> its token ids, or None when unknown
     next_id = 0
     for _ in range(steps):
-        op = rng.integers(0, 8 if extended else 5)
+        op = rng.integers(0, 10 if extended else 5)
         live = sorted(s for s in m.tables if s not in m.swapped)
         gone = sorted(m.swapped)
         try:
+            if op == 8:
+                if live:
+                    pick = [int(x) for x in rng.permutation(live)[:rng.integers(1, len(live) + 1)]]
+                    toks = [int(t) for t in rng.integers(0, 5, size=len(pick))]
+                    m.append_tokens(pick, toks)
+                    for s_, t_ in zip(pick, toks):
+                        if texts.get(s_) is not None:
+                            texts[s_] = texts[s_] + [t_]
+                continue
+            if op == 9:
+                known = [x for x in live if texts.get(x) is not None]
+                if known:
+                    src = known[rng.integers(len(known))]
+                    prompt = texts[src] + [int(t) for t in rng.integers(0, 5, size=int(rng.integers(1, 4)))]
+                    got = m.add_seq_tokens(next_id, prompt)
+                    assert got % block_size == 0 and got <= (len(prompt) - 1) // block_size * block_size
+                    texts[next_id] = prompt
+                    next_id += 1
+                continue
             if op == 5:
                 if live:
                     m.swap_out([int(x) for x in rng.permutation(live)[:rng.integers(1, min(3, len(live)) + 1)]])
@@ -184,6 +222,7 @@ def random_ops(seed, steps=400, num_blocks=48, block_size=4, extended=False):
                 n = int(rng.integers(1, len(p) + 1))
                 tail = list(rng.integers(0, 5, size=int(rng.integers(0, 3))))
                 m.add_seq_tokens(next_id, p[:n] + tail)
+                texts[next_id] = [int(t) for t in p[:n] + tail]
                 next_id += 1
                 continue
             if op == 0 or not live:
@@ -195,14 +234,20 @@ def random_ops(seed, steps=400, num_blocks=48, block_size=4, extended=False):
                 m.add_seq(next_id, len(shared) * block_size + int(rng.integers(0, 9)), shared)
                 next_id += 1
             elif op == 1:
-                m.fork(live[rng.integers(len(live))], next_id)
+                parent = live[rng.integers(len(live))]
+                m.fork(parent, next_id)
+                texts[next_id] = None if texts.get(parent) is None else list(texts[parent])
                 next_id += 1
             elif op == 2:
-                pick = rng.permutation(live)[:rng.integers(1, len(live) + 1)]
-                m.append_slots([int(s) for s in pick])
+                pick = [int(s) for s in rng.permutation(live)[:rng.integers(1, len(live) + 1)]]
+                m.append_slots(pick)
+                for s_ in pick:
+                    texts[s_] = None
             elif op == 3:
                 every = sorted(m.tables)
-                m.free_seq(every[rng.integers(len(every))])
+                victim = every[rng.integers(len(every))]
+                m.free_seq(victim)
+                texts.pop(victim, None)
             else:
                 s = live[rng.integers(len(live))]
                 if m.lens[s]:
@@ -212,6 +257,7 @@ def random_ops(seed, steps=400, num_blocks=48, block_size=4, extended=False):
             assert e.code == ERR_OOM
         finally:
             check_invariants(m)
+            check_histories(m, texts)
     return m
 
 
@@ -350,3 +396,55 @@ def test_prefix_cache_oom_is_all_or_nothing():
         m.add_seq_tokens(1, list(range(8)) + list(range(50, 60)))   # 2 cached + 3 fresh > 1 free
     assert e.value.code == ERR_OOM
     assert before == (list(m.free), list(m.ref), dict(m.cached)) and 1 not in m.tables
+
+
+def decode_registration_example(m):
+    """Hand-worked: 8 blocks of 4, free list 0..7.  Returns what the checks compare."""
+    out = {}
+
+    def table(seq, width):
+        t, _ = m.export_tables([seq], width)
+        return [int(x) for x in np.asarray(t)[0]]
+    out["admit0"] = m.add_seq_tokens(0, [1, 2, 3, 4, 5, 6])   # block 0 full (registered), block 1 holds 5, 6
+    out["cached0"] = m.num_cached_blocks()
+    m.append_tokens([0], [7])
+    out["cached1"] = m.num_cached_blocks()                      # block 1 not full yet
+    slots, pairs = m.append_tokens([0], [8])                    # completes block 1
+    out["slot8"] = [int(x) for x in slots]
+    out["cached2"] = m.num_cached_blocks()
+    out["admit1"] = m.add_seq_tokens(1, [1, 2, 3, 4, 5, 6, 7, 8, 9])   # continues the generated text
+    out["table1"] = table(1, 3)
+    m.append_slots([0])                                         # history of 0 ends here
+    for t in (10, 11, 12):
+        m.append_tokens([0], [t])                               # fills block 3 of seq 0: not registered
+    out["cached3"] = m.num_cached_blocks()
+    out["table0"] = table(0, 3)
+    m.fork(1, 2)                                                # the child keeps 1's history
+    _, pairs = m.append_tokens([1, 2], [10, 10])                # 1 copies its shared last block (2 -> 4)
+    out["pairs"] = [tuple(int(v) for v in p) for p in pairs]
+    m.append_tokens([1, 2], [11, 11])
+    m.append_tokens([1, 2], [12, 12])                           # equal texts: 1 registers, 2 finds the hash taken
+    out["cached4"] = m.num_cached_blocks()
+    out["table1_after"], out["table2"] = table(1, 3), table(2, 3)
+    return out
+
+
+def test_decode_filled_blocks_register():
+    m = BlockManagerModel(8, 4, list(range(8)))
+    out = decode_registration_example(m)
+    assert out["admit0"] == 0 and out["cached0"] == 1 and out["cached1"] == 1
+    assert out["slot8"] == [1 * 4 + 3] and out["cached2"] == 2
+    h0 = block_hash(0, [1, 2, 3, 4])
+    h1 = block_hash(h0, [5, 6, 7, 8])
+    assert m.cached[h0] == 0 and m.cached[h1] == 1
+    assert out["admit1"] == 8 and out["table1"] == [0, 1, 2]
+    assert out["cached3"] == 2 and out["table0"] == [0, 1, 3]
+    assert out["pairs"] == [(2, 4)] and out["table1_after"] == [0, 1, 4] and out["table2"] == [0, 1, 2]
+    h2 = block_hash(h1, [9, 10, 11, 12])
+    assert out["cached4"] == 3 and m.cached[h2] == 4
+    check_invariants(m)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_decode_registration_under_random_operations(seed):
+    random_ops(300 + seed, extended=True)

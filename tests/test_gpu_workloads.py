@@ -316,3 +316,38 @@ def test_prefix_cached_admission(pkv):
     tables, clens = ls.tables(ids, 20)
     assert all(tables[r][:12].tolist() == tables[0][:12].tolist() for r in ids)
     decode_and_compare(pkv, pool, wl.bf16_normal(rng, (len(ids), Hq, D)), tables, clens, wl.fp32_scale(D), Hq)
+
+
+def test_decode_filled_blocks_serve_a_continuation(pkv):
+    """Blocks a sequence fills while decoding register in the prefix cache
+    (append_tokens), so a later request whose prompt continues the generated text
+    takes them from the cache, writes only its uncached tokens, and attends exactly
+    as the oracle does over the same text."""
+    rng = wl.rng_for(920)
+    Hq, Hkv, D, bs, nb = 32, 8, 128, 16, 64
+    order = rng.permutation(nb).astype(np.int32)
+    ls = Lockstep(pkv, nb, bs, order)
+    pool = Pool(pkv, rng, nb, Hkv, bs, D)
+    prompt = [int(t) for t in rng.integers(0, 32000, size=40)]    # blocks 0, 1 full; 32..39 in block 2
+    gen = [int(t) for t in rng.integers(0, 32000, size=45)]       # positions 40..84: blocks 2, 3, 4 complete
+    text = prompt + gen
+    tk, tv = wl.new_tokens(rng, len(text), Hkv, D)                  # K/V of every position of the text
+    assert ls.cpp.add_seq_tokens(0, prompt) == ls.ref.add_seq_tokens(0, prompt) == 0
+    pool.write(tk[:40], tv[:40], ls.slots(0, 0, 40))
+    for i, tok in enumerate(gen):
+        slots, pairs = ls.cpp.append_tokens([0], [tok])
+        rslots, rpairs = ls.ref.append_tokens([0], [tok])
+        assert slots.tolist() == rslots and len(pairs) == len(rpairs) == 0
+        pool.write(tk[40 + i:41 + i], tv[40 + i:41 + i], slots)
+    assert ls.cpp.num_cached_blocks() == ls.ref.num_cached_blocks() == 5
+    tail = [int(t) for t in rng.integers(0, 32000, size=7)]
+    toks = text + tail                                              # 92 tokens
+    got = ls.cpp.add_seq_tokens(1, toks)
+    assert got == ls.ref.add_seq_tokens(1, toks) == 5 * bs          # every full block of the text
+    nk, nv = wl.new_tokens(rng, len(tail), Hkv, D)
+    pool.write(np.concatenate([tk[got:], nk]), np.concatenate([tv[got:], nv]), ls.slots(1, got, len(toks) - got))
+    pool.check()
+    tables, clens = ls.tables([0, 1], 6)
+    assert tables[1][:5].tolist() == tables[0][:5].tolist() and tables[1][5] != tables[0][5]
+    assert clens.tolist() == [len(text), len(toks)]
+    decode_and_compare(pkv, pool, wl.bf16_normal(rng, (2, Hq, D)), tables, clens, wl.fp32_scale(D), Hq)

@@ -788,10 +788,10 @@ def oracle_sample_fp8(w, step_inputs, n_seqs, rng):
     return items
 
 
-def cpu_baseline_fp8(w, step_inputs, budget_s=10.0):
+def time_oracle_fp8(w, items, budget_s):
+    """The 8-bit decode oracle on sampled sequences, 1 thread; KV bytes at 1 B/value."""
     from threadpoolctl import threadpool_limits
     from oracle import fp8
-    items = oracle_sample_fp8(w, step_inputs, 64, wl.rng_for(77))
     done = n = 0
     t0 = time.perf_counter()
     with threadpool_limits(limits=1):
@@ -801,7 +801,12 @@ def cpu_baseline_fp8(w, step_inputs, budget_s=10.0):
             n += 1
             if time.perf_counter() - t0 > budget_s:
                 break
-    dt = time.perf_counter() - t0
+    return done, time.perf_counter() - t0, n
+
+
+def cpu_baseline_fp8(w, step_inputs, budget_s=10.0):
+    items = oracle_sample_fp8(w, step_inputs, 64, wl.rng_for(77))
+    done, dt, n = time_oracle_fp8(w, items, budget_s)
     return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{n} sequences of the {w.name} batch over the 8-bit pool (all {w.Hq} heads each), "
                       f"float64 NumPy, 1 thread, {dt:.1f} s"}
@@ -1112,7 +1117,8 @@ def run_reference(args, rank, world, local_rank):
         return run_reference_prefill(args, world, device)
     if args.workload == SWAP_WORKLOAD:
         return run_reference_swap(args, world)
-    w = Workload(args.workload, 2, seed=1000, device=device)
+    kv8 = args.kv == "fp8"
+    w = Workload(args.workload, 2, seed=1000, device=device, kv8=kv8)
     bm = w.new_manager()
     ids = list(range(w.B))
     bm.append_slots(ids)
@@ -1120,27 +1126,28 @@ def run_reference(args, rank, world, local_rank):
     q, _, _ = w.host_step_inputs()
     st = {"tables": torch.from_numpy(tables), "host_lens": lens, "q": to_dev(q, device)}
     rng = wl.rng_for(78)
+    sample_fn, timer = (oracle_sample_fp8, time_oracle_fp8) if kv8 else (oracle_sample, time_oracle)
     # size each step's sample so the whole run stays near --ref-budget seconds
-    probe = oracle_sample(w, st, 2, rng)
-    _, dt_probe, n_probe = time_oracle(w, probe, 1e9)
+    probe = sample_fn(w, st, 2, rng)
+    _, dt_probe, n_probe = timer(w, probe, 1e9)
     per_seq = dt_probe / max(n_probe, 1)
     per_step = int(max(1, min(64, args.ref_budget / max(per_seq, 1e-6) / (args.warmup + args.steps))))
     for _ in range(args.warmup):
-        time_oracle(w, oracle_sample(w, st, per_step, rng), 1e9)
+        timer(w, sample_fn(w, st, per_step, rng), 1e9)
     kv = 0
     dt_total = 0.0
     for _ in range(args.steps):
-        b, dt, _n = time_oracle(w, oracle_sample(w, st, per_step, rng), 1e9)
+        b, dt, _n = timer(w, sample_fn(w, st, per_step, rng), 1e9)
         kv += b
         dt_total += dt
     value = kv / dt_total / 1e9
-    sample = (f"{per_step} random sequences of the {w.name} batch per step (all {w.Hq} heads), float64 NumPy oracle, "
-              f"1 thread")
+    sample = (f"{per_step} random sequences of the {w.name} batch per step (all {w.Hq} heads"
+              f"{', 8-bit pool' if kv8 else ''}), float64 NumPy oracle, 1 thread")
     return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * dt_total / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "num_seqs": w.B, "num_heads": w.Hq, "num_kv_heads": w.Hkv,
-                       "head_dim": w.D, "block_size": w.bs},
+            "config": {"workload": w.name + ("+fp8" if kv8 else ""), "kv_dtype": args.kv, "num_seqs": w.B,
+                       "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D, "block_size": w.bs},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -96,3 +96,20 @@ def test_all_cores_oracle_counts_every_sequence():
     done, dt, cores = bench.time_oracle_all_cores(w, items)
     assert done == cores * int(b.context_lens.sum()) * b.num_kv_heads * b.head_dim * 4  # `cores` passes
     assert cores >= 1 and dt > 0
+
+
+def test_fp8_oracle_timer_counts_one_byte_per_value():
+    """The 8-bit oracle timer (CPU-baseline leg and reference arm) counts K and V at 1 B each."""
+    import types
+    import workloads as wl
+    b = wl.make_decode_batch("llama7b", num_seqs=3, num_heads=4, num_kv_heads=2, length_scale=0.02, with_data=False)
+    rng = wl.rng_for(3)
+    shape = (b.num_blocks, b.num_kv_heads, b.block_size, b.head_dim)
+    kc, vc = wl.e4m3_codes(rng, shape), wl.e4m3_codes(rng, shape)
+    ks, vs = wl.kv_scales(rng, b.num_kv_heads), wl.kv_scales(rng, b.num_kv_heads)
+    q = wl.bf16_normal(rng, (b.num_seqs, b.num_heads, b.head_dim))
+    w = types.SimpleNamespace(Hkv=b.num_kv_heads, D=b.head_dim, scale=b.scale)
+    items = [(q[s:s + 1], kc, vc, ks, vs, b.block_tables[s:s + 1], b.context_lens[s:s + 1]) for s in range(b.num_seqs)]
+    done, dt, n = bench.time_oracle_fp8(w, items, 60.0)
+    assert n == b.num_seqs and dt > 0
+    assert done == int(b.context_lens.sum()) * b.num_kv_heads * b.head_dim * 2

@@ -336,3 +336,34 @@ def test_block_manager_decode_registration_example(pkv):
     cpp = pkv.BlockManager(8, 4, list(range(8)))
     assert decode_registration_example(cpp) == decode_registration_example(model)
     same_state(cpp, model)
+
+
+def test_fp8_argument_errors_before_any_device_work(pkv):
+    """The 8-bit entry points check shapes, paths and pointers on the host."""
+    lib = pkv.library()
+    fake = ctypes.c_void_p(0x1000)
+    args = dict(out=fake, out_dtype=0, query=fake, kc=fake, vc=fake, ks=fake, vs=fake, tables=fake, max_blocks=4,
+                lens=fake, max_ctx=64, B=2, Hq=8, Hkv=2, D=128, bs=16, NB=8, scale=0.1, part=0, path=0, ws=fake,
+                ws_bytes=1 << 20)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.pkv_paged_attention_decode_fp8(a["out"], a["out_dtype"], a["query"], a["kc"], a["vc"], a["ks"],
+                                                  a["vs"], a["tables"], a["max_blocks"], a["lens"], a["max_ctx"],
+                                                  a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"], a["scale"],
+                                                  a["part"], a["path"], a["ws"], a["ws_bytes"], None, None)
+
+    assert call(ks=None) == pkv.PKV_ERR_INVALID                  # the 8-bit pool needs its scales
+    assert call(vs=None) == pkv.PKV_ERR_INVALID
+    assert call(D=64) == pkv.PKV_ERR_UNSUPPORTED                 # head_dim 128 only
+    assert call(Hq=2, path=pkv.PATH_TENSOR) == pkv.PKV_ERR_UNSUPPORTED   # tensor cores need grouped heads
+    assert call(Hq=64, Hkv=2, path=pkv.PATH_TENSOR) == pkv.PKV_ERR_UNSUPPORTED  # group 32 > 16
+    assert call(path=7) == pkv.PKV_ERR_INVALID
+    assert call(ws_bytes=16) == pkv.PKV_ERR_INVALID
+    assert call(B=0) == pkv.PKV_OK
+    q = (fake, fake, fake, fake, fake, fake, fake)
+    assert lib.pkv_reshape_and_cache_fp8(*q, 4, 8, 2, 96, 16, None, None) == pkv.PKV_ERR_UNSUPPORTED
+    assert lib.pkv_reshape_and_cache_fp8(*q, 4, 8, 2, 128, 8, None, None) == pkv.PKV_ERR_UNSUPPORTED
+    assert lib.pkv_reshape_and_cache_fp8(*q, 0, 8, 2, 128, 16, None, None) == pkv.PKV_OK
+    assert lib.pkv_reshape_and_cache_fp8(fake, fake, fake, fake, fake, None, fake, 4, 8, 2, 128, 16, None,
+                                         None) == pkv.PKV_ERR_INVALID

@@ -3,7 +3,7 @@
 ``python -m paged_kv_cache_423_b200.build`` (or ``build_library()``) compiles every
 source under ``csrc/`` into ``_build/*.o`` in parallel and links
 ``paged_kv_cache_423_b200/libpkv.so``.  The CUDA runtime is linked statically, so the
-library loads on machines without a GPU (the driver is only needed once a call
+library loads on machines without a GPU (the NVIDIA driver is only needed once a call
 touches the device).  ptxas register/shared-memory reports go to
 ``_build/ptxas.log``.  Rebuilds only when a source or header is newer than the
 library.

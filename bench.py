@@ -739,7 +739,10 @@ def time_oracle_all_cores(w, items):
     import shutil
     import tempfile
     cores = len(os.sched_getaffinity(0))
-    folder = tempfile.mkdtemp(prefix="pkv_oracle_", dir="/dev/shm" if os.path.isdir("/dev/shm") else None)
+    need = sum(sum(np.asarray(x).nbytes for x in item) for item in items)
+    shm = "/dev/shm"
+    use_shm = os.path.isdir(shm) and shutil.disk_usage(shm).free > 2 * need + (64 << 20)
+    folder = tempfile.mkdtemp(prefix="pkv_oracle_", dir=shm if use_shm else None)
     try:
         for i, (q, kc, vc, table, lens) in enumerate(items):
             for k, arr in (("q", q), ("kc", kc), ("vc", vc), ("table", table), ("lens", lens)):

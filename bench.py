@@ -624,6 +624,32 @@ def run_trace(args, rank, world, local_rank):
     seq_steps = 0
     kv_bytes = 0
     launches = 0
+    # CPU-baseline leg: the oracle on one sampled sequence of every 20th timed step, outside
+    # the timed decode work; its output also checks the GPU's bf16 output for that sequence.
+    oracle_leg = rank == 0 and not args.no_cpu_baseline
+    ora = {"bytes": 0, "s": 0.0, "n": 0, "max_abs": 0.0, "error": None}
+    ora_rng = wl.rng_for(2003)
+
+    def oracle_sample_step(ids, tables, lens, q, out):
+        from threadpoolctl import threadpool_limits
+        from oracle import paged_attention
+        i = int(ora_rng.integers(len(ids)))
+        L = int(lens[i])
+        need = -(-L // p.block_size)
+        blocks = torch.from_numpy(tables[i][:need].astype(np.int64)).to(device)
+        kh = kc[blocks].view(torch.int16).cpu().numpy().view(np.uint16)
+        vh = vc[blocks].view(torch.int16).cpu().numpy().view(np.uint16)
+        qh = q[i:i + 1].view(torch.int16).cpu().numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        with threadpool_limits(limits=1):
+            ref = paged_attention.paged_decode(qh, kh, vh, np.arange(need, dtype=np.int32)[None, :],
+                                               np.array([L], np.int32), scale)
+        ora["s"] += time.perf_counter() - t0
+        ora["bytes"] += L * p.num_kv_heads * p.head_dim * 4
+        ora["n"] += 1
+        got = out[i:i + 1].float().cpu().numpy()
+        ora["max_abs"] = max(ora["max_abs"], float(np.abs(got - ref).max()))
+
     with ClockSampler(device) as clocks:
         for step in range(p.steps):
             ids = sorted(running)
@@ -649,6 +675,11 @@ def run_trace(args, rank, world, local_rank):
                     seq_steps += len(ids)
                     kv_bytes += int(lens.astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 4
                     launches += 3 + (1 if len(pairs) else 0) + 1  # + the split merge
+                    if oracle_leg and ora["error"] is None and (step - args.warmup) % 20 == 0:
+                        try:
+                            oracle_sample_step(ids, tables, lens, q, out)
+                        except Exception as e:  # the trace figure stands without its baseline
+                            ora["error"] = f"{type(e).__name__}: {e}"
                 for sid in ids:
                     running[sid] -= 1
                     if running[sid] == 0:
@@ -671,7 +702,14 @@ def run_trace(args, rank, world, local_rank):
                        "num_blocks": p.num_blocks, "admitted": next_id,
                        "timed": "copy_blocks + reshape_and_cache + paged_attention_decode per step"},
             "seq_steps_per_s": round(seq_steps / (t_ms * 1e-3), 1), "pct_hbm_peak": round(100 * value / peak, 2),
-            "gpu_launches": launches, "clocks": clocks.summary()}
+            "gpu_launches": launches, "clocks": clocks.summary(),
+            **({"cpu_baseline": ({"unavailable": ora["error"]} if ora["error"] or not ora["n"] else
+                                 {"value": round(ora["bytes"] / ora["s"] / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                  "kind": "oracle",
+                                  "sample": f"one sequence of every 20th timed step ({ora['n']} sequences, all "
+                                            f"{p.num_heads} heads), float64 NumPy, 1 thread, {ora['s']:.1f} s",
+                                  "max_abs_vs_gpu_bf16_out": round(ora["max_abs"], 5)})}
+               if oracle_leg else {})}
 
 
 # ---------------------------------------------------------------------------

@@ -244,6 +244,24 @@ def decode_bytes(lens, Hq, Hkv, D, bs, kv_elem_bytes=2):
     return kv, kv + 2 * len(lens) * Hq * D * 2 + blocks * 4 + len(lens) * 4
 
 
+def unique_kv_bytes(tables, lens, Hkv, D, bs, kv_elem_bytes=2):
+    """KV bytes of one decode call with every physical block counted once: for each
+    distinct block, the rows any sequence reads from it (a shared prefix block is read
+    through many tables but holds its bytes once)."""
+    tables = np.asarray(tables)
+    lens = np.asarray(lens, np.int64)
+    rows = np.zeros(int(tables.max()) + 1 if tables.size else 1, np.int64)
+    for s, L in enumerate(lens):
+        need = -(-int(L) // bs)
+        if need == 0:
+            continue
+        r = np.full(need, bs, np.int64)
+        if L % bs:
+            r[-1] = L % bs
+        np.maximum.at(rows, tables[s][:need].astype(np.int64), r)
+    return int(rows.sum()) * Hkv * D * 2 * kv_elem_bytes
+
+
 def e4m3_pool(shape, gen, device):
     """Seeded e4m3 codes drawn as bit patterns on the device (sign, exponent around 8,
     uniform mantissa, never NaN), like workloads.e4m3_codes."""
@@ -365,7 +383,8 @@ def run_ours(args, rank, world, local_rank):
         states.append(dict(q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
                            slots=torch.from_numpy(slots).to(device), pairs=torch.from_numpy(pairs).to(device),
                            n_pairs=len(pairs), tables=torch.from_numpy(tables).to(device),
-                           lens=torch.from_numpy(lens).to(device), max_len=int(lens.max()), host_lens=lens))
+                           lens=torch.from_numpy(lens).to(device), max_len=int(lens.max()), host_lens=lens,
+                           unique_kv=unique_kv_bytes(tables, lens, w.Hkv, w.D, w.bs, 1 if kv8 else 2)))
     bm.close()
     max_len_all = int(w.lens0.max()) + max(n_states, args.e2e_steps + args.warmup) + 1
     ws = torch.empty(pkv.paged_attention_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.bs, max_len_all),
@@ -390,7 +409,7 @@ def run_ours(args, rank, world, local_rank):
         step(i)
     torch.cuda.synchronize()
     launches = 0
-    kv_total = bytes_total = 0
+    kv_total = bytes_total = unique_total = 0
     g = w.Hq // w.Hkv
     uses_tensor = path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16)
     # write, plan, decode (+ copy_blocks when a fork copied blocks) (+ the merge of a split context)
@@ -400,6 +419,7 @@ def run_ours(args, rank, world, local_rank):
         kv, alg = decode_bytes(st["host_lens"], w.Hq, w.Hkv, w.D, w.bs, 1 if kv8 else 2)
         kv_total += kv
         bytes_total += alg
+        unique_total += alg - kv + st["unique_kv"]
         launches += 3 + (1 if st["n_pairs"] else 0) + merge
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
@@ -427,7 +447,9 @@ def run_ours(args, rank, world, local_rank):
     e2e = run_e2e(args, w, pkv, device, path, ws, out, status, max_len_all) if not args.no_e2e else None
 
     peak, peak_kind = measured_hbm_gbs()
-    dec_gbs = bytes_total / (dec_ms * 1e-3) / 1e9
+    # the roofline counts every physical block once (a shared prefix is one copy of bytes);
+    # the same as the logical count when no blocks are shared
+    dec_gbs = unique_total / (dec_ms * 1e-3) / 1e9
     read_gbs = stream_read_gbs(pkv, device)
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -445,7 +467,8 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": recorded_traffic(w.name + ("+fp8" if kv8 else ""),
                                                  ("decode_gqa_tc_fp8" if kv8 else "decode_gqa_tc") if uses_tensor
                                                  else "decode_simt"),
-                     "algorithmic_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": unique_total // args.steps,
+                     "logical_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
                      "kernel": ("paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"
                                 " + split merge" if kv8 and uses_tensor
                                 else "paged_attention_decode_fp8: plan + CUDA-core streaming kernel (e4m3 tiles)" if kv8

@@ -113,3 +113,43 @@ def test_fp8_oracle_timer_counts_one_byte_per_value():
     done, dt, n = bench.time_oracle_fp8(w, items, 60.0)
     assert n == b.num_seqs and dt > 0
     assert done == int(b.context_lens.sum()) * b.num_kv_heads * b.head_dim * 2
+
+
+def _distinct_slots(tables, lens, bs):
+    return len({int(tables[s][t // bs]) * bs + t % bs for s, L in enumerate(lens) for t in range(L)})
+
+
+def test_unique_kv_bytes_counts_each_physical_slot_once():
+    per_slot = 2 * 128 * 2 * 2  # Hkv=2, D=128, K and V, bf16
+    # two sequences share block 7 (a full prefix block), then go their own ways; the
+    # shorter one also reads a partial block; block 0 (padding) is past every length
+    tables = np.array([[7, 3, 0], [7, 5, 9]], np.int32)
+    lens = [20, 37]
+    u = bench.unique_kv_bytes(tables, lens, Hkv=2, D=128, bs=16)
+    assert u == _distinct_slots(tables, lens, 16) * per_slot == (16 + 4 + 16 + 5) * per_slot
+    kv, _ = bench.decode_bytes(lens, Hq=8, Hkv=2, D=128, bs=16)
+    assert kv - u == 16 * per_slot  # the shared block is the only difference
+    # nothing shared: the same as the logical count; e4m3 halves it
+    tables = np.array([[1, 2], [3, 4], [5, 0]], np.int32)
+    lens = [32, 17, 0]
+    assert bench.unique_kv_bytes(tables, lens, 2, 128, 16) == bench.decode_bytes(lens, 8, 2, 128, 16)[0]
+    assert bench.unique_kv_bytes(tables, lens, 2, 128, 16, 1) * 2 == bench.decode_bytes(lens, 8, 2, 128, 16)[0]
+
+
+def test_unique_kv_bytes_on_random_forked_tables():
+    rng = np.random.default_rng(5)
+    bs = 8
+    for _ in range(20):
+        n_shared = int(rng.integers(0, 4))
+        B = int(rng.integers(1, 6))
+        shared = rng.permutation(np.arange(1, 200))[:n_shared]
+        own = iter(rng.permutation(np.arange(200, 400)))
+        tables = np.zeros((B, 10), np.int32)
+        lens = []
+        for s in range(B):
+            L = int(rng.integers(0, 10 * bs + 1))
+            tables[s, :n_shared] = shared
+            for b in range(n_shared, 10):
+                tables[s, b] = next(own)
+            lens.append(L)
+        assert bench.unique_kv_bytes(tables, lens, 1, 4, bs, 1) == _distinct_slots(tables, lens, bs) * 8

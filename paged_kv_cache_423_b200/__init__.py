@@ -160,6 +160,19 @@ def _ptr(t, dtype=None, name="tensor"):
     return c_void_p(t.data_ptr())
 
 
+def _same_device(what, *tensors):
+    """The library launches on the current device, so every CUDA tensor of one call must
+    live there (pinned host tensors, where a call takes them, are exempt)."""
+    cur = None
+    for t in tensors:
+        if t is None or not getattr(t, "is_cuda", False):
+            continue
+        if cur is None:
+            cur = _torch().cuda.current_device()
+        if t.device.index != cur:
+            raise ValueError(f"{what}: every CUDA tensor must be on the current device cuda:{cur}, got {t.device}")
+
+
 def _stream(stream):
     torch = _torch()
     if stream is None:
@@ -174,6 +187,7 @@ def _stream(stream):
 def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, status=None, stream=None):
     """Write key/value [T, Hkv, D] bf16 into the pools [NB, Hkv, bs, D] at slot_mapping [T] int64."""
     torch = _torch()
+    _same_device("reshape_and_cache", key, value, key_cache, value_cache, slot_mapping, status)
     T, Hkv, D = key.shape
     NB, Hkv2, bs, D2 = key_cache.shape
     if value.shape != key.shape or value_cache.shape != key_cache.shape or (Hkv, D) != (Hkv2, D2):
@@ -203,6 +217,7 @@ def copy_blocks(key_caches, value_caches, block_mapping, status=None, stream=Non
     for kc, vc in zip(key_caches, value_caches):
         if kc.shape != key_caches[0].shape or vc.shape != key_caches[0].shape:
             raise ValueError("copy_blocks: every pool must have the same shape")
+    _same_device("copy_blocks", *key_caches, *value_caches, block_mapping, status)
     ks = (c_void_p * len(key_caches))(*[_ptr(k, torch.bfloat16, "key_cache").value for k in key_caches])
     vs = (c_void_p * len(value_caches))(*[_ptr(v, torch.bfloat16, "value_cache").value for v in value_caches])
     mapping = _ptr(block_mapping, torch.int64, "block_mapping") if n else c_void_p(0)
@@ -234,6 +249,7 @@ def paged_attention_decode(out, query, key_cache, value_cache, block_tables, con
     block_tables [B, max_blocks] int32, context_lens [B] int32 (device), max_context_len
     a host bound, workspace a uint8 device tensor of paged_attention_workspace_size bytes."""
     torch = _torch()
+    _same_device("paged_attention_decode", out, query, key_cache, value_cache, block_tables, context_lens, workspace, status)
     B, Hq, D = query.shape
     NB, Hkv, bs, D2 = key_cache.shape
     if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
@@ -266,6 +282,7 @@ def paged_attention_decode_static(out, query, key_cache, value_cache, block_tabl
     per GPU).  Calls on one device must not overlap on the GPU; the first call on a
     device should come before any stream capture."""
     torch = _torch()
+    _same_device("paged_attention_decode_static", out, query, key_cache, value_cache, block_tables, context_lens, status)
     B, Hq, D = query.shape
     NB, Hkv, bs, D2 = key_cache.shape
     if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
@@ -289,6 +306,7 @@ def reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_sc
     """Quantising write of key/value [T, Hkv, D] bf16 into 8-bit pools [NB, Hkv, bs, D] uint8
     (e4m3 codes) with per-kv-head float32 scales k_scale, v_scale [Hkv]."""
     torch = _torch()
+    _same_device("reshape_and_cache_fp8", key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale, status)
     T, Hkv, D = key.shape
     NB, Hkv2, bs, D2 = key_cache.shape
     if value.shape != key.shape or value_cache.shape != key_cache.shape or (Hkv, D) != (Hkv2, D2):
@@ -311,6 +329,8 @@ def paged_attention_decode_fp8(out, query, key_cache, value_cache, k_scale, v_sc
     otherwise as paged_attention_decode (same workspace size).  path: PATH_AUTO (tensor
     cores for 2 <= group <= 16), PATH_SIMT or PATH_TENSOR."""
     torch = _torch()
+    _same_device("paged_attention_decode_fp8", out, query, key_cache, value_cache, k_scale, v_scale, block_tables,
+                 context_lens, workspace, status)
     B, Hq, D = query.shape
     NB, Hkv, bs, D2 = key_cache.shape
     if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
@@ -348,6 +368,7 @@ def swap_blocks(src_pool, dst_pool, block_mapping, status=None, stream=None):
     dtype): dst_pool[d] = src_pool[s] for every (s, d) of block_mapping [n, 2] int64 (device or
     pinned host).  One kernel launch."""
     torch = _torch()
+    _same_device("swap_blocks", src_pool, dst_pool, block_mapping, status)
     if src_pool.dtype != dst_pool.dtype or src_pool.shape[1:] != dst_pool.shape[1:]:
         raise ValueError("swap_blocks: pools must share dtype and block shape")
     n = int(block_mapping.shape[0]) if block_mapping.numel() else 0
@@ -367,6 +388,7 @@ def stream_read(buf, sink, stream=None):
     """Read the contiguous device tensor `buf` once, XOR-folding its 32-bit words into
     sink (a 1-element int32 device tensor, set by the caller).  A bandwidth reference."""
     torch = _torch()
+    _same_device("stream_read", buf, sink)
     nbytes = buf.numel() * buf.element_size()
     rc = library().pkv_stream_read(_ptr(buf, None, "buf"), nbytes, _ptr(sink, torch.int32, "sink"), _stream(stream))
     _check(rc, "stream_read")
@@ -387,6 +409,8 @@ def paged_attention_prefill(out, query, key_cache, value_cache, block_tables, qu
     query_start [B+1] int32 and context_lens [B] int32 (device), max_context_len a host
     bound, workspace a uint8 device tensor of paged_attention_prefill_workspace_size bytes."""
     torch = _torch()
+    _same_device("paged_attention_prefill", out, query, key_cache, value_cache, block_tables, query_start, context_lens,
+                 workspace, status)
     T, Hq, D = query.shape
     NB, Hkv, bs, D2 = key_cache.shape
     B = int(context_lens.shape[0])

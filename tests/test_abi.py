@@ -367,3 +367,21 @@ def test_fp8_argument_errors_before_any_device_work(pkv):
     assert lib.pkv_reshape_and_cache_fp8(*q, 0, 8, 2, 128, 16, None, None) == pkv.PKV_OK
     assert lib.pkv_reshape_and_cache_fp8(fake, fake, fake, fake, fake, None, fake, 4, 8, 2, 128, 16, None,
                                          None) == pkv.PKV_ERR_INVALID
+
+
+def test_binding_rejects_tensors_off_the_current_device(pkv, monkeypatch):
+    """The binding checks devices before passing pointers: the library launches on the
+    current device, so a tensor on another GPU would be a bad pointer there."""
+    import types
+
+    import torch
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+
+    def fake(index, cuda=True):
+        return types.SimpleNamespace(is_cuda=cuda, device=types.SimpleNamespace(index=index))
+
+    pkv._same_device("op", fake(0), None, fake(0), fake(None, cuda=False))  # host tensors are exempt
+    with pytest.raises(ValueError, match="current device cuda:0"):
+        pkv._same_device("op", fake(0), fake(1))
+    with pytest.raises(ValueError, match="op: every CUDA tensor"):
+        pkv._same_device("op", fake(1))

@@ -102,14 +102,15 @@ def source_digest(kind: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(key: str, kind: str):
-    """DRAM bytes (read + write) per launch of the profiled kernel from profiles/traffic.json, or None."""
+def recorded_traffic(key: str, kind: str, layout=None):
+    """DRAM bytes (read + write) per launch of the profiled kernel from profiles/traffic.json, or
+    None unless the entry was captured on the same kernel sources and the same table layout."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             entry = json.load(f).get(key)
     except Exception:
         return None
-    if not entry or entry.get("sources") != source_digest(kind):
+    if not entry or entry.get("sources") != source_digest(kind) or entry.get("layout") != layout:
         return None
     return int(entry["dram_bytes_per_launch"])
 
@@ -303,6 +304,9 @@ class Workload:
             self.key_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
             self.value_cache = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
         self.rng = wl.rng_for(seed + 1)
+        # the shared-prefix batch: one copy of the prompt's blocks in every table
+        self.shared_blocks = wl.PREFIX_TOKENS // self.bs if name == "prefix_beams" else 0
+        self.layout = f"shared prompt: {self.shared_blocks} blocks in every table" if self.shared_blocks else None
 
     def write(self, k, v, slots, status):
         if self.kv8:
@@ -323,15 +327,26 @@ class Workload:
                                             ws, path=path, status=status)
 
     def new_manager(self):
-        bm = self.pkv.BlockManager(self.NB, self.bs, self.free_order)
-        for s in range(self.B):
-            bm.add_seq(s, int(self.lens0[s]) - 1)
-        return bm
+        return build_manager(self.pkv, self.NB, self.bs, self.free_order, self.lens0 - 1, self.shared_blocks,
+                             self.max_blocks)
 
     def host_step_inputs(self):
         q = wl.bf16_normal(self.rng, (self.B, self.Hq, self.D))
         k, v = wl.new_tokens(self.rng, self.B, self.Hkv, self.D)
         return q, k, v
+
+
+def build_manager(pkv, num_blocks, bs, free_order, lens, shared_blocks, max_blocks):
+    """The batch in the C++ allocator: sequence s holds lens[s] tokens; with
+    shared_blocks = P, sequence 0's first P blocks (one system prompt) are also the
+    first P blocks of every other table (reference count B), the rest private."""
+    bm = pkv.BlockManager(num_blocks, bs, free_order)
+    prefix = ()
+    for s in range(len(lens)):
+        bm.add_seq(s, int(lens[s]), prefix)
+        if s == 0 and shared_blocks:
+            prefix = bm.export_tables([0], max_blocks)[0][0, :shared_blocks].tolist()
+    return bm
 
 
 def aggregate_over_ranks(ms_local, units_local, dist=None, device=None):
@@ -466,7 +481,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(dec_gbs / peak, 4),
                      "traffic": recorded_traffic(w.name + ("+fp8" if kv8 else ""),
                                                  ("decode_gqa_tc_fp8" if kv8 else "decode_gqa_tc") if uses_tensor
-                                                 else "decode_simt"),
+                                                 else "decode_simt", w.layout),
                      "algorithmic_bytes_per_launch": unique_total // args.steps,
                      "logical_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
                      "kernel": ("paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"

@@ -153,3 +153,37 @@ def test_unique_kv_bytes_on_random_forked_tables():
                 tables[s, b] = next(own)
             lens.append(L)
         assert bench.unique_kv_bytes(tables, lens, 1, 4, bs, 1) == _distinct_slots(tables, lens, bs) * 8
+
+
+def test_bench_prefix_batch_shares_the_prompt_blocks(pkv):
+    """The timed shared-prefix batch: every table starts with the same prompt blocks
+    (reference count B), the suffixes are private, and its unique KV bytes are the
+    prompt once plus the suffixes."""
+    import workloads as wl
+    b = wl.make_decode_batch("prefix_beams", with_data=False)
+    bs, B = b.block_size, b.num_seqs
+    shared = wl.PREFIX_TOKENS // bs
+    lens = b.context_lens.astype(np.int64)
+    nb = int(np.ceil(1.2 * np.sum(-(-lens // bs))))
+    order = wl.rng_for(7).permutation(nb).astype(np.int32)
+    mb = int(np.max(-(-lens // bs)))
+    bm = bench.build_manager(pkv, nb, bs, order, lens, shared, mb)
+    tables, got = bm.export_tables(range(B), mb)
+    assert (got == lens).all()
+    assert (tables[:, :shared] == tables[0, :shared]).all()
+    for blk in tables[0, :shared]:
+        assert bm.refcount(int(blk)) == B
+    private = [int(x) for s in range(B) for x in tables[s, shared:-(-int(lens[s]) // bs)]]
+    assert len(set(private)) == len(private) and not set(private) & set(tables[0, :shared].tolist())
+    assert bm.num_free() == nb - shared - len(private)
+    per_token = b.num_kv_heads * b.head_dim * 2 * 2
+    u = bench.unique_kv_bytes(tables, lens, b.num_kv_heads, b.head_dim, bs)
+    assert u == (wl.PREFIX_TOKENS + int((lens - wl.PREFIX_TOKENS).sum())) * per_token
+    assert bench.decode_bytes(lens, b.num_heads, b.num_kv_heads, b.head_dim, bs)[0] - u == \
+        (B - 1) * wl.PREFIX_TOKENS * per_token
+    # every other workload stays unshared
+    bm2 = bench.build_manager(pkv, nb, bs, order, lens[:4], 0, mb)
+    t2, _ = bm2.export_tables(range(4), mb)
+    assert bench.unique_kv_bytes(t2, lens[:4], 8, 128, bs) == bench.decode_bytes(lens[:4], 32, 8, 128, bs)[0]
+    bm.close()
+    bm2.close()

@@ -187,3 +187,17 @@ def test_bench_prefix_batch_shares_the_prompt_blocks(pkv):
     assert bench.unique_kv_bytes(t2, lens[:4], 8, 128, bs) == bench.decode_bytes(lens[:4], 32, 8, 128, bs)[0]
     bm.close()
     bm2.close()
+
+
+def test_l2_flush_only_for_small_working_sets():
+    import workloads as wl
+    per_token = 8 * 128 * 2 * 2
+    b = wl.make_decode_batch("prefix_beams", with_data=False)
+    lens = b.context_lens.astype(np.int64)
+    shared_unique = (wl.PREFIX_TOKENS + int((lens - wl.PREFIX_TOKENS).sum())) * per_token
+    assert bench.needs_l2_flush(shared_unique)            # 0.135 GB: flushed
+    assert bench.needs_l2_flush(shared_unique // 2)       # the e4m3 pool too
+    for name in ("llama7b", "llama13b_mixed_bs16", "long_trace"):
+        c = wl.make_decode_batch(name, with_data=False)
+        kv = bench.decode_bytes(c.context_lens, c.num_heads, c.num_kv_heads, c.head_dim, c.block_size, 1)[0]
+        assert not bench.needs_l2_flush(kv), name         # >= 4x L2 even at one byte per value

@@ -203,7 +203,10 @@ def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, status=N
 
 
 def copy_blocks(key_caches, value_caches, block_mapping, status=None, stream=None):
-    """Copy (src, dst) blocks of block_mapping [n, 2] int64 in every layer's K and V pool."""
+    """Copy (src, dst) blocks of block_mapping [n, 2] int64 in every layer's K and V pool.
+
+    Pools are bf16 or 8-bit (uint8 e4m3 codes), all of one dtype and shape; the copy is
+    bytewise, so an 8-bit pool passes its block bytes as half as many 2-byte elements."""
     torch = _torch()
     if len(key_caches) != len(value_caches):
         raise ValueError("copy_blocks: layer count mismatch")
@@ -212,14 +215,20 @@ def copy_blocks(key_caches, value_caches, block_mapping, status=None, stream=Non
         raise ValueError("copy_blocks: block_mapping must be [n, 2]")
     if not key_caches:
         return
+    dtype = key_caches[0].dtype
+    if dtype not in (torch.bfloat16, torch.uint8):
+        raise TypeError(f"copy_blocks: pools must be bf16 or uint8 (e4m3 codes), got {dtype}")
     NB = key_caches[0].shape[0]
-    block_elems = int(np.prod(key_caches[0].shape[1:]))
+    block_bytes = int(np.prod(key_caches[0].shape[1:])) * key_caches[0].element_size()
+    if block_bytes % 16:
+        raise ValueError("copy_blocks: a block must be a multiple of 16 bytes")
+    block_elems = block_bytes // 2
     for kc, vc in zip(key_caches, value_caches):
         if kc.shape != key_caches[0].shape or vc.shape != key_caches[0].shape:
             raise ValueError("copy_blocks: every pool must have the same shape")
     _same_device("copy_blocks", *key_caches, *value_caches, block_mapping, status)
-    ks = (c_void_p * len(key_caches))(*[_ptr(k, torch.bfloat16, "key_cache").value for k in key_caches])
-    vs = (c_void_p * len(value_caches))(*[_ptr(v, torch.bfloat16, "value_cache").value for v in value_caches])
+    ks = (c_void_p * len(key_caches))(*[_ptr(k, dtype, "key_cache").value for k in key_caches])
+    vs = (c_void_p * len(value_caches))(*[_ptr(v, dtype, "value_cache").value for v in value_caches])
     mapping = _ptr(block_mapping, torch.int64, "block_mapping") if n else c_void_p(0)
     rc = library().pkv_copy_blocks(ks, vs, len(key_caches), mapping, n, NB, block_elems,
                                    _ptr(status, torch.int32, "status"), _stream(stream))

@@ -385,3 +385,14 @@ def test_binding_rejects_tensors_off_the_current_device(pkv, monkeypatch):
         pkv._same_device("op", fake(0), fake(1))
     with pytest.raises(ValueError, match="op: every CUDA tensor"):
         pkv._same_device("op", fake(1))
+
+
+def test_copy_blocks_pool_types_checked_before_device_work(pkv):
+    import torch
+    m = torch.zeros((1, 2), dtype=torch.int64)
+    with pytest.raises(TypeError, match="bf16 or uint8"):
+        pkv.copy_blocks([torch.zeros((4, 1, 16, 64))], [torch.zeros((4, 1, 16, 64))], m)
+    with pytest.raises(ValueError, match="multiple of 16 bytes"):
+        pkv.copy_blocks([torch.zeros((4, 1, 1, 15), dtype=torch.uint8)], [torch.zeros((4, 1, 1, 15), dtype=torch.uint8)], m)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):  # types pass, then the pointer check
+        pkv.copy_blocks([torch.zeros((4, 1, 16, 64), dtype=torch.uint8)], [torch.zeros((4, 1, 16, 64), dtype=torch.uint8)], m)

@@ -64,6 +64,26 @@ def test_copy_blocks_bit_exact(pkv, layers, n):
         assert np.array_equal(host_bits(dks[l]), exp_k[l]) and np.array_equal(host_bits(dvs[l]), exp_v[l])
 
 
+@pytest.mark.parametrize("layers,n", [(1, 5), (2, 17)])
+def test_copy_blocks_8bit_pools_bit_exact(pkv, layers, n):
+    """Copy-on-write over e4m3 pools: the same bytewise copy, every code kept."""
+    rng = wl.rng_for(240 + n)
+    NB, Hkv, bs, D = 48, 8, 16, 128
+    ks = [rng.integers(0, 256, size=(NB, Hkv, bs, D), dtype=np.uint8) for _ in range(layers)]
+    vs = [rng.integers(0, 256, size=(NB, Hkv, bs, D), dtype=np.uint8) for _ in range(layers)]
+    perm = rng.permutation(NB)
+    pairs = np.stack([perm[:n], perm[n:2 * n]], axis=1).astype(np.int64)
+    exp_k, exp_v = cache_ops.copy_blocks(ks, vs, pairs)
+    dks = [torch.from_numpy(a).cuda() for a in ks]
+    dvs = [torch.from_numpy(a).cuda() for a in vs]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.copy_blocks(dks, dvs, torch.from_numpy(pairs).cuda(), status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    for l in range(layers):
+        assert np.array_equal(dks[l].cpu().numpy(), exp_k[l]) and np.array_equal(dvs[l].cpu().numpy(), exp_v[l])
+
+
 def test_copy_blocks_bad_pair(pkv):
     rng = wl.rng_for(230)
     kc = wl.bf16_normal(rng, (4, 1, 16, 64))

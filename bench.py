@@ -29,6 +29,10 @@ Other rows, same JSON line (`--workload` / `--kv`):
                            one step = the chunks' K/V written + paged_attention_prefill;
                            value in TFLOP/s (4 * D per visible (row, key) per head),
                            roofline against the measured bf16 tensor peak.
+  --workload prefix_beams [--beams 4]
+                           128 sequences sharing one 1024-token prompt (the prompt's blocks
+                           in every table); with --beams N each is first forked into N beams,
+                           so the first step copies every shared partial last block but one.
   --workload swap_llama13b one step = 256 13B-shaped blocks swapped out to pinned host
                            memory and 256 swapped in (K and V); GB/s against the
                            pinned-memory copy bandwidth measured in the same run.
@@ -284,15 +288,19 @@ def e4m3_pool(shape, gen, device):
 
 
 class Workload:
-    def __init__(self, name: str, steps: int, seed: int, device, kv8: bool = False):
+    def __init__(self, name: str, steps: int, seed: int, device, kv8: bool = False, beams: int = 1):
         import torch
         import paged_kv_cache_423_b200 as pkv
         self.name = name
         self.kv8 = kv8
+        self.beams = beams
         b = wl.make_decode_batch(name, with_data=False, extra_blocks=0)
-        self.B, self.Hq, self.Hkv, self.D, self.bs = b.num_seqs, b.num_heads, b.num_kv_heads, b.head_dim, b.block_size
+        self.parents = b.num_seqs
+        self.B, self.Hq, self.Hkv, self.D, self.bs = b.num_seqs * beams, b.num_heads, b.num_kv_heads, b.head_dim, b.block_size
+        self.seq_ids = beam_ids(self.parents, beams)  # row order of every step's tensors
         self.scale = b.scale
-        self.lens0 = b.context_lens.copy()            # context lengths after the first appended token
+        self.parent_lens0 = b.context_lens.copy()
+        self.lens0 = np.repeat(b.context_lens, beams)  # per row: context length after the first appended token
         growth = steps + 1
         need_final = int(np.sum(-(-(self.lens0 + growth) // self.bs)))
         self.NB = max(b.num_blocks, int(math.ceil(1.2 * need_final)))
@@ -316,6 +324,9 @@ class Workload:
         # the shared-prefix batch: one copy of the prompt's blocks in every table
         self.shared_blocks = wl.PREFIX_TOKENS // self.bs if name == "prefix_beams" else 0
         self.layout = f"shared prompt: {self.shared_blocks} blocks in every table" if self.shared_blocks else None
+        if beams > 1:
+            self.layout = (self.layout + "; " if self.layout else "") + f"{beams} beams forked from every sequence"
+        self.label = name + (f"+beams{beams}" if beams > 1 else "") + ("+fp8" if kv8 else "")
 
     def write(self, k, v, slots, status):
         if self.kv8:
@@ -336,8 +347,8 @@ class Workload:
                                             ws, path=path, status=status)
 
     def new_manager(self):
-        return build_manager(self.pkv, self.NB, self.bs, self.free_order, self.lens0 - 1, self.shared_blocks,
-                             self.max_blocks)
+        return build_manager(self.pkv, self.NB, self.bs, self.free_order, self.parent_lens0 - 1, self.shared_blocks,
+                             self.max_blocks, self.beams)
 
     def host_step_inputs(self):
         q = wl.bf16_normal(self.rng, (self.B, self.Hq, self.D))
@@ -345,16 +356,33 @@ class Workload:
         return q, k, v
 
 
-def build_manager(pkv, num_blocks, bs, free_order, lens, shared_blocks, max_blocks):
+def beam_ids(parents: int, beams: int) -> list:
+    """Row order of a batch of `parents` sequences with `beams` beams each: every parent
+    id followed by its children (ids parents + (beams - 1) * s + k).  Appends in this
+    order give a shared partial last block a copy for every beam but the last, which
+    writes in place."""
+    ids = []
+    for s in range(parents):
+        ids.append(s)
+        ids.extend(parents + (beams - 1) * s + k for k in range(beams - 1))
+    return ids
+
+
+def build_manager(pkv, num_blocks, bs, free_order, lens, shared_blocks, max_blocks, beams=1):
     """The batch in the C++ allocator: sequence s holds lens[s] tokens; with
     shared_blocks = P, sequence 0's first P blocks (one system prompt) are also the
-    first P blocks of every other table (reference count B), the rest private."""
+    first P blocks of every other table (reference count B), the rest private; with
+    beams > 1 every sequence is then forked into that many beams (`beam_ids`)."""
     bm = pkv.BlockManager(num_blocks, bs, free_order)
     prefix = ()
     for s in range(len(lens)):
         bm.add_seq(s, int(lens[s]), prefix)
         if s == 0 and shared_blocks:
             prefix = bm.export_tables([0], max_blocks)[0][0, :shared_blocks].tolist()
+    parents = len(lens)
+    for s in range(parents):
+        for k in range(beams - 1):
+            bm.fork(s, parents + (beams - 1) * s + k)
     return bm
 
 
@@ -391,8 +419,8 @@ def run_ours(args, rank, world, local_rank):
     n_states = min(total, args.states)
     kv8 = args.kv == "fp8"
     w = Workload(args.workload, max(n_states, min(total, args.e2e_steps + args.warmup)), seed=1000 + rank,
-                 device=device, kv8=kv8)
-    seq_ids = list(range(w.B))
+                 device=device, kv8=kv8, beams=args.beams)
+    seq_ids = w.seq_ids
 
     # ---- the allocator runs ahead of timing: `n_states` consecutive decode steps of
     # the batch.  Timed step i replays state i % n_states, so the batch keeps its
@@ -489,7 +517,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 KV, bf16 q" if kv8 else "bf16", "data": "synthetic",
-        "config": {"workload": w.name + ("+fp8" if kv8 else ""), "kv_dtype": args.kv, "num_seqs": w.B, "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D,
+        "config": {"workload": w.label, "kv_dtype": args.kv, "num_seqs": w.B, "beams": w.beams, "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D,
                    "block_size": w.bs, "mean_context": float(np.mean(w.lens0)), "num_blocks": w.NB,
                    "kv_bytes_per_step": kv_total // args.steps, "path": args.path,
                    "l2": ("L2 flushed before each timed step (a 252 MB write, outside the step's events): the"
@@ -500,7 +528,7 @@ def run_ours(args, rank, world, local_rank):
         "pct_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4),
-                     "traffic": recorded_traffic(w.name + ("+fp8" if kv8 else ""),
+                     "traffic": recorded_traffic(w.label,
                                                  ("decode_gqa_tc_fp8" if kv8 else "decode_gqa_tc") if uses_tensor
                                                  else "decode_simt", w.layout),
                      "algorithmic_bytes_per_launch": unique_total // args.steps,
@@ -542,7 +570,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     ke = max(1, min(args.steps, args.e2e_steps))
     n = args.warmup + ke
     bm = w.new_manager()
-    seq_ids = list(range(w.B))
+    seq_ids = w.seq_ids
     compute = torch.cuda.current_stream()
     copy = torch.cuda.Stream(device=device)
     nq, nk = w.B * w.Hq * w.D, w.B * w.Hkv * w.D
@@ -859,7 +887,7 @@ def cpu_baseline(w, step_inputs, budget_s=10.0):
     items = oracle_sample(w, step_inputs, 64, wl.rng_for(77))
     done, dt, n = time_oracle(w, items, budget_s)
     out = {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-           "sample": f"{n} sequences of the {w.name} batch (all {w.Hq} heads each), float64 NumPy, 1 thread, "
+           "sample": f"{n} sequences of the {w.label} batch (all {w.Hq} heads each), float64 NumPy, 1 thread, "
                      f"{dt:.1f} s"}
     try:
         done_all, dt_all, cores = time_oracle_all_cores(w, items[:n])
@@ -908,7 +936,7 @@ def cpu_baseline_fp8(w, step_inputs, budget_s=10.0):
     items = oracle_sample_fp8(w, step_inputs, 64, wl.rng_for(77))
     done, dt, n = time_oracle_fp8(w, items, budget_s)
     return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} sequences of the {w.name} batch over the 8-bit pool (all {w.Hq} heads each), "
+            "sample": f"{n} sequences of the {w.label} batch over the 8-bit pool (all {w.Hq} heads each), "
                       f"float64 NumPy, 1 thread, {dt:.1f} s"}
 
 
@@ -1218,9 +1246,9 @@ def run_reference(args, rank, world, local_rank):
     if args.workload == SWAP_WORKLOAD:
         return run_reference_swap(args, world)
     kv8 = args.kv == "fp8"
-    w = Workload(args.workload, 2, seed=1000, device=device, kv8=kv8)
+    w = Workload(args.workload, 2, seed=1000, device=device, kv8=kv8, beams=args.beams)
     bm = w.new_manager()
-    ids = list(range(w.B))
+    ids = w.seq_ids
     bm.append_slots(ids)
     tables, lens = bm.export_tables(ids, w.max_blocks)
     q, _, _ = w.host_step_inputs()
@@ -1241,12 +1269,12 @@ def run_reference(args, rank, world, local_rank):
         kv += b
         dt_total += dt
     value = kv / dt_total / 1e9
-    sample = (f"{per_step} random sequences of the {w.name} batch per step (all {w.Hq} heads"
+    sample = (f"{per_step} random sequences of the {w.label} batch per step (all {w.Hq} heads"
               f"{', 8-bit pool' if kv8 else ''}), float64 NumPy oracle, 1 thread")
     return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * dt_total / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name + ("+fp8" if kv8 else ""), "kv_dtype": args.kv, "num_seqs": w.B,
+            "config": {"workload": w.label, "kv_dtype": args.kv, "num_seqs": w.B, "beams": w.beams,
                        "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D, "block_size": w.bs},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
@@ -1315,6 +1343,8 @@ def main():
                     choices=sorted(wl.WORKLOADS) + sorted(wl.PREFILL_WORKLOADS) + [SWAP_WORKLOAD])
     ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16", help="element type of the decode pool")
     ap.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--beams", type=int, default=1,
+                    help="prefix_beams only: fork every sequence into this many beams before the first step")
     ap.add_argument("--trace", action="store_true",
                     help="run the long-context continuous-batching trace step by step (the fifth workload)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1324,6 +1354,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.beams < 1 or (args.beams > 1 and (args.workload != "prefix_beams" or args.trace)):
+        raise SystemExit("--beams N > 1 applies to --workload prefix_beams only")
     rank, world, local_rank = rank_info()
     if args.impl == "reference":
         res = run_reference(args, rank, world, local_rank)

@@ -201,3 +201,70 @@ def test_l2_flush_only_for_small_working_sets():
         c = wl.make_decode_batch(name, with_data=False)
         kv = bench.decode_bytes(c.context_lens, c.num_heads, c.num_kv_heads, c.head_dim, c.block_size, 1)[0]
         assert not bench.needs_l2_flush(kv), name         # >= 4x L2 even at one byte per value
+
+
+def test_beam_ids_group_each_parent_with_its_beams():
+    assert bench.beam_ids(3, 1) == [0, 1, 2]
+    assert bench.beam_ids(2, 4) == [0, 2, 3, 4, 1, 5, 6, 7]
+    ids = bench.beam_ids(128, 4)
+    assert sorted(ids) == list(range(512))
+
+
+def test_bench_beam_batch_matches_the_allocator_model(pkv):
+    """The forked shared-prefix batch: the C++ allocator as the bench builds it against
+    the reference model driven by the same operations; the first append copies every
+    shared partial last block for all beams but the last (which writes in place)."""
+    from oracle.block_manager import BlockManagerModel
+    import workloads as wl
+    bs, parents, beams, shared = 16, 6, 4, 4
+    rng = wl.rng_for(11)
+    lens = (shared * bs + rng.integers(10, 60, size=parents)).astype(np.int64)
+    lens[0] = shared * bs + 32                       # one parent ends on a block boundary: no copy
+    nb = 200
+    order = rng.permutation(nb).astype(np.int32)
+    mb = 16
+    bm = bench.build_manager(pkv, nb, bs, order, lens, shared, mb, beams)
+    ids = bench.beam_ids(parents, beams)
+    model = BlockManagerModel(nb, bs, initial_order=order)
+    model.add_seq(0, int(lens[0]))
+    prefix = model.tables[0][:shared]
+    for s in range(1, parents):
+        model.add_seq(s, int(lens[s]), prefix)
+    for s in range(parents):
+        for k in range(beams - 1):
+            model.fork(s, parents + (beams - 1) * s + k)
+    for step in range(3):
+        slots, pairs = bm.append_slots(ids)
+        mslots, mpairs = model.append_slots(ids)
+        assert slots.tolist() == list(mslots) and pairs.tolist() == [list(p) for p in mpairs]
+        if step == 0:
+            partial = int(np.sum(lens % bs != 0))
+            assert len(pairs) == (beams - 1) * partial
+        else:
+            assert len(pairs) == 0
+        t, l = bm.export_tables(ids, mb)
+        mt, ml = model.export_tables(ids, mb)
+        assert t.tolist() == mt and l.tolist() == ml
+    for blk in prefix:
+        assert bm.refcount(int(blk)) == parents * beams
+    # distinct bytes: the prompt once, every parent's full suffix blocks once, each beam's own last block
+    u = bench.unique_kv_bytes(t, l, 1, 8, bs, 1)
+    assert u == len({int(t[r][p // bs]) * bs + p % bs for r in range(len(ids)) for p in range(int(l[r]))}) * 16
+    bm.close()
+
+
+def test_workload_default_path_is_unforked_and_unshared(pkv):
+    """The bench's Workload on the CPU for the tiny batch: ids in order, no beams, no
+    shared blocks, the manager's tables and lengths those of plain add_seq calls."""
+    import torch
+    w = bench.Workload("tiny", 4, seed=3, device=torch.device("cpu"))
+    assert w.seq_ids == list(range(w.B)) and w.beams == 1 and w.shared_blocks == 0 and w.layout is None
+    assert w.label == "tiny"
+    bm = w.new_manager()
+    ref = pkv.BlockManager(w.NB, w.bs, w.free_order)
+    for s in range(w.B):
+        ref.add_seq(s, int(w.lens0[s]) - 1)
+    a, b = bm.export_tables(w.seq_ids, w.max_blocks), ref.export_tables(range(w.B), w.max_blocks)
+    assert a[0].tolist() == b[0].tolist() and a[1].tolist() == b[1].tolist()
+    bm.close()
+    ref.close()

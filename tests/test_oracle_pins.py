@@ -259,6 +259,53 @@ def test_paged_equals_contiguous_layout():
     assert np.array_equal(paged, contig)
 
 
+@pytest.mark.parametrize("prompt_len", [10, 12, 13])
+def test_beam_fork_copy_on_write_gives_each_beam_its_own_sequence(prompt_len):
+    """Outcome School explainer, "内存共享": beams share blocks until they diverge.  A
+    prompt forked into 4 beams, each appending its own tokens (allocator model -> copy of
+    the shared partial block -> cache write -> gather through the tables), must give
+    every beam the attention of its own contiguous sequence (the prompt, then its own
+    tokens); no beam's write may reach another beam.  Prompt lengths 10 and 13 leave a
+    partial last block (three copies on the first append), 12 ends on a boundary."""
+    from oracle.block_manager import BlockManagerModel
+    rng = wl.rng_for(400 + prompt_len)
+    bs, Hkv, Hq, D, beams, nb = 4, 2, 4, 8, 4, 40
+    scale = wl.fp32_scale(D)
+    m = BlockManagerModel(nb, bs, initial_order=rng.permutation(nb).astype(np.int32))
+    m.add_seq(0, prompt_len)
+    for b in range(1, beams):
+        m.fork(0, b)
+    ids = list(range(beams))
+    kc = wl.bf16_normal(rng, (nb, Hkv, bs, D))
+    vc = wl.bf16_normal(rng, (nb, Hkv, bs, D))
+    pk = wl.bf16_normal(rng, (prompt_len, Hkv, D))
+    pv = wl.bf16_normal(rng, (prompt_len, Hkv, D))
+    kc, vc = cache_ops.reshape_and_cache(pk, pv, kc, vc, np.asarray(m.slots(0, 0, prompt_len), np.int64))
+    own_k = [[pk[t] for t in range(prompt_len)] for _ in range(beams)]
+    own_v = [[pv[t] for t in range(prompt_len)] for _ in range(beams)]
+    for step in range(5):
+        slots, pairs = m.append_slots(ids)
+        if step == 0:
+            assert len(pairs) == (0 if prompt_len % bs == 0 else beams - 1)
+        if len(pairs):
+            ks, vs = cache_ops.copy_blocks([kc], [vc], np.asarray(pairs, np.int64))
+            kc, vc = ks[0], vs[0]
+        nk = wl.bf16_normal(rng, (beams, Hkv, D))
+        nv = wl.bf16_normal(rng, (beams, Hkv, D))
+        kc, vc = cache_ops.reshape_and_cache(nk, nv, kc, vc, np.asarray(slots, np.int64))
+        for b in range(beams):
+            own_k[b].append(nk[b])
+            own_v[b].append(nv[b])
+        q = wl.bf16_normal(rng, (beams, Hq, D))
+        tables, lens = m.export_tables(ids, 8)
+        got = paged_attention.paged_decode(q, kc, vc, np.asarray(tables, np.int32), np.asarray(lens, np.int32), scale)
+        L = prompt_len + step + 1
+        ck = np.stack([np.stack(own_k[b], axis=1) for b in range(beams)])   # [beams, Hkv, L, D]
+        cv = np.stack([np.stack(own_v[b], axis=1) for b in range(beams)])
+        exp = paged_attention.contiguous_decode(q, ck, cv, np.full(beams, L, np.int32), scale)
+        assert np.array_equal(got, exp)
+
+
 def test_golden_block_table_figure_gather():
     """The figure's request A (Block 0 -> 3, Block 1 -> 7): positions 0..31 are read
     from physical blocks 3 then 7, in that order."""

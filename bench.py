@@ -525,6 +525,7 @@ def run_ours(args, rank, world, local_rank):
                           if flush_l2 else "inputs larger than L2 (distinct KV per step >= 4x the 126 MB L2)"),
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "seq_steps_per_s": round(seq_steps, 1),
+        "seq_steps_per_s_decode_call": round(w.B * args.steps / (dec_ms * 1e-3), 1),
         "pct_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4),

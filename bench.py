@@ -710,6 +710,7 @@ def run_trace(args, rank, world, local_rank):
     for length, budget in initial:
         admit(length, budget)
     t_ms = 0.0
+    alloc_s = 0.0  # host allocator time of the timed steps (append, export, frees)
     seq_steps = 0
     kv_bytes = 0
     launches = 0
@@ -743,8 +744,10 @@ def run_trace(args, rank, world, local_rank):
         for step in range(p.steps):
             ids = sorted(running)
             if ids:
+                a0 = time.perf_counter()
                 slots, pairs = bm.append_slots(ids)
                 tables, lens = bm.export_tables(ids, max_blocks)
+                a_s = time.perf_counter() - a0
                 d_slots = torch.from_numpy(slots).to(device)
                 d_tables = torch.from_numpy(tables).to(device)
                 d_lens = torch.from_numpy(lens).to(device)
@@ -761,6 +764,7 @@ def run_trace(args, rank, world, local_rank):
                 torch.cuda.synchronize()
                 if step >= args.warmup:
                     t_ms += e0.elapsed_time(e1)
+                    alloc_s += a_s
                     seq_steps += len(ids)
                     kv_bytes += int(lens.astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 4
                     launches += 3 + (1 if len(pairs) else 0) + 1  # + the split merge
@@ -769,11 +773,14 @@ def run_trace(args, rank, world, local_rank):
                             oracle_sample_step(ids, tables, lens, q, out)
                         except Exception as e:  # the trace figure stands without its baseline
                             ora["error"] = f"{type(e).__name__}: {e}"
+                a0 = time.perf_counter()
                 for sid in ids:
                     running[sid] -= 1
                     if running[sid] == 0:
                         bm.free_seq(sid)
                         del running[sid]
+                if step >= args.warmup:
+                    alloc_s += time.perf_counter() - a0
             for length, budget in arrivals[step]:
                 if len(running) < p.max_batch:
                     admit(length, budget)
@@ -791,6 +798,9 @@ def run_trace(args, rank, world, local_rank):
                        "num_blocks": p.num_blocks, "admitted": next_id,
                        "timed": "copy_blocks + reshape_and_cache + paged_attention_decode per step"},
             "seq_steps_per_s": round(seq_steps / (t_ms * 1e-3), 1), "pct_hbm_peak": round(100 * value / peak, 2),
+            # the same with the host allocator's time per step added (it runs between the steps here)
+            "seq_steps_per_s_with_allocator": round(seq_steps / (t_ms * 1e-3 + alloc_s), 1),
+            "allocator_us_per_step": round(1e6 * alloc_s / max(1, args.steps), 2),
             "gpu_launches": launches, "clocks": clocks.summary(),
             **({"cpu_baseline": ({"unavailable": ora["error"]} if ora["error"] or not ora["n"] else
                                  {"value": round(ora["bytes"] / ora["s"] / 1e9, 4), "unit": "GB/s", "cores": 1,

@@ -796,6 +796,8 @@ def run_trace(args, rank, world, local_rank):
             "config": {"workload": "long_trace_continuous", "max_batch": p.max_batch, "num_heads": p.num_heads,
                        "num_kv_heads": p.num_kv_heads, "head_dim": p.head_dim, "block_size": p.block_size,
                        "num_blocks": p.num_blocks, "admitted": next_id,
+                       "initial_lengths": f"U{{{p.len_lo}..{p.len_hi}}}", "budgets": f"U{{{p.budget_lo}..{p.budget_hi}}}",
+                       "arrivals": f"Bernoulli({p.arrival_p}) per free slot per step, lengths U{{{p.len_lo}..{p.len_hi}}}",
                        "timed": "copy_blocks + reshape_and_cache + paged_attention_decode per step"},
             "seq_steps_per_s": round(seq_steps / (t_ms * 1e-3), 1), "pct_hbm_peak": round(100 * value / peak, 2),
             # the same with the host allocator's time per step added (it runs between the steps here)

@@ -125,6 +125,17 @@ SPEC_HBM_GBS = 8000.0  # B200 HBM3e nominal (DGX figure)
 L2_BYTES = 126 * 1000 ** 2  # B200 L2
 
 
+# The length mixes the batches are drawn with (workloads.draw_lengths), recorded in each line.
+LENGTH_MIX = {
+    "tiny": "{1, 7, 16, 33}",
+    "llama7b": "U{10..2000}",
+    "llama13b_mixed_bs16": "70% geometric(mean 50), 30% U{1000..2000}",
+    "llama13b_mixed_bs32": "70% geometric(mean 50), 30% U{1000..2000}",
+    "prefix_beams": f"{wl.PREFIX_TOKENS}-token shared prompt + U{{10..500}}",
+    "long_trace": "U{5000..32000} (a static batch)",
+}
+
+
 def needs_l2_flush(distinct_bytes_per_step: int) -> bool:
     """Steps whose distinct KV is under 4x the L2 could be served partly from what the
     previous step left there, so the timed loop flushes the L2 between them."""
@@ -518,7 +529,8 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 KV, bf16 q" if kv8 else "bf16", "data": "synthetic",
         "config": {"workload": w.label, "kv_dtype": args.kv, "num_seqs": w.B, "beams": w.beams, "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D,
-                   "block_size": w.bs, "mean_context": float(np.mean(w.lens0)), "num_blocks": w.NB,
+                   "block_size": w.bs, "lengths": LENGTH_MIX[w.name], "mean_context": float(np.mean(w.lens0)),
+                   "num_blocks": w.NB,
                    "kv_bytes_per_step": kv_total // args.steps, "path": args.path,
                    "l2": ("L2 flushed before each timed step (a 252 MB write, outside the step's events): the"
                           " distinct KV per step is under 4x the 126 MB L2; e2e steps are pipelined, not flushed"

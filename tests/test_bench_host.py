@@ -268,3 +268,8 @@ def test_workload_default_path_is_unforked_and_unshared(pkv):
     assert a[0].tolist() == b[0].tolist() and a[1].tolist() == b[1].tolist()
     bm.close()
     ref.close()
+
+
+def test_every_decode_workload_records_its_length_mix():
+    import workloads as wl
+    assert set(bench.LENGTH_MIX) == set(wl.WORKLOADS)

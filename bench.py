@@ -397,6 +397,16 @@ def build_manager(pkv, num_blocks, bs, free_order, lens, shared_blocks, max_bloc
     return bm
 
 
+def pool_usage(num_blocks: int, num_free: int, lens, bs: int) -> dict:
+    """Pool blocks in use against the blocks the tables reference (each table's view);
+    sharing shows as `saved_by_sharing` > 0."""
+    referenced = int(np.sum(-(-np.asarray(lens, np.int64) // bs)))
+    used = num_blocks - num_free
+    return {"blocks": num_blocks, "used": used, "utilisation": round(used / num_blocks, 4),
+            "referenced_by_tables": referenced,
+            "saved_by_sharing": round(1 - used / referenced, 4) if referenced else 0.0}
+
+
 def aggregate_over_ranks(ms_local, units_local, dist=None, device=None):
     """Whole-job timing: the slowest rank's time and the units all ranks processed.
 
@@ -448,6 +458,7 @@ def run_ours(args, rank, world, local_rank):
                            n_pairs=len(pairs), tables=torch.from_numpy(tables).to(device),
                            lens=torch.from_numpy(lens).to(device), max_len=int(lens.max()), host_lens=lens,
                            unique_kv=unique_kv_bytes(tables, lens, w.Hkv, w.D, w.bs, 1 if kv8 else 2)))
+    pool = pool_usage(w.NB, bm.num_free(), lens, w.bs)  # after the last prepared step
     bm.close()
     max_len_all = int(w.lens0.max()) + max(n_states, args.e2e_steps + args.warmup) + 1
     ws = torch.empty(pkv.paged_attention_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.bs, max_len_all),
@@ -530,7 +541,7 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 KV, bf16 q" if kv8 else "bf16", "data": "synthetic",
         "config": {"workload": w.label, "kv_dtype": args.kv, "num_seqs": w.B, "beams": w.beams, "num_heads": w.Hq, "num_kv_heads": w.Hkv, "head_dim": w.D,
                    "block_size": w.bs, "lengths": LENGTH_MIX[w.name], "mean_context": float(np.mean(w.lens0)),
-                   "num_blocks": w.NB,
+                   "num_blocks": w.NB, "pool": pool,
                    "kv_bytes_per_step": kv_total // args.steps, "path": args.path,
                    "l2": ("L2 flushed before each timed step (a 252 MB write, outside the step's events): the"
                           " distinct KV per step is under 4x the 126 MB L2; e2e steps are pipelined, not flushed"

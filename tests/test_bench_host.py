@@ -273,3 +273,20 @@ def test_workload_default_path_is_unforked_and_unshared(pkv):
 def test_every_decode_workload_records_its_length_mix():
     import workloads as wl
     assert set(bench.LENGTH_MIX) == set(wl.WORKLOADS)
+
+
+def test_pool_usage_shows_what_sharing_saves(pkv):
+    import workloads as wl
+    b = wl.make_decode_batch("prefix_beams", with_data=False)
+    bs, B = b.block_size, b.num_seqs
+    lens = b.context_lens.astype(np.int64)
+    nb = int(np.ceil(1.2 * np.sum(-(-lens // bs))))
+    order = wl.rng_for(7).permutation(nb).astype(np.int32)
+    bm = bench.build_manager(pkv, nb, bs, order, lens, wl.PREFIX_TOKENS // bs, int(np.max(-(-lens // bs))))
+    u = bench.pool_usage(nb, bm.num_free(), lens, bs)
+    ref = int(np.sum(-(-lens // bs)))
+    assert u["referenced_by_tables"] == ref and u["used"] == ref - (B - 1) * (wl.PREFIX_TOKENS // bs)
+    assert 0.7 < u["saved_by_sharing"] < 0.9 and u["utilisation"] == round(u["used"] / nb, 4)
+    plain = bench.pool_usage(nb, nb - ref, lens, bs)
+    assert plain["saved_by_sharing"] == 0.0
+    bm.close()

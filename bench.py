@@ -483,7 +483,7 @@ def run_ours(args, rank, world, local_rank):
         step(i)
     torch.cuda.synchronize()
     launches = 0
-    kv_total = bytes_total = unique_total = 0
+    kv_total = bytes_total = unique_total = unique_kv_total = 0
     g = w.Hq // w.Hkv
     uses_tensor = path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16)
     # write, plan, decode (+ copy_blocks when a fork copied blocks) (+ the merge of a split context)
@@ -494,6 +494,7 @@ def run_ours(args, rank, world, local_rank):
         kv_total += kv
         bytes_total += alg
         unique_total += alg - kv + st["unique_kv"]
+        unique_kv_total += st["unique_kv"]
         launches += 3 + (1 if st["n_pairs"] else 0) + merge
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
@@ -549,7 +550,9 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "seq_steps_per_s": round(seq_steps, 1),
         "seq_steps_per_s_decode_call": round(w.B * args.steps / (dec_ms * 1e-3), 1),
-        "pct_hbm_peak": round(100 * value / world / peak, 2),
+        # of the HBM peak, on distinct KV bytes (a shared block's bytes once; the same as
+        # `value` unless tables share blocks, when logical GB/s can exceed the peak)
+        "pct_hbm_peak": round(100 * value * (unique_kv_total / kv_total if kv_total else 1.0) / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4),
                      "traffic": recorded_traffic(w.label,

@@ -290,3 +290,29 @@ def test_pool_usage_shows_what_sharing_saves(pkv):
     plain = bench.pool_usage(nb, nb - ref, lens, bs)
     assert plain["saved_by_sharing"] == 0.0
     bm.close()
+
+
+def _run_bench(*args):
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], capture_output=True, text=True,
+                          timeout=600, cwd=root)
+
+
+def test_reference_arm_without_a_device_prints_one_line_and_exits_0():
+    import json
+    if torch.cuda.is_available():
+        import pytest
+        pytest.skip("a CUDA device is present; this checks the host-only fallback")
+    r = _run_bench("--impl", "reference", "--steps", "2", "--warmup", "3")
+    assert r.returncode == 0
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and "unavailable" in out
+
+
+def test_beams_only_for_the_shared_prefix_workload():
+    r = _run_bench("--workload", "llama7b", "--beams", "4", "--warmup", "3")
+    assert r.returncode != 0 and "prefix_beams only" in r.stderr

@@ -18,6 +18,8 @@
  *     Device tensors must start on a 16-byte boundary (PKV_ERR_INVALID otherwise).
  *   - Kernel calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  A return of PKV_OK means the work was enqueued.
+ *   - Kernels launch on the calling thread's current CUDA device; every device
+ *     pointer of a call, and `stream`, must belong to that device.
  *   - Argument errors are reported before anything is enqueued and leave all
  *     memory untouched.  Data-dependent errors found on the device (an index out
  *     of range) never trap: the offending row/block is skipped and a bit is OR-ed

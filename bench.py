@@ -592,8 +592,9 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     would run it: per step the C++ allocator produces slots and tables on the host;
     q, new K, new V (one pinned buffer per step) and the allocator output (a small
     pinned buffer, double-buffered) go host->device on a copy stream while the
-    previous step's kernels run; the step's output comes back to pinned memory and
-    is read on the host one step later."""
+    previous step's kernels run; the step's output comes back to pinned memory on a
+    stream of its own (beside the next step's kernels) and is read on the host one
+    step later."""
     import torch
     ke = max(1, min(args.steps, args.e2e_steps))
     n = args.warmup + ke
@@ -601,6 +602,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     seq_ids = w.seq_ids
     compute = torch.cuda.current_stream()
     copy = torch.cuda.Stream(device=device)
+    d2h = torch.cuda.Stream(device=device)          # results back to the host beside the next step
     nq, nk = w.B * w.Hq * w.D, w.B * w.Hkv * w.D
     # per-step pinned q | k | v (bf16 bits)
     host_qkv = []
@@ -621,6 +623,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     outs = [out, torch.empty_like(out)]
     h2d_done = [torch.cuda.Event() for _ in range(n)]
     comp_done = [torch.cuda.Event() for _ in range(n)]
+    d2h_done = [torch.cuda.Event() for _ in range(n)]
     stats = {"h2d": 0, "d2h": 0, "kv": 0, "checksum": 0.0}
 
     def step(i):
@@ -653,11 +656,16 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
             d_pairs = dm[o_pairs:o_pairs + pairs.nbytes].view(torch.int64).view(-1, 2)
             w.copy(d_pairs, status)
         w.write(dk, dv, d_slots, status)
+        if i >= 2:
+            compute.wait_event(d2h_done[i - 2])    # outs[b] has been copied out
         w.decode(outs[b], dq, d_tables, d_lens, max_len_bound, ws, path, status)
-        out_host[b].copy_(outs[b], non_blocking=True)
         comp_done[i].record(compute)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(comp_done[i])
+            out_host[b].copy_(outs[b], non_blocking=True)
+            d2h_done[i].record(d2h)
         if i >= 1:                                 # read the previous step's result on the host
-            comp_done[i - 1].synchronize()
+            d2h_done[i - 1].synchronize()
             stats["checksum"] += float(out_host[(i - 1) % 2][0, 0, 0])
         if i >= args.warmup:
             stats["h2d"] += host_qkv[i].numel() * 2 + slots.nbytes + pairs.nbytes + tables.nbytes + lens.nbytes
@@ -672,7 +680,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     compute.wait_event(t0)
     for i in range(args.warmup, n):
         step(i)
-    comp_done[n - 1].synchronize()                 # the last step's result
+    d2h_done[n - 1].synchronize()                  # the last step's result
     stats["checksum"] += float(out_host[(n - 1) % 2][0, 0, 0])
     t1.record(compute)
     torch.cuda.synchronize()
@@ -682,7 +690,8 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
             "h2d_bytes_per_step": stats["h2d"] // ke, "d2h_bytes_per_step": stats["d2h"] // ke,
             "ms_per_step": round(ms / ke, 4), "steps": ke,
             "seq_steps_per_s": round(w.B * ke / (ms * 1e-3), 1),
-            "pipelining": "H2D of step i+1 on a copy stream overlaps the kernels of step i; results read one step later"}
+            "pipelining": "H2D of step i+1 on a copy stream and D2H of step i-1 on a result stream overlap the"
+                          " kernels of step i; results read one step later"}
 
 
 # ---------------------------------------------------------------------------

@@ -316,3 +316,65 @@ def test_reference_arm_without_a_device_prints_one_line_and_exits_0():
 def test_beams_only_for_the_shared_prefix_workload():
     r = _run_bench("--workload", "llama7b", "--beams", "4", "--warmup", "3")
     assert r.returncode != 0 and "prefix_beams only" in r.stderr
+
+
+class _FakeEvent:
+    def __init__(self, enable_timing=False):
+        self.recorded = False
+
+    def record(self, stream=None):
+        self.recorded = True
+
+    def synchronize(self):
+        assert self.recorded, "waited on an event that was never recorded"
+
+    def elapsed_time(self, other):
+        return 2.0
+
+
+class _FakeStream:
+    def __init__(self, device=None):
+        pass
+
+    def wait_event(self, ev):
+        pass
+
+
+def test_e2e_host_logic_with_stand_in_streams(pkv, monkeypatch):
+    """The e2e harness's host logic on the CPU: streams, events and pinning replaced by
+    stand-ins and the three kernels by stubs (the stub decode writes a known output).
+    Checks the per-step byte accounting, the KV bytes and that every step's output is
+    read back once."""
+    import contextlib
+    import types
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Stream", _FakeStream)
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    w = bench.Workload("tiny", 8, seed=5, device=torch.device("cpu"))
+    calls = {"write": 0, "decode": 0, "copy": 0}
+
+    def write(k, v, slots, status):
+        assert k.shape == (w.B, w.Hkv, w.D) and slots.shape == (w.B,)
+        calls["write"] += 1
+
+    def decode(out, q, tables, lens, max_len, ws, path, status):
+        assert q.shape == (w.B, w.Hq, w.D) and tables.shape == (w.B, w.max_blocks) and lens.shape == (w.B,)
+        out.fill_(1.0)
+        calls["decode"] += 1
+
+    w.write, w.decode = write, decode
+    w.copy = lambda pairs, status: calls.__setitem__("copy", calls["copy"] + 1)
+    args = types.SimpleNamespace(steps=4, e2e_steps=4, warmup=3)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16)
+    res = bench.run_e2e(args, w, pkv, torch.device("cpu"), 0, None, out, None, 1024)
+    assert calls["write"] == calls["decode"] == 7 and calls["copy"] == 0
+    per_step_in = 2 * w.B * (w.Hq + 2 * w.Hkv) * w.D + 8 * w.B + 4 * w.B * w.max_blocks + 4 * w.B
+    assert res["h2d_bytes_per_step"] == per_step_in
+    assert res["d2h_bytes_per_step"] == 2 * w.B * w.Hq * w.D
+    assert res["steps"] == 4 and res["ms_per_step"] == 0.5
+    # KV of the timed steps: the allocator's lengths at steps 3..6 (lens0 at step 0)
+    kv = sum(int((w.lens0 + i).sum()) for i in range(3, 7)) * w.Hkv * w.D * 2 * 2
+    assert res["value"] == round(kv / (2.0 * 1e-3) / 1e9, 1)

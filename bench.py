@@ -426,11 +426,17 @@ def to_dev(bits, device):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
 
 
+def bench_device(local_rank: int):
+    """The CUDA device of this rank (one process per GPU)."""
+    import torch
+    return torch.device(f"cuda:{local_rank}")
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import paged_kv_cache_423_b200 as pkv
 
-    device = torch.device(f"cuda:{local_rank}")
+    device = bench_device(local_rank)
     torch.cuda.set_device(device)
     dist = None
     if world > 1:

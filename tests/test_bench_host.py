@@ -378,3 +378,81 @@ def test_e2e_host_logic_with_stand_in_streams(pkv, monkeypatch):
     # KV of the timed steps: the allocator's lengths at steps 3..6 (lens0 at step 0)
     kv = sum(int((w.lens0 + i).sum()) for i in range(3, 7)) * w.Hkv * w.D * 2 * 2
     assert res["value"] == round(kv / (2.0 * 1e-3) / 1e9, 1)
+
+
+class _FakeClocks:
+    def __init__(self, device):
+        pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+    def summary(self):
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": []}
+
+
+def _stand_in_run_ours(monkeypatch, pkv, calls, **overrides):
+    import contextlib
+    import types
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Stream", _FakeStream)
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    monkeypatch.setattr(bench, "bench_device", lambda local_rank: torch.device("cpu"))
+    monkeypatch.setattr(bench, "ClockSampler", _FakeClocks)
+    monkeypatch.setattr(bench, "stream_read_gbs", lambda pkv, device: 7000.0)
+
+    def count(name):
+        def f(self, *a, **k):
+            calls[name] = calls.get(name, 0) + 1
+        return f
+    monkeypatch.setattr(bench.Workload, "write", count("write"))
+    monkeypatch.setattr(bench.Workload, "copy", count("copy"))
+    monkeypatch.setattr(bench.Workload, "decode", count("decode"))
+    args = types.SimpleNamespace(workload="tiny", steps=5, warmup=3, states=4, e2e_steps=3, kv="bf16", path="auto",
+                                 beams=1, no_e2e=False, no_cpu_baseline=True, cpu_budget=1.0)
+    for k, v in overrides.items():
+        setattr(args, k, v)
+    return bench.run_ours(args, 0, 1, 0)
+
+
+def test_run_ours_host_logic_with_stand_ins(pkv, monkeypatch):
+    """The decode bench's host logic on the CPU (stand-in streams, events, clocks and
+    kernels) for the tiny batch: every contract key, the launch count, the L2 flush of a
+    small working set, and distinct bytes equal to logical bytes with nothing shared."""
+    calls = {}
+    res = _stand_in_run_ours(monkeypatch, pkv, calls)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in res, key
+    assert calls["decode"] == 3 + 5 + 3 + 3 and "copy" not in calls   # warm-up, timed, e2e warm-up and timed
+    assert res["gpu_launches"] == 5 * 3                                # write, plan, decode per step (no split)
+    assert res["config"]["l2"].startswith("L2 flushed")                # 29 KB of KV is far below 4x L2
+    assert res["config"]["pool"]["saved_by_sharing"] == 0.0
+    r = res["roofline"]
+    assert r["algorithmic_bytes_per_launch"] == r["logical_bytes_per_launch"]
+    assert res["ms_per_step"] == 2.0                                   # the stand-in events' elapsed time
+
+
+def test_run_ours_beam_phase_with_stand_ins(pkv, monkeypatch):
+    """The shared-prefix batch forked into 4 beams (6 prompts here): copies on the first
+    prepared step only, distinct bytes well below logical, sharing visible in the pool."""
+    import workloads as wl
+    orig = wl.make_decode_batch
+    monkeypatch.setattr(wl, "make_decode_batch", lambda name, **k: orig(name, num_seqs=6, **k))
+    calls = {}
+    res = _stand_in_run_ours(monkeypatch, pkv, calls, workload="prefix_beams", beams=4, steps=4, states=4)
+    cfg = res["config"]
+    assert cfg["num_seqs"] == 24 and cfg["beams"] == 4 and cfg["workload"] == "prefix_beams+beams4"
+    assert cfg["pool"]["saved_by_sharing"] > 0.5
+    r = res["roofline"]
+    assert r["algorithmic_bytes_per_launch"] < 0.5 * r["logical_bytes_per_launch"]
+    assert r["traffic"] is None                      # no capture on this layout
+    # the first prepared step carries the copies; timed steps replay states 3, 0, 1, 2
+    assert calls.get("copy", 0) >= 1

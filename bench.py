@@ -714,7 +714,7 @@ def run_trace(args, rank, world, local_rank):
     import torch
     import paged_kv_cache_423_b200 as pkv
 
-    device = torch.device(f"cuda:{local_rank}")
+    device = bench_device(local_rank)
     torch.cuda.set_device(device)
     p = wl.TraceParams(steps=args.warmup + args.steps)
     initial, arrivals = wl.trace_events(p, seed=2000 + rank)
@@ -1095,7 +1095,7 @@ def prefill_oracle_rate(pw, q_bits, budget_s, rng):
 
 def run_prefill(args, rank, world, local_rank):
     import torch
-    device = torch.device(f"cuda:{local_rank}")
+    device = bench_device(local_rank)
     torch.cuda.set_device(device)
     dist = None
     if world > 1:
@@ -1198,7 +1198,7 @@ SWAP_PAIRS = 256
 def run_swap(args, rank, world, local_rank):
     import torch
     import paged_kv_cache_423_b200 as pkv
-    device = torch.device(f"cuda:{local_rank}")
+    device = bench_device(local_rank)
     torch.cuda.set_device(device)
     dist = None
     if world > 1:
@@ -1292,7 +1292,7 @@ def run_reference(args, rank, world, local_rank):
     import torch
     if rank != 0:
         return None
-    device = torch.device(f"cuda:{local_rank}") if torch.cuda.is_available() else None
+    device = bench_device(local_rank) if torch.cuda.is_available() else None
     if device is None:
         return {"impl": "reference", "unavailable": "no CUDA device to hold the synthetic workload"}
     torch.cuda.set_device(device)

@@ -456,3 +456,37 @@ def test_run_ours_beam_phase_with_stand_ins(pkv, monkeypatch):
     assert r["traffic"] is None                      # no capture on this layout
     # the first prepared step carries the copies; timed steps replay states 3, 0, 1, 2
     assert calls.get("copy", 0) >= 1
+
+
+def test_run_trace_host_logic_with_stand_ins(pkv, monkeypatch):
+    """The continuous-batching trace bench on the CPU with a shrunken trace (4 slots,
+    short contexts, small pool) and stubbed kernels: admissions, frees and the recorded
+    readings, allocator time reported, seq-steps with it below those without."""
+    import contextlib
+    import types
+    import workloads as wl
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(bench, "bench_device", lambda local_rank: torch.device("cpu"))
+    monkeypatch.setattr(bench, "ClockSampler", _FakeClocks)
+    orig = wl.TraceParams
+    monkeypatch.setattr(wl, "TraceParams", lambda steps: orig(max_batch=4, num_heads=8, num_kv_heads=2, head_dim=64,
+                                                             block_size=16, len_lo=40, len_hi=120, budget_lo=1,
+                                                             budget_hi=6, steps=steps, num_blocks=256))
+    kernel_calls = {"decode": 0, "write": 0}
+    monkeypatch.setattr(pkv, "reshape_and_cache",
+                        lambda *a, **k: kernel_calls.__setitem__("write", kernel_calls["write"] + 1))
+    monkeypatch.setattr(pkv, "paged_attention_decode",
+                        lambda *a, **k: kernel_calls.__setitem__("decode", kernel_calls["decode"] + 1))
+    monkeypatch.setattr(pkv, "copy_blocks", lambda *a, **k: None)
+    args = types.SimpleNamespace(steps=20, warmup=3, no_cpu_baseline=True)
+    res = bench.run_trace(args, 0, 1, 0)
+    cfg = res["config"]
+    assert cfg["workload"] == "long_trace_continuous" and cfg["admitted"] > 4
+    assert cfg["initial_lengths"] == "U{40..120}" and cfg["budgets"] == "U{1..6}"
+    assert cfg["arrivals"].startswith("Bernoulli(0.5) per free slot per step")
+    assert 0 < kernel_calls["decode"] <= 23
+    assert res["allocator_us_per_step"] > 0
+    assert res["seq_steps_per_s_with_allocator"] < res["seq_steps_per_s"]

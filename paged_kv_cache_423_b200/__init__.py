@@ -42,7 +42,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 
 
 def library_path() -> str:
-    return os.path.join(_HERE, "libpkv.so")
+    """The in-tree libpkv.so, or the build named by the PKV_LIBRARY environment variable
+    (another build of the same sources, e.g. the one-stage-ring variant a test compares)."""
+    return os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpkv.so")
 
 
 class PkvError(RuntimeError):

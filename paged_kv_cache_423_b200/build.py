@@ -7,6 +7,10 @@ library loads on machines without a GPU (the NVIDIA driver is only needed once a
 touches the device).  ptxas register/shared-memory reports go to
 ``_build/ptxas.log``.  Rebuilds only when a source or header is newer than the
 library.
+
+``variant="depth1"`` builds ``libpkv_depth1.so`` (objects under ``_build/depth1``) with the
+CUDA-core decode kernel's per-warp copy ring at one stage, so every copy waits for the
+previous stage's compute; a test compares it bit for bit with the default build.
 """
 from __future__ import annotations
 
@@ -27,6 +31,11 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xptxas", "-v",
               "--expt-relaxed-constexpr", "-Xcompiler", "-fvisibility=hidden"]
 CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-fvisibility=hidden"]
+VARIANTS = {"depth1": ["-DPKV_SIMT_STAGES=1", "-DPKV_SIMT_STAGES8=1"]}
+
+
+def lib_path(variant: str | None = None) -> str:
+    return LIB if variant is None else os.path.join(PKG, f"libpkv_{variant}.so")
 
 
 def nvcc() -> str:
@@ -47,18 +56,19 @@ def _inputs():
     return files
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB):
+def is_stale(variant: str | None = None) -> bool:
+    lib = lib_path(variant)
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
-def _compile(src: str) -> tuple[str, str]:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, build_dir: str = BUILD, extra_defs=()) -> tuple[str, str]:
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     inc = ["-I", INCLUDE, "-I", CSRC]
     # Exported symbols carry default visibility through the header's extern "C" block.
-    defs = ["-DPKV_BUILD"]
+    defs = ["-DPKV_BUILD", *extra_defs]
     if src.endswith(".cu"):
         cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *inc, *defs, "-c", src, "-o", obj]
     else:
@@ -70,26 +80,30 @@ def _compile(src: str) -> tuple[str, str]:
     return obj, res.stderr
 
 
-def build_library(force: bool = False, verbose: bool = False) -> str:
-    if not force and not is_stale():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build_library(force: bool = False, verbose: bool = False, variant: str | None = None) -> str:
+    lib = lib_path(variant)
+    if not force and not is_stale(variant):
+        return lib
+    build_dir = BUILD if variant is None else os.path.join(BUILD, variant)
+    extra = () if variant is None else VARIANTS[variant]
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(_compile, srcs))
-    with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+        results = list(ex.map(lambda src: _compile(src, build_dir, extra), srcs))
+    with open(os.path.join(build_dir, "ptxas.log"), "w") as f:
         for (obj, log), src in zip(results, srcs):
             f.write(f"==== {os.path.basename(src)}\n{log}\n")
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *[o for o, _ in results], "-cudart", "static"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"linking libpkv.so failed:\n{' '.join(cmd)}\n{res.stdout}\n{res.stderr}")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     if verbose:
-        print(f"built {LIB}")
-    return LIB
+        print(f"built {lib}")
+    return lib
 
 
 if __name__ == "__main__":
-    build_library(force="--force" in sys.argv, verbose=True)
+    v = sys.argv[sys.argv.index("--variant") + 1] if "--variant" in sys.argv else None
+    build_library(force="--force" in sys.argv, verbose=True, variant=v)

@@ -396,3 +396,23 @@ def test_copy_blocks_pool_types_checked_before_device_work(pkv):
         pkv.copy_blocks([torch.zeros((4, 1, 1, 15), dtype=torch.uint8)], [torch.zeros((4, 1, 1, 15), dtype=torch.uint8)], m)
     with pytest.raises(ValueError, match="must be a CUDA tensor"):  # types pass, then the pointer check
         pkv.copy_blocks([torch.zeros((4, 1, 16, 64), dtype=torch.uint8)], [torch.zeros((4, 1, 16, 64), dtype=torch.uint8)], m)
+
+
+def test_one_stage_ring_variant_builds_and_loads_through_the_override(pkv):
+    """The build variant the ring-depth race check compares exports every declared symbol,
+    and the binding loads it when PKV_LIBRARY names it (in a fresh process)."""
+    import subprocess
+    import sys
+    from paged_kv_cache_423_b200 import build as pkv_build
+    lib1 = pkv_build.build_library(variant="depth1")
+    assert lib1.endswith("libpkv_depth1.so") and lib1 != pkv.library_path()
+    lib = ctypes.CDLL(lib1)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = "import paged_kv_cache_423_b200 as p; p.library(); print(p.library_path()); print(p.library().pkv_version())"
+    r = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, PKV_LIBRARY=lib1), cwd=root,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    path, version = r.stdout.split()
+    assert path == lib1 and int(version) == pkv.library().pkv_version()

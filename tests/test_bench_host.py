@@ -496,3 +496,14 @@ def test_run_trace_host_logic_with_stand_ins(pkv, monkeypatch):
     assert res["seq_steps_per_s_with_allocator"] < res["seq_steps_per_s"]
     import json
     json.dumps(res)
+
+
+def test_cpu_baseline_leg_with_stand_ins(pkv, monkeypatch):
+    """The oracle leg of the decode line (1 core, then every core over spawned workers)
+    on the tiny batch, through the same stand-ins."""
+    calls = {}
+    res = _stand_in_run_ours(monkeypatch, pkv, calls, no_cpu_baseline=False, cpu_budget=1.0)
+    cb = res["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0 and cb["unit"] == "GB/s"
+    assert "tiny batch" in cb["sample"]
+    assert cb["all_cores"]["cores"] >= 1 and cb["all_cores"]["value"] > 0

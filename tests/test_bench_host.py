@@ -339,6 +339,9 @@ class _FakeStream:
     def wait_event(self, ev):
         pass
 
+    def synchronize(self):
+        pass
+
 
 def test_e2e_host_logic_with_stand_in_streams(pkv, monkeypatch):
     """The e2e harness's host logic on the CPU: streams, events and pinning replaced by
@@ -507,3 +510,39 @@ def test_cpu_baseline_leg_with_stand_ins(pkv, monkeypatch):
     assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0 and cb["unit"] == "GB/s"
     assert "tiny batch" in cb["sample"]
     assert cb["all_cores"]["cores"] >= 1 and cb["all_cores"]["value"] > 0
+
+
+def test_run_prefill_host_logic_with_stand_ins(pkv, monkeypatch):
+    """The chunked-prefill line on the CPU with a shrunken batch and stubbed kernels:
+    contract keys, launches, FLOPs per step, and the e2e byte counts."""
+    import contextlib
+    import json
+    import types
+    import workloads as wl
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    monkeypatch.setattr(bench, "bench_device", lambda local_rank: torch.device("cpu"))
+    monkeypatch.setattr(bench, "ClockSampler", _FakeClocks)
+    orig = wl.make_prefill_batch
+    monkeypatch.setattr(wl, "make_prefill_batch",
+                        lambda name, **k: orig(name, num_seqs=3, length_scale=0.05, num_heads=8, num_kv_heads=4, **k))
+    calls = {"write": 0, "prefill": 0}
+    monkeypatch.setattr(pkv, "reshape_and_cache", lambda *a, **k: calls.__setitem__("write", calls["write"] + 1))
+    monkeypatch.setattr(pkv, "paged_attention_prefill",
+                        lambda *a, **k: calls.__setitem__("prefill", calls["prefill"] + 1))
+    args = types.SimpleNamespace(workload="chunked_prefill_13b", steps=4, warmup=3, e2e_steps=2,
+                                 no_cpu_baseline=True, cpu_budget=1.0)
+    res = bench.run_prefill(args, 0, 1, 0)
+    json.dumps(res)
+    assert calls["prefill"] == 3 + 4 + 2 and calls["write"] == calls["prefill"]
+    cfg = res["config"]
+    T, Hq, Hkv, D = cfg["query_tokens"], cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"]
+    assert (Hq, Hkv) == (8, 4) and T == sum(cfg["query_lens"])
+    assert cfg["flops_per_step"] == bench.prefill_flops(np.array(cfg["query_lens"]), np.array(cfg["context_lens"]),
+                                                        Hq, D)
+    assert res["gpu_launches"] == 3 * 4 and res["roofline"]["bound"] == "tensor"
+    assert res["e2e"]["h2d_bytes_per_step"] == 2 * T * (Hq + 2 * Hkv) * D
+    assert res["e2e"]["d2h_bytes_per_step"] == 2 * T * Hq * D

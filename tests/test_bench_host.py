@@ -546,3 +546,29 @@ def test_run_prefill_host_logic_with_stand_ins(pkv, monkeypatch):
     assert res["gpu_launches"] == 3 * 4 and res["roofline"]["bound"] == "tensor"
     assert res["e2e"]["h2d_bytes_per_step"] == 2 * T * (Hq + 2 * Hkv) * D
     assert res["e2e"]["d2h_bytes_per_step"] == 2 * T * Hq * D
+
+
+def test_run_swap_host_logic_with_stand_ins(pkv, monkeypatch):
+    """The swap line on the CPU with small blocks and a stubbed swap kernel: four calls
+    per step (K and V out, K and V in), bytes per step, and the JSON line."""
+    import json
+    import types
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    monkeypatch.setattr(bench, "bench_device", lambda local_rank: torch.device("cpu"))
+    monkeypatch.setattr(bench, "ClockSampler", _FakeClocks)
+    monkeypatch.setattr(bench, "SWAP_SHAPE", (2, 16, 8))
+    seen = []
+    monkeypatch.setattr(pkv, "swap_blocks", lambda src, dst, pairs, **k: seen.append((src.shape[0], dst.shape[0],
+                                                                                        tuple(pairs.shape))))
+    args = types.SimpleNamespace(steps=5, warmup=3, no_cpu_baseline=True, cpu_budget=1.0)
+    res = bench.run_swap(args, 0, 1, 0)
+    json.dumps(res)
+    assert len(seen) == 4 * (3 + 5)
+    assert {s[2] for s in seen} == {(bench.SWAP_PAIRS, 2)}
+    assert seen[0][:2] == (4096, 1024) and seen[2][:2] == (1024, 4096)      # out to the host pool, then back in
+    block = 2 * 16 * 8 * 2
+    assert res["config"]["block_bytes"] == block and res["config"]["bytes_per_step"] == 4 * bench.SWAP_PAIRS * block

@@ -572,3 +572,21 @@ def test_run_swap_host_logic_with_stand_ins(pkv, monkeypatch):
     assert seen[0][:2] == (4096, 1024) and seen[2][:2] == (1024, 4096)      # out to the host pool, then back in
     block = 2 * 16 * 8 * 2
     assert res["config"]["block_bytes"] == block and res["config"]["bytes_per_step"] == 4 * bench.SWAP_PAIRS * block
+
+
+def test_reference_arm_with_stand_ins(pkv, monkeypatch):
+    """The reference arm (the oracle timed on the host) on the tiny batch, its device
+    stood in by the CPU: the JSON line with impl, cpu_baseline and a zero-copy e2e."""
+    import json
+    import types
+    monkeypatch.setattr(torch.cuda, "is_available", lambda: True)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(bench, "bench_device", lambda local_rank: torch.device("cpu"))
+    args = types.SimpleNamespace(workload="tiny", steps=2, warmup=3, kv="bf16", beams=1, ref_budget=2.0,
+                                 cpu_budget=1.0)
+    res = bench.run_reference(args, 0, 1, 0)
+    json.dumps(res)
+    assert res["impl"] == "reference" and res["value"] > 0 and res["unit"] == "GB/s"
+    assert res["cpu_baseline"]["kind"] == "oracle" and res["cpu_baseline"]["value"] == res["value"]
+    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["d2h_bytes_per_step"] == 0
+    assert res["config"]["workload"] == "tiny"

@@ -298,10 +298,53 @@ def e4m3_pool(shape, gen, device):
     return ((sign << 7) | (exp << 3) | mant).to(torch.uint8)
 
 
+class ModelManager:
+    """The allocator's reference model (`oracle.block_manager.BlockManagerModel`) with the
+    C++ manager's array outputs.  The reference arm builds its tables with it, so that it
+    loads nothing from the library; the operations are the same, so the tables are too."""
+
+    def __init__(self, num_blocks, block_size, initial_order=None):
+        from oracle.block_manager import BlockManagerModel
+        self.m = BlockManagerModel(num_blocks, block_size, initial_order=initial_order)
+
+    def add_seq(self, seq_id, num_tokens, shared_prefix_blocks=()):
+        self.m.add_seq(seq_id, num_tokens, [int(b) for b in shared_prefix_blocks])
+
+    def fork(self, parent, child):
+        self.m.fork(parent, child)
+
+    def append_slots(self, seq_ids):
+        slots, pairs = self.m.append_slots([int(s) for s in seq_ids])
+        return np.asarray(slots, np.int64), np.asarray(pairs, np.int64).reshape(-1, 2)
+
+    def slots(self, seq_id, start, count):
+        return np.asarray(self.m.slots(seq_id, start, count), np.int64)
+
+    def export_tables(self, seq_ids, max_blocks):
+        ids = [int(s) for s in seq_ids]
+        tables, lens = self.m.export_tables(ids, max_blocks)
+        return np.asarray(tables, np.int32).reshape(len(ids), max_blocks), np.asarray(lens, np.int32)
+
+    def num_free(self):
+        return self.m.num_free()
+
+    def refcount(self, b):
+        return self.m.refcount(b)
+
+    def close(self):
+        pass
+
+
 class Workload:
-    def __init__(self, name: str, steps: int, seed: int, device, kv8: bool = False, beams: int = 1):
+    def __init__(self, name: str, steps: int, seed: int, device, kv8: bool = False, beams: int = 1,
+                 native: bool = True):
+        """native=False (the reference arm): the library is not loaded and the batch's
+        tables come from the allocator's reference model."""
         import torch
-        import paged_kv_cache_423_b200 as pkv
+        if native:
+            import paged_kv_cache_423_b200 as pkv
+        else:
+            pkv = None
         self.name = name
         self.kv8 = kv8
         self.beams = beams
@@ -358,7 +401,8 @@ class Workload:
                                             ws, path=path, status=status)
 
     def new_manager(self):
-        return build_manager(self.pkv, self.NB, self.bs, self.free_order, self.parent_lens0 - 1, self.shared_blocks,
+        factory = self.pkv.BlockManager if self.pkv is not None else ModelManager
+        return build_manager(factory, self.NB, self.bs, self.free_order, self.parent_lens0 - 1, self.shared_blocks,
                              self.max_blocks, self.beams)
 
     def host_step_inputs(self):
@@ -379,12 +423,13 @@ def beam_ids(parents: int, beams: int) -> list:
     return ids
 
 
-def build_manager(pkv, num_blocks, bs, free_order, lens, shared_blocks, max_blocks, beams=1):
-    """The batch in the C++ allocator: sequence s holds lens[s] tokens; with
+def build_manager(new_manager, num_blocks, bs, free_order, lens, shared_blocks, max_blocks, beams=1):
+    """The batch in an allocator made by `new_manager(num_blocks, bs, free_order)` (the C++
+    `BlockManager`, or `ModelManager` for the reference arm): sequence s holds lens[s] tokens; with
     shared_blocks = P, sequence 0's first P blocks (one system prompt) are also the
     first P blocks of every other table (reference count B), the rest private; with
     beams > 1 every sequence is then forked into that many beams (`beam_ids`)."""
-    bm = pkv.BlockManager(num_blocks, bs, free_order)
+    bm = new_manager(num_blocks, bs, free_order)
     prefix = ()
     for s in range(len(lens)):
         bm.add_seq(s, int(lens[s]), prefix)
@@ -1013,14 +1058,19 @@ class PrefillWorkload:
     drawn on the host and uploaded before timing; the allocator gives tables and the
     chunk tokens' slots."""
 
-    def __init__(self, name, n_states, seed, device):
+    def __init__(self, name, n_states, seed, device, native=True):
+        """native=False (the reference arm): the library is not loaded, the tables come
+        from the allocator's reference model and no workspace is allocated."""
         import torch
-        import paged_kv_cache_423_b200 as pkv
+        if native:
+            import paged_kv_cache_423_b200 as pkv
+        else:
+            pkv = None
         self.pkv = pkv
         b = wl.make_prefill_batch(name, with_data=False)
         self.b = b
         self.name = name
-        bm = pkv.BlockManager(b.num_blocks, b.block_size, b.free_order)
+        bm = (pkv.BlockManager if native else ModelManager)(b.num_blocks, b.block_size, b.free_order)
         ids = list(range(b.num_seqs))
         slots = []
         for s in ids:
@@ -1045,8 +1095,9 @@ class PrefillWorkload:
             q = wl.bf16_normal(rng, (T, b.num_heads, b.head_dim))
             k, v = wl.new_tokens(rng, T, b.num_kv_heads, b.head_dim)
             self.host.append((q, k, v))
-        self.ws = torch.empty(pkv.paged_attention_prefill_workspace_size(b.num_seqs, T, b.num_heads, b.num_kv_heads),
-                              dtype=torch.uint8, device=device)
+        self.ws = None if pkv is None else torch.empty(
+            pkv.paged_attention_prefill_workspace_size(b.num_seqs, T, b.num_heads, b.num_kv_heads),
+            dtype=torch.uint8, device=device)
         self.flops = prefill_flops(b.query_lens, b.context_lens, b.num_heads, b.head_dim)
 
     def step(self, q, k, v, out, status, ev=None, stream=None):
@@ -1301,7 +1352,7 @@ def run_reference(args, rank, world, local_rank):
     if args.workload == SWAP_WORKLOAD:
         return run_reference_swap(args, world)
     kv8 = args.kv == "fp8"
-    w = Workload(args.workload, 2, seed=1000, device=device, kv8=kv8, beams=args.beams)
+    w = Workload(args.workload, 2, seed=1000, device=device, kv8=kv8, beams=args.beams, native=False)
     bm = w.new_manager()
     ids = w.seq_ids
     bm.append_slots(ids)
@@ -1337,7 +1388,7 @@ def run_reference(args, rank, world, local_rank):
 
 
 def run_reference_prefill(args, world, device):
-    pw = PrefillWorkload(args.workload, 1, seed=2000, device=device)
+    pw = PrefillWorkload(args.workload, 1, seed=2000, device=device, native=False)
     rng = wl.rng_for(80)
     per_step = max(0.05, args.ref_budget / (args.warmup + args.steps))
     for _ in range(args.warmup):

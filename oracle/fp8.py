@@ -112,12 +112,6 @@ def reshape_and_cache_fp8(key_bits, value_bits, key_cache_codes, value_cache_cod
     return kc, vc
 
 
-def dequantize_pool(codes, scales):
-    """float64 values of a quantised pool [NB, Hkv, bs, D] with per-kv-head scales."""
-    vals = e4m3_to_f64(codes)
-    return vals * np.asarray(scales, np.float64)[None, :, None, None]
-
-
 def paged_decode_fp8(query_bits, key_cache_codes, value_cache_codes, k_scale, v_scale, block_tables, context_lens,
                      scale):
     """Decode attention over the dequantised pool: float64 [B, Hq, D]."""

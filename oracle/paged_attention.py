@@ -77,15 +77,6 @@ def paged_decode(query_bits, key_cache_bits, value_cache_bits, block_tables, con
     return out
 
 
-def paged_decode_rows(query_bits, key_cache_bits, value_cache_bits, block_tables, context_lens, scale, seqs):
-    """The same definition restricted to the listed sequences: float64 [len(seqs), Hq, D].
-
-    Used to check sampled rows of full-size workloads one sequence at a time."""
-    seqs = list(seqs)
-    return paged_decode(query_bits[seqs], key_cache_bits, value_cache_bits,
-                        np.asarray(block_tables)[seqs], np.asarray(context_lens)[seqs], scale)
-
-
 def contiguous_decode(query_bits, keys_bits, values_bits, context_lens, scale):
     """Attention over the traditional contiguous layout (vLLM 初探 §1.4: one
     [heads, seq_len, head_dim] slab per request, pre-reserved to a maximum length).
@@ -108,7 +99,3 @@ def contiguous_decode(query_bits, keys_bits, values_bits, context_lens, scale):
             out[s, h] = attend(q_all[s, h], keys, values, scale64)
     return out
 
-
-def kv_bytes(context_lens, num_kv_heads: int, head_dim: int) -> int:
-    """Algorithmic K+V bytes one decode call must read: each valid (token, kv head) once, bf16."""
-    return int(np.asarray(context_lens, dtype=np.int64).sum()) * num_kv_heads * head_dim * 2 * 2

@@ -4,6 +4,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -167,7 +168,7 @@ def test_bench_prefix_batch_shares_the_prompt_blocks(pkv):
     nb = int(np.ceil(1.2 * np.sum(-(-lens // bs))))
     order = wl.rng_for(7).permutation(nb).astype(np.int32)
     mb = int(np.max(-(-lens // bs)))
-    bm = bench.build_manager(pkv, nb, bs, order, lens, shared, mb)
+    bm = bench.build_manager(pkv.BlockManager, nb, bs, order, lens, shared, mb)
     tables, got = bm.export_tables(range(B), mb)
     assert (got == lens).all()
     assert (tables[:, :shared] == tables[0, :shared]).all()
@@ -182,7 +183,7 @@ def test_bench_prefix_batch_shares_the_prompt_blocks(pkv):
     assert bench.decode_bytes(lens, b.num_heads, b.num_kv_heads, b.head_dim, bs)[0] - u == \
         (B - 1) * wl.PREFIX_TOKENS * per_token
     # every other workload stays unshared
-    bm2 = bench.build_manager(pkv, nb, bs, order, lens[:4], 0, mb)
+    bm2 = bench.build_manager(pkv.BlockManager, nb, bs, order, lens[:4], 0, mb)
     t2, _ = bm2.export_tables(range(4), mb)
     assert bench.unique_kv_bytes(t2, lens[:4], 8, 128, bs) == bench.decode_bytes(lens[:4], 32, 8, 128, bs)[0]
     bm.close()
@@ -223,7 +224,7 @@ def test_bench_beam_batch_matches_the_allocator_model(pkv):
     nb = 200
     order = rng.permutation(nb).astype(np.int32)
     mb = 16
-    bm = bench.build_manager(pkv, nb, bs, order, lens, shared, mb, beams)
+    bm = bench.build_manager(pkv.BlockManager, nb, bs, order, lens, shared, mb, beams)
     ids = bench.beam_ids(parents, beams)
     model = BlockManagerModel(nb, bs, initial_order=order)
     model.add_seq(0, int(lens[0]))
@@ -282,7 +283,7 @@ def test_pool_usage_shows_what_sharing_saves(pkv):
     lens = b.context_lens.astype(np.int64)
     nb = int(np.ceil(1.2 * np.sum(-(-lens // bs))))
     order = wl.rng_for(7).permutation(nb).astype(np.int32)
-    bm = bench.build_manager(pkv, nb, bs, order, lens, wl.PREFIX_TOKENS // bs, int(np.max(-(-lens // bs))))
+    bm = bench.build_manager(pkv.BlockManager, nb, bs, order, lens, wl.PREFIX_TOKENS // bs, int(np.max(-(-lens // bs))))
     u = bench.pool_usage(nb, bm.num_free(), lens, bs)
     ref = int(np.sum(-(-lens // bs)))
     assert u["referenced_by_tables"] == ref and u["used"] == ref - (B - 1) * (wl.PREFIX_TOKENS // bs)
@@ -574,11 +575,14 @@ def test_run_swap_host_logic_with_stand_ins(pkv, monkeypatch):
     assert res["config"]["block_bytes"] == block and res["config"]["bytes_per_step"] == 4 * bench.SWAP_PAIRS * block
 
 
-def test_reference_arm_with_stand_ins(pkv, monkeypatch):
+def test_reference_arm_with_stand_ins(monkeypatch):
     """The reference arm (the oracle timed on the host) on the tiny batch, its device
-    stood in by the CPU: the JSON line with impl, cpu_baseline and a zero-copy e2e."""
+    stood in by the CPU: the JSON line with impl, cpu_baseline and a zero-copy e2e.
+    The library is made unimportable for the call: the arm depends on nothing it ships."""
     import json
+    import sys
     import types
+    monkeypatch.setitem(sys.modules, "paged_kv_cache_423_b200", None)
     monkeypatch.setattr(torch.cuda, "is_available", lambda: True)
     monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
     monkeypatch.setattr(bench, "bench_device", lambda local_rank: torch.device("cpu"))
@@ -590,3 +594,34 @@ def test_reference_arm_with_stand_ins(pkv, monkeypatch):
     assert res["cpu_baseline"]["kind"] == "oracle" and res["cpu_baseline"]["value"] == res["value"]
     assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["d2h_bytes_per_step"] == 0
     assert res["config"]["workload"] == "tiny"
+
+
+@pytest.mark.parametrize("workload,beams", [("prefix_beams", 1), ("prefix_beams", 4), ("llama7b", 1)])
+def test_reference_arm_tables_equal_the_native_ones(pkv, workload, beams):
+    """The reference arm builds its batch with the allocator's reference model; the same
+    operations on the C++ allocator give the same tables, lengths, slots and copy pairs."""
+    w = bench.Workload(workload, 2, seed=1000, device=torch.device("cpu"), beams=beams, native=False)
+    assert w.pkv is None
+    native = bench.build_manager(pkv.BlockManager, w.NB, w.bs, w.free_order, w.parent_lens0 - 1, w.shared_blocks,
+                                 w.max_blocks, w.beams)
+    model = w.new_manager()
+    for _ in range(2):
+        a, b = native.append_slots(w.seq_ids), model.append_slots(w.seq_ids)
+        assert a[0].tolist() == b[0].tolist() and a[1].tolist() == b[1].tolist()
+        ta, la = native.export_tables(w.seq_ids, w.max_blocks)
+        tb, lb = model.export_tables(w.seq_ids, w.max_blocks)
+        assert ta.dtype == tb.dtype and ta.tolist() == tb.tolist() and la.tolist() == lb.tolist()
+    assert native.num_free() == model.num_free()
+    native.close()
+
+
+def test_reference_prefill_batch_without_the_library(pkv, monkeypatch):
+    """The prefill reference leg's batch from the allocator's reference model equals the
+    native one (slots, tables, lengths), with the library unimportable while it is built."""
+    import sys
+    native = bench.PrefillWorkload("chunked_prefill_13b", 1, seed=2000, device=torch.device("cpu"))
+    monkeypatch.setitem(sys.modules, "paged_kv_cache_423_b200", None)
+    ref = bench.PrefillWorkload("chunked_prefill_13b", 1, seed=2000, device=torch.device("cpu"), native=False)
+    assert ref.pkv is None and ref.ws is None
+    for k in ("slots", "tables", "lens", "qstart"):
+        assert torch.equal(getattr(native, k), getattr(ref, k)), k

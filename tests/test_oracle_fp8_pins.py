@@ -70,7 +70,17 @@ def pin_quantize_division(mod):
     return True
 
 
-CODEC_PINS = [pin_code_values, pin_rounding_every_bf16, pin_hand_cases, pin_quantize_division]
+def pin_table_lookup_every_code(mod):
+    """The vectorised lookup e4m3_to_f64 over all 256 codes, laid out as a [2, 8, 16] block, against
+    torch's float8_e4m3fn -> float64 conversion (NaN codes stay NaN, the shape is kept)."""
+    codes = np.arange(256, dtype=np.uint8).reshape(2, 8, 16)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = mod.e4m3_to_f64(codes)
+    nan = np.isnan(ref)
+    return got.shape == ref.shape and np.array_equal(nan, np.isnan(got)) and np.array_equal(ref[~nan], got[~nan])
+
+
+CODEC_PINS = [pin_code_values, pin_rounding_every_bf16, pin_hand_cases, pin_quantize_division, pin_table_lookup_every_code]
 
 
 @pytest.mark.parametrize("pin", CODEC_PINS, ids=lambda p: p.__name__)
@@ -178,6 +188,8 @@ MUTATIONS = {
     "bias_8": ("return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)", "return sign * (1.0 + m / 8.0) * 2.0 ** (e - 8)"),
     "k_scale_for_values": ("* float(np.float32(v_scale[kvh]))", "* float(np.float32(k_scale[kvh]))"),
     "scale_by_query_head": ("* float(np.float32(k_scale[kvh]))", "* float(np.float32(k_scale[h % len(k_scale)]))"),
+    "lookup_drops_sign": ("return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]",
+                          "return E4M3_TABLE[np.asarray(codes, dtype=np.uint8) & 0x7F]"),
     "multiply_not_divide": ("(np.asarray(x_f32, np.float32) / np.float32(scale_f32))",
                             "(np.asarray(x_f32, np.float32) * np.float32(scale_f32))"),
 }

@@ -419,3 +419,60 @@ def test_pins_catch_planted_mistake(name):
         if not ok:
             caught.append(pin.__name__)
     assert caught, f"no pin catches mutation {name}"
+
+
+# ---------------------------------------------------------------------------
+# The bf16 widening every attention oracle starts from
+# ---------------------------------------------------------------------------
+
+def pin_bf16_widening_every_pattern(widen):
+    """All 65,536 bf16 bit patterns against torch's own bfloat16 -> float64 conversion
+    (bf16 is the upper half of a float32, so widening is exact); NaN patterns must stay
+    NaN, and the result keeps the input's shape."""
+    bits = np.arange(65536, dtype=np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    got = widen(bits.reshape(256, 256)).reshape(-1)
+    nan = np.isnan(ref)
+    return np.array_equal(nan, np.isnan(got)) and np.array_equal(ref[~nan], got[~nan])
+
+
+def pin_bf16_widening_hand_cases(widen):
+    """Worked by hand from the bf16 layout (1 sign, 8 exponent bits with bias 127, 7 mantissa bits)."""
+    cases = {0x3F80: 1.0, 0xBF80: -1.0, 0x4000: 2.0, 0x3FC0: 1.5, 0x4049: 3.140625, 0x0001: 2.0 ** -133,
+             0x7F7F: (2 - 2 ** -7) * 2.0 ** 127, 0x0000: 0.0, 0x7F80: math.inf, 0xFF80: -math.inf}
+    got = widen(np.array(list(cases), dtype=np.uint16))
+    return all(g == v for g, v in zip(got, cases.values()))
+
+
+WIDEN_PINS = [pin_bf16_widening_every_pattern, pin_bf16_widening_hand_cases]
+
+
+@pytest.mark.parametrize("pin", WIDEN_PINS, ids=lambda p: p.__name__)
+def test_bf16_widening_pin(pin):
+    assert pin(paged_attention.bf16_bits_to_f64)
+
+
+WIDEN_MUTATIONS = {
+    # the bits read as IEEE half precision instead of bfloat16
+    "read_as_float16": ("return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)",
+                        "return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)"),
+    "shift_by_15": ("astype(np.uint32) << 16)", "astype(np.uint32) << 15)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(WIDEN_MUTATIONS))
+def test_widening_pins_catch_planted_mistake(name):
+    old, new = WIDEN_MUTATIONS[name]
+    src = inspect.getsource(paged_attention)
+    assert old in src, name
+    ns = {}
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), ns)
+    caught = [p.__name__ for p in WIDEN_PINS if not _safe(p, ns["bf16_bits_to_f64"])]
+    assert caught, f"no pin catches mutation {name}"
+
+
+def _safe(pin, impl):
+    try:
+        return pin(impl)
+    except Exception:
+        return False

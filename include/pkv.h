@@ -190,7 +190,14 @@ PKV_API int pkv_paged_attention_decode(void* out, int out_dtype, const void* que
  *     is enqueued.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture starts.
+ *     before any stream capture starts.  With CUDA's lazy module loading (the
+ *     default) the array's PKV_STATIC_SCRATCH_BYTES are also taken from device
+ *     memory only then, so make the first call before handing the rest of device
+ *     memory to another allocator.
+ *   - The address is kept for the life of the process: after cudaDeviceReset on a
+ *     device this entry point must not be used on that device again.
+ *   - Sizes the workspace variant refuses (an unsupported block_size or head_dim,
+ *     and so on) give the same return code as pkv_paged_attention_decode.
  *   - All calls on one device share the array.  Calls whose kernels overlap on the
  *     GPU (for example on two streams without ordering between them) race and give
  *     wrong results; order them on one stream or use the workspace variant.

@@ -27,10 +27,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
 #include <type_traits>
 
 #include "decode_common.cuh"
+#include "launch_setup.cuh"
 #include "pkv_internal.h"
 
 // Warps per CTA, ring stages per warp, and dynamic (counter) instead of static
@@ -747,18 +747,20 @@ static int launch_simt(const DecodeArgs& a, cudaStream_t stream) {
   constexpr int stages = KV8 ? kSimtStages8 : kSimtStages;
   auto kernel = decode_simt_kernel<D, OUT_F32, kSimtWarps, stages, KV8>;
   const size_t smem = sizeof(WarpRing<D, stages, KV8>) * kSimtWarps;
-  static std::once_flag once;
-  static int blocks_per_sm = 0;
-  static cudaError_t setup_err = cudaSuccess;
-  std::call_once(once, [&] {
-    setup_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (setup_err == cudaSuccess)
-      setup_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kernel, kSimtWarps * 32, smem);
-  });
-  if (setup_err != cudaSuccess)
-    return set_error(PKV_ERR_CUDA, "decode (simt) setup: %s", cudaGetErrorString(setup_err));
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
+  static PerDevice<int> setup;  // blocks per SM, found once on each device
+  int dev = 0, sms = 0, blocks_per_sm = 0;
+  cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (simt): cudaGetDevice: %s", cudaGetErrorString(de));
+  const int st = setup.get(
+      dev,
+      [&](int& bps) {
+        cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (r == cudaSuccess) r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kernel, kSimtWarps * 32, smem);
+        return static_cast<int>(r);
+      },
+      &blocks_per_sm, static_cast<int>(cudaErrorInvalidDevice));
+  if (st != 0)
+    return set_error(PKV_ERR_CUDA, "decode (simt) setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::max(1, sms * std::max(1, blocks_per_sm));
   kernel<<<grid, kSimtWarps * 32, smem, stream>>>(a);
@@ -822,13 +824,12 @@ extern "C" size_t pkv_paged_attention_workspace_size(int num_seqs, int num_heads
 // Shared by the bf16 and the 8-bit entry points; `k_scale` != null selects the
 // 8-bit (e4m3) pool (head_dim 128), read by the CUDA-core kernel or, for grouped
 // query heads, by the tensor-core kernel that widens each tile to f16.
-static int decode_impl(void* out, int out_dtype, const void* query, const void* key_cache, const void* value_cache,
-                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
-                       int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
-                       int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
-                       int partition_tokens, int path, void* workspace, size_t workspace_bytes, int32_t* status,
-                       pkv_stream_t stream) {
-  const bool kv8 = k_scale != nullptr;
+namespace pkv {
+// The checks of a decode call that need no pointer: sizes, output type, path and partition.
+// Returns PKV_OK (and the partition to use in *partition_out) or the call's error code.
+int decode_check_sizes(int out_dtype, bool kv8, int max_blocks_per_seq, int max_context_len, int num_seqs,
+                       int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                       int partition_tokens, int path, int* partition_out) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: bad sizes");
@@ -863,6 +864,24 @@ static int decode_impl(void* out, int out_dtype, const void* query, const void* 
                      "(partition_tokens %d, block_size %d)", partition_tokens, block_size);
   if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(65535) * partition)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: max_context_len too large for the split");
+  *partition_out = partition;
+  return PKV_OK;
+}
+}  // namespace pkv
+
+static int decode_impl(void* out, int out_dtype, const void* query, const void* key_cache, const void* value_cache,
+                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                       int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
+                       int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                       int partition_tokens, int path, void* workspace, size_t workspace_bytes, int32_t* status,
+                       pkv_stream_t stream) {
+  const bool kv8 = k_scale != nullptr;
+  int partition = 0;
+  const int rc_sizes = decode_check_sizes(out_dtype, kv8, max_blocks_per_seq, max_context_len, num_seqs, num_heads,
+                                          num_kv_heads, head_dim, block_size, num_blocks, partition_tokens, path, &partition);
+  if (rc_sizes != PKV_OK) return rc_sizes;
+  const int group = num_heads / num_kv_heads;
+  const bool use_tensor = path == PKV_PATH_TENSOR || (path == PKV_PATH_AUTO && tensor_path_supports(group, head_dim));
   if (num_seqs == 0) return PKV_OK;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !workspace ||
       (kv8 && !v_scale))

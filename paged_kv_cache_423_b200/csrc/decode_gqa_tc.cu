@@ -31,9 +31,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "decode_common.cuh"
+#include "launch_setup.cuh"
 #include "pkv_internal.h"
 #include "tcgen05_common.cuh"
 
@@ -653,12 +653,10 @@ template <int N, bool OUT_F32>
 static int launch(const Args& args, cudaStream_t stream) {
   auto kernel = decode_gqa_tc_kernel<kStages, N, OUT_F32>;
   const int smem = Layout<kStages, N>::alloc;
-  static std::once_flag once;
-  static cudaError_t setup = cudaSuccess;
-  std::call_once(once, [&] { setup = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
-  if (setup != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) setup: %s", cudaGetErrorString(setup));
+  static PerDevice<int> setup;
   int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
+  const int st = set_smem_limit_once(setup, kernel, smem, &dev);
+  if (st != 0) return set_error(PKV_ERR_CUDA, "decode (tensor) setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   kernel<<<std::max(1, sms), kThreads, smem, stream>>>(args);
   cudaError_t e = cudaGetLastError();

@@ -32,9 +32,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "decode_common.cuh"
+#include "launch_setup.cuh"
 #include "pkv_internal.h"
 #include "tcgen05_common.cuh"
 
@@ -796,13 +796,11 @@ static int encode_map(CUtensorMap* map, const void* base, uint64_t rows, bool e4
 template <bool OUT_F32, int NH>
 static int launch(const Args& args, cudaStream_t stream) {
   auto kernel = decode_gqa_tc_fp8_kernel<OUT_F32, NH>;
-  static std::once_flag once;
-  static cudaError_t setup = cudaSuccess;
-  std::call_once(once,
-                 [&] { setup = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes); });
-  if (setup != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) setup: %s", cudaGetErrorString(setup));
+  static PerDevice<int> setup;
   int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
+  const int st = set_smem_limit_once(setup, kernel, kSmemBytes, &dev);
+  if (st != 0)
+    return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   kernel<<<std::max(1, sms), kThreads, kSmemBytes, stream>>>(args);
   cudaError_t e = cudaGetLastError();

@@ -14,7 +14,12 @@
 // stand-in, not a device address): the device address is looked up once per device
 // with cudaGetSymbolAddress, with that device current, on the first call made
 // there.  That first call on each device should therefore happen before any stream
-// capture begins.  All calls on a device share the one array and it keeps the
+// capture begins.  With CUDA's lazy module loading (the default) the array itself is
+// also placed in device memory only then, so an application that hands all device
+// memory to its own allocator should make the first call before it does.  The
+// looked-up address is kept for the life of the process: after a device reset
+// (cudaDeviceReset) it is stale, so this entry point must not be used on that device
+// again.  All calls on a device share the one array and it keeps the
 // previous call's contents; the plan kernel re-zeroes everything that must start
 // at zero on every call, but two calls whose kernels overlap on the GPU (for
 // example on two streams) race on the array and corrupt each other's results.
@@ -62,10 +67,16 @@ extern "C" int pkv_paged_attention_decode_static(void* out, int out_dtype, const
                                                  pkv_stream_t stream) {
   using namespace pkv;
   clear_error();
+  // Sizes the workspace variant refuses give its return code, before the scratch is looked up.
+  int partition = 0;
+  const int rc_sizes = decode_check_sizes(out_dtype, false, max_blocks_per_seq, max_context_len, num_seqs, num_heads,
+                                          num_kv_heads, head_dim, block_size, num_blocks, partition_tokens, path,
+                                          &partition);
+  if (rc_sizes != PKV_OK) return rc_sizes;
+  if (num_seqs == 0) return PKV_OK;
   const size_t need = pkv_paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                                          max_context_len, partition_tokens);
-  if (need == 0 && num_seqs != 0)
-    return set_error(PKV_ERR_INVALID, "paged_attention_decode_static: bad sizes");
+  if (need == 0) return set_error(PKV_ERR_INVALID, "paged_attention_decode_static: bad sizes");
   if (need > static_cast<size_t>(PKV_STATIC_SCRATCH_BYTES))
     return set_error(PKV_ERR_INVALID,
                      "paged_attention_decode_static: these sizes need %zu bytes of scratch, more than the %zu-byte "

@@ -39,9 +39,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "decode_common.cuh"
+#include "launch_setup.cuh"
 #include "pkv_internal.h"
 #include "tcgen05_common.cuh"
 
@@ -743,11 +743,10 @@ static int encode_q_map(CUtensorMap* map, const void* base, int total_q, int num
 template <bool OUT_F32>
 static int launch_main(const Args& args, int grid, cudaStream_t stream) {
   auto kernel = prefill_tc_kernel<OUT_F32>;
-  static std::once_flag once;
-  static cudaError_t setup = cudaSuccess;
-  std::call_once(once,
-                 [&] { setup = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes); });
-  if (setup != cudaSuccess) return set_error(PKV_ERR_CUDA, "prefill setup: %s", cudaGetErrorString(setup));
+  static PerDevice<int> setup;
+  int dev = 0;
+  const int st = set_smem_limit_once(setup, kernel, kSmemBytes, &dev);
+  if (st != 0) return set_error(PKV_ERR_CUDA, "prefill setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   kernel<<<grid, kThreads, kSmemBytes, stream>>>(args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));

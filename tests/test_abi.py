@@ -416,3 +416,21 @@ def test_one_stage_ring_variant_builds_and_loads_through_the_override(pkv):
     assert r.returncode == 0, r.stderr
     path, version = r.stdout.split()
     assert path == lib1 and int(version) == pkv.library().pkv_version()
+
+
+def test_launch_setup_runs_once_per_device(tmp_path):
+    """Kernel attributes belong to each device's context, so the launchers set them up once
+    per device (csrc/per_device.h).  The bookkeeping is plain C++: compiled with g++ and run
+    here, it must set each device up on first use only, keep a value per device, retry a
+    failed set-up, refuse out-of-range indices, and run one set-up per device under 16 threads."""
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("g++ not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = tmp_path / "per_device_test"
+    subprocess.run([gxx, "-std=c++17", "-O1", "-pthread", "-I", os.path.join(root, "paged_kv_cache_423_b200", "csrc"),
+                    os.path.join(root, "tests", "native", "per_device_test.cpp"), "-o", str(exe)], check=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", res.stdout + res.stderr

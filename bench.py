@@ -33,6 +33,8 @@ Other rows, same JSON line (`--workload` / `--kv`):
                            128 sequences sharing one 1024-token prompt (the prompt's blocks
                            in every table); with --beams N each is first forked into N beams,
                            so the first step copies every shared partial last block but one.
+                           The decode is the shared-prefix decode (the allocator's tables
+                           planned on the host once per step; --shared off for the plain one).
   --workload swap_llama13b one step = 256 13B-shaped blocks swapped out to pinned host
                            memory and 256 swapped in (K and V); GB/s against the
                            pinned-memory copy bandwidth measured in the same run.
@@ -94,6 +96,8 @@ KERNEL_SOURCES = {
     "decode_gqa_tc": ["decode_gqa_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
     "decode_gqa_tc_fp8": ["decode_gqa_tc_fp8.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
     "prefill": ["prefill_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
+    "shared": ["shared_decode.cu", "shared_plan.cpp", "prefill_tc.cu", "decode_gqa_tc.cu", "decode.cu",
+               "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
 }
 
 
@@ -191,8 +195,10 @@ def rank_info():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples the SM clock and the clock-event reasons through NVML every ~1 ms
-    while the timed region runs (a thread; NVML reads only, nothing is set)."""
+    """Samples the SM clock and the clock-event reasons through NVML back to back (a
+    pause of 0.2 ms between samples) while the timed region runs (a thread; NVML reads
+    only, nothing is set).  Entering waits for the first sample, so a timed region of a
+    few milliseconds still gets several."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
@@ -236,10 +242,13 @@ class ClockSampler:
                 except Exception as e:
                     self.err = str(e)
                     return
-                time.sleep(0.001)
+                time.sleep(0.0002)
 
         self._thread = threading.Thread(target=poll, daemon=True)
         self._thread.start()
+        t0 = time.perf_counter()
+        while not self.samples and self.err is None and time.perf_counter() - t0 < 1.0:
+            time.sleep(0.0001)
         return self
 
     def __exit__(self, *exc):
@@ -392,8 +401,13 @@ class Workload:
     def copy(self, pairs, status):
         self.pkv.copy_blocks([self.key_cache], [self.value_cache], pairs, status=status)
 
-    def decode(self, out, q, tables, lens, max_len, ws, path, status):
-        if self.kv8:
+    def decode(self, out, q, tables, lens, max_len, ws, path, status, shared=None):
+        """shared = (device plan, its info, the shared-prefix workspace) for the shared-prefix decode."""
+        if shared is not None:
+            plan, info, sws = shared
+            self.pkv.paged_attention_decode_shared(out, q, self.key_cache, self.value_cache, tables, lens, self.scale,
+                                                   plan, info, sws, status=status)
+        elif self.kv8:
             self.pkv.paged_attention_decode_fp8(out, q, self.key_cache, self.value_cache, self.k_scale, self.v_scale,
                                                 tables, lens, max_len, self.scale, ws, path=path, status=status)
         else:
@@ -409,6 +423,17 @@ class Workload:
         q = wl.bf16_normal(self.rng, (self.B, self.Hq, self.D))
         k, v = wl.new_tokens(self.rng, self.B, self.Hkv, self.D)
         return q, k, v
+
+
+def shared_decode_applies(args, w) -> bool:
+    """The shared-prefix decode: on request, or by default for the shared-prompt workload;
+    it needs a bf16 pool and the tensor-core decode's head shapes."""
+    g = w.Hq // w.Hkv
+    ok = not w.kv8 and w.D == 128 and 2 <= g <= 16 and args.path != "simt"
+    choice = getattr(args, "shared", "auto")
+    if choice == "on" and not ok:
+        raise SystemExit("--shared on needs a bf16 pool, head_dim 128 and 2 <= num_heads / num_kv_heads <= 16")
+    return ok and (choice == "on" or (choice == "auto" and w.shared_blocks > 0))
 
 
 def beam_ids(parents: int, beams: int) -> list:
@@ -498,13 +523,19 @@ def run_ours(args, rank, world, local_rank):
     # the batch.  Timed step i replays state i % n_states, so the batch keeps its
     # configured length mix however many steps are timed (a replayed state rewrites
     # its own token into its own slot, then decodes the same contexts).
+    g = w.Hq // w.Hkv
+    use_shared = shared_decode_applies(args, w)
     bm = w.new_manager()
     states = []
     for _ in range(n_states):
         slots, pairs = bm.append_slots(seq_ids)
         tables, lens = bm.export_tables(seq_ids, w.max_blocks)
         q, k, v = w.host_step_inputs()
-        states.append(dict(q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
+        plan = None
+        if use_shared:
+            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs)
+            plan = (torch.from_numpy(plan_h).to(device), info)
+        states.append(dict(plan=plan, q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
                            slots=torch.from_numpy(slots).to(device), pairs=torch.from_numpy(pairs).to(device),
                            n_pairs=len(pairs), tables=torch.from_numpy(tables).to(device),
                            lens=torch.from_numpy(lens).to(device), max_len=int(lens.max()), host_lens=lens,
@@ -518,6 +549,10 @@ def run_ours(args, rank, world, local_rank):
     status = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
     path = {"auto": 0, "simt": 1, "tensor": 2}[args.path]
+    sws = None
+    if use_shared:
+        sws = torch.empty(max(pkv.paged_attention_decode_shared_workspace_size(st["plan"][1], w.Hq, w.Hkv, w.D)
+                              for st in states), dtype=torch.uint8, device=device)
 
     def step(i, ev=None):
         st = states[i % n_states]
@@ -526,7 +561,8 @@ def run_ours(args, rank, world, local_rank):
         w.write(st["k"], st["v"], st["slots"], status)
         if ev is not None:
             ev[0].record(stream)
-        w.decode(out, st["q"], st["tables"], st["lens"], max_len_all, ws, path, status)
+        w.decode(out, st["q"], st["tables"], st["lens"], max_len_all, ws, path, status,
+                 shared=(st["plan"][0], st["plan"][1], sws) if use_shared else None)
         if ev is not None:
             ev[1].record(stream)
 
@@ -535,7 +571,6 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     launches = 0
     kv_total = bytes_total = unique_total = unique_kv_total = 0
-    g = w.Hq // w.Hkv
     uses_tensor = path == 2 or (path == 0 and w.D == 128 and 2 <= g <= 16)
     # write, plan, decode (+ copy_blocks when a fork copied blocks) (+ the merge of a split context)
     merge = 1 if uses_tensor and max_len_all > split_tokens(w.B, w.Hkv, w.bs, max_len_all, True) else 0
@@ -546,7 +581,10 @@ def run_ours(args, rank, world, local_rank):
         bytes_total += alg
         unique_total += alg - kv + st["unique_kv"]
         unique_kv_total += st["unique_kv"]
-        launches += 3 + (1 if st["n_pairs"] else 0) + merge
+        if use_shared:  # write, setup, shared phase (when there are segments), plan, decode, merge
+            launches += 5 + (1 if st["plan"][1].num_entries else 0) + (1 if st["n_pairs"] else 0)
+        else:
+            launches += 3 + (1 if st["n_pairs"] else 0) + merge
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -580,7 +618,7 @@ def run_ours(args, rank, world, local_rank):
     seq_steps = world * w.B * args.steps / (ms_max * 1e-3)
 
     # ---- e2e through the public API with host buffers
-    e2e = run_e2e(args, w, pkv, device, path, ws, out, status, max_len_all) if not args.no_e2e else None
+    e2e = run_e2e(args, w, pkv, device, path, ws, out, status, max_len_all, sws) if not args.no_e2e else None
 
     peak, peak_kind = measured_hbm_gbs()
     # the roofline counts every physical block once (a shared prefix is one copy of bytes);
@@ -595,6 +633,7 @@ def run_ours(args, rank, world, local_rank):
                    "block_size": w.bs, "lengths": LENGTH_MIX[w.name], "mean_context": float(np.mean(w.lens0)),
                    "num_blocks": w.NB, "pool": pool,
                    "kv_bytes_per_step": kv_total // args.steps, "path": args.path,
+                   "decode": "shared-prefix" if use_shared else "plain",
                    "l2": ("L2 flushed before each timed step (a 252 MB write, outside the step's events): the"
                           " distinct KV per step is under 4x the 126 MB L2; e2e steps are pipelined, not flushed"
                           if flush_l2 else "inputs larger than L2 (distinct KV per step >= 4x the 126 MB L2)"),
@@ -606,12 +645,16 @@ def run_ours(args, rank, world, local_rank):
         "pct_hbm_peak": round(100 * value * (unique_kv_total / kv_total if kv_total else 1.0) / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4),
-                     "traffic": recorded_traffic(w.label,
+                     "traffic": recorded_traffic(w.label + ("+shared" if use_shared else ""),
+                                                 "shared" if use_shared else
                                                  ("decode_gqa_tc_fp8" if kv8 else "decode_gqa_tc") if uses_tensor
                                                  else "decode_simt", w.layout),
                      "algorithmic_bytes_per_launch": unique_total // args.steps,
                      "logical_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
-                     "kernel": ("paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"
+                     "kernel": ("paged_attention_decode_shared: setup + shared phase (tcgen05 prefill kernel, every"
+                                " key visible, partials) + plan + tcgen05 decode of the private remainders + merge;"
+                                " traffic = the DRAM bytes of all of them" if use_shared
+                                else "paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"
                                 " + split merge" if kv8 and uses_tensor
                                 else "paged_attention_decode_fp8: plan + CUDA-core streaming kernel (e4m3 tiles)" if kv8
                                 else "paged_attention_decode: plan + tcgen05 kernel + split merge" if uses_tensor
@@ -638,14 +681,15 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
-def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
+def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None):
     """End to end through the public API with host buffers, pipelined as a server
     would run it: per step the C++ allocator produces slots and tables on the host;
     q, new K, new V (one pinned buffer per step) and the allocator output (a small
     pinned buffer, double-buffered) go host->device on a copy stream while the
     previous step's kernels run; the step's output comes back to pinned memory on a
     stream of its own (beside the next step's kernels) and is read on the host one
-    step later."""
+    step later.  With the shared-prefix decode (`sws` its workspace) the host also plans
+    each step from the allocator's tables, and the plan travels with them."""
     import torch
     ke = max(1, min(args.steps, args.e2e_steps))
     n = args.warmup + ke
@@ -666,7 +710,16 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
     o_slots, o_pairs = 0, al(8 * w.B)
     o_tab = o_pairs + al(16 * w.B)
     o_lens = o_tab + al(4 * w.B * w.max_blocks)
-    meta_bytes = o_lens + al(4 * w.B)
+    o_plan = o_lens + al(4 * w.B)
+    plan_cap = 0
+    if sws is not None:  # room for the largest plan: sized on a dry run of the allocator
+        probe = w.new_manager()
+        for _ in range(n):
+            probe.append_slots(seq_ids)
+            t_, l_ = probe.export_tables(seq_ids, w.max_blocks)
+            plan_cap = max(plan_cap, int(pkv.shared_plan(t_, l_, w.Hq, w.Hkv, w.bs)[1].bytes))
+        probe.close()
+    meta_bytes = o_plan + al(plan_cap)
     host_meta = [torch.empty(meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     dev_qkv = [torch.empty(nq + 2 * nk, dtype=torch.int16, device=device) for _ in range(2)]
     dev_meta = [torch.empty(meta_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
@@ -689,6 +742,13 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
         hm[o_lens:o_lens + lens.nbytes] = lens.view(np.uint8)
         if len(pairs):
             hm[o_pairs:o_pairs + pairs.nbytes] = pairs.reshape(-1).view(np.uint8)
+        plan_bytes = 0
+        if sws is not None:
+            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs)
+            plan_bytes = plan_h.nbytes
+            if plan_bytes > plan_cap:
+                raise RuntimeError("e2e: a step's shared-prefix plan outgrew the pinned buffer")
+            hm[o_plan:o_plan + plan_bytes] = plan_h
         with torch.cuda.stream(copy):
             if i >= 2:
                 copy.wait_event(comp_done[i - 2])  # device buffers b are free again
@@ -709,7 +769,8 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
         w.write(dk, dv, d_slots, status)
         if i >= 2:
             compute.wait_event(d2h_done[i - 2])    # outs[b] has been copied out
-        w.decode(outs[b], dq, d_tables, d_lens, max_len_bound, ws, path, status)
+        shared = (dm[o_plan:o_plan + plan_cap], info, sws) if sws is not None else None
+        w.decode(outs[b], dq, d_tables, d_lens, max_len_bound, ws, path, status, shared=shared)
         comp_done[i].record(compute)
         with torch.cuda.stream(d2h):
             d2h.wait_event(comp_done[i])
@@ -719,7 +780,8 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound):
             d2h_done[i - 1].synchronize()
             stats["checksum"] += float(out_host[(i - 1) % 2][0, 0, 0])
         if i >= args.warmup:
-            stats["h2d"] += host_qkv[i].numel() * 2 + slots.nbytes + pairs.nbytes + tables.nbytes + lens.nbytes
+            stats["h2d"] += (host_qkv[i].numel() * 2 + slots.nbytes + pairs.nbytes + tables.nbytes + lens.nbytes
+                             + plan_bytes)
             stats["d2h"] += out_host[b].numel() * 2
             stats["kv"] += int(np.asarray(lens, np.int64).sum()) * w.Hkv * w.D * 2 * (1 if w.kv8 else 2)
 
@@ -1451,6 +1513,9 @@ def main():
     ap.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--beams", type=int, default=1,
                     help="prefix_beams only: fork every sequence into this many beams before the first step")
+    ap.add_argument("--shared", choices=["auto", "on", "off"], default="auto",
+                    help="shared-prefix decode (blocks that adjacent rows share read once per kv head): auto = on "
+                         "for the shared-prompt workload over a bf16 pool")
     ap.add_argument("--trace", action="store_true",
                     help="run the long-context continuous-batching trace step by step (the fifth workload)")
     ap.add_argument("--no-e2e", action="store_true")

@@ -303,6 +303,87 @@ PKV_API int pkv_paged_attention_prefill(void* out, int out_dtype, const void* qu
                                         size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
 
 /*
+ * Shared-prefix decode — decode attention that reads each block shared by several
+ * tables once per kv head instead of once per table.  Outcome School explainer,
+ * "内存共享": requests with a common system prompt, and the beams of one request, map
+ * the same physical blocks; vLLM 初探 §1.4 counts the memory this saves (30-50% with
+ * shared system prompts).  The result is that of pkv_paged_attention_decode.
+ *
+ * Softmax attention over a sequence's tokens splits exactly over any partition of
+ * those tokens: with each part's unnormalised sum o_i, its running maximum m_i and its
+ * weight sum l_i (base-2 scores), out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i,
+ * M = max_i m_i.  The plan cuts every row's tokens into a chain of shared segments
+ * (runs of whole blocks that a range of ADJACENT rows holds in common, at the same
+ * positions of their tables) followed by the row's private remainder.  Run:
+ *   1. shared phase: each segment is a dense contraction of all its rows' query heads
+ *      against the segment's keys (the tensor-core prefill kernel with every key
+ *      visible and unnormalised partial results), cut into key chunks for parallelism;
+ *   2. private phase: every row's remainder through the tensor-core decode (grouped
+ *      heads, head_dim 128), writing partial results only;
+ *   3. merge: per (row, head), the formula above over the row's shared partials and
+ *      its private partitions.
+ *
+ * pkv_shared_plan (host only, nothing touches the GPU) builds the plan from host
+ * copies of the tables and lengths.  Rows share a segment only when they are adjacent
+ * in the batch (order the rows so that sharers sit together: a prompt's requests, a
+ * parent and its beams) and the segment's blocks are full for every one of them.
+ *   block_tables   host [num_seqs, max_blocks_per_seq] int32; context_lens host [num_seqs]
+ *                  (0 <= L <= max_blocks_per_seq * block_size, else PKV_ERR_INVALID)
+ *   min_rows       fewest rows a segment serves (>= 2)
+ *   key_chunk      tokens per part of a segment: a multiple of 128, or 0 = automatic
+ *                  (the largest of 2048 .. 128 that still gives about two work items per SM)
+ *   plan           host buffer of plan_bytes, or NULL to only fill `info` (info->bytes
+ *                  is then the size to provide); too small a buffer is PKV_ERR_INVALID
+ *   info           host, filled on success: counts and the byte offset of each section
+ * Copy the plan's first info->bytes bytes to device memory (16-byte aligned) for the run.
+ */
+typedef struct pkv_shared_plan_info {
+  int32_t num_seqs;          /* rows the plan was made for */
+  int32_t num_segments;      /* shared segments found */
+  int32_t num_parts;         /* segments cut into key chunks */
+  int32_t num_entries;       /* shared-phase work entries (pairs of 128-row query tiles of a part) */
+  int32_t num_partials;      /* (part, row) partial results of the shared phase */
+  int32_t max_suffix_len;    /* longest private remainder of a row, tokens */
+  int32_t key_chunk;         /* tokens per part */
+  int32_t group;             /* num_heads / num_kv_heads */
+  int32_t block_size;
+  int32_t max_blocks_per_seq;
+  int64_t shared_row_tokens; /* sum over rows of the tokens their segments serve */
+  int64_t shared_tokens;     /* sum over segments of their tokens (each read once per kv head) */
+  uint64_t off_entries;      /* int4[num_entries]: first row, 0, rows of tile A | rows of tile B << 8, part */
+  uint64_t off_parts;        /* int4[2 * num_parts]: (table row, first block, keys, first row),
+                                (rows, first partial, 0, 0) */
+  uint64_t off_suffix_lens;  /* int32[num_seqs]: tokens of each row's private remainder */
+  uint64_t off_block_offset; /* int32[num_seqs]: table index where the remainder starts */
+  uint64_t off_row_start;    /* int32[num_seqs + 1]: CSR of each row's shared partials */
+  uint64_t off_row_ids;      /* int32[num_partials] */
+  uint64_t bytes;            /* plan size */
+} pkv_shared_plan_info;
+
+PKV_API int pkv_shared_plan(const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                            int num_seqs, int num_heads, int num_kv_heads, int block_size, int min_rows,
+                            int key_chunk, void* plan, size_t plan_bytes, pkv_shared_plan_info* info);
+
+/*
+ * Run of a shared-prefix plan.  Arguments as for pkv_paged_attention_decode, plus
+ *   plan        device copy of the plan made for these tables and lengths (16-byte aligned)
+ *   info        host, the plan's info
+ *   workspace   device, pkv_paged_attention_decode_shared_workspace_size() bytes, 256-byte aligned
+ * bf16 pools only; head_dim 128; 2 <= num_heads / num_kv_heads <= 16 (the tensor-core
+ * decode) — else PKV_ERR_UNSUPPORTED.  block_tables and context_lens must be those the
+ * plan was made from (the private phase re-validates lengths and table entries).
+ */
+PKV_API size_t pkv_paged_attention_decode_shared_workspace_size(const pkv_shared_plan_info* info, int num_heads,
+                                                                int num_kv_heads, int head_dim);
+PKV_API int pkv_paged_attention_decode_shared(void* out, int out_dtype, const void* query, const void* key_cache,
+                                              const void* value_cache, const int32_t* block_tables,
+                                              int max_blocks_per_seq, const int32_t* context_lens,
+                                              int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                              int block_size, int num_blocks, float scale, const void* plan,
+                                              const pkv_shared_plan_info* info, void* workspace,
+                                              size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
+
+/*
  * Host block manager — free list + reference counts + per-sequence block tables.
  * Outcome School explainer, "vLLM的核心创新：PagedAttention" (a block only when needed,
  * any free block serves any request, finished requests return all blocks at once)

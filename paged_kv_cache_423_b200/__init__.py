@@ -23,6 +23,7 @@ __all__ = [
     "paged_attention_decode", "paged_attention_decode_static", "STATIC_SCRATCH_BYTES",
     "paged_attention_prefill_workspace_size", "paged_attention_prefill", "reshape_and_cache_fp8",
     "paged_attention_decode_fp8", "swap_blocks", "BlockManager", "stream_read",
+    "SharedPlanInfo", "shared_plan", "paged_attention_decode_shared_workspace_size", "paged_attention_decode_shared",
 ]
 
 PKV_OK = 0
@@ -114,6 +115,29 @@ _SIGNATURES = {
     "pkv_bm_seq_blocks": (c_int, [c_void_p, c_int64]),
     "pkv_bm_export_tables": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_int, c_void_p]),
 }
+
+
+class SharedPlanInfo(ctypes.Structure):
+    """pkv_shared_plan_info: counts and byte offsets of a shared-prefix plan."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("num_seqs", "num_segments", "num_parts", "num_entries", "num_partials",
+                                               "max_suffix_len", "key_chunk", "group", "block_size",
+                                               "max_blocks_per_seq")] + \
+               [("shared_row_tokens", ctypes.c_int64), ("shared_tokens", ctypes.c_int64)] + \
+               [(n, ctypes.c_uint64) for n in ("off_entries", "off_parts", "off_suffix_lens", "off_block_offset",
+                                                "off_row_start", "off_row_ids", "bytes")]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+_SIGNATURES["pkv_shared_plan"] = (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                          c_void_p, c_size_t, ctypes.POINTER(SharedPlanInfo)])
+_SIGNATURES["pkv_paged_attention_decode_shared_workspace_size"] = (c_size_t, [ctypes.POINTER(SharedPlanInfo), c_int,
+                                                                              c_int, c_int])
+_SIGNATURES["pkv_paged_attention_decode_shared"] = (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                            c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                            c_float, c_void_p, ctypes.POINTER(SharedPlanInfo),
+                                                            c_void_p, c_size_t, c_void_p, c_void_p])
 
 
 def library():
@@ -445,6 +469,59 @@ def paged_attention_prefill(out, query, key_cache, value_cache, block_tables, qu
 # ---------------------------------------------------------------------------
 # Host block manager
 # ---------------------------------------------------------------------------
+
+def shared_plan(block_tables, context_lens, num_heads, num_kv_heads, block_size, min_rows=2, key_chunk=0):
+    """Host plan of the shared-prefix decode from host tables [B, max_blocks] int32 and lengths
+    [B] int32 (NumPy).  Returns (plan, info): plan a uint8 NumPy array of info.bytes bytes to
+    copy to the device, info a SharedPlanInfo."""
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    if tables.ndim != 2 or lens.shape != (tables.shape[0],):
+        raise ValueError("shared_plan: block_tables must be [B, max_blocks], context_lens [B]")
+    B, mb = tables.shape
+    info = SharedPlanInfo()
+    lib = library()
+    _check(lib.pkv_shared_plan(_np_ptr(tables), mb, _np_ptr(lens), B, num_heads, num_kv_heads, block_size, min_rows,
+                               key_chunk, None, 0, ctypes.byref(info)), "shared_plan")
+    plan = np.zeros(int(info.bytes), np.uint8)
+    _check(lib.pkv_shared_plan(_np_ptr(tables), mb, _np_ptr(lens), B, num_heads, num_kv_heads, block_size, min_rows,
+                               key_chunk, _np_ptr(plan), plan.nbytes, ctypes.byref(info)), "shared_plan")
+    return plan, info
+
+
+def paged_attention_decode_shared_workspace_size(info, num_heads, num_kv_heads, head_dim) -> int:
+    return int(library().pkv_paged_attention_decode_shared_workspace_size(ctypes.byref(info), num_heads, num_kv_heads,
+                                                                          head_dim))
+
+
+def paged_attention_decode_shared(out, query, key_cache, value_cache, block_tables, context_lens, scale, plan, info,
+                                  workspace, status=None, stream=None):
+    """Shared-prefix decode: the result of paged_attention_decode, with blocks that adjacent
+    rows share read once per kv head.  plan: the device copy (uint8 tensor) of shared_plan's
+    plan for these tables and lengths; info: its SharedPlanInfo."""
+    torch = _torch()
+    _same_device("paged_attention_decode_shared", out, query, key_cache, value_cache, block_tables, context_lens, plan,
+                 workspace, status)
+    B, Hq, D = query.shape
+    NB, Hkv, bs, D2 = key_cache.shape
+    if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
+        raise ValueError("paged_attention_decode_shared: shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("paged_attention_decode_shared: block_tables must be [B, max_blocks], context_lens [B]")
+    out_dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(out.dtype)
+    if out_dtype is None:
+        raise TypeError("paged_attention_decode_shared: out must be bf16 or f32")
+    if plan.numel() * plan.element_size() < int(info.bytes):
+        raise ValueError("paged_attention_decode_shared: the device plan is smaller than info.bytes")
+    rc = library().pkv_paged_attention_decode_shared(
+        _ptr(out, None, "out"), out_dtype, _ptr(query, torch.bfloat16, "query"),
+        _ptr(key_cache, torch.bfloat16, "key_cache"), _ptr(value_cache, torch.bfloat16, "value_cache"),
+        _ptr(block_tables, torch.int32, "block_tables"), int(block_tables.shape[1]),
+        _ptr(context_lens, torch.int32, "context_lens"), B, Hq, Hkv, D, bs, NB, float(scale),
+        _ptr(plan, torch.uint8, "plan"), ctypes.byref(info), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "paged_attention_decode_shared")
+
 
 def _np_ptr(a):
     return c_void_p(a.ctypes.data) if a is not None and a.size else c_void_p(0)

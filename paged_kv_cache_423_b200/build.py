@@ -11,6 +11,12 @@ library.
 ``variant="depth1"`` builds ``libpkv_depth1.so`` (objects under ``_build/depth1``) with the
 CUDA-core decode kernel's per-warp copy ring at one stage, so every copy waits for the
 previous stage's compute; a test compares it bit for bit with the default build.
+
+``variant="shortwait"`` builds ``libpkv_shortwait.so`` whose CUDA-core decode and prefill
+kernels give up a pipeline wait after a few hundred nanoseconds of polling instead of one
+second, so an ordinary launch takes its expiry path (flag PKV_DEV_TIMEOUT, let copies land,
+wait for MMAs, free tensor memory, return); a test checks the flag and that the context
+stays usable.  No wait is removed and the drains keep their one-second limit.
 """
 from __future__ import annotations
 
@@ -31,7 +37,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xptxas", "-v",
               "--expt-relaxed-constexpr", "-Xcompiler", "-fvisibility=hidden"]
 CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-fvisibility=hidden"]
-VARIANTS = {"depth1": ["-DPKV_SIMT_STAGES=1", "-DPKV_SIMT_STAGES8=1"]}
+VARIANTS = {"depth1": ["-DPKV_SIMT_STAGES=1", "-DPKV_SIMT_STAGES8=1"],
+            "shortwait": ["-DPKV_SHORT_WAITS"]}
 
 
 def lib_path(variant: str | None = None) -> str:

@@ -477,7 +477,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   bool timed_out = false;
   while (consumed < issued) {
     const int slot = consumed % STAGES;
-    if (!mbar_wait(&ring.full[slot], (consumed / STAGES) & 1)) {
+    if (!__all_sync(kFull, pipe_wait(&ring.full[slot], (consumed / STAGES) & 1))) {  // warp-uniform
       timed_out = true;
       break;
     }
@@ -769,7 +769,7 @@ static int launch_simt(const DecodeArgs& a, cudaStream_t stream) {
   return PKV_OK;
 }
 
-static int launch_plan(const DecodeArgs& a, const int32_t* context_lens, int max_context_len, cudaStream_t stream) {
+int launch_decode_plan(const DecodeArgs& a, const int32_t* context_lens, int max_context_len, cudaStream_t stream) {
   plan_kernel<<<1, kPlanThreads, 0, stream>>>(context_lens, a.num_seqs, max_context_len,
                                               a.max_blocks * a.block_size, a.partition,
                                               const_cast<PlanEntry*>(a.entries),
@@ -818,7 +818,7 @@ extern "C" size_t pkv_paged_attention_workspace_size(int num_seqs, int num_heads
                                       : resolve_partition(partition_tokens, true, num_seqs, num_kv_heads, block_size,
                                                           max_context_len);
   if (p < 0) return 0;
-  return workspace_layout(num_seqs, num_heads, head_dim, max_context_len, p).total;
+  return workspace_layout(num_seqs, num_heads, head_dim, max_context_len, p, false, num_kv_heads).total;
 }
 
 // Shared by the bf16 and the 8-bit entry points; `k_scale` != null selects the
@@ -890,7 +890,8 @@ static int decode_impl(void* out, int out_dtype, const void* query, const void* 
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: tensors must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: workspace must be 256-byte aligned");
-  const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim, max_context_len, partition);
+  const WorkspaceLayout w =
+      workspace_layout(num_seqs, num_heads, head_dim, max_context_len, partition, false, num_kv_heads);
   if (workspace_bytes < w.total)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode: workspace of %zu bytes, %zu needed", workspace_bytes,
                      w.total);
@@ -916,6 +917,10 @@ static int decode_impl(void* out, int out_dtype, const void* query, const void* 
   a.arrive = reinterpret_cast<int32_t*>(ws + w.off_arrive);
   a.part_o = reinterpret_cast<float*>(ws + w.off_part_o);
   a.part_ml = reinterpret_cast<float2*>(ws + w.off_part_ml);
+  if (kv8 && use_tensor) {
+    a.q_split = ws + w.off_qsplit;
+    a.q_inv = reinterpret_cast<float*>(ws + w.off_qinv);
+  }
   a.status = status;
   a.context_lens = context_lens;
   a.max_context_len = max_context_len;
@@ -931,7 +936,7 @@ static int decode_impl(void* out, int out_dtype, const void* query, const void* 
   a.scale_log2 = scale * 1.4426950408889634f;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int rc = launch_plan(a, context_lens, max_context_len, s);
+  int rc = launch_decode_plan(a, context_lens, max_context_len, s);
   if (rc != PKV_OK) return rc;
   const bool out_f32 = out_dtype == PKV_DTYPE_F32;
   if (kv8 && use_tensor) return launch_decode_tensor_fp8(a, head_dim, out_f32, s);

@@ -49,6 +49,15 @@ struct DecodeArgs {
   int partition;               // tokens per partition
   int max_parts;
   float scale_log2;            // scale * log2(e): scores are kept in base-2 units
+  // Shared-prefix decode, private phase (tensor-core path only): each row's table is read from
+  // position block_offset[row] on, and every item writes its partial (o, m, l), also unsplit
+  // ones; the merge of the shared-prefix decode combines them.  Null / 0 otherwise.
+  const int32_t* block_offset;
+  int always_partial;
+  // 8-bit tensor-core path: the queries split once per call into e4m3 [hi; lo] rows (32 rows of
+  // 128 codes per (sequence, kv head)) and the power of two 2^-e of each head (16 per unit).
+  uint8_t* q_split;
+  float* q_inv;
 };
 
 // Workspace layout, identical for every decode path.
@@ -56,7 +65,13 @@ struct WorkspaceLayout {
   int partition = 0;
   int max_parts = 0;
   size_t off_count = 0, off_arrive = 0, off_entries = 0, off_part_o = 0, off_part_ml = 0, total = 0;
+  size_t off_qsplit = 0, off_qinv = 0;  // only when the tensor-core path can run (split queries of the 8-bit pool)
 };
+
+// Bytes of split queries per (sequence, kv head) unit: 32 rows of 128 e4m3 codes, and 16 scales.
+constexpr size_t kQSplitUnitBytes = 32 * 128;
+constexpr size_t kQInvUnitBytes = 16 * sizeof(float);
+bool tensor_path_supports(int group, int head_dim);
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -81,7 +96,7 @@ inline int auto_partition_tokens_tensor(int num_seqs, int num_kv_heads, int bloc
 }
 
 inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int max_context_len,
-                                        int partition) {
+                                        int partition, bool force_partials = false, int num_kv_heads = 0) {
   WorkspaceLayout w;
   w.partition = partition;
   w.max_parts = max_context_len <= 0 ? 1 : (max_context_len + partition - 1) / partition;
@@ -93,21 +108,49 @@ inline WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_di
   w.off_entries = off;
   off = align256(off + static_cast<size_t>(num_seqs) * w.max_parts * sizeof(PlanEntry));
   w.off_part_o = off;
-  if (w.max_parts > 1) {
+  if (w.max_parts > 1 || force_partials) {
     off = align256(off + static_cast<size_t>(num_seqs) * num_heads * w.max_parts * head_dim * sizeof(float));
     w.off_part_ml = off;
     off = align256(off + static_cast<size_t>(num_seqs) * num_heads * w.max_parts * sizeof(float2));
   } else {
     w.off_part_ml = off;
   }
+  if (num_kv_heads > 0 && num_heads % num_kv_heads == 0 && tensor_path_supports(num_heads / num_kv_heads, head_dim)) {
+    const size_t units = static_cast<size_t>(num_seqs) * num_kv_heads;
+    w.off_qsplit = off;
+    off = align256(off + units * kQSplitUnitBytes);
+    w.off_qinv = off;
+    off = align256(off + units * kQInvUnitBytes);
+  }
   w.total = off;
   return w;
 }
 
+// The shared phase of the shared-prefix decode: the prefill kernel in segment mode over the
+// plan's entries and parts (prefill_tc.cu).
+struct SegmentLaunch {
+  const void* query;            // [num_seqs, num_heads, 128] bf16
+  const void* key_cache;
+  const void* value_cache;
+  const int32_t* block_tables;
+  const int32_t* plan_count;    // [0] entries, [1] work-item counter (zero before the launch)
+  const int4* entries;
+  const int4* parts;
+  float* part_o;
+  float2* part_ml;
+  int32_t* status;
+  int num_entries;              // grid sizing (host)
+  int max_blocks, num_seqs, num_heads, num_kv_heads, block_size, num_blocks;
+  float scale;
+};
+int launch_prefill_segments(const SegmentLaunch& launch, cudaStream_t stream);
+
 // Launchers living in other translation units.
+// The decode plan kernel (decode.cu): validates context_lens, sorts (sequence, partition)
+// entries longest first into a.entries, zeroes a.plan_count's counter and a.arrive.
+int launch_decode_plan(const DecodeArgs& a, const int32_t* context_lens, int max_context_len, cudaStream_t stream);
 int launch_decode_tensor(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
 int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
-bool tensor_path_supports(int group, int head_dim);
 // Merge of split partitions (no launch when max_parts <= 1), after a tensor-core decode.
 int launch_merge_partials(const DecodeArgs& a, bool out_f32, cudaStream_t stream);
 

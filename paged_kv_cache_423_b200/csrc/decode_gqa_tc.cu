@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       const int tok0 = e.y * a.partition;
       const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - tok0);
       const int nblk = (ntok + a.block_size - 1) / a.block_size;
-      const int32_t* row = a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size;
+      const int32_t* row = a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size +
+                           (a.block_offset ? a.block_offset[e.x] : 0);
       int4 t = make_int4(0, 0, 0, 0);
       if (lane < nblk) t.x = __ldg(row + lane);
       if (lane + 32 < nblk) t.y = __ldg(row + lane + 32);
@@ -540,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         for (int h = 0; h < N; ++h) {
           if (h >= g) break;
           const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
-          if (nparts == 1) {
+          if (nparts == 1 && !a.always_partial) {
             store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[h] / l : 0.f);
           } else {
             // unnormalised partial; a separate kernel merges the partitions
@@ -661,7 +662,7 @@ static int launch(const Args& args, cudaStream_t stream) {
   kernel<<<std::max(1, sms), kThreads, smem, stream>>>(args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) launch: %s", cudaGetErrorString(e));
-  return launch_merge_partials(args.a, OUT_F32, stream);
+  return args.a.always_partial ? PKV_OK : launch_merge_partials(args.a, OUT_F32, stream);
 }
 
 }  // namespace tc

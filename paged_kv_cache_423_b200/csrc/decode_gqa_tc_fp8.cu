@@ -21,10 +21,13 @@
 //              same represented values.
 //   The K scale and 2^-e join the score scale, the V scale the output.
 //
-// Roles: warps 0-3 softmax (thread = TMEM lane = token row of a tile), warp 4 TMA
-// producer, warp 5 MMA issuer (fixed order: S of tile n+1, then O += Vᵀ·P of tile
-// n), warp 6 splits each item's queries as soon as they land.  Work items, plan,
-// workspace and the merge of split partitions are those of the bf16 decode paths.
+// The queries are split into their e4m3 terms once per call, before the main kernel,
+// by split_queries_kernel (one warp per (sequence, kv head)), into the workspace; the
+// producer loads an item's split rows and head scales with its first tile, so no MMA
+// waits for a split.  Roles: warps 0-7 softmax (two groups; thread = TMEM lane = token
+// row of a tile), warp 8 TMA producer, warp 9 MMA issuer (fixed order: S of tile n+1,
+// then O += Vᵀ·P of tile n).  Work items, plan, workspace and the merge of split
+// partitions are those of the bf16 decode paths.
 // Every wait is bounded; on a timeout the CTA flags PKV_DEV_TIMEOUT, lets its copies
 // land, waits for its MMAs, frees its tensor memory and exits.
 #include <cuda.h>
@@ -51,15 +54,14 @@ constexpr int kStages = 5;                 // e4m3 staging ring
 constexpr int kRow8 = kD;                  // bytes of one e4m3 row
 constexpr int kStage8 = 2 * kTile * kRow8; // K then V: 32 KiB
 constexpr int kVOff = kTile * kRow8;       // V within a stage
-constexpr int kQSlot = 4096;               // bf16 queries (2 halves x 16 rows x 128 B), then e4m3 [hi; lo] in place
+constexpr int kQSlot = 4096;               // e4m3 [hi; lo] queries: 32 rows x 128 codes (from the split kernel)
 constexpr int kQSlots = 6;                 // by item ordinal; a slot is refilled 6 items later
 constexpr int kPTerm = kTile * 16;         // one e5m2 term of P: 128 tokens x 16 heads
 constexpr int kPBytes = 3 * kPTerm;        // [hi | mid | lo]
 constexpr int kSoftmax = 256;              // warps 0-7: two groups of 4 (head pairs 0, 2, .. and 1, 3, ..)
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kQueryWarp = 10;
-constexpr int kThreads = 384;              // 3 warpgroups; warp 11 only lends registers
+constexpr int kThreads = 384;              // 3 warpgroups; warps 10-11 only lend registers
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); the
 // control warpgroup drops to 88 and the two softmax warpgroups rise to 208:
 // 128 x (208 + 208 + 88) = 64512, and per scheduler (one warp of each group)
@@ -85,18 +87,18 @@ constexpr int kOffP = kOffQ + kQSlots * kQSlot;
 constexpr int kOffRed = kOffP + 2 * kPBytes;
 constexpr int kOffMeta = kOffRed + 2 * 3 * 4 * 16 * 4;  // [group][maxima | sums of even | odd items][4 warps][16]
 constexpr int kOffScale = kOffMeta + kStages * 16;  // [stage] (k_scale, v_scale) of the item
-constexpr int kOffQinv = kOffScale + kStages * 8;   // [q slot][16] 2^-e of each head
+constexpr int kOffQinv = (kOffScale + kStages * 8 + 15) / 16 * 16;  // [q slot][16] 2^-e of each head (bulk copies)
 constexpr int kOffBar = kOffQinv + kQSlots * 16 * 4;
-constexpr int kBars = 2 * kStages + kQSlots + 2 * 4 + 1;
+constexpr int kBars = 2 * kStages + 2 * 4 + 1;
 constexpr int kOffMisc = kOffBar + kBars * 8;
 constexpr int kSmemBytes = kOffMisc + 32 + 1024;
-static_assert(kOffBar % 8 == 0 && kOffMeta % 16 == 0 && kOffQ % 1024 == 0, "alignment");
+static_assert(kOffBar % 8 == 0 && kOffMeta % 16 == 0 && kOffQ % 1024 == 0 && kOffQinv % 16 == 0, "alignment");
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 
 struct alignas(64) Args {
   CUtensorMap tm_k;  // e4m3 pool as [rows, 128] bytes, box 128 x 16, 128-byte swizzle
   CUtensorMap tm_v;
-  CUtensorMap tm_q;  // bf16 queries as [B * Hq, 128], box 64 x 16, 128-byte swizzle
+  CUtensorMap tm_q;  // split e4m3 queries as [units * 32, 128] bytes, box 128 x 32, 128-byte swizzle
   DecodeArgs a;
 };
 
@@ -175,15 +177,15 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, floa
 }
 
 // Pipeline (per CTA, persistent over work items; n counts tiles):
-//   producer     -> full[s]    : e4m3 K, V (and the bf16 queries on an item's first tile) in stage s
-//   query warp   -> q_ready[j] : the queries of the item in q slot j split into e4m3 hi/lo
+//   producer     -> full[s]    : e4m3 K, V (and an item's split queries and head scales on its
+//                                first tile) in stage s
 //   MMA          -> s_full[b]  : S of the b-th valid tile (mod 2) in TMEM
 //   softmax      -> s_free[b]  : that S read (8 warps)
 //   softmax      -> p_full[b]  : P of that tile in shared buffer b (and its stale V rows zeroed; 8 warps)
 //   MMA          -> o_bar[b]   : its O += Vᵀ·P done (P buffer b reusable)
-//   MMA + softmax + query warp -> empty[s] : stage s done with: its P·V complete
-//                  (commit; a plain arrival for a tile with no rows), metadata read by
-//                  the 8 softmax warps and the query warp (10 arrivals)
+//   MMA + softmax -> empty[s] : stage s done with: its P·V complete (commit; a plain
+//                  arrival for a tile with no rows), metadata read by the 8 softmax warps
+//                  (9 arrivals)
 // Each tile's heads are split between the two softmax groups; they take every
 // decision that touches the shared O accumulator (a rescale restarts it) together.
 // NH (4, 8 or 16 >= g) bounds the heads the softmax works on; the operand layouts
@@ -204,8 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;
-  uint64_t* q_ready = empty + kStages;
-  uint64_t* s_full = q_ready + kQSlots;
+  uint64_t* s_full = empty + kStages;
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_bar = p_full + 2;
@@ -222,9 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 8 + 1);
+      mbar_init(&empty[s], 1 + 8);
     }
-    for (int j = 0; j < kQSlots; ++j) mbar_init(&q_ready[j], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&s_free[b], 8);
@@ -327,11 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         }
         const bool with_q = tile == 0 && ntok > 0;
         if (lane == 0) {
-          meta[slot] = make_int4(e.x, kvh | (qslot << 16) | (((item_ord / kQSlots) & 1) << 20), e.y | (e.z << 16),
+          meta[slot] = make_int4(e.x, kvh | (qslot << 16), e.y | (e.z << 16),
                                  n_valid | (mask << 8) | (tile == 0 ? kMetaFirst : 0) |
                                      (tile == ntiles - 1 ? kMetaLast : 0));
           mscale[slot] = sc_cur;
-          mbar_arrive_expect_tx(&full[slot], __popc(mask) * kChunkTx + (with_q ? kQSlot : 0));
+          mbar_arrive_expect_tx(&full[slot], __popc(mask) * kChunkTx + (with_q ? kQSlot + 16 * 4 : 0));
         }
         __syncwarp();
         if (ok) {
@@ -341,10 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
           tc::tma_load_2d(dst + kVOff, &args.tm_v, 0, r, &full[slot], policy);
         }
         if (with_q && lane == 0) {
-          const int qrow = e.x * a.num_heads + kvh * g;
-          unsigned char* qd = q_ring + qslot * kQSlot;
-          tc::tma_load_2d(qd, &args.tm_q, 0, qrow, &full[slot], policy);
-          tc::tma_load_2d(qd + kN * 128, &args.tm_q, 64, qrow, &full[slot], policy);
+          const int64_t unit = static_cast<int64_t>(e.x) * a.num_kv_heads + kvh;
+          tc::tma_load_2d(q_ring + qslot * kQSlot, &args.tm_q, 0, static_cast<int>(unit * 32), &full[slot], policy);
+          bulk_copy_g2s(qinv + qslot * 16, a.q_inv + unit * 16, 16 * 4, &full[slot], policy);
         }
       }
       item = item_nxt;
@@ -372,71 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
     }
     // Let this CTA's last copies land before the final barrier.
     for (int k = max(0, n - kStages); k < n; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1);
-  } else if (warp == kQueryWarp) {
-    // ================= query split: bf16 -> e4m3 [hi; lo] with a power of two per head =================
-    // Lane l takes head r = l / 2 and half h = l % 2 (dims 64h .. 64h+63) of the bf16 slot.
-    const int r = lane >> 1, h = lane & 1;
-    for (int n = 0;; ++n) {
-      const int slot = n % kStages;
-      if (!mbar_wait(&full[slot], (n / kStages) & 1)) {
-        *abort_flag = 1;
-        set_status(a.status, PKV_DEV_TIMEOUT);
-        break;
-      }
-      const int4 mt = meta[slot];
-      if (mt.w & kMetaEnd) break;
-      if ((mt.w & kMetaFirst) && (mt.w & 0xff) > 0) {
-        const int qs = (mt.y >> 16) & 0xf;
-        unsigned char* qb = q_ring + qs * kQSlot;
-        // bf16 row r of half h: 128 bytes, 16-byte chunk c at (c ^ (r % 8)) * 16
-        uint4 v[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          v[c] = *reinterpret_cast<const uint4*>(qb + h * 2048 + r * 128 + ((c ^ (r & 7)) << 4));
-        float m = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
-        }
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        // 2^e with the head's largest |q| * 2^e in [128, 256)
-        const int E = static_cast<int>((__float_as_uint(m) >> 23) & 0xff);
-        const int e = E == 0 ? 0 : min(134 - E, 126);
-        const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-        __syncwarp();  // every bf16 value read before the slot is rewritten
-        // e4m3 rows: hi of head r at row r, lo at row 16 + r (128 bytes, 128-byte
-        // swizzle); dims 64h + 16j .. sit in 16-byte chunk 4h + j
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 x0 = v[2 * j], x1 = v[2 * j + 1];  // dims 64h + 16j + 0..7, + 8..15
-          const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-          uint32_t s[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) s[i] = split_q2(bf16lo(w[i]) * up, bf16hi(w[i]) * up);
-          uint4 hi4, lo4;
-          hi4.x = __byte_perm(s[0], s[1], 0x5410);
-          hi4.y = __byte_perm(s[2], s[3], 0x5410);
-          hi4.z = __byte_perm(s[4], s[5], 0x5410);
-          hi4.w = __byte_perm(s[6], s[7], 0x5410);
-          lo4.x = __byte_perm(s[0], s[1], 0x7632);
-          lo4.y = __byte_perm(s[2], s[3], 0x7632);
-          lo4.z = __byte_perm(s[4], s[5], 0x7632);
-          lo4.w = __byte_perm(s[6], s[7], 0x7632);
-          const int pc = ((4 * h + j) ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4*>(qb + r * 128 + pc) = hi4;
-          *reinterpret_cast<uint4*>(qb + (16 + r) * 128 + pc) = lo4;
-        }
-        if (h == 0) qinv[qs * 16 + r] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-        fence_proxy_async_smem();  // the split queries, before the MMAs read them
-      }
-      __syncwarp();
-      // every item's first tile completes one phase of its slot's barrier (an empty
-      // item's too), so the phase of item i in slot i % 6 is (i / 6) & 1 for all roles
-      if ((mt.w & kMetaFirst) && lane == 0) mbar_arrive(&q_ready[(mt.y >> 16) & 0xf]);
-      if (lane == 0) mbar_arrive(&empty[slot]);  // metadata read
-    }
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer (one thread) =================
     if (lane == 0) {
@@ -482,7 +416,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         const int4 mt = meta[slot];
         if (mt.w & kMetaEnd) break;
         const int nv = mt.w & 0xff;
-        const bool first = mt.w & kMetaFirst;
         if (nv == 0) {
           if (prev_slot >= 0) issue_pv();
           mbar_arrive(&empty[slot]);
@@ -490,7 +423,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         }
         // S = K·[hi; lo]ᵀ of tile n
         const int qs = (mt.y >> 16) & 0xf;
-        if (first && !wait(&q_ready[qs], (mt.y >> 20) & 1)) break;
         const int b = q_valid & 1;
         if (q_valid >= 2 && !wait(&s_free[b], ((q_valid >> 1) - 1) & 1)) break;
         tc::tc_fence_after();
@@ -625,8 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         out_scale = sc.y;
         obuf ^= 1;
         if (n_valid > 0) {
-          const int qs = (mt.y >> 16) & 0xf;
-          bad |= !mbar_wait(&q_ready[qs], (mt.y >> 20) & 1);
+          const int qs = (mt.y >> 16) & 0xf;  // its split queries and head scales landed with this tile
           const float base = a.scale_log2 * sc.x;
 #pragma unroll
           for (int j = 0; j < NL; ++j) hscale[j] = base * qinv[qs * 16 + head(j)];
@@ -773,18 +704,70 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---- query split ------------------------------------------------------------------
+//
+// Once per call, before the main kernel: every (sequence, kv head) unit's g query heads as
+// e4m3 [hi; lo] rows, one warp per unit.  Lane l takes head r = l / 2, half h = l % 2 (dims
+// 64h .. 64h+63).  The head's largest |q| is brought into [128, 256) by a power of two 2^e;
+// hi is q·2^e rounded to e4m3, lo the remainder rounded to e4m3.  Row r holds hi of head r,
+// row 16 + r its lo, 128 codes each (plain rows: the main kernel's tensor map applies the
+// 128-byte swizzle on load); rows of heads g .. 15 are zero.  2^-e goes to q_inv[unit][r].
+constexpr int kSplitWarps = 4;
+
+__global__ void __launch_bounds__(kSplitWarps * 32) split_queries_kernel(const DecodeArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kSplitWarps + warp;
+  if (unit >= static_cast<int64_t>(a.num_seqs) * a.num_kv_heads) return;  // warp-uniform
+  const int seq = static_cast<int>(unit / a.num_kv_heads), kvh = static_cast<int>(unit % a.num_kv_heads);
+  const int g = a.group;
+  const int r = lane >> 1, h = lane & 1;
+  const bool live = r < g;
+  const uint4* src = reinterpret_cast<const uint4*>(a.query + (static_cast<int64_t>(seq) * a.num_heads + kvh * g +
+                                                               (live ? r : 0)) * kD + 64 * h);
+  uint4 v[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) v[c] = live ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+  float m = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
+  }
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  const int E = static_cast<int>((__float_as_uint(m) >> 23) & 0xff);
+  const int e = E == 0 ? 0 : min(134 - E, 126);
+  const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+  uint8_t* dst = a.q_split + unit * static_cast<int64_t>(kQSplitUnitBytes);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 x0 = v[2 * j], x1 = v[2 * j + 1];  // dims 64h + 16j + 0..7, + 8..15
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    uint32_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = split_q2(bf16lo(w[i]) * up, bf16hi(w[i]) * up);
+    const uint4 hi4 = make_uint4(__byte_perm(q[0], q[1], 0x5410), __byte_perm(q[2], q[3], 0x5410),
+                                 __byte_perm(q[4], q[5], 0x5410), __byte_perm(q[6], q[7], 0x5410));
+    const uint4 lo4 = make_uint4(__byte_perm(q[0], q[1], 0x7632), __byte_perm(q[2], q[3], 0x7632),
+                                 __byte_perm(q[4], q[5], 0x7632), __byte_perm(q[6], q[7], 0x7632));
+    *reinterpret_cast<uint4*>(dst + r * 128 + (4 * h + j) * 16) = hi4;
+    *reinterpret_cast<uint4*>(dst + (16 + r) * 128 + (4 * h + j) * 16) = lo4;
+  }
+  if (h == 0) a.q_inv[unit * 16 + r] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+}
+
 // ---- host side -----------------------------------------------------------------
 
-// 2-D view [rows, 128] with a 128-byte swizzle: the e4m3 pool (box 128 codes x 16
-// rows) or the bf16 queries (box 64 values x 16 rows).
-static int encode_map(CUtensorMap* map, const void* base, uint64_t rows, bool e4m3, const char* what) {
+// 2-D view [rows, 128] bytes with a 128-byte swizzle, box 128 x box_rows: the e4m3 pool
+// (16-row slices) or the split queries (32 rows per unit).
+static int encode_map(CUtensorMap* map, const void* base, uint64_t rows, int box_rows, const char* what) {
   auto encode = tc::tensor_map_encoder();
   if (!encode) return set_error(PKV_ERR_CUDA, "decode (8-bit tensor): cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * (e4m3 ? 1 : 2)};
-  cuuint32_t box[2] = {e4m3 ? 128u : 64u, e4m3 ? static_cast<cuuint32_t>(kChunk) : static_cast<cuuint32_t>(kN)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                       const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -817,11 +800,19 @@ int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cu
   tc8::Args args;
   args.a = a;
   const uint64_t pool_rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
-  int rc = tc8::encode_map(&args.tm_k, a.key_cache8, pool_rows, true, "key_cache");
-  if (rc == PKV_OK) rc = tc8::encode_map(&args.tm_v, a.value_cache8, pool_rows, true, "value_cache");
-  if (rc == PKV_OK)
-    rc = tc8::encode_map(&args.tm_q, a.query, static_cast<uint64_t>(a.num_seqs) * a.num_heads, false, "query");
+  if (!a.q_split || !a.q_inv) return set_error(PKV_ERR_INVALID, "decode (8-bit tensor): no split-query workspace");
+  const uint64_t units = static_cast<uint64_t>(a.num_seqs) * a.num_kv_heads;
+  int rc = tc8::encode_map(&args.tm_k, a.key_cache8, pool_rows, tc8::kChunk, "key_cache");
+  if (rc == PKV_OK) rc = tc8::encode_map(&args.tm_v, a.value_cache8, pool_rows, tc8::kChunk, "value_cache");
+  if (rc == PKV_OK) rc = tc8::encode_map(&args.tm_q, a.q_split, units * 32, 32, "split queries");
   if (rc != PKV_OK) return rc;
+  if (units > 0) {
+    const unsigned grid = static_cast<unsigned>((units + tc8::kSplitWarps - 1) / tc8::kSplitWarps);
+    tc8::split_queries_kernel<<<grid, tc8::kSplitWarps * 32, 0, stream>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+      return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) query split launch: %s", cudaGetErrorString(e));
+  }
   if (a.group <= 4)
     rc = out_f32 ? tc8::launch<true, 4>(args, stream) : tc8::launch<false, 4>(args, stream);
   else if (a.group <= 8)

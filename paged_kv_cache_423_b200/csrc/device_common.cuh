@@ -85,6 +85,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// The short wait of the failure-path test build (PKV_SHORT_WAITS): 16 polls, a few hundred
+// nanoseconds, so that an ordinary launch runs into its expiry path.  No wait is removed.
+__device__ __forceinline__ bool mbar_wait_short(uint64_t* bar, uint32_t parity) {
+#pragma unroll 1
+  for (int i = 0; i < 16; ++i)
+    if (mbar_test(bar, parity)) return true;
+  return false;
+}
+
+// Pipeline waits of the CUDA-core decode and of the prefill kernel: bounded by kWaitLimitNs,
+// or by the short poll in the failure-path test build.  Their end-of-kernel drains (copies
+// landing, MMAs completing) always take mbar_wait.
+__device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity) {
+#ifdef PKV_SHORT_WAITS
+  return mbar_wait_short(bar, parity);
+#else
+  return mbar_wait(bar, parity);
+#endif
+}
+
 // Bulk copy global -> shared (async proxy), completion counted on `bar` in bytes.
 // Both addresses 16-byte aligned, bytes a multiple of 16.  Streaming data: the L2
 // line is marked evict-first.

@@ -65,15 +65,23 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 384;              // 3 warpgroups; warps 10-11 only lend registers
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); the
-// producer/MMA warpgroup drops to 88 and the two softmax warpgroups rise to 208:
-// 128 x (208 + 208 + 88) = 64512 <= 64512, and per scheduler (one warp of each
-// group) 32 x 504 = 16128 <= 16384 registers.
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsControl = 88;
+// producer/MMA warpgroup drops to 120 and the two softmax warpgroups rise to 192:
+// 128 x (192 + 192 + 120) = 64512 <= 64512, and per scheduler (one warp of each
+// group) 32 x 504 = 16128 <= 16384 registers.  ptxas fits both roles without
+// spilling at these counts (at 208 / 88 the control warps spilled).
+constexpr int kRegsSoftmax = 192;
+constexpr int kRegsControl = 120;
 static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;
+// Share of the softmax exponentials computed by a polynomial on the FMA pipe (one pair of
+// scores in kPolyEvery; 0 = none): the SFU issues 16 exponentials per clock per SM, about as
+// many as a stage's MMAs take, so part of them moves to the 128-wide FMA pipe.
+#ifndef PKV_PREFILL_POLY_EVERY
+#define PKV_PREFILL_POLY_EVERY 4
+#endif
+constexpr int kPolyEvery = PKV_PREFILL_POLY_EVERY;
 
 // shared memory (offsets from a 1024-aligned base)
 constexpr int kOffQ = 0;                                   // [2 tiles]
@@ -96,6 +104,11 @@ struct PrefillArgs {
   const int32_t* block_tables;
   const int32_t* plan_count;  // [0] entries, [1] work-item counter
   const int4* entries;        // x = first packed row, y = its position, z = tokens A | tokens B << 8, w = sequence
+                              // (segment mode: w = part, y unused)
+  const int4* parts;          // segment mode: [2 * part] (table row, first block, keys, first row),
+                              //               [2 * part + 1] (rows, first partial, 0, 0)
+  float* part_o;              // segment mode: unnormalised partial outputs [partial][head][128]
+  float2* part_ml;            // segment mode: (held maximum in base-2 units, weight sum) [partial][head]
   int32_t* status;
   int max_blocks;
   int num_heads;
@@ -115,7 +128,10 @@ struct alignas(64) Args {
   PrefillArgs a;
 };
 
-template <bool OUT_F32>
+// SEG = false: causal prefill, normalised output rows.  SEG = true: the shared phase of
+// the shared-prefix decode — every query row of an item sees all keys of its part (a run
+// of whole blocks of one table row), and the epilogue writes unnormalised partials.
+template <bool OUT_F32, bool SEG>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ Args args) {
   const PrefillArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
@@ -199,7 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     bool failed = false;
     auto wait_slot = [&](uint64_t* bar, int fills, int depth) -> bool {
       if (failed) return false;
-      if (fills >= depth && !mbar_wait(bar, ((fills / depth) - 1) & 1)) {
+      // warp-uniform: every lane takes the same branch (the copies below are per lane)
+      if (fills >= depth && !__all_sync(0xffffffffu, pipe_wait(bar, ((fills / depth) - 1) & 1))) {
         fail();
         failed = true;
       }
@@ -207,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     };
     // the item whose stages the K side is issuing
     int64_t item = grab();
-    int kvh = 0, row0 = 0, pos0 = 0, ntok_a = 0, ntok_b = 0, nkeys = 0, nst = 0, j = 0;
+    int kvh = 0, row0 = 0, pos0 = 0, ntok_a = 0, ntok_b = 0, nkeys = 0, nst = 0, j = 0, meta_x = 0;
     const int32_t* table = nullptr;
     int tab_cur = -1, tab_nxt = -1, win = 0;
     // Table entries come 32 slices (4 stages) at a time, one window ahead: lane l
@@ -220,13 +237,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int4 e = a.entries[item / a.num_kv_heads];
       kvh = static_cast<int>(item % a.num_kv_heads);
       row0 = e.x;
-      pos0 = e.y;
       ntok_a = e.z & 0xff;
       ntok_b = (e.z >> 8) & 0xff;
-      nkeys = pos0 + ntok_a + ntok_b;
+      if constexpr (SEG) {
+        // the stage metadata carries the pair's first partial id and the part's key count
+        const int4 pd0 = a.parts[2 * e.w], pd1 = a.parts[2 * e.w + 1];
+        nkeys = pd0.z;
+        meta_x = pd1.y + (e.x - pd0.w);
+        pos0 = nkeys;
+        table = a.block_tables + static_cast<int64_t>(pd0.x) * a.max_blocks + pd0.y;
+      } else {
+        pos0 = e.y;
+        nkeys = pos0 + ntok_a + ntok_b;
+        meta_x = row0;
+        table = a.block_tables + static_cast<int64_t>(e.w) * a.max_blocks;
+      }
       nst = (nkeys + kKeys - 1) / kKeys;
       j = 0;
-      table = a.block_tables + static_cast<int64_t>(e.w) * a.max_blocks;
       win = 0;
       tab_cur = load_window(0);
       tab_nxt = load_window(1);
@@ -270,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       if (!wait_slot(&meta_free[kn % kMetaSlots], kn, kMetaSlots)) return false;
       const int ks = kn % kKStages;
       if (lane == 0) {
-        meta[kn % kMetaSlots] = make_int4(row0, pos0, ntok_a | (ntok_b << 8) | (kvh << 16),
+        meta[kn % kMetaSlots] = make_int4(meta_x, pos0, ntok_a | (ntok_b << 8) | (kvh << 16),
                                           j | static_cast<int>(mask << 18) | (j == 0 ? kFirst : 0) |
                                               (j == nst - 1 ? kLast : 0));
         mbar_arrive(&meta_full[kn % kMetaSlots]);
@@ -357,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       int q_items = 0;
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t parity) {
-        if (ok && !mbar_wait(bar, parity)) {
+        if (ok && !pipe_wait(bar, parity)) {
           ok = false;
           fail();
         }
@@ -450,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     bool has_pv = false;
     int c = 0;  // stages of this tile processed (phases of s_full / p_full / o_bar)
     for (int n = 0;; ++n) {
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&meta_full[n % kMetaSlots], (n / kMetaSlots) & 1));
+      bool ok = __all_sync(0xffffffffu, pipe_wait(&meta_full[n % kMetaSlots], (n / kMetaSlots) & 1));
       const int4 mt = meta[n % kMetaSlots];
       __syncwarp();
       if (lane == 0) mbar_arrive(&meta_free[n % kMetaSlots]);
@@ -464,6 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int j = mt.w & 0x3ffff;
       const uint32_t mask = (mt.w >> 18) & 0xffu;
       const bool first = mt.w & kFirst, last = mt.w & kLast;
+      // causal: row0 = packed row, pos0 = its position; segment mode: row0 = partial id, mt.y = keys
       const int row0 = mt.x + t * a.tile_tokens, pos0 = mt.y + t * a.tile_tokens;
       if (first) {
         m_used = -INFINITY;
@@ -472,14 +500,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       }
       const int tl = m >> a.group_shift;
       const bool valid_row = tl < ntok;
-      const int limit = pos0 + (valid_row ? tl : ntok - 1);  // last visible key position
+      const int limit = SEG ? mt.y - 1 : pos0 + (valid_row ? tl : ntok - 1);  // last visible key position
       const int kbase = j * kKeys;
-      const int nvalid = min(kKeys, mt.y + ntok_a + ntok_b - kbase);
+      const int nvalid = min(kKeys, (SEG ? mt.y : mt.y + ntok_a + ntok_b) - kbase);
       if (t == 0 && (nvalid < kKeys || mask != 0xffu)) {
         // V rows past the context or in a slice that was not loaded may hold anything
         // (even NaN): zero them once the stage's copies have landed, before P·V.
         const int vs = n % kVStages;
-        ok &= mbar_wait(&v_full[vs], (n / kVStages) & 1);
+        ok &= pipe_wait(&v_full[vs], (n / kVStages) & 1);
         if (m >= nvalid || !((mask >> (m / kChunk)) & 1u)) {
           unsigned char* vrow = v_ring + vs * kTileBytes + m * 128;
 #pragma unroll
@@ -490,14 +518,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         fence_proxy_async_smem();
       }
       // ---- S row (its arrival also means every earlier MMA of this tile is done)
-      ok &= mbar_wait(&s_full[t], c & 1);
+      ok &= pipe_wait(&s_full[t], c & 1);
       tc::tc_fence_after();
       float s[kKeys];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) tc::tmem_load32f_nowait(tmem + lane_base + col_s + q4 * 32, s + q4 * 32);
       tc::tmem_wait_ld();
       // ---- causal / context mask and the row maximum
-      if (!(kbase + kKeys - 1 <= pos0 && mask == 0xffu)) {
+      if (!(kbase + kKeys - 1 <= (SEG ? mt.y - 1 : pos0) && mask == 0xffu)) {
 #pragma unroll
         for (int k = 0; k < kKeys; ++k) {
           const bool vis = kbase + k <= limit && ((mask >> (k / kChunk)) & 1u);
@@ -547,8 +575,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float x0 = s[h * 32 + 2 * i], x1 = s[h * 32 + 2 * i + 1];
-          const float p0 = any ? fast_exp2(fmaf(x0, a.scale_log2, neg_m)) : 0.f;
-          const float p1 = any ? fast_exp2(fmaf(x1, a.scale_log2, neg_m)) : 0.f;
+          // one pair in kPolyEvery takes the FMA-pipe exponential, the rest the SFU's
+          const bool poly = kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1;
+          const float e0 = fmaf(x0, a.scale_log2, neg_m), e1 = fmaf(x1, a.scale_log2, neg_m);
+          const float p0 = any ? (poly ? tc::poly_exp2(e0) : fast_exp2(e0)) : 0.f;
+          const float p1 = any ? (poly ? tc::poly_exp2(e1) : fast_exp2(e1)) : 0.f;
           w[i] = pack_bf16x2(p0, p1);
           ls8[(2 * i) & 7] += bf16lo(w[i]);
           ls8[(2 * i + 1) & 7] += bf16hi(w[i]);
@@ -564,17 +595,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       ++c;
       if (last) {
         // ---- epilogue: O / l of this row, once the item's last P·V is done
-        ok &= mbar_wait(&o_bar[t], (c - 1) & 1);
+        ok &= pipe_wait(&o_bar[t], (c - 1) & 1);
         tc::tc_fence_after();
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         const int64_t orow = (static_cast<int64_t>(row0 + tl) * a.num_heads + kvh * g + (m & (g - 1))) * kD;
+        if constexpr (SEG) {
+          if (valid_row) a.part_ml[orow / kD] = make_float2(m_used, lsum);
+        }
         uint32_t r[32];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           tc::tmem_load32_nowait(tmem + lane_base + col_o + q4 * 32, r);
           tc::tmem_wait_ld();
           if (valid_row) {
-            if constexpr (OUT_F32) {
+            if constexpr (SEG) {
+              float4* dst = reinterpret_cast<float4*>(a.part_o + orow + q4 * 32);
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                dst[k] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                                     __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+            } else if constexpr (OUT_F32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow + q4 * 32);
 #pragma unroll
               for (int k = 0; k < 8; ++k)
@@ -740,9 +780,9 @@ static int encode_q_map(CUtensorMap* map, const void* base, int total_q, int num
   return PKV_OK;
 }
 
-template <bool OUT_F32>
+template <bool OUT_F32, bool SEG = false>
 static int launch_main(const Args& args, int grid, cudaStream_t stream) {
-  auto kernel = prefill_tc_kernel<OUT_F32>;
+  auto kernel = prefill_tc_kernel<OUT_F32, SEG>;
   static PerDevice<int> setup;
   int dev = 0;
   const int st = set_smem_limit_once(setup, kernel, kSmemBytes, &dev);
@@ -760,6 +800,41 @@ static int max_entries(int num_seqs, int total_q, int group) {
 }
 
 }  // namespace pf
+
+int launch_prefill_segments(const SegmentLaunch& L, cudaStream_t s) {
+  const int group = L.num_heads / L.num_kv_heads;
+  pf::Args args;
+  pf::PrefillArgs& a = args.a;
+  a.out = nullptr;
+  a.block_tables = L.block_tables;
+  a.plan_count = L.plan_count;
+  a.entries = L.entries;
+  a.parts = L.parts;
+  a.part_o = L.part_o;
+  a.part_ml = L.part_ml;
+  a.status = L.status;
+  a.max_blocks = L.max_blocks;
+  a.num_heads = L.num_heads;
+  a.num_kv_heads = L.num_kv_heads;
+  a.block_size = L.block_size;
+  a.num_blocks = L.num_blocks;
+  a.group = group;
+  a.group_shift = __builtin_ctz(static_cast<unsigned>(group));
+  a.tile_tokens = pf::kRows / group;
+  a.scale_log2 = L.scale * 1.4426950408889634f;
+  const uint64_t pool_rows = static_cast<uint64_t>(L.num_blocks) * L.num_kv_heads * L.block_size;
+  int rc = pf::encode_kv_map(&args.tm_k, L.key_cache, pool_rows, "key_cache");
+  if (rc == PKV_OK) rc = pf::encode_kv_map(&args.tm_v, L.value_cache, pool_rows, "value_cache");
+  if (rc == PKV_OK) rc = pf::encode_q_map(&args.tm_q, L.query, L.num_seqs, L.num_heads, group);
+  if (rc != PKV_OK) return rc;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t items = static_cast<int64_t>(L.num_entries) * L.num_kv_heads;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, items)));
+  return pf::launch_main<true, true>(args, grid, s);
+}
+
 }  // namespace pkv
 
 using namespace pkv;
@@ -863,5 +938,5 @@ extern "C" int pkv_paged_attention_prefill(void* out, int out_dtype, const void*
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t items = static_cast<int64_t>(pf::max_entries(num_seqs, total_q, group)) * num_kv_heads;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, items)));
-  return p.out_f32 ? pf::launch_main<true>(args, grid, s) : pf::launch_main<false>(args, grid, s);
+  return p.out_f32 ? pf::launch_main<true, false>(args, grid, s) : pf::launch_main<false, false>(args, grid, s);
 }

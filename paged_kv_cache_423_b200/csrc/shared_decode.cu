@@ -1,0 +1,371 @@
+// Shared-prefix decode: the run of a plan made by pkv_shared_plan (shared_plan.cpp).
+//
+// Blocks that adjacent rows hold in common (a shared system prompt, a parent's blocks in
+// its beams; Outcome School explainer, "内存共享") are attended to once per kv head for
+// all of those rows, as one dense contraction on the tensor cores; each row's private
+// remainder goes through the tensor-core decode; a merge combines the partial results
+// by log-sum-exp rescaling, which reproduces softmax attention over the whole context
+// (intelliparadigm article "PagedAttention：操作系统分页思想的跨界创新" §2.1).
+//
+// Launches, in order on the caller's stream:
+//   shared_setup_kernel   checks the plan against the call (sizes, ranges, that every
+//                         row's shared tokens plus its remainder equal its context
+//                         length) and writes checked copies of the remainders; a plan
+//                         that does not fit sets PKV_DEV_BAD_CONTEXT and every output
+//                         row becomes zero
+//   prefill_tc_kernel     segment mode: all query heads of a part's rows against the
+//                         part's keys, unnormalised partials (o, m, l)
+//   plan_kernel +
+//   decode_gqa_tc_kernel  the remainders, every item writing its partial
+//   shared_merge_kernel   out = sum 2^(m_i - M) o_i / sum 2^(m_i - M) l_i per (row, head)
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "decode_common.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+namespace sp {
+
+constexpr int kD = 128;
+constexpr int kSetupThreads = 1024;
+constexpr int kMergeWarps = 4;
+
+struct Layout {
+  size_t off_count = 0, off_lens = 0, off_offset = 0, off_seg_o = 0, off_seg_ml = 0, off_decode = 0, total = 0;
+  WorkspaceLayout dec;
+  int partition = 0;
+};
+
+// Workspace: [plan count, work counter, bad flag] | checked remainders | checked block offsets |
+// shared partials (o, then (m, l)) | the private phase's decode workspace (partials forced).
+static Layout layout(const pkv_shared_plan_info& in, int num_heads, int num_kv_heads) {
+  Layout L;
+  const int B = in.num_seqs;
+  L.partition = auto_partition_tokens_tensor(B, num_kv_heads, in.block_size, in.max_suffix_len);
+  size_t off = 0;
+  L.off_count = off;
+  off = align256(off + 4 * sizeof(int32_t));
+  L.off_lens = off;
+  off = align256(off + static_cast<size_t>(B) * sizeof(int32_t));
+  L.off_offset = off;
+  off = align256(off + static_cast<size_t>(B) * sizeof(int32_t));
+  L.off_seg_o = off;
+  off = align256(off + static_cast<size_t>(in.num_partials) * num_heads * kD * sizeof(float));
+  L.off_seg_ml = off;
+  off = align256(off + static_cast<size_t>(in.num_partials) * num_heads * sizeof(float2));
+  L.off_decode = off;
+  L.dec = workspace_layout(B, num_heads, kD, in.max_suffix_len, L.partition, true);
+  L.total = off + L.dec.total;
+  return L;
+}
+
+struct SetupArgs {
+  const int4* entries;
+  const int4* parts;
+  const int32_t* suffix_lens;
+  const int32_t* block_offset;
+  const int32_t* row_start;
+  const int32_t* row_ids;
+  const int32_t* context_lens;
+  int32_t* count;          // [0] shared-phase entries, [1] its work counter, [2] bad plan
+  int32_t* v_lens;         // checked remainders (0 for every row of a bad plan)
+  int32_t* v_offset;
+  int32_t* status;
+  int num_seqs, num_entries, num_parts, num_partials, max_blocks, block_size, tile_rows, max_suffix_len;
+};
+
+__global__ void __launch_bounds__(kSetupThreads) shared_setup_kernel(const SetupArgs p) {
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  bool mine = false;
+  for (int i = threadIdx.x; i < p.num_parts; i += blockDim.x) {
+    const int4 d0 = p.parts[2 * i], d1 = p.parts[2 * i + 1];
+    const int64_t nblk = d0.z >= 1 ? (static_cast<int64_t>(d0.z) + p.block_size - 1) / p.block_size : 0;
+    mine |= d0.x < 0 || d0.x >= p.num_seqs || d0.y < 0 || d0.z < 1 || d0.y + nblk > p.max_blocks || d0.w < 0 ||
+            d1.x < 1 || static_cast<int64_t>(d0.w) + d1.x > p.num_seqs || d1.y < 0 ||
+            static_cast<int64_t>(d1.y) + d1.x > p.num_partials;
+  }
+  for (int i = threadIdx.x; i < p.num_entries; i += blockDim.x) {
+    const int4 e = p.entries[i];
+    if (e.w < 0 || e.w >= p.num_parts) {
+      mine = true;
+      continue;
+    }
+    const int4 d0 = p.parts[2 * e.w], d1 = p.parts[2 * e.w + 1];
+    const int na = e.z & 0xff, nb = (e.z >> 8) & 0xff;
+    mine |= (e.z >> 16) != 0 || na < 1 || na > p.tile_rows || nb > p.tile_rows || (nb > 0 && na != p.tile_rows) ||
+            e.x < d0.w || static_cast<int64_t>(e.x) + na + nb > static_cast<int64_t>(d0.w) + d1.x;
+  }
+  for (int r = threadIdx.x; r < p.num_seqs; r += blockDim.x) {
+    const int off = p.block_offset[r], sl = p.suffix_lens[r], L = p.context_lens[r];
+    const bool ok = off >= 0 && off <= p.max_blocks && sl >= 0 && sl <= p.max_suffix_len &&
+                    static_cast<int64_t>(sl) <= static_cast<int64_t>(p.max_blocks - off) * p.block_size &&
+                    static_cast<int64_t>(off) * p.block_size + sl == L;
+    mine |= !ok;
+    const int a = p.row_start[r], b = p.row_start[r + 1];
+    mine |= a < 0 || b < a || b > p.num_partials || (r == 0 && a != 0) ||
+            (r == p.num_seqs - 1 && b != p.num_partials);
+    if (a >= 0 && b <= p.num_partials)
+      for (int k = a; k < b; ++k) mine |= p.row_ids[k] < 0 || p.row_ids[k] >= p.num_partials;
+  }
+  if (mine) atomicOr(&bad, 1);
+  __syncthreads();
+  for (int r = threadIdx.x; r < p.num_seqs; r += blockDim.x) {
+    p.v_lens[r] = bad ? 0 : p.suffix_lens[r];
+    p.v_offset[r] = bad ? 0 : p.block_offset[r];
+  }
+  if (threadIdx.x == 0) {
+    p.count[0] = bad ? 0 : p.num_entries;
+    p.count[1] = 0;
+    p.count[2] = bad;
+    if (bad) set_status(p.status, PKV_DEV_BAD_CONTEXT);
+  }
+}
+
+struct MergeArgs {
+  void* out;
+  const float* dec_o;       // private phase partials [row * Hq + h][max_parts][128]
+  const float2* dec_ml;
+  const float* seg_o;       // shared partials [id][h][128]
+  const float2* seg_ml;
+  const int32_t* v_lens;
+  const int32_t* row_start;
+  const int32_t* row_ids;
+  const int32_t* bad;
+  int num_seqs, num_heads, partition, max_parts;
+};
+
+// One warp per (row, head); lane l owns output values 4l .. 4l+3.
+template <bool OUT_F32>
+__global__ void __launch_bounds__(kMergeWarps * 32) shared_merge_kernel(const MergeArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kMergeWarps + warp;
+  if (unit >= static_cast<int64_t>(a.num_seqs) * a.num_heads) return;
+  const int r = static_cast<int>(unit / a.num_heads), h = static_cast<int>(unit % a.num_heads);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float Ls = 0.f;
+  if (*a.bad == 0) {
+    const int sl = a.v_lens[r];
+    const int np = sl == 0 ? 1 : (sl + a.partition - 1) / a.partition;
+    const int s0 = a.row_start[r], s1 = a.row_start[r + 1];
+    const float2* dml = a.dec_ml + unit * a.max_parts;
+    float M = -INFINITY;
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, dml[p].x);
+    for (int k = s0 + lane; k < s1; k += 32) M = fmaxf(M, a.seg_ml[static_cast<int64_t>(a.row_ids[k]) * a.num_heads + h].x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    auto add = [&](float2 ml, const float* o) {
+      const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+      Ls = fmaf(w, ml.y, Ls);
+      const float4 v = *reinterpret_cast<const float4*>(o + lane * 4);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    };
+    for (int p = 0; p < np; ++p) add(dml[p], a.dec_o + (unit * a.max_parts + p) * kD);
+    for (int k = s0; k < s1; ++k) {
+      const int64_t id = static_cast<int64_t>(a.row_ids[k]) * a.num_heads + h;
+      add(a.seg_ml[id], a.seg_o + id * kD);
+    }
+  }
+  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+  const int64_t o = unit * kD + lane * 4;
+  if constexpr (OUT_F32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(a.out) + o) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  } else {
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + o) =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+  }
+}
+
+}  // namespace sp
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" size_t pkv_paged_attention_decode_shared_workspace_size(const pkv_shared_plan_info* info, int num_heads,
+                                                                   int num_kv_heads, int head_dim) {
+  if (!info || info->num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim != sp::kD ||
+      info->num_partials < 0 || info->max_suffix_len < 0 || (info->block_size != 16 && info->block_size != 32))
+    return 0;
+  return sp::layout(*info, num_heads, num_kv_heads).total;
+}
+
+extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const void* query, const void* key_cache,
+                                                 const void* value_cache, const int32_t* block_tables,
+                                                 int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                                 int num_blocks, float scale, const void* plan,
+                                                 const pkv_shared_plan_info* info, void* workspace,
+                                                 size_t workspace_bytes, int32_t* status, pkv_stream_t stream) {
+  clear_error();
+  if (!info) return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: null info");
+  const pkv_shared_plan_info& in = *info;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: bad sizes");
+  if (out_dtype != PKV_DTYPE_BF16 && out_dtype != PKV_DTYPE_F32)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: out_dtype %d", out_dtype);
+  if (block_size != 16 && block_size != 32)
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_shared: block_size %d not in {16,32}", block_size);
+  if (num_heads % num_kv_heads != 0 || !tensor_path_supports(num_heads / num_kv_heads, head_dim))
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_shared: needs head_dim 128 and 2 <= num_heads / "
+                     "num_kv_heads <= 16 (got %d, %d / %d)", head_dim, num_heads, num_kv_heads);
+  if (num_kv_heads >= (1 << 15))
+    return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_shared: num_kv_heads %d", num_kv_heads);
+  const int group = num_heads / num_kv_heads;
+  if (in.num_seqs != num_seqs || in.group != group || in.block_size != block_size ||
+      in.max_blocks_per_seq != max_blocks_per_seq || in.num_entries < 0 || in.num_parts < 0 ||
+      in.num_partials < 0 || in.max_suffix_len < 0 || in.max_suffix_len > max_blocks_per_seq * block_size)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: the plan was made for other sizes");
+  if (static_cast<int64_t>(num_blocks) * num_kv_heads * block_size > (static_cast<int64_t>(1) << 31))
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: pool too large");
+  if (static_cast<int64_t>(in.num_entries) * num_kv_heads > (int64_t{1} << 30))
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: too many shared-phase entries");
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !plan || !workspace)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: null pointer");
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(plan))
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: tensors and the plan must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: workspace must be 256-byte aligned");
+  const uint64_t offs[] = {in.off_entries, in.off_parts, in.off_suffix_lens, in.off_block_offset, in.off_row_start,
+                           in.off_row_ids};
+  for (uint64_t o : offs)
+    if (o % 16 != 0 || o > in.bytes) return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: bad plan offsets");
+  if (in.off_entries + static_cast<uint64_t>(in.num_entries) * 16 > in.bytes ||
+      in.off_parts + static_cast<uint64_t>(in.num_parts) * 32 > in.bytes ||
+      in.off_suffix_lens + static_cast<uint64_t>(num_seqs) * 4 > in.bytes ||
+      in.off_block_offset + static_cast<uint64_t>(num_seqs) * 4 > in.bytes ||
+      in.off_row_start + static_cast<uint64_t>(num_seqs + 1) * 4 > in.bytes ||
+      in.off_row_ids + static_cast<uint64_t>(in.num_partials) * 4 > in.bytes)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: plan sections exceed its size");
+  const sp::Layout L = sp::layout(in, num_heads, num_kv_heads);
+  if (workspace_bytes < L.total)
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: workspace of %zu bytes, %zu needed",
+                     workspace_bytes, L.total);
+
+  const unsigned char* pl = static_cast<const unsigned char*>(plan);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* count = reinterpret_cast<int32_t*>(ws + L.off_count);
+  int32_t* v_lens = reinterpret_cast<int32_t*>(ws + L.off_lens);
+  int32_t* v_offset = reinterpret_cast<int32_t*>(ws + L.off_offset);
+  float* seg_o = reinterpret_cast<float*>(ws + L.off_seg_o);
+  float2* seg_ml = reinterpret_cast<float2*>(ws + L.off_seg_ml);
+  unsigned char* dws = ws + L.off_decode;
+  const int4* entries = reinterpret_cast<const int4*>(pl + in.off_entries);
+  const int4* parts = reinterpret_cast<const int4*>(pl + in.off_parts);
+  const int32_t* row_start = reinterpret_cast<const int32_t*>(pl + in.off_row_start);
+  const int32_t* row_ids = reinterpret_cast<const int32_t*>(pl + in.off_row_ids);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // ---- check the plan against the call
+  sp::SetupArgs sa{};
+  sa.entries = entries;
+  sa.parts = parts;
+  sa.suffix_lens = reinterpret_cast<const int32_t*>(pl + in.off_suffix_lens);
+  sa.block_offset = reinterpret_cast<const int32_t*>(pl + in.off_block_offset);
+  sa.row_start = row_start;
+  sa.row_ids = row_ids;
+  sa.context_lens = context_lens;
+  sa.count = count;
+  sa.v_lens = v_lens;
+  sa.v_offset = v_offset;
+  sa.status = status;
+  sa.num_seqs = num_seqs;
+  sa.num_entries = in.num_entries;
+  sa.num_parts = in.num_parts;
+  sa.num_partials = in.num_partials;
+  sa.max_blocks = max_blocks_per_seq;
+  sa.block_size = block_size;
+  sa.tile_rows = 128 / group;
+  sa.max_suffix_len = in.max_suffix_len;
+  sp::shared_setup_kernel<<<1, sp::kSetupThreads, 0, s>>>(sa);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "shared setup launch: %s", cudaGetErrorString(e));
+
+  // ---- shared phase
+  if (in.num_entries > 0) {
+    SegmentLaunch sl{};
+    sl.query = query;
+    sl.key_cache = key_cache;
+    sl.value_cache = value_cache;
+    sl.block_tables = block_tables;
+    sl.plan_count = count;
+    sl.entries = entries;
+    sl.parts = parts;
+    sl.part_o = seg_o;
+    sl.part_ml = seg_ml;
+    sl.status = status;
+    sl.num_entries = in.num_entries;
+    sl.max_blocks = max_blocks_per_seq;
+    sl.num_seqs = num_seqs;
+    sl.num_heads = num_heads;
+    sl.num_kv_heads = num_kv_heads;
+    sl.block_size = block_size;
+    sl.num_blocks = num_blocks;
+    sl.scale = scale;
+    const int rc = launch_prefill_segments(sl, s);
+    if (rc != PKV_OK) return rc;
+  }
+
+  // ---- private phase: the remainders through the tensor-core decode, partials only
+  DecodeArgs a{};
+  a.out = out;
+  a.query = static_cast<const __nv_bfloat16*>(query);
+  a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
+  a.value_cache = static_cast<const __nv_bfloat16*>(value_cache);
+  a.block_tables = block_tables;
+  a.plan_count = reinterpret_cast<const int32_t*>(dws + L.dec.off_count);
+  a.entries = reinterpret_cast<const PlanEntry*>(dws + L.dec.off_entries);
+  a.arrive = reinterpret_cast<int32_t*>(dws + L.dec.off_arrive);
+  a.part_o = reinterpret_cast<float*>(dws + L.dec.off_part_o);
+  a.part_ml = reinterpret_cast<float2*>(dws + L.dec.off_part_ml);
+  a.status = status;
+  a.context_lens = v_lens;
+  a.max_context_len = in.max_suffix_len;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.group = group;
+  a.partition = L.partition;
+  a.max_parts = L.dec.max_parts;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.block_offset = v_offset;
+  a.always_partial = 1;
+  int rc = launch_decode_plan(a, v_lens, in.max_suffix_len, s);
+  if (rc == PKV_OK) rc = launch_decode_tensor(a, head_dim, out_dtype == PKV_DTYPE_F32, s);
+  if (rc != PKV_OK) return rc;
+
+  // ---- merge
+  sp::MergeArgs m{};
+  m.out = out;
+  m.dec_o = a.part_o;
+  m.dec_ml = a.part_ml;
+  m.seg_o = seg_o;
+  m.seg_ml = seg_ml;
+  m.v_lens = v_lens;
+  m.row_start = row_start;
+  m.row_ids = row_ids;
+  m.bad = count + 2;
+  m.num_seqs = num_seqs;
+  m.num_heads = num_heads;
+  m.partition = L.partition;
+  m.max_parts = L.dec.max_parts;
+  const int64_t units = static_cast<int64_t>(num_seqs) * num_heads;
+  const unsigned grid = static_cast<unsigned>((units + sp::kMergeWarps - 1) / sp::kMergeWarps);
+  if (out_dtype == PKV_DTYPE_F32)
+    sp::shared_merge_kernel<true><<<grid, sp::kMergeWarps * 32, 0, s>>>(m);
+  else
+    sp::shared_merge_kernel<false><<<grid, sp::kMergeWarps * 32, 0, s>>>(m);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "shared merge launch: %s", cudaGetErrorString(e));
+  return PKV_OK;
+}

@@ -138,6 +138,27 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for softmax weights x = score - held maximum (x <= 8 here), to take part
+// of the exponentials off the SFU.  Range reduction: x = j + f, j = rint(x) from the 1.5 * 2^23
+// rounding add (j lands in the sum's low mantissa bits), f = x - j in [-1/2, 1/2] exactly.  2^f is
+// a cubic 1 + f (c1 + f (c2 + f c3)) whose coefficients minimise the largest relative error over
+// [-1/2, 1/2] with p(0) = 1 (a linear-programming fit over a dense grid of f): relative error at
+// most 1.02e-4, exact at integers.  2^j is added to the exponent field as j << 23.  Inputs at or
+// below -127 (and -inf) give +0; results below 2^-126 are not accurate (they only feed bf16
+// weights next to a weight of about 1).
+constexpr float kExp2C1 = 0.6932829f;
+constexpr float kExp2C2 = 0.24221095f;
+constexpr float kExp2C3 = 0.05500893f;
+__device__ __forceinline__ float poly_exp2(float x) {
+  x = fmaxf(x, -127.f);
+  const float t = x + 12582912.f;  // 1.5 * 2^23
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(f, kExp2C3, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, 1.f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, A and B both bf16 (or both f16),
 // A/B major-ness, N >> 3 and M >> 4.
 __host__ __device__ constexpr uint32_t instr_desc(int m, int n, bool a_mn_major, bool b_mn_major, bool f16 = false) {

@@ -364,7 +364,7 @@ def test_e2e_host_logic_with_stand_in_streams(pkv, monkeypatch):
         assert k.shape == (w.B, w.Hkv, w.D) and slots.shape == (w.B,)
         calls["write"] += 1
 
-    def decode(out, q, tables, lens, max_len, ws, path, status):
+    def decode(out, q, tables, lens, max_len, ws, path, status, shared=None):
         assert q.shape == (w.B, w.Hq, w.D) and tables.shape == (w.B, w.max_blocks) and lens.shape == (w.B,)
         out.fill_(1.0)
         calls["decode"] += 1
@@ -625,3 +625,19 @@ def test_reference_prefill_batch_without_the_library(pkv, monkeypatch):
     assert ref.pkv is None and ref.ws is None
     for k in ("slots", "tables", "lens", "qstart"):
         assert torch.equal(getattr(native, k), getattr(ref, k)), k
+
+
+def test_shared_decode_applies_only_where_it_can_run():
+    import types
+    args = lambda shared="auto", path="auto": types.SimpleNamespace(shared=shared, path=path)  # noqa: E731
+    w = lambda kv8=False, shared_blocks=64, Hq=32, Hkv=8, D=128: types.SimpleNamespace(  # noqa: E731
+        kv8=kv8, shared_blocks=shared_blocks, Hq=Hq, Hkv=Hkv, D=D)
+    assert bench.shared_decode_applies(args(), w())                    # the shared-prompt batch
+    assert not bench.shared_decode_applies(args(), w(shared_blocks=0))  # nothing shared: plain decode
+    assert bench.shared_decode_applies(args("on"), w(shared_blocks=0))
+    assert not bench.shared_decode_applies(args("off"), w())
+    assert not bench.shared_decode_applies(args(), w(kv8=True))        # bf16 pools only
+    assert not bench.shared_decode_applies(args(path="simt"), w())
+    assert not bench.shared_decode_applies(args(), w(Hq=40, Hkv=40))   # MHA: no tensor-core decode
+    with pytest.raises(SystemExit):
+        bench.shared_decode_applies(args("on"), w(Hq=40, Hkv=40))

@@ -743,12 +743,9 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
         if len(pairs):
             hm[o_pairs:o_pairs + pairs.nbytes] = pairs.reshape(-1).view(np.uint8)
         plan_bytes = 0
-        if sws is not None:
-            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs)
+        if sws is not None:  # planned straight into the pinned buffer (raises if it outgrew it)
+            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs, out=hm[o_plan:o_plan + plan_cap])
             plan_bytes = plan_h.nbytes
-            if plan_bytes > plan_cap:
-                raise RuntimeError("e2e: a step's shared-prefix plan outgrew the pinned buffer")
-            hm[o_plan:o_plan + plan_bytes] = plan_h
         with torch.cuda.stream(copy):
             if i >= 2:
                 copy.wait_event(comp_done[i - 2])  # device buffers b are free again

@@ -331,7 +331,7 @@ PKV_API int pkv_paged_attention_prefill(void* out, int out_dtype, const void* qu
  *                  (0 <= L <= max_blocks_per_seq * block_size, else PKV_ERR_INVALID)
  *   min_rows       fewest rows a segment serves (>= 2)
  *   key_chunk      tokens per part of a segment: a multiple of 128, or 0 = automatic
- *                  (the largest of 2048 .. 128 that still gives about two work items per SM)
+ *                  (the largest of 2048 .. 128 that gives at least 64 shared-phase work items)
  *   plan           host buffer of plan_bytes, or NULL to only fill `info` (info->bytes
  *                  is then the size to provide); too small a buffer is PKV_ERR_INVALID
  *   info           host, filled on success: counts and the byte offset of each section
@@ -371,7 +371,13 @@ PKV_API int pkv_shared_plan(const int32_t* block_tables, int max_blocks_per_seq,
  *   workspace   device, pkv_paged_attention_decode_shared_workspace_size() bytes, 256-byte aligned
  * bf16 pools only; head_dim 128; 2 <= num_heads / num_kv_heads <= 16 (the tensor-core
  * decode) — else PKV_ERR_UNSUPPORTED.  block_tables and context_lens must be those the
- * plan was made from (the private phase re-validates lengths and table entries).
+ * plan was made from: the call checks on the device that every row's shared tokens plus its
+ * remainder equal its context length (and the plan's ranges); a plan that does not fit sets
+ * PKV_DEV_BAD_CONTEXT and every output row is zero.
+ * The shared phase runs on a side stream of the library, forked from `stream` after the
+ * checks and joined back before the merge (event waits, so the call as a whole stays ordered
+ * on `stream`); the side stream and its two events are created on the first call on each
+ * device — make that call before any stream capture — and kept until the process exits.
  */
 PKV_API size_t pkv_paged_attention_decode_shared_workspace_size(const pkv_shared_plan_info* info, int num_heads,
                                                                 int num_kv_heads, int head_dim);

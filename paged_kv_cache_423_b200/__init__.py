@@ -470,10 +470,12 @@ def paged_attention_prefill(out, query, key_cache, value_cache, block_tables, qu
 # Host block manager
 # ---------------------------------------------------------------------------
 
-def shared_plan(block_tables, context_lens, num_heads, num_kv_heads, block_size, min_rows=2, key_chunk=0):
+def shared_plan(block_tables, context_lens, num_heads, num_kv_heads, block_size, min_rows=2, key_chunk=0, out=None):
     """Host plan of the shared-prefix decode from host tables [B, max_blocks] int32 and lengths
     [B] int32 (NumPy).  Returns (plan, info): plan a uint8 NumPy array of info.bytes bytes to
-    copy to the device, info a SharedPlanInfo."""
+    copy to the device, info a SharedPlanInfo.  With `out` (a contiguous uint8 NumPy array, for
+    example a view of pinned memory) the plan is written there in one call and a view of its
+    first info.bytes bytes is returned; too small a buffer raises."""
     tables = np.ascontiguousarray(block_tables, dtype=np.int32)
     lens = np.ascontiguousarray(context_lens, dtype=np.int32)
     if tables.ndim != 2 or lens.shape != (tables.shape[0],):
@@ -481,6 +483,12 @@ def shared_plan(block_tables, context_lens, num_heads, num_kv_heads, block_size,
     B, mb = tables.shape
     info = SharedPlanInfo()
     lib = library()
+    if out is not None:
+        if out.dtype != np.uint8 or out.ndim != 1 or not out.flags.c_contiguous:
+            raise ValueError("shared_plan: out must be a contiguous 1-D uint8 array")
+        _check(lib.pkv_shared_plan(_np_ptr(tables), mb, _np_ptr(lens), B, num_heads, num_kv_heads, block_size,
+                                   min_rows, key_chunk, _np_ptr(out), out.nbytes, ctypes.byref(info)), "shared_plan")
+        return out[:int(info.bytes)], info
     _check(lib.pkv_shared_plan(_np_ptr(tables), mb, _np_ptr(lens), B, num_heads, num_kv_heads, block_size, min_rows,
                                key_chunk, None, 0, ctypes.byref(info)), "shared_plan")
     plan = np.zeros(int(info.bytes), np.uint8)

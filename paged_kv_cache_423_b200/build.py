@@ -13,8 +13,7 @@ CUDA-core decode kernel's per-warp copy ring at one stage, so every copy waits f
 previous stage's compute; a test compares it bit for bit with the default build.
 
 ``variant="shortwait"`` builds ``libpkv_shortwait.so`` whose CUDA-core decode and prefill
-kernels give up a pipeline wait after a few hundred nanoseconds of polling instead of one
-second, so an ordinary launch takes its expiry path (flag PKV_DEV_TIMEOUT, let copies land,
+kernels give up a pipeline wait after one poll instead of one second, so an ordinary launch takes its expiry path (flag PKV_DEV_TIMEOUT, let copies land,
 wait for MMAs, free tensor memory, return); a test checks the flag and that the context
 stays usable.  No wait is removed and the drains keep their one-second limit.
 """

@@ -50,8 +50,8 @@ constexpr int kConsumers = 128;        // warps 0-3: softmax, one thread per TME
 constexpr int kProducerWarp = 4;       // TMA loads
 constexpr int kMmaWarp = 5;            // tcgen05.mma issue
 constexpr int kThreads = kConsumers + 64;
-constexpr int kTmemCols = 64;          // S double buffer in columns [0,16) and [16,32), O in [32,48)
-constexpr uint32_t kColO = 32;
+constexpr int kTmemCols = 64;          // S double buffer in columns [0,16) and [16,32), O of even / odd
+constexpr uint32_t kColO = 32;         // items in [32,48) and [48,64)
 constexpr uint32_t kChunkTx = 4 * kChunk * 128;  // K and V, two halves each
 
 struct alignas(64) Args {
@@ -72,9 +72,10 @@ struct Layout {
   static constexpr int off_q = off_v + STAGES * kTileBytes;
   static constexpr int off_p = off_q + kQSlots * 4096;    // q slots sized for N <= 16
   static constexpr int off_red = off_p + 2 * 4096;        // P double buffer: 2 K-atoms of N rows x 128 B each
-  static constexpr int off_meta = off_red + 2 * 4 * 16 * 4;
+  static constexpr int off_meta = off_red + 3 * 4 * 16 * 4;  // [maxima | sums of even items | odd items][4 warps][16]
   static constexpr int off_bar = off_meta + STAGES * 16;
-  static constexpr int kBars = 2 * STAGES + 8;            // full, empty, s_full[2], s_free[2], p_full[2], o_bar[2]
+  // full, empty, s_full[2], s_free[2], p_full[2], o_bar[2], drain
+  static constexpr int kBars = 2 * STAGES + 9;
   static constexpr int off_misc = off_bar + kBars * 8;
   static constexpr int bytes = off_misc + 32;
   static constexpr int alloc = bytes + 1024;              // slack to align the base to 1024
@@ -128,8 +129,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_bar = p_full + 2;
+  uint64_t* drain = o_bar + 2;  // the MMA thread's last commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::off_misc + 4);
+  // [P buffer]: bit 0 = the P·V starts a fresh accumulation, bit 1 = the O buffer of its item
   volatile int* restart_flag = reinterpret_cast<volatile int*>(smem + L::off_misc + 8);  // [2]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -147,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       mbar_init(&p_full[b], 4);
       mbar_init(&o_bar[b], 1);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -336,13 +340,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
             const int b = p_valid & 1;
             if (mbar_test(&p_full[b], (p_valid >> 1) & 1)) {
               tc_fence_after();
-              const bool restart = restart_flag[b] != 0;
+              const int rf = restart_flag[b];
+              const bool restart = rf & 1;
+              const uint32_t o_col = kColO + ((rf >> 1) & 1) * 16;
               const uint32_t v_addr = smem_addr(v_ring + slot * kTileBytes);
               const uint32_t p_addr = p_addr0 + b * 4096;
               const int kt = ((mt.w & 0xff) + 15) / 16;
               for (int kk = 0; kk < kt; ++kk) {
                 // P: MN-major, unswizzled; 8-token groups 128 B apart, heads 8..15 2 KiB on
-                umma(tmem + kColO, smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024),
+                umma(tmem + o_col, smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024),
                      smem_desc_plain(p_addr + kk * 256, 128, 2048), idesc_pv, kk > 0 || !restart);
               }
               umma_commit(&o_bar[b]);
@@ -369,6 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           }
         }
       }
+      // every MMA this thread issued has finished before tensor memory is freed
+      umma_commit(drain);
+      mbar_wait(drain, 0);
     }
     __syncwarp();
   } else {
@@ -380,6 +389,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
     bool restart = true;           // the next P·V starts a fresh TMEM accumulation
     bool pv_since_restart = false;
     int n_valid_tiles = 0;
+    int obuf = 1;  // O buffer of the current item (alternates per item)
+    // An item's output is written one tile later, after the next tile's P is released, so
+    // its last P·V completes meanwhile instead of being waited for.
+    bool fin = false;
+    int4 f_mt = make_int4(0, 0, 0, 0);
+    float f_o[N], f_lp[N], f_m[N];
+    int f_ob = 0, f_b = 0;
+    bool f_has_o = false;
     uint32_t ob_next = 0;     // bit b: parity of the phase the next P·V on o_bar[b] completes
     uint32_t ob_pending = 0;  // bit b: the last P·V on o_bar[b] has not been waited for yet
     auto wait_ob = [&](int b) -> bool {
@@ -388,11 +405,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       return mbar_wait(&o_bar[b], ((ob_next >> b) & 1) ^ 1u);
     };
 
+    // ---- the held item's output: O = registers + TMEM, denominators, output or partial
+    auto finalize = [&]() {
+      fin = false;
+      bool ok = true;
+      float ot[N];
+      if (f_has_o) {
+        ok = wait_ob(f_b);  // its last P·V (the latest on P buffer f_b)
+        tc_fence_after();
+        float o[N];
+        tmem_load_row<N>(tmem + lane_base + kColO + f_ob * 16, o);
+        tc_fence_before();
+#pragma unroll
+        for (int h = 0; h < N; ++h) ot[h] = f_o[h] + o[h];
+      } else {
+#pragma unroll
+        for (int h = 0; h < N; ++h) ot[h] = f_o[h];
+      }
+      if (!ok) *abort_flag = 1;
+      float* red2 = red + 64 + f_ob * 64;  // consecutive items use different halves
+      const float wsum = warp_col16<false>(f_lp, lane);
+      if ((lane & 1) == 0) red2[warp * 16 + (lane >> 1)] = wsum;
+      named_barrier_sync(1, kConsumers);
+      const int seq = f_mt.x, kvh = f_mt.y & 0xffff, part = f_mt.z & 0xffff, nparts = f_mt.z >> 16;
+      const int d = tid;
+      const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
+#pragma unroll
+      for (int h = 0; h < N; ++h) {
+        if (h >= g) break;
+        const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
+        if (nparts == 1 && !a.always_partial) {
+          store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[h] / l : 0.f);
+        } else {
+          // unnormalised partial; a separate kernel merges the partitions
+          const int64_t pidx = (unit0 + h) * a.max_parts + part;
+          a.part_o[pidx * kD + d] = ot[h];
+          if (d == 0) a.part_ml[pidx] = make_float2(f_m[h], l);
+        }
+      }
+    };
+    bool ended = false;
+
     for (int n = 0;; ++n) {
       const int slot = n % STAGES;
       bool bad = !mbar_wait(&full[slot], (n / STAGES) & 1);
       const int4 mt = meta[slot];
-      if (mt.w & kMetaEnd) break;
+      if (mt.w & kMetaEnd) {
+        ended = true;
+        break;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
       const int n_valid = mt.w & 0xff;
@@ -403,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         for (int h = 0; h < N; ++h) m_used[h] = -INFINITY, lp[h] = 0.f, o_reg[h] = 0.f;
         restart = true;
         pv_since_restart = false;
+        obuf ^= 1;
       }
       if (n_valid > 0) {
         const int b = n_valid_tiles & 1;
@@ -453,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         bool need_any = true;  // an item's first tile always sets the held maximum
         if (!first) {
           write_p();
-          if (tid == 0) restart_flag[b] = restart;
+          if (tid == 0) restart_flag[b] = (restart ? 1 : 0) | (obuf << 1);
           fence_proxy_async_smem();
           need_any = named_barrier_or(1, kConsumers, need || bad);
           if (*abort_flag) break;
@@ -464,8 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           // (re)write P.
           const float wmax = warp_col16<true>(x, lane);
           if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = wmax;
-          bool ok = wait_ob(0);
-          ok &= wait_ob(1);
+          bool ok = true;
+          if (pv_since_restart) {  // this item's O is folded below: its P·Vs must be complete
+            ok = wait_ob(0);
+            ok &= wait_ob(1);
+          }
           if (!ok) *abort_flag = 1;
           named_barrier_sync(1, kConsumers);
           if (*abort_flag) break;
@@ -485,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           tc_fence_after();
           if (pv_since_restart) {
             float o[N];
-            tmem_load_row<N>(tmem + lane_base + kColO, o);
+            tmem_load_row<N>(tmem + lane_base + kColO + obuf * 16, o);
 #pragma unroll
             for (int h = 0; h < N; ++h) o_reg[h] = (o_reg[h] + o[h]) * alpha[h];
           } else {
@@ -498,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
           restart = true;
           pv_since_restart = false;
           write_p();
-          if (tid == 0) restart_flag[b] = 1;
+          if (tid == 0) restart_flag[b] = 1 | (obuf << 1);
           fence_proxy_async_smem();
           named_barrier_sync(1, kConsumers);
         }
@@ -513,46 +578,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         pv_since_restart = true;
         ++n_valid_tiles;
       }
+      if (fin) finalize();  // the previous item: its last P·V ran while this tile was processed
       if (last) {
-        // ---- finalize the item: O = registers + TMEM, denominators, output or partial
-        bool ok = wait_ob(0);
-        ok &= wait_ob(1);
-        tc_fence_after();
-        float ot[N];
-        if (pv_since_restart) {
-          float o[N];
-          tmem_load_row<N>(tmem + lane_base + kColO, o);
+        fin = true;
+        f_mt = mt;
 #pragma unroll
-          for (int h = 0; h < N; ++h) ot[h] = o_reg[h] + o[h];
-        } else {
-#pragma unroll
-          for (int h = 0; h < N; ++h) ot[h] = o_reg[h];
-        }
-        tc_fence_before();
-        if (!ok) *abort_flag = 1;
-        float* red2 = red + 64;
-        const float wsum = warp_col16<false>(lp, lane);
-        if ((lane & 1) == 0) red2[warp * 16 + (lane >> 1)] = wsum;
-        named_barrier_sync(1, kConsumers);
-        const int seq = mt.x, kvh = mt.y & 0xffff, part = mt.z & 0xffff, nparts = mt.z >> 16;
-        const int d = tid;
-        const int64_t unit0 = static_cast<int64_t>(seq) * a.num_heads + kvh * g;
-#pragma unroll
-        for (int h = 0; h < N; ++h) {
-          if (h >= g) break;
-          const float l = red2[h] + red2[16 + h] + red2[32 + h] + red2[48 + h];
-          if (nparts == 1 && !a.always_partial) {
-            store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[h] / l : 0.f);
-          } else {
-            // unnormalised partial; a separate kernel merges the partitions
-            const int64_t pidx = (unit0 + h) * a.max_parts + part;
-            a.part_o[pidx * kD + d] = ot[h];
-            if (d == 0) a.part_ml[pidx] = make_float2(m_used[h], l);
-          }
-        }
-        // red2 is rewritten only after the next item's barriers
+        for (int h = 0; h < N; ++h) f_o[h] = o_reg[h], f_lp[h] = lp[h], f_m[h] = m_used[h];
+        f_ob = obuf;
+        f_has_o = pv_since_restart;
+        f_b = (n_valid_tiles - 1) & 1;  // P buffer of the item's last valid tile
       }
     }
+    if (ended && fin) finalize();
     if (*abort_flag && tid == 0) set_status(a.status, PKV_DEV_TIMEOUT);
   }
   tc_fence_before();

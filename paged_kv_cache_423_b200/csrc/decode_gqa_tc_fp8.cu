@@ -50,50 +50,73 @@ constexpr int kTile = 128;                 // tokens per tile (MMA M of S)
 constexpr int kChunk = 16;                 // rows per TMA box: a 16-row slice of one (block, kv head)
 constexpr int kD = 128;
 constexpr int kN = 16;                     // query heads of one kv head (g <= 16)
-constexpr int kStages = 5;                 // e4m3 staging ring
 constexpr int kRow8 = kD;                  // bytes of one e4m3 row
 constexpr int kStage8 = 2 * kTile * kRow8; // K then V: 32 KiB
 constexpr int kVOff = kTile * kRow8;       // V within a stage
 constexpr int kQSlot = 4096;               // e4m3 [hi; lo] queries: 32 rows x 128 codes (from the split kernel)
-constexpr int kQSlots = 6;                 // by item ordinal; a slot is refilled 6 items later
 constexpr int kPTerm = kTile * 16;         // one e5m2 term of P: 128 tokens x 16 heads
 constexpr int kPBytes = 3 * kPTerm;        // [hi | mid | lo]
-constexpr int kSoftmax = 256;              // warps 0-7: two groups of 4 (head pairs 0, 2, .. and 1, 3, ..)
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 384;              // 3 warpgroups; warps 10-11 only lend registers
-// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); the
-// control warpgroup drops to 88 and the two softmax warpgroups rise to 208:
-// 128 x (208 + 208 + 88) = 64512, and per scheduler (one warp of each group)
-// 32 x 504 = 16128 <= 16384 registers.
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsControl = 88;
-static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 256;        // S double buffer [0,32), [32,64) (hi | lo); O of even / odd items
 constexpr uint32_t kColO = 64;             // at [64,112) / [128,176) (3 terms of 16 heads each)
 constexpr uint32_t kOStride = 64;
 constexpr uint32_t kChunkTx = 2 * kChunk * kRow8;  // K and V of one slice
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kPShift = 7.f;             // P is stored times 2^7 (at most 2^15)
-// Stage metadata: x = sequence, y = kv head | q slot << 16 | phase of the slot's barrier << 20,
-// z = partition | partitions << 16,
+// Stage metadata: x = sequence, y = kv head | q slot << 16, z = partition | partitions << 16,
 // w = valid rows (8 bits) | slice mask << 8 | first << 16 | last << 17 | end of stream << 18
 constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
 
-// shared memory
-constexpr int kOffStage = 0;
-constexpr int kOffQ = kOffStage + kStages * kStage8;
-constexpr int kOffP = kOffQ + kQSlots * kQSlot;
-constexpr int kOffRed = kOffP + 2 * kPBytes;
-constexpr int kOffMeta = kOffRed + 2 * 3 * 4 * 16 * 4;  // [group][maxima | sums of even | odd items][4 warps][16]
-constexpr int kOffScale = kOffMeta + kStages * 16;  // [stage] (k_scale, v_scale) of the item
-constexpr int kOffQinv = (kOffScale + kStages * 8 + 15) / 16 * 16;  // [q slot][16] 2^-e of each head (bulk copies)
-constexpr int kOffBar = kOffQinv + kQSlots * 16 * 4;
-constexpr int kBars = 2 * kStages + 2 * 4 + 1;
-constexpr int kOffMisc = kOffBar + kBars * 8;
-constexpr int kSmemBytes = kOffMisc + 32 + 1024;
-static_assert(kOffBar % 8 == 0 && kOffMeta % 16 == 0 && kOffQ % 1024 == 0 && kOffQinv % 16 == 0, "alignment");
-static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+// Two shapes of the CTA.
+//   GROUPS = 2: one CTA per SM; two softmax warpgroups split each tile's head pairs
+//     (warps 0-7), warp 8 the TMA producer, warp 9 the MMA issuer, warps 10-11 only lend
+//     registers; 5 stages.  Registers: launched at 168 per thread (384 x 168 = 64512), the
+//     control warpgroup drops to 88 and the softmax warpgroups rise to 208:
+//     128 x (208 + 208 + 88) = 64512, and per scheduler (one warp of each group)
+//     32 x 504 = 16128 <= 16384.
+//   GROUPS = 1: two CTAs per SM, so two independent item streams (each CTA's
+//     MMA -> softmax -> MMA chain) overlap on one SM; one softmax warpgroup takes every head
+//     (warps 0-3), warp 4 the producer, warp 5 the MMA issuer, warps 6-7 lend registers;
+//     2 stages each.  Registers: launched at 128 (2 x 256 x 128 = 65536), softmax 184,
+//     control 72: 128 x (184 + 72) = 32768 per CTA, and per scheduler 2 CTAs x 32 x 256 =
+//     16384.
+template <int GROUPS>
+struct Cfg {
+  static constexpr int kStages = GROUPS == 2 ? 5 : 2;
+  static constexpr int kQSlots = kStages + 1;  // by item ordinal; a slot is refilled kQSlots items later
+  static constexpr int kSoftmax = 128 * GROUPS;
+  static constexpr int kProducerWarp = 4 * GROUPS;
+  static constexpr int kMmaWarp = 4 * GROUPS + 1;
+  static constexpr int kThreads = 128 * (GROUPS + 1);
+  static constexpr int kCtasPerSm = GROUPS == 2 ? 1 : 2;
+  static constexpr int kLaunchRegs = GROUPS == 2 ? 168 : 128;
+  static constexpr int kRegsSoftmax = GROUPS == 2 ? 208 : 184;
+  static constexpr int kRegsControl = GROUPS == 2 ? 88 : 72;
+  static_assert(128 * (GROUPS * kRegsSoftmax + kRegsControl) <= kThreads * kLaunchRegs,
+                "register split exceeds the launch");
+  static_assert(kThreads * kLaunchRegs * kCtasPerSm <= 65536, "registers of an SM");
+  // shared memory
+  static constexpr int kOffStage = 0;
+  static constexpr int kOffQ = kOffStage + kStages * kStage8;
+  static constexpr int kOffP = kOffQ + kQSlots * kQSlot;
+  static constexpr int kOffRed = kOffP + 2 * kPBytes;
+  static constexpr int kOffMeta = kOffRed + 2 * 3 * 4 * 16 * 4;  // [group][maxima | sums of even | odd items][4 warps][16]
+  static constexpr int kOffScale = kOffMeta + kStages * 16;  // [stage] (k_scale, v_scale) of the item
+  static constexpr int kOffQinv = (kOffScale + kStages * 8 + 15) / 16 * 16;  // [q slot][16] 2^-e of each head
+  static constexpr int kOffBar = kOffQinv + kQSlots * 16 * 4;
+  static constexpr int kBars = 2 * kStages + 2 * 4 + 1;
+  static constexpr int kOffMisc = kOffBar + kBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
+  static_assert(kOffBar % 8 == 0 && kOffMeta % 16 == 0 && kOffQ % 1024 == 0 && kOffQinv % 16 == 0, "alignment");
+  static_assert(kSmemBytes * kCtasPerSm <= 232448, "shared memory of an SM");
+};
+
+// Head slots (NH = 4, 8 or 16 >= g) served with one softmax warpgroup per CTA and two CTAs per
+// SM (GROUPS = 1); larger groups take the two-warpgroup CTA.  Measured on a B200 (e4m3 pools):
+// the long-context batch (g = 8) 3,440 against 3,350 GB/s, the shared-prompt batch (g = 4) 660
+// against 552 GB/s of distinct bytes.
+#ifndef PKV_FP8_ONE_GROUP_MAX_NH
+#define PKV_FP8_ONE_GROUP_MAX_NH 8
+#endif
 
 struct alignas(64) Args {
   CUtensorMap tm_k;  // e4m3 pool as [rows, 128] bytes, box 128 x 16, 128-byte swizzle
@@ -190,8 +213,15 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, floa
 // decision that touches the shared O accumulator (a rescale restarts it) together.
 // NH (4, 8 or 16 >= g) bounds the heads the softmax works on; the operand layouts
 // keep 16 head slots.
-template <bool OUT_F32, int NH>
-__global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __grid_constant__ Args args) {
+template <bool OUT_F32, int NH, int GROUPS>
+__global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm)
+    decode_gqa_tc_fp8_kernel(const __grid_constant__ Args args) {
+  using C = Cfg<GROUPS>;
+  constexpr int kStages = C::kStages, kQSlots = C::kQSlots, kSoftmax = C::kSoftmax;
+  constexpr int kProducerWarp = C::kProducerWarp, kMmaWarp = C::kMmaWarp;
+  constexpr int kOffStage = C::kOffStage, kOffQ = C::kOffQ, kOffP = C::kOffP, kOffRed = C::kOffRed;
+  constexpr int kOffMeta = C::kOffMeta, kOffScale = C::kOffScale, kOffQinv = C::kOffQinv, kOffBar = C::kOffBar;
+  constexpr int kOffMisc = C::kOffMisc;
   const DecodeArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -223,12 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 8);
+      mbar_init(&empty[s], 1 + 4 * GROUPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 8);
-      mbar_init(&p_full[b], 8);
+      mbar_init(&s_free[b], 4 * GROUPS);
+      mbar_init(&p_full[b], 4 * GROUPS);
       mbar_init(&o_bar[b], 1);
     }
     mbar_init(drain, 1);
@@ -247,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
   if (warp >= kProducerWarp) {
   // The control warpgroup gives registers back; the branch is uniform per warpgroup,
   // as setmaxnreg requires, and dominates the code that runs with the new count.
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegsControl));
   if (warp == kProducerWarp) {
     // ================= producer: e4m3 slices and an item's queries =================
     const uint64_t policy = l2_policy_kv();
@@ -447,18 +477,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
     __syncwarp();
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegsSoftmax));
     // ================= softmax: thread = token row of the tile = TMEM lane =================
-    // Group G (warps 4G .. 4G+3) takes head pairs G, G+2, G+4, ..: local head j is
-    // head 4 (j / 2) + 2G + j % 2.  Both groups walk every tile together.
-    constexpr int NL = NH / 2;               // heads of one group
+    // With two groups, group G (warps 4G .. 4G+3) takes head pairs G, G+2, G+4, ..: local
+    // head j is head 4 (j / 2) + 2G + j % 2, and both groups walk every tile together.  One
+    // group takes every head (local head j = head j).
+    constexpr int NL = NH / GROUPS;          // heads of one group
     constexpr int kColLanes = 32 / NL;       // lanes sharing one column after warp_col
     const int G = warp >> 2;
     const int t = tid & 127;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float* red_max = red + G * 192;          // [4 warps][16]
     float* red_sums = red_max + 64;          // [item parity][4 warps][16]
-    auto head = [&](int j) { return 4 * (j >> 1) + 2 * G + (j & 1); };
+    auto head = [&](int j) { return GROUPS == 2 ? 4 * (j >> 1) + 2 * G + (j & 1) : j; };
     float m_used[NL], lp[NL], o_reg[NL], hscale[NL];
 #pragma unroll
     for (int j = 0; j < NL; ++j) m_used[j] = -INFINITY, lp[j] = 0.f, o_reg[j] = 0.f, hscale[j] = 0.f;
@@ -489,7 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
       tc::tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < NL; ++j) {
-        const int h0 = 4 * (j >> 1) + (j & 1);  // head of group 0; group 1's is h0 + 2
+        // register indices stay compile-time: group 1's heads are group 0's plus 2
+        const int h0 = GROUPS == 2 ? 4 * (j >> 1) + (j & 1) : j;
         o[j] = G ? o3[h0 + 2] + o3[kN + h0 + 2] + o3[2 * kN + h0 + 2] : o3[h0] + o3[kN + h0] + o3[2 * kN + h0];
       }
     };
@@ -581,15 +613,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         if (!valid) {
           // V rows outside the context may hold anything (even NaN codes): zero them
           // (each group half of the row)
-          uint4* vr = reinterpret_cast<uint4*>(stage8 + slot * kStage8 + kVOff + t * kRow8) + 4 * G;
+          uint4* vr = reinterpret_cast<uint4*>(stage8 + slot * kStage8 + kVOff + t * kRow8) + (8 / GROUPS) * G;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) vr[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 8 / GROUPS; ++c) vr[c] = make_uint4(0, 0, 0, 0);
         }
         float x[NL];
         bool need = false;
 #pragma unroll
         for (int j = 0; j < NL; ++j) {
-          const int h0 = 4 * (j >> 1) + (j & 1);
+          const int h0 = GROUPS == 2 ? 4 * (j >> 1) + (j & 1) : j;  // compile-time register indices
           const float sv = G ? s[h0 + 2] + s[kN + h0 + 2] : s[h0] + s[kN + h0];
           x[j] = (valid && head(j) < g) ? sv * hscale[j] : -INFINITY;
           need |= x[j] > m_used[j] + kRescaleLog2;
@@ -598,7 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
         // term's 16-byte chunk at (t/8)*128 + (t%8)*16 of its 2 KiB third of the buffer.
         float pv[NL];
         auto write_p = [&]() {
-          unsigned char* row = p_tile + (t >> 3) * 128 + (t & 7) * 16 + 2 * G;
+          // global head pair of local pair k: 2k + G with two groups, k with one (2 bytes per pair)
+          unsigned char* row = p_tile + (t >> 3) * 128 + (t & 7) * 16 + (GROUPS == 2 ? 2 * G : 0);
 #pragma unroll
           for (int k = 0; k < NL / 2; ++k) {
             const int j0 = 2 * k, j1 = 2 * k + 1;
@@ -611,9 +644,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_fp8_kernel(const __
             pv[j0] = f16lo(sum);
             pv[j1] = f16hi(sum);
             // the codes are the top bytes of the two f16 halves
-            *reinterpret_cast<uint16_t*>(row + 4 * k) = static_cast<uint16_t>(__byte_perm(ph, 0, 0x0031));
-            *reinterpret_cast<uint16_t*>(row + kPTerm + 4 * k) = static_cast<uint16_t>(__byte_perm(pm, 0, 0x0031));
-            *reinterpret_cast<uint16_t*>(row + 2 * kPTerm + 4 * k) = static_cast<uint16_t>(__byte_perm(pl, 0, 0x0031));
+            const int pk = GROUPS == 2 ? 4 * k : 2 * k;
+            *reinterpret_cast<uint16_t*>(row + pk) = static_cast<uint16_t>(__byte_perm(ph, 0, 0x0031));
+            *reinterpret_cast<uint16_t*>(row + kPTerm + pk) = static_cast<uint16_t>(__byte_perm(pm, 0, 0x0031));
+            *reinterpret_cast<uint16_t*>(row + 2 * kPTerm + pk) = static_cast<uint16_t>(__byte_perm(pl, 0, 0x0031));
           }
         };
         if (bad) *abort_flag = 1;
@@ -778,14 +812,17 @@ static int encode_map(CUtensorMap* map, const void* base, uint64_t rows, int box
 
 template <bool OUT_F32, int NH>
 static int launch(const Args& args, cudaStream_t stream) {
-  auto kernel = decode_gqa_tc_fp8_kernel<OUT_F32, NH>;
+  constexpr int GROUPS = NH <= PKV_FP8_ONE_GROUP_MAX_NH ? 1 : 2;
+  using C = Cfg<GROUPS>;
+  constexpr int kSmemBytes = C::kSmemBytes;
+  auto kernel = decode_gqa_tc_fp8_kernel<OUT_F32, NH, GROUPS>;
   static PerDevice<int> setup;
   int dev = 0, sms = 0;
   const int st = set_smem_limit_once(setup, kernel, kSmemBytes, &dev);
   if (st != 0)
     return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  kernel<<<std::max(1, sms), kThreads, kSmemBytes, stream>>>(args);
+  kernel<<<std::max(1, sms * C::kCtasPerSm), C::kThreads, kSmemBytes, stream>>>(args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) launch: %s", cudaGetErrorString(e));
   return PKV_OK;

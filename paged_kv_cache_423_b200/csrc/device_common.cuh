@@ -85,13 +85,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// The short wait of the failure-path test build (PKV_SHORT_WAITS): 16 polls, a few hundred
-// nanoseconds, so that an ordinary launch runs into its expiry path.  No wait is removed.
+// The short wait of the failure-path test build (PKV_SHORT_WAITS): one poll, so that an
+// ordinary launch runs into its expiry path (with 16 polls, copies served from L2 often landed
+// in time).  No wait is removed.
 __device__ __forceinline__ bool mbar_wait_short(uint64_t* bar, uint32_t parity) {
-#pragma unroll 1
-  for (int i = 0; i < 16; ++i)
-    if (mbar_test(bar, parity)) return true;
-  return false;
+  return mbar_test(bar, parity);
 }
 
 // Pipeline waits of the CUDA-core decode and of the prefill kernel: bounded by kWaitLimitNs,

@@ -76,10 +76,13 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;
 // Share of the softmax exponentials computed by a polynomial on the FMA pipe (one pair of
-// scores in kPolyEvery; 0 = none): the SFU issues 16 exponentials per clock per SM, about as
-// many as a stage's MMAs take, so part of them moves to the 128-wide FMA pipe.
+// scores in kPolyEvery; 0 = none, the default).  The SFU issues 16 exponentials per clock per
+// SM, about as many as a stage's MMAs take; but measured on a B200 every share made the kernel
+// slower (13B chunked batch: 746 TFLOP/s with none, 677 with one pair in 8, 637 with one in 4,
+// 528 with one in 2): the softmax is bound by instruction issue, and the polynomial adds
+// instructions.  The option stays for other shapes; its function is tested either way.
 #ifndef PKV_PREFILL_POLY_EVERY
-#define PKV_PREFILL_POLY_EVERY 4
+#define PKV_PREFILL_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = PKV_PREFILL_POLY_EVERY;
 

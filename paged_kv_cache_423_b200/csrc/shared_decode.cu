@@ -7,22 +7,31 @@
 // by log-sum-exp rescaling, which reproduces softmax attention over the whole context
 // (intelliparadigm article "PagedAttention：操作系统分页思想的跨界创新" §2.1).
 //
-// Launches, in order on the caller's stream:
+// Launches, on the caller's stream unless noted:
 //   shared_setup_kernel   checks the plan against the call (sizes, ranges, that every
 //                         row's shared tokens plus its remainder equal its context
 //                         length) and writes checked copies of the remainders; a plan
 //                         that does not fit sets PKV_DEV_BAD_CONTEXT and every output
 //                         row becomes zero
-//   prefill_tc_kernel     segment mode: all query heads of a part's rows against the
-//                         part's keys, unnormalised partials (o, m, l)
+//   prefill_tc_kernel     segment mode, on a side stream forked after the set-up: all query
+//                         heads of a part's rows against the part's keys, unnormalised
+//                         partials (o, m, l)
 //   plan_kernel +
-//   decode_gqa_tc_kernel  the remainders, every item writing its partial
-//   shared_merge_kernel   out = sum 2^(m_i - M) o_i / sum 2^(m_i - M) l_i per (row, head)
+//   decode_gqa_tc_kernel  the remainders, every item writing its partial, beside the shared
+//                         phase (the two write disjoint partials, and each kernel's CTAs take
+//                         the SMs the other leaves)
+//   shared_merge_kernel   after both (the side stream joins back): out = sum 2^(m_i - M) o_i /
+//                         sum 2^(m_i - M) l_i per (row, head)
+// The side stream and its two events are created on the first call on each device and kept
+// until the process exits; the enqueue of a call is serialised per device, so calls from
+// several host threads stay correct.
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "decode_common.cuh"
+#include "per_device.h"
 #include "pkv_internal.h"
 
 namespace pkv {
@@ -123,6 +132,26 @@ __global__ void __launch_bounds__(kSetupThreads) shared_setup_kernel(const Setup
     p.count[2] = bad;
     if (bad) set_status(p.status, PKV_DEV_BAD_CONTEXT);
   }
+}
+
+// The side stream of the shared phase and the fork / join events, one set per device.
+struct Side {
+  cudaStream_t stream;
+  cudaEvent_t fork, join;
+};
+static PerDevice<Side> g_side;
+static std::mutex g_side_mutex[kMaxDevices];
+
+static int side_for(int dev, Side* out) {
+  return g_side.get(
+      dev,
+      [](Side& s) {
+        cudaError_t e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+        return static_cast<int>(e);
+      },
+      out, static_cast<int>(cudaErrorInvalidDevice));
 }
 
 struct MergeArgs {
@@ -288,8 +317,23 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "shared setup launch: %s", cudaGetErrorString(e));
 
-  // ---- shared phase
+  // ---- shared phase, on the side stream
+  int dev = 0;
+  cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess) return set_error(PKV_ERR_CUDA, "shared decode: cudaGetDevice: %s", cudaGetErrorString(de));
+  if (dev < 0 || dev >= kMaxDevices) return set_error(PKV_ERR_INVALID, "shared decode: device %d out of range", dev);
+  sp::Side side{};
   if (in.num_entries > 0) {
+    const int st = sp::side_for(dev, &side);
+    if (st != 0)
+      return set_error(PKV_ERR_CUDA, "shared decode: side stream: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
+  }
+  std::unique_lock<std::mutex> lock(sp::g_side_mutex[dev], std::defer_lock);
+  if (in.num_entries > 0) {
+    lock.lock();
+    e = cudaEventRecord(side.fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.fork, 0);
+    if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "shared decode: fork: %s", cudaGetErrorString(e));
     SegmentLaunch sl{};
     sl.query = query;
     sl.key_cache = key_cache;
@@ -309,8 +353,13 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
     sl.block_size = block_size;
     sl.num_blocks = num_blocks;
     sl.scale = scale;
-    const int rc = launch_prefill_segments(sl, s);
-    if (rc != PKV_OK) return rc;
+    int rc = launch_prefill_segments(sl, side.stream);
+    e = cudaEventRecord(side.join, side.stream);
+    if (rc == PKV_OK && e != cudaSuccess) rc = set_error(PKV_ERR_CUDA, "shared decode: join: %s", cudaGetErrorString(e));
+    if (rc != PKV_OK) {
+      cudaStreamWaitEvent(s, side.join, 0);  // leave the caller's stream joined
+      return rc;
+    }
   }
 
   // ---- private phase: the remainders through the tensor-core decode, partials only
@@ -342,6 +391,10 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
   a.always_partial = 1;
   int rc = launch_decode_plan(a, v_lens, in.max_suffix_len, s);
   if (rc == PKV_OK) rc = launch_decode_tensor(a, head_dim, out_dtype == PKV_DTYPE_F32, s);
+  if (in.num_entries > 0) {
+    e = cudaStreamWaitEvent(s, side.join, 0);  // the merge reads the shared partials
+    if (rc == PKV_OK && e != cudaSuccess) rc = set_error(PKV_ERR_CUDA, "shared decode: join: %s", cudaGetErrorString(e));
+  }
   if (rc != PKV_OK) return rc;
 
   // ---- merge

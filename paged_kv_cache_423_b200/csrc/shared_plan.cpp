@@ -26,7 +26,9 @@ namespace pkv {
 namespace {
 
 constexpr int kTileRows = 128;       // query rows of one tile of the shared phase (MMA M)
-constexpr int kItemsTarget = 296;    // two work items per SM of a 148-SM B200
+// Shared-phase work items the automatic key chunk aims for: the phase runs beside the private
+// decode, so it needs no full wave of its own, and longer chunks leave fewer partials to merge.
+constexpr int kItemsTarget = 64;
 
 struct Segment {
   int row0, nrows, block0, nblocks;

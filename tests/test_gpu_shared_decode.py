@@ -157,3 +157,30 @@ def test_runs_on_a_non_default_stream(pkv):
     with torch.cuda.stream(s):
         out, _ = run_shared(pkv, db)
     compare(out.cpu().numpy(), oracle_out(b))
+
+
+def test_two_calls_on_two_streams(pkv):
+    """Two batches decoded on two caller streams without ordering between them: each call
+    forks its shared phase onto the library's side stream and joins it back, so both
+    results stay right."""
+    b1, b2 = beam_batch(13, steps=1), beam_batch(14, steps=2)
+    d1, d2 = DeviceBatch(b1), DeviceBatch(b2)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    outs = []
+    for db, st in ((d1, s1), (d2, s2)):
+        with torch.cuda.stream(st):
+            b = db.b
+            plan, info = pkv.shared_plan(b.block_tables, b.context_lens, b.num_heads, b.num_kv_heads, b.block_size)
+            plan_d = torch.from_numpy(plan).cuda()
+            ws = torch.empty(pkv.paged_attention_decode_shared_workspace_size(info, b.num_heads, b.num_kv_heads, 128),
+                             dtype=torch.uint8, device="cuda")
+            out = torch.empty((b.num_seqs, b.num_heads, 128), dtype=torch.float32, device="cuda")
+            status = torch.zeros(1, dtype=torch.int32, device="cuda")
+            pkv.paged_attention_decode_shared(out, db.query, db.key_cache, db.value_cache, db.tables, db.lens, b.scale,
+                                              plan_d, info, ws, status=status)
+            outs.append((out, status, plan_d, ws))
+    torch.cuda.synchronize()
+    for (out, status, _, _), b in zip(outs, (b1, b2)):
+        assert status.item() == 0
+        compare(out.cpu().numpy(), oracle_out(b))

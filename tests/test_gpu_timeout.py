@@ -4,9 +4,9 @@ Every mbarrier wait of the kernels gives up after a limit (one second of %global
 and the kernel then flags PKV_DEV_TIMEOUT, lets its copies in flight land, waits for its
 MMAs, frees its tensor memory and returns, so a scheduling bug cannot hang the GPU.  A
 second build of the library (`build_library(variant="shortwait")`) shortens the pipeline
-waits of the CUDA-core decode and of the prefill kernel to a few hundred nanoseconds of
-polling -- no wait is removed, and the end-of-kernel drains keep their full limit -- so
-ordinary decode and prefill launches run into that path.  In a child process the test
+waits of the CUDA-core decode and of the prefill kernel to a single poll -- no wait is
+removed, and the end-of-kernel drains keep their full limit -- so ordinary decode and
+prefill launches run into that path.  In a child process the test
 requires (1) every short-wait call to return with PKV_DEV_TIMEOUT in its status word and
 (2) the default build, loaded afterwards into the same process and CUDA context, to give
 the oracle's results with a clean status: the context stays usable."""

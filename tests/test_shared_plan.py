@@ -237,3 +237,14 @@ def test_workspace_size_of_the_shared_run(pkv):
     n = pkv.paged_attention_decode_shared_workspace_size(info, 32, 8, 128)
     assert n >= info.num_partials * 32 * (128 * 4 + 8)
     assert pkv.paged_attention_decode_shared_workspace_size(info, 32, 8, 64) == 0
+
+
+def test_plan_into_a_caller_buffer(pkv):
+    """One call into a caller-provided buffer gives the same plan; a short buffer raises."""
+    tables, lens, bs = beam_batch(2)
+    plan, info = pkv.shared_plan(tables, lens, 32, 8, bs)
+    buf = np.full(plan.nbytes + 100, 0xAB, np.uint8)
+    got, info2 = pkv.shared_plan(tables, lens, 32, 8, bs, out=buf)
+    assert got.nbytes == plan.nbytes and np.array_equal(got, plan) and info2.as_dict() == info.as_dict()
+    with pytest.raises(pkv.PkvError):
+        pkv.shared_plan(tables, lens, 32, 8, bs, out=np.zeros(plan.nbytes - 16, np.uint8))

@@ -1,7 +1,7 @@
 """The launches of the bounded-wait expiry test.
 
 Run as a script with PKV_LIBRARY naming the short-wait build (its CUDA-core decode and
-prefill kernels give up a pipeline wait after a few hundred nanoseconds), it runs a small
+prefill kernels give up a pipeline wait after one poll), it runs a small
 decode (CUDA-core path, unsplit and split) and a small chunked prefill through that build
 and records each call's device status word; then, in the same process and CUDA context,
 it loads the default build named by its second argument and runs the same decode and

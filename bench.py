@@ -855,6 +855,7 @@ def run_trace(args, rank, world, local_rank):
     for length, budget in initial:
         admit(length, budget)
     t_ms = 0.0
+    span_ms = 0.0  # first kernel start to last kernel end per step, host launch gaps included
     alloc_s = 0.0  # host allocator time of the timed steps (append, export, frees)
     seq_steps = 0
     kv_bytes = 0
@@ -899,16 +900,22 @@ def run_trace(args, rank, world, local_rank):
                 q = torch.randn((len(ids), p.num_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
                 k = torch.randn((len(ids), p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
                 out = torch.empty((len(ids), p.num_heads, p.head_dim), dtype=torch.bfloat16, device=device)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                if len(pairs):
-                    pkv.copy_blocks([kc], [vc], torch.from_numpy(pairs).to(device), status=status)
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                pairs_d = torch.from_numpy(pairs).to(device) if len(pairs) else None
+                ev[0].record(stream)
+                if pairs_d is not None:
+                    pkv.copy_blocks([kc], [vc], pairs_d, status=status)
                 pkv.reshape_and_cache(k, k, kc, vc, d_slots, status=status)
+                ev[1].record(stream)
+                ev[2].record(stream)
                 pkv.paged_attention_decode(out, q, kc, vc, d_tables, d_lens, max_len, scale, ws, status=status)
-                e1.record(stream)
+                ev[3].record(stream)
                 torch.cuda.synchronize()
                 if step >= args.warmup:
-                    t_ms += e0.elapsed_time(e1)
+                    # the step's kernels: the cache write (and copies), then the decode call; the
+                    # host's marshalling of the decode call between the two is not device work
+                    t_ms += ev[0].elapsed_time(ev[1]) + ev[2].elapsed_time(ev[3])
+                    span_ms += ev[0].elapsed_time(ev[3])
                     alloc_s += a_s
                     seq_steps += len(ids)
                     kv_bytes += int(lens.astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 4
@@ -943,7 +950,10 @@ def run_trace(args, rank, world, local_rank):
                        "num_blocks": p.num_blocks, "admitted": next_id,
                        "initial_lengths": f"U{{{p.len_lo}..{p.len_hi}}}", "budgets": f"U{{{p.budget_lo}..{p.budget_hi}}}",
                        "arrivals": f"Bernoulli({p.arrival_p}) per free slot per step, lengths U{{{p.len_lo}..{p.len_hi}}}",
-                       "timed": "copy_blocks + reshape_and_cache + paged_attention_decode per step"},
+                       "timed": "copy_blocks + reshape_and_cache, and paged_attention_decode, per step (events"
+                                " around each call: the host's marshalling between the calls is excluded;"
+                                " ms_per_step_span includes it)"},
+            "ms_per_step_span": round(span_ms / max(1, args.steps), 4),
             "seq_steps_per_s": round(seq_steps / (t_ms * 1e-3), 1), "pct_hbm_peak": round(100 * value / peak, 2),
             # the same with the host allocator's time per step added (it runs between the steps here)
             "seq_steps_per_s_with_allocator": round(seq_steps / (t_ms * 1e-3 + alloc_s), 1),

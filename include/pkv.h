@@ -285,7 +285,8 @@ PKV_API int pkv_swap_blocks(const void* src_pool, void* dst_pool, const int64_t*
  *   query_start  device [num_seqs + 1] int32, non-decreasing, query_start[num_seqs] <= total_q
  *   context_lens device [num_seqs] int32, n <= L <= min(max_context_len, max_blocks_per_seq*block_size)
  *   workspace    device, pkv_paged_attention_prefill_workspace_size() bytes, 256-byte aligned
- * head_dim must be 128 and num_heads / num_kv_heads must divide 128 (PKV_ERR_UNSUPPORTED).
+ * head_dim must be 128 and num_heads / num_kv_heads must divide 128 (PKV_ERR_UNSUPPORTED);
+ * scale must be finite and positive (PKV_ERR_INVALID: hidden keys are -inf scores).
  * A sequence whose numbers break the rules above sets PKV_DEV_BAD_CONTEXT and its rows
  * (when their range is valid) are written as zeros; a table entry outside the pool sets
  * PKV_DEV_BAD_BLOCK and its 16-row slice of keys is skipped.  The pages leave the
@@ -370,7 +371,7 @@ PKV_API int pkv_shared_plan(const int32_t* block_tables, int max_blocks_per_seq,
  *   info        host, the plan's info
  *   workspace   device, pkv_paged_attention_decode_shared_workspace_size() bytes, 256-byte aligned
  * bf16 pools only; head_dim 128; 2 <= num_heads / num_kv_heads <= 16 (the tensor-core
- * decode) — else PKV_ERR_UNSUPPORTED.  block_tables and context_lens must be those the
+ * decode) — else PKV_ERR_UNSUPPORTED; scale finite and positive, else PKV_ERR_INVALID.  block_tables and context_lens must be those the
  * plan was made from: the call checks on the device that every row's shared tokens plus its
  * remainder equal its context length (and the plan's ranges); a plan that does not fit sets
  * PKV_DEV_BAD_CONTEXT and every output row is zero.

@@ -178,30 +178,6 @@ __device__ __forceinline__ int load_item_table(const DecodeArgs& a, const PlanEn
   return __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + lane);
 }
 
-// ---- packed fp32x2 arithmetic (two lanes of fp32 in one 64-bit register pair)
-__device__ __forceinline__ uint64_t f2pack(float x, float y) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
-  return r;
-}
-__device__ __forceinline__ float2 f2unpack(uint64_t v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-// bf16 pair word -> packed (lo, hi) fp32 pair, exactly.
-__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2pack(bf16lo(w), bf16hi(w)); }
-
 // a0 += q.lo * k.lo, a1 += q.hi * k.hi with bf16 operands and fp32 accumulation
 // (sm_100 mixed-precision FMA; the bf16 x bf16 product is exact in fp32).
 __device__ __forceinline__ void dot_bf16x2(float& a0, float& a1, uint32_t q, uint32_t k) {

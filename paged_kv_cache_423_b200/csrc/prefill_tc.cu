@@ -39,6 +39,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "decode_common.cuh"
 #include "launch_setup.cuh"
@@ -566,30 +567,35 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       }
       lsum *= alpha;
       // ---- P = 2^(s * scale_log2 - m) as bf16 pairs, stored over S (columns 0-63 of
-      //      the tile's block: keys 2i, 2i+1 in column i)
+      //      the tile's block: keys 2i, 2i+1 in column i).  Pairs of scores go through packed
+      //      fp32x2 arithmetic: one fma.rn.f32x2 for scale and maximum, and the row sum adds
+      //      the rounded bf16 pairs with add.rn.f32x2.  A row with no visible key yet holds
+      //      -inf as its maximum: neg_m is then 0 and every score of the stage is -inf, so its
+      //      weights are 0 without a select.
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      const bool any = m_used != -INFINITY;
-      float ls8[8];
+      const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(neg_m, neg_m);
+      uint64_t ls2[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ls8[i] = 0.f;
+      for (int i = 0; i < 4; ++i) ls2[i] = f2pack(0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float x0 = s[h * 32 + 2 * i], x1 = s[h * 32 + 2 * i + 1];
+          const float2 e = f2unpack(ffma2(f2pack(s[h * 32 + 2 * i], s[h * 32 + 2 * i + 1]), sc2, nm2));
           // one pair in kPolyEvery takes the FMA-pipe exponential, the rest the SFU's
           const bool poly = kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1;
-          const float e0 = fmaf(x0, a.scale_log2, neg_m), e1 = fmaf(x1, a.scale_log2, neg_m);
-          const float p0 = any ? (poly ? tc::poly_exp2(e0) : fast_exp2(e0)) : 0.f;
-          const float p1 = any ? (poly ? tc::poly_exp2(e1) : fast_exp2(e1)) : 0.f;
+          const float p0 = poly ? tc::poly_exp2(e.x) : fast_exp2(e.x);
+          const float p1 = poly ? tc::poly_exp2(e.y) : fast_exp2(e.y);
           w[i] = pack_bf16x2(p0, p1);
-          ls8[(2 * i) & 7] += bf16lo(w[i]);
-          ls8[(2 * i + 1) & 7] += bf16hi(w[i]);
+          ls2[i & 3] = fadd2(ls2[i & 3], bf16x2_to_f2(w[i]));
         }
         tc::tmem_store16(tmem + lane_base + col_s + h * 16, w);
       }
-      lsum += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+      {
+        const float2 l0 = f2unpack(fadd2(ls2[0], ls2[1])), l1 = f2unpack(fadd2(ls2[2], ls2[3]));
+        lsum += (l0.x + l0.y) + (l1.x + l1.y);
+      }
       tc::tmem_wait_st();
       tc::tc_fence_before();     // P and the rescaled O, before the MMA reads them
       __syncwarp();
@@ -875,6 +881,8 @@ extern "C" int pkv_paged_attention_prefill(void* out, int out_dtype, const void*
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_prefill: group %d does not divide 128", group);
   if (num_kv_heads >= (1 << 15) || max_context_len >= (1 << 25))
     return set_error(PKV_ERR_INVALID, "paged_attention_prefill: sizes out of range");
+  if (!(scale > 0.f) || !std::isfinite(scale))  // masked keys are -inf scores: a scale of 0 would make them NaN
+    return set_error(PKV_ERR_INVALID, "paged_attention_prefill: scale must be finite and positive");
   if (static_cast<int64_t>(num_blocks) * num_kv_heads * block_size > (static_cast<int64_t>(1) << 31))
     return set_error(PKV_ERR_INVALID, "paged_attention_prefill: pool too large");
   if (num_seqs == 0 || total_q == 0) return PKV_OK;

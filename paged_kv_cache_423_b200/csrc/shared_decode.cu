@@ -28,6 +28,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "decode_common.cuh"
@@ -246,6 +247,8 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
                      "num_kv_heads <= 16 (got %d, %d / %d)", head_dim, num_heads, num_kv_heads);
   if (num_kv_heads >= (1 << 15))
     return set_error(PKV_ERR_UNSUPPORTED, "paged_attention_decode_shared: num_kv_heads %d", num_kv_heads);
+  if (!(scale > 0.f) || !std::isfinite(scale))  // the shared phase masks keys with -inf scores
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: scale must be finite and positive");
   const int group = num_heads / num_kv_heads;
   if (in.num_seqs != num_seqs || in.group != group || in.block_size != block_size ||
       in.max_blocks_per_seq != max_blocks_per_seq || in.num_entries < 0 || in.num_parts < 0 ||

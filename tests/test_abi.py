@@ -105,6 +105,9 @@ def test_prefill_argument_errors_before_any_device_work(pkv):
     assert call(ws_bytes=64) == pkv.PKV_ERR_INVALID
     assert b"workspace" in lib.pkv_last_error_string()
     assert call(qstart=None) == pkv.PKV_ERR_INVALID
+    for bad_scale in (0.0, -0.1, float("inf"), float("nan")):  # hidden keys are -inf scores
+        assert call(scale=bad_scale) == pkv.PKV_ERR_INVALID
+        assert b"scale" in lib.pkv_last_error_string()
     assert call(T=0) == pkv.PKV_OK                        # no rows: nothing to do
     assert call(B=0) == pkv.PKV_OK
 

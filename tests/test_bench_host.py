@@ -498,6 +498,7 @@ def test_run_trace_host_logic_with_stand_ins(pkv, monkeypatch):
     assert 0 < kernel_calls["decode"] <= 23
     assert res["allocator_us_per_step"] > 0
     assert res["seq_steps_per_s_with_allocator"] < res["seq_steps_per_s"]
+    assert res["ms_per_step_span"] > 0   # first kernel start to last kernel end, launch gaps included
     import json
     json.dumps(res)
 
@@ -641,3 +642,35 @@ def test_shared_decode_applies_only_where_it_can_run():
     assert not bench.shared_decode_applies(args(), w(Hq=40, Hkv=40))   # MHA: no tensor-core decode
     with pytest.raises(SystemExit):
         bench.shared_decode_applies(args("on"), w(Hq=40, Hkv=40))
+
+
+def test_e2e_shared_prefix_plan_travels_with_each_step(pkv, monkeypatch):
+    """With the shared-prefix decode the e2e harness plans every step on the host, straight
+    into the pinned buffer, and the plan's bytes count as host-to-device traffic; the decode
+    gets the device plan, its info and the shared workspace."""
+    import contextlib
+    import types
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _FakeStream())
+    monkeypatch.setattr(torch.cuda, "Stream", _FakeStream)
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    w = bench.Workload("tiny", 8, seed=5, device=torch.device("cpu"))
+    sws = torch.empty(16, dtype=torch.uint8)
+    seen = []
+
+    def decode(out, q, tables, lens, max_len, ws, path, status, shared=None):
+        plan, info, ws_shared = shared
+        assert ws_shared is sws and plan.dtype == torch.uint8 and plan.numel() >= info.bytes
+        seen.append(int(info.bytes))
+        out.fill_(1.0)
+
+    w.write, w.decode = (lambda *a, **k: None), decode
+    w.copy = lambda pairs, status: None
+    args = types.SimpleNamespace(steps=4, e2e_steps=4, warmup=3)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16)
+    res = bench.run_e2e(args, w, pkv, torch.device("cpu"), 0, None, out, None, 1024, sws)
+    assert len(seen) == 7 and all(b > 0 for b in seen)
+    plain = 2 * w.B * (w.Hq + 2 * w.Hkv) * w.D + 8 * w.B + 4 * w.B * w.max_blocks + 4 * w.B
+    assert res["h2d_bytes_per_step"] == plain + sum(seen[3:]) // 4

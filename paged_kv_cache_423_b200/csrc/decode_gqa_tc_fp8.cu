@@ -51,38 +51,41 @@ constexpr int kChunk = 16;                 // rows per TMA box: a 16-row slice o
 constexpr int kD = 128;
 constexpr int kN = 16;                     // query heads of one kv head (g <= 16)
 constexpr int kRow8 = kD;                  // bytes of one e4m3 row
-constexpr int kStage8 = 2 * kTile * kRow8; // K then V: 32 KiB
-constexpr int kVOff = kTile * kRow8;       // V within a stage
+constexpr int kTile8 = kTile * kRow8;      // one K or V tile: 16 KiB
 constexpr int kQSlot = 4096;               // e4m3 [hi; lo] queries: 32 rows x 128 codes (from the split kernel)
 constexpr int kPTerm = kTile * 16;         // one e5m2 term of P: 128 tokens x 16 heads
 constexpr int kPBytes = 3 * kPTerm;        // [hi | mid | lo]
 constexpr uint32_t kTmemCols = 256;        // S double buffer [0,32), [32,64) (hi | lo); O of even / odd items
 constexpr uint32_t kColO = 64;             // at [64,112) / [128,176) (3 terms of 16 heads each)
 constexpr uint32_t kOStride = 64;
-constexpr uint32_t kChunkTx = 2 * kChunk * kRow8;  // K and V of one slice
+constexpr uint32_t kSliceTx = kChunk * kRow8;  // one 16-row slice of K or of V
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kPShift = 7.f;             // P is stored times 2^7 (at most 2^15)
 // Stage metadata: x = sequence, y = kv head | q slot << 16, z = partition | partitions << 16,
 // w = valid rows (8 bits) | slice mask << 8 | first << 16 | last << 17 | end of stream << 18
 constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
 
+// K and V of a tile travel in separate rings: a K slot is free again once the tile's S = K·Qᵀ
+// is done, a V slot only once its O += Vᵀ·P is, so K (and with it the next tiles' S) runs a
+// stage further ahead than a shared K+V stage would allow.
 // Two shapes of the CTA.
 //   GROUPS = 2: one CTA per SM; two softmax warpgroups split each tile's head pairs
 //     (warps 0-7), warp 8 the TMA producer, warp 9 the MMA issuer, warps 10-11 only lend
-//     registers; 5 stages.  Registers: launched at 168 per thread (384 x 168 = 64512), the
+//     registers; 5 K and 4 V slots.  Registers: launched at 168 per thread (384 x 168 = 64512), the
 //     control warpgroup drops to 88 and the softmax warpgroups rise to 208:
 //     128 x (208 + 208 + 88) = 64512, and per scheduler (one warp of each group)
 //     32 x 504 = 16128 <= 16384.
 //   GROUPS = 1: two CTAs per SM, so two independent item streams (each CTA's
 //     MMA -> softmax -> MMA chain) overlap on one SM; one softmax warpgroup takes every head
 //     (warps 0-3), warp 4 the producer, warp 5 the MMA issuer, warps 6-7 lend registers;
-//     2 stages each.  Registers: launched at 128 (2 x 256 x 128 = 65536), softmax 184,
+//     3 K and 2 V slots each.  Registers: launched at 128 (2 x 256 x 128 = 65536), softmax 184,
 //     control 72: 128 x (184 + 72) = 32768 per CTA, and per scheduler 2 CTAs x 32 x 256 =
 //     16384.
 template <int GROUPS>
 struct Cfg {
-  static constexpr int kStages = GROUPS == 2 ? 5 : 2;
-  static constexpr int kQSlots = kStages + 1;  // by item ordinal; a slot is refilled kQSlots items later
+  static constexpr int kKStages = GROUPS == 2 ? 5 : 3;
+  static constexpr int kVStages = GROUPS == 2 ? 4 : 2;
+  static constexpr int kQSlots = kKStages + 1;  // by item ordinal; a slot is refilled kQSlots items later
   static constexpr int kSoftmax = 128 * GROUPS;
   static constexpr int kProducerWarp = 4 * GROUPS;
   static constexpr int kMmaWarp = 4 * GROUPS + 1;
@@ -95,19 +98,20 @@ struct Cfg {
                 "register split exceeds the launch");
   static_assert(kThreads * kLaunchRegs * kCtasPerSm <= 65536, "registers of an SM");
   // shared memory
-  static constexpr int kOffStage = 0;
-  static constexpr int kOffQ = kOffStage + kStages * kStage8;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKStages * kTile8;
+  static constexpr int kOffQ = kOffV + kVStages * kTile8;
   static constexpr int kOffP = kOffQ + kQSlots * kQSlot;
   static constexpr int kOffRed = kOffP + 2 * kPBytes;
   static constexpr int kOffMeta = kOffRed + 2 * 3 * 4 * 16 * 4;  // [group][maxima | sums of even | odd items][4 warps][16]
-  static constexpr int kOffScale = kOffMeta + kStages * 16;  // [stage] (k_scale, v_scale) of the item
-  static constexpr int kOffQinv = (kOffScale + kStages * 8 + 15) / 16 * 16;  // [q slot][16] 2^-e of each head
+  static constexpr int kOffScale = kOffMeta + kKStages * 16;  // [K slot] (k_scale, v_scale) of the item
+  static constexpr int kOffQinv = (kOffScale + kKStages * 8 + 15) / 16 * 16;  // [q slot][16] 2^-e of each head
   static constexpr int kOffBar = kOffQinv + kQSlots * 16 * 4;
-  static constexpr int kBars = 2 * kStages + 2 * 4 + 1;
+  static constexpr int kBars = 2 * kKStages + 2 * kVStages + 2 * 4 + 1;
   static constexpr int kOffMisc = kOffBar + kBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;
   static_assert(kOffBar % 8 == 0 && kOffMeta % 16 == 0 && kOffQ % 1024 == 0 && kOffQinv % 16 == 0, "alignment");
-  static_assert(kSmemBytes * kCtasPerSm <= 232448, "shared memory of an SM");
+  static_assert((kSmemBytes + 1024) * kCtasPerSm <= 233472, "shared memory of an SM (1 KiB reserved per CTA)");
 };
 
 // Head slots (NH = 4, 8 or 16 >= g) served with one softmax warpgroup per CTA and two CTAs per
@@ -200,15 +204,17 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx, floa
 }
 
 // Pipeline (per CTA, persistent over work items; n counts tiles):
-//   producer     -> full[s]    : e4m3 K, V (and an item's split queries and head scales on its
-//                                first tile) in stage s
-//   MMA          -> s_full[b]  : S of the b-th valid tile (mod 2) in TMEM
-//   softmax      -> s_free[b]  : that S read (8 warps)
-//   softmax      -> p_full[b]  : P of that tile in shared buffer b (and its stale V rows zeroed; 8 warps)
-//   MMA          -> o_bar[b]   : its O += Vᵀ·P done (P buffer b reusable)
-//   MMA + softmax -> empty[s] : stage s done with: its P·V complete (commit; a plain
-//                  arrival for a tile with no rows), metadata read by the 8 softmax warps
-//                  (9 arrivals)
+//   producer     -> k_full[n % K]  : K of tile n (and an item's split queries and head scales
+//                                    on its first tile), with the tile's metadata
+//   producer     -> v_full[n % V]  : V of tile n, issued after the K of tile n+1
+//   MMA          -> s_full[b]      : S of the b-th valid tile (mod 2) in TMEM
+//   softmax      -> s_free[b]      : that S read
+//   softmax      -> p_full[b]      : P of that tile in shared buffer b (and its stale V rows zeroed)
+//   MMA          -> o_bar[b]       : its O += Vᵀ·P done (P buffer b reusable)
+//   MMA + softmax -> k_empty[n % K] : K slot done with: its S complete (commit; a plain arrival
+//                    for a tile with no rows), metadata read by every softmax warp
+//   MMA          -> v_empty[n % V] : V slot done with: its O += Vᵀ·P complete (commit; a plain
+//                    arrival for a tile with no rows)
 // Each tile's heads are split between the two softmax groups; they take every
 // decision that touches the shared O accumulator (a rescale restarts it) together.
 // NH (4, 8 or 16 >= g) bounds the heads the softmax works on; the operand layouts
@@ -217,16 +223,17 @@ template <bool OUT_F32, int NH, int GROUPS>
 __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm)
     decode_gqa_tc_fp8_kernel(const __grid_constant__ Args args) {
   using C = Cfg<GROUPS>;
-  constexpr int kStages = C::kStages, kQSlots = C::kQSlots, kSoftmax = C::kSoftmax;
+  constexpr int kKStages = C::kKStages, kVStages = C::kVStages, kQSlots = C::kQSlots, kSoftmax = C::kSoftmax;
   constexpr int kProducerWarp = C::kProducerWarp, kMmaWarp = C::kMmaWarp;
-  constexpr int kOffStage = C::kOffStage, kOffQ = C::kOffQ, kOffP = C::kOffP, kOffRed = C::kOffRed;
+  constexpr int kOffK = C::kOffK, kOffV = C::kOffV, kOffQ = C::kOffQ, kOffP = C::kOffP, kOffRed = C::kOffRed;
   constexpr int kOffMeta = C::kOffMeta, kOffScale = C::kOffScale, kOffQinv = C::kOffQinv, kOffBar = C::kOffBar;
   constexpr int kOffMisc = C::kOffMisc;
   const DecodeArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* stage8 = smem + kOffStage;
+  unsigned char* k_ring = smem + kOffK;
+  unsigned char* v_ring = smem + kOffV;
   unsigned char* q_ring = smem + kOffQ;
   unsigned char* p_buf = smem + kOffP;
   float* red = reinterpret_cast<float*>(smem + kOffRed);
@@ -234,9 +241,11 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
   float2* mscale = reinterpret_cast<float2*>(smem + kOffScale);
   float* qinv = reinterpret_cast<float*>(smem + kOffQinv);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* full = bars;
-  uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;
+  uint64_t* k_full = bars;                 // [K slot]: K (and on an item's first tile its queries) landed
+  uint64_t* k_empty = k_full + kKStages;   // [K slot]: S done with K, metadata read by the softmax warps
+  uint64_t* v_full = k_empty + kKStages;   // [V slot]: V landed
+  uint64_t* v_empty = v_full + kVStages;   // [V slot]: O += Vᵀ·P done with V
+  uint64_t* s_full = v_empty + kVStages;
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_bar = p_full + 2;
@@ -251,9 +260,13 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
   const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4 * GROUPS);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1 + 4 * GROUPS);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -320,14 +333,32 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
     int4 tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
     float2 sc_nxt = load_scales(item_nxt);
     PlanEntry e_nx2 = load_entry(item_nx2);
-    int n = 0, item_ord = 0;
+    // Tile n's K (with its metadata, and an item's queries on its first tile) goes out before
+    // tile n-1's V, so the S side runs a tile ahead of the V side.  Each lane remembers its V
+    // slice (source row, or -1) of the last K-issued tile for that V fill.
+    int n = 0, vn = 0, item_ord = 0;  // K fills and V fills issued
     bool failed = false;
-    auto acquire = [&](int slot) -> bool {
-      if (n >= kStages && !mbar_wait(&empty[slot], ((n / kStages) - 1) & 1)) {
+    auto acquire = [&](uint64_t* empty_bar, int fills, int depth) -> bool {
+      // warp-uniform: the copies below are per lane
+      if (fills >= depth && !__all_sync(0xffffffffu, mbar_wait(&empty_bar[fills % depth], ((fills / depth) - 1) & 1))) {
         *abort_flag = 1;
         set_status(a.status, PKV_DEV_TIMEOUT);
         return false;
       }
+      return true;
+    };
+    int pend_row = -1;
+    uint32_t pend_mask = 0;
+    bool pending = false;  // the V of the last K-issued tile is still to go
+    auto issue_v = [&]() -> bool {
+      if (!acquire(v_empty, vn, kVStages)) return false;
+      const int vs = vn % kVStages;
+      if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], __popc(pend_mask) * kSliceTx);
+      __syncwarp();
+      if (pend_row >= 0)
+        tc::tma_load_2d(v_ring + vs * kTile8 + lane * kChunk * kRow8, &args.tm_v, 0, pend_row, &v_full[vs], policy);
+      ++vn;
+      pending = false;
       return true;
     };
     while (item < n_items && !failed && !*abort_flag) {
@@ -337,7 +368,7 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       const int ntiles = ntok == 0 ? 1 : (ntok + kTile - 1) / kTile;
       const int qslot = item_ord % kQSlots;
       for (int tile = 0; tile < ntiles; ++tile, ++n) {
-        const int slot = n % kStages;
+        const int slot = n % kKStages;
         const int n_valid = max(0, min(kTile, ntok - tile * kTile));
         const int nchunks = (n_valid + kChunk - 1) / kChunk;
         const int ltok = tile * kTile + lane * kChunk;  // this lane's slice (lane < nchunks)
@@ -351,7 +382,7 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
         const bool ok = mine && phys >= 0 && phys < a.num_blocks;
         const uint32_t mask = __ballot_sync(0xffffffffu, ok);
         if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
-        if (!acquire(slot)) {
+        if (!acquire(k_empty, n, kKStages)) {
           failed = true;
           break;
         }
@@ -361,20 +392,25 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
                                  n_valid | (mask << 8) | (tile == 0 ? kMetaFirst : 0) |
                                      (tile == ntiles - 1 ? kMetaLast : 0));
           mscale[slot] = sc_cur;
-          mbar_arrive_expect_tx(&full[slot], __popc(mask) * kChunkTx + (with_q ? kQSlot + 16 * 4 : 0));
+          mbar_arrive_expect_tx(&k_full[slot], __popc(mask) * kSliceTx + (with_q ? kQSlot + 16 * 4 : 0));
         }
         __syncwarp();
-        if (ok) {
-          const int r = (phys * a.num_kv_heads + kvh) * a.block_size + ltok % a.block_size;
-          unsigned char* dst = stage8 + slot * kStage8 + lane * kChunk * kRow8;
-          tc::tma_load_2d(dst, &args.tm_k, 0, r, &full[slot], policy);
-          tc::tma_load_2d(dst + kVOff, &args.tm_v, 0, r, &full[slot], policy);
-        }
+        const int r = ok ? (phys * a.num_kv_heads + kvh) * a.block_size + ltok % a.block_size : -1;
+        if (ok) tc::tma_load_2d(k_ring + slot * kTile8 + lane * kChunk * kRow8, &args.tm_k, 0, r, &k_full[slot], policy);
         if (with_q && lane == 0) {
           const int64_t unit = static_cast<int64_t>(e.x) * a.num_kv_heads + kvh;
-          tc::tma_load_2d(q_ring + qslot * kQSlot, &args.tm_q, 0, static_cast<int>(unit * 32), &full[slot], policy);
-          bulk_copy_g2s(qinv + qslot * 16, a.q_inv + unit * 16, 16 * 4, &full[slot], policy);
+          tc::tma_load_2d(q_ring + qslot * kQSlot, &args.tm_q, 0, static_cast<int>(unit * 32), &k_full[slot], policy);
+          bulk_copy_g2s(qinv + qslot * 16, a.q_inv + unit * 16, 16 * 4, &k_full[slot], policy);
         }
+        // then the previous tile's V
+        if (pending && !issue_v()) {
+          failed = true;
+          ++n;
+          break;
+        }
+        pend_row = r;
+        pend_mask = mask;
+        pending = true;
       }
       item = item_nxt;
       item_nxt = item_nx2;
@@ -388,19 +424,22 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       sc_nxt = load_scales(item_nxt);
       e_nx2 = load_entry(item_nx2);
     }
+    if (!failed && !*abort_flag && pending && !issue_v()) failed = true;
     if (!failed && !*abort_flag) {
-      const int slot = n % kStages;
-      if (acquire(slot)) {
+      // end of stream: a K fill with no data
+      const int slot = n % kKStages;
+      if (acquire(k_empty, n, kKStages)) {
         if (lane == 0) {
           meta[slot] = make_int4(0, 0, 0, kMetaEnd);
-          mbar_arrive_expect_tx(&full[slot], 0);
+          mbar_arrive_expect_tx(&k_full[slot], 0);
         }
         ++n;
       }
       __syncwarp();
     }
     // Let this CTA's last copies land before the final barrier.
-    for (int k = max(0, n - kStages); k < n; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1);
+    for (int k = max(0, n - kKStages); k < n; ++k) mbar_wait(&k_full[k % kKStages], (k / kKStages) & 1);
+    for (int k = max(0, vn - kVStages); k < vn; ++k) mbar_wait(&v_full[k % kVStages], (k / kVStages) & 1);
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer (one thread) =================
     if (lane == 0) {
@@ -409,7 +448,7 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       constexpr uint32_t idesc_pv = tc::instr_desc_e4m3(kD, 3 * kN) | (1u << 10) | (1u << 15) | (1u << 16);
       const uint32_t p_addr0 = smem_addr(p_buf);
       int q_valid = 0, p_valid = 0;  // valid tiles that got their QK / PV
-      int prev_slot = -1, prev_nv = 0;
+      int prev_v = -1, prev_nv = 0;  // the held tile: its V fill (= tile index), its valid rows
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t parity) {
         if (ok && !mbar_wait(bar, parity)) {
@@ -422,12 +461,14 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       // O += Vᵀ·P of the held tile (its P in buffer p_valid & 1)
       auto issue_pv = [&]() {
         const int b = p_valid & 1;
+        const int vs = prev_v % kVStages;
+        if (!wait(&v_full[vs], (prev_v / kVStages) & 1)) return;
         if (!wait(&p_full[b], (p_valid >> 1) & 1)) return;
         tc::tc_fence_after();
         const int rf = restart_flag[b];
         const bool restart = rf & 1;
         const uint32_t o_col = kColO + ((rf >> 1) & 1) * kOStride;
-        const uint32_t v_addr = smem_addr(stage8 + prev_slot * kStage8 + kVOff);
+        const uint32_t v_addr = smem_addr(v_ring + vs * kTile8);
         const uint32_t p_addr = p_addr0 + b * kPBytes;
         const int kt = (prev_nv + 31) / 32;
         for (int kk = 0; kk < kt; ++kk) {
@@ -436,19 +477,22 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
                       tc::smem_desc_plain(p_addr + kk * 512, 128, kPTerm), idesc_pv, kk > 0 || !restart);
         }
         tc::umma_commit(&o_bar[b]);
-        tc::umma_commit(&empty[prev_slot]);
+        tc::umma_commit(&v_empty[vs]);
         ++p_valid;
-        prev_slot = -1;
+        prev_v = -1;
       };
       for (int n = 0; ok; ++n) {
-        const int slot = n % kStages;
-        if (!wait(&full[slot], (n / kStages) & 1)) break;
+        const int slot = n % kKStages;
+        if (!wait(&k_full[slot], (n / kKStages) & 1)) break;
         const int4 mt = meta[slot];
         if (mt.w & kMetaEnd) break;
         const int nv = mt.w & 0xff;
         if (nv == 0) {
-          if (prev_slot >= 0) issue_pv();
-          mbar_arrive(&empty[slot]);
+          if (prev_v >= 0) issue_pv();
+          // a tile with no rows: no S to wait for, and its V fill carries no data; release both
+          mbar_arrive(&k_empty[slot]);
+          if (!wait(&v_full[n % kVStages], (n / kVStages) & 1)) break;
+          mbar_arrive(&v_empty[n % kVStages]);
           continue;
         }
         // S = K·[hi; lo]ᵀ of tile n
@@ -456,20 +500,21 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
         const int b = q_valid & 1;
         if (q_valid >= 2 && !wait(&s_free[b], ((q_valid >> 1) - 1) & 1)) break;
         tc::tc_fence_after();
-        const uint32_t k_addr = smem_addr(stage8 + slot * kStage8);
+        const uint32_t k_addr = smem_addr(k_ring + slot * kTile8);
         const uint32_t q_addr = smem_addr(q_ring + qs * kQSlot);
 #pragma unroll
         for (int kk = 0; kk < kD / 32; ++kk)
           tc::umma_f8(tmem + b * 32, tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024),
                       tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024), idesc_qk, kk > 0);
         tc::umma_commit(&s_full[b]);
+        tc::umma_commit(&k_empty[slot]);  // K is free once S is done
         ++q_valid;
         // then O += Vᵀ·P of the previous valid tile
-        if (prev_slot >= 0) issue_pv();
-        prev_slot = slot;
+        if (prev_v >= 0) issue_pv();
+        prev_v = n;
         prev_nv = nv;
       }
-      if (ok && prev_slot >= 0) issue_pv();
+      if (ok && prev_v >= 0) issue_pv();
       // every MMA of this CTA is done before the tensor memory is freed
       tc::umma_commit(drain);
       mbar_wait(drain, 0);
@@ -568,8 +613,8 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
     };
     bool ended = false;
     for (int n = 0;; ++n) {
-      const int slot = n % kStages;
-      bool bad = !mbar_wait(&full[slot], (n / kStages) & 1);
+      const int slot = n % kKStages;
+      bool bad = !mbar_wait(&k_full[slot], (n / kKStages) & 1);
       const int4 mt = meta[slot];
       const float2 sc = mscale[slot];
       if (bad) *abort_flag = 1;
@@ -596,7 +641,7 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);  // metadata (and this item's query scales) read
+      if (lane == 0) mbar_arrive(&k_empty[slot]);  // metadata (and this item's query scales) read
       if (n_valid > 0) {
         const int b = n_valid_tiles & 1;
         unsigned char* p_tile = p_buf + b * kPBytes;
@@ -610,12 +655,16 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
         if (lane == 0) mbar_arrive(&s_free[b]);
         bad |= !wait_ob(b);  // P buffer b: the P·V of two valid tiles back is done
         const bool valid = t < n_valid && ((mask >> (t / kChunk)) & 1);
-        if (!valid) {
-          // V rows outside the context may hold anything (even NaN codes): zero them
-          // (each group half of the row)
-          uint4* vr = reinterpret_cast<uint4*>(stage8 + slot * kStage8 + kVOff + t * kRow8) + (8 / GROUPS) * G;
+        if (n_valid < kTile || mask != 0xffu) {  // uniform: the tile has rows outside the context
+          // V rows outside the context may hold anything (even NaN codes): zero them once the
+          // tile's V has landed (each group half of the row)
+          const int vs = n % kVStages;
+          bad |= !mbar_wait(&v_full[vs], (n / kVStages) & 1);
+          if (!valid) {
+            uint4* vr = reinterpret_cast<uint4*>(v_ring + vs * kTile8 + t * kRow8) + (8 / GROUPS) * G;
 #pragma unroll
-          for (int c = 0; c < 8 / GROUPS; ++c) vr[c] = make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < 8 / GROUPS; ++c) vr[c] = make_uint4(0, 0, 0, 0);
+          }
         }
         float x[NL];
         bool need = false;

@@ -81,10 +81,16 @@ constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
 //     3 K and 2 V slots each.  Registers: launched at 128 (2 x 256 x 128 = 65536), softmax 184,
 //     control 72: 128 x (184 + 72) = 32768 per CTA, and per scheduler 2 CTAs x 32 x 256 =
 //     16384.
+#ifndef PKV_FP8_K2
+#define PKV_FP8_K2 5
+#endif
+#ifndef PKV_FP8_V2
+#define PKV_FP8_V2 4
+#endif
 template <int GROUPS>
 struct Cfg {
-  static constexpr int kKStages = GROUPS == 2 ? 5 : 3;
-  static constexpr int kVStages = GROUPS == 2 ? 4 : 2;
+  static constexpr int kKStages = GROUPS == 2 ? PKV_FP8_K2 : 3;
+  static constexpr int kVStages = GROUPS == 2 ? PKV_FP8_V2 : 2;
   static constexpr int kQSlots = kKStages + 1;  // by item ordinal; a slot is refilled kQSlots items later
   static constexpr int kSoftmax = 128 * GROUPS;
   static constexpr int kProducerWarp = 4 * GROUPS;

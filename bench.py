@@ -112,15 +112,18 @@ def source_digest(kind: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(key: str, kind: str, layout=None):
+def recorded_traffic(key: str, kind: str, units: int, layout=None):
     """DRAM bytes (read + write) per launch of the profiled kernel from profiles/traffic.json, or
-    None unless the entry was captured on the same kernel sources and the same table layout."""
+    None unless the entry was captured on the same kernel sources, the same table layout and a
+    batch of the same size (`units`: the algorithmic bytes, or flops, of one launch)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             entry = json.load(f).get(key)
     except Exception:
         return None
     if not entry or entry.get("sources") != source_digest(kind) or entry.get("layout") != layout:
+        return None
+    if entry.get("algorithmic_per_launch") != int(units):
         return None
     return int(entry["dram_bytes_per_launch"])
 
@@ -648,7 +651,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": recorded_traffic(w.label + ("+shared" if use_shared else ""),
                                                  "shared" if use_shared else
                                                  ("decode_gqa_tc_fp8" if kv8 else "decode_gqa_tc") if uses_tensor
-                                                 else "decode_simt", w.layout),
+                                                 else "decode_simt", unique_total // args.steps, w.layout),
                      "algorithmic_bytes_per_launch": unique_total // args.steps,
                      "logical_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
                      "kernel": ("paged_attention_decode_shared: setup + shared phase (tcgen05 prefill kernel, every"
@@ -662,9 +665,9 @@ def run_ours(args, rank, world, local_rank):
                      "ms_per_launch": round(dec_ms / args.steps, 4),
                      "ms_per_launch_median": round(statistics.median(a.elapsed_time(b) for a, b in dec_events), 4),
                      # the same achieved figure against the other two denominators
-                     "peaks_gbs": {"copy_measured": peak, "read_stream_in_run": round(read_gbs, 1),
+                     "peaks_gbs": {f"copy_{peak_kind}": peak, "read_stream_in_run": round(read_gbs, 1),
                                    "spec": SPEC_HBM_GBS},
-                     "frac_of": {"copy_measured": round(dec_gbs / peak, 4),
+                     "frac_of": {f"copy_{peak_kind}": round(dec_gbs / peak, 4),
                                  "read_stream_in_run": round(dec_gbs / read_gbs, 4),
                                  "spec": round(dec_gbs / SPEC_HBM_GBS, 4)}},
         "gpu_launches": launches,
@@ -1287,7 +1290,7 @@ def run_prefill(args, rank, world, local_rank):
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "pct_tensor_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(b.name, "prefill"),
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(b.name, "prefill", pw.flops),
                      "algorithmic_flops_per_launch": pw.flops, "peak_kind": peak_kind,
                      "kernel": "paged_attention_prefill: plan + tcgen05 kernel",
                      "ms_per_launch": round(k_ms / args.steps, 4)},

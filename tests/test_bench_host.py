@@ -459,11 +459,31 @@ def test_run_ours_beam_phase_with_stand_ins(pkv, monkeypatch):
     assert cfg["pool"]["saved_by_sharing"] > 0.5
     r = res["roofline"]
     assert r["algorithmic_bytes_per_launch"] < 0.5 * r["logical_bytes_per_launch"]
-    assert r["traffic"] is None                      # no capture on this layout
+    assert r["traffic"] is None                      # the capture was of the 128-prompt batch
     # the first prepared step carries the copies; timed steps replay states 3, 0, 1, 2
     assert calls.get("copy", 0) >= 1
     import json
     json.dumps(res)
+
+
+def test_recorded_traffic_only_for_the_captured_batch(tmp_path, monkeypatch):
+    """A recorded ncu figure is reported only for the kernel sources, table layout and batch
+    size it was captured on."""
+    import json
+    (tmp_path / "profiles").mkdir()
+    digest = bench.source_digest("decode_simt")
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({
+        "b": {"dram_bytes_per_launch": 1234, "sources": digest, "algorithmic_per_launch": 1000},
+        "shared": {"dram_bytes_per_launch": 99, "sources": digest, "algorithmic_per_launch": 10, "layout": "x"}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_digest", lambda kind: digest)
+    assert bench.recorded_traffic("b", "decode_simt", 1000) == 1234
+    assert bench.recorded_traffic("b", "decode_simt", 999) is None          # another batch size
+    assert bench.recorded_traffic("b", "decode_simt", 1000, "x") is None    # another layout
+    assert bench.recorded_traffic("shared", "decode_simt", 10, "x") == 99
+    assert bench.recorded_traffic("missing", "decode_simt", 1000) is None
+    monkeypatch.setattr(bench, "source_digest", lambda kind: "changed")
+    assert bench.recorded_traffic("b", "decode_simt", 1000) is None          # sources changed
 
 
 def test_run_trace_host_logic_with_stand_ins(pkv, monkeypatch):

@@ -817,7 +817,13 @@ def run_trace(args, rank, world, local_rank):
     while the pool allows (their prompt K/V is written by one reshape_and_cache call,
     a synthetic prefill, outside the timed decode work).  Device time of the decode
     work (copy_blocks if any, reshape_and_cache, paged_attention_decode) is summed
-    over the timed steps with CUDA events."""
+    over the timed steps with CUDA events.
+
+    The host never waits for the device inside the loop, as a serving loop would not: each
+    step's tables, lengths and slots go up from pinned memory without blocking, so the host
+    (allocator, launches) runs ahead and a step's kernels are queued before the device reaches
+    them.  Events are read after the last step; the oracle's sampled sequences are gathered on
+    the device at their step and checked at the end."""
     import torch
     import paged_kv_cache_423_b200 as pkv
 
@@ -843,6 +849,13 @@ def run_trace(args, rank, world, local_rank):
     running = {}
     next_id = 0
 
+    def up(a):
+        """Host array -> device tensor without a host wait (pinned staging on a GPU)."""
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if device.type != "cuda":
+            return t.to(device)
+        return t.pin_memory().to(device, non_blocking=True)
+
     def admit(length, budget):
         nonlocal next_id
         if -(-length // p.block_size) > bm.num_free():
@@ -850,35 +863,40 @@ def run_trace(args, rank, world, local_rank):
         sid = next_id
         next_id += 1
         bm.add_seq(sid, length - 1)
-        slots = torch.from_numpy(bm.slots(sid, 0, length - 1)).to(device)
+        slots = up(bm.slots(sid, 0, length - 1))
         k = torch.randn((length - 1, p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
         pkv.reshape_and_cache(k, k, kc, vc, slots, status=status)
         running[sid] = budget
 
     for length, budget in initial:
         admit(length, budget)
-    t_ms = 0.0
-    span_ms = 0.0  # first kernel start to last kernel end per step, host launch gaps included
     alloc_s = 0.0  # host allocator time of the timed steps (append, export, frees)
     seq_steps = 0
     kv_bytes = 0
     launches = 0
+    timed = []  # the events of each timed step
     # CPU-baseline leg: the oracle on one sampled sequence of every 20th timed step, outside
     # the timed decode work; its output also checks the GPU's bf16 output for that sequence.
     oracle_leg = rank == 0 and not args.no_cpu_baseline
     ora = {"bytes": 0, "s": 0.0, "n": 0, "max_abs": 0.0, "error": None}
     ora_rng = wl.rng_for(2003)
+    samples = []
 
-    def oracle_sample_step(ids, tables, lens, q, out):
-        from threadpoolctl import threadpool_limits
-        from oracle import paged_attention
+    def oracle_sample_stash(ids, tables, lens, q, out):
+        """Device copies of one sequence's query, output and blocks, taken in stream order
+        after its step (the pool changes later)."""
         i = int(ora_rng.integers(len(ids)))
         L = int(lens[i])
         need = -(-L // p.block_size)
-        blocks = torch.from_numpy(tables[i][:need].astype(np.int64)).to(device)
-        kh = kc[blocks].view(torch.int16).cpu().numpy().view(np.uint16)
-        vh = vc[blocks].view(torch.int16).cpu().numpy().view(np.uint16)
-        qh = q[i:i + 1].view(torch.int16).cpu().numpy().view(np.uint16)
+        blocks = up(tables[i][:need].astype(np.int64))
+        samples.append((L, need, q[i:i + 1].clone(), out[i:i + 1].clone(), kc[blocks], vc[blocks]))
+
+    def oracle_check(L, need, q1, out1, kb, vb):
+        from threadpoolctl import threadpool_limits
+        from oracle import paged_attention
+        kh = kb.view(torch.int16).cpu().numpy().view(np.uint16)
+        vh = vb.view(torch.int16).cpu().numpy().view(np.uint16)
+        qh = q1.view(torch.int16).cpu().numpy().view(np.uint16)
         t0 = time.perf_counter()
         with threadpool_limits(limits=1):
             ref = paged_attention.paged_decode(qh, kh, vh, np.arange(need, dtype=np.int32)[None, :],
@@ -886,7 +904,7 @@ def run_trace(args, rank, world, local_rank):
         ora["s"] += time.perf_counter() - t0
         ora["bytes"] += L * p.num_kv_heads * p.head_dim * 4
         ora["n"] += 1
-        got = out[i:i + 1].float().cpu().numpy()
+        got = out1.float().cpu().numpy()
         ora["max_abs"] = max(ora["max_abs"], float(np.abs(got - ref).max()))
 
     with ClockSampler(device) as clocks:
@@ -897,14 +915,14 @@ def run_trace(args, rank, world, local_rank):
                 slots, pairs = bm.append_slots(ids)
                 tables, lens = bm.export_tables(ids, max_blocks)
                 a_s = time.perf_counter() - a0
-                d_slots = torch.from_numpy(slots).to(device)
-                d_tables = torch.from_numpy(tables).to(device)
-                d_lens = torch.from_numpy(lens).to(device)
+                d_slots = up(slots)
+                d_tables = up(tables)
+                d_lens = up(lens)
                 q = torch.randn((len(ids), p.num_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
                 k = torch.randn((len(ids), p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
                 out = torch.empty((len(ids), p.num_heads, p.head_dim), dtype=torch.bfloat16, device=device)
                 ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-                pairs_d = torch.from_numpy(pairs).to(device) if len(pairs) else None
+                pairs_d = up(pairs) if len(pairs) else None
                 ev[0].record(stream)
                 if pairs_d is not None:
                     pkv.copy_blocks([kc], [vc], pairs_d, status=status)
@@ -913,21 +931,14 @@ def run_trace(args, rank, world, local_rank):
                 ev[2].record(stream)
                 pkv.paged_attention_decode(out, q, kc, vc, d_tables, d_lens, max_len, scale, ws, status=status)
                 ev[3].record(stream)
-                torch.cuda.synchronize()
                 if step >= args.warmup:
-                    # the step's kernels: the cache write (and copies), then the decode call; the
-                    # host's marshalling of the decode call between the two is not device work
-                    t_ms += ev[0].elapsed_time(ev[1]) + ev[2].elapsed_time(ev[3])
-                    span_ms += ev[0].elapsed_time(ev[3])
+                    timed.append(ev)
                     alloc_s += a_s
                     seq_steps += len(ids)
                     kv_bytes += int(lens.astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 4
                     launches += 3 + (1 if len(pairs) else 0) + 1  # + the split merge
-                    if oracle_leg and ora["error"] is None and (step - args.warmup) % 20 == 0:
-                        try:
-                            oracle_sample_step(ids, tables, lens, q, out)
-                        except Exception as e:  # the trace figure stands without its baseline
-                            ora["error"] = f"{type(e).__name__}: {e}"
+                    if oracle_leg and (step - args.warmup) % 20 == 0:
+                        oracle_sample_stash(ids, tables, lens, q, out)
                 a0 = time.perf_counter()
                 for sid in ids:
                     running[sid] -= 1
@@ -939,7 +950,17 @@ def run_trace(args, rank, world, local_rank):
             for length, budget in arrivals[step]:
                 if len(running) < p.max_batch:
                     admit(length, budget)
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+    # the step's kernels: the cache write (and copies), then the decode call; the host's
+    # marshalling of the decode call between the two is not device work
+    t_ms = sum(ev[0].elapsed_time(ev[1]) + ev[2].elapsed_time(ev[3]) for ev in timed)
+    span_ms = sum(ev[0].elapsed_time(ev[3]) for ev in timed)
+    for smp in samples:
+        if ora["error"] is None:
+            try:
+                oracle_check(*smp)
+            except Exception as e:  # the trace figure stands without its baseline
+                ora["error"] = f"{type(e).__name__}: {e}"
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item():#x}")
     bm.close()
@@ -954,8 +975,9 @@ def run_trace(args, rank, world, local_rank):
                        "initial_lengths": f"U{{{p.len_lo}..{p.len_hi}}}", "budgets": f"U{{{p.budget_lo}..{p.budget_hi}}}",
                        "arrivals": f"Bernoulli({p.arrival_p}) per free slot per step, lengths U{{{p.len_lo}..{p.len_hi}}}",
                        "timed": "copy_blocks + reshape_and_cache, and paged_attention_decode, per step (events"
-                                " around each call: the host's marshalling between the calls is excluded;"
-                                " ms_per_step_span includes it)"},
+                                " around each call; the host runs ahead of the device, with pinned asynchronous"
+                                " uploads and no wait inside the loop; ms_per_step_span = first kernel start"
+                                " to last kernel end of a step)"},
             "ms_per_step_span": round(span_ms / max(1, args.steps), 4),
             "seq_steps_per_s": round(seq_steps / (t_ms * 1e-3), 1), "pct_hbm_peak": round(100 * value / peak, 2),
             # the same with the host allocator's time per step added (it runs between the steps here)

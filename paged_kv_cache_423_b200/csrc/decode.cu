@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(kPlanThreads)
                 int32_t* __restrict__ arrive, int n_arrive, int32_t* status) {
   __shared__ int bucket[kPlanBuckets];
   __shared__ int warp_total[32];
+  griddep_launch_dependents();  // the decode kernel may be scheduled now; it waits for this one to end
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < kPlanBuckets; i += blockDim.x) bucket[i] = 0;
   for (int i = tid; i < n_arrive; i += blockDim.x) arrive[i] = 0;
@@ -306,6 +307,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   Ring& ring = reinterpret_cast<Ring*>(smem_raw)[warp];
   const int qk_row = LaneMap<D, KV8>::row(lane), qk_half = LaneMap<D, KV8>::half(lane);
 
+  griddep_wait();  // the plan kernel before this one has finished
   const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_heads;
   // Work distribution over the plan (longest items first): every warp starts with
   // items w and w + #warps; after that it takes the next unclaimed item from a
@@ -739,8 +741,8 @@ static int launch_simt(const DecodeArgs& a, cudaStream_t stream) {
     return set_error(PKV_ERR_CUDA, "decode (simt) setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::max(1, sms * std::max(1, blocks_per_sm));
-  kernel<<<grid, kSimtWarps * 32, smem, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_after_previous(kernel, dim3(grid), dim3(kSimtWarps * 32), smem, stream, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (simt) launch: %s", cudaGetErrorString(e));
   return PKV_OK;
 }

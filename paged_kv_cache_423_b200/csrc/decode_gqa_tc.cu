@@ -8,10 +8,12 @@
 // softmax(q·Kᵀ)·V over the pages of the block table) on the CUDA cores.
 //
 // Work item = (sequence, partition, kv head), handed out from the same sorted plan
-// as the CUDA-core kernel.  A tile is 128 tokens = 8 slices of 16 rows; each slice
-// of a (block, kv head) tile arrives by TMA (2-D tensor map over the pool viewed as
-// [num_blocks * Hkv * block_size, head_dim], box 64 x 16, 128-byte swizzle), which
-// is exactly the K-major operand layout of the MMA.  Per tile:
+// as the CUDA-core kernel.  A tile is 128 tokens = 8 slices of 16 rows (4 of 32 when
+// the block size is a multiple of 32); each slice of a (block, kv head) tile arrives
+// by TMA (2-D tensor map over the pool viewed as [num_blocks * Hkv * block_size,
+// head_dim], box 64 columns x 16 or 32 rows, 128-byte swizzle), which is exactly the
+// K-major operand layout of the MMA.  The TMA engine's time per box is what limits a
+// single producer warp, so the larger box is used wherever the pool allows it.  Per tile:
 //   S[128 x N]  = K[128 x D] · Q[N x D]ᵀ          (A = K, K-major; B = Q, K-major)
 //   softmax over the 128 rows of each of the g columns (fp32, base 2, online)
 //   O[D x N]    = Vᵀ[D x 128] · P[128 x N]         (A = V, MN-major; B = P, K-major)
@@ -42,7 +44,7 @@ namespace pkv {
 namespace tc {
 
 constexpr int kTile = 128;             // tokens per tile (MMA M)
-constexpr int kChunk = 16;             // rows per TMA box
+constexpr int kChunk = 16;             // rows per validity bit (and per TMA box at block size 16)
 constexpr int kD = 128;                // head_dim of this path
 constexpr int kHalfBytes = kTile * 128;  // one 64-column half of a K or V tile: 16 KiB
 constexpr int kTileBytes = 2 * kHalfBytes;
@@ -52,7 +54,6 @@ constexpr int kMmaWarp = 5;            // tcgen05.mma issue
 constexpr int kThreads = kConsumers + 64;
 constexpr int kTmemCols = 64;          // S double buffer in columns [0,16) and [16,32), O of even / odd
 constexpr uint32_t kColO = 32;         // items in [32,48) and [48,64)
-constexpr uint32_t kChunkTx = 4 * kChunk * 128;  // K and V, two halves each
 
 struct alignas(64) Args {
   CUtensorMap tm_k;
@@ -60,6 +61,9 @@ struct alignas(64) Args {
   CUtensorMap tm_q;
   DecodeArgs a;
 };
+
+// Rows per TMA box: 32 where every 32-row slice stays inside one block, else 16.
+__host__ __device__ constexpr int box_rows(int block_size) { return block_size % 32 == 0 ? 32 : kChunk; }
 
 // ---- shared memory layout -------------------------------------------------
 
@@ -137,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = a.group;
-  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
+  griddep_launch_dependents();  // the merge kernel may be scheduled now; it waits for this one to end
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -162,6 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The set-up above overlaps the plan kernel; its work list is read only after it has finished.
+  griddep_wait();
+  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
 
   if (warp == kProducerWarp) {
     // ================= producer =================
@@ -185,8 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       return t;
     };
     // Items are taken from a global counter in plan order (longest first), so CTAs
-    // that finish early take more.  Item ids, plan entries and table slices are
-    // fetched up to two items ahead.
+    // that finish early take more.  The next item is claimed when the current one's last
+    // tile is issued (its counter, entry and table slice then load while the ring
+    // drains), not earlier: a claimed item waits for this CTA alone, so claiming ahead
+    // would hold work back from CTAs that run out at the end.
     int* work_counter = const_cast<int*>(a.plan_count) + 1;
     auto grab = [&]() -> int64_t {
       int v = 0;
@@ -194,13 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       return __shfl_sync(0xffffffffu, v, 0);
     };
     int64_t item = grab();
-    int64_t item_nxt = grab();
-    int64_t item_nx2 = grab();
+    int64_t item_nxt = n_items;
     PlanEntry e_cur = load_entry(item);
     int4 tab_cur = item < n_items ? load_tab(e_cur) : make_int4(0, 0, 0, 0);
-    PlanEntry e_nxt = load_entry(item_nxt);
-    int4 tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
-    PlanEntry e_nx2 = load_entry(item_nx2);
+    const int crow = box_rows(a.block_size);
     int n = 0;  // fills issued
     int item_ord = 0;
     bool failed = false;
@@ -220,13 +226,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
       const int qslot = item_ord % L::kQSlots;
       for (int tile = 0; tile < ntiles; ++tile, ++n) {
         const int slot = n % STAGES;
+        if (tile == ntiles - 1) item_nxt = grab();
         if (!acquire(slot)) {
           failed = true;
           break;
         }
         const int n_valid = max(0, min(kTile, ntok - tile * kTile));
-        const int nchunks = (n_valid + kChunk - 1) / kChunk;
-        const int ltok = tile * kTile + lane * kChunk;  // this lane's chunk (lane < nchunks)
+        const int nchunks = (n_valid + crow - 1) / crow;
+        const int ltok = tile * kTile + lane * crow;  // this lane's box (lane < nchunks)
         const int blk = min(127, ltok / a.block_size);
         const int p0 = __shfl_sync(0xffffffffu, tab_cur.x, blk & 31);
         const int p1 = __shfl_sync(0xffffffffu, tab_cur.y, blk & 31);
@@ -235,19 +242,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         const int phys = blk < 32 ? p0 : blk < 64 ? p1 : blk < 96 ? p2 : p3;
         const bool mine = lane < nchunks;
         const bool ok = mine && phys >= 0 && phys < a.num_blocks;
-        const uint32_t mask = __ballot_sync(0xffffffffu, ok);
+        const uint32_t boxes = __ballot_sync(0xffffffffu, ok);
+        // validity per 16-row slice (a 32-row box covers two)
+        uint32_t mask = boxes;
+        if (crow == 32) {
+          mask = 0;
+#pragma unroll
+          for (int i = 0; i < kTile / 32; ++i)
+            if ((boxes >> i) & 1) mask |= 3u << (2 * i);
+        }
         if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
         const bool with_q = tile == 0 && ntok > 0;
         if (lane == 0) {
           meta[slot] = make_int4(e.x, kvh | (qslot << 16), e.y | (e.z << 16),
                                  n_valid | (mask << 8) | (tile == 0 ? kMetaFirst : 0) | (tile == ntiles - 1 ? kMetaLast : 0));
-          mbar_arrive_expect_tx(&full[slot], __popc(mask) * kChunkTx + (with_q ? L::kQBytes : 0));
+          // K and V of each landed box, two 64-column halves each
+          mbar_arrive_expect_tx(&full[slot], __popc(boxes) * (4u * crow * 128u) + (with_q ? L::kQBytes : 0));
         }
         __syncwarp();
         if (ok) {
           const int row = (phys * a.num_kv_heads + kvh) * a.block_size + ltok % a.block_size;
-          unsigned char* kd = k_ring + slot * kTileBytes + lane * kChunk * 128;
-          unsigned char* vd = v_ring + slot * kTileBytes + lane * kChunk * 128;
+          unsigned char* kd = k_ring + slot * kTileBytes + lane * crow * 128;
+          unsigned char* vd = v_ring + slot * kTileBytes + lane * crow * 128;
           tma_load_2d(kd, &args.tm_k, 0, row, &full[slot], policy);
           tma_load_2d(kd + kHalfBytes, &args.tm_k, 64, row, &full[slot], policy);
           tma_load_2d(vd, &args.tm_v, 0, row, &full[slot], policy);
@@ -263,14 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gqa_tc_kernel(const __grid
         }
       }
       item = item_nxt;
-      item_nxt = item_nx2;
-      item_nx2 = grab();
       ++item_ord;
-      e_cur = e_nxt;
-      tab_cur = tab_nxt;
-      e_nxt = e_nx2;
-      tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
-      e_nx2 = load_entry(item_nx2);
+      e_cur = load_entry(item);
+      tab_cur = item < n_items ? load_tab(e_cur) : make_int4(0, 0, 0, 0);
     }
     if (!failed && !*abort_flag) {
       // end-of-stream marker: a fill with no data
@@ -614,6 +625,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_partials_kernel(const 
   int L = a.context_lens[seq];
   if (L < 0 || L > a.max_context_len || L > a.max_blocks * a.block_size) L = 0;  // as the plan does
   const int nparts = L == 0 ? 1 : (L + a.partition - 1) / a.partition;
+  griddep_wait();  // the decode kernel has finished: its partials are visible
   if (nparts <= 1) return;  // written directly by the main kernel
   const int64_t unit = static_cast<int64_t>(seq) * a.num_heads + h;
   const float2* ml = a.part_ml + unit * a.max_parts;
@@ -696,8 +708,8 @@ static int launch(const Args& args, cudaStream_t stream) {
   const int st = set_smem_limit_once(setup, kernel, smem, &dev);
   if (st != 0) return set_error(PKV_ERR_CUDA, "decode (tensor) setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  kernel<<<std::max(1, sms), kThreads, smem, stream>>>(args);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_after_previous(kernel, dim3(std::max(1, sms)), dim3(kThreads), smem, stream, args);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (tensor) launch: %s", cudaGetErrorString(e));
   return args.a.always_partial ? PKV_OK : launch_merge_partials(args.a, OUT_F32, stream);
 }
@@ -706,12 +718,10 @@ static int launch(const Args& args, cudaStream_t stream) {
 
 int launch_merge_partials(const DecodeArgs& a, bool out_f32, cudaStream_t stream) {
   if (a.max_parts <= 1) return PKV_OK;
-  const int grid = a.num_seqs * a.num_heads;
-  if (out_f32)
-    tc::merge_partials_kernel<true><<<grid, tc::kMergeWarps * 32, 0, stream>>>(a);
-  else
-    tc::merge_partials_kernel<false><<<grid, tc::kMergeWarps * 32, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  const dim3 grid(a.num_seqs * a.num_heads), block(tc::kMergeWarps * 32);
+  cudaError_t e = out_f32 ? launch_after_previous(tc::merge_partials_kernel<true>, grid, block, 0, stream, a)
+                          : launch_after_previous(tc::merge_partials_kernel<false>, grid, block, 0, stream, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode merge launch: %s", cudaGetErrorString(e));
   return PKV_OK;
 }
@@ -725,8 +735,9 @@ int launch_decode_tensor(const DecodeArgs& a, int head_dim, bool out_f32, cudaSt
   args.a = a;
   constexpr int n = 16;
   const uint64_t pool_rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
-  int rc = tc::encode_map(&args.tm_k, a.key_cache, pool_rows, tc::kChunk, "key_cache");
-  if (rc == PKV_OK) rc = tc::encode_map(&args.tm_v, a.value_cache, pool_rows, tc::kChunk, "value_cache");
+  const uint32_t rows = static_cast<uint32_t>(tc::box_rows(a.block_size));
+  int rc = tc::encode_map(&args.tm_k, a.key_cache, pool_rows, rows, "key_cache");
+  if (rc == PKV_OK) rc = tc::encode_map(&args.tm_v, a.value_cache, pool_rows, rows, "value_cache");
   if (rc == PKV_OK)
     rc = tc::encode_map(&args.tm_q, a.query, static_cast<uint64_t>(a.num_seqs) * a.num_heads, n, "query");
   if (rc != PKV_OK) return rc;

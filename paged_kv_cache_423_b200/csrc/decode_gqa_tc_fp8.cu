@@ -47,7 +47,7 @@ namespace tc8 {
 using tc::fast_exp2;
 
 constexpr int kTile = 128;                 // tokens per tile (MMA M of S)
-constexpr int kChunk = 16;                 // rows per TMA box: a 16-row slice of one (block, kv head)
+constexpr int kChunk = 16;                 // rows per validity bit (and per TMA box at block size 16)
 constexpr int kD = 128;
 constexpr int kN = 16;                     // query heads of one kv head (g <= 16)
 constexpr int kRow8 = kD;                  // bytes of one e4m3 row
@@ -58,12 +58,15 @@ constexpr int kPBytes = 3 * kPTerm;        // [hi | mid | lo]
 constexpr uint32_t kTmemCols = 256;        // S double buffer [0,32), [32,64) (hi | lo); O of even / odd items
 constexpr uint32_t kColO = 64;             // at [64,112) / [128,176) (3 terms of 16 heads each)
 constexpr uint32_t kOStride = 64;
-constexpr uint32_t kSliceTx = kChunk * kRow8;  // one 16-row slice of K or of V
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kPShift = 7.f;             // P is stored times 2^7 (at most 2^15)
 // Stage metadata: x = sequence, y = kv head | q slot << 16, z = partition | partitions << 16,
 // w = valid rows (8 bits) | slice mask << 8 | first << 16 | last << 17 | end of stream << 18
 constexpr int kMetaFirst = 1 << 16, kMetaLast = 1 << 17, kMetaEnd = 1 << 18;
+
+// Rows per TMA box: 32 where every 32-row slice stays inside one block, else 16 (the TMA
+// engine's time per box limits a producer warp, so the larger box is used where it can be).
+__host__ __device__ constexpr int box_rows(int block_size) { return block_size % 32 == 0 ? 32 : kChunk; }
 
 // K and V of a tile travel in separate rings: a K slot is free again once the tile's S = K·Qᵀ
 // is done, a V slot only once its O += Vᵀ·P is, so K (and with it the next tiles' S) runs a
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = a.group;
-  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
+  griddep_launch_dependents();  // the merge kernel may be scheduled now; it waits for this one to end
 
   if (tid == 0) {
     for (int s = 0; s < kKStages; ++s) {
@@ -292,6 +295,10 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The set-up above overlaps the kernels before this one (plan, query split); the work list
+  // and the split queries are read only after they have finished.
+  griddep_wait();
+  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
 
   if (warp >= kProducerWarp) {
   // The control warpgroup gives registers back; the branch is uniform per warpgroup,
@@ -328,17 +335,14 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       if (lane == 0) v = atomicAdd(work_counter, 1);
       return __shfl_sync(0xffffffffu, v, 0);
     };
-    // item ids, entries, scales and table slices are fetched ahead, as in the bf16 kernel
+    // The next item is claimed when the current one's last tile is issued, as in the bf16
+    // kernel: a claimed item waits for this CTA alone.
     int64_t item = grab();
-    int64_t item_nxt = grab();
-    int64_t item_nx2 = grab();
+    int64_t item_nxt = n_items;
     PlanEntry e_cur = load_entry(item);
     int4 tab_cur = item < n_items ? load_tab(e_cur) : make_int4(0, 0, 0, 0);
     float2 sc_cur = load_scales(item);
-    PlanEntry e_nxt = load_entry(item_nxt);
-    int4 tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
-    float2 sc_nxt = load_scales(item_nxt);
-    PlanEntry e_nx2 = load_entry(item_nx2);
+    const int crow = box_rows(a.block_size);
     // Tile n's K (with its metadata, and an item's queries on its first tile) goes out before
     // tile n-1's V, so the S side runs a tile ahead of the V side.  Each lane remembers its V
     // slice (source row, or -1) of the last K-issued tile for that V fill.
@@ -354,15 +358,15 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       return true;
     };
     int pend_row = -1;
-    uint32_t pend_mask = 0;
+    uint32_t pend_boxes = 0;
     bool pending = false;  // the V of the last K-issued tile is still to go
     auto issue_v = [&]() -> bool {
       if (!acquire(v_empty, vn, kVStages)) return false;
       const int vs = vn % kVStages;
-      if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], __popc(pend_mask) * kSliceTx);
+      if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], __popc(pend_boxes) * static_cast<uint32_t>(crow * kRow8));
       __syncwarp();
       if (pend_row >= 0)
-        tc::tma_load_2d(v_ring + vs * kTile8 + lane * kChunk * kRow8, &args.tm_v, 0, pend_row, &v_full[vs], policy);
+        tc::tma_load_2d(v_ring + vs * kTile8 + lane * crow * kRow8, &args.tm_v, 0, pend_row, &v_full[vs], policy);
       ++vn;
       pending = false;
       return true;
@@ -375,9 +379,10 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       const int qslot = item_ord % kQSlots;
       for (int tile = 0; tile < ntiles; ++tile, ++n) {
         const int slot = n % kKStages;
+        if (tile == ntiles - 1) item_nxt = grab();
         const int n_valid = max(0, min(kTile, ntok - tile * kTile));
-        const int nchunks = (n_valid + kChunk - 1) / kChunk;
-        const int ltok = tile * kTile + lane * kChunk;  // this lane's slice (lane < nchunks)
+        const int nchunks = (n_valid + crow - 1) / crow;
+        const int ltok = tile * kTile + lane * crow;  // this lane's box (lane < nchunks)
         const int blk = min(127, ltok / a.block_size);
         const int p0 = __shfl_sync(0xffffffffu, tab_cur.x, blk & 31);
         const int p1 = __shfl_sync(0xffffffffu, tab_cur.y, blk & 31);
@@ -386,7 +391,15 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
         const int phys = blk < 32 ? p0 : blk < 64 ? p1 : blk < 96 ? p2 : p3;
         const bool mine = lane < nchunks;
         const bool ok = mine && phys >= 0 && phys < a.num_blocks;
-        const uint32_t mask = __ballot_sync(0xffffffffu, ok);
+        const uint32_t boxes = __ballot_sync(0xffffffffu, ok);
+        // validity per 16-row slice (a 32-row box covers two)
+        uint32_t mask = boxes;
+        if (crow == 32) {
+          mask = 0;
+#pragma unroll
+          for (int i = 0; i < kTile / 32; ++i)
+            if ((boxes >> i) & 1) mask |= 3u << (2 * i);
+        }
         if (mine && !ok) set_status(a.status, PKV_DEV_BAD_BLOCK);
         if (!acquire(k_empty, n, kKStages)) {
           failed = true;
@@ -398,11 +411,12 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
                                  n_valid | (mask << 8) | (tile == 0 ? kMetaFirst : 0) |
                                      (tile == ntiles - 1 ? kMetaLast : 0));
           mscale[slot] = sc_cur;
-          mbar_arrive_expect_tx(&k_full[slot], __popc(mask) * kSliceTx + (with_q ? kQSlot + 16 * 4 : 0));
+          mbar_arrive_expect_tx(&k_full[slot],
+                                __popc(boxes) * static_cast<uint32_t>(crow * kRow8) + (with_q ? kQSlot + 16 * 4 : 0));
         }
         __syncwarp();
         const int r = ok ? (phys * a.num_kv_heads + kvh) * a.block_size + ltok % a.block_size : -1;
-        if (ok) tc::tma_load_2d(k_ring + slot * kTile8 + lane * kChunk * kRow8, &args.tm_k, 0, r, &k_full[slot], policy);
+        if (ok) tc::tma_load_2d(k_ring + slot * kTile8 + lane * crow * kRow8, &args.tm_k, 0, r, &k_full[slot], policy);
         if (with_q && lane == 0) {
           const int64_t unit = static_cast<int64_t>(e.x) * a.num_kv_heads + kvh;
           tc::tma_load_2d(q_ring + qslot * kQSlot, &args.tm_q, 0, static_cast<int>(unit * 32), &k_full[slot], policy);
@@ -415,20 +429,14 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
           break;
         }
         pend_row = r;
-        pend_mask = mask;
+        pend_boxes = boxes;
         pending = true;
       }
       item = item_nxt;
-      item_nxt = item_nx2;
-      item_nx2 = grab();
       ++item_ord;
-      e_cur = e_nxt;
-      tab_cur = tab_nxt;
-      sc_cur = sc_nxt;
-      e_nxt = e_nx2;
-      tab_nxt = item_nxt < n_items ? load_tab(e_nxt) : make_int4(0, 0, 0, 0);
-      sc_nxt = load_scales(item_nxt);
-      e_nx2 = load_entry(item_nx2);
+      e_cur = load_entry(item);
+      tab_cur = item < n_items ? load_tab(e_cur) : make_int4(0, 0, 0, 0);
+      sc_cur = load_scales(item);
     }
     if (!failed && !*abort_flag && pending && !issue_v()) failed = true;
     if (!failed && !*abort_flag) {
@@ -803,10 +811,9 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
 // 128-byte swizzle on load); rows of heads g .. 15 are zero.  2^-e goes to q_inv[unit][r].
 constexpr int kSplitWarps = 4;
 
-__global__ void __launch_bounds__(kSplitWarps * 32) split_queries_kernel(const DecodeArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kSplitWarps + warp;
-  if (unit >= static_cast<int64_t>(a.num_seqs) * a.num_kv_heads) return;  // warp-uniform
+// One (sequence, kv head): its g query rows split into e4m3 [hi; lo] rows and a power-of-two
+// scale per head (lane = row r, half h).
+__device__ __forceinline__ void split_unit(const DecodeArgs& a, int64_t unit, int lane) {
   const int seq = static_cast<int>(unit / a.num_kv_heads), kvh = static_cast<int>(unit % a.num_kv_heads);
   const int g = a.group;
   const int r = lane >> 1, h = lane & 1;
@@ -845,6 +852,16 @@ __global__ void __launch_bounds__(kSplitWarps * 32) split_queries_kernel(const D
   if (h == 0) a.q_inv[unit * 16 + r] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
 }
 
+__global__ void __launch_bounds__(kSplitWarps * 32) split_queries_kernel(const DecodeArgs a) {
+  griddep_launch_dependents();  // the decode kernel may be scheduled now
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kSplitWarps + warp;
+  // The split reads only the caller's queries and writes only its own rows, so it runs beside
+  // the plan kernel before it; it waits for the plan only to end after it.
+  if (unit < static_cast<int64_t>(a.num_seqs) * a.num_kv_heads) split_unit(a, unit, lane);  // warp-uniform
+  griddep_wait();
+}
+
 // ---- host side -----------------------------------------------------------------
 
 // 2-D view [rows, 128] bytes with a 128-byte swizzle, box 128 x box_rows: the e4m3 pool
@@ -877,8 +894,9 @@ static int launch(const Args& args, cudaStream_t stream) {
   if (st != 0)
     return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  kernel<<<std::max(1, sms * C::kCtasPerSm), C::kThreads, kSmemBytes, stream>>>(args);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e =
+      launch_after_previous(kernel, dim3(std::max(1, sms * C::kCtasPerSm)), dim3(C::kThreads), kSmemBytes, stream, args);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) launch: %s", cudaGetErrorString(e));
   return PKV_OK;
 }
@@ -894,14 +912,16 @@ int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cu
   const uint64_t pool_rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
   if (!a.q_split || !a.q_inv) return set_error(PKV_ERR_INVALID, "decode (8-bit tensor): no split-query workspace");
   const uint64_t units = static_cast<uint64_t>(a.num_seqs) * a.num_kv_heads;
-  int rc = tc8::encode_map(&args.tm_k, a.key_cache8, pool_rows, tc8::kChunk, "key_cache");
-  if (rc == PKV_OK) rc = tc8::encode_map(&args.tm_v, a.value_cache8, pool_rows, tc8::kChunk, "value_cache");
+  const int rows = tc8::box_rows(a.block_size);
+  int rc = tc8::encode_map(&args.tm_k, a.key_cache8, pool_rows, rows, "key_cache");
+  if (rc == PKV_OK) rc = tc8::encode_map(&args.tm_v, a.value_cache8, pool_rows, rows, "value_cache");
   if (rc == PKV_OK) rc = tc8::encode_map(&args.tm_q, a.q_split, units * 32, 32, "split queries");
   if (rc != PKV_OK) return rc;
   if (units > 0) {
     const unsigned grid = static_cast<unsigned>((units + tc8::kSplitWarps - 1) / tc8::kSplitWarps);
-    tc8::split_queries_kernel<<<grid, tc8::kSplitWarps * 32, 0, stream>>>(a);
-    const cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_after_previous(tc8::split_queries_kernel, dim3(grid), dim3(tc8::kSplitWarps * 32), 0,
+                                          stream, a);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess)
       return set_error(PKV_ERR_CUDA, "decode (8-bit tensor) query split launch: %s", cudaGetErrorString(e));
   }

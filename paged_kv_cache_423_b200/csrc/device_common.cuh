@@ -23,6 +23,17 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization
+// (launch_after_previous) may be scheduled while the kernel before it in the stream still
+// runs.  griddep_wait() returns once that kernel has completed and its writes are visible
+// (at once for a normal launch); every thread of such a kernel passes it before reading what
+// the earlier kernel writes, and before leaving, so the kernels of one call complete in order.
+// griddep_launch_dependents() lets the stream's next kernel, if so launched, be scheduled.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }

@@ -22,4 +22,24 @@ inline int set_smem_limit_once(PerDevice<int>& setup, Kernel kernel, int smem, i
       nullptr, static_cast<int>(cudaErrorInvalidDevice));
 }
 
+// Launches `kernel` with programmatic stream serialization: it may be scheduled (and run
+// up to its griddep_wait()) while the previous kernel of `stream` is still running, which
+// hides the launch gap between the kernels of one call.  The kernel must call griddep_wait()
+// in every thread before it reads the previous kernel's output or returns.
+template <typename... KernelParams, typename... Args>
+inline cudaError_t launch_after_previous(void (*kernel)(KernelParams...), dim3 grid, dim3 block, size_t smem,
+                                         cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 }  // namespace pkv

@@ -486,10 +486,12 @@ def test_recorded_traffic_only_for_the_captured_batch(tmp_path, monkeypatch):
     assert bench.recorded_traffic("b", "decode_simt", 1000) is None          # sources changed
 
 
-def test_run_trace_host_logic_with_stand_ins(pkv, monkeypatch):
+@pytest.mark.parametrize("oracle_leg", [False, True])
+def test_run_trace_host_logic_with_stand_ins(pkv, monkeypatch, oracle_leg):
     """The continuous-batching trace bench on the CPU with a shrunken trace (4 slots,
     short contexts, small pool) and stubbed kernels: admissions, frees and the recorded
-    readings, allocator time reported, seq-steps with it below those without."""
+    readings, allocator time reported, seq-steps with it below those without; with the
+    oracle leg, one sampled sequence per 20 timed steps is stashed and checked after the loop."""
     import contextlib
     import types
     import workloads as wl
@@ -509,8 +511,13 @@ def test_run_trace_host_logic_with_stand_ins(pkv, monkeypatch):
     monkeypatch.setattr(pkv, "paged_attention_decode",
                         lambda *a, **k: kernel_calls.__setitem__("decode", kernel_calls["decode"] + 1))
     monkeypatch.setattr(pkv, "copy_blocks", lambda *a, **k: None)
-    args = types.SimpleNamespace(steps=20, warmup=3, no_cpu_baseline=True)
+    args = types.SimpleNamespace(steps=20, warmup=3, no_cpu_baseline=not oracle_leg)
     res = bench.run_trace(args, 0, 1, 0)
+    if oracle_leg:
+        cb = res["cpu_baseline"]
+        assert cb["kind"] == "oracle" and cb["cores"] == 1 and "1 sequences" in cb["sample"], cb
+    else:
+        assert "cpu_baseline" not in res
     cfg = res["config"]
     assert cfg["workload"] == "long_trace_continuous" and cfg["admitted"] > 4
     assert cfg["initial_lengths"] == "U{40..120}" and cfg["budgets"] == "U{1..6}"

@@ -83,15 +83,19 @@ inline int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size,
   return p < block_size ? block_size : p;
 }
 
-// The tensor-core path pays a fixed cost per item (softmax denominators, output or
-// partial, and later a merge): it takes longer splits, up to 2048 tokens, as long
-// as about 16 items per SM remain for load balance.  Never shorter than the
-// CUDA-core split, so a workspace sized for that split always suffices.
+// The tensor-core path pays a fixed cost per item (the first tile's maximum, the
+// output or partial, and later a merge): it takes longer splits, up to 2048 tokens, as
+// long as about 16 items per SM remain for load balance.  With at least 4 (sequence,
+// kv head) units per SM it never splits below 512 tokens: items of one or two tiles
+// would cost about as much in per-item work as in streaming, and the units alone
+// balance the SMs.  Never shorter than the CUDA-core split, so a workspace sized for
+// that split always suffices.
 inline int auto_partition_tokens_tensor(int num_seqs, int num_kv_heads, int block_size, int max_context_len) {
   const int base = auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len);
+  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
   int p = kMaxPartition;
-  while (p > base && static_cast<int64_t>(num_seqs) * num_kv_heads * ((max_context_len + p - 1) / p) < 16 * 148)
-    p /= 2;
+  while (p > base && units * ((max_context_len + p - 1) / p) < 16 * 148) p /= 2;
+  if (units >= 4 * 148 && p < 512) p = 512;
   return p > base ? p : base;
 }
 

@@ -163,7 +163,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = a.group;
-  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -194,6 +193,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The set-up above overlaps the plan kernel (when launched after it); its work list is
+  // read only after it has finished.
+  griddep_wait();
+  const int64_t n_items = static_cast<int64_t>(a.plan_count[0]) * a.num_kv_heads;
   auto fail = [&]() {
     *abort_flag = 1;
     set_status(a.status, PKV_DEV_TIMEOUT);
@@ -689,6 +692,7 @@ __device__ __forceinline__ int plan_bucket(int len, int max_len) {
 __global__ void __launch_bounds__(kPlanThreads) prefill_plan_kernel(const PlanArgs p) {
   __shared__ int cnt[kPlanBuckets];
   __shared__ int total;
+  griddep_launch_dependents();  // the prefill kernel may be scheduled now; it waits for this one to end
   for (int i = threadIdx.x; i < kPlanBuckets; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   const int pair_tokens = 2 * p.tile_tokens;
@@ -789,15 +793,21 @@ static int encode_q_map(CUtensorMap* map, const void* base, int total_q, int num
   return PKV_OK;
 }
 
+// after_plan: launched right after the plan kernel on the same stream, chained to it (the
+// shared-prefix decode's segment launch follows an event wait on its side stream instead).
 template <bool OUT_F32, bool SEG = false>
-static int launch_main(const Args& args, int grid, cudaStream_t stream) {
+static int launch_main(const Args& args, int grid, cudaStream_t stream, bool after_plan) {
   auto kernel = prefill_tc_kernel<OUT_F32, SEG>;
   static PerDevice<int> setup;
   int dev = 0;
   const int st = set_smem_limit_once(setup, kernel, kSmemBytes, &dev);
   if (st != 0) return set_error(PKV_ERR_CUDA, "prefill setup: %s", cudaGetErrorString(static_cast<cudaError_t>(st)));
-  kernel<<<grid, kThreads, kSmemBytes, stream>>>(args);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaSuccess;
+  if (after_plan)
+    e = launch_after_previous(kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, args);
+  else
+    kernel<<<grid, kThreads, kSmemBytes, stream>>>(args);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
   return PKV_OK;
 }
@@ -841,7 +851,7 @@ int launch_prefill_segments(const SegmentLaunch& L, cudaStream_t s) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t items = static_cast<int64_t>(L.num_entries) * L.num_kv_heads;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, items)));
-  return pf::launch_main<true, true>(args, grid, s);
+  return pf::launch_main<true, true>(args, grid, s, false);
 }
 
 }  // namespace pkv
@@ -949,5 +959,5 @@ extern "C" int pkv_paged_attention_prefill(void* out, int out_dtype, const void*
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t items = static_cast<int64_t>(pf::max_entries(num_seqs, total_q, group)) * num_kv_heads;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, items)));
-  return p.out_f32 ? pf::launch_main<true, false>(args, grid, s) : pf::launch_main<false, false>(args, grid, s);
+  return p.out_f32 ? pf::launch_main<true, false>(args, grid, s, true) : pf::launch_main<false, false>(args, grid, s, true);
 }

@@ -115,7 +115,9 @@ def source_digest(kind: str) -> str:
 def recorded_traffic(key: str, kind: str, units: int, layout=None):
     """DRAM bytes (read + write) per launch of the profiled kernel from profiles/traffic.json, or
     None unless the entry was captured on the same kernel sources, the same table layout and a
-    batch of the same size (`units`: the algorithmic bytes, or flops, of one launch)."""
+    batch of the same size: `units` (the algorithmic bytes, or flops, of one launch) within 5% of
+    the capture's.  Contexts grow by a token per step, so a run with another step count has a
+    slightly different mean; the recorded bytes are scaled by the ratio of the units."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             entry = json.load(f).get(key)
@@ -123,9 +125,10 @@ def recorded_traffic(key: str, kind: str, units: int, layout=None):
         return None
     if not entry or entry.get("sources") != source_digest(kind) or entry.get("layout") != layout:
         return None
-    if entry.get("algorithmic_per_launch") != int(units):
+    rec = entry.get("algorithmic_per_launch")
+    if not rec or abs(int(units) - rec) > 0.05 * rec:
         return None
-    return int(entry["dram_bytes_per_launch"])
+    return int(round(entry["dram_bytes_per_launch"] * int(units) / rec))
 
 
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e nominal (DGX figure)

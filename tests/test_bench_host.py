@@ -478,7 +478,8 @@ def test_recorded_traffic_only_for_the_captured_batch(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "source_digest", lambda kind: digest)
     assert bench.recorded_traffic("b", "decode_simt", 1000) == 1234
-    assert bench.recorded_traffic("b", "decode_simt", 999) is None          # another batch size
+    assert bench.recorded_traffic("b", "decode_simt", 1040) == round(1234 * 1.04)  # more steps: scaled
+    assert bench.recorded_traffic("b", "decode_simt", 900) is None          # another batch size
     assert bench.recorded_traffic("b", "decode_simt", 1000, "x") is None    # another layout
     assert bench.recorded_traffic("shared", "decode_simt", 10, "x") == 99
     assert bench.recorded_traffic("missing", "decode_simt", 1000) is None

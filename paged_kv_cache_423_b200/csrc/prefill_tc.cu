@@ -132,6 +132,18 @@ struct alignas(64) Args {
   PrefillArgs a;
 };
 
+// a0 += w.lo, a1 += w.hi for the two bf16 values of w, each by fma.rn.f32.bf16 with 1 as the
+// other factor: exact product, one rounding of the sum.
+__device__ __forceinline__ void add_bf16x2(float& a0, float& a1, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi, one;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "mov.b16 one, 0x3F80;\n\t"
+      "fma.rn.f32.bf16 %0, lo, one, %0;\n\t"
+      "fma.rn.f32.bf16 %1, hi, one, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(w));
+}
+
 // SEG = false: causal prefill, normalised output rows.  SEG = true: the shared phase of
 // the shared-prefix decode — every query row of an item sees all keys of its part (a run
 // of whole blocks of one table row), and the epilogue writes unnormalised partials.
@@ -571,15 +583,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       lsum *= alpha;
       // ---- P = 2^(s * scale_log2 - m) as bf16 pairs, stored over S (columns 0-63 of
       //      the tile's block: keys 2i, 2i+1 in column i).  Pairs of scores go through packed
-      //      fp32x2 arithmetic: one fma.rn.f32x2 for scale and maximum, and the row sum adds
-      //      the rounded bf16 pairs with add.rn.f32x2.  A row with no visible key yet holds
-      //      -inf as its maximum: neg_m is then 0 and every score of the stage is -inf, so its
-      //      weights are 0 without a select.
+      //      fp32x2 arithmetic: one fma.rn.f32x2 for scale and maximum.  The row sum adds the
+      //      rounded bf16 values into eight fp32 accumulators with the mixed-precision FMA
+      //      (x·1 + acc: one rounding, the same sum as an fp32 add of the widened value,
+      //      without widening it first).  A row with no visible key yet holds -inf as its
+      //      maximum: neg_m is then 0 and every score of the stage is -inf, so its weights
+      //      are 0 without a select.
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(neg_m, neg_m);
-      uint64_t ls2[4];
+      float ls[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ls2[i] = f2pack(0.f, 0.f);
+      for (int i = 0; i < 8; ++i) ls[i] = 0.f;
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         uint32_t w[16];
@@ -591,13 +605,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           const float p0 = poly ? tc::poly_exp2(e.x) : fast_exp2(e.x);
           const float p1 = poly ? tc::poly_exp2(e.y) : fast_exp2(e.y);
           w[i] = pack_bf16x2(p0, p1);
-          ls2[i & 3] = fadd2(ls2[i & 3], bf16x2_to_f2(w[i]));
+          add_bf16x2(ls[2 * (i & 3)], ls[2 * (i & 3) + 1], w[i]);
         }
         tc::tmem_store16(tmem + lane_base + col_s + h * 16, w);
       }
       {
-        const float2 l0 = f2unpack(fadd2(ls2[0], ls2[1])), l1 = f2unpack(fadd2(ls2[2], ls2[3]));
-        lsum += (l0.x + l0.y) + (l1.x + l1.y);
+        const float l0x = ls[0] + ls[2], l0y = ls[1] + ls[3], l1x = ls[4] + ls[6], l1y = ls[5] + ls[7];
+        lsum += (l0x + l0y) + (l1x + l1y);
       }
       tc::tmem_wait_st();
       tc::tc_fence_before();     // P and the rescaled O, before the MMA reads them

@@ -112,8 +112,12 @@ def test_fp8_oracle_timer_counts_one_byte_per_value():
     w = types.SimpleNamespace(Hkv=b.num_kv_heads, D=b.head_dim, scale=b.scale)
     items = [(q[s:s + 1], kc, vc, ks, vs, b.block_tables[s:s + 1], b.context_lens[s:s + 1]) for s in range(b.num_seqs)]
     done, dt, n = bench.time_oracle_fp8(w, items, 60.0)
-    assert n == b.num_seqs and dt > 0
+    assert n == b.num_seqs and dt > 0                      # one pass (the reference arm's timing)
     assert done == int(b.context_lens.sum()) * b.num_kv_heads * b.head_dim * 2
+    done, dt, n = bench.time_oracle_fp8(w, items, 0.3, repeat=True)
+    assert n > b.num_seqs and dt >= 0.3                    # passes until the budget (the CPU-baseline leg)
+    per = [int(l) * b.num_kv_heads * b.head_dim * 2 for l in b.context_lens]
+    assert done == sum(per[i % b.num_seqs] for i in range(n))
 
 
 def _distinct_slots(tables, lens, bs):

@@ -693,12 +693,15 @@ def run_ours(args, rank, world, local_rank):
 def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None):
     """End to end through the public API with host buffers, pipelined as a server
     would run it: per step the C++ allocator produces slots and tables on the host;
-    q, new K, new V (one pinned buffer per step) and the allocator output (a small
-    pinned buffer, double-buffered) go host->device on a copy stream while the
-    previous step's kernels run; the step's output comes back to pinned memory on a
-    stream of its own (beside the next step's kernels) and is read on the host one
-    step later.  With the shared-prefix decode (`sws` its workspace) the host also plans
-    each step from the allocator's tables, and the plan travels with them."""
+    q, new K, new V (one pinned buffer per step) go host->device on a copy stream as soon
+    as the step before has been launched (beside its kernels), and the allocator output
+    (a small pinned buffer, double-buffered) once the allocator has run; the step's
+    output comes back to pinned memory on a stream of its own (beside the next step's
+    kernels) and is read on the host two steps later (outputs triple-buffered), so the
+    host never waits for the step that runs while it prepares the next.  Every timed
+    step's copies are issued inside the timed region.  With the shared-prefix decode (`sws` its workspace)
+    the host also plans each step from the allocator's tables, and the plan travels with
+    them."""
     import torch
     ke = max(1, min(args.steps, args.e2e_steps))
     n = args.warmup + ke
@@ -732,17 +735,41 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
     host_meta = [torch.empty(meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     dev_qkv = [torch.empty(nq + 2 * nk, dtype=torch.int16, device=device) for _ in range(2)]
     dev_meta = [torch.empty(meta_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
-    out_host = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    outs = [out, torch.empty_like(out)]
+    out_host = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    outs = [out, torch.empty_like(out), torch.empty_like(out)]
     h2d_done = [torch.cuda.Event() for _ in range(n)]
+    qkv_done = [torch.cuda.Event() for _ in range(n)]
     comp_done = [torch.cuda.Event() for _ in range(n)]
     d2h_done = [torch.cuda.Event() for _ in range(n)]
-    stats = {"h2d": 0, "d2h": 0, "kv": 0, "checksum": 0.0}
+    stats = {"h2d": 0, "d2h": 0, "kv": 0, "checksum": 0.0, "host_s": 0.0}
+    # the step's device views, made once per buffer (the host loop is part of what is timed)
+    views = []
+    for b in range(2):
+        dm = dev_meta[b]
+        views.append({"q": dev_qkv[b][:nq].view(torch.bfloat16).view(w.B, w.Hq, w.D),
+                      "k": dev_qkv[b][nq:nq + nk].view(torch.bfloat16).view(w.B, w.Hkv, w.D),
+                      "v": dev_qkv[b][nq + nk:].view(torch.bfloat16).view(w.B, w.Hkv, w.D),
+                      "slots": dm[o_slots:o_slots + 8 * w.B].view(torch.int64),
+                      "tables": dm[o_tab:o_tab + 4 * w.B * w.max_blocks].view(torch.int32).view(w.B, w.max_blocks),
+                      "lens": dm[o_lens:o_lens + 4 * w.B].view(torch.int32),
+                      "plan": dm[o_plan:o_plan + plan_cap]})
 
-    def step(i):
+    def upload_qkv(i):
+        """Step i's q, new K and new V to the device, once step i-2 is done with the buffer."""
+        with torch.cuda.stream(copy):
+            if i >= 2:
+                copy.wait_event(comp_done[i - 2])
+            dev_qkv[i % 2].copy_(host_qkv[i], non_blocking=True)
+            qkv_done[i].record(copy)
+
+    def step(i, prefetch_next):
         b = i % 2
+        t_in = time.perf_counter()
+        wait_s = 0.0
         if i >= 2:
+            tw = time.perf_counter()
             h2d_done[i - 2].synchronize()          # host_meta[b] is free again
+            wait_s += time.perf_counter() - tw
         slots, pairs = bm.append_slots(seq_ids)
         tables, lens = bm.export_tables(seq_ids, w.max_blocks)
         hm = host_meta[b].numpy()
@@ -758,49 +785,53 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
         with torch.cuda.stream(copy):
             if i >= 2:
                 copy.wait_event(comp_done[i - 2])  # device buffers b are free again
-            dev_qkv[b].copy_(host_qkv[i], non_blocking=True)
             dev_meta[b].copy_(host_meta[b], non_blocking=True)
             h2d_done[i].record(copy)
+        compute.wait_event(qkv_done[i])
         compute.wait_event(h2d_done[i])
-        dq = dev_qkv[b][:nq].view(torch.bfloat16).view(w.B, w.Hq, w.D)
-        dk = dev_qkv[b][nq:nq + nk].view(torch.bfloat16).view(w.B, w.Hkv, w.D)
-        dv = dev_qkv[b][nq + nk:].view(torch.bfloat16).view(w.B, w.Hkv, w.D)
-        dm = dev_meta[b]
-        d_slots = dm[o_slots:o_slots + 8 * w.B].view(torch.int64)
-        d_tables = dm[o_tab:o_tab + 4 * w.B * w.max_blocks].view(torch.int32).view(w.B, w.max_blocks)
-        d_lens = dm[o_lens:o_lens + 4 * w.B].view(torch.int32)
+        vw = views[b]
         if len(pairs):
-            d_pairs = dm[o_pairs:o_pairs + pairs.nbytes].view(torch.int64).view(-1, 2)
+            d_pairs = dev_meta[b][o_pairs:o_pairs + pairs.nbytes].view(torch.int64).view(-1, 2)
             w.copy(d_pairs, status)
-        w.write(dk, dv, d_slots, status)
-        if i >= 2:
-            compute.wait_event(d2h_done[i - 2])    # outs[b] has been copied out
-        shared = (dm[o_plan:o_plan + plan_cap], info, sws) if sws is not None else None
-        w.decode(outs[b], dq, d_tables, d_lens, max_len_bound, ws, path, status, shared=shared)
+        w.write(vw["k"], vw["v"], vw["slots"], status)
+        r = i % 3                                  # output buffers
+        if i >= 3:
+            compute.wait_event(d2h_done[i - 3])    # outs[r] has been copied out
+        shared = (vw["plan"], info, sws) if sws is not None else None
+        w.decode(outs[r], vw["q"], vw["tables"], vw["lens"], max_len_bound, ws, path, status, shared=shared)
         comp_done[i].record(compute)
         with torch.cuda.stream(d2h):
             d2h.wait_event(comp_done[i])
-            out_host[b].copy_(outs[b], non_blocking=True)
+            out_host[r].copy_(outs[r], non_blocking=True)
             d2h_done[i].record(d2h)
-        if i >= 1:                                 # read the previous step's result on the host
-            d2h_done[i - 1].synchronize()
-            stats["checksum"] += float(out_host[(i - 1) % 2][0, 0, 0])
+        if prefetch_next:                          # the next step's inputs go up beside this step's kernels
+            upload_qkv(i + 1)
+        if i >= 2:                                 # read the result of two steps back on the host
+            tw = time.perf_counter()
+            d2h_done[i - 2].synchronize()
+            wait_s += time.perf_counter() - tw
+            stats["checksum"] += float(out_host[(i - 2) % 3][0, 0, 0])
         if i >= args.warmup:
+            stats["host_s"] += time.perf_counter() - t_in - wait_s
             stats["h2d"] += (host_qkv[i].numel() * 2 + slots.nbytes + pairs.nbytes + tables.nbytes + lens.nbytes
                              + plan_bytes)
-            stats["d2h"] += out_host[b].numel() * 2
+            stats["d2h"] += out_host[r].numel() * 2
             stats["kv"] += int(np.asarray(lens, np.int64).sum()) * w.Hkv * w.D * 2 * (1 if w.kv8 else 2)
 
+    if args.warmup > 0:
+        upload_qkv(0)
     for i in range(args.warmup):
-        step(i)
+        step(i, prefetch_next=i + 1 < args.warmup)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(copy)
     compute.wait_event(t0)
+    upload_qkv(args.warmup)                        # the first timed step's inputs, inside the timed region
     for i in range(args.warmup, n):
-        step(i)
-    d2h_done[n - 1].synchronize()                  # the last step's result
-    stats["checksum"] += float(out_host[(n - 1) % 2][0, 0, 0])
+        step(i, prefetch_next=i + 1 < n)
+    for j in range(max(0, n - 2), n):              # the last two steps' results
+        d2h_done[j].synchronize()
+        stats["checksum"] += float(out_host[j % 3][0, 0, 0])
     t1.record(compute)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
@@ -809,8 +840,10 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
             "h2d_bytes_per_step": stats["h2d"] // ke, "d2h_bytes_per_step": stats["d2h"] // ke,
             "ms_per_step": round(ms / ke, 4), "steps": ke,
             "seq_steps_per_s": round(w.B * ke / (ms * 1e-3), 1),
+            # host time per step outside its waits (allocator, planning, staging, launches)
+            "host_busy_ms_per_step": round(1e3 * stats["host_s"] / ke, 4),
             "pipelining": "H2D of step i+1 on a copy stream and D2H of step i-1 on a result stream overlap the"
-                          " kernels of step i; results read one step later"}
+                          " kernels of step i; results read on the host two steps later"}
 
 
 # ---------------------------------------------------------------------------

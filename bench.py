@@ -98,6 +98,8 @@ KERNEL_SOURCES = {
     "prefill": ["prefill_tc.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
     "shared": ["shared_decode.cu", "shared_plan.cpp", "prefill_tc.cu", "decode_gqa_tc.cu", "decode.cu",
                "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
+    "shared_fp8": ["shared_decode.cu", "shared_plan.cpp", "prefill_tc.cu", "decode_gqa_tc_fp8.cu", "decode_gqa_tc.cu",
+                   "decode.cu", "decode_common.cuh", "device_common.cuh", "tcgen05_common.cuh"],
 }
 
 
@@ -412,7 +414,12 @@ class Workload:
 
     def decode(self, out, q, tables, lens, max_len, ws, path, status, shared=None):
         """shared = (device plan, its info, the shared-prefix workspace) for the shared-prefix decode."""
-        if shared is not None:
+        if shared is not None and self.kv8:
+            plan, info, sws = shared
+            self.pkv.paged_attention_decode_shared_fp8(out, q, self.key_cache, self.value_cache, self.k_scale,
+                                                       self.v_scale, tables, lens, self.scale, plan, info, sws,
+                                                       status=status)
+        elif shared is not None:
             plan, info, sws = shared
             self.pkv.paged_attention_decode_shared(out, q, self.key_cache, self.value_cache, tables, lens, self.scale,
                                                    plan, info, sws, status=status)
@@ -436,12 +443,12 @@ class Workload:
 
 def shared_decode_applies(args, w) -> bool:
     """The shared-prefix decode: on request, or by default for the shared-prompt workload;
-    it needs a bf16 pool and the tensor-core decode's head shapes."""
+    it needs the tensor-core decode's head shapes (bf16 or 8-bit pool)."""
     g = w.Hq // w.Hkv
-    ok = not w.kv8 and w.D == 128 and 2 <= g <= 16 and args.path != "simt"
+    ok = w.D == 128 and 2 <= g <= 16 and args.path != "simt"
     choice = getattr(args, "shared", "auto")
     if choice == "on" and not ok:
-        raise SystemExit("--shared on needs a bf16 pool, head_dim 128 and 2 <= num_heads / num_kv_heads <= 16")
+        raise SystemExit("--shared on needs head_dim 128 and 2 <= num_heads / num_kv_heads <= 16")
     return ok and (choice == "on" or (choice == "auto" and w.shared_blocks > 0))
 
 
@@ -560,8 +567,10 @@ def run_ours(args, rank, world, local_rank):
     path = {"auto": 0, "simt": 1, "tensor": 2}[args.path]
     sws = None
     if use_shared:
-        sws = torch.empty(max(pkv.paged_attention_decode_shared_workspace_size(st["plan"][1], w.Hq, w.Hkv, w.D)
-                              for st in states), dtype=torch.uint8, device=device)
+        size_fn = (pkv.paged_attention_decode_shared_fp8_workspace_size if kv8
+                   else pkv.paged_attention_decode_shared_workspace_size)
+        sws = torch.empty(max(size_fn(st["plan"][1], w.Hq, w.Hkv, w.D) for st in states), dtype=torch.uint8,
+                          device=device)
 
     def step(i, ev=None):
         st = states[i % n_states]
@@ -590,8 +599,10 @@ def run_ours(args, rank, world, local_rank):
         bytes_total += alg
         unique_total += alg - kv + st["unique_kv"]
         unique_kv_total += st["unique_kv"]
-        if use_shared:  # write, setup, shared phase (when there are segments), plan, decode, merge
-            launches += 5 + (1 if st["plan"][1].num_entries else 0) + (1 if st["n_pairs"] else 0)
+        if use_shared:  # write, setup, [widening and] shared phase (when there are segments), plan,
+            # [query split,] decode, merge
+            launches += (5 + (1 if st["plan"][1].num_entries else 0) * (2 if kv8 else 1) + (1 if kv8 else 0)
+                         + (1 if st["n_pairs"] else 0))
         else:
             launches += 3 + (1 if st["n_pairs"] else 0) + merge
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -655,12 +666,16 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4),
                      "traffic": recorded_traffic(w.label + ("+shared" if use_shared else ""),
-                                                 "shared" if use_shared else
+                                                 ("shared_fp8" if kv8 else "shared") if use_shared else
                                                  ("decode_gqa_tc_fp8" if kv8 else "decode_gqa_tc") if uses_tensor
                                                  else "decode_simt", unique_total // args.steps, w.layout),
                      "algorithmic_bytes_per_launch": unique_total // args.steps,
                      "logical_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
-                     "kernel": ("paged_attention_decode_shared: setup + shared phase (tcgen05 prefill kernel, every"
+                     "kernel": ("paged_attention_decode_shared_fp8: setup + shared phase (the shared blocks widened"
+                                " to bf16, tcgen05 prefill kernel, every key visible, partials) + plan + query split +"
+                                " tcgen05 kind::f8f6f4 decode of the private remainders + merge; traffic = the DRAM"
+                                " bytes of all of them" if use_shared and kv8
+                                else "paged_attention_decode_shared: setup + shared phase (tcgen05 prefill kernel, every"
                                 " key visible, partials) + plan + tcgen05 decode of the private remainders + merge;"
                                 " traffic = the DRAM bytes of all of them" if use_shared
                                 else "paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"

@@ -353,7 +353,8 @@ typedef struct pkv_shared_plan_info {
   int64_t shared_tokens;     /* sum over segments of their tokens (each read once per kv head) */
   uint64_t off_entries;      /* int4[num_entries]: first row, 0, rows of tile A | rows of tile B << 8, part */
   uint64_t off_parts;        /* int4[2 * num_parts]: (table row, first block, keys, first row),
-                                (rows, first partial, 0, 0) */
+                                (rows, first partial, first scratch block, 0); parts' scratch blocks
+                                follow each other in plan order, shared_tokens / block_size in all */
   uint64_t off_suffix_lens;  /* int32[num_seqs]: tokens of each row's private remainder */
   uint64_t off_block_offset; /* int32[num_seqs]: table index where the remainder starts */
   uint64_t off_row_start;    /* int32[num_seqs + 1]: CSR of each row's shared partials */
@@ -370,7 +371,7 @@ PKV_API int pkv_shared_plan(const int32_t* block_tables, int max_blocks_per_seq,
  *   plan        device copy of the plan made for these tables and lengths (16-byte aligned)
  *   info        host, the plan's info
  *   workspace   device, pkv_paged_attention_decode_shared_workspace_size() bytes, 256-byte aligned
- * bf16 pools only; head_dim 128; 2 <= num_heads / num_kv_heads <= 16 (the tensor-core
+ * bf16 pools (the 8-bit form follows); head_dim 128; 2 <= num_heads / num_kv_heads <= 16 (the tensor-core
  * decode) — else PKV_ERR_UNSUPPORTED; scale finite and positive, else PKV_ERR_INVALID.  block_tables and context_lens must be those the
  * plan was made from: the call checks on the device that every row's shared tokens plus its
  * remainder equal its context length (and the plan's ranges); a plan that does not fit sets
@@ -389,6 +390,33 @@ PKV_API int pkv_paged_attention_decode_shared(void* out, int out_dtype, const vo
                                               int block_size, int num_blocks, float scale, const void* plan,
                                               const pkv_shared_plan_info* info, void* workspace,
                                               size_t workspace_bytes, int32_t* status, pkv_stream_t stream);
+
+/*
+ * The same over an 8-bit (e4m3) pool: key_cache / value_cache are [num_blocks, num_kv_heads,
+ * block_size, 128] uint8 codes with one float32 scale per kv head in k_scale / v_scale
+ * (device), as for pkv_paged_attention_decode_fp8, whose result this is (intelliparadigm
+ * article §4.2 and §5: fp8 KV loading; Outcome School explainer, "内存共享": shared blocks).
+ * The shared phase first widens the codes of the plan's shared blocks into two bf16 scratch
+ * pools inside the workspace (exact: every e4m3 value is a bf16 value), then runs with each
+ * kv head's key scale folded into its scores and its value scale into its partial outputs;
+ * the private phase is the 8-bit tensor-core decode.  Workspace:
+ * pkv_paged_attention_decode_shared_fp8_workspace_size() bytes, the bf16 call's plus the split
+ * queries, two scratch pools of info->shared_tokens * num_kv_heads * 128 * 2 bytes and a table
+ * of num_seqs * max_blocks_per_seq int32.  A table entry of a shared block outside the pool
+ * sets PKV_DEV_BAD_BLOCK and its keys are left out, as in every decode.  Errors as for the
+ * bf16 call; null scales are PKV_ERR_INVALID.
+ */
+PKV_API size_t pkv_paged_attention_decode_shared_fp8_workspace_size(const pkv_shared_plan_info* info,
+                                                                    int num_heads, int num_kv_heads, int head_dim);
+PKV_API int pkv_paged_attention_decode_shared_fp8(void* out, int out_dtype, const void* query,
+                                                  const void* key_cache, const void* value_cache,
+                                                  const float* k_scale, const float* v_scale,
+                                                  const int32_t* block_tables, int max_blocks_per_seq,
+                                                  const int32_t* context_lens, int num_seqs, int num_heads,
+                                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                                  float scale, const void* plan, const pkv_shared_plan_info* info,
+                                                  void* workspace, size_t workspace_bytes, int32_t* status,
+                                                  pkv_stream_t stream);
 
 /*
  * Host block manager — free list + reference counts + per-sequence block tables.

@@ -24,6 +24,7 @@ __all__ = [
     "paged_attention_prefill_workspace_size", "paged_attention_prefill", "reshape_and_cache_fp8",
     "paged_attention_decode_fp8", "swap_blocks", "BlockManager", "stream_read",
     "SharedPlanInfo", "shared_plan", "paged_attention_decode_shared_workspace_size", "paged_attention_decode_shared",
+    "paged_attention_decode_shared_fp8_workspace_size", "paged_attention_decode_shared_fp8",
 ]
 
 PKV_OK = 0
@@ -138,6 +139,13 @@ _SIGNATURES["pkv_paged_attention_decode_shared"] = (c_int, [c_void_p, c_int, c_v
                                                             c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                             c_float, c_void_p, ctypes.POINTER(SharedPlanInfo),
                                                             c_void_p, c_size_t, c_void_p, c_void_p])
+_SIGNATURES["pkv_paged_attention_decode_shared_fp8_workspace_size"] = (c_size_t, [ctypes.POINTER(SharedPlanInfo),
+                                                                                  c_int, c_int, c_int])
+_SIGNATURES["pkv_paged_attention_decode_shared_fp8"] = (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                                                c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int,
+                                                                c_int, c_int, c_int, c_int, c_int, c_float, c_void_p,
+                                                                ctypes.POINTER(SharedPlanInfo), c_void_p, c_size_t,
+                                                                c_void_p, c_void_p])
 
 
 def library():
@@ -529,6 +537,41 @@ def paged_attention_decode_shared(out, query, key_cache, value_cache, block_tabl
         _ptr(plan, torch.uint8, "plan"), ctypes.byref(info), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
     _check(rc, "paged_attention_decode_shared")
+
+
+def paged_attention_decode_shared_fp8_workspace_size(info, num_heads, num_kv_heads, head_dim) -> int:
+    return int(library().pkv_paged_attention_decode_shared_fp8_workspace_size(ctypes.byref(info), num_heads,
+                                                                              num_kv_heads, head_dim))
+
+
+def paged_attention_decode_shared_fp8(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, context_lens,
+                                      scale, plan, info, workspace, status=None, stream=None):
+    """Shared-prefix decode over 8-bit pools [NB, Hkv, bs, 128] uint8 with per-kv-head scales:
+    the result of paged_attention_decode_fp8; otherwise as paged_attention_decode_shared (its
+    workspace from paged_attention_decode_shared_fp8_workspace_size)."""
+    torch = _torch()
+    _same_device("paged_attention_decode_shared_fp8", out, query, key_cache, value_cache, k_scale, v_scale,
+                 block_tables, context_lens, plan, workspace, status)
+    B, Hq, D = query.shape
+    NB, Hkv, bs, D2 = key_cache.shape
+    if out.shape != query.shape or D2 != D or value_cache.shape != key_cache.shape:
+        raise ValueError("paged_attention_decode_shared_fp8: shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("paged_attention_decode_shared_fp8: block_tables must be [B, max_blocks], context_lens [B]")
+    out_dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(out.dtype)
+    if out_dtype is None:
+        raise TypeError("paged_attention_decode_shared_fp8: out must be bf16 or f32")
+    if plan.numel() * plan.element_size() < int(info.bytes):
+        raise ValueError("paged_attention_decode_shared_fp8: the device plan is smaller than info.bytes")
+    rc = library().pkv_paged_attention_decode_shared_fp8(
+        _ptr(out, None, "out"), out_dtype, _ptr(query, torch.bfloat16, "query"),
+        _ptr(key_cache, torch.uint8, "key_cache"), _ptr(value_cache, torch.uint8, "value_cache"),
+        _ptr(k_scale, torch.float32, "k_scale"), _ptr(v_scale, torch.float32, "v_scale"),
+        _ptr(block_tables, torch.int32, "block_tables"), int(block_tables.shape[1]),
+        _ptr(context_lens, torch.int32, "context_lens"), B, Hq, Hkv, D, bs, NB, float(scale),
+        _ptr(plan, torch.uint8, "plan"), ctypes.byref(info), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(rc, "paged_attention_decode_shared_fp8")
 
 
 def _np_ptr(a):

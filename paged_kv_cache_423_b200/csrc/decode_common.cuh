@@ -146,6 +146,10 @@ struct SegmentLaunch {
   int num_entries;              // grid sizing (host)
   int max_blocks, num_seqs, num_heads, num_kv_heads, block_size, num_blocks;
   float scale;
+  // pools of widened 8-bit codes: per-kv-head factors of the scores and of the partial
+  // outputs (null for bf16 pools)
+  const float* k_scale = nullptr;
+  const float* v_scale = nullptr;
 };
 int launch_prefill_segments(const SegmentLaunch& launch, cudaStream_t stream);
 

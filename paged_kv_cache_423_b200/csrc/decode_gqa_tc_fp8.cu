@@ -316,7 +316,8 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
       const int tok0 = e.y * a.partition;
       const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - tok0);
       const int nblk = (ntok + a.block_size - 1) / a.block_size;
-      const int32_t* row = a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size;
+      const int32_t* row = a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size +
+                           (a.block_offset ? a.block_offset[e.x] : 0);
       int4 t = make_int4(0, 0, 0, 0);
       if (lane < nblk) t.x = __ldg(row + lane);
       if (lane + 32 < nblk) t.y = __ldg(row + lane + 32);
@@ -614,14 +615,15 @@ __global__ void __launch_bounds__(Cfg<GROUPS>::kThreads, Cfg<GROUPS>::kCtasPerSm
         const int h = head(j);
         if (h >= g) break;  // heads of a group increase with j
         const float l = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
-        if (nparts == 1) {
+        if (nparts == 1 && !a.always_partial) {
           store_out<OUT_F32>(a, (unit0 + h) * kD + d, l > 0.f ? ot[j] / l : 0.f);
         } else {
-          // unnormalised partial (weights times 2^7 in both o and l); the merge
-          // kernel combines the partitions
+          // unnormalised partial; the weights are held times 2^7 in both o and l, so the
+          // partial's maximum is recorded as the held one minus 7 (o and l are then the sums
+          // of 2^(x - m) (v, 1), as every partial a merge combines)
           const int64_t pidx = (unit0 + h) * a.max_parts + part;
           a.part_o[pidx * kD + d] = ot[j];
-          if (d == 0) a.part_ml[pidx] = make_float2(f_m[j], l);
+          if (d == 0) a.part_ml[pidx] = make_float2(f_m[j] - kPShift, l);
         }
       }
     };
@@ -932,7 +934,7 @@ int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cu
   else
     rc = out_f32 ? tc8::launch<true, 16>(args, stream) : tc8::launch<false, 16>(args, stream);
   if (rc != PKV_OK) return rc;
-  return launch_merge_partials(a, out_f32, stream);
+  return a.always_partial ? PKV_OK : launch_merge_partials(a, out_f32, stream);
 }
 
 }  // namespace pkv

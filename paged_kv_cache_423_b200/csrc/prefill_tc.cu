@@ -110,7 +110,7 @@ struct PrefillArgs {
   const int4* entries;        // x = first packed row, y = its position, z = tokens A | tokens B << 8, w = sequence
                               // (segment mode: w = part, y unused)
   const int4* parts;          // segment mode: [2 * part] (table row, first block, keys, first row),
-                              //               [2 * part + 1] (rows, first partial, 0, 0)
+                              //               [2 * part + 1] (rows, first partial, first scratch block, 0)
   float* part_o;              // segment mode: unnormalised partial outputs [partial][head][128]
   float2* part_ml;            // segment mode: (held maximum in base-2 units, weight sum) [partial][head]
   int32_t* status;
@@ -123,6 +123,10 @@ struct PrefillArgs {
   int group_shift;            // log2(group)
   int tile_tokens;            // 128 / group
   float scale_log2;
+  // segment mode over widened 8-bit blocks: per-kv-head factors of the scores and of the
+  // partial outputs (the codes' scales), or null
+  const float* k_scale;
+  const float* v_scale;
 };
 
 struct alignas(64) Args {
@@ -493,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t col_s = t * 128, col_o = kColO + t * 128;
     float m_used = -INFINITY, lsum = 0.f;
+    float sl2 = a.scale_log2;  // score scale (base 2) of the item; segment mode may fold in the key scale
     bool has_pv = false;
     int c = 0;  // stages of this tile processed (phases of s_full / p_full / o_bar)
     for (int n = 0;; ++n) {
@@ -516,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         m_used = -INFINITY;
         lsum = 0.f;
         has_pv = false;
+        if constexpr (SEG) sl2 = a.k_scale ? a.scale_log2 * __ldg(a.k_scale + kvh) : a.scale_log2;
       }
       const int tl = m >> a.group_shift;
       const bool valid_row = tl < ntok;
@@ -558,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       for (int k = 8; k < kKeys; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], s[k]);
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float mxs = mx * a.scale_log2;
+      const float mxs = mx * sl2;
       // A row rescales only when its maximum grew past the threshold; the tensor-memory
       // accesses are warp-collective, so the warp rescales together (alpha = 1 for the
       // rows that keep their maximum).  Every P·V of the tile is complete here.
@@ -590,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       //      maximum: neg_m is then 0 and every score of the stage is -inf, so its weights
       //      are 0 without a select.
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(neg_m, neg_m);
+      const uint64_t sc2 = f2pack(sl2, sl2), nm2 = f2pack(neg_m, neg_m);
       float ls[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) ls[i] = 0.f;
@@ -625,8 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         tc::tc_fence_after();
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         const int64_t orow = (static_cast<int64_t>(row0 + tl) * a.num_heads + kvh * g + (m & (g - 1))) * kD;
+        float vsc = 1.f;  // segment mode over widened 8-bit blocks: the value scale of the kv head
         if constexpr (SEG) {
           if (valid_row) a.part_ml[orow / kD] = make_float2(m_used, lsum);
+          if (a.v_scale) vsc = __ldg(a.v_scale + kvh);
         }
         uint32_t r[32];
 #pragma unroll
@@ -638,8 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
               float4* dst = reinterpret_cast<float4*>(a.part_o + orow + q4 * 32);
 #pragma unroll
               for (int k = 0; k < 8; ++k)
-                dst[k] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
-                                     __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+                dst[k] = make_float4(__uint_as_float(r[4 * k]) * vsc, __uint_as_float(r[4 * k + 1]) * vsc,
+                                     __uint_as_float(r[4 * k + 2]) * vsc, __uint_as_float(r[4 * k + 3]) * vsc);
             } else if constexpr (OUT_F32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow + q4 * 32);
 #pragma unroll
@@ -855,6 +863,8 @@ int launch_prefill_segments(const SegmentLaunch& L, cudaStream_t s) {
   a.group_shift = __builtin_ctz(static_cast<unsigned>(group));
   a.tile_tokens = pf::kRows / group;
   a.scale_log2 = L.scale * 1.4426950408889634f;
+  a.k_scale = L.k_scale;
+  a.v_scale = L.v_scale;
   const uint64_t pool_rows = static_cast<uint64_t>(L.num_blocks) * L.num_kv_heads * L.block_size;
   int rc = pf::encode_kv_map(&args.tm_k, L.key_cache, pool_rows, "key_cache");
   if (rc == PKV_OK) rc = pf::encode_kv_map(&args.tm_v, L.value_cache, pool_rows, "value_cache");
@@ -963,6 +973,8 @@ extern "C" int pkv_paged_attention_prefill(void* out, int out_dtype, const void*
   a.group_shift = __builtin_ctz(static_cast<unsigned>(group));
   a.tile_tokens = pf::kRows / group;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.k_scale = nullptr;
+  a.v_scale = nullptr;
   const uint64_t pool_rows = static_cast<uint64_t>(num_blocks) * num_kv_heads * block_size;
   int rc = pf::encode_kv_map(&args.tm_k, key_cache, pool_rows, "key_cache");
   if (rc == PKV_OK) rc = pf::encode_kv_map(&args.tm_v, value_cache, pool_rows, "value_cache");

@@ -22,9 +22,15 @@
 //                         the SMs the other leaves)
 //   shared_merge_kernel   after both (the side stream joins back): out = sum 2^(m_i - M) o_i /
 //                         sum 2^(m_i - M) l_i per (row, head)
+// Over an 8-bit (e4m3) pool the shared phase first widens the codes of every part's blocks
+// into bf16 scratch pools (scratch_fill_kernel, on the side stream: exact, every e4m3 value
+// is a bf16 value) and runs on them with the kv head's key scale folded into its score scale
+// and its value scale into its partial outputs; the private phase is the 8-bit tensor-core
+// decode.
 // The side stream and its two events are created on the first call on each device and kept
 // until the process exits; the enqueue of a call is serialised per device, so calls from
 // several host threads stay correct.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -44,13 +50,17 @@ constexpr int kMergeWarps = 4;
 
 struct Layout {
   size_t off_count = 0, off_lens = 0, off_offset = 0, off_seg_o = 0, off_seg_ml = 0, off_decode = 0, total = 0;
+  size_t off_scr_k = 0, off_scr_v = 0, off_scr_tab = 0;  // 8-bit pools only
+  int64_t scratch_blocks = 0;
   WorkspaceLayout dec;
   int partition = 0;
 };
 
 // Workspace: [plan count, work counter, bad flag] | checked remainders | checked block offsets |
-// shared partials (o, then (m, l)) | the private phase's decode workspace (partials forced).
-static Layout layout(const pkv_shared_plan_info& in, int num_heads, int num_kv_heads) {
+// shared partials (o, then (m, l)) | the private phase's decode workspace (partials forced) |
+// 8-bit pools: the widened K and V scratch pools [scratch block][kv head][block_size][128] bf16
+// and their table [num_seqs][max_blocks] (written where a part's blocks sit in the call's table).
+static Layout layout(const pkv_shared_plan_info& in, int num_heads, int num_kv_heads, bool kv8) {
   Layout L;
   const int B = in.num_seqs;
   L.partition = auto_partition_tokens_tensor(B, num_kv_heads, in.block_size, in.max_suffix_len);
@@ -66,8 +76,19 @@ static Layout layout(const pkv_shared_plan_info& in, int num_heads, int num_kv_h
   L.off_seg_ml = off;
   off = align256(off + static_cast<size_t>(in.num_partials) * num_heads * sizeof(float2));
   L.off_decode = off;
-  L.dec = workspace_layout(B, num_heads, kD, in.max_suffix_len, L.partition, true);
-  L.total = off + L.dec.total;
+  L.dec = workspace_layout(B, num_heads, kD, in.max_suffix_len, L.partition, true, kv8 ? num_kv_heads : 0);
+  off = align256(off + L.dec.total);
+  if (kv8) {
+    L.scratch_blocks = in.block_size > 0 ? in.shared_tokens / in.block_size : 0;
+    const size_t pool = static_cast<size_t>(L.scratch_blocks) * num_kv_heads * in.block_size * kD * 2;
+    L.off_scr_k = off;
+    off = align256(off + pool);
+    L.off_scr_v = off;
+    off = align256(off + pool);
+    L.off_scr_tab = off;
+    off = align256(off + static_cast<size_t>(B) * in.max_blocks_per_seq * sizeof(int32_t));
+  }
+  L.total = off;
   return L;
 }
 
@@ -132,6 +153,76 @@ __global__ void __launch_bounds__(kSetupThreads) shared_setup_kernel(const Setup
     p.count[1] = 0;
     p.count[2] = bad;
     if (bad) set_status(p.status, PKV_DEV_BAD_CONTEXT);
+  }
+}
+
+// ---- 8-bit pools: the shared phase's blocks widened into bf16 scratch pools
+struct ScratchArgs {
+  const int4* parts;
+  const int32_t* block_tables;
+  const uint8_t* key8;
+  const uint8_t* value8;
+  __nv_bfloat16* key_s;
+  __nv_bfloat16* value_s;
+  int32_t* table_s;
+  const int32_t* bad;   // the set-up's verdict on the plan
+  int32_t* status;
+  int num_parts, num_seqs, max_blocks, block_size, num_blocks, num_kv_heads;
+  int64_t scratch_blocks;
+};
+
+constexpr int kScratchThreads = 256;
+constexpr int kScratchSplit = 4;  // CTAs sharing one (part, kv head)
+
+// Four e4m3 codes (low byte first) as four bf16 values, exactly (through f16, which holds
+// every e4m3 value; so does bf16).
+__device__ __forceinline__ uint2 e4m3x4_to_bf16x4(uint32_t w) {
+  uint32_t h01, h23;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(h01), "=r"(h23)
+      : "r"(w));
+  const __half2 a = *reinterpret_cast<const __half2*>(&h01), b = *reinterpret_cast<const __half2*>(&h23);
+  return make_uint2(pack_bf16x2(__low2float(a), __high2float(a)), pack_bf16x2(__low2float(b), __high2float(b)));
+}
+
+// CTA (part, kv head, z) widens blocks z, z + kScratchSplit, .. of the part for one kv head
+// into scratch blocks base + j, and (kv head 0) points the scratch table's entry of the block
+// at it, or at -1 for a table entry outside the pool (the shared phase then flags
+// PKV_DEV_BAD_BLOCK and masks its keys, as over a bf16 pool).
+__global__ void __launch_bounds__(kScratchThreads) scratch_fill_kernel(const ScratchArgs p) {
+  if (*p.bad) return;
+  const int part = blockIdx.x, kvh = blockIdx.y;
+  const int4 d0 = p.parts[2 * part], d1 = p.parts[2 * part + 1];
+  const int row = d0.x, pos0 = d0.y, nblk = d0.z / p.block_size, base = d1.z;
+  if (row < 0 || row >= p.num_seqs || pos0 < 0 || nblk < 0 || pos0 + nblk > p.max_blocks || base < 0 ||
+      base + static_cast<int64_t>(nblk) > p.scratch_blocks) {
+    if (threadIdx.x == 0 && kvh == 0 && blockIdx.z == 0) set_status(p.status, PKV_DEV_BAD_CONTEXT);
+    return;
+  }
+  const int codes = p.block_size * kD;  // one (block, kv head) tile
+  for (int j = blockIdx.z; j < nblk; j += gridDim.z) {
+    const int64_t tpos = static_cast<int64_t>(row) * p.max_blocks + pos0 + j;
+    const int phys = p.block_tables[tpos];
+    const bool ok = phys >= 0 && phys < p.num_blocks;
+    if (kvh == 0 && threadIdx.x == 0) p.table_s[tpos] = ok ? base + j : -1;
+    if (!ok) continue;
+    const int64_t src = (static_cast<int64_t>(phys) * p.num_kv_heads + kvh) * codes;
+    const int64_t dst = (static_cast<int64_t>(base + j) * p.num_kv_heads + kvh) * codes;
+    const uint4* ks = reinterpret_cast<const uint4*>(p.key8 + src);
+    const uint4* vs = reinterpret_cast<const uint4*>(p.value8 + src);
+    uint4* kd = reinterpret_cast<uint4*>(p.key_s + dst);
+    uint4* vd = reinterpret_cast<uint4*>(p.value_s + dst);
+    for (int i = threadIdx.x; i < codes / 16; i += blockDim.x) {  // 16 codes -> 32 bytes
+      const uint4 kw = __ldg(ks + i), vw = __ldg(vs + i);
+      uint2 a = e4m3x4_to_bf16x4(kw.x), b = e4m3x4_to_bf16x4(kw.y), c = e4m3x4_to_bf16x4(kw.z),
+            d = e4m3x4_to_bf16x4(kw.w);
+      kd[2 * i] = make_uint4(a.x, a.y, b.x, b.y);
+      kd[2 * i + 1] = make_uint4(c.x, c.y, d.x, d.y);
+      a = e4m3x4_to_bf16x4(vw.x), b = e4m3x4_to_bf16x4(vw.y), c = e4m3x4_to_bf16x4(vw.z), d = e4m3x4_to_bf16x4(vw.w);
+      vd[2 * i] = make_uint4(a.x, a.y, b.x, b.y);
+      vd[2 * i + 1] = make_uint4(c.x, c.y, d.x, d.y);
+    }
   }
 }
 
@@ -218,22 +309,33 @@ __global__ void __launch_bounds__(kMergeWarps * 32) shared_merge_kernel(const Me
 
 using namespace pkv;
 
-extern "C" size_t pkv_paged_attention_decode_shared_workspace_size(const pkv_shared_plan_info* info, int num_heads,
-                                                                   int num_kv_heads, int head_dim) {
+static size_t shared_workspace_size(const pkv_shared_plan_info* info, int num_heads, int num_kv_heads, int head_dim,
+                                    bool kv8) {
   if (!info || info->num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim != sp::kD ||
-      info->num_partials < 0 || info->max_suffix_len < 0 || (info->block_size != 16 && info->block_size != 32))
+      info->num_partials < 0 || info->max_suffix_len < 0 || (info->block_size != 16 && info->block_size != 32) ||
+      info->shared_tokens < 0 || info->max_blocks_per_seq <= 0)
     return 0;
-  return sp::layout(*info, num_heads, num_kv_heads).total;
+  return sp::layout(*info, num_heads, num_kv_heads, kv8).total;
 }
 
-extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const void* query, const void* key_cache,
-                                                 const void* value_cache, const int32_t* block_tables,
-                                                 int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
-                                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
-                                                 int num_blocks, float scale, const void* plan,
-                                                 const pkv_shared_plan_info* info, void* workspace,
-                                                 size_t workspace_bytes, int32_t* status, pkv_stream_t stream) {
-  clear_error();
+extern "C" size_t pkv_paged_attention_decode_shared_workspace_size(const pkv_shared_plan_info* info, int num_heads,
+                                                                   int num_kv_heads, int head_dim) {
+  return shared_workspace_size(info, num_heads, num_kv_heads, head_dim, false);
+}
+
+extern "C" size_t pkv_paged_attention_decode_shared_fp8_workspace_size(const pkv_shared_plan_info* info,
+                                                                       int num_heads, int num_kv_heads,
+                                                                       int head_dim) {
+  return shared_workspace_size(info, num_heads, num_kv_heads, head_dim, true);
+}
+
+// kv8: the pools hold e4m3 codes with per-kv-head scales k_scale / v_scale.
+static int shared_impl(bool kv8, void* out, int out_dtype, const void* query, const void* key_cache,
+                       const void* value_cache, const float* k_scale, const float* v_scale,
+                       const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                       int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                       const void* plan, const pkv_shared_plan_info* info, void* workspace, size_t workspace_bytes,
+                       int32_t* status, pkv_stream_t stream) {
   if (!info) return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: null info");
   const pkv_shared_plan_info& in = *info;
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
@@ -259,7 +361,8 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
   if (static_cast<int64_t>(in.num_entries) * num_kv_heads > (int64_t{1} << 30))
     return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: too many shared-phase entries");
   if (num_seqs == 0) return PKV_OK;
-  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !plan || !workspace)
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !plan || !workspace ||
+      (kv8 && (!k_scale || !v_scale)))
     return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: null pointer");
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(plan))
     return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: tensors and the plan must be 16-byte aligned");
@@ -276,7 +379,10 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
       in.off_row_start + static_cast<uint64_t>(num_seqs + 1) * 4 > in.bytes ||
       in.off_row_ids + static_cast<uint64_t>(in.num_partials) * 4 > in.bytes)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: plan sections exceed its size");
-  const sp::Layout L = sp::layout(in, num_heads, num_kv_heads);
+  if (in.shared_tokens < 0 || in.shared_tokens % block_size != 0 ||
+      (kv8 && in.shared_tokens / block_size * num_kv_heads * block_size > (int64_t{1} << 31)))
+    return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: bad shared token count in the plan info");
+  const sp::Layout L = sp::layout(in, num_heads, num_kv_heads, kv8);
   if (workspace_bytes < L.total)
     return set_error(PKV_ERR_INVALID, "paged_attention_decode_shared: workspace of %zu bytes, %zu needed",
                      workspace_bytes, L.total);
@@ -342,6 +448,43 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
     sl.key_cache = key_cache;
     sl.value_cache = value_cache;
     sl.block_tables = block_tables;
+    int seg_blocks = num_blocks;
+    if (kv8) {
+      // the parts' blocks widened into the scratch pools, on the side stream before the shared phase
+      sp::ScratchArgs sc{};
+      sc.parts = parts;
+      sc.block_tables = block_tables;
+      sc.key8 = static_cast<const uint8_t*>(key_cache);
+      sc.value8 = static_cast<const uint8_t*>(value_cache);
+      sc.key_s = reinterpret_cast<__nv_bfloat16*>(ws + L.off_scr_k);
+      sc.value_s = reinterpret_cast<__nv_bfloat16*>(ws + L.off_scr_v);
+      sc.table_s = reinterpret_cast<int32_t*>(ws + L.off_scr_tab);
+      sc.bad = count + 2;
+      sc.status = status;
+      sc.num_parts = in.num_parts;
+      sc.num_seqs = num_seqs;
+      sc.max_blocks = max_blocks_per_seq;
+      sc.block_size = block_size;
+      sc.num_blocks = num_blocks;
+      sc.num_kv_heads = num_kv_heads;
+      sc.scratch_blocks = L.scratch_blocks;
+      if (in.num_parts > 0) {
+        sp::scratch_fill_kernel<<<dim3(in.num_parts, num_kv_heads, sp::kScratchSplit), sp::kScratchThreads, 0,
+                                  side.stream>>>(sc);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) {
+          cudaEventRecord(side.join, side.stream);
+          cudaStreamWaitEvent(s, side.join, 0);  // leave the caller's stream joined
+          return set_error(PKV_ERR_CUDA, "shared decode: scratch launch: %s", cudaGetErrorString(e));
+        }
+      }
+      sl.key_cache = sc.key_s;
+      sl.value_cache = sc.value_s;
+      sl.block_tables = sc.table_s;
+      sl.k_scale = k_scale;
+      sl.v_scale = v_scale;
+      seg_blocks = static_cast<int>(L.scratch_blocks);
+    }
     sl.plan_count = count;
     sl.entries = entries;
     sl.parts = parts;
@@ -354,7 +497,7 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
     sl.num_heads = num_heads;
     sl.num_kv_heads = num_kv_heads;
     sl.block_size = block_size;
-    sl.num_blocks = num_blocks;
+    sl.num_blocks = seg_blocks;
     sl.scale = scale;
     int rc = launch_prefill_segments(sl, side.stream);
     e = cudaEventRecord(side.join, side.stream);
@@ -369,8 +512,17 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
   DecodeArgs a{};
   a.out = out;
   a.query = static_cast<const __nv_bfloat16*>(query);
-  a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
-  a.value_cache = static_cast<const __nv_bfloat16*>(value_cache);
+  if (kv8) {
+    a.key_cache8 = static_cast<const uint8_t*>(key_cache);
+    a.value_cache8 = static_cast<const uint8_t*>(value_cache);
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.q_split = dws + L.dec.off_qsplit;
+    a.q_inv = reinterpret_cast<float*>(dws + L.dec.off_qinv);
+  } else {
+    a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
+    a.value_cache = static_cast<const __nv_bfloat16*>(value_cache);
+  }
   a.block_tables = block_tables;
   a.plan_count = reinterpret_cast<const int32_t*>(dws + L.dec.off_count);
   a.entries = reinterpret_cast<const PlanEntry*>(dws + L.dec.off_entries);
@@ -393,7 +545,9 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
   a.block_offset = v_offset;
   a.always_partial = 1;
   int rc = launch_decode_plan(a, v_lens, in.max_suffix_len, s);
-  if (rc == PKV_OK) rc = launch_decode_tensor(a, head_dim, out_dtype == PKV_DTYPE_F32, s);
+  if (rc == PKV_OK)
+    rc = kv8 ? launch_decode_tensor_fp8(a, head_dim, out_dtype == PKV_DTYPE_F32, s)
+             : launch_decode_tensor(a, head_dim, out_dtype == PKV_DTYPE_F32, s);
   if (in.num_entries > 0) {
     e = cudaStreamWaitEvent(s, side.join, 0);  // the merge reads the shared partials
     if (rc == PKV_OK && e != cudaSuccess) rc = set_error(PKV_ERR_CUDA, "shared decode: join: %s", cudaGetErrorString(e));
@@ -424,4 +578,32 @@ extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "shared merge launch: %s", cudaGetErrorString(e));
   return PKV_OK;
+}
+
+extern "C" int pkv_paged_attention_decode_shared(void* out, int out_dtype, const void* query, const void* key_cache,
+                                                 const void* value_cache, const int32_t* block_tables,
+                                                 int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                                 int num_blocks, float scale, const void* plan,
+                                                 const pkv_shared_plan_info* info, void* workspace,
+                                                 size_t workspace_bytes, int32_t* status, pkv_stream_t stream) {
+  clear_error();
+  return shared_impl(false, out, out_dtype, query, key_cache, value_cache, nullptr, nullptr, block_tables,
+                     max_blocks_per_seq, context_lens, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                     num_blocks, scale, plan, info, workspace, workspace_bytes, status, stream);
+}
+
+extern "C" int pkv_paged_attention_decode_shared_fp8(void* out, int out_dtype, const void* query,
+                                                     const void* key_cache, const void* value_cache,
+                                                     const float* k_scale, const float* v_scale,
+                                                     const int32_t* block_tables, int max_blocks_per_seq,
+                                                     const int32_t* context_lens, int num_seqs, int num_heads,
+                                                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                                     float scale, const void* plan, const pkv_shared_plan_info* info,
+                                                     void* workspace, size_t workspace_bytes, int32_t* status,
+                                                     pkv_stream_t stream) {
+  clear_error();
+  return shared_impl(true, out, out_dtype, query, key_cache, value_cache, k_scale, v_scale, block_tables,
+                     max_blocks_per_seq, context_lens, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                     num_blocks, scale, plan, info, workspace, workspace_bytes, status, stream);
 }

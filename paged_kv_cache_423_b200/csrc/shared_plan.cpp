@@ -185,10 +185,12 @@ extern "C" int pkv_shared_plan(const int32_t* block_tables, int max_blocks_per_s
   int32_t* row_start = reinterpret_cast<int32_t*>(base + in.off_row_start);
   int32_t* row_ids = reinterpret_cast<int32_t*>(base + in.off_row_ids);
 
-  // partial ids: part i covers rows row0 .. row0 + nrows - 1 with ids first .. first + nrows - 1
+  // partial ids: part i covers rows row0 .. row0 + nrows - 1 with ids first .. first + nrows - 1;
+  // its blocks take the scratch blocks base .. base + keys / block_size - 1 (the 8-bit run
+  // widens every part's blocks into a scratch pool in this order)
   std::vector<int> first(parts.size());
   std::vector<int> per_row(num_seqs + 1, 0);
-  int next_id = 0, e = 0;
+  int next_id = 0, e = 0, next_block = 0;
   for (size_t i = 0; i < parts.size(); ++i) {
     const Segment& sg = segs[parts[i].seg];
     first[i] = next_id;
@@ -200,6 +202,8 @@ extern "C" int pkv_shared_plan(const int32_t* block_tables, int max_blocks_per_s
     d[3] = sg.row0;
     d[4] = sg.nrows;
     d[5] = first[i];
+    d[6] = next_block;
+    next_block += parts[i].nkeys / block_size;
     for (int r0 = 0; r0 < sg.nrows; r0 += pair_rows, ++e) {
       const int na = std::min(tile_rows, sg.nrows - r0);
       const int nb = std::max(0, std::min(tile_rows, sg.nrows - r0 - tile_rows));

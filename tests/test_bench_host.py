@@ -470,6 +470,25 @@ def test_run_ours_beam_phase_with_stand_ins(pkv, monkeypatch):
     json.dumps(res)
 
 
+def test_run_ours_shared_prefix_over_an_8bit_pool_with_stand_ins(pkv, monkeypatch):
+    """The shared-prompt batch over an 8-bit pool takes the shared-prefix decode: launches per
+    step include the widening of the shared blocks and the query split."""
+    import workloads as wl
+    orig = wl.make_decode_batch
+    monkeypatch.setattr(wl, "make_decode_batch", lambda name, **k: orig(name, num_seqs=6, **k))
+    calls = {}
+    res = _stand_in_run_ours(monkeypatch, pkv, calls, workload="prefix_beams", kv="fp8", steps=4, states=4)
+    cfg = res["config"]
+    assert cfg["decode"] == "shared-prefix" and cfg["kv_dtype"] == "fp8"
+    r = res["roofline"]
+    assert r["kernel"].startswith("paged_attention_decode_shared_fp8")
+    assert r["algorithmic_bytes_per_launch"] < r["logical_bytes_per_launch"]
+    # per step: write, setup, widening + shared phase, plan, query split, decode, merge
+    assert res["gpu_launches"] == 4 * 8
+    import json
+    json.dumps(res)
+
+
 def test_recorded_traffic_only_for_the_captured_batch(tmp_path, monkeypatch):
     """A recorded ncu figure is reported only for the kernel sources, table layout and batch
     size it was captured on."""
@@ -669,7 +688,7 @@ def test_shared_decode_applies_only_where_it_can_run():
     assert not bench.shared_decode_applies(args(), w(shared_blocks=0))  # nothing shared: plain decode
     assert bench.shared_decode_applies(args("on"), w(shared_blocks=0))
     assert not bench.shared_decode_applies(args("off"), w())
-    assert not bench.shared_decode_applies(args(), w(kv8=True))        # bf16 pools only
+    assert bench.shared_decode_applies(args(), w(kv8=True))            # the 8-bit pool too
     assert not bench.shared_decode_applies(args(path="simt"), w())
     assert not bench.shared_decode_applies(args(), w(Hq=40, Hkv=40))   # MHA: no tensor-core decode
     with pytest.raises(SystemExit):

@@ -72,8 +72,11 @@ def check_plan(tables, lens, bs, g, plan, info, min_rows=2):
     # every part: its rows hold its blocks, full
     got_segs = set()
     id_of = {}
-    for p, (trow, blk0, nkeys, row0, nrows, first, z0, z1) in enumerate(parts.tolist()):
-        assert z0 == 0 and z1 == 0 and trow == row0 and 1 <= nkeys <= info.key_chunk and nkeys % bs == 0
+    scratch = 0
+    for p, (trow, blk0, nkeys, row0, nrows, first, base, z1) in enumerate(parts.tolist()):
+        assert z1 == 0 and trow == row0 and 1 <= nkeys <= info.key_chunk and nkeys % bs == 0
+        assert base == scratch  # scratch blocks of the 8-bit run, consecutive in plan order
+        scratch += nkeys // bs
         nblk = nkeys // bs
         for r in range(row0, row0 + nrows):
             for k in range(blk0, blk0 + nblk):
@@ -108,6 +111,7 @@ def check_plan(tables, lens, bs, g, plan, info, min_rows=2):
     nk = [parts[entries[e][3]][2] for e in range(len(entries))]
     assert nk == sorted(nk, reverse=True)
     assert info.shared_row_tokens == sum(depth) * bs
+    assert scratch * bs == info.shared_tokens
 
 
 def beam_batch(seed, parents=6, beams=4, prompt_blocks=3, bs=16, steps=2):

@@ -105,6 +105,7 @@ struct SetupArgs {
   int32_t* v_offset;
   int32_t* status;
   int num_seqs, num_entries, num_parts, num_partials, max_blocks, block_size, tile_rows, max_suffix_len;
+  int64_t scratch_blocks;  // 8-bit run: the scratch pools' blocks (each part's base is checked), else -1
 };
 
 __global__ void __launch_bounds__(kSetupThreads) shared_setup_kernel(const SetupArgs p) {
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(kSetupThreads) shared_setup_kernel(const Setup
     mine |= d0.x < 0 || d0.x >= p.num_seqs || d0.y < 0 || d0.z < 1 || d0.y + nblk > p.max_blocks || d0.w < 0 ||
             d1.x < 1 || static_cast<int64_t>(d0.w) + d1.x > p.num_seqs || d1.y < 0 ||
             static_cast<int64_t>(d1.y) + d1.x > p.num_partials;
+    if (p.scratch_blocks >= 0) mine |= d0.z % p.block_size != 0 || d1.z < 0 || d1.z + nblk > p.scratch_blocks;
   }
   for (int i = threadIdx.x; i < p.num_entries; i += blockDim.x) {
     const int4 e = p.entries[i];
@@ -422,6 +424,7 @@ static int shared_impl(bool kv8, void* out, int out_dtype, const void* query, co
   sa.block_size = block_size;
   sa.tile_rows = 128 / group;
   sa.max_suffix_len = in.max_suffix_len;
+  sa.scratch_blocks = kv8 ? L.scratch_blocks : -1;
   sp::shared_setup_kernel<<<1, sp::kSetupThreads, 0, s>>>(sa);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "shared setup launch: %s", cudaGetErrorString(e));

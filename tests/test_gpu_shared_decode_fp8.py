@@ -5,8 +5,9 @@ share blocks, not results; intelliparadigm article §4.2, §5: fp8 KV).  The poo
 e4m3 bit patterns with per-kv-head scales, as for the 8-bit decode tests.  Batches: a shared
 system prompt (small, and full size on sampled rows), beam forks with copy-on-write after
 appends (nested segments), several key-chunk sizes, block size 32, a batch with no sharing, a
-plan that no longer fits the lengths (flagged, zero output) and a shared block outside the
-pool (flagged).  Tolerance as for decode (fp32 output)."""
+plan that no longer fits the lengths (flagged, zero output), a plan whose scratch blocks run
+past the scratch pools (flagged, zero output) and a shared block outside the pool (flagged).
+Tolerance as for decode (fp32 output)."""
 import numpy as np
 import pytest
 import torch
@@ -134,3 +135,22 @@ def test_shared_block_outside_the_pool_is_flagged(pkv):
     assert info.num_segments == 1
     assert status.item() & pkv.PKV_DEV_BAD_BLOCK
     assert torch.isfinite(out).all()
+
+
+def test_plan_with_a_bad_scratch_base_is_flagged_and_zeroed(pkv):
+    """A part whose scratch blocks would run past the scratch pools: the plan check rejects the
+    plan (PKV_DEV_BAD_CONTEXT, zero rows) before anything is widened or read."""
+    p = Pool8(wl.make_decode_batch("prefix_beams", num_seqs=8, length_scale=0.3), 1280)
+    b = p.b
+    plan, info = pkv.shared_plan(b.block_tables, b.context_lens, b.num_heads, b.num_kv_heads, b.block_size)
+    words = plan.view(np.int32)
+    words[info.off_parts // 4 + 6] = 1 << 20  # part 0's first scratch block
+    ws = torch.empty(pkv.paged_attention_decode_shared_fp8_workspace_size(info, b.num_heads, b.num_kv_heads,
+                                                                          b.head_dim), dtype=torch.uint8, device="cuda")
+    out = torch.full((b.num_seqs, b.num_heads, b.head_dim), float("nan"), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_attention_decode_shared_fp8(out, p.query, p.kc_d, p.vc_d, p.ks_d, p.vs_d, p.tables, p.lens, b.scale,
+                                          torch.from_numpy(plan).cuda(), info, ws, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & pkv.PKV_DEV_BAD_CONTEXT
+    assert torch.all(out == 0)

@@ -170,13 +170,15 @@ __device__ __forceinline__ int item_stages(const PlanEntry& e, int partition, in
   return ntok == 0 ? 1 : (ntok + stage_tok - 1) / stage_tok;
 }
 
-// Load lane j's table entry for the item (block tok0/bs + j), 0 past the item.
+// Load lane j's table entry for the item (block tok0/bs + j, from the row's block_offset on
+// when there is one), 0 past the item.
 __device__ __forceinline__ int load_item_table(const DecodeArgs& a, const PlanEntry& e, int lane) {
   const int tok0 = e.y * a.partition;
   const int ntok = e.w == 0 ? 0 : min(a.partition, e.w - tok0);
   const int nblk = (ntok + a.block_size - 1) / a.block_size;
   if (lane >= nblk) return 0;
-  return __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + lane);
+  const int off = a.block_offset ? __ldg(a.block_offset + e.x) : 0;
+  return __ldg(a.block_tables + static_cast<int64_t>(e.x) * a.max_blocks + tok0 / a.block_size + off + lane);
 }
 
 // a0 += q.lo * k.lo, a1 += q.hi * k.hi with bf16 operands and fp32 accumulation
@@ -664,8 +666,15 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
       l *= 0.5f;  // every row's weight was held by its two lanes
-      if (nparts == 1) {
+      if (nparts == 1 && !a.always_partial) {
         store_row<D, OUT_F32>(a, seq, qh, lane, of, l > 0.f ? 1.f / l : 0.f);
+      } else if (a.always_partial) {
+        // every item's partial for the caller's merge (the shared-prefix decode's private phase)
+        const int64_t pidx = (static_cast<int64_t>(seq) * a.num_heads + qh) * a.max_parts + part;
+        float* po = a.part_o + pidx * D + lane * EPL;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) po[j] = of[j];
+        if (lane == 0) a.part_ml[pidx] = make_float2(m, l);
       } else {
         const int64_t unit = static_cast<int64_t>(seq) * a.num_heads + qh;
         const int64_t pidx = unit * a.max_parts + part;
@@ -745,6 +754,12 @@ static int launch_simt(const DecodeArgs& a, cudaStream_t stream) {
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(PKV_ERR_CUDA, "decode (simt) launch: %s", cudaGetErrorString(e));
   return PKV_OK;
+}
+
+int launch_decode_simt(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream) {
+  if (a.key_cache8) return out_f32 ? launch_simt<128, true, true>(a, stream) : launch_simt<128, false, true>(a, stream);
+  if (head_dim == 128) return out_f32 ? launch_simt<128, true>(a, stream) : launch_simt<128, false>(a, stream);
+  return out_f32 ? launch_simt<64, true>(a, stream) : launch_simt<64, false>(a, stream);
 }
 
 int launch_decode_plan(const DecodeArgs& a, const int32_t* context_lens, int max_context_len, cudaStream_t stream) {

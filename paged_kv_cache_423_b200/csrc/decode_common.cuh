@@ -158,6 +158,8 @@ int launch_prefill_segments(const SegmentLaunch& launch, cudaStream_t stream);
 // entries longest first into a.entries, zeroes a.plan_count's counter and a.arrive.
 int launch_decode_plan(const DecodeArgs& a, const int32_t* context_lens, int max_context_len, cudaStream_t stream);
 int launch_decode_tensor(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
+// The CUDA-core decode (bf16 pools, or 8-bit ones when a.key_cache8 is set; decode.cu).
+int launch_decode_simt(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
 int launch_decode_tensor_fp8(const DecodeArgs& a, int head_dim, bool out_f32, cudaStream_t stream);
 // Merge of split partitions (no launch when max_parts <= 1), after a tensor-core decode.
 int launch_merge_partials(const DecodeArgs& a, bool out_f32, cudaStream_t stream);

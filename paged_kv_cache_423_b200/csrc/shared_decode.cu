@@ -46,6 +46,16 @@ namespace sp {
 
 constexpr int kD = 128;
 constexpr int kSetupThreads = 1024;
+// Private remainders of at most this many tokens (one tile of the tensor-core decode) go
+// through the CUDA-core decode (a warp per (row, query head, partition), little fixed work per
+// item), longer ones through the tensor-core decode (one item per (row, kv head, partition),
+// tiles of 128 tokens).  Measured on the shared-prompt batch forked into 4 beams (remainders of
+// at most 32 tokens) the CUDA-core phase is faster; with the prompt batch's remainders of up to
+// 500 tokens the tensor-core one is.
+#ifndef PKV_SHARED_SIMT_MAX
+#define PKV_SHARED_SIMT_MAX 128
+#endif
+constexpr int kSimtSuffixMax = PKV_SHARED_SIMT_MAX;
 constexpr int kMergeWarps = 4;
 
 struct Layout {
@@ -54,6 +64,7 @@ struct Layout {
   int64_t scratch_blocks = 0;
   WorkspaceLayout dec;
   int partition = 0;
+  bool private_simt = false;  // the private phase on the CUDA-core decode
 };
 
 // Workspace: [plan count, work counter, bad flag] | checked remainders | checked block offsets |
@@ -63,7 +74,9 @@ struct Layout {
 static Layout layout(const pkv_shared_plan_info& in, int num_heads, int num_kv_heads, bool kv8) {
   Layout L;
   const int B = in.num_seqs;
-  L.partition = auto_partition_tokens_tensor(B, num_kv_heads, in.block_size, in.max_suffix_len);
+  L.private_simt = in.max_suffix_len <= kSimtSuffixMax;
+  L.partition = L.private_simt ? auto_partition_tokens(B, num_kv_heads, in.block_size, in.max_suffix_len)
+                               : auto_partition_tokens_tensor(B, num_kv_heads, in.block_size, in.max_suffix_len);
   size_t off = 0;
   L.off_count = off;
   off = align256(off + 4 * sizeof(int32_t));
@@ -549,8 +562,9 @@ static int shared_impl(bool kv8, void* out, int out_dtype, const void* query, co
   a.always_partial = 1;
   int rc = launch_decode_plan(a, v_lens, in.max_suffix_len, s);
   if (rc == PKV_OK)
-    rc = kv8 ? launch_decode_tensor_fp8(a, head_dim, out_dtype == PKV_DTYPE_F32, s)
-             : launch_decode_tensor(a, head_dim, out_dtype == PKV_DTYPE_F32, s);
+    rc = L.private_simt ? launch_decode_simt(a, head_dim, out_dtype == PKV_DTYPE_F32, s)
+         : kv8          ? launch_decode_tensor_fp8(a, head_dim, out_dtype == PKV_DTYPE_F32, s)
+                        : launch_decode_tensor(a, head_dim, out_dtype == PKV_DTYPE_F32, s);
   if (in.num_entries > 0) {
     e = cudaStreamWaitEvent(s, side.join, 0);  // the merge reads the shared partials
     if (rc == PKV_OK && e != cudaSuccess) rc = set_error(PKV_ERR_CUDA, "shared decode: join: %s", cudaGetErrorString(e));

@@ -184,3 +184,13 @@ def test_two_calls_on_two_streams(pkv):
     for (out, status, _, _), b in zip(outs, (b1, b2)):
         assert status.item() == 0
         compare(out.cpu().numpy(), oracle_out(b))
+
+
+def test_long_remainders_match_oracle(pkv):
+    """Private remainders past one 128-token tile go through the tensor-core decode (shorter ones
+    through the CUDA-core decode, as in the beam batches here): a shared prompt with long remainders."""
+    lens = 1024 + np.array([1100, 1350, 1600, 1200, 1500], np.int32)
+    b = wl.make_decode_batch("prefix_beams", lengths=lens, seed=91)
+    out, info = run_shared(pkv, DeviceBatch(b))
+    assert info.num_segments == 1 and info.max_suffix_len > 1024
+    compare(out.cpu().numpy(), oracle_out(b))

@@ -154,3 +154,14 @@ def test_plan_with_a_bad_scratch_base_is_flagged_and_zeroed(pkv):
     torch.cuda.synchronize()
     assert status.item() & pkv.PKV_DEV_BAD_CONTEXT
     assert torch.all(out == 0)
+
+
+def test_long_remainders_match_oracle(pkv):
+    """Private remainders past one 128-token tile go through the 8-bit tensor-core decode (shorter
+    ones through the 8-bit CUDA-core decode, as in the beam batches here): a shared prompt with long
+    remainders."""
+    lens = 1024 + np.array([1100, 1350, 1600, 1200, 1500], np.int32)
+    p = Pool8(wl.make_decode_batch("prefix_beams", lengths=lens, seed=92), 1290)
+    out, info = run_shared(pkv, p)
+    assert info.num_segments == 1 and info.max_suffix_len > 1024
+    compare(out.cpu().numpy(), p.oracle())

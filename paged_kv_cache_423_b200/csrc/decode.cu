@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(kPlanThreads)
 // fixed cost of a stage (wait, reductions, softmax) is spread over as many bytes.
 template <bool KV8>
 constexpr int stage_tokens() { return KV8 ? 2 * kStageTokens : kStageTokens; }
+// Values per lane of the 8-bit pool's P·V accumulators (a 16-byte chunk of a head_dim-128 row).
+constexpr int kPV8 = 16;
 
 template <int D, int STAGES, bool KV8 = false>
 struct __align__(128) WarpRing {
@@ -153,7 +155,7 @@ struct __align__(128) WarpRing {
   KvT v[STAGES][ST * D];
   __nv_bfloat16 q[STAGES][D];
   float2 p[ST];  // (p_t, p_t) of the stage being consumed, read back as packed pairs
-                 // (8-bit pool: p_t rounded to f16 in the low half of .x)
+                 // (8-bit pool: p_t rounded to f16, packed as 32 halves in the first 64 bytes)
   uint64_t full[STAGES];
   int4 meta[STAGES];  // x seq, y query head, z part | nparts << 16, w n_valid | flags (first, last, q present)
 };
@@ -194,10 +196,10 @@ __device__ __forceinline__ void dot_bf16x2(float& a0, float& a1, uint32_t q, uin
 }
 
 template <int D, bool OUT_F32>
-__device__ __forceinline__ void store_row(const DecodeArgs& a, int seq, int qh, int lane, const float* o,
+__device__ __forceinline__ void store_row(const DecodeArgs& a, int seq, int qh, int col, const float* o,
                                           float inv) {
   constexpr int EPL = D / 32;
-  const int64_t base = (static_cast<int64_t>(seq) * a.num_heads + qh) * D + lane * EPL;
+  const int64_t base = (static_cast<int64_t>(seq) * a.num_heads + qh) * D + col;
   if constexpr (OUT_F32) {
     float* out = static_cast<float*>(a.out) + base;
     if constexpr (EPL == 4)
@@ -272,15 +274,25 @@ __device__ __forceinline__ void dot_f16x2(float& a0, float& a1, uint32_t x, uint
       : "+f"(a0), "+f"(a1)
       : "r"(x), "r"(y));
 }
-// a += p * x.lo, b += p * x.hi (p an f16 in the low half of `p16`)
+// a += p * x.lo, b += p * x.hi with p the low (HI = false) or high f16 of `p16`
+template <bool HI>
 __device__ __forceinline__ void axpy_f16x2(float& a, float& b, uint32_t p16, uint32_t x) {
-  asm("{\n\t.reg .b16 pl, ph, xl, xh;\n\t"
-      "mov.b32 {pl, ph}, %2;\n\t"
-      "mov.b32 {xl, xh}, %3;\n\t"
-      "fma.rn.f32.f16 %0, pl, xl, %0;\n\t"
-      "fma.rn.f32.f16 %1, pl, xh, %1;\n\t}"
-      : "+f"(a), "+f"(b)
-      : "r"(p16), "r"(x));
+  if constexpr (HI)
+    asm("{\n\t.reg .b16 pl, ph, xl, xh;\n\t"
+        "mov.b32 {pl, ph}, %2;\n\t"
+        "mov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, ph, xl, %0;\n\t"
+        "fma.rn.f32.f16 %1, ph, xh, %1;\n\t}"
+        : "+f"(a), "+f"(b)
+        : "r"(p16), "r"(x));
+  else
+    asm("{\n\t.reg .b16 pl, ph, xl, xh;\n\t"
+        "mov.b32 {pl, ph}, %2;\n\t"
+        "mov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, pl, xl, %0;\n\t"
+        "fma.rn.f32.f16 %1, pl, xh, %1;\n\t}"
+        : "+f"(a), "+f"(b)
+        : "r"(p16), "r"(x));
 }
 __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   uint32_t r;
@@ -438,13 +450,15 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
   constexpr int NQ = KV8 ? 2 * NC : NC;
   uint4 qv[NQ];
   uint64_t o[NPAIR];            // packed fp32 output accumulators
-  float o8[KV8 ? 2 * EPL : 1];  // 8-bit pool: scalar fp32 accumulators, two sets (even / odd tokens)
+  // 8-bit pool: fp32 accumulators of the lane's 16 values (a 16-byte chunk of a row) over the
+  // rows of its row group; the four row groups are added once per item
+  float o8[KV8 ? kPV8 : 1];
   float score_scale = a.scale_log2, out_scale = 1.f;
   float m = -INFINITY, lsum = 0.f;
 #pragma unroll
   for (int i = 0; i < NQ; ++i) qv[i] = make_uint4(0, 0, 0, 0);
 #pragma unroll
-  for (int j = 0; j < (KV8 ? 2 * EPL : 1); ++j) o8[j] = 0.f;
+  for (int j = 0; j < (KV8 ? kPV8 : 1); ++j) o8[j] = 0.f;
 #pragma unroll
   for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
 
@@ -471,7 +485,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       for (int j = 0; j < NPAIR; ++j) o[j] = f2pack(0.f, 0.f);
       if constexpr (KV8) {
 #pragma unroll
-        for (int j = 0; j < 2 * EPL; ++j) o8[j] = 0.f;
+        for (int j = 0; j < kPV8; ++j) o8[j] = 0.f;
         if (mt.w & 0x400) {
           // q to f16 for the mixed-precision products.  bf16 values of magnitude
           // >= 2^15 would overflow f16: then the whole vector is scaled by 2^-16
@@ -556,8 +570,9 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
         m = m_new;
         lsum = fmaf(lsum, alpha, f16lo_to_f32(p16a) + f16lo_to_f32(p16b));
         if (qk_half == 0) {
-          ring.p[qk_row] = make_float2(__uint_as_float(p16a), 0.f);
-          ring.p[qk_row + kStageTokens] = make_float2(__uint_as_float(p16b), 0.f);
+          uint16_t* p16 = reinterpret_cast<uint16_t*>(ring.p);
+          p16[qk_row] = static_cast<uint16_t>(p16a);
+          p16[qk_row + kStageTokens] = static_cast<uint16_t>(p16b);
         }
       } else {
       // ---- scores: two lanes per row, bf16 x bf16 products accumulated in fp32
@@ -586,32 +601,32 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       __syncwarp();
       // ---- P·V: packed fp32 pairs, rows past n_valid never touched (stale rows may be NaN)
       if constexpr (KV8) {
-        // ---- P·V over e4m3 rows: lane l owns values 4l..4l+3; f16 x f16 products, fp32 sums
+        // ---- P·V over e4m3 rows: row group g = lane / 8 takes rows 8g..8g+7 of the stage and
+        // lane l its 16-byte chunk l % 8 of each (16 values); f16 x f16 products, fp32 sums.
+        // Rows past n_valid are not loaded (stale rows may hold NaN codes).
 #pragma unroll
-        for (int j = 0; j < 2 * EPL; ++j) o8[j] *= alpha;
-        const uint8_t* vb = ring.v[slot] + lane * EPL;
-        const float2* pr = ring.p;
-        // even and odd tokens accumulate into separate sets (shorter dependency chains)
-        int t = 0;
-#pragma unroll 4
-        for (; t + 1 < n_valid; t += 2) {
-          const uint32_t pw0 = __float_as_uint(pr[t].x), pw1 = __float_as_uint(pr[t + 1].x);
-          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vb + t * D);
-          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vb + (t + 1) * D);
-          uint32_t v01, v23, u01, u23;
-          e4m3x4_to_f16x2x2(w0, v01, v23);
-          e4m3x4_to_f16x2x2(w1, u01, u23);
-          axpy_f16x2(o8[0], o8[1], pw0, v01);
-          axpy_f16x2(o8[2], o8[3], pw0, v23);
-          axpy_f16x2(o8[4], o8[5], pw1, u01);
-          axpy_f16x2(o8[6], o8[7], pw1, u23);
-        }
-        if (t < n_valid) {
-          const uint32_t pw0 = __float_as_uint(pr[t].x);
-          uint32_t v01, v23;
-          e4m3x4_to_f16x2x2(*reinterpret_cast<const uint32_t*>(vb + t * D), v01, v23);
-          axpy_f16x2(o8[0], o8[1], pw0, v01);
-          axpy_f16x2(o8[2], o8[3], pw0, v23);
+        for (int j = 0; j < kPV8; ++j) o8[j] *= alpha;
+        const int g = lane >> 3;
+        const uint8_t* vb = ring.v[slot] + g * 8 * D + (lane & 7) * 16;
+        const uint4 pw = reinterpret_cast<const uint4*>(ring.p)[g];  // p of rows 8g..8g+7 (f16)
+        const uint32_t pws[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          uint4 w = make_uint4(0, 0, 0, 0);
+          if (g * 8 + k < n_valid) w = *reinterpret_cast<const uint4*>(vb + k * D);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v01, v23;
+            e4m3x4_to_f16x2x2(ws[c], v01, v23);
+            if (k & 1) {
+              axpy_f16x2<true>(o8[4 * c], o8[4 * c + 1], pws[k >> 1], v01);
+              axpy_f16x2<true>(o8[4 * c + 2], o8[4 * c + 3], pws[k >> 1], v23);
+            } else {
+              axpy_f16x2<false>(o8[4 * c], o8[4 * c + 1], pws[k >> 1], v01);
+              axpy_f16x2<false>(o8[4 * c + 2], o8[4 * c + 3], pws[k >> 1], v23);
+            }
+          }
         }
       } else {
       const uint64_t alpha2 = f2pack(alpha, alpha);
@@ -651,9 +666,27 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
     if (last) {
       const int seq = mt.x, qh = mt.y, part = mt.z & 0xffff, nparts = mt.z >> 16;
       float of[EPL];
+      // the lane's first output column: 8-bit pool, after the row groups' sums are scattered,
+      // values 4g..4g+3 of its chunk
+      const int col = KV8 ? (lane & 7) * 16 + (lane >> 3) * 4 : lane * EPL;
       if constexpr (KV8) {
+        // Add the four row groups' sums, each lane keeping 4 of its chunk's 16 values: across
+        // lanes l and l ^ 16 (groups g, g ^ 2) the halves 8 (g >> 1).. go to their owner, then
+        // across l and l ^ 8 (g, g ^ 1) the quarters 4 (g & 1)...
+        const bool hi = lane & 16, odd = lane & 8;
+        float h8[8], q4[4];
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) of[j] = (o8[j] + o8[EPL + j]) * out_scale;  // the value scale of the kv head
+        for (int j = 0; j < 8; ++j) {
+          const float give = hi ? o8[j] : o8[8 + j];
+          h8[j] = (hi ? o8[8 + j] : o8[j]) + __shfl_xor_sync(kFull, give, 16);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float give = odd ? h8[j] : h8[4 + j];
+          q4[j] = (odd ? h8[4 + j] : h8[j]) + __shfl_xor_sync(kFull, give, 8);
+        }
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) of[j] = q4[j] * out_scale;  // the value scale of the kv head
       } else {
 #pragma unroll
         for (int j = 0; j < NPAIR; ++j) {
@@ -667,18 +700,18 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
       for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
       l *= 0.5f;  // every row's weight was held by its two lanes
       if (nparts == 1 && !a.always_partial) {
-        store_row<D, OUT_F32>(a, seq, qh, lane, of, l > 0.f ? 1.f / l : 0.f);
+        store_row<D, OUT_F32>(a, seq, qh, col, of, l > 0.f ? 1.f / l : 0.f);
       } else if (a.always_partial) {
         // every item's partial for the caller's merge (the shared-prefix decode's private phase)
         const int64_t pidx = (static_cast<int64_t>(seq) * a.num_heads + qh) * a.max_parts + part;
-        float* po = a.part_o + pidx * D + lane * EPL;
+        float* po = a.part_o + pidx * D + col;
 #pragma unroll
         for (int j = 0; j < EPL; ++j) po[j] = of[j];
         if (lane == 0) a.part_ml[pidx] = make_float2(m, l);
       } else {
         const int64_t unit = static_cast<int64_t>(seq) * a.num_heads + qh;
         const int64_t pidx = unit * a.max_parts + part;
-        float* po = a.part_o + pidx * D + lane * EPL;
+        float* po = a.part_o + pidx * D + col;
 #pragma unroll
         for (int j = 0; j < EPL; ++j) po[j] = of[j];
         if (lane == 0) a.part_ml[pidx] = make_float2(m, l);
@@ -696,7 +729,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
           float acc[EPL], Ls = 0.f;
 #pragma unroll
           for (int j = 0; j < EPL; ++j) acc[j] = 0.f;
-          const float* pb = a.part_o + unit * a.max_parts * D + lane * EPL;
+          const float* pb = a.part_o + unit * a.max_parts * D + col;
           for (int p = 0; p < nparts; ++p) {
             const float2 mlp = __ldcg(&ml[p]);
             const float w = exp2f(mlp.x - M);
@@ -704,7 +737,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(const __grid_co
 #pragma unroll
             for (int j = 0; j < EPL; ++j) acc[j] = fmaf(w, __ldcg(pb + static_cast<int64_t>(p) * D + j), acc[j]);
           }
-          store_row<D, OUT_F32>(a, seq, qh, lane, acc, Ls > 0.f ? 1.f / Ls : 0.f);
+          store_row<D, OUT_F32>(a, seq, qh, col, acc, Ls > 0.f ? 1.f / Ls : 0.f);
           if (lane == 0) a.arrive[unit] = 0;
         }
       }

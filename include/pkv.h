@@ -319,8 +319,10 @@ PKV_API int pkv_paged_attention_prefill(void* out, int out_dtype, const void* qu
  *   1. shared phase: each segment is a dense contraction of all its rows' query heads
  *      against the segment's keys (the tensor-core prefill kernel with every key
  *      visible and unnormalised partial results), cut into key chunks for parallelism;
- *   2. private phase: every row's remainder through the tensor-core decode (grouped
- *      heads, head_dim 128), writing partial results only;
+ *   2. private phase: every row's remainder through a decode kernel writing partial
+ *      results only: the CUDA-core decode when no remainder is longer than 128 tokens
+ *      (one tile; many short items, as after beams fork), else the tensor-core decode
+ *      (grouped heads, head_dim 128);
  *   3. merge: per (row, head), the formula above over the row's shared partials and
  *      its private partitions.
  *
@@ -399,7 +401,7 @@ PKV_API int pkv_paged_attention_decode_shared(void* out, int out_dtype, const vo
  * The shared phase first widens the codes of the plan's shared blocks into two bf16 scratch
  * pools inside the workspace (exact: every e4m3 value is a bf16 value), then runs with each
  * kv head's key scale folded into its scores and its value scale into its partial outputs;
- * the private phase is the 8-bit tensor-core decode.  Workspace:
+ * the private phase is the 8-bit decode (CUDA cores or tensor cores, by the same rule).  Workspace:
  * pkv_paged_attention_decode_shared_fp8_workspace_size() bytes, the bf16 call's plus the split
  * queries, two scratch pools of info->shared_tokens * num_kv_heads * 128 * 2 bytes and a table
  * of num_seqs * max_blocks_per_seq int32.  A table entry of a shared block outside the pool

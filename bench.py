@@ -134,6 +134,9 @@ def recorded_traffic(key: str, kind: str, units: int, layout=None):
 
 
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e nominal (DGX figure)
+# The shared-prefix decode's private phase runs on the CUDA-core decode when no row's remainder
+# is longer than this (one 128-token tile), else on the tensor-core decode (csrc/shared_decode.cu).
+SHARED_SIMT_SUFFIX_MAX = 128
 L2_BYTES = 126 * 1000 ** 2  # B200 L2
 
 
@@ -600,8 +603,10 @@ def run_ours(args, rank, world, local_rank):
         unique_total += alg - kv + st["unique_kv"]
         unique_kv_total += st["unique_kv"]
         if use_shared:  # write, setup, [widening and] shared phase (when there are segments), plan,
-            # [query split,] decode, merge
-            launches += (5 + (1 if st["plan"][1].num_entries else 0) * (2 if kv8 else 1) + (1 if kv8 else 0)
+            # [query split (8-bit tensor-core private phase),] decode, merge
+            info = st["plan"][1]
+            launches += (5 + (1 if info.num_entries else 0) * (2 if kv8 else 1)
+                         + (1 if kv8 and info.max_suffix_len > SHARED_SIMT_SUFFIX_MAX else 0)
                          + (1 if st["n_pairs"] else 0))
         else:
             launches += 3 + (1 if st["n_pairs"] else 0) + merge
@@ -672,12 +677,14 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": unique_total // args.steps,
                      "logical_bytes_per_launch": bytes_total // args.steps, "peak_kind": peak_kind,
                      "kernel": ("paged_attention_decode_shared_fp8: setup + shared phase (the shared blocks widened"
-                                " to bf16, tcgen05 prefill kernel, every key visible, partials) + plan + query split +"
-                                " tcgen05 kind::f8f6f4 decode of the private remainders + merge; traffic = the DRAM"
-                                " bytes of all of them" if use_shared and kv8
+                                " to bf16, tcgen05 prefill kernel, every key visible, partials) + plan + decode of"
+                                " the private remainders (CUDA cores when none passes 128 tokens, else query split +"
+                                " tcgen05 kind::f8f6f4) + merge; traffic = the DRAM bytes of all of them"
+                                if use_shared and kv8
                                 else "paged_attention_decode_shared: setup + shared phase (tcgen05 prefill kernel, every"
-                                " key visible, partials) + plan + tcgen05 decode of the private remainders + merge;"
-                                " traffic = the DRAM bytes of all of them" if use_shared
+                                " key visible, partials) + plan + decode of the private remainders (CUDA cores when"
+                                " none passes 128 tokens, else tcgen05) + merge; traffic = the DRAM bytes of all of"
+                                " them" if use_shared
                                 else "paged_attention_decode_fp8: plan + tcgen05 kind::f8f6f4 kernel on the e4m3 tiles"
                                 " + split merge" if kv8 and uses_tensor
                                 else "paged_attention_decode_fp8: plan + CUDA-core streaming kernel (e4m3 tiles)" if kv8

@@ -725,3 +725,12 @@ def test_e2e_shared_prefix_plan_travels_with_each_step(pkv, monkeypatch):
     assert len(seen) == 7 and all(b > 0 for b in seen)
     plain = 2 * w.B * (w.Hq + 2 * w.Hkv) * w.D + 8 * w.B + 4 * w.B * w.max_blocks + 4 * w.B
     assert res["h2d_bytes_per_step"] == plain + sum(seen[3:]) // 4
+
+
+def test_shared_private_rule_matches_the_library():
+    """bench.py counts the 8-bit query split only when the shared-prefix decode's private phase
+    is on the tensor cores; its remainder bound must be the library's."""
+    import re
+    src = open(os.path.join(bench.ROOT, "paged_kv_cache_423_b200", "csrc", "shared_decode.cu")).read()
+    m = re.search(r"#define PKV_SHARED_SIMT_MAX (\d+)", src)
+    assert m and int(m.group(1)) == bench.SHARED_SIMT_SUFFIX_MAX

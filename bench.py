@@ -444,6 +444,16 @@ class Workload:
         return q, k, v
 
 
+def shared_min_rows(args) -> int:
+    """Fewest rows a shared segment serves.  Over a bf16 pool a segment of 2 rows already saves
+    reads; over an 8-bit pool a segment's blocks are first widened to bf16 scratch (a read of the
+    codes, a write and a read of twice their bytes), which costs more than 4 rows reading the
+    codes themselves: there segments start at 5 rows (4-beam batch: 0.139 against 0.175 ms per
+    call with 4-row segments; 0.185 against 0.136 ms the other way round over bf16)."""
+    mr = getattr(args, "min_rows", None)
+    return mr if mr is not None else (5 if getattr(args, "kv", "bf16") == "fp8" else 2)
+
+
 def shared_decode_applies(args, w) -> bool:
     """The shared-prefix decode: on request, or by default for the shared-prompt workload;
     it needs the tensor-core decode's head shapes (bf16 or 8-bit pool)."""
@@ -552,7 +562,7 @@ def run_ours(args, rank, world, local_rank):
         q, k, v = w.host_step_inputs()
         plan = None
         if use_shared:
-            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs)
+            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args))
             plan = (torch.from_numpy(plan_h).to(device), info)
         states.append(dict(plan=plan, q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
                            slots=torch.from_numpy(slots).to(device), pairs=torch.from_numpy(pairs).to(device),
@@ -659,6 +669,7 @@ def run_ours(args, rank, world, local_rank):
                    "num_blocks": w.NB, "pool": pool,
                    "kv_bytes_per_step": kv_total // args.steps, "path": args.path,
                    "decode": "shared-prefix" if use_shared else "plain",
+                   **({"shared_min_rows": shared_min_rows(args)} if use_shared else {}),
                    "l2": ("L2 flushed before each timed step (a 252 MB write, outside the step's events): the"
                           " distinct KV per step is under 4x the 126 MB L2; e2e steps are pipelined, not flushed"
                           if flush_l2 else "inputs larger than L2 (distinct KV per step >= 4x the 126 MB L2)"),
@@ -751,7 +762,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
         for _ in range(n):
             probe.append_slots(seq_ids)
             t_, l_ = probe.export_tables(seq_ids, w.max_blocks)
-            plan_cap = max(plan_cap, int(pkv.shared_plan(t_, l_, w.Hq, w.Hkv, w.bs)[1].bytes))
+            plan_cap = max(plan_cap, int(pkv.shared_plan(t_, l_, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args))[1].bytes))
         probe.close()
     meta_bytes = o_plan + al(plan_cap)
     host_meta = [torch.empty(meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
@@ -802,7 +813,8 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
             hm[o_pairs:o_pairs + pairs.nbytes] = pairs.reshape(-1).view(np.uint8)
         plan_bytes = 0
         if sws is not None:  # planned straight into the pinned buffer (raises if it outgrew it)
-            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs, out=hm[o_plan:o_plan + plan_cap])
+            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args),
+                                           out=hm[o_plan:o_plan + plan_cap])
             plan_bytes = plan_h.nbytes
         with torch.cuda.stream(copy):
             if i >= 2:
@@ -1617,6 +1629,9 @@ def main():
     ap.add_argument("--shared", choices=["auto", "on", "off"], default="auto",
                     help="shared-prefix decode (blocks that adjacent rows share read once per kv head): auto = on "
                          "for the shared-prompt workload over a bf16 pool")
+    ap.add_argument("--min-rows", type=int, default=None,
+                    help="fewest rows a shared segment serves in the shared-prefix decode's plan"
+                         " (default 2 over bf16 pools, 5 over 8-bit pools)")
     ap.add_argument("--trace", action="store_true",
                     help="run the long-context continuous-batching trace step by step (the fifth workload)")
     ap.add_argument("--no-e2e", action="store_true")

@@ -42,11 +42,11 @@ class Pool8:
                                        np.asarray(b.block_tables)[rows], np.asarray(b.context_lens)[rows], b.scale)
 
 
-def run_shared(pkv, p, key_chunk=0, out_dtype=torch.float32, lens=None, plan_tables=None, status=None):
+def run_shared(pkv, p, key_chunk=0, out_dtype=torch.float32, lens=None, plan_tables=None, status=None, min_rows=2):
     b = p.b
     tables_h = b.block_tables if plan_tables is None else plan_tables
     plan, info = pkv.shared_plan(tables_h, b.context_lens, b.num_heads, b.num_kv_heads, b.block_size,
-                                 key_chunk=key_chunk)
+                                 min_rows=min_rows, key_chunk=key_chunk)
     plan_d = torch.from_numpy(plan).cuda()
     ws = torch.empty(pkv.paged_attention_decode_shared_fp8_workspace_size(info, b.num_heads, b.num_kv_heads,
                                                                           b.head_dim),
@@ -78,6 +78,15 @@ def test_beam_forks_match_oracle(pkv, steps, heads):
     p = Pool8(beam_batch(70 + steps, steps=steps, Hq=heads[0], Hkv=heads[1]), 1210 + steps)
     out, info = run_shared(pkv, p)
     assert info.num_segments >= 1
+    compare(out.cpu().numpy(), p.oracle())
+
+
+@pytest.mark.parametrize("steps", [1, 3])
+def test_beam_forks_without_beam_segments(pkv, steps):
+    """Segments of at least 5 rows only (the choice for 8-bit pools): the beams' parent blocks
+    stay in their private remainders, read by the 8-bit decode; the result is the same."""
+    p = Pool8(beam_batch(75 + steps, steps=steps), 1215 + steps)
+    out, info = run_shared(pkv, p, min_rows=5)
     compare(out.cpu().numpy(), p.oracle())
 
 

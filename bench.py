@@ -892,11 +892,13 @@ def run_trace(args, rank, world, local_rank):
     work (copy_blocks if any, reshape_and_cache, paged_attention_decode) is summed
     over the timed steps with CUDA events.
 
-    The host never waits for the device inside the loop, as a serving loop would not: each
-    step's tables, lengths and slots go up from pinned memory without blocking, so the host
-    (allocator, launches) runs ahead and a step's kernels are queued before the device reaches
-    them.  Events are read after the last step; the oracle's sampled sequences are gathered on
-    the device at their step and checked at the end."""
+    The allocator's decisions depend on nothing the device computes, so they are made first, on
+    the host, for every step (appends, copy-on-write pairs, tables, frees, admissions; their time
+    is reported as allocator_us_per_step), and each step's tables, lengths, slots, pairs and
+    inputs are staged on the device.  The timed pass then issues the device work in the serving
+    loop's order with the host only launching, so the host stays ahead of the device and a slow
+    host adds no idle time between a step's events.  Events are read after the last step; the
+    oracle's sampled sequences are gathered on the device at their step and checked at the end."""
     import torch
     import paged_kv_cache_423_b200 as pkv
 
@@ -929,6 +931,8 @@ def run_trace(args, rank, world, local_rank):
             return t.to(device)
         return t.pin_memory().to(device, non_blocking=True)
 
+    pending = []  # prompt writes of the sequences admitted since the last step: (slots, length)
+
     def admit(length, budget):
         nonlocal next_id
         if -(-length // p.block_size) > bm.num_free():
@@ -936,14 +940,43 @@ def run_trace(args, rank, world, local_rank):
         sid = next_id
         next_id += 1
         bm.add_seq(sid, length - 1)
-        slots = up(bm.slots(sid, 0, length - 1))
-        k = torch.randn((length - 1, p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
-        pkv.reshape_and_cache(k, k, kc, vc, slots, status=status)
+        pending.append((up(bm.slots(sid, 0, length - 1)), length))
         running[sid] = budget
 
+    # ---- pass 1, host only: the allocator's decisions for every step (appends, copy-on-write
+    # pairs, tables, frees, admissions), each step's inputs staged on the device
     for length, budget in initial:
         admit(length, budget)
     alloc_s = 0.0  # host allocator time of the timed steps (append, export, frees)
+    plan = []
+    for step in range(p.steps):
+        ids = sorted(running)
+        rec = {"admits": pending[:], "n": len(ids)}
+        pending.clear()
+        if ids:
+            a0 = time.perf_counter()
+            slots, pairs = bm.append_slots(ids)
+            tables, lens = bm.export_tables(ids, max_blocks)
+            a_s = time.perf_counter() - a0
+            rec.update(slots=up(slots), pairs=up(pairs) if len(pairs) else None, tables=up(tables), lens=up(lens),
+                       tables_h=tables, lens_h=lens, ids=ids,
+                       q=torch.randn((len(ids), p.num_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16),
+                       k=torch.randn((len(ids), p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16),
+                       ev=[torch.cuda.Event(enable_timing=True) for _ in range(4)])
+            a0 = time.perf_counter()
+            for sid in ids:
+                running[sid] -= 1
+                if running[sid] == 0:
+                    bm.free_seq(sid)
+                    del running[sid]
+            if step >= args.warmup:
+                alloc_s += a_s + time.perf_counter() - a0
+        for length, budget in arrivals[step]:
+            if len(running) < p.max_batch:
+                admit(length, budget)
+        plan.append(rec)
+    torch.cuda.synchronize()
+
     seq_steps = 0
     kv_bytes = 0
     launches = 0
@@ -980,49 +1013,33 @@ def run_trace(args, rank, world, local_rank):
         got = out1.float().cpu().numpy()
         ora["max_abs"] = max(ora["max_abs"], float(np.abs(got - ref).max()))
 
+    # ---- pass 2: the device work in the order the serving loop issues it; the host only
+    # launches, so it stays ahead of the device and no host time falls between a step's events
+    out_all = torch.empty((p.max_batch, p.num_heads, p.head_dim), dtype=torch.bfloat16, device=device)
     with ClockSampler(device) as clocks:
-        for step in range(p.steps):
-            ids = sorted(running)
-            if ids:
-                a0 = time.perf_counter()
-                slots, pairs = bm.append_slots(ids)
-                tables, lens = bm.export_tables(ids, max_blocks)
-                a_s = time.perf_counter() - a0
-                d_slots = up(slots)
-                d_tables = up(tables)
-                d_lens = up(lens)
-                q = torch.randn((len(ids), p.num_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
-                k = torch.randn((len(ids), p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
-                out = torch.empty((len(ids), p.num_heads, p.head_dim), dtype=torch.bfloat16, device=device)
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-                pairs_d = up(pairs) if len(pairs) else None
-                ev[0].record(stream)
-                if pairs_d is not None:
-                    pkv.copy_blocks([kc], [vc], pairs_d, status=status)
-                pkv.reshape_and_cache(k, k, kc, vc, d_slots, status=status)
-                ev[1].record(stream)
-                ev[2].record(stream)
-                pkv.paged_attention_decode(out, q, kc, vc, d_tables, d_lens, max_len, scale, ws, status=status)
-                ev[3].record(stream)
-                if step >= args.warmup:
-                    timed.append(ev)
-                    alloc_s += a_s
-                    seq_steps += len(ids)
-                    kv_bytes += int(lens.astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 4
-                    launches += 3 + (1 if len(pairs) else 0) + 1  # + the split merge
-                    if oracle_leg and (step - args.warmup) % 20 == 0:
-                        oracle_sample_stash(ids, tables, lens, q, out)
-                a0 = time.perf_counter()
-                for sid in ids:
-                    running[sid] -= 1
-                    if running[sid] == 0:
-                        bm.free_seq(sid)
-                        del running[sid]
-                if step >= args.warmup:
-                    alloc_s += time.perf_counter() - a0
-            for length, budget in arrivals[step]:
-                if len(running) < p.max_batch:
-                    admit(length, budget)
+        for step, rec in enumerate(plan):
+            for slots_d, length in rec["admits"]:  # synthetic prefill of the admitted prompts
+                k = torch.randn((length - 1, p.num_kv_heads, p.head_dim), generator=g, device=device).to(torch.bfloat16)
+                pkv.reshape_and_cache(k, k, kc, vc, slots_d, status=status)
+            if rec["n"] == 0:
+                continue
+            ev, out = rec["ev"], out_all[:rec["n"]]
+            ev[0].record(stream)
+            if rec["pairs"] is not None:
+                pkv.copy_blocks([kc], [vc], rec["pairs"], status=status)
+            pkv.reshape_and_cache(rec["k"], rec["k"], kc, vc, rec["slots"], status=status)
+            ev[1].record(stream)
+            ev[2].record(stream)
+            pkv.paged_attention_decode(out, rec["q"], kc, vc, rec["tables"], rec["lens"], max_len, scale, ws,
+                                       status=status)
+            ev[3].record(stream)
+            if step >= args.warmup:
+                timed.append(ev)
+                seq_steps += rec["n"]
+                kv_bytes += int(rec["lens_h"].astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 4
+                launches += 3 + (1 if rec["pairs"] is not None else 0) + 1  # + the split merge
+                if oracle_leg and (step - args.warmup) % 20 == 0:
+                    oracle_sample_stash(rec["ids"], rec["tables_h"], rec["lens_h"], rec["q"], out)
         torch.cuda.synchronize()
     # the step's kernels: the cache write (and copies), then the decode call; the host's
     # marshalling of the decode call between the two is not device work
@@ -1048,12 +1065,12 @@ def run_trace(args, rank, world, local_rank):
                        "initial_lengths": f"U{{{p.len_lo}..{p.len_hi}}}", "budgets": f"U{{{p.budget_lo}..{p.budget_hi}}}",
                        "arrivals": f"Bernoulli({p.arrival_p}) per free slot per step, lengths U{{{p.len_lo}..{p.len_hi}}}",
                        "timed": "copy_blocks + reshape_and_cache, and paged_attention_decode, per step (events"
-                                " around each call; the host runs ahead of the device, with pinned asynchronous"
-                                " uploads and no wait inside the loop; ms_per_step_span = first kernel start"
-                                " to last kernel end of a step)"},
+                                " around each call; the allocator's decisions for all steps made and staged on the"
+                                " device first, the timed pass only launching, so the host stays ahead of the device;"
+                                " ms_per_step_span = first kernel start to last kernel end of a step)"},
             "ms_per_step_span": round(span_ms / max(1, args.steps), 4),
             "seq_steps_per_s": round(seq_steps / (t_ms * 1e-3), 1), "pct_hbm_peak": round(100 * value / peak, 2),
-            # the same with the host allocator's time per step added (it runs between the steps here)
+            # the same with the host allocator's time per step added (made before the timed pass here)
             "seq_steps_per_s_with_allocator": round(seq_steps / (t_ms * 1e-3 + alloc_s), 1),
             "allocator_us_per_step": round(1e6 * alloc_s / max(1, args.steps), 2),
             "gpu_launches": launches, "clocks": clocks.summary(),

@@ -562,7 +562,8 @@ def run_ours(args, rank, world, local_rank):
         q, k, v = w.host_step_inputs()
         plan = None
         if use_shared:
-            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args))
+            plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args),
+                                           key_chunk=getattr(args, "key_chunk", 0))
             plan = (torch.from_numpy(plan_h).to(device), info)
         states.append(dict(plan=plan, q=to_dev(q, device), k=to_dev(k, device), v=to_dev(v, device),
                            slots=torch.from_numpy(slots).to(device), pairs=torch.from_numpy(pairs).to(device),
@@ -762,7 +763,8 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
         for _ in range(n):
             probe.append_slots(seq_ids)
             t_, l_ = probe.export_tables(seq_ids, w.max_blocks)
-            plan_cap = max(plan_cap, int(pkv.shared_plan(t_, l_, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args))[1].bytes))
+            plan_cap = max(plan_cap, int(pkv.shared_plan(t_, l_, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args),
+                                           key_chunk=getattr(args, "key_chunk", 0))[1].bytes))
         probe.close()
     meta_bytes = o_plan + al(plan_cap)
     host_meta = [torch.empty(meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
@@ -814,7 +816,7 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
         plan_bytes = 0
         if sws is not None:  # planned straight into the pinned buffer (raises if it outgrew it)
             plan_h, info = pkv.shared_plan(tables, lens, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args),
-                                           out=hm[o_plan:o_plan + plan_cap])
+                                           key_chunk=getattr(args, "key_chunk", 0), out=hm[o_plan:o_plan + plan_cap])
             plan_bytes = plan_h.nbytes
         with torch.cuda.stream(copy):
             if i >= 2:
@@ -1649,6 +1651,8 @@ def main():
     ap.add_argument("--min-rows", type=int, default=None,
                     help="fewest rows a shared segment serves in the shared-prefix decode's plan"
                          " (default 2 over bf16 pools, 5 over 8-bit pools)")
+    ap.add_argument("--key-chunk", type=int, default=0,
+                    help="keys per part of a shared segment in the shared-prefix decode's plan (0 = automatic)")
     ap.add_argument("--trace", action="store_true",
                     help="run the long-context continuous-batching trace step by step (the fifth workload)")
     ap.add_argument("--no-e2e", action="store_true")

@@ -374,7 +374,7 @@ class Workload:
         b = wl.make_decode_batch(name, with_data=False, extra_blocks=0)
         self.parents = b.num_seqs
         self.B, self.Hq, self.Hkv, self.D, self.bs = b.num_seqs * beams, b.num_heads, b.num_kv_heads, b.head_dim, b.block_size
-        self.seq_ids = beam_ids(self.parents, beams)  # row order of every step's tensors
+        self.seq_ids = np.asarray(beam_ids(self.parents, beams), np.int64)  # row order of every step's tensors
         self.scale = b.scale
         self.parent_lens0 = b.context_lens.copy()
         self.lens0 = np.repeat(b.context_lens, beams)  # per row: context length after the first appended token
@@ -1017,7 +1017,7 @@ def run_trace(args, rank, world, local_rank):
 
     # ---- pass 2: the device work in the order the serving loop issues it; the host only
     # launches, so it stays ahead of the device and no host time falls between a step's events
-    out_all = torch.empty((p.max_batch, p.num_heads, p.head_dim), dtype=torch.bfloat16, device=device)
+    out_all = torch.zeros((p.max_batch, p.num_heads, p.head_dim), dtype=torch.bfloat16, device=device)
     with ClockSampler(device) as clocks:
         for step, rec in enumerate(plan):
             for slots_d, length in rec["admits"]:  # synthetic prefill of the admitted prompts

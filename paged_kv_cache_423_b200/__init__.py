@@ -118,6 +118,15 @@ _SIGNATURES = {
 }
 
 
+def _id_array(seq_ids) -> np.ndarray:
+    """Sequence ids as a contiguous int64 array (an int64 array is used as it is; any other
+    iterable is read once)."""
+    if isinstance(seq_ids, np.ndarray) and seq_ids.dtype == np.int64 and seq_ids.flags.c_contiguous:
+        return seq_ids
+    return np.ascontiguousarray(seq_ids if isinstance(seq_ids, (np.ndarray, list, tuple)) else list(seq_ids),
+                                dtype=np.int64)
+
+
 class SharedPlanInfo(ctypes.Structure):
     """pkv_shared_plan_info: counts and byte offsets of a shared-prefix plan."""
     _fields_ = [(n, ctypes.c_int32) for n in ("num_seqs", "num_segments", "num_parts", "num_entries", "num_partials",
@@ -639,7 +648,7 @@ class BlockManager:
         _check(library().pkv_bm_fork(self._h, parent, child), "bm_fork")
 
     def append_slots(self, seq_ids):
-        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        ids = _id_array(seq_ids)
         slots = np.zeros(len(ids), np.int64)
         pairs = np.zeros((max(len(ids), 1), 2), np.int64)
         n_cow = c_int(0)
@@ -650,7 +659,7 @@ class BlockManager:
     def append_tokens(self, seq_ids, tokens):
         """append_slots with the token id of each new position; a sequence created from
         token ids registers every block these tokens complete in the prefix cache."""
-        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        ids = _id_array(seq_ids)
         toks = np.ascontiguousarray(list(tokens), dtype=np.int32)
         if len(toks) != len(ids):
             raise ValueError("append_tokens: one token per sequence")
@@ -682,7 +691,7 @@ class BlockManager:
         return r
 
     def export_tables(self, seq_ids, max_blocks: int):
-        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        ids = _id_array(seq_ids)
         tables = np.zeros((len(ids), max_blocks), np.int32)
         lens = np.zeros(len(ids), np.int32)
         _check(library().pkv_bm_export_tables(self._h, _np_ptr(ids), len(ids), _np_ptr(tables), max_blocks,
@@ -706,7 +715,7 @@ class BlockManager:
         return bool(r)
 
     def _swap(self, fn, seq_ids, what):
-        ids = np.ascontiguousarray(list(seq_ids), dtype=np.int64)
+        ids = _id_array(seq_ids)
         cap = max(self.num_blocks, self.num_host_blocks, 1)
         pairs = np.zeros((cap, 2), np.int64)
         n = c_int(0)

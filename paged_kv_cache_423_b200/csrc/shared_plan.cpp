@@ -86,11 +86,16 @@ extern "C" int pkv_shared_plan(const int32_t* block_tables, int max_blocks_per_s
       int s = r + 1;
       while (s < w.r1 && full(s, w.k) && at(s, w.k) == at(r, w.k)) ++s;
       if (s - r >= min_rows) {
-        int k2 = w.k + 1;
-        for (;; ++k2) {
-          bool same = true;
-          for (int q = r; q < s && same; ++q) same = full(q, k2) && at(q, k2) == at(r, k2);
-          if (!same) break;
+        // k2: the first position past w.k where some row of r..s-1 has no full block or a
+        // block other than row r's (each row's table scanned along its own memory)
+        int k2 = max_blocks_per_seq;
+        const int32_t* base = block_tables + static_cast<int64_t>(r) * max_blocks_per_seq;
+        for (int q = r; q < s; ++q) {
+          const int32_t* row = block_tables + static_cast<int64_t>(q) * max_blocks_per_seq;
+          const int lim = std::min(k2, std::min(context_lens[q] / block_size, max_blocks_per_seq));
+          int k = w.k + 1;
+          while (k < lim && row[k] == base[k]) ++k;
+          k2 = k;
         }
         segs.push_back({r, s - r, w.k, k2 - w.k});
         for (int q = r; q < s; ++q) depth[q] = k2;

@@ -263,7 +263,7 @@ def test_workload_default_path_is_unforked_and_unshared(pkv):
     shared blocks, the manager's tables and lengths those of plain add_seq calls."""
     import torch
     w = bench.Workload("tiny", 4, seed=3, device=torch.device("cpu"))
-    assert w.seq_ids == list(range(w.B)) and w.beams == 1 and w.shared_blocks == 0 and w.layout is None
+    assert list(w.seq_ids) == list(range(w.B)) and w.beams == 1 and w.shared_blocks == 0 and w.layout is None
     assert w.label == "tiny"
     bm = w.new_manager()
     ref = pkv.BlockManager(w.NB, w.bs, w.free_order)

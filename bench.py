@@ -180,14 +180,14 @@ def stream_read_gbs(pkv, device, nbytes=4 << 30, reps=10):
 
 def split_tokens(num_seqs, num_kv_heads, block_size, max_context_len, tensor):
     """The library's automatic split of a context (tokens per partition) for a call:
-    the CUDA-core path takes the largest of 512..64 that leaves >= 4096 work items,
+    the CUDA-core path takes the largest of 512..64 that leaves >= 16384 work items,
     the tensor-core paths the largest of 2048.. down to that which leaves >= 16 items
     per SM, and not below 512 with at least 4 (sequence, kv head) units per SM.  Used
     to count the launches of a step (a split context adds the merge)."""
     def items(p):
         return num_seqs * num_kv_heads * -(-max_context_len // p)
     base = 512
-    while base > 64 and items(base) < 4096:
+    while base > 64 and items(base) < 16384:
         base //= 2
     base = max(base, block_size)
     if not tensor:

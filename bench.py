@@ -181,7 +181,7 @@ def stream_read_gbs(pkv, device, nbytes=4 << 30, reps=10):
 def split_tokens(num_seqs, num_kv_heads, block_size, max_context_len, tensor):
     """The library's automatic split of a context (tokens per partition) for a call:
     the CUDA-core path takes the largest of 512..64 that leaves >= 16384 work items,
-    the tensor-core paths the largest of 2048.. down to that which leaves >= 16 items
+    the tensor-core paths the largest of 2048.. down to that which leaves >= 8 items
     per SM, and not below 512 with at least 4 (sequence, kv head) units per SM.  Used
     to count the launches of a step (a split context adds the merge)."""
     def items(p):
@@ -193,7 +193,7 @@ def split_tokens(num_seqs, num_kv_heads, block_size, max_context_len, tensor):
     if not tensor:
         return base
     p = 2048
-    while p > base and items(p) < 16 * 148:
+    while p > base and items(p) < 8 * 148:
         p //= 2
     if num_seqs * num_kv_heads >= 4 * 148 and p < 512:
         p = 512

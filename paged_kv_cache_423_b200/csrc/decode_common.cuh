@@ -92,16 +92,21 @@ inline int auto_partition_tokens(int num_seqs, int num_kv_heads, int block_size,
 
 // The tensor-core path pays a fixed cost per item (the first tile's maximum, the
 // output or partial, and later a merge): it takes longer splits, up to 2048 tokens, as
-// long as about 16 items per SM remain for load balance.  With at least 4 (sequence,
+// long as about 8 items per SM remain for load balance (long-context batch, 16 x
+// U{5k..32k}: 2048-token splits, 5,764 -> 5,852 GB/s bf16 and 5,107 -> 5,348 e4m3
+// against the 1024 that a target of 16 per SM gave; 32 per SM was slower still).  With at least 4 (sequence,
 // kv head) units per SM it never splits below 512 tokens: items of one or two tiles
 // would cost about as much in per-item work as in streaming, and the units alone
 // balance the SMs.  Never shorter than the CUDA-core split, so a workspace sized for
 // that split always suffices.
+#ifndef PKV_TC_ITEMS_PER_SM
+#define PKV_TC_ITEMS_PER_SM 8
+#endif
 inline int auto_partition_tokens_tensor(int num_seqs, int num_kv_heads, int block_size, int max_context_len) {
   const int base = auto_partition_tokens(num_seqs, num_kv_heads, block_size, max_context_len);
   const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
   int p = kMaxPartition;
-  while (p > base && units * ((max_context_len + p - 1) / p) < 16 * 148) p /= 2;
+  while (p > base && units * ((max_context_len + p - 1) / p) < PKV_TC_ITEMS_PER_SM * 148) p /= 2;
   if (units >= 4 * 148 && p < 512) p = 512;
   return p > base ? p : base;
 }

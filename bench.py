@@ -758,14 +758,21 @@ def run_e2e(args, w, pkv, device, path, ws, out, status, max_len_bound, sws=None
     o_lens = o_tab + al(4 * w.B * w.max_blocks)
     o_plan = o_lens + al(4 * w.B)
     plan_cap = 0
-    if sws is not None:  # room for the largest plan: sized on a dry run of the allocator
+    if sws is not None:  # room for the largest plan and workspace: sized on a dry run of the allocator
+        size_fn = (pkv.paged_attention_decode_shared_fp8_workspace_size if w.kv8
+                   else pkv.paged_attention_decode_shared_workspace_size)
+        ws_need = sws.numel()
         probe = w.new_manager()
         for _ in range(n):
             probe.append_slots(seq_ids)
             t_, l_ = probe.export_tables(seq_ids, w.max_blocks)
-            plan_cap = max(plan_cap, int(pkv.shared_plan(t_, l_, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args),
-                                           key_chunk=getattr(args, "key_chunk", 0))[1].bytes))
+            info_ = pkv.shared_plan(t_, l_, w.Hq, w.Hkv, w.bs, min_rows=shared_min_rows(args),
+                                    key_chunk=getattr(args, "key_chunk", 0))[1]
+            plan_cap = max(plan_cap, int(info_.bytes))
+            ws_need = max(ws_need, size_fn(info_, w.Hq, w.Hkv, w.D))
         probe.close()
+        if ws_need > sws.numel():  # the e2e run goes further than the timed steps' states
+            sws = torch.empty(ws_need, dtype=torch.uint8, device=device)
     meta_bytes = o_plan + al(plan_cap)
     host_meta = [torch.empty(meta_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     dev_qkv = [torch.empty(nq + 2 * nk, dtype=torch.int16, device=device) for _ in range(2)]

@@ -15,6 +15,7 @@
 // prompt blocks are registered under a chain hash of their token ids; a later prompt
 // takes its longest registered leading run.  A registered block with no references
 // stays registered in the free list until the list hands it out again.
+#include <algorithm>
 #include <cstring>
 #include <deque>
 #include <new>
@@ -96,6 +97,7 @@ struct pkv_bm {
     bool tracked = false;
     uint64_t parent = 0;           // chain hash of the last full block
     std::vector<int32_t> partial;  // token ids of the block being filled
+    uint64_t stamp = 0;            // the last append call that listed it (repeats are rejected)
   };
   int num_blocks = 0;
   int block_size = 0;
@@ -113,6 +115,9 @@ struct pkv_bm {
   // Scratch for the dry run of append_slots: per-block pending reference change.
   std::vector<int32_t> pending;
   std::vector<int32_t> touched;
+  // Scratch of append calls: the listed sequences, and the call's stamp.
+  std::vector<Seq*> listed;
+  uint64_t append_calls = 0;
 
   bool valid_block(int32_t b) const { return b >= 0 && b < num_blocks; }
   int blocks_for(int tokens) const { return (tokens + block_size - 1) / block_size; }
@@ -258,15 +263,17 @@ static int append_impl(pkv_bm* bm, const int64_t* seq_ids, const int32_t* tokens
   if (!bm || n < 0 || (n > 0 && (!seq_ids || !slots_out || !cow_pairs_out)) || !n_cow_out)
     return set_error(PKV_ERR_INVALID, "pkv_bm_append_slots: bad arguments");
   *n_cow_out = 0;
-  // Validate ids (known, distinct) and resolve them once.
-  std::vector<pkv_bm::Seq*> seqs(n);
-  std::unordered_map<int64_t, int> seen;
-  seen.reserve(static_cast<size_t>(n) * 2);
+  // Validate ids (known, distinct: a sequence already stamped by this call is a repeat) and
+  // resolve them once.
+  std::vector<pkv_bm::Seq*>& seqs = bm->listed;
+  seqs.resize(static_cast<size_t>(n));
+  const uint64_t stamp = ++bm->append_calls;
   for (int i = 0; i < n; ++i) {
     auto it = bm->seqs.find(seq_ids[i]);
-    if (it == bm->seqs.end() || it->second.swapped || !seen.emplace(seq_ids[i], i).second)
+    if (it == bm->seqs.end() || it->second.swapped || it->second.stamp == stamp)
       return set_error(PKV_ERR_INVALID, "pkv_bm_append_slots: unknown, repeated or swapped-out sequence %lld",
                        (long long)seq_ids[i]);
+    it->second.stamp = stamp;
     seqs[i] = &it->second;
   }
   // Dry run: count fresh blocks, following reference counts as earlier sequences
@@ -388,18 +395,19 @@ extern "C" int pkv_bm_export_tables(const pkv_bm* bm, const int64_t* seq_ids, in
                                     int max_blocks, int32_t* context_lens) {
   if (!bm || n < 0 || max_blocks < 0 || (n > 0 && (!seq_ids || !context_lens || (max_blocks > 0 && !tables))))
     return set_error(PKV_ERR_INVALID, "pkv_bm_export_tables: bad arguments");
+  std::vector<const pkv_bm::Seq*> seqs(static_cast<size_t>(n));
   for (int i = 0; i < n; ++i) {
     auto it = bm->seqs.find(seq_ids[i]);
     if (it == bm->seqs.end() || it->second.swapped || static_cast<int>(it->second.table.size()) > max_blocks)
       return set_error(PKV_ERR_INVALID, "pkv_bm_export_tables: unknown sequence %lld or table longer than %d",
                        (long long)seq_ids[i], max_blocks);
+    seqs[i] = &it->second;
   }
   for (int i = 0; i < n; ++i) {
-    const auto& s = bm->seqs.find(seq_ids[i])->second;
+    const auto& s = *seqs[i];
     int32_t* row = tables + static_cast<size_t>(i) * max_blocks;
-    size_t k = 0;
-    for (; k < s.table.size(); ++k) row[k] = s.table[k];
-    for (; k < static_cast<size_t>(max_blocks); ++k) row[k] = 0;
+    std::copy(s.table.begin(), s.table.end(), row);
+    std::fill(row + s.table.size(), row + max_blocks, 0);
     context_lens[i] = s.len;
   }
   return PKV_OK;

@@ -437,3 +437,21 @@ def test_launch_setup_runs_once_per_device(tmp_path):
                     os.path.join(root, "tests", "native", "per_device_test.cpp"), "-o", str(exe)], check=True)
     res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0 and res.stdout.strip() == "ok", res.stdout + res.stderr
+
+
+def test_sequence_ids_in_any_form(pkv):
+    """The allocator takes sequence ids as a list, a tuple, an int64 array (used as it is),
+    an array of another integer type or any iterable; the results are the same."""
+    import numpy as np
+    forms = [[0, 1, 2], (0, 1, 2), np.array([0, 1, 2], np.int64), np.array([0, 1, 2], np.int32), iter([0, 1, 2]),
+             {0: None, 1: None, 2: None}.keys()]
+    results = []
+    for ids in forms:
+        bm = pkv.BlockManager(16, 4, list(range(16)))
+        for s in range(3):
+            bm.add_seq(s, 3 + s)
+        slots, pairs = bm.append_slots(ids)
+        tables, lens = bm.export_tables([0, 1, 2], 4)
+        results.append((slots.tolist(), pairs.tolist(), tables.tolist(), lens.tolist()))
+        bm.close()
+    assert all(r == results[0] for r in results)

@@ -734,3 +734,13 @@ def test_shared_private_rule_matches_the_library():
     src = open(os.path.join(bench.ROOT, "paged_kv_cache_423_b200", "csrc", "shared_decode.cu")).read()
     m = re.search(r"#define PKV_SHARED_SIMT_MAX (\d+)", src)
     assert m and int(m.group(1)) == bench.SHARED_SIMT_SUFFIX_MAX
+
+
+def test_shared_plan_options_by_pool():
+    """Segments of 2 rows over bf16 pools and of 5 over 8-bit pools unless --min-rows says
+    otherwise."""
+    import types
+    assert bench.shared_min_rows(types.SimpleNamespace(kv="bf16")) == 2
+    assert bench.shared_min_rows(types.SimpleNamespace(kv="fp8")) == 5
+    assert bench.shared_min_rows(types.SimpleNamespace(kv="fp8", min_rows=3)) == 3
+    assert bench.shared_min_rows(types.SimpleNamespace(kv="bf16", min_rows=None)) == 2
